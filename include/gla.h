@@ -1,0 +1,182 @@
+/*
+ * gla.h -- C ABI of libgla, the B200 (sm_100a) Simple Gated Linear Attention
+ * mixer library.
+ *
+ * The mixer (page "AWS serve Laplace 3B di i14 con uno stato fisso di 29,5 MB",
+ * section "GLA sostituisce i token conservati con uno stato ricorrente": every
+ * layer replaces softmax attention with Simple GLA, which updates a
+ * fixed-size matrix state per token) computes, per (batch, head), with a
+ * scalar log-decay a_t <= 0 per token and head:
+ *
+ *     S_t = exp(a_t) * S_{t-1} + k_t^T v_t         S: dk x dv, fp32
+ *     o_t = scale * q_t S_t                         scale: normally dk^-1/2
+ *
+ * Shapes follow page "Como i14 llevo Laplace 3B a AWS Trainium2", section
+ * "Diseno esencial de Laplace 3B": H = 16 heads, dk = 96, dv = 192.
+ *
+ * Conventions shared by every entry point
+ *   - Every tensor pointer is DEVICE memory owned by the caller.  libgla never
+ *     allocates, never frees and never synchronises (except the two status
+ *     readers at the end of this file, which say so).
+ *   - Every call is asynchronous on the caller's stream and returns a
+ *     gla_status.  Argument errors are detected on the host before anything
+ *     is launched; in that case nothing is written.
+ *   - Layout is token-major: [B, T, H, d] with d innermost and contiguous.
+ *     Base pointers must be 16-byte aligned (GLA_ERR_MISALIGNED otherwise).
+ *   - No exception crosses this ABI.
+ *   - Preconditions not checked on the device: a_t <= 0 and finite; inputs
+ *     finite.
+ *   - Device-side waits (on TMA / tensor-core completion barriers) are
+ *     bounded.  A wait that runs out records GLA_ERR_TIMEOUT in a device status
+ *     word, the kernel releases what it holds and returns; read the word with
+ *     gla_get_device_status().
+ */
+#ifndef GLA_H
+#define GLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gla_status {
+    GLA_OK = 0,
+    GLA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, workspace too small */
+    GLA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. dk != 96)    */
+    GLA_ERR_MISALIGNED = 3,    /* pointer or stride not 16-byte aligned        */
+    GLA_ERR_CUDA = 4,          /* a CUDA call failed; see gla_last_cuda_error  */
+    GLA_ERR_TIMEOUT = 5        /* a bounded device-side wait ran out           */
+} gla_status;
+
+typedef enum gla_dtype {
+    GLA_BF16 = 0,              /* bf16 q/k/v/o/dO; fp32 state and decay        */
+    GLA_F32 = 1                /* fp32 everywhere (forward only)               */
+} gla_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gla_status_string(gla_status s);
+
+/* cudaError_t of the last failed CUDA call made by libgla on this host thread
+ * (0 when none). */
+int gla_last_cuda_error(void);
+
+/* Number of kernel launches libgla has issued from this process (all
+ * threads), for launch accounting by callers. */
+unsigned long long gla_launch_count(void);
+
+/* ---------------------------------------------------------------------------
+ * Chunked prefill / training forward.
+ *
+ * The chunked form ("Como i14 ...", section "Adaptaciones para AWS
+ * Trainium2", item 1: T = 2048 processed as 16 chunks of 128 tokens) is an
+ * exact reorganisation of the recurrence above.  Chunk size is 128.
+ *
+ *   q, k    [B, T, H, dk]  dt       token stride ld_qkv elements (0 = packed:
+ *   v       [B, T, H, dv]  dt       H*dk for q and k, H*dv for v); head stride
+ *                                   dk (q, k) or dv (v); batch stride T*ld.
+ *                                   ld_qkv lets q/k/v be views into one fused
+ *                                   projection buffer (e.g. 9216 per token).
+ *   a       [B, T, H]      fp32     log-decay, contiguous.
+ *   s0      [B, H, dk, dv] fp32     initial state; NULL means zeros.
+ *   o       [B, T, H, dv]  dt       output, contiguous.
+ *   s_final [B, H, dk, dv] fp32     final state S_T; NULL to skip.
+ *   ws      workspace of ws_bytes >= gla_chunk_workspace_bytes(B,T,H,dk,dv,0)
+ *           (may be NULL when that size is 0).  Its contents on entry do not
+ *           matter and are undefined on return.
+ *   scale   multiplies q once (normally dk^-1/2); must be > 0 and finite.
+ *   dt      GLA_BF16 (tensor-core path: fp32 accumulation, fp32 state) or
+ *           GLA_F32 (fp32 CUDA-core path, for small problems).
+ * Supported: dk == 96, dv == 192, B, H >= 1, T >= 1 (any T; the last chunk may
+ * be partial).  ld_qkv must be a multiple of 8 and >= the packed stride.
+ * ------------------------------------------------------------------------ */
+size_t gla_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int for_bwd);
+
+gla_status gla_chunk_fwd(const void* q, const void* k, const void* v, const float* a,
+                         const float* s0, void* o, float* s_final, void* ws, size_t ws_bytes,
+                         int B, int T, int H, int dk, int dv, int64_t ld_qkv, float scale,
+                         gla_dtype dt, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Chunked backward (the sequential chunk backward of "Como i14 ...", section
+ * "Adaptaciones para AWS Trainium2", item 3).  Same inputs as the forward plus
+ *   dO       [B, T, H, dv]  dt     upstream gradient of o, contiguous.
+ *   ds_final [B, H, dk, dv] fp32   upstream gradient of S_T; NULL means zero.
+ * Outputs (contiguous):
+ *   grad_q, grad_k [B, T, H, dk] dt;  grad_v [B, T, H, dv] dt;
+ *   grad_a [B, T, H] fp32;  grad_s0 [B, H, dk, dv] fp32 (NULL to skip).
+ * grad_q is the gradient with respect to the unscaled q that was passed in.
+ * ws_bytes >= gla_chunk_workspace_bytes(B,T,H,dk,dv,1).  dt must be GLA_BF16.
+ * ------------------------------------------------------------------------ */
+gla_status gla_chunk_bwd(const void* q, const void* k, const void* v, const float* a,
+                         const float* s0, const void* dO, const float* ds_final,
+                         void* grad_q, void* grad_k, void* grad_v, float* grad_a,
+                         float* grad_s0, void* ws, size_t ws_bytes, int B, int T, int H, int dk,
+                         int dv, int64_t ld_qkv, float scale, gla_dtype dt, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * One decode step for N sequences (the fixed per-sequence state of "AWS serve
+ * Laplace 3B ...", section "Lo stato di Laplace 3B resta fisso durante
+ * l'inferenza"; 1,280 concurrent sequences in "Como i14 ...", section
+ * "Resultados de entrenamiento e inferencia").  For every (n, h):
+ *     S <- exp(a[n,h]) * S + k[n,h]^T v[n,h]     (in place, fp32)
+ *     o[n,h] = scale * q[n,h] S                   (the updated S)
+ *   state    [N_slots, H, dk, dv] fp32, updated in place.
+ *   slot_idx [N] int32: state slot of sequence n (NULL = identity, N_slots = N).
+ *            Slots must be distinct within one call and < N_slots (not
+ *            checked on the device).
+ *   q, k     [N, H, dk] bf16;  v [N, H, dv] bf16;  a [N, H] fp32 (contiguous).
+ *   o        [N, H, dv] fp32.
+ * Supported: dk == 96, dv == 192.
+ * ------------------------------------------------------------------------ */
+gla_status gla_decode_step(float* state, const int32_t* slot_idx, const void* q, const void* k,
+                           const void* v, const float* a, float* o, int N, int H, int dk, int dv,
+                           float scale, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Front end of each layer ("Como i14 ...", section "Diseno esencial de
+ * Laplace 3B": the residual vector goes through LayerNorm, then a causal
+ * depthwise Conv1d of width 4 with SiLU, a 4-gram summary before the mixer):
+ *     xn[t]   = LayerNorm(x[t]) over D   (biased variance, eps inside the root,
+ *                                          then * gamma + beta) if apply_ln,
+ *               else x[t]
+ *     y[t,c]  = SiLU( sum_{j<W} w[c,j] * xn[t-(W-1)+j, c] + bias[c] )
+ * Positions before t = 0 come from conv_state_in (zeros when NULL).
+ *   x, y            [B, T, D] bf16, contiguous.
+ *   ln_gamma/beta   [D] fp32, NULL = 1 / 0.
+ *   w               [D, W] fp32 (w[c, W-1] multiplies the current token).
+ *   bias            [D] fp32 or NULL.
+ *   conv_state_in   [B, W-1, D] fp32 or NULL: the last W-1 conv inputs (xn)
+ *                   before t = 0, oldest first.
+ *   conv_state_out  [B, W-1, D] fp32 or NULL: the last W-1 conv inputs of
+ *                   this call, for the next call.  Must not alias
+ *                   conv_state_in.
+ * Supported: W == 4, D % 8 == 0, 8 <= D <= 4096.
+ * ------------------------------------------------------------------------ */
+gla_status conv1d_silu_causal(const void* x, int apply_ln, const float* ln_gamma,
+                              const float* ln_beta, float ln_eps, const float* w,
+                              const float* bias, const float* conv_state_in,
+                              float* conv_state_out, void* y, int B, int T, int D, int W,
+                              cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Device status.  gla_get_device_status SYNCHRONISES the stream, copies the
+ * device status word of the current device (0 or a gla_status recorded by a
+ * kernel, e.g. GLA_ERR_TIMEOUT) into *device_status and clears it.
+ * gla_set_wait_limit_ns sets the bound on every device-side wait of later
+ * launches (default 2e9 ns; 0 restores the default).
+ * gla_selftest_wait_timeout launches one kernel whose only wait is on a
+ * barrier that nothing completes, so the bound runs out by design and the
+ * kernel returns having recorded GLA_ERR_TIMEOUT; it lets callers check the
+ * failure path without faulting or hanging the GPU.
+ * ------------------------------------------------------------------------ */
+gla_status gla_get_device_status(cudaStream_t stream, int* device_status);
+gla_status gla_set_wait_limit_ns(unsigned long long ns);
+gla_status gla_selftest_wait_timeout(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GLA_H */

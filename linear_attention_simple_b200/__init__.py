@@ -1,1 +1,302 @@
-"""Simple GLA mixer on B200 (placeholder until the binding lands)."""
+"""libgla -- Simple Gated Linear Attention mixer for B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/gla.h``: the functions below
+have the same names as the exported C entry points and only marshal
+arguments (check dtypes/devices/strides, allocate outputs with PyTorch when
+the caller passes none, pass raw pointers and the current CUDA stream).
+Every step of the computation runs in the kernels of ``libgla.so``; there is
+no CPU or PyTorch fallback.  Importing this package does not load the
+library; the first call does, and raises ``GlaLibraryMissing`` when
+``libgla.so`` has not been built (``python -m linear_attention_simple_b200.build``).
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "GlaError", "GlaLibraryMissing", "lib", "gla_status_string", "gla_launch_count",
+    "gla_chunk_workspace_bytes", "gla_chunk_fwd", "gla_chunk_bwd", "gla_decode_step",
+    "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
+    "gla_selftest_wait_timeout", "EXPORTED_SYMBOLS", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgla.so")
+
+EXPORTED_SYMBOLS = (
+    "gla_status_string", "gla_last_cuda_error", "gla_launch_count",
+    "gla_chunk_workspace_bytes", "gla_chunk_fwd", "gla_chunk_bwd", "gla_decode_step",
+    "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
+    "gla_selftest_wait_timeout",
+)
+
+GLA_BF16, GLA_F32 = 0, 1
+STATUS = {0: "GLA_OK", 1: "GLA_ERR_INVALID_ARG", 2: "GLA_ERR_UNSUPPORTED",
+          3: "GLA_ERR_MISALIGNED", 4: "GLA_ERR_CUDA", 5: "GLA_ERR_TIMEOUT"}
+
+
+class GlaLibraryMissing(RuntimeError):
+    pass
+
+
+class GlaError(RuntimeError):
+    def __init__(self, fn, status, cuda_err=0):
+        self.status = status
+        self.cuda_error = cuda_err
+        msg = "%s failed: %s" % (fn, STATUS.get(status, str(status)))
+        if status == 4:
+            msg += " (cudaError %d)" % cuda_err
+        super().__init__(msg)
+
+
+_LIB = None
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_i64 = ctypes.c_int64
+_f = ctypes.c_float
+
+
+def lib():
+    """Load libgla.so (once).  Raises GlaLibraryMissing if it is not built."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise GlaLibraryMissing("libgla.so not found at %s; build it with "
+                                "`python -m linear_attention_simple_b200.build`" % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    L.gla_status_string.restype = ctypes.c_char_p
+    L.gla_status_string.argtypes = [_i]
+    L.gla_last_cuda_error.restype = _i
+    L.gla_launch_count.restype = ctypes.c_ulonglong
+    L.gla_chunk_workspace_bytes.restype = ctypes.c_size_t
+    L.gla_chunk_workspace_bytes.argtypes = [_i, _i, _i, _i, _i, _i]
+    L.gla_chunk_fwd.restype = _i
+    L.gla_chunk_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                                _i, _i, _i, _i, _i, _i64, _f, _i, _vp]
+    L.gla_chunk_bwd.restype = _i
+    L.gla_chunk_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                _vp, ctypes.c_size_t, _i, _i, _i, _i, _i, _i64, _f, _i, _vp]
+    L.gla_decode_step.restype = _i
+    L.gla_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
+    L.conv1d_silu_causal.restype = _i
+    L.conv1d_silu_causal.argtypes = [_vp, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _vp,
+                                     _i, _i, _i, _i, _vp]
+    L.gla_get_device_status.restype = _i
+    L.gla_get_device_status.argtypes = [_vp, ctypes.POINTER(_i)]
+    L.gla_set_wait_limit_ns.restype = _i
+    L.gla_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    L.gla_selftest_wait_timeout.restype = _i
+    L.gla_selftest_wait_timeout.argtypes = [_vp]
+    _LIB = L
+    return L
+
+
+def _check(fn, status):
+    if status != 0:
+        raise GlaError(fn, status, lib().gla_last_cuda_error())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dt(t):
+    if t.dtype == torch.bfloat16:
+        return GLA_BF16
+    if t.dtype == torch.float32:
+        return GLA_F32
+    raise TypeError("q/k/v must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _token_stride(x, B, T, H, d):
+    """Token stride (elements) of a [B,T,H,d] view whose head and feature
+    dims are packed; raises if the view is not of that form."""
+    if x.shape != (B, T, H, d):
+        raise ValueError("expected shape %s, got %s" % ((B, T, H, d), tuple(x.shape)))
+    s = x.stride()
+    if s[3] != 1 or s[2] != d:
+        raise ValueError("head and feature dims must be packed (strides %s)" % (s,))
+    if B > 1 and T > 0 and s[0] != T * s[1]:
+        raise ValueError("batch stride must be T * token stride (strides %s)" % (s,))
+    return s[1]
+
+
+def _need(x, name, dtype, shape=None, contiguous=True):
+    if x is None:
+        return
+    if not x.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if x.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, x.dtype))
+    if shape is not None and tuple(x.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(x.shape)))
+    if contiguous and not x.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def gla_status_string(status):
+    return lib().gla_status_string(int(status)).decode()
+
+
+def gla_launch_count():
+    return int(lib().gla_launch_count())
+
+
+def gla_chunk_workspace_bytes(B, T, H, dk=96, dv=192, for_bwd=False):
+    return int(lib().gla_chunk_workspace_bytes(B, T, H, dk, dv, 1 if for_bwd else 0))
+
+
+def _qkv_strides(q, k, v):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    lq = _token_stride(q, B, T, H, dk)
+    lk = _token_stride(k, B, T, H, dk)
+    lv = _token_stride(v, B, T, H, dv)
+    if lq == H * dk and lk == H * dk and lv == H * dv:
+        return 0
+    if not (lq == lk == lv):
+        raise ValueError("q, k and v must share one token stride when not packed "
+                         "(got %d, %d, %d)" % (lq, lk, lv))
+    return lq
+
+
+def gla_chunk_fwd(q, k, v, a, s0=None, o=None, s_final=None, ws=None, scale=None,
+                  want_final_state=True, stream=None):
+    """Chunked forward.  q, k [B,T,H,dk]; v [B,T,H,dv] (bf16 or fp32, may be
+    views into one fused projection buffer); a [B,T,H] fp32; s0 [B,H,dk,dv]
+    fp32 or None.  Returns (o, s_final)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dt(q)
+    for name, x in (("k", k), ("v", v)):
+        if x.dtype != q.dtype:
+            raise TypeError("%s must have the dtype of q" % name)
+    ld = _qkv_strides(q, k, v)
+    _need(a, "a", torch.float32, (B, T, H))
+    _need(s0, "s0", torch.float32, (B, H, dk, dv))
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    _need(o, "o", q.dtype, (B, T, H, dv))
+    if s_final is None and want_final_state:
+        s_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(s_final, "s_final", torch.float32, (B, H, dk, dv))
+    need = gla_chunk_workspace_bytes(B, T, H, dk, dv, False) if dt == GLA_BF16 else 0
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if scale is None:
+        scale = dk ** -0.5
+    st = lib().gla_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(s0), _ptr(o),
+                             _ptr(s_final), _ptr(ws), 0 if ws is None else ws.numel(),
+                             B, T, H, dk, dv, ld, float(scale), dt, _stream(stream))
+    _check("gla_chunk_fwd", st)
+    return o, s_final
+
+
+def gla_chunk_bwd(q, k, v, a, dO, s0=None, ds_final=None, grads=None, ws=None, scale=None,
+                  want_grad_s0=True, stream=None):
+    """Chunked backward.  Returns (dq, dk, dv, da, ds0)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dt(q)
+    ld = _qkv_strides(q, k, v)
+    _need(a, "a", torch.float32, (B, T, H))
+    _need(dO, "dO", q.dtype, (B, T, H, dv))
+    _need(s0, "s0", torch.float32, (B, H, dk, dv))
+    _need(ds_final, "ds_final", torch.float32, (B, H, dk, dv))
+    dev = q.device
+    if grads is None:
+        grads = (torch.empty((B, T, H, dk), dtype=q.dtype, device=dev),
+                 torch.empty((B, T, H, dk), dtype=q.dtype, device=dev),
+                 torch.empty((B, T, H, dv), dtype=q.dtype, device=dev),
+                 torch.empty((B, T, H), dtype=torch.float32, device=dev),
+                 torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+                 if want_grad_s0 else None)
+    gq, gk, gv, ga, gs0 = grads
+    _need(gq, "grad_q", q.dtype, (B, T, H, dk))
+    _need(gk, "grad_k", q.dtype, (B, T, H, dk))
+    _need(gv, "grad_v", q.dtype, (B, T, H, dv))
+    _need(ga, "grad_a", torch.float32, (B, T, H))
+    _need(gs0, "grad_s0", torch.float32, (B, H, dk, dv))
+    need = gla_chunk_workspace_bytes(B, T, H, dk, dv, True)
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    if scale is None:
+        scale = dk ** -0.5
+    st = lib().gla_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(s0), _ptr(dO),
+                             _ptr(ds_final), _ptr(gq), _ptr(gk), _ptr(gv), _ptr(ga), _ptr(gs0),
+                             _ptr(ws), 0 if ws is None else ws.numel(), B, T, H, dk, dv, ld,
+                             float(scale), dt, _stream(stream))
+    _check("gla_chunk_bwd", st)
+    return gq, gk, gv, ga, gs0
+
+
+def gla_decode_step(state, q, k, v, a, o=None, slot_idx=None, scale=None, stream=None):
+    """In-place decode step.  state [N_slots,H,dk,dv] fp32; q, k [N,H,dk] and
+    v [N,H,dv] bf16; a [N,H] fp32; slot_idx [N] int32 or None.  Returns o."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    _need(state, "state", torch.float32)
+    if state.dim() != 4 or tuple(state.shape[1:]) != (H, dk, dv):
+        raise ValueError("state must be [N_slots, %d, %d, %d]" % (H, dk, dv))
+    _need(q, "q", torch.bfloat16, (N, H, dk))
+    _need(k, "k", torch.bfloat16, (N, H, dk))
+    _need(v, "v", torch.bfloat16, (N, H, dv))
+    _need(a, "a", torch.float32, (N, H))
+    _need(slot_idx, "slot_idx", torch.int32, (N,))
+    if slot_idx is None and state.shape[0] != N:
+        raise ValueError("without slot_idx the state must have N slots")
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=torch.float32, device=q.device)
+    _need(o, "o", torch.float32, (N, H, dv))
+    if scale is None:
+        scale = dk ** -0.5
+    st = lib().gla_decode_step(_ptr(state), _ptr(slot_idx), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+                               _ptr(o), N, H, dk, dv, float(scale), _stream(stream))
+    _check("gla_decode_step", st)
+    return o
+
+
+def conv1d_silu_causal(x, w, apply_ln=True, ln_gamma=None, ln_beta=None, ln_eps=1e-5,
+                       bias=None, conv_state_in=None, conv_state_out=None, y=None,
+                       stream=None):
+    """LayerNorm -> causal depthwise conv -> SiLU.  x [B,T,D] bf16; w [D,W]
+    fp32.  Returns y (and fills conv_state_out [B,W-1,D] fp32 if given)."""
+    B, T, D = x.shape
+    W = w.shape[1]
+    _need(x, "x", torch.bfloat16, (B, T, D))
+    _need(w, "w", torch.float32, (D, W))
+    _need(ln_gamma, "ln_gamma", torch.float32, (D,))
+    _need(ln_beta, "ln_beta", torch.float32, (D,))
+    _need(bias, "bias", torch.float32, (D,))
+    _need(conv_state_in, "conv_state_in", torch.float32, (B, W - 1, D))
+    _need(conv_state_out, "conv_state_out", torch.float32, (B, W - 1, D))
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", torch.bfloat16, (B, T, D))
+    st = lib().conv1d_silu_causal(_ptr(x), 1 if apply_ln else 0, _ptr(ln_gamma), _ptr(ln_beta),
+                                  float(ln_eps), _ptr(w), _ptr(bias), _ptr(conv_state_in),
+                                  _ptr(conv_state_out), _ptr(y), B, T, D, W, _stream(stream))
+    _check("conv1d_silu_causal", st)
+    return y
+
+
+def gla_get_device_status(stream=None):
+    """Synchronise the stream and return (and clear) the device status word."""
+    out = ctypes.c_int(0)
+    _check("gla_get_device_status", lib().gla_get_device_status(_stream(stream),
+                                                                ctypes.byref(out)))
+    return out.value
+
+
+def gla_set_wait_limit_ns(ns):
+    _check("gla_set_wait_limit_ns", lib().gla_set_wait_limit_ns(int(ns)))
+
+
+def gla_selftest_wait_timeout(stream=None):
+    _check("gla_selftest_wait_timeout", lib().gla_selftest_wait_timeout(_stream(stream)))

@@ -1,0 +1,75 @@
+// gla_internal.h -- declarations shared by the libgla translation units
+// (host launchers, the wait-control block, tile constants).  Not part of the
+// public ABI; the public ABI is include/gla.h.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime_api.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/gla.h"
+
+namespace gla {
+
+// Bounded-wait control passed by value to every kernel that waits.
+struct WaitCtl {
+    int* status;                   // device status word (first error wins)
+    unsigned long long limit_ns;   // wall-time bound of each wait
+};
+
+// Chunk geometry of the tensor-core path.
+constexpr int kChunk = 128;        // tokens per chunk (M of every MMA)
+constexpr int kDk = 96;
+constexpr int kDv = 192;
+
+// Host-side helpers implemented in gla_host.cu.
+WaitCtl wait_ctl_for_current_device(gla_status* err);
+gla_status check_launch(const char* what);
+void count_launch(unsigned n = 1);
+
+// Encode a tiled tensor map over a bf16 (or fp32) [d3][d2][d1][d0] tensor.
+// dims[i] elements, strides_bytes[i] for i >= 1 (dim 0 contiguous), box[i].
+gla_status make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box, int elem_bytes,
+                     int swizzle_bytes);
+
+// ---- launchers (one per kernel family), all asynchronous on `st`.
+gla_status launch_decode(float* state, const int32_t* slot_idx, const void* q, const void* k,
+                         const void* v, const float* a, float* o, int N, int H, float scale,
+                         cudaStream_t st);
+
+gla_status launch_conv(const void* x, int apply_ln, const float* g, const float* b, float eps,
+                       const float* w, const float* bias, const float* cs_in, float* cs_out,
+                       void* y, int B, int T, int D, cudaStream_t st);
+
+gla_status launch_fwd_f32(const float* q, const float* k, const float* v, const float* a,
+                          const float* s0, float* o, float* s_final, int B, int T, int H,
+                          int64_t ld_qk, int64_t ld_v, float scale, const WaitCtl& ctl,
+                          cudaStream_t st);
+
+// Chunked bf16 paths (chunk_fwd.cu / chunk_bwd.cu).
+struct ChunkProblem {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* a;
+    int B, T, H;
+    int64_t ld_qk, ld_v;           // token strides in elements
+    float scale;
+};
+
+size_t fwd_workspace_bytes(int B, int T, int H);
+size_t bwd_workspace_bytes(int B, int T, int H);
+
+gla_status run_chunk_fwd(const ChunkProblem& p, const float* s0, void* o, float* s_final,
+                         void* ws, size_t ws_bytes, const WaitCtl& ctl, cudaStream_t st);
+
+gla_status run_chunk_bwd(const ChunkProblem& p, const float* s0, const void* dO,
+                         const float* ds_final, void* dq, void* dk, void* dv, float* da,
+                         float* ds0, void* ws, size_t ws_bytes, const WaitCtl& ctl,
+                         cudaStream_t st);
+
+gla_status launch_wait_selftest(const WaitCtl& ctl, cudaStream_t st);
+
+}  // namespace gla

@@ -1,0 +1,205 @@
+"""GPU parity: decode step, LayerNorm/conv/SiLU front end, fp32 forward, and
+the bounded-wait failure path.  Every CUDA result is compared element by
+element with the fp64 oracle on the same seeded inputs.
+
+Tolerances (relative L2 = ||x - ref|| / ||ref||, ref = oracle):
+  fp32 decode (state and o)      <= 1e-5
+  fp32 forward (o and S_T)       <= 1e-5
+  bf16 front end output y        <= 1e-2, max-abs <= 5e-2
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_simple_b200 as gla
+from linear_attention_simple_b200 import inputs
+from oracle import recurrent
+
+pytestmark = pytest.mark.gpu
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def rel(x, ref):
+    return float(np.linalg.norm(x - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    from linear_attention_simple_b200 import build
+    build.build()
+    gla.lib()
+
+
+# ------------------------------------------------------------------ decode
+
+@pytest.mark.parametrize("N,H", [(1, 1), (37, 3), (256, 16)])
+def test_decode_parity(N, H):
+    d = inputs.decode_inputs(N, H, seed=20 + N, device="cuda")[0]
+    st0 = _np(d["state"])
+    o = gla.gla_decode_step(d["state"], d["q"], d["k"], d["v"], d["a"])
+    ref_state, ref_o = recurrent.decode(st0, _np(d["q"]), _np(d["k"]), _np(d["v"]), _np(d["a"]))
+    assert rel(_np(d["state"]), ref_state) <= 1e-5
+    assert rel(_np(o), ref_o) <= 1e-5
+    assert gla.gla_get_device_status() == 0
+
+
+def test_decode_slot_indirection_leaves_other_slots_untouched():
+    N, H, slots = 40, 4, 96
+    d = inputs.decode_inputs(N, H, seed=31, device="cuda", n_slots=slots)[0]
+    g = torch.Generator().manual_seed(5)
+    idx = torch.randperm(slots, generator=g)[:N].to(torch.int32).cuda()
+    before = d["state"].clone()
+    o = gla.gla_decode_step(d["state"], d["q"], d["k"], d["v"], d["a"], slot_idx=idx)
+    ref_state, ref_o = recurrent.decode(_np(before), _np(d["q"]), _np(d["k"]), _np(d["v"]),
+                                        _np(d["a"]), slot_idx=idx.cpu().numpy())
+    assert rel(_np(d["state"]), ref_state) <= 1e-5
+    assert rel(_np(o), ref_o) <= 1e-5
+    untouched = sorted(set(range(slots)) - set(idx.cpu().tolist()))
+    assert torch.equal(d["state"][untouched], before[untouched])      # bit-exact
+
+
+def test_decode_repeated_steps_match_recurrence():
+    """T decode steps from S_0 equal the forward recurrence over T tokens."""
+    N, H, T = 8, 2, 5
+    d = inputs.chunk_inputs(N, T, H, seed=33, device="cuda", s0_std=0.1)
+    state = d["s0"].clone()
+    outs = []
+    for t in range(T):
+        outs.append(gla.gla_decode_step(state, d["q"][:, t].contiguous(), d["k"][:, t].contiguous(),
+                                        d["v"][:, t].contiguous(), d["a"][:, t].contiguous()))
+    ref_o, ref_s = recurrent.fwd(_np(d["q"]), _np(d["k"]), _np(d["v"]), _np(d["a"]), _np(d["s0"]))
+    assert rel(np.stack([_np(x) for x in outs], axis=1), ref_o) <= 1e-5
+    assert rel(_np(state), ref_s) <= 1e-5
+
+
+def test_decode_full_size_sampled():
+    """1280 sequences x 16 heads (one layer of the 24-layer step, the launch the
+    benchmark times), checked on 96 sampled (sequence, head) units."""
+    N, H = 1280, 16
+    d = inputs.decode_inputs(N, H, seed=1004, device="cuda")[0]
+    g = torch.Generator().manual_seed(7)
+    units = torch.randperm(N * H, generator=g)[:96]
+    units = torch.cat([units, torch.tensor([0, N * H - 1])])
+    n_idx, h_idx = units // H, units % H
+    st0 = d["state"][n_idx, h_idx].clone()
+    o = gla.gla_decode_step(d["state"], d["q"], d["k"], d["v"], d["a"])
+    ref_state, ref_o = recurrent.decode(_np(st0)[:, None], _np(d["q"][n_idx, h_idx])[:, None],
+                                        _np(d["k"][n_idx, h_idx])[:, None],
+                                        _np(d["v"][n_idx, h_idx])[:, None],
+                                        _np(d["a"][n_idx, h_idx])[:, None])
+    assert rel(_np(d["state"][n_idx, h_idx]), ref_state[:, 0]) <= 1e-5
+    assert rel(_np(o[n_idx, h_idx]), ref_o[:, 0]) <= 1e-5
+
+
+# --------------------------------------------------------------- front end
+
+def _front_check(y, ref):
+    assert rel(y, ref) <= 1e-2
+    assert float(np.max(np.abs(y - ref))) <= 5e-2
+
+
+@pytest.mark.parametrize("B,T,D,hist,affine", [(1, 1, 256, False, False), (2, 37, 256, True, True),
+                                               (3, 300, 3072, True, False), (1, 2, 64, True, True)])
+def test_front_end_parity(B, T, D, hist, affine):
+    d = inputs.front_inputs(B, T, D, seed=40 + T, device="cuda", with_state=hist)
+    g = b = bias = None
+    if affine:
+        g = inputs.randn((D,), 41, "cuda", std=0.5) + 1.0
+        b = inputs.randn((D,), 42, "cuda", std=0.5)
+        bias = inputs.randn((D,), 43, "cuda", std=0.5)
+    cs_out = torch.empty((B, 3, D), dtype=torch.float32, device="cuda")
+    y = gla.conv1d_silu_causal(d["x"], d["w"], ln_gamma=g, ln_beta=b, bias=bias,
+                               conv_state_in=d["conv_state"], conv_state_out=cs_out)
+    ref_y, ref_cs = recurrent.ln_conv_silu(_np(d["x"]), _np(d["w"]), ln=True,
+                                           ln_gamma=None if g is None else _np(g),
+                                           ln_beta=None if b is None else _np(b),
+                                           bias=None if bias is None else _np(bias),
+                                           conv_state=None if d["conv_state"] is None
+                                           else _np(d["conv_state"]))
+    _front_check(_np(y), ref_y)
+    assert rel(_np(cs_out), ref_cs) <= 1e-5
+
+
+def test_front_end_without_layernorm():
+    d = inputs.front_inputs(2, 50, 512, seed=44, device="cuda", with_state=True)
+    y = gla.conv1d_silu_causal(d["x"], d["w"], apply_ln=False, conv_state_in=d["conv_state"])
+    ref_y, _ = recurrent.ln_conv_silu(_np(d["x"]), _np(d["w"]), ln=False,
+                                      conv_state=_np(d["conv_state"]))
+    _front_check(_np(y), ref_y)
+
+
+def test_front_end_chained_calls_equal_one_call():
+    """Carrying conv_state_out into the next call reproduces the unsplit run."""
+    B, T, D, split = 1, 90, 512, 41
+    d = inputs.front_inputs(B, T, D, seed=45, device="cuda")
+    y_full = gla.conv1d_silu_causal(d["x"], d["w"])
+    cs = torch.empty((B, 3, D), dtype=torch.float32, device="cuda")
+    y1 = gla.conv1d_silu_causal(d["x"][:, :split].contiguous(), d["w"], conv_state_out=cs)
+    y2 = gla.conv1d_silu_causal(d["x"][:, split:].contiguous(), d["w"], conv_state_in=cs)
+    y_split = torch.cat([y1, y2], dim=1)
+    # bf16 outputs: the two runs do the same fp32 arithmetic per element
+    assert rel(_np(y_split), _np(y_full)) <= 1e-6
+
+
+def test_front_end_full_size_sampled():
+    """T = 65536, D = 3072 (the long-context prefill front end, as benchmarked),
+    checked on sampled tokens including CTA boundaries and both ends."""
+    B, T, D = 1, 65536, 3072
+    d = inputs.front_inputs(B, T, D, seed=1005, device="cuda")
+    y = gla.conv1d_silu_causal(d["x"], d["w"])
+    g = torch.Generator().manual_seed(9)
+    toks = sorted(set(torch.randint(0, T, (40,), generator=g).tolist()) |
+                  {0, 1, 2, 3, 221, 222, 223, 224, T - 1})
+    x = _np(d["x"])
+    w = _np(d["w"])
+    ys = _np(y)
+    got, ref = [], []
+    for t in toks:
+        lo = max(0, t - 3)
+        r, _ = recurrent.ln_conv_silu(x[:, lo:t + 1], w)
+        got.append(ys[:, t])
+        ref.append(r[:, -1])
+    _front_check(np.stack(got), np.stack(ref))
+
+
+# -------------------------------------------------------------- fp32 path
+
+@pytest.mark.parametrize("B,T,H,s0", [(1, 256, 1, False), (2, 77, 3, True), (1, 1, 1, True)])
+def test_fwd_fp32_parity(B, T, H, s0):
+    d = inputs.chunk_inputs(B, T, H, dtype=torch.float32, seed=50 + T, device="cuda",
+                            s0_std=0.1 if s0 else None)
+    o, sf = gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], s0=d["s0"])
+    ro, rs = recurrent.fwd(_np(d["q"]), _np(d["k"]), _np(d["v"]), _np(d["a"]),
+                           None if d["s0"] is None else _np(d["s0"]))
+    assert rel(_np(o), ro) <= 1e-5
+    assert rel(_np(sf), rs) <= 1e-5
+
+
+def test_fwd_empty_sequence_copies_state():
+    d = inputs.chunk_inputs(2, 0, 3, seed=51, device="cuda", s0_std=0.1)
+    o, sf = gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], s0=d["s0"])
+    torch.cuda.synchronize()
+    assert o.numel() == 0
+    assert torch.equal(sf, d["s0"])
+
+
+# ------------------------------------------------------ failure detection
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    gla.gla_set_wait_limit_ns(5_000_000)          # 5 ms
+    try:
+        assert gla.gla_get_device_status() == 0
+        gla.gla_selftest_wait_timeout()
+        assert gla.gla_get_device_status() == 5     # GLA_ERR_TIMEOUT, then cleared
+        assert gla.gla_get_device_status() == 0
+    finally:
+        gla.gla_set_wait_limit_ns(0)
+    # the context is still usable
+    d = inputs.decode_inputs(4, 2, seed=52, device="cuda")[0]
+    st0 = _np(d["state"])
+    o = gla.gla_decode_step(d["state"], d["q"], d["k"], d["v"], d["a"])
+    ref_state, ref_o = recurrent.decode(st0, _np(d["q"]), _np(d["k"]), _np(d["v"]), _np(d["a"]))
+    assert rel(_np(o), ref_o) <= 1e-5

@@ -1,7 +1,183 @@
-// chunk_fwd.cu -- placeholder, replaced by the tensor-core kernel.
-#include "gla_internal.h"
+// chunk_fwd.cu -- host side of the chunked bf16 forward, plus the segment
+// combine kernel.
+//
+// Work split.  The chunk recurrence is sequential per (batch, head), so with
+// B*H units the fused kernel has B*H CTAs.  When B*H alone cannot fill the
+// GPU (long prefill: T = 65,536 at B*H = 16), each unit's chunks are cut into
+// nseg segments and processed in three steps:
+//   1. state-only pass over segments 0..nseg-2 from a zero state: each
+//      segment's local end state L_g (fp32) and total log2-decay G_g;
+//   2. combine (CUDA cores, elementwise over dk x dv): the true state
+//      entering each segment, S_{g+1} = 2^{G_g} S_g + L_g, S_0 = s0;
+//   3. fused output pass over all segments from those states.
+// This is exact (the state is linear in its inputs); it trades one extra
+// read of k and v for nseg-fold parallelism.
+#include <cstring>
+
+#include "chunk_state.cuh"
+
 namespace gla {
-size_t fwd_workspace_bytes(int, int, int) { return 0; }
-gla_status run_chunk_fwd(const ChunkProblem&, const float*, void*, float*, void*, size_t,
-                         const WaitCtl&, cudaStream_t) { return GLA_ERR_UNSUPPORTED; }
+namespace {
+
+constexpr int kTargetCtas = 148;                 // one wave of B200 SMs
+constexpr int64_t kSS = static_cast<int64_t>(kDk) * kDv;
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int num_chunks(int T) { return (T + kChunk - 1) / kChunk; }
+
+void segment_plan(int units, int NC, int* nseg, int* cps)
+{
+    int n = units >= kTargetCtas / 2 ? 1 : kTargetCtas / units;
+    n = n < 1 ? 1 : (n > NC ? NC : n);
+    int c = (NC + n - 1) / n;
+    *cps = c;
+    *nseg = (NC + c - 1) / c;
+}
+
+__global__ void __launch_bounds__(256) seg_combine_kernel(float* __restrict__ states,
+                                                          const float* __restrict__ g2,
+                                                          const float* __restrict__ s0, int nseg,
+                                                          int units)
+{
+    const int64_t n4 = kSS / 4;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= n4 * units) return;
+    const int64_t unit = idx / n4, e4 = idx - unit * n4;
+    float4* st = reinterpret_cast<float4*>(states);
+    float4 x = s0 ? reinterpret_cast<const float4*>(s0)[unit * n4 + e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int g = 0; g < nseg; ++g) {
+        float4* slot = st + (unit * nseg + g) * n4 + e4;
+        const float4 l = (g < nseg - 1) ? *slot : make_float4(0.f, 0.f, 0.f, 0.f);
+        *slot = x;
+        if (g < nseg - 1) {
+            const float f = exp2f(g2[unit * nseg + g]);
+            x.x = fmaf(f, x.x, l.x);
+            x.y = fmaf(f, x.y, l.y);
+            x.z = fmaf(f, x.z, l.z);
+            x.w = fmaf(f, x.w, l.w);
+        }
+    }
+}
+
+template <bool W, bool R>
+gla_status launch_state_t(const StateParams& p, dim3 grid, cudaStream_t st)
+{
+    const uint32_t bytes = chunk::Smem<W>::BYTES;
+    cudaError_t e = cudaFuncSetAttribute(gla_chunk_state_kernel<W, R>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return check_launch("cudaFuncSetAttribute");
+    gla_chunk_state_kernel<W, R><<<grid, 256, bytes, st>>>(p);
+    count_launch();
+    return check_launch("gla_chunk_state_kernel");
+}
+
+}  // namespace
+
+gla_status make_token_map(CUtensorMap* m, const void* base, int d, int H, int T, int B,
+                          int64_t ld, int box_d, int swizzle)
+{
+    const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(H),
+                              static_cast<uint64_t>(T), static_cast<uint64_t>(B)};
+    const uint64_t strides[4] = {2, static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(ld) * 2,
+                                 static_cast<uint64_t>(T) * ld * 2};
+    const uint32_t box[4] = {static_cast<uint32_t>(box_d), 1, 128, 1};
+    return make_tmap(m, base, 4, dims, strides, box, 2, swizzle);
+}
+
+gla_status make_state_map(CUtensorMap* m, void* base, int64_t nstates)
+{
+    const uint64_t dims[3] = {static_cast<uint64_t>(kDv), static_cast<uint64_t>(kDk),
+                              static_cast<uint64_t>(nstates)};
+    const uint64_t strides[3] = {2, static_cast<uint64_t>(kDv) * 2,
+                                 static_cast<uint64_t>(kDk) * kDv * 2};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(kDk), 1};
+    return make_tmap(m, base, 3, dims, strides, box, 2, 128);
+}
+
+gla_status launch_state_kernel(bool with_o, bool reverse, const StateParams& p, dim3 grid,
+                               cudaStream_t st)
+{
+    if (with_o && !reverse) return launch_state_t<true, false>(p, grid, st);
+    if (!with_o && !reverse) return launch_state_t<false, false>(p, grid, st);
+    if (!with_o && reverse) return launch_state_t<false, true>(p, grid, st);
+    return GLA_ERR_UNSUPPORTED;
+}
+
+size_t fwd_workspace_bytes(int B, int T, int H)
+{
+    const int units = B * H, NC = num_chunks(T);
+    int nseg, cps;
+    segment_plan(units, NC, &nseg, &cps);
+    if (nseg == 1) return 0;
+    return align256(static_cast<size_t>(units) * nseg * kSS * sizeof(float)) +
+           align256(static_cast<size_t>(units) * nseg * sizeof(float));
+}
+
+gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float* s_final,
+                         void* ws, size_t ws_bytes, const WaitCtl& ctl, cudaStream_t st)
+{
+    (void)ws_bytes;
+    const int units = pr.B * pr.H, NC = num_chunks(pr.T);
+    int nseg, cps;
+    segment_plan(units, NC, &nseg, &cps);
+
+    StateParams p;
+    memset(&p, 0, sizeof(p));
+    gla_status s;
+    if ((s = make_token_map(&p.tm_q, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
+    if ((s = make_token_map(&p.tm_u, pr.k, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
+    if ((s = make_token_map(&p.tm_y, pr.v, kDv, pr.H, pr.T, pr.B, pr.ld_v, 64, 128)) != GLA_OK) return s;
+    if ((s = make_token_map(&p.tm_o, o, kDv, pr.H, pr.T, pr.B, static_cast<int64_t>(pr.H) * kDv, 64,
+                            128)) != GLA_OK)
+        return s;
+    p.a = pr.a;
+    p.B = pr.B;
+    p.T = pr.T;
+    p.H = pr.H;
+    p.NC = NC;
+    p.chunks_per_seg = cps;
+    p.scale = pr.scale;
+    p.ctl = ctl;
+    p.store_h = 0;
+
+    if (nseg == 1) {
+        p.s_init = s0;
+        p.init_unit_stride = kSS;
+        p.s_out = s_final;
+        p.out_unit_stride = kSS;
+        p.out_last_only = 1;
+        return launch_state_kernel(true, false, p, dim3(1, pr.H, pr.B), st);
+    }
+
+    float* states = static_cast<float*>(ws);
+    float* g2 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                         align256(static_cast<size_t>(units) * nseg * kSS * sizeof(float)));
+    // 1. local end states of segments 0..nseg-2
+    StateParams pre = p;
+    pre.s_init = nullptr;
+    pre.s_out = states;
+    pre.out_unit_stride = nseg * kSS;
+    pre.out_seg_stride = kSS;
+    pre.out_last_only = 0;
+    pre.g2_out = g2;
+    pre.g2_unit_stride = nseg;
+    if ((s = launch_state_kernel(false, false, pre, dim3(nseg - 1, pr.H, pr.B), st)) != GLA_OK) return s;
+    // 2. states entering every segment
+    const int64_t n4 = static_cast<int64_t>(units) * (kSS / 4);
+    seg_combine_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(states, g2, s0, nseg,
+                                                                               units);
+    count_launch();
+    if ((s = check_launch("seg_combine_kernel")) != GLA_OK) return s;
+    // 3. fused output pass
+    p.s_init = states;
+    p.init_unit_stride = nseg * kSS;
+    p.init_seg_stride = kSS;
+    p.s_out = s_final;
+    p.out_unit_stride = kSS;
+    p.out_seg_stride = 0;
+    p.out_last_only = 1;
+    return launch_state_kernel(true, false, p, dim3(nseg, pr.H, pr.B), st);
+}
+
 }  // namespace gla

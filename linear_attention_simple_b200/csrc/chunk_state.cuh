@@ -1,0 +1,559 @@
+// chunk_state.cuh -- the sequential-over-chunks Simple GLA kernel on tcgen05.
+//
+// One CTA owns one (batch, head, segment of chunks) and walks its chunks in
+// order (forward) or in reverse, keeping the fp32 dk x dv state in tensor
+// memory.  The chunked form ("Como i14 llevo Laplace 3B a AWS Trainium2",
+// section "Adaptaciones para AWS Trainium2", item 1: chunks of 128 tokens;
+// item 3: the backward walks the chunks sequentially) with, for a chunk of
+// tokens i, j and in-chunk cumulative log-decay b_i (gamma = b_last):
+//
+//   forward  o_i  = scale ( e^{b_i} q_i S_prev + sum_{j<=i} e^{b_i-b_j} (q_i.k_j) v_j )
+//            S    = e^{gamma} S_prev + sum_j e^{gamma-b_j} k_j^T v_j
+//   reverse  D    = e^{gamma} D_next + sum_i (scale e^{b_i} q_i)^T dO_i
+//
+// Template modes
+//   WITH_O   forward with the output fused in: per chunk four tcgen05.mma
+//            groups -- scores = Q K^T (128x128x96), O = Q~ S_prev
+//            (128x192x96, fp16 operands), O += P V (128x192x128, P split
+//            into two bf16 terms P_hi + P_lo), S += K~^T V (128pad x 192 x
+//            128) -- plus the masked-decay P tile on CUDA cores.  The
+//            state itself is always fp32 in tensor memory; only the MMA
+//            operand copies are 16-bit.
+//   !WITH_O  state only: S (or D) += U~^T Y per chunk, optionally storing the
+//            bf16 state before each chunk's update (for the backward).
+//   REVERSE  walks chunks from last to first (the dL/dS pass).
+//
+// Operand layouts (all validated against the hardware): q and k tiles are
+// TMA-loaded as three 32-wide SW64 boxes ([3][128][32], K-major for the
+// scores; the k tile doubles as the MN-major A operand of the state product,
+// whose fourth 32-row block is a permanent zero block); v tiles are three
+// 64-wide SW128 boxes ([3][128][64], MN-major B); the bf16 state copy is
+// [3][96][64] SW128 (MN-major B of O = Q~ S); P_hi is [2][128][64] SW128
+// (K-major A) and reuses the state copy's buffer once O = Q~ S has run;
+// P_lo uses the output staging buffer, which is free until the epilogue.
+//
+// Every wait is bounded; on timeout the CTA stops at the next block-wide
+// barrier, drains its in-flight copies and tensor-core work (again bounded),
+// frees its tensor memory and returns with GLA_ERR_TIMEOUT recorded.
+#pragma once
+
+#include "gla_device.cuh"
+
+namespace gla {
+
+struct StateParams {
+    CUtensorMap tm_q;       // q tile loads (WITH_O)
+    CUtensorMap tm_u;       // scaled operand: k (forward) or q (reverse)
+    CUtensorMap tm_y;       // v (forward) or dO (reverse)
+    CUtensorMap tm_o;       // o tile stores (WITH_O)
+    CUtensorMap tm_h;       // per-chunk bf16 state stores (store_h)
+    const float* a;         // [B, T, H] log-decay
+    const float* s_init;    // initial state per (unit, seg) or null (zeros)
+    float* s_out;           // state after the segment, or null
+    float* g2_out;          // total log2-decay of each segment, or null
+    int64_t init_unit_stride, init_seg_stride;   // elements
+    int64_t out_unit_stride, out_seg_stride;     // elements
+    int B, T, H, NC, chunks_per_seg;
+    int out_last_only;      // write s_out only from the last segment
+    int g2_unit_stride;     // segments per unit in g2_out
+    int store_h;            // store the bf16 state entering each chunk
+    float scale;
+    WaitCtl ctl;
+};
+
+namespace chunk {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Shared-memory map (bytes from a 1024-aligned base).
+template <bool WITH_O>
+struct Smem;
+template <>
+struct Smem<true> {
+    static constexpr uint32_t Q = 0;          // [3][128][32] bf16 SW64
+    static constexpr uint32_t U = 24576;      // k tile  [3][128][32] bf16 SW64
+    static constexpr uint32_t Z = 49152;      // zero block (4th M block of U^T)
+    static constexpr uint32_t Y = 57344;      // v tile  [3][128][64] bf16 SW128
+    static constexpr uint32_t X = 106496;     // state copy [3][96][64] / P [2][128][64]
+    static constexpr uint32_t O = 143360;     // output staging [3][128][64]
+    static constexpr uint32_t MISC = 192512;
+    static constexpr uint32_t BYTES = MISC + 1024 + 1024;   // + alignment slack
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t TM_SC = 0, TM_O = 128, TM_S = 320;
+};
+template <>
+struct Smem<false> {
+    static constexpr uint32_t Q = 0;          // unused
+    static constexpr uint32_t U = 0;
+    static constexpr uint32_t Z = 24576;
+    static constexpr uint32_t Y = 32768;
+    static constexpr uint32_t X = 81920;
+    static constexpr uint32_t O = 0;          // unused
+    static constexpr uint32_t MISC = 118784;
+    static constexpr uint32_t BYTES = MISC + 1024 + 1024;
+    static constexpr uint32_t TMEM_COLS = 256;
+    static constexpr uint32_t TM_SC = 0, TM_O = 0, TM_S = 0;
+};
+
+constexpr uint32_t kTileQK = 3 * 128 * 64;     // 24576 bytes
+constexpr uint32_t kTileV = 3 * 128 * 128;     // 49152 bytes
+
+constexpr uint32_t kIdScores = idesc_bf16_f32(128, 128, 0, 0);
+constexpr uint32_t kIdOut = idesc_bf16_f32(128, 192, 0, 1);
+// O = Q~ S_prev runs in fp16 (10-bit mantissa) on rescaled copies: Q~ * 2^5
+// and S_prev * 2^-5, so the product is unchanged while |S| up to ~2e6 stays
+// inside the fp16 range.
+constexpr uint32_t kIdInter = idesc_f16_f32(128, 192, 0, 1);
+constexpr float kInterUp = 32.0f, kInterDown = 1.0f / 32.0f;
+constexpr uint32_t kIdState = idesc_bf16_f32(128, 192, 1, 1);
+
+__device__ __forceinline__ void named_sync(int id, int n)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ uint4 scale8(uint4 v, float f)
+{
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = pack_bf16(bf16_lo(w[i]) * f, bf16_hi(w[i]) * f);
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ uint4 scale8_to_f16(uint4 v, float f)
+{
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = pack_f16(bf16_lo(w[i]) * f, bf16_hi(w[i]) * f);
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Scale the 64-byte row segment `row` of block `blk` of a [3][128][32] SW64
+// tile in place (the swizzle only permutes 16-byte chunks within a row);
+// TO_F16 also converts the bf16 elements to fp16.
+template <bool TO_F16 = false>
+__device__ __forceinline__ void scale_row_sw64(uint8_t* tile, int row, int blk, float f)
+{
+    uint4* p = reinterpret_cast<uint4*>(tile + blk * 8192 + row * 64);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) p[c] = TO_F16 ? scale8_to_f16(p[c], f) : scale8(p[c], f);
+}
+
+__device__ __forceinline__ uint4 pack8_f16(const uint32_t* r, float f)
+{
+    return make_uint4(pack_f16(__uint_as_float(r[0]) * f, __uint_as_float(r[1]) * f),
+                      pack_f16(__uint_as_float(r[2]) * f, __uint_as_float(r[3]) * f),
+                      pack_f16(__uint_as_float(r[4]) * f, __uint_as_float(r[5]) * f),
+                      pack_f16(__uint_as_float(r[6]) * f, __uint_as_float(r[7]) * f));
+}
+
+__device__ __forceinline__ uint4 pack8(const uint32_t* r)
+{
+    return make_uint4(pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1])),
+                      pack_bf16(__uint_as_float(r[2]), __uint_as_float(r[3])),
+                      pack_bf16(__uint_as_float(r[4]), __uint_as_float(r[5])),
+                      pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7])));
+}
+
+}  // namespace chunk
+
+template <bool WITH_O, bool REVERSE>
+__global__ void __launch_bounds__(256, 1) gla_chunk_state_kernel(const __grid_constant__ StateParams p)
+{
+    using L = chunk::Smem<WITH_O>;
+    using namespace chunk;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const uint32_t sb = smem_u32(sm);
+    uint64_t* bar_q = reinterpret_cast<uint64_t*>(sm + L::MISC);
+    uint64_t* bar_u = bar_q + 1;
+    uint64_t* bar_y = bar_q + 2;
+    uint64_t* bar_m = bar_q + 3;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_q + 4);
+    float* b2s = reinterpret_cast<float*>(sm + L::MISC + 64);   // 128 floats
+    float* wsum = b2s + 128;                                     // 4 floats
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int unit = b * p.H + h;
+    const int c_begin = seg * p.chunks_per_seg;
+    const int c_end = min(p.NC, c_begin + p.chunks_per_seg);
+    const int nchunks = c_end - c_begin;
+    const WaitCtl ctl = p.ctl;
+
+    // thread <-> TMEM lane / tile row: warp w covers lanes 32*(w%4) .. +31,
+    // column half (w/4).  State rows exist only for lanes < 96.
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int half = warp >> 2;
+    const bool srow = quad < 3;
+
+    if (tid == 0) {
+        mbar_init(bar_q, 1);
+        mbar_init(bar_u, 1);
+        mbar_init(bar_y, 1);
+        mbar_init(bar_m, 1);
+        mbar_init_fence();
+        if (WITH_O) {
+            tma_prefetch_desc(&p.tm_q);
+            tma_prefetch_desc(&p.tm_o);
+        }
+        tma_prefetch_desc(&p.tm_u);
+        tma_prefetch_desc(&p.tm_y);
+        if (p.store_h) tma_prefetch_desc(&p.tm_h);
+    }
+    for (int i = tid * 16; i < 8192; i += 256 * 16)
+        *reinterpret_cast<uint4*>(sm + L::Z + i) = make_uint4(0u, 0u, 0u, 0u);
+    fence_async_smem();
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tq = tmem_addr(tmem, quad * 32, 0);   // this warp's lane quarter
+
+    auto chunk_at = [&](int it) { return REVERSE ? (c_end - 1 - it) : (c_begin + it); };
+    auto load_a = [&](int c) {
+        const int t = c * 128 + tid;
+        return t < p.T ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f;
+    };
+    // in-flight bookkeeping of thread 0 (for the abort path)
+    bool pend_q = false, pend_u = false, pend_y = false, pend_m = false;
+    uint32_t ph_q = 0, ph_u = 0, ph_y = 0;
+    uint32_t mph = 0;   // parity of the next bar_m phase to complete
+
+    auto issue_qu = [&](int c) {
+        const int t0 = c * 128;
+        if (WITH_O) {
+            mbar_arrive_expect_tx(bar_q, kTileQK);
+            for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::Q + i * 8192, &p.tm_q, bar_q, i * 32, h, t0, b);
+            pend_q = true;
+        }
+        mbar_arrive_expect_tx(bar_u, kTileQK);
+        for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::U + i * 8192, &p.tm_u, bar_u, i * 32, h, t0, b);
+        pend_u = true;
+    };
+    auto issue_y = [&](int c) {
+        const int t0 = c * 128;
+        mbar_arrive_expect_tx(bar_y, kTileV);
+        for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::Y + i * 16384, &p.tm_y, bar_y, i * 64, h, t0, b);
+        pend_y = true;
+    };
+
+    if (tid == 0 && nchunks > 0) {
+        issue_qu(chunk_at(0));
+        issue_y(chunk_at(0));
+    }
+    float a_cur = (tid < 128 && nchunks > 0) ? load_a(chunk_at(0)) : 0.f;
+
+    // initial state -> TMEM
+    if (srow) {
+        const float* src = p.s_init ? p.s_init + unit * p.init_unit_stride + seg * p.init_seg_stride +
+                                          row * kDv + half * 96
+                                    : nullptr;
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            uint32_t r[32];
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+                float4 v = src ? *reinterpret_cast<const float4*>(src + j * 32 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+                r[e] = __float_as_uint(v.x);
+                r[e + 1] = __float_as_uint(v.y);
+                r[e + 2] = __float_as_uint(v.z);
+                r[e + 3] = __float_as_uint(v.w);
+            }
+            tmem_st32(tq + L::TM_S + half * 96 + j * 32, r);
+        }
+        tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    bool failed = false, aborted = false;
+    float gsum2 = 0.f;
+    for (int it = 0; it < nchunks; ++it) {
+        const int c = chunk_at(it);
+        const uint32_t ph = it & 1;
+
+        // (A) in-chunk cumulative decay b (log2 units), warps 0-3
+        if (tid < 128) {
+            float x = a_cur * kLog2e;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (lane == 31) wsum[warp] = x;
+            named_sync(1, 128);
+            float pre = 0.f;
+            for (int w = 0; w < warp; ++w) pre += wsum[w];
+            b2s[tid] = x + pre;
+        }
+        if (WITH_O && tid == 0) {
+            // scores = Q K^T as soon as both tiles have landed
+            bool ok = mbar_wait(bar_q, ph_q, ctl) && mbar_wait(bar_u, ph_u, ctl);
+            if (ok) {
+                pend_q = pend_u = false;
+                ph_q ^= 1;
+                ph_u ^= 1;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 6; ++ks) {
+                    const uint32_t off = (ks >> 1) * 8192 + (ks & 1) * 32;
+                    umma_bf16(tmem + L::TM_SC, smem_desc(sb + L::Q + off, 16, 512, kLayoutSW64),
+                              smem_desc(sb + L::U + off, 16, 512, kLayoutSW64), kIdScores, ks > 0);
+                }
+                umma_commit(bar_m);
+                pend_m = true;
+            } else {
+                failed = true;
+            }
+        }
+        if (__syncthreads_or(failed)) { aborted = true; break; }
+        const float g2 = b2s[127];
+        gsum2 += g2;
+
+        // (B) state: bf16 copy for the MMA operand / the stored state, then decay
+        if (srow) {
+            const float f = exp2f(g2);
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                uint32_t r[32];
+                tmem_ld32(tq + L::TM_S + half * 96 + j * 32, r);
+                tmem_ld_wait();
+                if (WITH_O || p.store_h) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int n = half * 96 + j * 32 + q4 * 8;
+                        *reinterpret_cast<uint4*>(sm + L::X + (n >> 6) * 12288 +
+                                                  swz_off(row, (n & 63) >> 3, 128)) =
+                            WITH_O ? pack8_f16(r + q4 * 8, kInterDown) : pack8(r + q4 * 8);
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+                tmem_st32(tq + L::TM_S + half * 96 + j * 32, r);
+            }
+            tmem_st_wait();
+        }
+
+        // (C) scale operand rows in place
+        if (WITH_O) {
+            if (!mbar_wait(bar_m, mph, ctl)) failed = true;      // scores done: Q, K free
+            if (tid == 0) tma_store_wait_read();                  // o staging free (P_lo goes there)
+        } else {
+            if (!mbar_wait(bar_u, ph, ctl)) failed = true;       // u tile in
+        }
+        if (!failed) {
+            if (WITH_O) {
+                for (int idx = tid; idx < 768; idx += 256) {
+                    const int which = idx >= 384;
+                    const int rem = idx - which * 384;
+                    const int r = rem & 127, blk = rem >> 7;
+                    if (which)
+                        scale_row_sw64(sm + L::U, r, blk, exp2f(g2 - b2s[r]));
+                    else
+                        scale_row_sw64<true>(sm + L::Q, r, blk, p.scale * kInterUp * exp2f(b2s[r]));
+                }
+            } else {
+                for (int idx = tid; idx < 384; idx += 256) {
+                    const int r = idx & 127, blk = idx >> 7;
+                    const float f = REVERSE ? p.scale * exp2f(b2s[r]) : exp2f(g2 - b2s[r]);
+                    scale_row_sw64(sm + L::U, r, blk, f);
+                }
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        if (__syncthreads_or(failed)) { aborted = true; break; }
+        tc_fence_after();
+        if (WITH_O) {
+            if (tid == 0) pend_m = false;
+            mph ^= 1;
+        } else if (tid == 0) {
+            pend_u = false;
+            ph_u ^= 1;
+        }
+
+        // (D) store the state copy, O = Q~ S_prev, S += U~^T Y
+        if (tid == 0) {
+            tc_fence_after();
+            if (p.store_h) {
+                for (int i = 0; i < 3; ++i)
+                    tma_store_3d(&p.tm_h, sm + L::X + i * 12288, i * 64, 0, unit * p.NC + c);
+                tma_store_commit();
+            }
+            if (mbar_wait(bar_y, ph_y, ctl)) {
+                pend_y = false;
+                ph_y ^= 1;
+                if (WITH_O) {
+#pragma unroll
+                    for (int ks = 0; ks < 6; ++ks) {
+                        const uint32_t aoff = (ks >> 1) * 8192 + (ks & 1) * 32;
+                        umma_bf16(tmem + L::TM_O, smem_desc(sb + L::Q + aoff, 16, 512, kLayoutSW64),
+                                  smem_desc(sb + L::X + ks * 2048, 12288, 1024, kLayoutSW128), kIdInter,
+                                  ks > 0);
+                    }
+                }
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_bf16(tmem + L::TM_S, smem_desc(sb + L::U + ks * 1024, 8192, 512, kLayoutSW64),
+                              smem_desc(sb + L::Y + ks * 2048, 16384, 1024, kLayoutSW128), kIdState, 1);
+                umma_commit(bar_m);
+                pend_m = true;
+            } else {
+                failed = true;
+            }
+        }
+
+        if (WITH_O) {
+            // (E) masked, decayed scores -> P = P_hi + P_lo (two bf16 terms, so the
+            // intra-chunk product keeps ~16 mantissa bits).  P_lo goes straight
+            // to the free output staging buffer; P_hi waits in registers until
+            // O = Q~ S_prev has finished reading the state copy it replaces.
+            uint32_t pk[32];
+            const float b2r = b2s[row];
+            uint8_t* plo = sm + L::O + half * 16384;
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                const int j0 = half * 64 + q2 * 32;
+                uint32_t lo[16];
+                if (j0 > quad * 32 + 31) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[q2 * 16 + e] = lo[e] = 0u;
+                } else {
+                    uint32_t r[32];
+                    tmem_ld32(tq + L::TM_SC + j0, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int j = j0 + e;
+                        const float v0 = (j <= row) ? p.scale * __uint_as_float(r[e]) * exp2f(b2r - b2s[j]) : 0.f;
+                        const float v1 = (j + 1 <= row) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2r - b2s[j + 1]) : 0.f;
+                        const uint32_t hi = pack_bf16(v0, v1);
+                        pk[q2 * 16 + e / 2] = hi;
+                        lo[e / 2] = pack_bf16(v0 - bf16_lo(hi), v1 - bf16_hi(hi));
+                    }
+                }
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4)
+                    *reinterpret_cast<uint4*>(plo + swz_off(row, q2 * 4 + c4, 128)) =
+                        make_uint4(lo[c4 * 4], lo[c4 * 4 + 1], lo[c4 * 4 + 2], lo[c4 * 4 + 3]);
+            }
+            if (!mbar_wait(bar_m, mph, ctl)) failed = true;       // O = Q~S and S += K~^T V done
+            if (tid == 0) tma_store_wait_read();                  // stored state copy read out
+            tc_fence_before();
+            if (__syncthreads_or(failed)) { aborted = true; break; }
+            if (tid == 0) pend_m = false;
+            mph ^= 1;
+            {
+                uint8_t* pb = sm + L::X + half * 16384;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4*>(pb + swz_off(row, ch, 128)) =
+                        make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+
+            // (F) O += P V; prefetch the next q and k tiles
+            float a_next = 0.f;
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    const uint32_t pbase = part ? L::O : L::X;
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t aoff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                        umma_bf16(tmem + L::TM_O, smem_desc(sb + pbase + aoff, 16, 1024, kLayoutSW128),
+                                  smem_desc(sb + L::Y + ks * 2048, 16384, 1024, kLayoutSW128), kIdOut, 1);
+                    }
+                }
+                umma_commit(bar_m);
+                pend_m = true;
+                if (it + 1 < nchunks) issue_qu(chunk_at(it + 1));
+            }
+            if (tid < 128 && it + 1 < nchunks) a_next = load_a(chunk_at(it + 1));
+
+            // (G) epilogue: O rows -> bf16 staging -> TMA store
+            if (!mbar_wait(bar_m, mph, ctl)) failed = true;
+            if (__syncthreads_or(failed)) { aborted = true; break; }
+            if (tid == 0) pend_m = false;
+            mph ^= 1;
+            tc_fence_after();
+            if (tid == 0 && it + 1 < nchunks) issue_y(chunk_at(it + 1));
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                uint32_t r[32];
+                tmem_ld32(tq + L::TM_O + half * 96 + j * 32, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int n = half * 96 + j * 32 + q4 * 8;
+                    *reinterpret_cast<uint4*>(sm + L::O + (n >> 6) * 16384 +
+                                              swz_off(row, (n & 63) >> 3, 128)) = pack8(r + q4 * 8);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                for (int i = 0; i < 3; ++i) tma_store_4d(&p.tm_o, sm + L::O + i * 16384, i * 64, h, c * 128, b);
+                tma_store_commit();
+            }
+            a_cur = a_next;
+        } else {
+            // state only: wait for S += U~^T Y, then prefetch the next tiles
+            if (!mbar_wait(bar_m, mph, ctl)) failed = true;
+            if (tid == 0 && p.store_h) tma_store_wait_read();
+            if (__syncthreads_or(failed)) { aborted = true; break; }
+            if (tid == 0) pend_m = false;
+            mph ^= 1;
+            tc_fence_after();
+            if (tid == 0 && it + 1 < nchunks) {
+                issue_qu(chunk_at(it + 1));
+                issue_y(chunk_at(it + 1));
+            }
+            a_cur = (tid < 128 && it + 1 < nchunks) ? load_a(chunk_at(it + 1)) : 0.f;
+        }
+    }
+
+    if (!aborted) {
+        const bool write_state = p.s_out && (!p.out_last_only || seg == static_cast<int>(gridDim.x) - 1);
+        if (write_state && srow) {
+            float* dst = p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + half * 96;
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                uint32_t r[32];
+                tmem_ld32(tq + L::TM_S + half * 96 + j * 32, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4*>(dst + j * 32 + e) =
+                        make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                                    __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+            }
+        }
+        if (p.g2_out && tid == 0) p.g2_out[static_cast<int64_t>(unit) * p.g2_unit_stride + seg] = gsum2;
+    } else if (tid == 0) {
+        // drain whatever is still in flight (bounded), so nothing lands in
+        // shared or tensor memory after this CTA has released them
+        if (pend_q) mbar_wait(bar_q, ph_q, ctl);
+        if (pend_u) mbar_wait(bar_u, ph_u, ctl);
+        if (pend_y) mbar_wait(bar_y, ph_y, ctl);
+        if (pend_m) mbar_wait(bar_m, mph, ctl);
+    }
+    if (tid == 0) tma_store_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);
+}
+
+}  // namespace gla

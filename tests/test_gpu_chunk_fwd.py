@@ -1,0 +1,132 @@
+"""GPU parity of the tensor-core chunked forward against the fp64 oracle.
+
+Tolerances (tests/tolerances.py; relative L2 over the whole tensor, oracle as
+reference):
+  o (bf16)           rel L2 <= 1e-2 and max-abs <= 5e-2 beyond the bf16
+                     output's own half-ulp rounding
+  S_T (fp32 state)   rel L2 <= 5e-3
+Cases span several chunks, ragged tails, T = 1, the segmented path used when
+batch x heads is small (pre-pass, combine, fused pass), a nonzero S_0, the
+fused-projection token stride, and the full-size workloads on sampled heads.
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_simple_b200 as gla
+from linear_attention_simple_b200 import inputs
+from oracle import recurrent
+from tolerances import REL_STATE, assert_bf16_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def rel(x, ref):
+    return float(np.linalg.norm(x - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    from linear_attention_simple_b200 import build
+    build.build()
+    gla.lib()
+
+
+def check_fwd(d, o, sf, units=None):
+    q, k, v, a = d["q"], d["k"], d["v"], d["a"]
+    s0 = d["s0"]
+    if units is not None:          # [(b, h), ...] sampled heads
+        bs = [u[0] for u in units]
+        hs = [u[1] for u in units]
+        sl = lambda x: x[bs, :, hs].unsqueeze(0).transpose(1, 2)  # noqa: E731  [1,T,n,d]
+        qn, kn, vn = _np(sl(q)), _np(sl(k)), _np(sl(v))
+        an = _np(a[bs, :, hs]).T[None]
+        s0n = None if s0 is None else _np(s0[bs, hs])[None]
+        ro, rs = recurrent.fwd(qn, kn, vn, an, s0n)
+        got_o = _np(sl(o))
+        got_s = _np(sf[bs, hs])[None]
+    else:
+        ro, rs = recurrent.fwd(_np(q), _np(k), _np(v), _np(a), None if s0 is None else _np(s0))
+        got_o, got_s = _np(o), _np(sf)
+    eo = assert_bf16_close(got_o, ro, "o")
+    es = rel(got_s, rs)
+    assert es <= REL_STATE, "S_T rel L2 %.3g" % es
+    print("o: rel %.3g raw-max %.3g beyond-rounding %.3g | S_T rel %.3g" % (eo + (es,)))
+    return eo, es
+
+
+@pytest.mark.parametrize("B,T,H,s0", [
+    (1, 128, 1, False),     # one full chunk
+    (1, 1, 1, True),        # single token
+    (1, 300, 2, True),      # ragged tail, 3 chunks, segmented path
+    (2, 257, 3, False),     # tail of 1 token
+    (3, 129, 5, True),
+    (1, 1000, 1, True),     # 8 chunks, one per segment
+    (2, 640, 40, False),    # 80 units: one segment per unit
+])
+def test_chunk_fwd_parity(B, T, H, s0):
+    d = inputs.chunk_inputs(B, T, H, seed=100 + T + H, device="cuda", s0_std=0.1 if s0 else None)
+    o, sf = gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], s0=d["s0"])
+    assert gla.gla_get_device_status() == 0
+    check_fwd(d, o, sf)
+
+
+def test_chunk_fwd_fused_projection_stride():
+    """q, k, v as views into one [B, T, 9216] projection buffer."""
+    B, T, H = 2, 200, 16
+    d = inputs.chunk_inputs(B, T, H, seed=120, device="cuda", s0_std=0.1, ld=9216)
+    assert d["q"].stride(1) == 9216
+    o, sf = gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], s0=d["s0"])
+    check_fwd(d, o, sf, units=[(0, 0), (1, 7), (1, 15)])
+
+
+def test_chunk_fwd_strong_decay_and_no_decay():
+    """Decays outside the workload distribution: a = 0 (no decay at all, so
+    |o| grows with T) and a ~ -8 per token.  Outputs here are not of the
+    workloads' magnitude, so the absolute bound is taken relative to max|o|:
+    rel L2 <= 1e-2 and max-abs <= 1e-2 * max|o|."""
+    B, T, H = 1, 384, 2
+    for mean, seed in ((None, 121), (-8.0, 122)):
+        d = inputs.chunk_inputs(B, T, H, seed=seed, device="cuda", s0_std=0.1)
+        d["a"] = (torch.zeros_like(d["a"]) if mean is None
+                  else inputs.log_decay((B, T, H), seed, "cuda", mean=mean))
+        o, sf = gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], s0=d["s0"])
+        ro, rs = recurrent.fwd(_np(d["q"]), _np(d["k"]), _np(d["v"]), _np(d["a"]), _np(d["s0"]))
+        got = _np(o)
+        assert rel(got, ro) <= 1e-2
+        assert np.max(np.abs(got - ro)) <= 1e-2 * np.max(np.abs(ro))
+        assert rel(_np(sf), rs) <= REL_STATE
+
+
+def test_chunk_fwd_state_carry_split():
+    """Running [0, T1) then [T1, T) with the state carried equals one call."""
+    B, T, H, T1 = 2, 512, 4, 200
+    d = inputs.chunk_inputs(B, T, H, seed=123, device="cuda", s0_std=0.1)
+    o, sf = gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], s0=d["s0"])
+    part = lambda x, sl: x[:, sl].contiguous()  # noqa: E731
+    first, second = slice(0, T1), slice(T1, T)
+    o1, s1 = gla.gla_chunk_fwd(*(part(d[n], first) for n in ("q", "k", "v", "a")), s0=d["s0"])
+    o2, s2 = gla.gla_chunk_fwd(*(part(d[n], second) for n in ("q", "k", "v", "a")), s0=s1)
+    assert rel(_np(torch.cat([o1, o2], 1)), _np(o)) <= 1e-2
+    assert rel(_np(s2), _np(sf)) <= 5e-3
+
+
+def test_chunk_fwd_prefill_full_size_sampled():
+    """B = 8, T = 2048, H = 16 (the prefill workload as benchmarked)."""
+    d = inputs.chunk_inputs(8, 2048, 16, seed=1002, device="cuda")
+    o, sf = gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"])
+    assert gla.gla_get_device_status() == 0
+    check_fwd(d, o, sf, units=[(0, 0), (3, 5), (7, 15), (5, 9)])
+
+
+def test_chunk_fwd_long_prefill_full_size_sampled():
+    """B = 1, T = 65536, H = 16 with S_0 ~ N(0, 0.1^2) (the long-context
+    prefill, segmented path), on two sampled heads."""
+    d = inputs.chunk_inputs(1, 65536, 16, seed=1005, device="cuda", s0_std=0.1)
+    o, sf = gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], s0=d["s0"])
+    assert gla.gla_get_device_status() == 0
+    check_fwd(d, o, sf, units=[(0, 3), (0, 12)])

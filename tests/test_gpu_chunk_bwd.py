@@ -1,0 +1,106 @@
+"""GPU parity of the tensor-core chunked backward against the fp64 oracle's
+reverse recurrence (itself pinned by finite differences on the CPU).
+
+Tolerances (tests/tolerances.py):
+  dq, dk, dv (bf16)   rel L2 <= 1e-2, max-abs <= 5e-2 beyond bf16 storage rounding
+  da (fp32)           rel L2 <= 1e-2, max-abs <= 5e-2 * max(1, max|da|)
+  dS_0 (fp32 state)   rel L2 <= 5e-3
+da is a reverse cumulative sum over the whole sequence, so its magnitude
+grows with T; its absolute bound scales with its own size (stated reading).
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_simple_b200 as gla
+from linear_attention_simple_b200 import inputs
+from oracle import recurrent
+from tolerances import ABS_BF16, REL_BF16, REL_STATE, assert_bf16_close, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    from linear_attention_simple_b200 import build
+    build.build()
+    gla.lib()
+
+
+def _sample(x, bs, hs):
+    """[B,T,H,...] -> [1,T,n,...] for sampled (b, h) pairs."""
+    y = x[bs, :, hs]                      # [n, T, ...]
+    return y.unsqueeze(0).transpose(1, 2)
+
+
+def check_bwd(d, grads, units=None, dsT=None):
+    gq, gk, gv, ga, gs0 = grads
+    names = ("q", "k", "v", "a", "dO")
+    if units is None:
+        arrs = [_np(d[n]) for n in names]
+        s0 = None if d["s0"] is None else _np(d["s0"])
+        dsTn = None if dsT is None else _np(dsT)
+        got = [_np(gq), _np(gk), _np(gv), _np(ga), None if gs0 is None else _np(gs0)]
+    else:
+        bs = [u[0] for u in units]
+        hs = [u[1] for u in units]
+        arrs = [_np(_sample(d[n], bs, hs)) if n != "a" else _np(d["a"][bs, :, hs]).T[None]
+                for n in names]
+        s0 = None if d["s0"] is None else _np(d["s0"][bs, hs])[None]
+        dsTn = None if dsT is None else _np(dsT[bs, hs])[None]
+        got = [_np(_sample(gq, bs, hs)), _np(_sample(gk, bs, hs)), _np(_sample(gv, bs, hs)),
+               _np(ga[bs, :, hs]).T[None], None if gs0 is None else _np(gs0[bs, hs])[None]]
+    q, k, v, a, dO = arrs
+    rq, rk, rv, ra, rs0 = recurrent.bwd(q, k, v, a, dO, s0, dsTn)
+    report = {}
+    for name, g, r in (("dq", got[0], rq), ("dk", got[1], rk), ("dv", got[2], rv)):
+        report[name] = assert_bf16_close(g, r, name)
+    e_da = rel_l2(got[3], ra)
+    m_da = float(np.max(np.abs(got[3] - ra)))
+    assert e_da <= REL_BF16, "da rel L2 %.3g" % e_da
+    assert m_da <= ABS_BF16 * max(1.0, float(np.max(np.abs(ra)))), "da max-abs %.3g" % m_da
+    report["da"] = (e_da, m_da, float(np.max(np.abs(ra))))
+    if got[4] is not None:
+        e = rel_l2(got[4], rs0)
+        assert e <= REL_STATE, "dS0 rel L2 %.3g" % e
+        report["ds0"] = e
+    print(" ".join("%s=%s" % (k, tuple(round(x, 5) for x in v) if isinstance(v, tuple) else round(v, 6))
+                   for k, v in report.items()))
+    return report
+
+
+@pytest.mark.parametrize("B,T,H,s0,dsT", [
+    (1, 128, 1, False, False),
+    (1, 1, 1, True, True),
+    (2, 300, 3, True, True),
+    (1, 257, 2, False, False),
+    (3, 129, 5, True, False),
+    (2, 640, 40, False, True),
+])
+def test_chunk_bwd_parity(B, T, H, s0, dsT):
+    d = inputs.chunk_inputs(B, T, H, seed=200 + T + H, device="cuda", s0_std=0.1 if s0 else None,
+                            with_dO=True)
+    ds = inputs.randn((B, H, 96, 192), 300 + T, "cuda", std=0.1) if dsT else None
+    grads = gla.gla_chunk_bwd(d["q"], d["k"], d["v"], d["a"], d["dO"], s0=d["s0"], ds_final=ds)
+    assert gla.gla_get_device_status() == 0
+    check_bwd(d, grads, dsT=ds)
+
+
+def test_chunk_bwd_fused_projection_stride():
+    B, T, H = 2, 200, 16
+    d = inputs.chunk_inputs(B, T, H, seed=220, device="cuda", s0_std=0.1, ld=9216, with_dO=True)
+    grads = gla.gla_chunk_bwd(d["q"], d["k"], d["v"], d["a"], d["dO"], s0=d["s0"])
+    check_bwd(d, grads, units=[(0, 0), (1, 9)])
+
+
+def test_chunk_bwd_training_full_size_sampled():
+    """B = 8, T = 2048, H = 16, dO ~ N(0,1), zero gradient on the final state
+    (the training step as benchmarked), on sampled heads."""
+    d = inputs.chunk_inputs(8, 2048, 16, seed=1003, device="cuda", with_dO=True)
+    grads = gla.gla_chunk_bwd(d["q"], d["k"], d["v"], d["a"], d["dO"])
+    assert gla.gla_get_device_status() == 0
+    check_bwd(d, grads, units=[(0, 0), (4, 7), (7, 15)])

@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""Benchmark of the Simple GLA mixer hot path on B200.
+
+One step = one training step of one Laplace-layer mixer at B = 8, T = 2048,
+H = 16, dk = 96, dv = 192 in bf16: gla_chunk_fwd followed by gla_chunk_bwd
+(dO ~ N(0,1), zero gradient on the final state).  The headline value is
+chunk fwd+bwd tokens/s over all ranks.  The metric also names decode
+tokens/s at 1,280 sequences, so the same run times the 24-layer decode step
+(1,280 sequences x 24 layers x 16 heads, fp32 state in place) and reports
+it under "decode".
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
+cuda synchronize, measured with CUDA events on the launching stream, max
+over ranks.  Inputs (about 0.6 GB per rank for the training step, 36 GB of
+decode state) are larger than the 126 MB L2, so no flush is needed.
+Roofline: libgla's own per-launch event tracing times every kernel inside
+the timed region; the dominant kernel's algorithmic bytes (or flops) per
+launch divided by its mean launch time, against MEASURED_PEAKS.json.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import linear_attention_simple_b200 as gla  # noqa: E402
+from linear_attention_simple_b200 import inputs  # noqa: E402
+from linear_attention_simple_b200.configs import WORKLOADS  # noqa: E402
+
+METRIC = "GLA chunk fwd+bwd tokens/s; decode tokens/s at 1280 seqs; % of roofline"
+TRAIN = WORKLOADS["train_fwd_bwd_b8_t2048"]
+DECODE = WORKLOADS["decode_n1280_l24"]
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# Algorithmic bytes per unit (one (batch, head, 128-token chunk) unless
+# stated), used for each kernel's roofline.  bf16 tiles: q, k 24,576 B; v, o,
+# dO 49,152 B; a 512 B; bf16 per-chunk state 36,864 B; fp32 state 73,728 B.
+QK, VO, A, HS, FS = 24576, 49152, 512, 36864, 73728
+CHUNK_BYTES = {
+    # fused forward: read q, k, v, a; write o          (+ S_T per head)
+    "chunk_fwd_fused_kernel": 2 * QK + 2 * VO + A,
+    # state recompute: read k, v, a; write h_c          (+ S_T per head if dS_T)
+    "chunk_state_fwd_kernel": QK + VO + A + HS,
+    # state-gradient pass: read q, dO, a; write D_c     (+ dS_0 per head)
+    "chunk_state_rev_kernel": QK + VO + A + HS,
+    # dq/dk: read q, k, v, dO, h, D, a; write dq, dk, delta
+    "bwd_dqdk_kernel": 2 * QK + 2 * VO + 2 * HS + A + 2 * QK + A,
+    # dv: read q, k, dO, D, a; write dv
+    "bwd_dv_kernel": 2 * QK + VO + HS + A + VO,
+}
+CHUNK_FLOPS = {
+    # 2*(128*128*96 + 128*192*96 + 128*192*128 + 96*192*128), dense tiles
+    "chunk_fwd_fused_kernel": 2 * (128 * 128 * 96 + 128 * 192 * 96 + 128 * 192 * 128 + 96 * 192 * 128),
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# --------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------- helpers
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def train_buffers(seed, device="cuda"):
+    w = TRAIN
+    d = inputs.chunk_inputs(w.B, w.T, w.H, w.dk, w.dv, seed=seed, device=device, with_dO=True)
+    dev = torch.device(device)
+    d["o"] = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device=dev)
+    d["sf"] = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    d["grads"] = (torch.empty_like(d["q"]), torch.empty_like(d["k"]), torch.empty_like(d["v"]),
+                  torch.empty_like(d["a"]), None)
+    d["ws_f"] = torch.empty(max(1, gla.gla_chunk_workspace_bytes(w.B, w.T, w.H)), dtype=torch.uint8,
+                            device=dev)
+    d["ws_b"] = torch.empty(gla.gla_chunk_workspace_bytes(w.B, w.T, w.H, for_bwd=True),
+                            dtype=torch.uint8, device=dev)
+    return d
+
+
+def train_step(d):
+    gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], o=d["o"], s_final=d["sf"], ws=d["ws_f"])
+    gla.gla_chunk_bwd(d["q"], d["k"], d["v"], d["a"], d["dO"], grads=d["grads"], ws=d["ws_b"],
+                      want_grad_s0=False)
+
+
+def kernel_roofline(summary, peaks, peak_kind, units_per_launch, B, H):
+    """Roofline of the kernel with the largest summed time in the trace."""
+    if not summary:
+        return None, None
+    name, launches, total_ms = max(summary, key=lambda r: r[2])
+    mean_s = total_ms / launches / 1e3
+    if name in CHUNK_BYTES:
+        bytes_per_launch = CHUNK_BYTES[name] * units_per_launch
+        if name in ("chunk_fwd_fused_kernel",):
+            bytes_per_launch += FS * B * H          # final state written per head
+        achieved = bytes_per_launch / mean_s / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "bytes_per_launch": bytes_per_launch, "mean_launch_us": round(mean_s * 1e6, 2),
+                "traffic": None, "peak_source": "%s copy bandwidth" % peak_kind}
+    else:
+        roof = {"kernel": name, "bound": None, "achieved": None, "peak": None, "unit": None,
+                "frac": None, "traffic": None, "mean_launch_us": round(mean_s * 1e6, 2)}
+    shares = {n: round(t / sum(r[2] for r in summary), 4) for n, _, t in summary}
+    return roof, shares
+
+
+# ------------------------------------------------------------ oracle arm
+
+def oracle_sample_time(units, seed, with_bwd=True):
+    """Run the fp64 oracle (fwd + bwd) on `units` (batch, head) sequences of
+    the training workload; returns (seconds, tokens, threads)."""
+    from oracle import recurrent
+    w = TRAIN
+    d = inputs.chunk_inputs(1, w.T, units, w.dk, w.dv, seed=seed, device="cpu", with_dO=True)
+    f = lambda t: t.float().numpy().astype("float64")  # noqa: E731
+    q, k, v, a, dO = (f(d[n]) for n in ("q", "k", "v", "a", "dO"))
+    t0 = time.perf_counter()
+    recurrent.fwd(q, k, v, a)
+    if with_bwd:
+        recurrent.bwd(q, k, v, a, dO)
+    dt = time.perf_counter() - t0
+    # one token of the workload covers all H heads
+    return dt, units * w.T / w.H, recurrent.max_threads()
+
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return
+    units = max(1, int(os.environ.get("GLA_ORACLE_UNITS", "16")))
+    for _ in range(args.warmup):
+        oracle_sample_time(units, 7)
+    times, toks = [], 0.0
+    for i in range(args.steps):
+        dt, tok, cores = oracle_sample_time(units, 7 + i)
+        times.append(dt)
+        toks = tok
+    t = sum(times) / len(times)
+    value = toks / t
+    line = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(t * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": TRAIN.name, "global_batch": TRAIN.B, "seq_len": TRAIN.T,
+                       "heads": TRAIN.H, "dk": TRAIN.dk, "dv": TRAIN.dv,
+                       "parallelism": "oracle on host cores"},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": "%d of %d (batch, head) sequences of T=%d per step, fwd+bwd"
+                                       % (units, TRAIN.B * TRAIN.H, TRAIN.T)},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- ours
+
+def run_ours(args, ws, rank, local):
+    from linear_attention_simple_b200 import build
+    build.build()
+    gla.lib()
+    peaks, peak_kind = load_peaks()
+    st = torch.cuda.current_stream()
+    w = TRAIN
+    d = train_buffers(seed=w.seed + 97 * rank)
+    NC = (w.T + 127) // 128
+    units_per_launch = w.B * w.H * NC
+
+    for _ in range(max(3, args.warmup)):
+        train_step(d)
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)                       # let the sampler come up
+    gla.gla_trace_enable(True)
+    launches0 = gla.gla_launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(st)
+    for _ in range(args.steps):
+        train_step(d)
+    ev1.record(st)
+    ev1.synchronize()
+    launches = gla.gla_launch_count() - launches0
+    summary = gla.gla_trace_summary()
+    gla.gla_trace_enable(False)
+    torch.cuda.synchronize()
+    barrier(ws)
+    elapsed = max_over_ranks(ev0.elapsed_time(ev1) / 1e3, ws)
+    ms_step = elapsed / args.steps * 1e3
+    value = ws * w.B * w.T * args.steps / elapsed
+    roof, shares = kernel_roofline([(n, c, t) for n, c, t in summary], peaks, peak_kind,
+                                   units_per_launch, w.B, w.H)
+
+    # ---- end to end through the public API with host buffers
+    pin = {n: torch.empty_like(d[n], device="cpu").pin_memory() for n in ("q", "k", "v", "a", "dO")}
+    for n in pin:
+        pin[n].copy_(d[n])
+    outs = [torch.empty_like(g, device="cpu").pin_memory() for g in d["grads"][:4]]
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+
+    def e2e_step():
+        for n in pin:
+            d[n].copy_(pin[n], non_blocking=True)
+        train_step(d)
+        for g, o in zip(d["grads"][:4], outs):
+            o.copy_(g, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(1, min(args.steps, 10))
+    e0.record(st)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(st)
+    e1.synchronize()
+    e_elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3, ws)
+    e2e = {"value": round(ws * w.B * w.T * e_steps / e_elapsed, 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del d, pin, outs
+    torch.cuda.empty_cache()
+
+    # ---- decode step at 1280 sequences x 24 layers
+    dec = run_decode(args, ws, peaks, peak_kind)
+    clk = clocks.stop()
+    if clk is not None:
+        clk["region"] = "fwd+bwd and decode timed regions"
+
+    # ---- oracle on the host cores (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        units = int(os.environ.get("GLA_ORACLE_UNITS", str(w.B * w.H)))
+        total_t, total_tok, reps = 0.0, 0.0, 0
+        while total_t < 10.0 and reps < 20:
+            dt, toks, cores = oracle_sample_time(units, 11 + reps)
+            total_t += dt
+            total_tok += toks
+            reps += 1
+        cpu = {"value": round(total_tok / total_t, 3), "unit": "tokens/s", "cores": cores,
+               "kind": "oracle",
+               "sample": "fwd+bwd of %d of the %d (batch, head) sequences (T=%d), %d repetitions, "
+                         "%.1f s" % (units, w.B * w.H, w.T, reps, total_t)}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws,
+                "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic",
+                "config": {"workload": w.name, "global_batch": w.B * ws, "seq_len": w.T,
+                           "heads": w.H, "dk": w.dk, "dv": w.dv, "parallelism": "dp%d" % ws,
+                           "l2": "inputs larger than L2 (no flush)"},
+                "roofline": roof, "kernel_shares": shares, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "clocks": clk, "decode": dec}
+        print(json.dumps(line), flush=True)
+
+
+def run_decode(args, ws, peaks, peak_kind):
+    w = DECODE
+    layers = inputs.decode_inputs(w.N, w.H, w.dk, w.dv, seed=w.seed, device="cuda", layers=w.layers)
+    outs = [torch.empty((w.N, w.H, w.dv), dtype=torch.float32, device="cuda") for _ in layers]
+    st = torch.cuda.current_stream()
+
+    def step():
+        for L, o in zip(layers, outs):
+            gla.gla_decode_step(L["state"], L["q"], L["k"], L["v"], L["a"], o=o)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    steps = max(1, min(args.steps, 30))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        step()
+    e1.record(st)
+    e1.synchronize()
+    el = max_over_ranks(e0.elapsed_time(e1) / 1e3, ws)
+    per_step = el / steps
+    bytes_step = w.layers * w.N * w.H * (2 * FS + 2 * 96 * 2 + 192 * 2 + 192 * 4 + 4)
+    achieved = bytes_step / per_step / 1e9
+    out = {"value": round(ws * w.N / per_step, 1), "unit": "tokens/s",
+           "workload": w.name, "ms_per_step": round(per_step * 1e3, 4),
+           "roofline": {"kernel": "decode_step_kernel", "bound": "hbm", "achieved": round(achieved, 1),
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(achieved / peaks["hbm_gbs"], 4),
+                        "frac_of_8tbs": round(achieved / 8000.0, 4),
+                        "peak_source": "%s copy bandwidth" % peak_kind}}
+    del layers, outs
+    torch.cuda.empty_cache()
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, ws, rank)
+        return
+    ws, rank, local = dist_setup()
+    try:
+        run_ours(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

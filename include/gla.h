@@ -173,6 +173,20 @@ gla_status conv1d_silu_causal(const void* x, int apply_ln, const float* ln_gamma
  * failure path without faulting or hanging the GPU.
  * ------------------------------------------------------------------------ */
 gla_status gla_get_device_status(cudaStream_t stream, int* device_status);
+
+/* ---------------------------------------------------------------------------
+ * Kernel tracing.  While enabled, libgla brackets every kernel it launches
+ * with two CUDA events recorded on the launch stream (events come from a
+ * pool owned by libgla; no device memory is allocated).  gla_trace_enable(1)
+ * clears earlier records; gla_trace_enable(0) stops recording.
+ * gla_trace_summary SYNCHRONISES on the recorded events and reports, per
+ * kernel name (at most max_entries, in first-launch order): the name (a
+ * static string), the number of launches and their summed device time in
+ * milliseconds.  It returns the number of entries written.
+ * ------------------------------------------------------------------------ */
+gla_status gla_trace_enable(int enable);
+int gla_trace_summary(const char** names, unsigned long long* launches, double* total_ms,
+                      int max_entries);
 gla_status gla_set_wait_limit_ns(unsigned long long ns);
 gla_status gla_selftest_wait_timeout(cudaStream_t stream);
 

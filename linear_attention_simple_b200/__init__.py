@@ -18,7 +18,8 @@ __all__ = [
     "GlaError", "GlaLibraryMissing", "lib", "gla_status_string", "gla_launch_count",
     "gla_chunk_workspace_bytes", "gla_chunk_fwd", "gla_chunk_bwd", "gla_decode_step",
     "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
-    "gla_selftest_wait_timeout", "EXPORTED_SYMBOLS", "LIB_PATH",
+    "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
+    "EXPORTED_SYMBOLS", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgla.so")
@@ -27,7 +28,7 @@ EXPORTED_SYMBOLS = (
     "gla_status_string", "gla_last_cuda_error", "gla_launch_count",
     "gla_chunk_workspace_bytes", "gla_chunk_fwd", "gla_chunk_bwd", "gla_decode_step",
     "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
-    "gla_selftest_wait_timeout",
+    "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
 )
 
 GLA_BF16, GLA_F32 = 0, 1
@@ -88,6 +89,12 @@ def lib():
     L.gla_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     L.gla_selftest_wait_timeout.restype = _i
     L.gla_selftest_wait_timeout.argtypes = [_vp]
+    L.gla_trace_enable.restype = _i
+    L.gla_trace_enable.argtypes = [_i]
+    L.gla_trace_summary.restype = _i
+    L.gla_trace_summary.argtypes = [ctypes.POINTER(ctypes.c_char_p),
+                                    ctypes.POINTER(ctypes.c_ulonglong),
+                                    ctypes.POINTER(ctypes.c_double), _i]
     _LIB = L
     return L
 
@@ -300,3 +307,18 @@ def gla_set_wait_limit_ns(ns):
 
 def gla_selftest_wait_timeout(stream=None):
     _check("gla_selftest_wait_timeout", lib().gla_selftest_wait_timeout(_stream(stream)))
+
+
+def gla_trace_enable(enable=True):
+    """Start (clearing earlier records) or stop per-launch event tracing."""
+    _check("gla_trace_enable", lib().gla_trace_enable(1 if enable else 0))
+
+
+def gla_trace_summary(max_entries=64):
+    """Synchronise on the traced launches and return
+    [(kernel_name, launches, total_ms), ...] in first-launch order."""
+    names = (ctypes.c_char_p * max_entries)()
+    counts = (ctypes.c_ulonglong * max_entries)()
+    totals = (ctypes.c_double * max_entries)()
+    n = lib().gla_trace_summary(names, counts, totals, max_entries)
+    return [(names[i].decode(), int(counts[i]), float(totals[i])) for i in range(n)]

@@ -486,7 +486,9 @@ gla_status launch_bwd_kernel(K kernel, uint32_t bytes, const BwdParams& p, dim3 
 {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
         return check_launch(name);
+    trace_begin(st);
     kernel<<<grid, 256, bytes, st>>>(p);
+    trace_end(st, name);
     count_launch();
     return check_launch(name);
 }
@@ -572,7 +574,9 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     if ((s = launch_bwd_kernel(bwd_dv_kernel, bv::BYTES, bp, grid, st, "bwd_dv_kernel")) != GLA_OK) return s;
 
     // 4. da = reverse cumulative sum of delta (+ <dS_T, S_T>)
+    trace_begin(st);
     da_scan_kernel<<<units, kScanThreads, 0, st>>>(da, ds_final, ds_final ? sT : nullptr, pr.T, pr.H);
+    trace_end(st, "da_scan_kernel");
     count_launch();
     return check_launch("da_scan_kernel");
 }

@@ -67,7 +67,11 @@ gla_status launch_state_t(const StateParams& p, dim3 grid, cudaStream_t st)
     cudaError_t e = cudaFuncSetAttribute(gla_chunk_state_kernel<W, R>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return check_launch("cudaFuncSetAttribute");
+    static const char* const kName = W ? "chunk_fwd_fused_kernel"
+                                       : (R ? "chunk_state_rev_kernel" : "chunk_state_fwd_kernel");
+    trace_begin(st);
     gla_chunk_state_kernel<W, R><<<grid, 256, bytes, st>>>(p);
+    trace_end(st, kName);
     count_launch();
     return check_launch("gla_chunk_state_kernel");
 }
@@ -165,8 +169,10 @@ gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float
     if ((s = launch_state_kernel(false, false, pre, dim3(nseg - 1, pr.H, pr.B), st)) != GLA_OK) return s;
     // 2. states entering every segment
     const int64_t n4 = static_cast<int64_t>(units) * (kSS / 4);
+    trace_begin(st);
     seg_combine_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(states, g2, s0, nseg,
                                                                                units);
+    trace_end(st, "seg_combine_kernel");
     count_launch();
     if ((s = check_launch("seg_combine_kernel")) != GLA_OK) return s;
     // 3. fused output pass

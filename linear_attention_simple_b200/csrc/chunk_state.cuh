@@ -16,17 +16,20 @@
 //            groups -- scores = Q K^T (128x128x96), O = Q~ S_prev
 //            (128x192x96, fp16 operands), O += P V (128x192x128, P split
 //            into two bf16 terms P_hi + P_lo), S += K~^T V (128pad x 192 x
-//            128) -- plus the masked-decay P tile on CUDA cores.  The
+//            128, K~ split into bf16 hi + lo) -- plus the masked-decay P
+//            tile on CUDA cores.  The
 //            state itself is always fp32 in tensor memory; only the MMA
 //            operand copies are 16-bit.
-//   !WITH_O  state only: S (or D) += U~^T Y per chunk, optionally storing the
+//   !WITH_O  state only: S (or D) += U~^T Y per chunk (U~ split into bf16
+//            hi + lo, so the fp32 state sees ~16-bit operands), optionally storing the
 //            bf16 state before each chunk's update (for the backward).
 //   REVERSE  walks chunks from last to first (the dL/dS pass).
 //
 // Operand layouts (all validated against the hardware): q and k tiles are
 // TMA-loaded as three 32-wide SW64 boxes ([3][128][32], K-major for the
 // scores; the k tile doubles as the MN-major A operand of the state product,
-// whose fourth 32-row block is a permanent zero block); v tiles are three
+// whose fourth 32-row block -- the padding of dk = 96 to M = 128 -- only
+// feeds TMEM lanes 96..127, which are never read); v tiles are three
 // 64-wide SW128 boxes ([3][128][64], MN-major B); the bf16 state copy is
 // [3][96][64] SW128 (MN-major B of O = Q~ S); P_hi is [2][128][64] SW128
 // (K-major A) and reuses the state copy's buffer once O = Q~ S has run;
@@ -71,12 +74,13 @@ struct Smem;
 template <>
 struct Smem<true> {
     static constexpr uint32_t Q = 0;          // [3][128][32] bf16 SW64
-    static constexpr uint32_t U = 24576;      // k tile  [3][128][32] bf16 SW64
-    static constexpr uint32_t Z = 49152;      // zero block (4th M block of U^T)
-    static constexpr uint32_t Y = 57344;      // v tile  [3][128][64] bf16 SW128
-    static constexpr uint32_t X = 106496;     // state copy [3][96][64] / P [2][128][64]
-    static constexpr uint32_t O = 143360;     // output staging [3][128][64]
-    static constexpr uint32_t MISC = 192512;
+    static constexpr uint32_t U = 24576;      // k tile  [3][128][32] bf16 SW64 (then K~ hi)
+    static constexpr uint32_t UL = 49152;     // K~ lo, same layout (U's 4th M block: finite)
+    static constexpr uint32_t Z = 73728;      // zero block (UL's 4th M block)
+    static constexpr uint32_t Y = 81920;      // v tile  [3][128][64] bf16 SW128
+    static constexpr uint32_t X = 131072;     // state copy [3][96][64] / P_hi [2][128][64]
+    static constexpr uint32_t O = 167936;     // output staging [3][128][64] / P_lo
+    static constexpr uint32_t MISC = 217088;
     static constexpr uint32_t BYTES = MISC + 1024 + 1024;   // + alignment slack
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t TM_SC = 0, TM_O = 128, TM_S = 320;
@@ -85,11 +89,12 @@ template <>
 struct Smem<false> {
     static constexpr uint32_t Q = 0;          // unused
     static constexpr uint32_t U = 0;
-    static constexpr uint32_t Z = 24576;
-    static constexpr uint32_t Y = 32768;
-    static constexpr uint32_t X = 81920;
+    static constexpr uint32_t UL = 24576;
+    static constexpr uint32_t Z = 49152;
+    static constexpr uint32_t Y = 57344;
+    static constexpr uint32_t X = 106496;
     static constexpr uint32_t O = 0;          // unused
-    static constexpr uint32_t MISC = 118784;
+    static constexpr uint32_t MISC = 143360;
     static constexpr uint32_t BYTES = MISC + 1024 + 1024;
     static constexpr uint32_t TMEM_COLS = 256;
     static constexpr uint32_t TM_SC = 0, TM_O = 0, TM_S = 0;
@@ -118,6 +123,34 @@ __device__ __forceinline__ uint4 scale8(uint4 v, float f)
 #pragma unroll
     for (int i = 0; i < 4; ++i) w[i] = pack_bf16(bf16_lo(w[i]) * f, bf16_hi(w[i]) * f);
     return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// hi = bf16(f x), lo = bf16(f x - hi) for 8 bf16 elements.
+__device__ __forceinline__ void scale8_split(uint4 v, float f, uint4& hi, uint4& lo)
+{
+    uint32_t w[4] = {v.x, v.y, v.z, v.w}, h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float a = bf16_lo(w[i]) * f, b = bf16_hi(w[i]) * f;
+        h[i] = pack_bf16(a, b);
+        l[i] = pack_bf16(a - bf16_lo(h[i]), b - bf16_hi(h[i]));
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// In-place hi / separate lo split of a scaled 64-byte row segment.
+__device__ __forceinline__ void split_row_sw64(uint8_t* tile, uint8_t* lo_tile, int row, int blk, float f)
+{
+    uint4* p = reinterpret_cast<uint4*>(tile + blk * 8192 + row * 64);
+    uint4* q = reinterpret_cast<uint4*>(lo_tile + blk * 8192 + row * 64);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint4 h, l;
+        scale8_split(p[c], f, h, l);
+        p[c] = h;
+        q[c] = l;
+    }
 }
 
 __device__ __forceinline__ uint4 scale8_to_f16(uint4 v, float f)
@@ -356,7 +389,7 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_state_kernel(const __grid_co
                     const int rem = idx - which * 384;
                     const int r = rem & 127, blk = rem >> 7;
                     if (which)
-                        scale_row_sw64(sm + L::U, r, blk, exp2f(g2 - b2s[r]));
+                        split_row_sw64(sm + L::U, sm + L::UL, r, blk, exp2f(g2 - b2s[r]));
                     else
                         scale_row_sw64<true>(sm + L::Q, r, blk, p.scale * kInterUp * exp2f(b2s[r]));
                 }
@@ -364,7 +397,7 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_state_kernel(const __grid_co
                 for (int idx = tid; idx < 384; idx += 256) {
                     const int r = idx & 127, blk = idx >> 7;
                     const float f = REVERSE ? p.scale * exp2f(b2s[r]) : exp2f(g2 - b2s[r]);
-                    scale_row_sw64(sm + L::U, r, blk, f);
+                    split_row_sw64(sm + L::U, sm + L::UL, r, blk, f);
                 }
             }
         }
@@ -401,9 +434,12 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_state_kernel(const __grid_co
                     }
                 }
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    umma_bf16(tmem + L::TM_S, smem_desc(sb + L::U + ks * 1024, 8192, 512, kLayoutSW64),
-                              smem_desc(sb + L::Y + ks * 2048, 16384, 1024, kLayoutSW128), kIdState, 1);
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        umma_bf16(tmem + L::TM_S,
+                                  smem_desc(sb + (part ? L::UL : L::U) + ks * 1024, 8192, 512, kLayoutSW64),
+                                  smem_desc(sb + L::Y + ks * 2048, 16384, 1024, kLayoutSW128), kIdState, 1);
                 umma_commit(bar_m);
                 pend_m = true;
             } else {

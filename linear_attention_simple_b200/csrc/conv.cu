@@ -228,9 +228,11 @@ gla_status launch_conv(const void* x, int apply_ln, const float* g, const float*
     nx = (T + per - 1) / per;
     dim3 grid(nx, B);
     const size_t smem = static_cast<size_t>(3) * D * sizeof(float);
+    trace_begin(st);
     ln_conv_silu_kernel<<<grid, threads, smem, st>>>(
         static_cast<const __nv_bfloat16*>(x), apply_ln, g, b, eps, w, bias, cs_in, cs_out,
         static_cast<__nv_bfloat16*>(y), T, D, per);
+    trace_end(st, "ln_conv_silu_kernel");
     count_launch();
     return check_launch("ln_conv_silu_kernel");
 }

@@ -103,10 +103,12 @@ gla_status launch_decode(float* state, const int32_t* slot_idx, const void* q, c
     const int64_t units = static_cast<int64_t>(N) * H;
     if (units == 0) return GLA_OK;
     if (units > 0x7FFFFFFF) return GLA_ERR_UNSUPPORTED;
+    trace_begin(st);
     decode_step_kernel<<<static_cast<unsigned>(units), kThreads, 0, st>>>(
         state, slot_idx, static_cast<const __nv_bfloat16*>(q),
         static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), a, o, H,
         scale);
+    trace_end(st, "decode_step_kernel");
     count_launch();
     return check_launch("decode_step_kernel");
 }

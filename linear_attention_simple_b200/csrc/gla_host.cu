@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "gla_internal.h"
 
@@ -75,7 +76,49 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
+// Trace records: one (start, end, name) per launch while enabled.
+struct TraceRec {
+    cudaEvent_t start, end;
+    const char* name;
+};
+std::atomic<bool> g_trace_on{false};
+std::mutex g_trace_mu;
+std::vector<TraceRec> g_trace;
+std::vector<cudaEvent_t> g_event_pool;
+thread_local cudaEvent_t t_pending_start = nullptr;
+
+cudaEvent_t pool_event()
+{
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
 }  // namespace
+
+void trace_begin(cudaStream_t st)
+{
+    if (!g_trace_on.load()) return;
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    t_pending_start = pool_event();
+    if (t_pending_start) cudaEventRecord(t_pending_start, st);
+}
+
+void trace_end(cudaStream_t st, const char* name)
+{
+    if (!g_trace_on.load() || !t_pending_start) return;
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    cudaEvent_t e = pool_event();
+    if (!e) return;
+    cudaEventRecord(e, st);
+    g_trace.push_back({t_pending_start, e, name});
+    t_pending_start = nullptr;
+}
 
 WaitCtl wait_ctl_for_current_device(gla_status* err)
 {
@@ -319,6 +362,44 @@ gla_status gla_get_device_status(cudaStream_t stream, int* device_status)
     if (e != cudaSuccess) return cuda_fail(e);
     *device_status = h;
     return GLA_OK;
+}
+
+gla_status gla_trace_enable(int enable)
+{
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    for (auto& r : g_trace) {
+        cudaEventSynchronize(r.end);
+        g_event_pool.push_back(r.start);
+        g_event_pool.push_back(r.end);
+    }
+    g_trace.clear();
+    g_trace_on.store(enable != 0);
+    return GLA_OK;
+}
+
+int gla_trace_summary(const char** names, unsigned long long* launches, double* total_ms,
+                      int max_entries)
+{
+    std::lock_guard<std::mutex> lk(g_trace_mu);
+    int n = 0;
+    for (auto& r : g_trace) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.end) != cudaSuccess ||
+            cudaEventElapsedTime(&ms, r.start, r.end) != cudaSuccess)
+            continue;
+        int i = 0;
+        while (i < n && std::strcmp(names[i], r.name) != 0) ++i;
+        if (i == n) {
+            if (n >= max_entries) continue;
+            names[n] = r.name;
+            launches[n] = 0;
+            total_ms[n] = 0.0;
+            ++n;
+        }
+        launches[i] += 1;
+        total_ms[i] += ms;
+    }
+    return n;
 }
 
 gla_status gla_set_wait_limit_ns(unsigned long long ns)

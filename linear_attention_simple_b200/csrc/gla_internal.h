@@ -28,6 +28,11 @@ WaitCtl wait_ctl_for_current_device(gla_status* err);
 gla_status check_launch(const char* what);
 void count_launch(unsigned n = 1);
 
+// Tracing: trace_begin() before a launch, trace_end() after it; both are
+// no-ops unless tracing is enabled.  `name` must be a static string.
+void trace_begin(cudaStream_t st);
+void trace_end(cudaStream_t st, const char* name);
+
 // Encode a tiled tensor map over a bf16 (or fp32) [d3][d2][d1][d0] tensor.
 // dims[i] elements, strides_bytes[i] for i >= 1 (dim 0 contiguous), box[i].
 gla_status make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,

@@ -77,8 +77,10 @@ gla_status launch_fwd_f32(const float* q, const float* k, const float* v, const 
     (void)ctl;
     const int64_t units = static_cast<int64_t>(B) * H;
     if (units == 0) return GLA_OK;
+    trace_begin(st);
     fwd_f32_kernel<<<static_cast<unsigned>(units), kDv, 0, st>>>(q, k, v, a, s0, o, s_final, T, H,
                                                                  ld_qk, ld_v, scale);
+    trace_end(st, "fwd_f32_kernel");
     count_launch();
     return check_launch("fwd_f32_kernel");
 }

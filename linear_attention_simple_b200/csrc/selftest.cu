@@ -22,7 +22,9 @@ __global__ void wait_selftest_kernel(WaitCtl ctl)
 
 gla_status launch_wait_selftest(const WaitCtl& ctl, cudaStream_t st)
 {
+    trace_begin(st);
     wait_selftest_kernel<<<1, 32, 0, st>>>(ctl);
+    trace_end(st, "wait_selftest_kernel");
     count_launch();
     return check_launch("wait_selftest_kernel");
 }

@@ -100,6 +100,35 @@ gla_status gla_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          gla_dtype dt, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * gla_chunk_fwd for callers that cannot allocate device memory.  (The pages
+ * have no counterpart to this call; it exists for library users.)
+ *
+ * Some callers cannot obtain a workspace: a runtime that keeps all device
+ * memory in its own pool and forbids side allocations, a plugin host that
+ * does not let extensions call cudaMalloc, or a path that cannot afford the
+ * device synchronisation that cudaMalloc/cudaFree imply.  This call takes
+ * the arguments of gla_chunk_fwd without ws/ws_bytes and uses a fixed
+ * scratch array inside libgla instead; it allocates nothing.
+ *   - The array is GLA_NOALLOC_SCRATCH_BYTES per GPU that loads the library,
+ *     held until the process exits, and shared by every call on that GPU.
+ *   - Shapes whose workspace (gla_chunk_workspace_bytes) is larger are
+ *     rejected with GLA_ERR_UNSUPPORTED before anything is launched; use
+ *     gla_chunk_fwd with a workspace for those.
+ *   - Calls that overlap on the GPU (e.g. on two streams at once) race on the
+ *     shared array; order them.  The array's leftover contents never matter.
+ *   - The first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture starts.
+ * Everything else (layouts, validation, status codes) is as gla_chunk_fwd.
+ * ------------------------------------------------------------------------ */
+#define GLA_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+gla_status gla_chunk_fwd_noalloc(const void* q, const void* k, const void* v, const float* a,
+                                 const float* s0, void* o, float* s_final, int B, int T, int H,
+                                 int dk, int dv, int64_t ld_qkv, float scale, gla_dtype dt,
+                                 cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Chunked backward (the sequential chunk backward of "Como i14 ...", section
  * "Adaptaciones para AWS Trainium2", item 3).  Same inputs as the forward plus
  *   dO       [B, T, H, dv]  dt     upstream gradient of o, contiguous.

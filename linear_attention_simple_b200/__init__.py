@@ -19,7 +19,7 @@ __all__ = [
     "gla_chunk_workspace_bytes", "gla_chunk_fwd", "gla_chunk_bwd", "gla_decode_step",
     "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
-    "EXPORTED_SYMBOLS", "LIB_PATH",
+    "gla_chunk_fwd_noalloc", "EXPORTED_SYMBOLS", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgla.so")
@@ -29,6 +29,7 @@ EXPORTED_SYMBOLS = (
     "gla_chunk_workspace_bytes", "gla_chunk_fwd", "gla_chunk_bwd", "gla_decode_step",
     "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
+    "gla_chunk_fwd_noalloc",
 )
 
 GLA_BF16, GLA_F32 = 0, 1
@@ -89,6 +90,9 @@ def lib():
     L.gla_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
     L.gla_selftest_wait_timeout.restype = _i
     L.gla_selftest_wait_timeout.argtypes = [_vp]
+    L.gla_chunk_fwd_noalloc.restype = _i
+    L.gla_chunk_fwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                        _i64, _f, _i, _vp]
     L.gla_trace_enable.restype = _i
     L.gla_trace_enable.argtypes = [_i]
     L.gla_trace_summary.restype = _i
@@ -322,3 +326,30 @@ def gla_trace_summary(max_entries=64):
     totals = (ctypes.c_double * max_entries)()
     n = lib().gla_trace_summary(names, counts, totals, max_entries)
     return [(names[i].decode(), int(counts[i]), float(totals[i])) for i in range(n)]
+
+
+def gla_chunk_fwd_noalloc(q, k, v, a, s0=None, o=None, s_final=None, scale=None,
+                          want_final_state=True, stream=None):
+    """gla_chunk_fwd without a workspace, for callers that cannot allocate
+    device memory: libgla uses its built-in scratch array (shared by all
+    calls on a GPU; calls that overlap on the GPU race).  Shapes that need
+    more scratch than the array holds raise GlaError(GLA_ERR_UNSUPPORTED)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dt(q)
+    ld = _qkv_strides(q, k, v)
+    _need(a, "a", torch.float32, (B, T, H))
+    _need(s0, "s0", torch.float32, (B, H, dk, dv))
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    _need(o, "o", q.dtype, (B, T, H, dv))
+    if s_final is None and want_final_state:
+        s_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(s_final, "s_final", torch.float32, (B, H, dk, dv))
+    if scale is None:
+        scale = dk ** -0.5
+    st = lib().gla_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(s0), _ptr(o),
+                                     _ptr(s_final), B, T, H, dk, dv, ld, float(scale), dt,
+                                     _stream(stream))
+    _check("gla_chunk_fwd_noalloc", st)
+    return o, s_final

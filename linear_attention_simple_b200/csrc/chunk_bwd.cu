@@ -61,6 +61,9 @@ constexpr uint32_t BYTES = MISC + 2048 + 1024;
 constexpr uint32_t TM_SC = 0, TM_W = 128, TM_U = 320;
 }  // namespace bv
 
+// Threads: warps 0-7 are workers; warp 8 only issues TMA and tcgen05.mma.
+constexpr int kThreadsBwd = 288;
+
 __device__ __forceinline__ void named_sync128()
 {
     asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -131,7 +134,7 @@ __device__ __forceinline__ float bf16_at_sw64(const uint8_t* tile, int row, int 
 
 // ------------------------------------------------------------ dq, dk kernel
 
-__global__ void __launch_bounds__(256, 1) bwd_dqdk_kernel(const __grid_constant__ BwdParams p)
+__global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dqdk_kernel(const __grid_constant__ BwdParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -148,10 +151,12 @@ __global__ void __launch_bounds__(256, 1) bwd_dqdk_kernel(const __grid_constant_
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int unit = b * p.H + h;
     const int t0 = c * kChunk;
-    const int quad = warp & 3, half = warp >> 2, row = quad * 32 + lane;
+    const int quad = warp & 3, half = (warp >> 2) & 1, row = quad * 32 + lane;
+    const bool worker = warp < 8;
+    const bool issuer = warp == 8 && lane == 0;
     const WaitCtl ctl = p.ctl;
 
-    if (tid == 0) {
+    if (issuer) {
         mbar_init(bar_ld, 1);
         mbar_init(bar_m, 1);
         mbar_init_fence();
@@ -167,8 +172,9 @@ __global__ void __launch_bounds__(256, 1) bwd_dqdk_kernel(const __grid_constant_
     const uint32_t tq = tmem_addr(tmem, quad * 32, 0);
     bool failed = false;
     bool pend_ld = false, pend_m = false;
+    float dsum = 0.f;                        // this thread's share of q.dq - k.dk
 
-    if (tid == 0) {
+    if (issuer) {
         mbar_arrive_expect_tx(bar_ld, 2 * chunk::kTileQK + 2 * chunk::kTileV + 2 * 36864);
         for (int i = 0; i < 3; ++i) {
             tma_load_4d(sm + bq::Q + i * 8192, &p.tm_q, bar_ld, i * 32, h, t0, b);
@@ -208,14 +214,14 @@ __global__ void __launch_bounds__(256, 1) bwd_dqdk_kernel(const __grid_constant_
     if (!failed && !mbar_wait(bar_m, 0, ctl)) failed = true;
     tc_fence_before();
     if (__syncthreads_or(failed)) goto done;
-    if (tid == 0) pend_m = false;
+    if (issuer) pend_m = false;
     tc_fence_after();
     // dP (hi -> h buffer, lo -> D buffer; both consumed by the MMAs above)
-    masked_decay_tile(tq, bq::TM_DP, row, quad, half, b2s, p.scale, sm + bq::HS, sm + bq::DS);
+    if (worker) masked_decay_tile(tq, bq::TM_DP, row, quad, half, b2s, p.scale, sm + bq::HS, sm + bq::DS);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
+    if (issuer) {
         tc_fence_after();
         // Y = dP K (K as MN-major B, N = dk);  Z = dP^T Q (dP as MN-major A)
         for (int part = 0; part < 2; ++part) {
@@ -236,14 +242,13 @@ __global__ void __launch_bounds__(256, 1) bwd_dqdk_kernel(const __grid_constant_
     if (!mbar_wait(bar_m, 1, ctl)) failed = true;
     tc_fence_before();
     if (__syncthreads_or(failed)) goto done;
-    if (tid == 0) pend_m = false;
+    if (issuer) pend_m = false;
     tc_fence_after();
-    {
+    if (worker) {
         // epilogue: dq = scale e^{b} X + Y ; dk = Z + e^{gamma - b} W ; delta
         const float b2r = b2s[row];
         const float fq = p.scale * exp2f(b2r);
         const float fk = exp2f(b2s[127] - b2r);
-        float dsum = 0.f;
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
             const int d0 = half * 48 + j * 16;
@@ -277,19 +282,19 @@ __global__ void __launch_bounds__(256, 1) bwd_dqdk_kernel(const __grid_constant_
         if (half) dpart[row] = dsum;
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
-        if (!half && t0 + row < p.T)
-            p.delta[(static_cast<int64_t>(b) * p.T + t0 + row) * p.H + h] = dsum + dpart[row];
-        if (tid == 0) {
-            for (int i = 0; i < 3; ++i) {
-                tma_store_4d(&p.tm_dq, sm + bq::DO + i * 8192, i * 32, h, t0, b);
-                tma_store_4d(&p.tm_dk, sm + bq::DO + 24576 + i * 8192, i * 32, h, t0, b);
-            }
-            tma_store_commit();
+    }
+    __syncthreads();
+    if (worker && !half && t0 + row < p.T)
+        p.delta[(static_cast<int64_t>(b) * p.T + t0 + row) * p.H + h] = dsum + dpart[row];
+    if (issuer) {
+        for (int i = 0; i < 3; ++i) {
+            tma_store_4d(&p.tm_dq, sm + bq::DO + i * 8192, i * 32, h, t0, b);
+            tma_store_4d(&p.tm_dk, sm + bq::DO + 24576 + i * 8192, i * 32, h, t0, b);
         }
+        tma_store_commit();
     }
 done:
-    if (tid == 0) {
+    if (issuer) {
         if (pend_ld) mbar_wait(bar_ld, 0, ctl);
         if (pend_m) mbar_wait(bar_m, 0, ctl) && mbar_wait(bar_m, 1, ctl);
         tma_store_wait_all();
@@ -301,7 +306,7 @@ done:
 
 // ----------------------------------------------------------------- dv kernel
 
-__global__ void __launch_bounds__(256, 1) bwd_dv_kernel(const __grid_constant__ BwdParams p)
+__global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dv_kernel(const __grid_constant__ BwdParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -317,10 +322,12 @@ __global__ void __launch_bounds__(256, 1) bwd_dv_kernel(const __grid_constant__ 
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int unit = b * p.H + h;
     const int t0 = c * kChunk;
-    const int quad = warp & 3, half = warp >> 2, row = quad * 32 + lane;
+    const int quad = warp & 3, half = (warp >> 2) & 1, row = quad * 32 + lane;
+    const bool worker = warp < 8;
+    const bool issuer = warp == 8 && lane == 0;
     const WaitCtl ctl = p.ctl;
 
-    if (tid == 0) {
+    if (issuer) {
         mbar_init(bar_ld, 1);
         mbar_init(bar_m, 1);
         mbar_init_fence();
@@ -337,7 +344,7 @@ __global__ void __launch_bounds__(256, 1) bwd_dv_kernel(const __grid_constant__ 
     bool failed = false;
     bool pend_ld = false, pend_m = false;
 
-    if (tid == 0) {
+    if (issuer) {
         mbar_arrive_expect_tx(bar_ld, 2 * chunk::kTileQK + chunk::kTileV + 36864);
         for (int i = 0; i < 3; ++i) {
             tma_load_4d(sm + bv::Q + i * 8192, &p.tm_q, bar_ld, i * 32, h, t0, b);
@@ -372,13 +379,13 @@ __global__ void __launch_bounds__(256, 1) bwd_dv_kernel(const __grid_constant__ 
     if (!failed && !mbar_wait(bar_m, 0, ctl)) failed = true;
     tc_fence_before();
     if (__syncthreads_or(failed)) goto done;
-    if (tid == 0) pend_m = false;
+    if (issuer) pend_m = false;
     tc_fence_after();
-    masked_decay_tile(tq, bv::TM_SC, row, quad, half, b2s, p.scale, sm + bv::PH, sm + bv::PL);
+    if (worker) masked_decay_tile(tq, bv::TM_SC, row, quad, half, b2s, p.scale, sm + bv::PH, sm + bv::PL);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
+    if (issuer) {
         tc_fence_after();
         // U = P^T dO (P as MN-major A, dO as MN-major B)
         for (int part = 0; part < 2; ++part) {
@@ -394,9 +401,9 @@ __global__ void __launch_bounds__(256, 1) bwd_dv_kernel(const __grid_constant__ 
     if (!mbar_wait(bar_m, 1, ctl)) failed = true;
     tc_fence_before();
     if (__syncthreads_or(failed)) goto done;
-    if (tid == 0) pend_m = false;
+    if (issuer) pend_m = false;
     tc_fence_after();
-    {
+    if (worker) {
         // epilogue: dv = U + e^{gamma - b} W  -> staging in the dO buffer
         const float fk = exp2f(b2s[127] - b2s[row]);
 #pragma unroll
@@ -420,14 +427,14 @@ __global__ void __launch_bounds__(256, 1) bwd_dv_kernel(const __grid_constant__ 
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            for (int i = 0; i < 3; ++i) tma_store_4d(&p.tm_dv, sm + bv::DO + i * 16384, i * 64, h, t0, b);
-            tma_store_commit();
-        }
+    }
+    __syncthreads();
+    if (issuer) {
+        for (int i = 0; i < 3; ++i) tma_store_4d(&p.tm_dv, sm + bv::DO + i * 16384, i * 64, h, t0, b);
+        tma_store_commit();
     }
 done:
-    if (tid == 0) {
+    if (issuer) {
         if (pend_ld) mbar_wait(bar_ld, 0, ctl);
         if (pend_m) mbar_wait(bar_m, 0, ctl) && mbar_wait(bar_m, 1, ctl);
         tma_store_wait_all();
@@ -487,7 +494,7 @@ gla_status launch_bwd_kernel(K kernel, uint32_t bytes, const BwdParams& p, dim3 
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
         return check_launch(name);
     trace_begin(st);
-    kernel<<<grid, 256, bytes, st>>>(p);
+    kernel<<<grid, kThreadsBwd, bytes, st>>>(p);
     trace_end(st, name);
     count_launch();
     return check_launch(name);

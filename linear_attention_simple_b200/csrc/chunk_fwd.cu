@@ -14,6 +14,7 @@
 // read of k and v for nseg-fold parallelism.
 #include <cstring>
 
+#define GLA_CHUNK_KERNELS
 #include "chunk_state.cuh"
 
 namespace gla {
@@ -60,32 +61,29 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(float* __restrict__ st
     }
 }
 
-template <bool W, bool R>
-gla_status launch_state_t(const StateParams& p, dim3 grid, cudaStream_t st)
+template <typename K>
+gla_status launch_chunk_kernel(K kernel, uint32_t bytes, const char* name, const StateParams& p,
+                               dim3 grid, cudaStream_t st)
 {
-    const uint32_t bytes = chunk::Smem<W>::BYTES;
-    cudaError_t e = cudaFuncSetAttribute(gla_chunk_state_kernel<W, R>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return check_launch("cudaFuncSetAttribute");
-    static const char* const kName = W ? "chunk_fwd_fused_kernel"
-                                       : (R ? "chunk_state_rev_kernel" : "chunk_state_fwd_kernel");
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return check_launch("cudaFuncSetAttribute");
     trace_begin(st);
-    gla_chunk_state_kernel<W, R><<<grid, 256, bytes, st>>>(p);
-    trace_end(st, kName);
+    kernel<<<grid, chunk::kThreads, bytes, st>>>(p);
+    trace_end(st, name);
     count_launch();
-    return check_launch("gla_chunk_state_kernel");
+    return check_launch(name);
 }
 
 }  // namespace
 
 gla_status make_token_map(CUtensorMap* m, const void* base, int d, int H, int T, int B,
-                          int64_t ld, int box_d, int swizzle)
+                          int64_t ld, int box_d, int swizzle, int box_rows)
 {
     const uint64_t dims[4] = {static_cast<uint64_t>(d), static_cast<uint64_t>(H),
                               static_cast<uint64_t>(T), static_cast<uint64_t>(B)};
     const uint64_t strides[4] = {2, static_cast<uint64_t>(d) * 2, static_cast<uint64_t>(ld) * 2,
                                  static_cast<uint64_t>(T) * ld * 2};
-    const uint32_t box[4] = {static_cast<uint32_t>(box_d), 1, 128, 1};
+    const uint32_t box[4] = {static_cast<uint32_t>(box_d), 1, static_cast<uint32_t>(box_rows), 1};
     return make_tmap(m, base, 4, dims, strides, box, 2, swizzle);
 }
 
@@ -102,9 +100,15 @@ gla_status make_state_map(CUtensorMap* m, void* base, int64_t nstates)
 gla_status launch_state_kernel(bool with_o, bool reverse, const StateParams& p, dim3 grid,
                                cudaStream_t st)
 {
-    if (with_o && !reverse) return launch_state_t<true, false>(p, grid, st);
-    if (!with_o && !reverse) return launch_state_t<false, false>(p, grid, st);
-    if (!with_o && reverse) return launch_state_t<false, true>(p, grid, st);
+    if (with_o && !reverse)
+        return launch_chunk_kernel(gla_fwd_fused_kernel, chunk::FusedSmem::BYTES,
+                                   "chunk_fwd_fused_kernel", p, grid, st);
+    if (!with_o && !reverse)
+        return launch_chunk_kernel(gla_state_pass_kernel<false>, chunk::PassSmem::BYTES,
+                                   "chunk_state_fwd_kernel", p, grid, st);
+    if (!with_o && reverse)
+        return launch_chunk_kernel(gla_state_pass_kernel<true>, chunk::PassSmem::BYTES,
+                                   "chunk_state_rev_kernel", p, grid, st);
     return GLA_ERR_UNSUPPORTED;
 }
 
@@ -129,7 +133,7 @@ gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float
     StateParams p;
     memset(&p, 0, sizeof(p));
     gla_status s;
-    if ((s = make_token_map(&p.tm_q, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
+    if ((s = make_token_map(&p.tm_q, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64, 16)) != GLA_OK) return s;
     if ((s = make_token_map(&p.tm_u, pr.k, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&p.tm_y, pr.v, kDv, pr.H, pr.T, pr.B, pr.ld_v, 64, 128)) != GLA_OK) return s;
     if ((s = make_token_map(&p.tm_o, o, kDv, pr.H, pr.T, pr.B, static_cast<int64_t>(pr.H) * kDv, 64,

@@ -1,43 +1,52 @@
-// chunk_state.cuh -- the sequential-over-chunks Simple GLA kernel on tcgen05.
+// chunk_state.cuh -- the sequential-over-chunks Simple GLA kernels on tcgen05.
 //
-// One CTA owns one (batch, head, segment of chunks) and walks its chunks in
-// order (forward) or in reverse, keeping the fp32 dk x dv state in tensor
-// memory.  The chunked form ("Como i14 llevo Laplace 3B a AWS Trainium2",
-// section "Adaptaciones para AWS Trainium2", item 1: chunks of 128 tokens;
-// item 3: the backward walks the chunks sequentially) with, for a chunk of
-// tokens i, j and in-chunk cumulative log-decay b_i (gamma = b_last):
+// A CTA owns one (batch, head, segment of chunks) and walks its chunks in
+// order (or in reverse), keeping the fp32 dk x dv state in tensor memory as
+// an MMA accumulator.  The chunked form ("Como i14 llevo Laplace 3B a AWS
+// Trainium2", section "Adaptaciones para AWS Trainium2", item 1: chunks of
+// 128 tokens; item 3: the backward walks the chunks sequentially), for a
+// chunk with tokens i, j and in-chunk cumulative log-decay b (gamma = b_last):
 //
 //   forward  o_i  = scale ( e^{b_i} q_i S_prev + sum_{j<=i} e^{b_i-b_j} (q_i.k_j) v_j )
 //            S    = e^{gamma} S_prev + sum_j e^{gamma-b_j} k_j^T v_j
 //   reverse  D    = e^{gamma} D_next + sum_i (scale e^{b_i} q_i)^T dO_i
 //
-// Template modes
-//   WITH_O   forward with the output fused in: per chunk four tcgen05.mma
-//            groups -- scores = Q K^T (128x128x96), O = Q~ S_prev
-//            (128x192x96, fp16 operands), O += P V (128x192x128, P split
-//            into two bf16 terms P_hi + P_lo), S += K~^T V (128pad x 192 x
-//            128, K~ split into bf16 hi + lo) -- plus the masked-decay P
-//            tile on CUDA cores.  The
-//            state itself is always fp32 in tensor memory; only the MMA
-//            operand copies are 16-bit.
-//   !WITH_O  state only: S (or D) += U~^T Y per chunk (U~ split into bf16
-//            hi + lo, so the fp32 state sees ~16-bit operands), optionally storing the
-//            bf16 state before each chunk's update (for the backward).
-//   REVERSE  walks chunks from last to first (the dL/dS pass).
+// Two kernels:
 //
-// Operand layouts (all validated against the hardware): q and k tiles are
-// TMA-loaded as three 32-wide SW64 boxes ([3][128][32], K-major for the
+// gla_fwd_fused_kernel -- forward with the output fused in.  Per chunk:
+//   scores = Q K^T (tcgen05, 128x128x96); O = Q S_prev (128x192x96, the bf16
+//   state copy split into hi + lo terms); S += K~^T V (K~ = e^{gamma-b} K);
+//   O += P V (P split into bf16 hi + lo); epilogue o = r_i O_i.
+//   Decay factorisation: while the chunk's total decay spans at most 2^100,
+//   e^{b_i - b_j} = e^{b_i} e^{-b_j} is split into a column factor folded
+//   into P (P'_ij = (q_i.k_j) 2^{-b_j}) and a row factor applied in the
+//   epilogue (r_i = scale 2^{b_i}); every product stays finite and no
+//   per-element exponential or scaled copy of Q is needed.  Chunks with a
+//   steeper decay take the exact per-element path (P_ij with 2^{b_i - b_j},
+//   Q scaled by scale e^{b_i} in place, r_i = 1).
+//   The rows of the Q tile are permuted in 16-row blocks so that each of
+//   the four TMEM lane quarters (each owned by one SM sub-partition) gets an
+//   equal share of the causal triangle.
+//
+// gla_state_pass_kernel<REVERSE> -- state only: S (or D) += U~^T Y per chunk
+//   with U~ split into bf16 hi + lo, optionally storing the bf16 state before
+//   each chunk's update (the backward's h_c and D_c).  Tiles are double
+//   buffered: the next-but-one chunk's tiles load while a chunk computes.
+//
+// Operand layouts (validated against the hardware): q and k tiles are
+// TMA-loaded as three 32-wide SW64 boxes ([3][128][32]; K-major for the
 // scores; the k tile doubles as the MN-major A operand of the state product,
 // whose fourth 32-row block -- the padding of dk = 96 to M = 128 -- only
-// feeds TMEM lanes 96..127, which are never read); v tiles are three
-// 64-wide SW128 boxes ([3][128][64], MN-major B); the bf16 state copy is
-// [3][96][64] SW128 (MN-major B of O = Q~ S); P_hi is [2][128][64] SW128
-// (K-major A) and reuses the state copy's buffer once O = Q~ S has run;
-// P_lo uses the output staging buffer, which is free until the epilogue.
+// feeds TMEM lanes 96..127, which are never read); v tiles are three 64-wide
+// SW128 boxes ([3][128][64], MN-major B); state copies are [3][96][64] SW128;
+// P tiles are [2][128][64] SW128 (K-major A).
 //
-// Every wait is bounded; on timeout the CTA stops at the next block-wide
-// barrier, drains its in-flight copies and tensor-core work (again bounded),
-// frees its tensor memory and returns with GLA_ERR_TIMEOUT recorded.
+// Threads: warps 0-7 are workers (warp w reads TMEM lanes 32*(w%4) .. +31,
+// column half (w/4)); warp 8 only issues TMA copies and tcgen05.mma, so the
+// workers never stall behind the tensor core's issue queue.  Every wait is
+// bounded; on timeout the CTA stops at the next block-wide barrier, drains
+// its in-flight copies and tensor-core work (bounded), frees its tensor
+// memory and returns with GLA_ERR_TIMEOUT recorded.
 #pragma once
 
 #include "gla_device.cuh"
@@ -45,10 +54,10 @@
 namespace gla {
 
 struct StateParams {
-    CUtensorMap tm_q;       // q tile loads (WITH_O)
+    CUtensorMap tm_q;       // q tile loads, 16-row boxes (fused forward)
     CUtensorMap tm_u;       // scaled operand: k (forward) or q (reverse)
     CUtensorMap tm_y;       // v (forward) or dO (reverse)
-    CUtensorMap tm_o;       // o tile stores (WITH_O)
+    CUtensorMap tm_o;       // o tile stores (fused forward)
     CUtensorMap tm_h;       // per-chunk bf16 state stores (store_h)
     const float* a;         // [B, T, H] log-decay
     const float* s_init;    // initial state per (unit, seg) or null (zeros)
@@ -67,50 +76,47 @@ struct StateParams {
 namespace chunk {
 
 constexpr float kLog2e = 1.4426950408889634f;
-
-// Shared-memory map (bytes from a 1024-aligned base).
-template <bool WITH_O>
-struct Smem;
-template <>
-struct Smem<true> {
-    static constexpr uint32_t Q = 0;          // [3][128][32] bf16 SW64
-    static constexpr uint32_t U = 24576;      // k tile  [3][128][32] bf16 SW64 (then K~ hi)
-    static constexpr uint32_t UL = 49152;     // K~ lo, same layout (U's 4th M block: finite)
-    static constexpr uint32_t Z = 73728;      // zero block (UL's 4th M block)
-    static constexpr uint32_t Y = 81920;      // v tile  [3][128][64] bf16 SW128
-    static constexpr uint32_t X = 131072;     // state copy [3][96][64] / P_hi [2][128][64]
-    static constexpr uint32_t O = 167936;     // output staging [3][128][64] / P_lo
-    static constexpr uint32_t MISC = 217088;
-    static constexpr uint32_t BYTES = MISC + 1024 + 1024;   // + alignment slack
-    static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t TM_SC = 0, TM_O = 128, TM_S = 320;
-};
-template <>
-struct Smem<false> {
-    static constexpr uint32_t Q = 0;          // unused
-    static constexpr uint32_t U = 0;
-    static constexpr uint32_t UL = 24576;
-    static constexpr uint32_t Z = 49152;
-    static constexpr uint32_t Y = 57344;
-    static constexpr uint32_t X = 106496;
-    static constexpr uint32_t O = 0;          // unused
-    static constexpr uint32_t MISC = 143360;
-    static constexpr uint32_t BYTES = MISC + 1024 + 1024;
-    static constexpr uint32_t TMEM_COLS = 256;
-    static constexpr uint32_t TM_SC = 0, TM_O = 0, TM_S = 0;
-};
-
+constexpr int kWorkers = 256;
+constexpr int kThreads = kWorkers + 32;
 constexpr uint32_t kTileQK = 3 * 128 * 64;     // 24576 bytes
 constexpr uint32_t kTileV = 3 * 128 * 128;     // 49152 bytes
+constexpr float kFactorRange = 100.0f;         // max log2 span for the factorised decay
 
 constexpr uint32_t kIdScores = idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint32_t kIdOut = idesc_bf16_f32(128, 192, 0, 1);
-// O = Q~ S_prev runs in fp16 (10-bit mantissa) on rescaled copies: Q~ * 2^5
-// and S_prev * 2^-5, so the product is unchanged while |S| up to ~2e6 stays
-// inside the fp16 range.
-constexpr uint32_t kIdInter = idesc_f16_f32(128, 192, 0, 1);
-constexpr float kInterUp = 32.0f, kInterDown = 1.0f / 32.0f;
 constexpr uint32_t kIdState = idesc_bf16_f32(128, 192, 1, 1);
+
+// Shared-memory maps (bytes from a 1024-aligned base).
+struct FusedSmem {
+    static constexpr uint32_t Q = 0;          // q tile, permuted rows
+    static constexpr uint32_t U = 24576;      // k tile, then K~ (its 4th M block is Y: finite)
+    static constexpr uint32_t Y = 49152;      // v tile
+    static constexpr uint32_t X = 98304;      // state copy hi, then P_hi
+    static constexpr uint32_t XL = 135168;    // state copy lo
+    static constexpr uint32_t O = 172032;     // P_lo, then output staging
+    static constexpr uint32_t MISC = 221184;
+    static constexpr uint32_t BYTES = MISC + 2048 + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t TM_SC = 0, TM_O = 128, TM_S = 320;
+};
+struct PassSmem {
+    static constexpr uint32_t U0 = 0, U1 = 24576;   // U0's 4th M block is U1, U1's is UL
+    static constexpr uint32_t UL = 49152;           // U~ lo (its 4th M block is Z)
+    static constexpr uint32_t Z = 73728;            // zeros
+    static constexpr uint32_t Y0 = 81920, Y1 = 131072;
+    static constexpr uint32_t X = 180224;           // bf16 state copy (store_h)
+    static constexpr uint32_t MISC = 217088;
+    static constexpr uint32_t BYTES = MISC + 1024 + 1024;
+    static constexpr uint32_t TMEM_COLS = 256;
+    static constexpr uint32_t TM_S = 0;
+};
+
+// Token held by row r of the permuted q tile: 16-row block r/16 holds token
+// block perm16(r/16) (0, 7, 1, 6, 2, 5, 3, 4), so lane quarter q (rows
+// 32q..32q+31) holds token blocks {q, 7-q} and every quarter has the same
+// number of causal (i, j) pairs.
+__device__ __forceinline__ int perm16(int blk) { return (0x43526170u >> (4 * blk)) & 15; }
+__device__ __forceinline__ int row_token(int r) { return perm16(r >> 4) * 16 + (r & 15); }
 
 __device__ __forceinline__ void named_sync(int id, int n)
 {
@@ -139,6 +145,15 @@ __device__ __forceinline__ void scale8_split(uint4 v, float f, uint4& hi, uint4&
     lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
+// Scale the 64-byte row segment `row` of block `blk` of a [3][128][32] SW64
+// tile in place (the swizzle only permutes 16-byte chunks within a row).
+__device__ __forceinline__ void scale_row_sw64(uint8_t* tile, int row, int blk, float f)
+{
+    uint4* p = reinterpret_cast<uint4*>(tile + blk * 8192 + row * 64);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) p[c] = scale8(p[c], f);
+}
+
 // In-place hi / separate lo split of a scaled 64-byte row segment.
 __device__ __forceinline__ void split_row_sw64(uint8_t* tile, uint8_t* lo_tile, int row, int blk, float f)
 {
@@ -153,33 +168,6 @@ __device__ __forceinline__ void split_row_sw64(uint8_t* tile, uint8_t* lo_tile, 
     }
 }
 
-__device__ __forceinline__ uint4 scale8_to_f16(uint4 v, float f)
-{
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) w[i] = pack_f16(bf16_lo(w[i]) * f, bf16_hi(w[i]) * f);
-    return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// Scale the 64-byte row segment `row` of block `blk` of a [3][128][32] SW64
-// tile in place (the swizzle only permutes 16-byte chunks within a row);
-// TO_F16 also converts the bf16 elements to fp16.
-template <bool TO_F16 = false>
-__device__ __forceinline__ void scale_row_sw64(uint8_t* tile, int row, int blk, float f)
-{
-    uint4* p = reinterpret_cast<uint4*>(tile + blk * 8192 + row * 64);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) p[c] = TO_F16 ? scale8_to_f16(p[c], f) : scale8(p[c], f);
-}
-
-__device__ __forceinline__ uint4 pack8_f16(const uint32_t* r, float f)
-{
-    return make_uint4(pack_f16(__uint_as_float(r[0]) * f, __uint_as_float(r[1]) * f),
-                      pack_f16(__uint_as_float(r[2]) * f, __uint_as_float(r[3]) * f),
-                      pack_f16(__uint_as_float(r[4]) * f, __uint_as_float(r[5]) * f),
-                      pack_f16(__uint_as_float(r[6]) * f, __uint_as_float(r[7]) * f));
-}
-
 __device__ __forceinline__ uint4 pack8(const uint32_t* r)
 {
     return make_uint4(pack_bf16(__uint_as_float(r[0]), __uint_as_float(r[1])),
@@ -188,13 +176,118 @@ __device__ __forceinline__ uint4 pack8(const uint32_t* r)
                       pack_bf16(__uint_as_float(r[6]), __uint_as_float(r[7])));
 }
 
+// 8 fp32 values -> bf16 hi and lo (value - hi) terms.
+__device__ __forceinline__ void pack8_split(const uint32_t* r, uint4& hi, uint4& lo)
+{
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float a = __uint_as_float(r[2 * i]), b = __uint_as_float(r[2 * i + 1]);
+        h[i] = pack_bf16(a, b);
+        l[i] = pack_bf16(a - bf16_lo(h[i]), b - bf16_hi(h[i]));
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// Inclusive cumulative log2-decay of the chunk's 128 tokens, warps 0-3
+// (thread t holds token t's a).
+__device__ __forceinline__ float chunk_cumsum(float a, float* wsum, int warp, int lane)
+{
+    float x = a * kLog2e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    named_sync(1, 128);
+    float pre = 0.f;
+    for (int w = 0; w < warp; ++w) pre += wsum[w];
+    return x + pre;
+}
+
+// Load a [96][192] fp32 state (row `row`, columns half*96 .. +95) into TMEM.
+__device__ __forceinline__ void state_to_tmem(const float* src, uint32_t taddr)
+{
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        uint32_t r[32];
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+            const float4 v = src ? *reinterpret_cast<const float4*>(src + j * 32 + e)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            r[e] = __float_as_uint(v.x);
+            r[e + 1] = __float_as_uint(v.y);
+            r[e + 2] = __float_as_uint(v.z);
+            r[e + 3] = __float_as_uint(v.w);
+        }
+        tmem_st32(taddr + j * 32, r);
+    }
+    tmem_st_wait();
+}
+
+__device__ __forceinline__ void tmem_to_state(uint32_t taddr, float* dst)
+{
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        uint32_t r[32];
+        tmem_ld32(taddr + j * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + j * 32 + e) =
+                make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                            __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+    }
+}
+
+// State copy into [3][96][64] SW128 (row = dk index, n = dv column), for the
+// 96 columns half*96 .. +95 of this thread's row; then decay the state.
+template <bool SPLIT>
+__device__ __forceinline__ void state_copy_and_decay(uint32_t taddr, int row, int half, float f,
+                                                     uint8_t* hi, uint8_t* lo, bool copy)
+{
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        uint32_t r[32];
+        tmem_ld32(taddr + j * 32, r);
+        tmem_ld_wait();
+        if (copy) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const int n = half * 96 + j * 32 + q4 * 8;
+                const uint32_t off = (n >> 6) * 12288 + swz_off(row, (n & 63) >> 3, 128);
+                if (SPLIT) {
+                    uint4 h, l;
+                    pack8_split(r + q4 * 8, h, l);
+                    *reinterpret_cast<uint4*>(hi + off) = h;
+                    *reinterpret_cast<uint4*>(lo + off) = l;
+                } else {
+                    *reinterpret_cast<uint4*>(hi + off) = pack8(r + q4 * 8);
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+        tmem_st32(taddr + j * 32, r);
+    }
+    tmem_st_wait();
+}
+
 }  // namespace chunk
 
-template <bool WITH_O, bool REVERSE>
-__global__ void __launch_bounds__(256, 1) gla_chunk_state_kernel(const __grid_constant__ StateParams p)
+// The kernels are defined only in the translation unit that launches them
+// (chunk_fwd.cu defines GLA_CHUNK_KERNELS before including this header).
+#ifdef GLA_CHUNK_KERNELS
+
+// =====================================================================
+// Fused forward.
+// =====================================================================
+__global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const __grid_constant__ StateParams p)
 {
-    using L = chunk::Smem<WITH_O>;
     using namespace chunk;
+    using L = FusedSmem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -204,8 +297,9 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_state_kernel(const __grid_co
     uint64_t* bar_y = bar_q + 2;
     uint64_t* bar_m = bar_q + 3;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_q + 4);
-    float* b2s = reinterpret_cast<float*>(sm + L::MISC + 64);   // 128 floats
-    float* wsum = b2s + 128;                                     // 4 floats
+    float* b2s = reinterpret_cast<float*>(sm + L::MISC + 64);   // [128] by token
+    float* cfac = b2s + 128;                                     // [128] 2^{-b_j}
+    float* wsum = cfac + 128;                                    // [4]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -215,30 +309,27 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_state_kernel(const __grid_co
     const int nchunks = c_end - c_begin;
     const WaitCtl ctl = p.ctl;
 
-    // thread <-> TMEM lane / tile row: warp w covers lanes 32*(w%4) .. +31,
-    // column half (w/4).  State rows exist only for lanes < 96.
     const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    const int half = warp >> 2;
-    const bool srow = quad < 3;
+    const int row = quad * 32 + lane;         // TMEM lane = tile row (permuted token order)
+    const int tok = row_token(row);           // token of this row
+    const int half = (warp >> 2) & 1;
+    const bool worker = warp < 8;
+    const bool srow = worker && quad < 3;
+    const bool issuer = warp == 8 && lane == 0;
+    // largest token among this lane quarter's rows (columns beyond it are masked)
+    const int quad_max_tok = max(perm16(2 * quad), perm16(2 * quad + 1)) * 16 + 15;
 
-    if (tid == 0) {
+    if (issuer) {
         mbar_init(bar_q, 1);
         mbar_init(bar_u, 1);
         mbar_init(bar_y, 1);
         mbar_init(bar_m, 1);
         mbar_init_fence();
-        if (WITH_O) {
-            tma_prefetch_desc(&p.tm_q);
-            tma_prefetch_desc(&p.tm_o);
-        }
+        tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_u);
         tma_prefetch_desc(&p.tm_y);
-        if (p.store_h) tma_prefetch_desc(&p.tm_h);
+        tma_prefetch_desc(&p.tm_o);
     }
-    for (int i = tid * 16; i < 8192; i += 256 * 16)
-        *reinterpret_cast<uint4*>(sm + L::Z + i) = make_uint4(0u, 0u, 0u, 0u);
-    fence_async_smem();
     if (warp == 0) {
         tmem_alloc(tmem_slot, L::TMEM_COLS);
         tmem_relinquish();
@@ -247,90 +338,60 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_state_kernel(const __grid_co
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tq = tmem_addr(tmem, quad * 32, 0);   // this warp's lane quarter
+    const uint32_t tq = tmem_addr(tmem, quad * 32, 0);
 
-    auto chunk_at = [&](int it) { return REVERSE ? (c_end - 1 - it) : (c_begin + it); };
     auto load_a = [&](int c) {
         const int t = c * 128 + tid;
         return t < p.T ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f;
     };
-    // in-flight bookkeeping of thread 0 (for the abort path)
     bool pend_q = false, pend_u = false, pend_y = false, pend_m = false;
-    uint32_t ph_q = 0, ph_u = 0, ph_y = 0;
-    uint32_t mph = 0;   // parity of the next bar_m phase to complete
-
+    uint32_t ph_q = 0, ph_u = 0, ph_y = 0, mph = 0;
     auto issue_qu = [&](int c) {
         const int t0 = c * 128;
-        if (WITH_O) {
-            mbar_arrive_expect_tx(bar_q, kTileQK);
-            for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::Q + i * 8192, &p.tm_q, bar_q, i * 32, h, t0, b);
-            pend_q = true;
-        }
+        mbar_arrive_expect_tx(bar_q, kTileQK);
+        for (int i = 0; i < 3; ++i)
+            for (int r16 = 0; r16 < 8; ++r16)
+                tma_load_4d(sm + L::Q + i * 8192 + r16 * 1024, &p.tm_q, bar_q, i * 32, h,
+                            t0 + perm16(r16) * 16, b);
+        pend_q = true;
         mbar_arrive_expect_tx(bar_u, kTileQK);
         for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::U + i * 8192, &p.tm_u, bar_u, i * 32, h, t0, b);
         pend_u = true;
     };
     auto issue_y = [&](int c) {
-        const int t0 = c * 128;
         mbar_arrive_expect_tx(bar_y, kTileV);
-        for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::Y + i * 16384, &p.tm_y, bar_y, i * 64, h, t0, b);
+        for (int i = 0; i < 3; ++i)
+            tma_load_4d(sm + L::Y + i * 16384, &p.tm_y, bar_y, i * 64, h, c * 128, b);
         pend_y = true;
     };
 
-    if (tid == 0 && nchunks > 0) {
-        issue_qu(chunk_at(0));
-        issue_y(chunk_at(0));
+    if (issuer && nchunks > 0) {
+        issue_qu(c_begin);
+        issue_y(c_begin);
     }
-    float a_cur = (tid < 128 && nchunks > 0) ? load_a(chunk_at(0)) : 0.f;
-
-    // initial state -> TMEM
+    float a_cur = (tid < 128 && nchunks > 0) ? load_a(c_begin) : 0.f;
     if (srow) {
         const float* src = p.s_init ? p.s_init + unit * p.init_unit_stride + seg * p.init_seg_stride +
                                           row * kDv + half * 96
                                     : nullptr;
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-            uint32_t r[32];
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-                float4 v = src ? *reinterpret_cast<const float4*>(src + j * 32 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-                r[e] = __float_as_uint(v.x);
-                r[e + 1] = __float_as_uint(v.y);
-                r[e + 2] = __float_as_uint(v.z);
-                r[e + 3] = __float_as_uint(v.w);
-            }
-            tmem_st32(tq + L::TM_S + half * 96 + j * 32, r);
-        }
-        tmem_st_wait();
+        state_to_tmem(src, tq + L::TM_S + half * 96);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
 
     bool failed = false, aborted = false;
-    float gsum2 = 0.f;
     for (int it = 0; it < nchunks; ++it) {
-        const int c = chunk_at(it);
-        const uint32_t ph = it & 1;
+        const int c = c_begin + it;
 
-        // (A) in-chunk cumulative decay b (log2 units), warps 0-3
+        // (A) cumulative decay (warps 0-3) and column factors; scores MMA
         if (tid < 128) {
-            float x = a_cur * kLog2e;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            if (lane == 31) wsum[warp] = x;
-            named_sync(1, 128);
-            float pre = 0.f;
-            for (int w = 0; w < warp; ++w) pre += wsum[w];
-            b2s[tid] = x + pre;
+            const float x = chunk_cumsum(a_cur, wsum, warp, lane);
+            b2s[tid] = x;
+            cfac[tid] = exp2f(-x);
         }
-        if (WITH_O && tid == 0) {
-            // scores = Q K^T as soon as both tiles have landed
-            bool ok = mbar_wait(bar_q, ph_q, ctl) && mbar_wait(bar_u, ph_u, ctl);
-            if (ok) {
+        if (issuer) {
+            if (mbar_wait(bar_q, ph_q, ctl) && mbar_wait(bar_u, ph_u, ctl)) {
                 pend_q = pend_u = false;
                 ph_q ^= 1;
                 ph_u ^= 1;
@@ -349,97 +410,51 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_state_kernel(const __grid_co
         }
         if (__syncthreads_or(failed)) { aborted = true; break; }
         const float g2 = b2s[127];
-        gsum2 += g2;
+        const bool fast = -g2 <= kFactorRange;   // uniform: the factorised path is safe
 
-        // (B) state: bf16 copy for the MMA operand / the stored state, then decay
-        if (srow) {
-            const float f = exp2f(g2);
-#pragma unroll
-            for (int j = 0; j < 3; ++j) {
-                uint32_t r[32];
-                tmem_ld32(tq + L::TM_S + half * 96 + j * 32, r);
-                tmem_ld_wait();
-                if (WITH_O || p.store_h) {
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int n = half * 96 + j * 32 + q4 * 8;
-                        *reinterpret_cast<uint4*>(sm + L::X + (n >> 6) * 12288 +
-                                                  swz_off(row, (n & 63) >> 3, 128)) =
-                            WITH_O ? pack8_f16(r + q4 * 8, kInterDown) : pack8(r + q4 * 8);
-                    }
-                }
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
-                tmem_st32(tq + L::TM_S + half * 96 + j * 32, r);
-            }
-            tmem_st_wait();
-        }
+        // (B) state copy (bf16 hi + lo, the B operand of O = Q S_prev), decay
+        if (srow)
+            state_copy_and_decay<true>(tq + L::TM_S + half * 96, row, half, exp2f(g2), sm + L::X,
+                                       sm + L::XL, true);
 
-        // (C) scale operand rows in place
-        if (WITH_O) {
-            if (!mbar_wait(bar_m, mph, ctl)) failed = true;      // scores done: Q, K free
-            if (tid == 0) tma_store_wait_read();                  // o staging free (P_lo goes there)
-        } else {
-            if (!mbar_wait(bar_u, ph, ctl)) failed = true;       // u tile in
-        }
-        if (!failed) {
-            if (WITH_O) {
-                for (int idx = tid; idx < 768; idx += 256) {
-                    const int which = idx >= 384;
-                    const int rem = idx - which * 384;
-                    const int r = rem & 127, blk = rem >> 7;
-                    if (which)
-                        split_row_sw64(sm + L::U, sm + L::UL, r, blk, exp2f(g2 - b2s[r]));
-                    else
-                        scale_row_sw64<true>(sm + L::Q, r, blk, p.scale * kInterUp * exp2f(b2s[r]));
-                }
-            } else {
-                for (int idx = tid; idx < 384; idx += 256) {
-                    const int r = idx & 127, blk = idx >> 7;
-                    const float f = REVERSE ? p.scale * exp2f(b2s[r]) : exp2f(g2 - b2s[r]);
-                    split_row_sw64(sm + L::U, sm + L::UL, r, blk, f);
-                }
+        // (C) K~ = e^{gamma - b} K in place; on the exact path also
+        // Q~ = scale e^{b} Q (rows in permuted token order)
+        if (!mbar_wait(bar_m, mph, ctl)) failed = true;           // scores done: Q, K free
+        if (issuer) tma_store_wait_read();                          // o staging free (P_lo)
+        if (!failed && worker) {
+            for (int idx = tid; idx < 384; idx += kWorkers) {
+                const int r = idx & 127, blk = idx >> 7;
+                scale_row_sw64(sm + L::U, r, blk, exp2f(g2 - b2s[r]));
+                if (!fast) scale_row_sw64(sm + L::Q, r, blk, p.scale * exp2f(b2s[row_token(r)]));
             }
         }
         fence_async_smem();
         tc_fence_before();
         if (__syncthreads_or(failed)) { aborted = true; break; }
         tc_fence_after();
-        if (WITH_O) {
-            if (tid == 0) pend_m = false;
-            mph ^= 1;
-        } else if (tid == 0) {
-            pend_u = false;
-            ph_u ^= 1;
-        }
+        if (issuer) pend_m = false;
+        mph ^= 1;
 
-        // (D) store the state copy, O = Q~ S_prev, S += U~^T Y
-        if (tid == 0) {
-            tc_fence_after();
-            if (p.store_h) {
-                for (int i = 0; i < 3; ++i)
-                    tma_store_3d(&p.tm_h, sm + L::X + i * 12288, i * 64, 0, unit * p.NC + c);
-                tma_store_commit();
-            }
+        // (D) O = Q S_prev (hi, lo), S += K~^T V
+        if (issuer) {
             if (mbar_wait(bar_y, ph_y, ctl)) {
                 pend_y = false;
                 ph_y ^= 1;
-                if (WITH_O) {
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    const uint32_t sbase = part ? L::XL : L::X;
 #pragma unroll
                     for (int ks = 0; ks < 6; ++ks) {
                         const uint32_t aoff = (ks >> 1) * 8192 + (ks & 1) * 32;
                         umma_bf16(tmem + L::TM_O, smem_desc(sb + L::Q + aoff, 16, 512, kLayoutSW64),
-                                  smem_desc(sb + L::X + ks * 2048, 12288, 1024, kLayoutSW128), kIdInter,
-                                  ks > 0);
+                                  smem_desc(sb + sbase + ks * 2048, 12288, 1024, kLayoutSW128), kIdOut,
+                                  (part | ks) > 0);
                     }
                 }
 #pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        umma_bf16(tmem + L::TM_S,
-                                  smem_desc(sb + (part ? L::UL : L::U) + ks * 1024, 8192, 512, kLayoutSW64),
-                                  smem_desc(sb + L::Y + ks * 2048, 16384, 1024, kLayoutSW128), kIdState, 1);
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_bf16(tmem + L::TM_S, smem_desc(sb + L::U + ks * 1024, 8192, 512, kLayoutSW64),
+                              smem_desc(sb + L::Y + ks * 2048, 16384, 1024, kLayoutSW128), kIdState, 1);
                 umma_commit(bar_m);
                 pend_m = true;
             } else {
@@ -447,19 +462,17 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_state_kernel(const __grid_co
             }
         }
 
-        if (WITH_O) {
-            // (E) masked, decayed scores -> P = P_hi + P_lo (two bf16 terms, so the
-            // intra-chunk product keeps ~16 mantissa bits).  P_lo goes straight
-            // to the free output staging buffer; P_hi waits in registers until
-            // O = Q~ S_prev has finished reading the state copy it replaces.
-            uint32_t pk[32];
-            const float b2r = b2s[row];
+        // (E) P = P_hi + P_lo from the scores; P_lo to the output staging
+        // buffer at once, P_hi once O = Q S_prev has released the state copy
+        uint32_t pk[32];
+        if (worker) {
+            const float b2r = b2s[tok];
             uint8_t* plo = sm + L::O + half * 16384;
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 const int j0 = half * 64 + q2 * 32;
                 uint32_t lo[16];
-                if (j0 > quad * 32 + 31) {
+                if (j0 > quad_max_tok) {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) pk[q2 * 16 + e] = lo[e] = 0u;
                 } else {
@@ -469,8 +482,14 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_state_kernel(const __grid_co
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         const int j = j0 + e;
-                        const float v0 = (j <= row) ? p.scale * __uint_as_float(r[e]) * exp2f(b2r - b2s[j]) : 0.f;
-                        const float v1 = (j + 1 <= row) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2r - b2s[j + 1]) : 0.f;
+                        float v0, v1;
+                        if (fast) {
+                            v0 = (j <= tok) ? __uint_as_float(r[e]) * cfac[j] : 0.f;
+                            v1 = (j + 1 <= tok) ? __uint_as_float(r[e + 1]) * cfac[j + 1] : 0.f;
+                        } else {
+                            v0 = (j <= tok) ? p.scale * __uint_as_float(r[e]) * exp2f(b2r - b2s[j]) : 0.f;
+                            v1 = (j + 1 <= tok) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2r - b2s[j + 1]) : 0.f;
+                        }
                         const uint32_t hi = pack_bf16(v0, v1);
                         pk[q2 * 16 + e / 2] = hi;
                         lo[e / 2] = pack_bf16(v0 - bf16_lo(hi), v1 - bf16_hi(hi));
@@ -481,115 +500,276 @@ __global__ void __launch_bounds__(256, 1) gla_chunk_state_kernel(const __grid_co
                     *reinterpret_cast<uint4*>(plo + swz_off(row, q2 * 4 + c4, 128)) =
                         make_uint4(lo[c4 * 4], lo[c4 * 4 + 1], lo[c4 * 4 + 2], lo[c4 * 4 + 3]);
             }
-            if (!mbar_wait(bar_m, mph, ctl)) failed = true;       // O = Q~S and S += K~^T V done
-            if (tid == 0) tma_store_wait_read();                  // stored state copy read out
-            tc_fence_before();
-            if (__syncthreads_or(failed)) { aborted = true; break; }
-            if (tid == 0) pend_m = false;
-            mph ^= 1;
-            {
-                uint8_t* pb = sm + L::X + half * 16384;
+        }
+        if (!mbar_wait(bar_m, mph, ctl)) failed = true;               // O = Q S_prev, S update done
+        tc_fence_before();
+        if (__syncthreads_or(failed)) { aborted = true; break; }
+        if (issuer) pend_m = false;
+        mph ^= 1;
+        if (worker) {
+            uint8_t* pb = sm + L::X + half * 16384;
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    *reinterpret_cast<uint4*>(pb + swz_off(row, ch, 128)) =
-                        make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-            }
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4*>(pb + swz_off(row, ch, 128)) =
+                    make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
 
-            // (F) O += P V; prefetch the next q and k tiles
-            float a_next = 0.f;
-            if (tid == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    const uint32_t pbase = part ? L::O : L::X;
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t aoff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                        umma_bf16(tmem + L::TM_O, smem_desc(sb + pbase + aoff, 16, 1024, kLayoutSW128),
-                                  smem_desc(sb + L::Y + ks * 2048, 16384, 1024, kLayoutSW128), kIdOut, 1);
-                    }
-                }
-                umma_commit(bar_m);
-                pend_m = true;
-                if (it + 1 < nchunks) issue_qu(chunk_at(it + 1));
-            }
-            if (tid < 128 && it + 1 < nchunks) a_next = load_a(chunk_at(it + 1));
-
-            // (G) epilogue: O rows -> bf16 staging -> TMA store
-            if (!mbar_wait(bar_m, mph, ctl)) failed = true;
-            if (__syncthreads_or(failed)) { aborted = true; break; }
-            if (tid == 0) pend_m = false;
-            mph ^= 1;
+        // (F) O += P V; prefetch the next q and k tiles and decays
+        float a_next = 0.f;
+        if (issuer) {
             tc_fence_after();
-            if (tid == 0 && it + 1 < nchunks) issue_y(chunk_at(it + 1));
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t pbase = part ? L::O : L::X;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t aoff = (ks >> 2) * 16384 + (ks & 3) * 32;
+                    umma_bf16(tmem + L::TM_O, smem_desc(sb + pbase + aoff, 16, 1024, kLayoutSW128),
+                              smem_desc(sb + L::Y + ks * 2048, 16384, 1024, kLayoutSW128), kIdOut, 1);
+                }
+            }
+            umma_commit(bar_m);
+            pend_m = true;
+            if (it + 1 < nchunks) issue_qu(c + 1);
+        }
+        if (tid < 128 && it + 1 < nchunks) a_next = load_a(c + 1);
+
+        // (G) epilogue: o = r_i O_i -> bf16 staging (token order) -> TMA store
+        if (!mbar_wait(bar_m, mph, ctl)) failed = true;
+        if (__syncthreads_or(failed)) { aborted = true; break; }
+        if (issuer) pend_m = false;
+        mph ^= 1;
+        tc_fence_after();
+        if (issuer && it + 1 < nchunks) issue_y(c + 1);
+        if (worker) {
+            const float rf = fast ? p.scale * exp2f(b2s[tok]) : 1.0f;
 #pragma unroll
             for (int j = 0; j < 3; ++j) {
                 uint32_t r[32];
                 tmem_ld32(tq + L::TM_O + half * 96 + j * 32, r);
                 tmem_ld_wait();
 #pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * rf);
+#pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     const int n = half * 96 + j * 32 + q4 * 8;
                     *reinterpret_cast<uint4*>(sm + L::O + (n >> 6) * 16384 +
-                                              swz_off(row, (n & 63) >> 3, 128)) = pack8(r + q4 * 8);
+                                              swz_off(tok, (n & 63) >> 3, 128)) = pack8(r + q4 * 8);
                 }
             }
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (tid == 0) {
-                for (int i = 0; i < 3; ++i) tma_store_4d(&p.tm_o, sm + L::O + i * 16384, i * 64, h, c * 128, b);
-                tma_store_commit();
-            }
-            a_cur = a_next;
-        } else {
-            // state only: wait for S += U~^T Y, then prefetch the next tiles
-            if (!mbar_wait(bar_m, mph, ctl)) failed = true;
-            if (tid == 0 && p.store_h) tma_store_wait_read();
-            if (__syncthreads_or(failed)) { aborted = true; break; }
-            if (tid == 0) pend_m = false;
-            mph ^= 1;
-            tc_fence_after();
-            if (tid == 0 && it + 1 < nchunks) {
-                issue_qu(chunk_at(it + 1));
-                issue_y(chunk_at(it + 1));
-            }
-            a_cur = (tid < 128 && it + 1 < nchunks) ? load_a(chunk_at(it + 1)) : 0.f;
         }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (issuer) {
+            for (int i = 0; i < 3; ++i) tma_store_4d(&p.tm_o, sm + L::O + i * 16384, i * 64, h, c * 128, b);
+            tma_store_commit();
+        }
+        a_cur = a_next;
     }
 
     if (!aborted) {
         const bool write_state = p.s_out && (!p.out_last_only || seg == static_cast<int>(gridDim.x) - 1);
-        if (write_state && srow) {
-            float* dst = p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + half * 96;
-#pragma unroll
-            for (int j = 0; j < 3; ++j) {
-                uint32_t r[32];
-                tmem_ld32(tq + L::TM_S + half * 96 + j * 32, r);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; e += 4)
-                    *reinterpret_cast<float4*>(dst + j * 32 + e) =
-                        make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                                    __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
-            }
-        }
-        if (p.g2_out && tid == 0) p.g2_out[static_cast<int64_t>(unit) * p.g2_unit_stride + seg] = gsum2;
-    } else if (tid == 0) {
-        // drain whatever is still in flight (bounded), so nothing lands in
-        // shared or tensor memory after this CTA has released them
+        if (write_state && srow)
+            tmem_to_state(tq + L::TM_S + half * 96,
+                          p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + half * 96);
+    } else if (issuer) {
         if (pend_q) mbar_wait(bar_q, ph_q, ctl);
         if (pend_u) mbar_wait(bar_u, ph_u, ctl);
         if (pend_y) mbar_wait(bar_y, ph_y, ctl);
         if (pend_m) mbar_wait(bar_m, mph, ctl);
     }
-    if (tid == 0) tma_store_wait_all();
+    if (issuer) tma_store_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);
 }
+
+// =====================================================================
+// State-only pass (double-buffered tiles).
+// =====================================================================
+template <bool REVERSE>
+__global__ void __launch_bounds__(chunk::kThreads, 1) gla_state_pass_kernel(const __grid_constant__ StateParams p)
+{
+    using namespace chunk;
+    using L = PassSmem;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+    const uint32_t sb = smem_u32(sm);
+    uint64_t* bar_u = reinterpret_cast<uint64_t*>(sm + L::MISC);   // [2]
+    uint64_t* bar_y = bar_u + 2;                                    // [2]
+    uint64_t* bar_m = bar_u + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_u + 5);
+    float* b2s = reinterpret_cast<float*>(sm + L::MISC + 64);
+    float* wsum = b2s + 128;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int unit = b * p.H + h;
+    const int c_begin = seg * p.chunks_per_seg;
+    const int c_end = min(p.NC, c_begin + p.chunks_per_seg);
+    const int nchunks = c_end - c_begin;
+    const WaitCtl ctl = p.ctl;
+
+    const int quad = warp & 3, row = quad * 32 + lane, half = (warp >> 2) & 1;
+    const bool worker = warp < 8;
+    const bool srow = worker && quad < 3;
+    const bool issuer = warp == 8 && lane == 0;
+
+    if (issuer) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar_u + s, 1);
+            mbar_init(bar_y + s, 1);
+        }
+        mbar_init(bar_m, 1);
+        mbar_init_fence();
+        tma_prefetch_desc(&p.tm_u);
+        tma_prefetch_desc(&p.tm_y);
+        if (p.store_h) tma_prefetch_desc(&p.tm_h);
+    }
+    for (int i = tid * 16; i < 8192; i += kThreads * 16)
+        *reinterpret_cast<uint4*>(sm + L::Z + i) = make_uint4(0u, 0u, 0u, 0u);
+    fence_async_smem();
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, L::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tq = tmem_addr(tmem, quad * 32, 0);
+
+    auto chunk_at = [&](int it) { return REVERSE ? (c_end - 1 - it) : (c_begin + it); };
+    auto load_a = [&](int c) {
+        const int t = c * 128 + tid;
+        return t < p.T ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f;
+    };
+    int pend = 0;                              // bit s: stage s has loads in flight
+    uint32_t ph_ld[2] = {0u, 0u};
+    uint32_t mph = 0;
+    bool pend_m = false;
+    auto issue = [&](int c, int s) {
+        const int t0 = c * 128;
+        uint8_t* u = sm + (s ? L::U1 : L::U0);
+        uint8_t* y = sm + (s ? L::Y1 : L::Y0);
+        mbar_arrive_expect_tx(bar_u + s, kTileQK);
+        for (int i = 0; i < 3; ++i) tma_load_4d(u + i * 8192, &p.tm_u, bar_u + s, i * 32, h, t0, b);
+        mbar_arrive_expect_tx(bar_y + s, kTileV);
+        for (int i = 0; i < 3; ++i) tma_load_4d(y + i * 16384, &p.tm_y, bar_y + s, i * 64, h, t0, b);
+        pend |= 1 << s;
+    };
+
+    if (issuer) {
+        if (nchunks > 0) issue(chunk_at(0), 0);
+        if (nchunks > 1) issue(chunk_at(1), 1);
+    }
+    float a_cur = (tid < 128 && nchunks > 0) ? load_a(chunk_at(0)) : 0.f;
+    if (srow) {
+        const float* src = p.s_init ? p.s_init + unit * p.init_unit_stride + seg * p.init_seg_stride +
+                                          row * kDv + half * 96
+                                    : nullptr;
+        state_to_tmem(src, tq + L::TM_S + half * 96);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    bool failed = false, aborted = false;
+    float gsum2 = 0.f;
+    for (int it = 0; it < nchunks; ++it) {
+        const int c = chunk_at(it);
+        const int s = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        uint8_t* u = sm + (s ? L::U1 : L::U0);
+        const uint32_t ua = s ? L::U1 : L::U0, ya = s ? L::Y1 : L::Y0;
+        const float a_nxt = (tid < 128 && it + 1 < nchunks) ? load_a(chunk_at(it + 1)) : 0.f;
+
+        // (A) cumulative decay
+        if (tid < 128) b2s[tid] = chunk_cumsum(a_cur, wsum, warp, lane);
+        __syncthreads();
+        const float g2 = b2s[127];
+        gsum2 += g2;
+
+        // (B) store-copy (bf16) and decay of the state
+        if (srow)
+            state_copy_and_decay<false>(tq + L::TM_S + half * 96, row, half, exp2f(g2), sm + L::X,
+                                        nullptr, p.store_h != 0);
+
+        // (C) U~ = w U split into hi (in place) + lo
+        if (!mbar_wait(bar_u + s, ph, ctl)) failed = true;
+        if (!failed && worker) {
+            for (int idx = tid; idx < 384; idx += kWorkers) {
+                const int r = idx & 127, blk = idx >> 7;
+                const float f = REVERSE ? p.scale * exp2f(b2s[r]) : exp2f(g2 - b2s[r]);
+                split_row_sw64(u, sm + L::UL, r, blk, f);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        if (__syncthreads_or(failed)) { aborted = true; break; }
+        tc_fence_after();
+
+        // (D) store the state copy; S += U~^T Y
+        if (issuer) {
+            if (p.store_h) {
+                for (int i = 0; i < 3; ++i)
+                    tma_store_3d(&p.tm_h, sm + L::X + i * 12288, i * 64, 0, unit * p.NC + c);
+                tma_store_commit();
+            }
+            if (mbar_wait(bar_y + s, ph, ctl)) {
+                pend &= ~(1 << s);
+                ph_ld[s] ^= 1;
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    const uint32_t abase = part ? L::UL : ua;
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        umma_bf16(tmem + L::TM_S, smem_desc(sb + abase + ks * 1024, 8192, 512, kLayoutSW64),
+                                  smem_desc(sb + ya + ks * 2048, 16384, 1024, kLayoutSW128), kIdState, 1);
+                }
+                umma_commit(bar_m);
+                pend_m = true;
+            } else {
+                failed = true;
+            }
+        }
+
+        // (E) wait for the update; refill this stage with chunk it+2
+        if (!mbar_wait(bar_m, mph, ctl)) failed = true;
+        if (issuer && p.store_h) tma_store_wait_read();
+        if (__syncthreads_or(failed)) { aborted = true; break; }
+        if (issuer) pend_m = false;
+        mph ^= 1;
+        tc_fence_after();
+        if (issuer && it + 2 < nchunks) issue(chunk_at(it + 2), s);
+        a_cur = a_nxt;
+    }
+
+    if (!aborted) {
+        const bool write_state = p.s_out && (!p.out_last_only || seg == static_cast<int>(gridDim.x) - 1);
+        if (write_state && srow)
+            tmem_to_state(tq + L::TM_S + half * 96,
+                          p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + half * 96);
+        if (p.g2_out && tid == 0) p.g2_out[static_cast<int64_t>(unit) * p.g2_unit_stride + seg] = gsum2;
+    } else if (issuer) {
+        for (int s = 0; s < 2; ++s)
+            if (pend & (1 << s)) {
+                mbar_wait(bar_u + s, ph_ld[s], ctl);
+                mbar_wait(bar_y + s, ph_ld[s], ctl);
+            }
+        if (pend_m) mbar_wait(bar_m, mph, ctl);
+    }
+    if (issuer) tma_store_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);
+}
+
+#endif  // GLA_CHUNK_KERNELS
 
 }  // namespace gla

@@ -101,7 +101,7 @@ def _front_check(y, ref):
     assert float(np.max(np.abs(y - ref))) <= 5e-2
 
 
-@pytest.mark.parametrize("B,T,D,hist,affine", [(1, 1, 256, False, False), (2, 37, 256, True, True),
+@pytest.mark.parametrize("B,T,D,hist,affine", [(1, 1, 256, False, False), (2, 37, 256, True, True), (3, 1000, 4096, True, True), (1, 200, 64, True, False),
                                                (3, 300, 3072, True, False), (1, 2, 64, True, True)])
 def test_front_end_parity(B, T, D, hist, affine):
     d = inputs.front_inputs(B, T, D, seed=40 + T, device="cuda", with_state=hist)

@@ -40,6 +40,7 @@ struct BwdParams {
     CUtensorMap tm_q, tm_k, tm_v, tm_do;   // token tiles
     CUtensorMap tm_h, tm_d;                // per-chunk bf16 states
     CUtensorMap tm_dq, tm_dk, tm_dv;       // gradient stores
+    CUtensorMap tm_do32, tm_d32, tm_dv32;  // 32-column SW64 boxes (dv kernel)
     const float* a;
     float* delta;                          // [B, T, H]: q.dq - k.dk per token
     int B, T, H, NC;
@@ -54,12 +55,6 @@ constexpr uint32_t BYTES = MISC + 2048 + 1024;
 constexpr uint32_t TM_DP = 0, TM_X = 128, TM_W = 224, TM_Y = 320, TM_Z = 416;
 }  // namespace bq
 
-namespace bv {   // dv kernel shared-memory map
-constexpr uint32_t Q = 0, K = 24576, DO = 49152, DS = 98304, PH = 135168, PL = 167936;
-constexpr uint32_t MISC = 200704;
-constexpr uint32_t BYTES = MISC + 2048 + 1024;
-constexpr uint32_t TM_SC = 0, TM_W = 128, TM_U = 320;
-}  // namespace bv
 
 // Threads: warps 0-7 are workers; warp 8 only issues TMA and tcgen05.mma.
 constexpr int kThreadsBwd = 288;
@@ -305,8 +300,39 @@ done:
 }
 
 // ----------------------------------------------------------------- dv kernel
+//
+// One CTA per (batch, head, chunk, half of dv), 94 KB of shared memory and
+// 256 TMEM columns, so two CTAs share an SM and overlap each other's loads,
+// tensor work and CUDA-core work.  With gamma the chunk's total log-decay:
+//
+//   dv_j = e^{gamma - b_j} ( sum_{i >= j} P~_ji dO_i + k_j D )
+//   P~_ji = scale e^{b_i - gamma} (k_j . q_i)          (factorised path)
+//
+// scores^T = K Q^T lands in TMEM with lanes = j; each thread turns its own
+// lane's 64 columns in place into the bf16 hi and lo halves of P~ (P~ as the
+// A operand of a tcgen05.mma straight from tensor memory), and k_j D shares
+// the accumulator because both terms carry the same row factor.  Chunks whose
+// decay spans more than 2^100 take the exact path: P_ji = scale
+// e^{b_i - b_j} (k_j . q_i), K rows scaled by e^{gamma - b_j} in place before
+// K D, row factor 1.
+//
+// TMEM tile layout of P~ for one lane: K (token i) block kb = i / 32 holds
+// the hi words in columns 32 kb .. +15 and the lo words in 32 kb + 16 .. +31
+// (two bf16 per 32-bit column, even index in the low half).
 
-__global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dv_kernel(const __grid_constant__ BwdParams p)
+namespace bv {   // dv kernel shared-memory map
+constexpr uint32_t Q = 0, K = 24576, DO = 49152, DS = 73728;   // DO [3][128][32], DS [3][96][32] SW64
+constexpr uint32_t MISC = 92160;
+constexpr uint32_t BYTES = MISC + 1024 + 1024;
+constexpr uint32_t TM_T = 0, TM_DV = 128, TMEM_COLS = 256;
+}  // namespace bv
+
+__device__ __forceinline__ uint32_t ts_hi(uint32_t base, int ks)
+{
+    return base + 32 * (ks >> 1) + 8 * (ks & 1);
+}
+
+__global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dv_kernel(const __grid_constant__ BwdParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -316,16 +342,19 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dv_kernel(const __grid_con
     uint64_t* bar_m = bar_ld + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ld + 2);
     float* b2s = reinterpret_cast<float*>(sm + bv::MISC + 64);
-    float* wsum = b2s + 128;
+    float* cfs = b2s + 128;                  // [128] column factors scale 2^{b_i - gamma}
+    float* wsum = cfs + 128;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int c = blockIdx.x >> 1, dvh = blockIdx.x & 1, h = blockIdx.y, b = blockIdx.z;
     const int unit = b * p.H + h;
     const int t0 = c * kChunk;
     const int quad = warp & 3, half = (warp >> 2) & 1, row = quad * 32 + lane;
     const bool worker = warp < 8;
     const bool issuer = warp == 8 && lane == 0;
     const WaitCtl ctl = p.ctl;
+    const uint32_t idT = idesc_bf16_f32(128, 128, 0, 0);
+    const uint32_t idV = idesc_bf16_f32(128, 96, 0, 1);
 
     if (issuer) {
         mbar_init(bar_ld, 1);
@@ -333,7 +362,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dv_kernel(const __grid_con
         mbar_init_fence();
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 512);
+        tmem_alloc(tmem_slot, bv::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -341,29 +370,41 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dv_kernel(const __grid_con
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tq = tmem_addr(tmem, quad * 32, 0);
-    bool failed = false;
-    bool pend_ld = false, pend_m = false;
+    bool failed = false, pend_ld = false, pend_m = false;
+    uint32_t mph = 0;
 
     if (issuer) {
-        mbar_arrive_expect_tx(bar_ld, 2 * chunk::kTileQK + chunk::kTileV + 36864);
+        mbar_arrive_expect_tx(bar_ld, 2 * chunk::kTileQK + 24576 + 18432);
         for (int i = 0; i < 3; ++i) {
             tma_load_4d(sm + bv::Q + i * 8192, &p.tm_q, bar_ld, i * 32, h, t0, b);
             tma_load_4d(sm + bv::K + i * 8192, &p.tm_k, bar_ld, i * 32, h, t0, b);
-            tma_load_4d(sm + bv::DO + i * 16384, &p.tm_do, bar_ld, i * 64, h, t0, b);
-            tma_load_3d(sm + bv::DS + i * 12288, &p.tm_d, bar_ld, i * 64, 0, unit * p.NC + c);
+            tma_load_4d(sm + bv::DO + i * 8192, &p.tm_do32, bar_ld, dvh * 96 + i * 32, h, t0, b);
+            tma_load_3d(sm + bv::DS + i * 6144, &p.tm_d32, bar_ld, dvh * 96 + i * 32, 0, unit * p.NC + c);
         }
         pend_ld = true;
+    }
+    if (tid < 128) {
+        const int t = t0 + tid;
+        chunk_cumsum(t < p.T ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f, b2s, wsum, tid, warp,
+                     lane);
+    }
+    __syncthreads();
+    const float g2 = b2s[127];
+    const bool fast = -g2 <= chunk::kFactorRange;
+    if (tid < 128) cfs[tid] = p.scale * exp2f(b2s[tid] - g2);
+
+    // group 1: scores^T = K Q^T; on the factorised path also dv = K D
+    if (issuer) {
         if (mbar_wait(bar_ld, 0, ctl)) {
             pend_ld = false;
             tc_fence_after();
-            // scores = Q K^T ; W = K D
             for (int ks = 0; ks < 6; ++ks) {
                 const uint32_t off = (ks >> 1) * 8192 + (ks & 1) * 32;
                 const uint64_t ak = smem_desc(sb + bv::K + off, 16, 512, kLayoutSW64);
-                umma_bf16(tmem + bv::TM_SC, smem_desc(sb + bv::Q + off, 16, 512, kLayoutSW64), ak,
-                          idesc_bf16_f32(128, 128, 0, 0), ks > 0);
-                umma_bf16(tmem + bv::TM_W, ak, smem_desc(sb + bv::DS + ks * 2048, 12288, 1024, kLayoutSW128),
-                          idesc_bf16_f32(128, 192, 0, 1), ks > 0);
+                umma_bf16(tmem + bv::TM_T, ak, smem_desc(sb + bv::Q + off, 16, 512, kLayoutSW64), idT, ks > 0);
+                if (fast)
+                    umma_bf16(tmem + bv::TM_DV, ak, smem_desc(sb + bv::DS + ks * 1024, 6144, 512, kLayoutSW64), idV,
+                              ks > 0);
             }
             umma_commit(bar_m);
             pend_m = true;
@@ -371,77 +412,119 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dv_kernel(const __grid_con
             failed = true;
         }
     }
-    if (tid < 128) {
-        const int t = t0 + tid;
-        chunk_cumsum(t < p.T ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f, b2s, wsum,
-                     tid, warp, lane);
-    }
-    if (!failed && !mbar_wait(bar_m, 0, ctl)) failed = true;
+    if (!mbar_wait(bar_m, mph, ctl)) failed = true;
     tc_fence_before();
     if (__syncthreads_or(failed)) goto done;
-    if (issuer) pend_m = false;
     tc_fence_after();
-    if (worker) masked_decay_tile(tq, bv::TM_SC, row, quad, half, b2s, p.scale, sm + bv::PH, sm + bv::PL);
-    fence_async_smem();
+    if (issuer) pend_m = false;
+    mph ^= 1;
+
+    if (worker) {
+        // P~ (hi, lo) in place in tensor memory, this lane's 64 columns
+        const float b2j = b2s[row];
+#pragma unroll
+        for (int kb2 = 0; kb2 < 2; ++kb2) {
+            const int i0 = half * 64 + kb2 * 32;
+            const uint32_t col = bv::TM_T + i0;
+            uint32_t hi[16], lo[16];
+            if (i0 + 31 < quad * 32) {            // every i < j here: masked
+#pragma unroll
+                for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
+            } else {
+                uint32_t r[32];
+                tmem_ld32(tq + col, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const int i = i0 + e;
+                    float v0, v1;
+                    if (fast) {
+                        v0 = (i >= row) ? __uint_as_float(r[e]) * cfs[i] : 0.f;
+                        v1 = (i + 1 >= row) ? __uint_as_float(r[e + 1]) * cfs[i + 1] : 0.f;
+                    } else {
+                        v0 = (i >= row) ? p.scale * __uint_as_float(r[e]) * exp2f(b2s[i] - b2j) : 0.f;
+                        v1 = (i + 1 >= row) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2s[i + 1] - b2j) : 0.f;
+                    }
+                    const uint32_t hv = pack_bf16(v0, v1);
+                    hi[e / 2] = hv;
+                    lo[e / 2] = pack_bf16(v0 - bf16_lo(hv), v1 - bf16_hi(hv));
+                }
+            }
+            tmem_st16(tq + col, hi);
+            tmem_st16(tq + col + 16, lo);
+        }
+        tmem_st_wait();
+        if (!fast) {
+            // exact path: K rows scaled by e^{gamma - b_j} in place for K D
+            for (int idx = tid; idx < 384; idx += 256) {
+                const int r = idx & 127, blk = idx >> 7;
+                chunk::scale_row_sw64(sm + bv::K, r, blk, exp2f(g2 - b2s[r]));
+            }
+            fence_async_smem();
+        }
+    }
     tc_fence_before();
     __syncthreads();
+
+    // group 2: (exact path: dv = K~ D) ; dv += P~ dO  (A from tensor memory)
     if (issuer) {
         tc_fence_after();
-        // U = P^T dO (P as MN-major A, dO as MN-major B)
-        for (int part = 0; part < 2; ++part) {
-            const uint32_t pb = part ? bv::PL : bv::PH;
+        if (!fast)
+            for (int ks = 0; ks < 6; ++ks) {
+                const uint32_t off = (ks >> 1) * 8192 + (ks & 1) * 32;
+                umma_bf16(tmem + bv::TM_DV, smem_desc(sb + bv::K + off, 16, 512, kLayoutSW64),
+                          smem_desc(sb + bv::DS + ks * 1024, 6144, 512, kLayoutSW64), idV, ks > 0);
+            }
+        for (int part = 0; part < 2; ++part)
             for (int ks = 0; ks < 8; ++ks)
-                umma_bf16(tmem + bv::TM_U, smem_desc(sb + pb + ks * 2048, 16384, 1024, kLayoutSW128),
-                          smem_desc(sb + bv::DO + ks * 2048, 16384, 1024, kLayoutSW128),
-                          idesc_bf16_f32(128, 192, 1, 1), (part | ks) > 0);
-        }
+                umma_bf16_ts(tmem + bv::TM_DV, tmem + ts_hi(bv::TM_T, ks) + 16 * part,
+                             smem_desc(sb + bv::DO + ks * 1024, 8192, 512, kLayoutSW64), idV, 1);
         umma_commit(bar_m);
         pend_m = true;
     }
-    if (!mbar_wait(bar_m, 1, ctl)) failed = true;
+    if (!mbar_wait(bar_m, mph, ctl)) failed = true;
     tc_fence_before();
     if (__syncthreads_or(failed)) goto done;
-    if (issuer) pend_m = false;
     tc_fence_after();
+    if (issuer) pend_m = false;
     if (worker) {
-        // epilogue: dv = U + e^{gamma - b} W  -> staging in the dO buffer
-        const float fk = exp2f(b2s[127] - b2s[row]);
+        // epilogue: dv_j = f_j acc_j -> staging [3][128][32] SW64 in the dO buffer
+        const float f = fast ? exp2f(g2 - b2s[row]) : 1.0f;
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
-            const int n0 = half * 96 + j * 32;
-            uint32_t u[32], w[32];
-            tmem_ld32(tq + bv::TM_U + n0, u);
-            tmem_ld32(tq + bv::TM_W + n0, w);
+            const int n0 = half * 48 + j * 16;
+            uint32_t u[16];
+            tmem_ld16(tq + bv::TM_DV + n0, u);
             tmem_ld_wait();
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
+            for (int g = 0; g < 2; ++g) {
                 const int n = n0 + g * 8;
                 uint32_t pk[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    pk[e] = pack_bf16(fmaf(fk, __uint_as_float(w[g * 8 + 2 * e]), __uint_as_float(u[g * 8 + 2 * e])),
-                                      fmaf(fk, __uint_as_float(w[g * 8 + 2 * e + 1]), __uint_as_float(u[g * 8 + 2 * e + 1])));
-                *reinterpret_cast<uint4*>(sm + bv::DO + (n >> 6) * 16384 + swz_off(row, (n & 63) >> 3, 128)) =
+                    pk[e] = pack_bf16(f * __uint_as_float(u[g * 8 + 2 * e]), f * __uint_as_float(u[g * 8 + 2 * e + 1]));
+                *reinterpret_cast<uint4*>(sm + bv::DO + (n >> 5) * 8192 + swz_off(row, (n & 31) >> 3, 64)) =
                     make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
         }
         fence_async_smem();
-        tc_fence_before();
     }
+    tc_fence_before();
     __syncthreads();
     if (issuer) {
-        for (int i = 0; i < 3; ++i) tma_store_4d(&p.tm_dv, sm + bv::DO + i * 16384, i * 64, h, t0, b);
+        for (int i = 0; i < 3; ++i)
+            tma_store_4d(&p.tm_dv32, sm + bv::DO + i * 8192, dvh * 96 + i * 32, h, t0, b);
         tma_store_commit();
     }
 done:
     if (issuer) {
         if (pend_ld) mbar_wait(bar_ld, 0, ctl);
-        if (pend_m) mbar_wait(bar_m, 0, ctl) && mbar_wait(bar_m, 1, ctl);
+        if (pend_m) mbar_wait(bar_m, mph, ctl);
         tma_store_wait_all();
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 0) tmem_dealloc(tmem, bv::TMEM_COLS);
 }
 
 // ------------------------------------------------------------------ da scan
@@ -568,6 +651,9 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     if ((s = make_token_map(&bp.tm_dv, dv, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
     if ((s = make_state_map(&bp.tm_h, hbuf, static_cast<int64_t>(units) * NC)) != GLA_OK) return s;
     if ((s = make_state_map(&bp.tm_d, dbuf, static_cast<int64_t>(units) * NC)) != GLA_OK) return s;
+    if ((s = make_token_map(&bp.tm_do32, dO, kDv, pr.H, pr.T, pr.B, ldo, 32, 64)) != GLA_OK) return s;
+    if ((s = make_token_map(&bp.tm_dv32, dv, kDv, pr.H, pr.T, pr.B, ldo, 32, 64)) != GLA_OK) return s;
+    if ((s = make_state_map(&bp.tm_d32, dbuf, static_cast<int64_t>(units) * NC, 32)) != GLA_OK) return s;
     bp.a = pr.a;
     bp.delta = da;
     bp.B = pr.B;
@@ -578,7 +664,8 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     bp.ctl = ctl;
     const dim3 grid(NC, pr.H, pr.B);
     if ((s = launch_bwd_kernel(bwd_dqdk_kernel, bq::BYTES, bp, grid, st, "bwd_dqdk_kernel")) != GLA_OK) return s;
-    if ((s = launch_bwd_kernel(bwd_dv_kernel, bv::BYTES, bp, grid, st, "bwd_dv_kernel")) != GLA_OK) return s;
+    if ((s = launch_bwd_kernel(bwd_dv_kernel, bv::BYTES, bp, dim3(2 * NC, pr.H, pr.B), st, "bwd_dv_kernel")) != GLA_OK)
+        return s;
 
     // 4. da = reverse cumulative sum of delta (+ <dS_T, S_T>)
     trace_begin(st);

@@ -81,7 +81,7 @@ gla_status launch_wait_selftest(const WaitCtl& ctl, cudaStream_t st);
 struct StateParams;   // chunk_state.cuh
 gla_status make_token_map(CUtensorMap* m, const void* base, int d, int H, int T, int B,
                           int64_t ld, int box_d, int swizzle, int box_rows = 128);
-gla_status make_state_map(CUtensorMap* m, void* base, int64_t nstates);
+gla_status make_state_map(CUtensorMap* m, void* base, int64_t nstates, int box_cols = 64);
 gla_status launch_state_kernel(bool with_o, bool reverse, const StateParams& p, dim3 grid,
                                cudaStream_t st);
 

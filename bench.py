@@ -51,8 +51,8 @@ CHUNK_BYTES = {
     "chunk_state_fwd_kernel": QK + VO + A + HS,
     # state-gradient pass: read q, dO, a; write D_c     (+ dS_0 per head)
     "chunk_state_rev_kernel": QK + VO + A + HS,
-    # dq/dk: read q, k, v, dO, h, D, a; write dq, dk, delta
-    "bwd_dqdk_kernel": 2 * QK + 2 * VO + 2 * HS + A + 2 * QK + A,
+    # dq/dk: read q, k, v, dO, h, D, a; write dq, dk, q.dq and k.dk per token
+    "bwd_dqdk_kernel": 2 * QK + 2 * VO + 2 * HS + A + 2 * QK + 2 * A,
     # dv: read q, k, dO, D, a; write dv
     "bwd_dv_kernel": 2 * QK + VO + HS + A + VO,
 }

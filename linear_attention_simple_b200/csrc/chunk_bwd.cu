@@ -17,12 +17,13 @@
 //   1. state kernel, forward, state-only: h_c (bf16) for every chunk, and
 //      S_T when an upstream dS_T is given;
 //   2. state kernel, reverse: D_c (bf16) for every chunk, dS_0 = D_{-1};
-//   3. bwd_dqdk_kernel and bwd_dv_kernel: one CTA per (batch, head, chunk),
-//      fully parallel, tcgen05 for every contraction; dP and P are split
-//      into bf16 hi + lo terms; the row factors diag(...) are applied to
-//      separate TMEM accumulators in the epilogue, so no operand needs a
-//      scaled copy; the epilogue also emits q.dq - k.dk per token;
-//   4. da_scan_kernel: reverse cumulative sum over T (plus <dS_T, S_T>).
+//   3. bwd_dqdk_kernel (two CTAs per chunk: dq, dk) and bwd_dv_kernel (two
+//      CTAs per chunk: the halves of dv), fully parallel, tcgen05 for every
+//      contraction; the masked, decayed dP / P tiles stay in tensor memory
+//      as bf16 hi + lo and feed the next MMA from there; the epilogues also
+//      emit q.dq and k.dk per token and per chunk;
+//   4. da_finish_kernel: reverse cumulative sum over T (plus <dS_T, S_T>
+//      from state_dot_kernel when dS_T is given).
 #include <cstring>
 
 #include "chunk_state.cuh"
@@ -42,18 +43,13 @@ struct BwdParams {
     CUtensorMap tm_dq, tm_dk, tm_dv;       // gradient stores
     CUtensorMap tm_do32, tm_d32, tm_dv32;  // 32-column SW64 boxes (dv kernel)
     const float* a;
-    float* delta;                          // [B, T, H]: q.dq - k.dk per token
+    float* delta;                          // [B*H, T]: q.dq per token (role 0), k.dk (role 1) after it
+    float* ctot;                           // [B*H, NC, 2]: chunk totals of both halves
     int B, T, H, NC;
     float scale;
     WaitCtl ctl;
 };
 
-namespace bq {   // dq / dk kernel shared-memory map
-constexpr uint32_t Q = 0, K = 24576, V = 49152, DO = 98304, HS = 147456, DS = 184320;
-constexpr uint32_t MISC = 221184;
-constexpr uint32_t BYTES = MISC + 2048 + 1024;
-constexpr uint32_t TM_DP = 0, TM_X = 128, TM_W = 224, TM_Y = 320, TM_Z = 416;
-}  // namespace bq
 
 
 // Threads: warps 0-7 are workers; warp 8 only issues TMA and tcgen05.mma.
@@ -62,6 +58,11 @@ constexpr int kThreadsBwd = 288;
 __device__ __forceinline__ void named_sync128()
 {
     asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_sync256()
+{
+    asm volatile("bar.sync 2, 256;" ::: "memory");
 }
 
 // Inclusive cumulative log2-decay of the chunk's tokens, warps 0-3.
@@ -81,83 +82,97 @@ __device__ __forceinline__ void chunk_cumsum(float a, float* b2s, float* wsum, i
     b2s[tid] = x + pre;
 }
 
-// Masked, decayed 128x128 tile from TMEM (rows = this thread's lane, columns
-// half*64 .. +63), split into bf16 hi and lo, written [i][j] as a K-major
-// SW128 operand ([2][128][64]) at hi / lo.
-__device__ __forceinline__ void masked_decay_tile(uint32_t tq, uint32_t col0, int row, int quad,
-                                                  int half, const float* b2s, float scale,
-                                                  uint8_t* hi_base, uint8_t* lo_base)
-{
-    const float b2r = b2s[row];
-#pragma unroll
-    for (int q2 = 0; q2 < 2; ++q2) {
-        const int j0 = half * 64 + q2 * 32;
-        uint32_t hi[16], lo[16];
-        if (j0 > quad * 32 + 31) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
-        } else {
-            uint32_t r[32];
-            tmem_ld32(tq + col0 + j0, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-                const int j = j0 + e;
-                const float v0 = (j <= row) ? scale * __uint_as_float(r[e]) * exp2f(b2r - b2s[j]) : 0.f;
-                const float v1 = (j + 1 <= row) ? scale * __uint_as_float(r[e + 1]) * exp2f(b2r - b2s[j + 1]) : 0.f;
-                const uint32_t h = pack_bf16(v0, v1);
-                hi[e / 2] = h;
-                lo[e / 2] = pack_bf16(v0 - bf16_lo(h), v1 - bf16_hi(h));
-            }
-        }
-        uint8_t* hb = hi_base + half * 16384;
-        uint8_t* lb = lo_base + half * 16384;
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            const uint32_t off = swz_off(row, q2 * 4 + c4, 128);
-            *reinterpret_cast<uint4*>(hb + off) = make_uint4(hi[c4 * 4], hi[c4 * 4 + 1], hi[c4 * 4 + 2], hi[c4 * 4 + 3]);
-            *reinterpret_cast<uint4*>(lb + off) = make_uint4(lo[c4 * 4], lo[c4 * 4 + 1], lo[c4 * 4 + 2], lo[c4 * 4 + 3]);
-        }
-    }
-}
-
-__device__ __forceinline__ float bf16_at_sw64(const uint8_t* tile, int row, int d)
-{
-    const uint8_t* p = tile + (d >> 5) * 8192 + swz_off(row, (d & 31) >> 3, 64) + (d & 7) * 2;
-    return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p)) << 16);
-}
-
 // ------------------------------------------------------------ dq, dk kernel
+//
+// Two CTAs per chunk, role 0 (dq) and role 1 (dk), each 90 KB of shared
+// memory and 256 TMEM columns, so two share an SM.  With gamma the chunk's
+// total log-decay and T the masked tile of the dO / V products:
+//
+//   role 0:  dq_i = s e^{b_i} ( dO_i h^T + sum_{j <= i} (dO_i . v_j) e^{-b_j} k_j )
+//   role 1:  dk_j = e^{gamma - b_j} ( v_j D^T + sum_{i >= j} s e^{b_i - gamma} (v_j . dO_i) q_i )
+//
+// The contraction over dv (T = dO V^T for role 0, V dO^T for role 1, and the
+// state product into the accumulator) streams through two shared-memory
+// slots in three 64-column slices; T is then turned in place, in tensor
+// memory, into the bf16 hi and lo halves of the decayed tile and used as the
+// A operand of the MMA against K (role 0) or Q (role 1); the row factor is
+// applied in the epilogue.  Chunks whose decay spans more than 2^100 take
+// the exact path: the tile carries s e^{b_i - b_j}, the state product is
+// scaled in place by the row factor before the tile MMA, row factor 1.
+// Each role also writes its half of the per-token delta of the da sum,
+// q.dq (role 0) or k.dk (role 1), and that half's chunk total.
 
-__global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dqdk_kernel(const __grid_constant__ BwdParams p)
+namespace bq {   // dq / dk kernel shared-memory map
+constexpr uint32_t SLOT = 45056;         // dv slice: first [128][64], second [128][64], state [96][64], SW128
+constexpr uint32_t SECOND = 16384, STATE = 32768;
+constexpr uint32_t MISC = 2 * SLOT;
+constexpr uint32_t BYTES = MISC + 2048 + 1024;
+constexpr uint32_t TM_T = 0, TM_ACC = 128, TMEM_COLS = 256;
+constexpr uint32_t kSliceBytes = 2 * 16384 + 12288;
+constexpr uint32_t kTileBytes = 3 * 128 * 64;
+}  // namespace bq
+
+// TMEM column of the hi words of K step ks (16 tokens) of a tile kept as
+// [32-token block: 16 hi columns, 16 lo columns]; the lo words are 16 further.
+__device__ __forceinline__ uint32_t ts_hi(uint32_t base, int ks)
+{
+    return base + 32 * (ks >> 1) + 8 * (ks & 1);
+}
+
+// Phases of one mbarrier issued and waited for by the issuing thread.
+struct BarTrack {
+    int issued = 0, waited = 0;
+};
+
+__device__ __forceinline__ bool wait_next(uint64_t* bar, BarTrack& t, const WaitCtl& ctl)
+{
+    if (!mbar_wait(bar, t.waited & 1, ctl)) return false;
+    ++t.waited;
+    return true;
+}
+
+__device__ __forceinline__ void drain(uint64_t* bar, BarTrack& t, const WaitCtl& ctl)
+{
+    for (; t.waited < t.issued; ++t.waited) mbar_wait(bar, t.waited & 1, ctl);
+}
+
+__global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dqdk_kernel(const __grid_constant__ BwdParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(sm);
-    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + bq::MISC);
-    uint64_t* bar_m = bar_ld + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ld + 2);
+    uint64_t* bar_full = reinterpret_cast<uint64_t*>(sm + bq::MISC);   // [2] slot loaded
+    uint64_t* bar_free = bar_full + 2;                                  // [2] slot consumed
+    uint64_t* bar_done = bar_full + 4;                                  // all MMAs so far done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_full + 5);
     float* b2s = reinterpret_cast<float*>(sm + bq::MISC + 64);
-    float* wsum = b2s + 128;
-    float* dpart = wsum + 8;                 // [128]: delta partial of column half 1
+    float* cfs = b2s + 128;                  // [128] column factors of the fast path
+    float* wsum = cfs + 128;
+    float* dpart = wsum + 8;                 // [128] delta partial of column half 1
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int c = blockIdx.x >> 1, role = blockIdx.x & 1, h = blockIdx.y, b = blockIdx.z;
     const int unit = b * p.H + h;
     const int t0 = c * kChunk;
     const int quad = warp & 3, half = (warp >> 2) & 1, row = quad * 32 + lane;
     const bool worker = warp < 8;
     const bool issuer = warp == 8 && lane == 0;
     const WaitCtl ctl = p.ctl;
+    const CUtensorMap* tm_first = role ? &p.tm_v : &p.tm_do;
+    const CUtensorMap* tm_second = role ? &p.tm_do : &p.tm_v;
+    const CUtensorMap* tm_state = role ? &p.tm_d : &p.tm_h;
+    const CUtensorMap* tm_op = role ? &p.tm_q : &p.tm_k;      // B operand of the tile MMA
+    const CUtensorMap* tm_dot = role ? &p.tm_k : &p.tm_q;     // partner of the delta dot
+    BarTrack tr_full[2], tr_free[2], tr_done;
+    bool failed = false;
 
     if (issuer) {
-        mbar_init(bar_ld, 1);
-        mbar_init(bar_m, 1);
+        for (int i = 0; i < 5; ++i) mbar_init(bar_full + i, 1);
         mbar_init_fence();
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 512);
+        tmem_alloc(tmem_slot, bq::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -165,138 +180,225 @@ __global__ void __launch_bounds__(kThreadsBwd, 1) bwd_dqdk_kernel(const __grid_c
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tq = tmem_addr(tmem, quad * 32, 0);
-    bool failed = false;
-    bool pend_ld = false, pend_m = false;
-    float dsum = 0.f;                        // this thread's share of q.dq - k.dk
+
+    auto load_slice = [&](int sl) {
+        const int k = sl & 1;
+        uint8_t* base = sm + k * bq::SLOT;
+        mbar_arrive_expect_tx(bar_full + k, bq::kSliceBytes);
+        tma_load_4d(base, tm_first, bar_full + k, sl * 64, h, t0, b);
+        tma_load_4d(base + bq::SECOND, tm_second, bar_full + k, sl * 64, h, t0, b);
+        tma_load_3d(base + bq::STATE, tm_state, bar_full + k, sl * 64, 0, unit * p.NC + c);
+        ++tr_full[k].issued;
+    };
+    auto load_tile = [&](int k, const CUtensorMap* m) {
+        uint8_t* base = sm + k * bq::SLOT;
+        mbar_arrive_expect_tx(bar_full + k, bq::kTileBytes);
+        for (int i = 0; i < 3; ++i) tma_load_4d(base + i * 8192, m, bar_full + k, i * 32, h, t0, b);
+        ++tr_full[k].issued;
+    };
+    auto mma_slice = [&](int sl) {
+        const uint32_t base = sb + (sl & 1) * bq::SLOT;
+        for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t a = smem_desc(base + ks * 32, 16, 1024, kLayoutSW128);
+            umma_bf16(tmem + bq::TM_T, a, smem_desc(base + bq::SECOND + ks * 32, 16, 1024, kLayoutSW128),
+                      idesc_bf16_f32(128, 128, 0, 0), (sl | ks) > 0);
+            umma_bf16(tmem + bq::TM_ACC, a, smem_desc(base + bq::STATE + ks * 32, 16, 1024, kLayoutSW128),
+                      idesc_bf16_f32(128, 96, 0, 0), (sl | ks) > 0);
+        }
+    };
 
     if (issuer) {
-        mbar_arrive_expect_tx(bar_ld, 2 * chunk::kTileQK + 2 * chunk::kTileV + 2 * 36864);
-        for (int i = 0; i < 3; ++i) {
-            tma_load_4d(sm + bq::Q + i * 8192, &p.tm_q, bar_ld, i * 32, h, t0, b);
-            tma_load_4d(sm + bq::K + i * 8192, &p.tm_k, bar_ld, i * 32, h, t0, b);
-            tma_load_4d(sm + bq::V + i * 16384, &p.tm_v, bar_ld, i * 64, h, t0, b);
-            tma_load_4d(sm + bq::DO + i * 16384, &p.tm_do, bar_ld, i * 64, h, t0, b);
-            tma_load_3d(sm + bq::HS + i * 12288, &p.tm_h, bar_ld, i * 64, 0, unit * p.NC + c);
-            tma_load_3d(sm + bq::DS + i * 12288, &p.tm_d, bar_ld, i * 64, 0, unit * p.NC + c);
-        }
-        pend_ld = true;
-        if (mbar_wait(bar_ld, 0, ctl)) {
-            pend_ld = false;
-            tc_fence_after();
-            // dP_raw = dO V^T ; X = dO h^T ; W = V D^T
-            for (int ks = 0; ks < 12; ++ks) {
-                const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
-                const uint32_t soff = (ks >> 2) * 12288 + (ks & 3) * 32;
-                const uint64_t ado = smem_desc(sb + bq::DO + off, 16, 1024, kLayoutSW128);
-                const uint64_t av = smem_desc(sb + bq::V + off, 16, 1024, kLayoutSW128);
-                umma_bf16(tmem + bq::TM_DP, ado, av, idesc_bf16_f32(128, 128, 0, 0), ks > 0);
-                umma_bf16(tmem + bq::TM_X, ado, smem_desc(sb + bq::HS + soff, 16, 1024, kLayoutSW128),
-                          idesc_bf16_f32(128, 96, 0, 0), ks > 0);
-                umma_bf16(tmem + bq::TM_W, av, smem_desc(sb + bq::DS + soff, 16, 1024, kLayoutSW128),
-                          idesc_bf16_f32(128, 96, 0, 0), ks > 0);
-            }
-            umma_commit(bar_m);
-            pend_m = true;
-        } else {
-            failed = true;
-        }
+        load_slice(0);
+        load_slice(1);
     }
     if (tid < 128) {
         const int t = t0 + tid;
-        chunk_cumsum(t < p.T ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f, b2s, wsum,
-                     tid, warp, lane);
+        chunk_cumsum(t < p.T ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f, b2s, wsum, tid, warp,
+                     lane);
+        const float g2 = ((wsum[0] + wsum[1]) + wsum[2]) + wsum[3];   // the order b2s[127] sums in
+        const float b2 = b2s[tid];
+        cfs[tid] = role ? p.scale * exp2f(b2 - g2) : exp2f(-b2);
     }
-    if (!failed && !mbar_wait(bar_m, 0, ctl)) failed = true;
+    __syncthreads();
+    const float g2 = b2s[127];
+    const bool fast = -g2 <= chunk::kFactorRange;
+
+    // T and the state product over the three dv slices
+    if (issuer) {
+        bool ok = wait_next(bar_full, tr_full[0], ctl);
+        if (ok) {
+            tc_fence_after();
+            mma_slice(0);
+            umma_commit(bar_free);
+            ++tr_free[0].issued;
+            ok = wait_next(bar_full + 1, tr_full[1], ctl);
+        }
+        if (ok) {
+            tc_fence_after();
+            mma_slice(1);
+            umma_commit(bar_free + 1);
+            ++tr_free[1].issued;
+            ok = wait_next(bar_free, tr_free[0], ctl);
+        }
+        if (ok) {
+            load_slice(2);
+            ok = wait_next(bar_free + 1, tr_free[1], ctl);
+        }
+        if (ok) {
+            load_tile(1, tm_op);
+            ok = wait_next(bar_full, tr_full[0], ctl);
+        }
+        if (ok) {
+            tc_fence_after();
+            mma_slice(2);
+            umma_commit(bar_done);
+            ++tr_done.issued;
+            ok = wait_next(bar_done, tr_done, ctl);
+        }
+        if (ok) load_tile(0, tm_dot);   // slot 0 is free once every slice MMA is done
+        failed = !ok;
+    } else if (!mbar_wait(bar_done, 0, ctl)) {
+        failed = true;
+    }
     tc_fence_before();
     if (__syncthreads_or(failed)) goto done;
-    if (issuer) pend_m = false;
     tc_fence_after();
-    // dP (hi -> h buffer, lo -> D buffer; both consumed by the MMAs above)
-    if (worker) masked_decay_tile(tq, bq::TM_DP, row, quad, half, b2s, p.scale, sm + bq::HS, sm + bq::DS);
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (issuer) {
-        tc_fence_after();
-        // Y = dP K (K as MN-major B, N = dk);  Z = dP^T Q (dP as MN-major A)
-        for (int part = 0; part < 2; ++part) {
-            const uint32_t pb = part ? bq::DS : bq::HS;
-            for (int ks = 0; ks < 8; ++ks) {
-                umma_bf16(tmem + bq::TM_Y,
-                          smem_desc(sb + pb + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128),
-                          smem_desc(sb + bq::K + ks * 1024, 8192, 512, kLayoutSW64),
-                          idesc_bf16_f32(128, 96, 0, 1), (part | ks) > 0);
-                umma_bf16(tmem + bq::TM_Z, smem_desc(sb + pb + ks * 2048, 16384, 1024, kLayoutSW128),
-                          smem_desc(sb + bq::Q + ks * 1024, 8192, 512, kLayoutSW64),
-                          idesc_bf16_f32(128, 96, 1, 1), (part | ks) > 0);
+
+    if (worker) {
+        const float b2r = b2s[row];
+        const float rowf = role ? exp2f(g2 - b2r) : p.scale * exp2f(b2r);
+#pragma unroll
+        for (int kb2 = 0; kb2 < 2; ++kb2) {
+            const int c0 = half * 64 + kb2 * 32;
+            const uint32_t col = bq::TM_T + c0;
+            const bool dead = role ? (c0 + 31 < quad * 32) : (c0 > quad * 32 + 31);
+            uint32_t hi[16], lo[16];
+            if (dead) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
+            } else {
+                uint32_t r[32];
+                tmem_ld32(tq + col, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float v[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int cc = c0 + e + u;
+                        const bool keep = role ? (cc >= row) : (cc <= row);
+                        const float f = fast ? cfs[cc]
+                                             : p.scale * exp2f(role ? b2s[cc] - b2r : b2r - b2s[cc]);
+                        v[u] = keep ? __uint_as_float(r[e + u]) * f : 0.f;
+                    }
+                    const uint32_t hv = pack_bf16(v[0], v[1]);
+                    hi[e / 2] = hv;
+                    lo[e / 2] = pack_bf16(v[0] - bf16_lo(hv), v[1] - bf16_hi(hv));
+                }
+            }
+            tmem_st16(tq + col, hi);
+            tmem_st16(tq + col + 16, lo);
+        }
+        if (!fast) {
+            // exact path: the state product takes its row factor now
+#pragma unroll
+            for (int j = 0; j < 3; ++j) {
+                const uint32_t col = bq::TM_ACC + half * 48 + j * 16;
+                uint32_t u[16];
+                tmem_ld16(tq + col, u);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(rowf * __uint_as_float(u[e]));
+                tmem_st16(tq + col, u);
             }
         }
-        umma_commit(bar_m);
-        pend_m = true;
+        tmem_st_wait();
     }
-    if (!mbar_wait(bar_m, 1, ctl)) failed = true;
+    tc_fence_before();
+    __syncthreads();
+
+    // acc += tile (hi, lo) x K or Q, A from tensor memory
+    if (issuer) {
+        tc_fence_after();
+        bool ok = wait_next(bar_full + 1, tr_full[1], ctl);
+        if (ok) {
+            for (int part = 0; part < 2; ++part)
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_bf16_ts(tmem + bq::TM_ACC, tmem + ts_hi(bq::TM_T, ks) + 16 * part,
+                                 smem_desc(sb + bq::SLOT + ks * 1024, 8192, 512, kLayoutSW64),
+                                 idesc_bf16_f32(128, 96, 0, 1), 1);
+            umma_commit(bar_done);
+            ++tr_done.issued;
+            ok = wait_next(bar_done, tr_done, ctl) && wait_next(bar_full, tr_full[0], ctl);
+        }
+        failed = !ok;
+    } else if (!mbar_wait(bar_done, 1, ctl) || !mbar_wait(bar_full, 0, ctl)) {
+        failed = true;
+    }
     tc_fence_before();
     if (__syncthreads_or(failed)) goto done;
-    if (issuer) pend_m = false;
     tc_fence_after();
     if (worker) {
-        // epilogue: dq = scale e^{b} X + Y ; dk = Z + e^{gamma - b} W ; delta
-        const float b2r = b2s[row];
-        const float fq = p.scale * exp2f(b2r);
-        const float fk = exp2f(b2s[127] - b2r);
+        // epilogue: out = f acc -> staging [3][128][32] SW64 in slot 1; delta partial
+        const float f = fast ? (role ? exp2f(g2 - b2s[row]) : p.scale * exp2f(b2s[row])) : 1.0f;
+        float dsum = 0.f;
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
-            const int d0 = half * 48 + j * 16;
-            uint32_t x[16], y[16], z[16], w[16];
-            tmem_ld16(tq + bq::TM_X + d0, x);
-            tmem_ld16(tq + bq::TM_Y + d0, y);
-            tmem_ld16(tq + bq::TM_Z + d0, z);
-            tmem_ld16(tq + bq::TM_W + d0, w);
+            const int n0 = half * 48 + j * 16;
+            uint32_t u[16];
+            tmem_ld16(tq + bq::TM_ACC + n0, u);
             tmem_ld_wait();
-            float dq[16], dk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                dq[e] = fmaf(fq, __uint_as_float(x[e]), __uint_as_float(y[e]));
-                dk[e] = fmaf(fk, __uint_as_float(w[e]), __uint_as_float(z[e]));
-                dsum = fmaf(bf16_at_sw64(sm + bq::Q, row, d0 + e), dq[e], dsum);
-                dsum = fmaf(-bf16_at_sw64(sm + bq::K, row, d0 + e), dk[e], dsum);
-            }
-            // staging in the dO buffer: dq [3][128][32] SW64, dk right after
 #pragma unroll
             for (int g = 0; g < 2; ++g) {
-                const int d = d0 + g * 8;
-                const uint32_t off = (d >> 5) * 8192 + swz_off(row, (d & 31) >> 3, 64);
-                *reinterpret_cast<uint4*>(sm + bq::DO + off) =
-                    make_uint4(pack_bf16(dq[g * 8], dq[g * 8 + 1]), pack_bf16(dq[g * 8 + 2], dq[g * 8 + 3]),
-                               pack_bf16(dq[g * 8 + 4], dq[g * 8 + 5]), pack_bf16(dq[g * 8 + 6], dq[g * 8 + 7]));
-                *reinterpret_cast<uint4*>(sm + bq::DO + 24576 + off) =
-                    make_uint4(pack_bf16(dk[g * 8], dk[g * 8 + 1]), pack_bf16(dk[g * 8 + 2], dk[g * 8 + 3]),
-                               pack_bf16(dk[g * 8 + 4], dk[g * 8 + 5]), pack_bf16(dk[g * 8 + 6], dk[g * 8 + 7]));
+                const int n = n0 + g * 8;
+                const uint32_t off = (n >> 5) * 8192 + swz_off(row, (n & 31) >> 3, 64);
+                const uint4 w = *reinterpret_cast<const uint4*>(sm + off);   // q or k, slot 0
+                const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                uint32_t pk[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = f * __uint_as_float(u[g * 8 + 2 * e]);
+                    const float x1 = f * __uint_as_float(u[g * 8 + 2 * e + 1]);
+                    dsum = fmaf(bf16_lo(wv[e]), x0, dsum);
+                    dsum = fmaf(bf16_hi(wv[e]), x1, dsum);
+                    pk[e] = pack_bf16(x0, x1);
+                }
+                *reinterpret_cast<uint4*>(sm + bq::SLOT + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
         }
         if (half) dpart[row] = dsum;
         fence_async_smem();
         tc_fence_before();
+        named_sync256();
+        if (!half) {
+            const bool live = t0 + row < p.T;
+            float x = live ? dsum + dpart[row] : 0.f;
+            if (live) p.delta[(static_cast<int64_t>(role) * p.B * p.H + unit) * p.T + t0 + row] = x;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+            if (lane == 0) wsum[quad] = x;
+            named_sync128();
+            if (row == 0) p.ctot[(static_cast<int64_t>(unit) * p.NC + c) * 2 + role] = ((wsum[0] + wsum[1]) + wsum[2]) + wsum[3];
+        }
     }
     __syncthreads();
-    if (worker && !half && t0 + row < p.T)
-        p.delta[(static_cast<int64_t>(b) * p.T + t0 + row) * p.H + h] = dsum + dpart[row];
     if (issuer) {
-        for (int i = 0; i < 3; ++i) {
-            tma_store_4d(&p.tm_dq, sm + bq::DO + i * 8192, i * 32, h, t0, b);
-            tma_store_4d(&p.tm_dk, sm + bq::DO + 24576 + i * 8192, i * 32, h, t0, b);
-        }
+        const CUtensorMap* tm_out = role ? &p.tm_dk : &p.tm_dq;
+        for (int i = 0; i < 3; ++i) tma_store_4d(tm_out, sm + bq::SLOT + i * 8192, i * 32, h, t0, b);
         tma_store_commit();
     }
 done:
     if (issuer) {
-        if (pend_ld) mbar_wait(bar_ld, 0, ctl);
-        if (pend_m) mbar_wait(bar_m, 0, ctl) && mbar_wait(bar_m, 1, ctl);
+        drain(bar_full, tr_full[0], ctl);
+        drain(bar_full + 1, tr_full[1], ctl);
+        drain(bar_free, tr_free[0], ctl);
+        drain(bar_free + 1, tr_free[1], ctl);
+        drain(bar_done, tr_done, ctl);
         tma_store_wait_all();
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 0) tmem_dealloc(tmem, bq::TMEM_COLS);
 }
 
 // ----------------------------------------------------------------- dv kernel
@@ -326,11 +428,6 @@ constexpr uint32_t MISC = 92160;
 constexpr uint32_t BYTES = MISC + 1024 + 1024;
 constexpr uint32_t TM_T = 0, TM_DV = 128, TMEM_COLS = 256;
 }  // namespace bv
-
-__device__ __forceinline__ uint32_t ts_hi(uint32_t base, int ks)
-{
-    return base + 32 * (ks >> 1) + 8 * (ks & 1);
-}
 
 __global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dv_kernel(const __grid_constant__ BwdParams p)
 {
@@ -527,46 +624,69 @@ done:
     if (warp == 0) tmem_dealloc(tmem, bv::TMEM_COLS);
 }
 
-// ------------------------------------------------------------------ da scan
+// ------------------------------------------------------------------ da
 //
-// da_t = sum_{m >= t} delta_m + <dS_T, S_T>, one CTA per (batch, head):
-// each thread sums a contiguous span of tokens, the CTA scans the span
-// totals from the end, then every thread rewrites its span.
+// da_t = sum_{m >= t} (q_m . dq_m - k_m . dk_m) + <dS_T, S_T>.  One CTA of
+// 128 threads per (chunk, batch x head): the reverse inclusive scan of the
+// chunk's own tokens, plus the totals of every later chunk, plus the state
+// term (dS_T given) that state_dot_kernel wrote per (batch, head).
 
-constexpr int kScanThreads = 256;
+constexpr int kDaThreads = 128;
 
-__global__ void __launch_bounds__(kScanThreads) da_scan_kernel(float* __restrict__ da,
-                                                               const float* __restrict__ dsT,
-                                                               const float* __restrict__ sT,
-                                                               int T, int H)
+__global__ void __launch_bounds__(kDaThreads) da_finish_kernel(float* __restrict__ da,
+                                                               const float* __restrict__ delta,
+                                                               const float* __restrict__ ctot,
+                                                               const float* __restrict__ base, int T, int H,
+                                                               int NC, int units)
 {
-    __shared__ float tot[kScanThreads];
-    __shared__ float red[kScanThreads / 32];
-    const int unit = blockIdx.x;
-    const int b = unit / H, h = unit - b * H;
-    const int tid = threadIdx.x;
-    float* col = da + static_cast<int64_t>(b) * T * H + h;
-    float base = 0.f;
-    if (dsT) {
-        float s = 0.f;
-        for (int64_t e = tid; e < kSS; e += kScanThreads) s = fmaf(dsT[unit * kSS + e], sT[unit * kSS + e], s);
+    __shared__ float wtot[kDaThreads / 32], wsuf[kDaThreads / 32];
+    const int unit = blockIdx.x, c = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t = c * kChunk + tid;
+    const float* cu = ctot + static_cast<int64_t>(unit) * NC * 2;
+    float suf = 0.f;
+    for (int cc = c + 1 + tid; cc < NC; cc += kDaThreads) suf += cu[2 * cc] - cu[2 * cc + 1];
+    float x = 0.f;
+    if (t < T) x = delta[static_cast<int64_t>(unit) * T + t] - delta[(static_cast<int64_t>(units) + unit) * T + t];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if ((tid & 31) == 0) red[tid >> 5] = s;
-        __syncthreads();
-        for (int i = 0; i < kScanThreads / 32; ++i) base += red[i];
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_down_sync(0xffffffffu, x, o);
+        if (lane + o < 32) x += y;
+        suf += __shfl_xor_sync(0xffffffffu, suf, o);
     }
-    const int span = (T + kScanThreads - 1) / kScanThreads;
-    const int lo = tid * span, hi = min(T, lo + span);
-    float s = 0.f;
-    for (int t = lo; t < hi; ++t) s += col[static_cast<int64_t>(t) * H];
-    tot[tid] = s;
+    if (lane == 0) {
+        wtot[warp] = x;
+        wsuf[warp] = suf;
+    }
     __syncthreads();
-    float after = base;   // sum of all spans after this one
-    for (int i = tid + 1; i < kScanThreads; ++i) after += tot[i];
-    for (int t = hi - 1; t >= lo; --t) {
-        after += col[static_cast<int64_t>(t) * H];
-        col[static_cast<int64_t>(t) * H] = after;
+    float add = base ? base[unit] : 0.f;
+    for (int w = 0; w < kDaThreads / 32; ++w) {
+        add += wsuf[w];
+        if (w > warp) add += wtot[w];
+    }
+    if (t < T) da[(static_cast<int64_t>(unit / H) * T + t) * H + unit % H] = x + add;
+}
+
+// <dS_T, S_T> per (batch, head), one CTA each.
+__global__ void __launch_bounds__(256) state_dot_kernel(float* __restrict__ out, const float* __restrict__ dsT,
+                                                        const float* __restrict__ sT)
+{
+    __shared__ float red[8];
+    const int unit = blockIdx.x, tid = threadIdx.x;
+    const float4* x = reinterpret_cast<const float4*>(dsT + unit * kSS);
+    const float4* y = reinterpret_cast<const float4*>(sT + unit * kSS);
+    float s = 0.f;
+    for (int e = tid; e < kSS / 4; e += 256) {
+        const float4 a = x[e], b = y[e];
+        s = fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, s))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if ((tid & 31) == 0) red[tid >> 5] = s;
+    __syncthreads();
+    if (tid == 0) {
+        float r = 0.f;
+        for (int i = 0; i < 8; ++i) r += red[i];
+        out[unit] = r;
     }
 }
 
@@ -589,7 +709,8 @@ size_t bwd_workspace_bytes(int B, int T, int H)
 {
     const size_t units = static_cast<size_t>(B) * H, NC = num_chunks(T);
     const size_t states = align256(units * NC * kSS * 2);
-    return 2 * states + align256(units * kSS * sizeof(float));
+    return 2 * states + align256(units * kSS * sizeof(float)) + align256(2 * units * T * sizeof(float)) +
+           align256(units * NC * 2 * sizeof(float)) + align256(units * sizeof(float));
 }
 
 gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO,
@@ -604,6 +725,12 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     void* hbuf = wsb;
     void* dbuf = wsb + states;
     float* sT = reinterpret_cast<float*>(wsb + 2 * states);
+    size_t off = 2 * states + align256(static_cast<size_t>(units) * kSS * sizeof(float));
+    float* delta = reinterpret_cast<float*>(wsb + off);
+    off += align256(2 * static_cast<size_t>(units) * pr.T * sizeof(float));
+    float* ctot = reinterpret_cast<float*>(wsb + off);
+    off += align256(static_cast<size_t>(units) * NC * 2 * sizeof(float));
+    float* base = reinterpret_cast<float*>(wsb + off);
     const int64_t ldo = static_cast<int64_t>(pr.H) * kDv;
     gla_status s;
 
@@ -638,7 +765,7 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     rp.s_out = ds0;
     if ((s = launch_state_kernel(false, true, rp, dim3(1, pr.H, pr.B), st)) != GLA_OK) return s;
 
-    // 3. dq, dk (+ per-token delta into da) and dv
+    // 3. dq, dk (+ per-token delta halves and chunk totals) and dv
     BwdParams bp;
     memset(&bp, 0, sizeof(bp));
     const int64_t ldk = static_cast<int64_t>(pr.H) * kDk;
@@ -655,24 +782,34 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     if ((s = make_token_map(&bp.tm_dv32, dv, kDv, pr.H, pr.T, pr.B, ldo, 32, 64)) != GLA_OK) return s;
     if ((s = make_state_map(&bp.tm_d32, dbuf, static_cast<int64_t>(units) * NC, 32)) != GLA_OK) return s;
     bp.a = pr.a;
-    bp.delta = da;
+    bp.delta = delta;
+    bp.ctot = ctot;
     bp.B = pr.B;
     bp.T = pr.T;
     bp.H = pr.H;
     bp.NC = NC;
     bp.scale = pr.scale;
     bp.ctl = ctl;
-    const dim3 grid(NC, pr.H, pr.B);
-    if ((s = launch_bwd_kernel(bwd_dqdk_kernel, bq::BYTES, bp, grid, st, "bwd_dqdk_kernel")) != GLA_OK) return s;
+    if ((s = launch_bwd_kernel(bwd_dqdk_kernel, bq::BYTES, bp, dim3(2 * NC, pr.H, pr.B), st, "bwd_dqdk_kernel")) !=
+        GLA_OK)
+        return s;
     if ((s = launch_bwd_kernel(bwd_dv_kernel, bv::BYTES, bp, dim3(2 * NC, pr.H, pr.B), st, "bwd_dv_kernel")) != GLA_OK)
         return s;
 
     // 4. da = reverse cumulative sum of delta (+ <dS_T, S_T>)
+    if (ds_final) {
+        trace_begin(st);
+        state_dot_kernel<<<units, 256, 0, st>>>(base, ds_final, sT);
+        trace_end(st, "state_dot_kernel");
+        count_launch();
+        if ((s = check_launch("state_dot_kernel")) != GLA_OK) return s;
+    }
     trace_begin(st);
-    da_scan_kernel<<<units, kScanThreads, 0, st>>>(da, ds_final, ds_final ? sT : nullptr, pr.T, pr.H);
-    trace_end(st, "da_scan_kernel");
+    da_finish_kernel<<<dim3(units, NC), kDaThreads, 0, st>>>(da, delta, ctot, ds_final ? base : nullptr, pr.T, pr.H,
+                                                             NC, units);
+    trace_end(st, "da_finish_kernel");
     count_launch();
-    return check_launch("da_scan_kernel");
+    return check_launch("da_finish_kernel");
 }
 
 }  // namespace gla

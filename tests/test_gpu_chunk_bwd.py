@@ -104,3 +104,40 @@ def test_chunk_bwd_training_full_size_sampled():
     grads = gla.gla_chunk_bwd(d["q"], d["k"], d["v"], d["a"], d["dO"])
     assert gla.gla_get_device_status() == 0
     check_bwd(d, grads, units=[(0, 0), (4, 7), (7, 15)])
+
+
+@pytest.mark.parametrize("mean", [None, -8.0, 0.6])
+def test_chunk_bwd_strong_decay_and_no_decay(mean):
+    """Decays outside the workload distribution: a = 0 (no decay), a ~ -8 per
+    token (every chunk's decay spans far more than 2^100, the kernels' exact
+    path), and logsigmoid(N(0.6, 1)) (chunk decays between 2^-111 and 2^-93,
+    so fast and exact chunks mix in one sequence).  Magnitudes here are not the
+    workloads', so bounds are relative: rel L2 <= 1e-2 and max-abs <= 1e-2 *
+    max|ref| for dq, dk, dv, dS_0.
+
+    da is a sum of terms that cancel: under a ~ -8 the diagonal parts of q.dq
+    and k.dk cancel, and <dS_T, S_T> cancels k_T . (dS_T v_T), leaving da some
+    three orders of magnitude below the terms.  The per-chunk state copies the
+    kernels read are bf16, so da's absolute error is bounded by their rounding
+    of those terms; its bound is max-abs <= 1e-2 * the larger of max|da| and
+    the largest cancelling term (max |q.dq|, |k.dk|, |<dS_T, S_T>|)."""
+    B, T, H = 2, 512, 2
+    seed = 230 if mean is None else 231 + int(mean * 10)
+    d = inputs.chunk_inputs(B, T, H, seed=seed, device="cuda", s0_std=0.1, with_dO=True)
+    d["a"] = (torch.zeros_like(d["a"]) if mean is None
+              else inputs.log_decay((B, T, H), seed, "cuda", mean=mean))
+    ds = inputs.randn((B, H, 96, 192), seed + 1, "cuda", std=0.1)
+    grads = gla.gla_chunk_bwd(d["q"], d["k"], d["v"], d["a"], d["dO"], s0=d["s0"], ds_final=ds)
+    assert gla.gla_get_device_status() == 0
+    q, k, v, a, dO = [_np(d[n]) for n in ("q", "k", "v", "a", "dO")]
+    ref = recurrent.bwd(q, k, v, a, dO, _np(d["s0"]), _np(ds))
+    for name, g, r in zip(("dq", "dk", "dv", "ds0"), grads[:3] + grads[4:], ref[:3] + ref[4:]):
+        got = _np(g)
+        assert rel_l2(got, r) <= 1e-2, "%s rel L2 %.3g" % (name, rel_l2(got, r))
+        assert np.max(np.abs(got - r)) <= 1e-2 * np.max(np.abs(r)), name
+    _, s_T = recurrent.fwd(q, k, v, a, _np(d["s0"]))
+    terms = max(np.max(np.abs(np.einsum("bthd,bthd->bth", q, ref[0]))),
+                np.max(np.abs(np.einsum("bthd,bthd->bth", k, ref[1]))),
+                np.max(np.abs(np.einsum("bhij,bhij->bh", _np(ds), s_T))))
+    err = np.max(np.abs(_np(grads[3]) - ref[3]))
+    assert err <= 1e-2 * max(np.max(np.abs(ref[3])), terms), "da max-abs %.3g (terms %.3g)" % (err, terms)

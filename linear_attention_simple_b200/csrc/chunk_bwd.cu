@@ -739,7 +739,6 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     memset(&sp, 0, sizeof(sp));
     if ((s = make_token_map(&sp.tm_u, pr.k, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&sp.tm_y, pr.v, kDv, pr.H, pr.T, pr.B, pr.ld_v, 64, 128)) != GLA_OK) return s;
-    if ((s = make_state_map(&sp.tm_h, hbuf, static_cast<int64_t>(units) * NC)) != GLA_OK) return s;
     sp.a = pr.a;
     sp.s_init = s0;
     sp.init_unit_stride = kSS;
@@ -752,6 +751,7 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     sp.NC = NC;
     sp.chunks_per_seg = NC;
     sp.store_h = 1;
+    sp.h_out = hbuf;
     sp.scale = pr.scale;
     sp.ctl = ctl;
     if ((s = launch_state_kernel(false, false, sp, dim3(1, pr.H, pr.B), st)) != GLA_OK) return s;
@@ -760,7 +760,7 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     StateParams rp = sp;
     if ((s = make_token_map(&rp.tm_u, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&rp.tm_y, dO, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
-    if ((s = make_state_map(&rp.tm_h, dbuf, static_cast<int64_t>(units) * NC)) != GLA_OK) return s;
+    rp.h_out = dbuf;
     rp.s_init = ds_final;
     rp.s_out = ds0;
     if ((s = launch_state_kernel(false, true, rp, dim3(1, pr.H, pr.B), st)) != GLA_OK) return s;

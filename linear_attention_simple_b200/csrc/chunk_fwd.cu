@@ -63,12 +63,12 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(float* __restrict__ st
 
 template <typename K>
 gla_status launch_chunk_kernel(K kernel, uint32_t bytes, const char* name, const StateParams& p,
-                               dim3 grid, cudaStream_t st)
+                               dim3 grid, cudaStream_t st, int threads = chunk::kThreads)
 {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
         return check_launch("cudaFuncSetAttribute");
     trace_begin(st);
-    kernel<<<grid, chunk::kThreads, bytes, st>>>(p);
+    kernel<<<grid, threads, bytes, st>>>(p);
     trace_end(st, name);
     count_launch();
     return check_launch(name);
@@ -105,10 +105,10 @@ gla_status launch_state_kernel(bool with_o, bool reverse, const StateParams& p, 
                                    "chunk_fwd_fused_kernel", p, grid, st);
     if (!with_o && !reverse)
         return launch_chunk_kernel(gla_state_pass_kernel<false>, chunk::PassSmem::BYTES,
-                                   "chunk_state_fwd_kernel", p, grid, st);
+                                   "chunk_state_fwd_kernel", p, grid, st, chunk::kPassThreads);
     if (!with_o && reverse)
         return launch_chunk_kernel(gla_state_pass_kernel<true>, chunk::PassSmem::BYTES,
-                                   "chunk_state_rev_kernel", p, grid, st);
+                                   "chunk_state_rev_kernel", p, grid, st, chunk::kPassThreads);
     return GLA_ERR_UNSUPPORTED;
 }
 

@@ -28,10 +28,14 @@
 //   the four TMEM lane quarters (each owned by one SM sub-partition) gets an
 //   equal share of the causal triangle.
 //
-// gla_state_pass_kernel<REVERSE> -- state only: S (or D) += U~^T Y per chunk
-//   with U~ split into bf16 hi + lo, optionally storing the bf16 state before
-//   each chunk's update (the backward's h_c and D_c).  Tiles are double
-//   buffered: the next-but-one chunk's tiles load while a chunk computes.
+// gla_state_pass_kernel<REVERSE> -- state only: S (or D) = e^gamma S + U~^T Y
+//   per chunk with U~ split into bf16 hi + lo, optionally storing the bf16
+//   state before each chunk's update (the backward's h_c and D_c).  Twelve
+//   warps hold S in registers (dk row, a quarter of dv each); per chunk they write the
+//   next chunk's decayed U~^T (hi, lo) into one of two TMEM buffers while the
+//   current chunk's dS = U~^T Y runs on the tensor core with A read from
+//   TMEM, then fold dS into S and store the bf16 copy.  Warp 15 issues the
+//   loads (a three-stage ring, two chunks ahead) and the MMAs.
 //
 // Operand layouts (validated against the hardware): q and k tiles are
 // TMA-loaded as three 32-wide SW64 boxes ([3][128][32]; K-major for the
@@ -58,7 +62,6 @@ struct StateParams {
     CUtensorMap tm_u;       // scaled operand: k (forward) or q (reverse)
     CUtensorMap tm_y;       // v (forward) or dO (reverse)
     CUtensorMap tm_o;       // o tile stores (fused forward)
-    CUtensorMap tm_h;       // per-chunk bf16 state stores (store_h)
     const float* a;         // [B, T, H] log-decay
     const float* s_init;    // initial state per (unit, seg) or null (zeros)
     float* s_out;           // state after the segment, or null
@@ -68,7 +71,8 @@ struct StateParams {
     int B, T, H, NC, chunks_per_seg;
     int out_last_only;      // write s_out only from the last segment
     int g2_unit_stride;     // segments per unit in g2_out
-    int store_h;            // store the bf16 state entering each chunk
+    int store_h;            // store the bf16 state entering each chunk into h_out
+    void* h_out;            // bf16 [B*H*NC][96][192]
     float scale;
     WaitCtl ctl;
 };
@@ -78,6 +82,9 @@ namespace chunk {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kWorkers = 256;
 constexpr int kThreads = kWorkers + 32;
+// state pass: 16 warps; w % 4 < 3 for w < 15 are the 12 workers (TMEM lanes
+// 0..95 = the dk rows, four column quarters), warp 15 issues
+constexpr int kPassThreads = 512;
 constexpr uint32_t kTileQK = 3 * 128 * 64;     // 24576 bytes
 constexpr uint32_t kTileV = 3 * 128 * 128;     // 49152 bytes
 constexpr float kFactorRange = 100.0f;         // max log2 span for the factorised decay
@@ -85,6 +92,7 @@ constexpr float kFactorRange = 100.0f;         // max log2 span for the factoris
 constexpr uint32_t kIdScores = idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint32_t kIdOut = idesc_bf16_f32(128, 192, 0, 1);
 constexpr uint32_t kIdState = idesc_bf16_f32(128, 192, 1, 1);
+constexpr uint32_t kIdStateTs = idesc_bf16_f32(128, 192, 0, 1);   // A from tensor memory
 
 // Shared-memory maps (bytes from a 1024-aligned base).
 struct FusedSmem {
@@ -100,15 +108,15 @@ struct FusedSmem {
     static constexpr uint32_t TM_SC = 0, TM_O = 128, TM_S = 320;
 };
 struct PassSmem {
-    static constexpr uint32_t U0 = 0, U1 = 24576;   // U0's 4th M block is U1, U1's is UL
-    static constexpr uint32_t UL = 49152;           // U~ lo (its 4th M block is Z)
-    static constexpr uint32_t Z = 73728;            // zeros
-    static constexpr uint32_t Y0 = 81920, Y1 = 131072;
-    static constexpr uint32_t X = 180224;           // bf16 state copy (store_h)
-    static constexpr uint32_t MISC = 217088;
-    static constexpr uint32_t BYTES = MISC + 1024 + 1024;
-    static constexpr uint32_t TMEM_COLS = 256;
-    static constexpr uint32_t TM_S = 0;
+    // three stages of (U [3][128][32] SW64, Y [3][128][64] SW128)
+    static constexpr uint32_t STAGE = 73728, Y = 24576;
+    static constexpr int kStages = 3;
+    static constexpr uint32_t MISC = kStages * STAGE;
+    static constexpr uint32_t XPOSE = MISC + 1024;       // [12 warps][8 rows][96 B] store transpose
+    static constexpr uint32_t BYTES = XPOSE + 12 * 768 + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    // dS accumulator [192 cols]; U~^T hi (64 cols) + lo (64 cols) per buffer, two buffers
+    static constexpr uint32_t TM_DS = 0, TM_U = 256;
 };
 
 // Token held by row r of the permuted q tile: 16-row block r/16 holds token
@@ -592,7 +600,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const
 // State-only pass (double-buffered tiles).
 // =====================================================================
 template <bool REVERSE>
-__global__ void __launch_bounds__(chunk::kThreads, 1) gla_state_pass_kernel(const __grid_constant__ StateParams p)
+__global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(const __grid_constant__ StateParams p)
 {
     using namespace chunk;
     using L = PassSmem;
@@ -600,12 +608,13 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_state_pass_kernel(cons
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(sm);
-    uint64_t* bar_u = reinterpret_cast<uint64_t*>(sm + L::MISC);   // [2]
-    uint64_t* bar_y = bar_u + 2;                                    // [2]
-    uint64_t* bar_m = bar_u + 4;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_u + 5);
-    float* b2s = reinterpret_cast<float*>(sm + L::MISC + 64);
-    float* wsum = b2s + 128;
+    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + L::MISC);   // [3] stage loaded
+    uint64_t* bar_free = bar_ld + 3;                                // [3] stage's MMAs done
+    uint64_t* bar_split = bar_ld + 6;                               // [2] U~^T buffer written (384)
+    uint64_t* bar_mma = bar_ld + 8;                                 // [2] dS of chunk parity done
+    uint64_t* bar_read = bar_ld + 10;                               // dS read by the workers (384)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ld + 11);
+    constexpr uint32_t kWork = 384;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -614,26 +623,25 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_state_pass_kernel(cons
     const int c_end = min(p.NC, c_begin + p.chunks_per_seg);
     const int nchunks = c_end - c_begin;
     const WaitCtl ctl = p.ctl;
-
-    const int quad = warp & 3, row = quad * 32 + lane, half = (warp >> 2) & 1;
-    const bool worker = warp < 8;
-    const bool srow = worker && quad < 3;
-    const bool issuer = warp == 8 && lane == 0;
+    const int quad = warp & 3, row = quad * 32 + lane, qt = warp >> 2;
+    const bool worker = warp < 15 && quad < 3;     // TMEM lanes 0..95: row = dk index
+    const bool issuer = warp == 15 && lane == 0;
+    const bool producer = warp == 11 && lane == 0;
 
     if (issuer) {
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(bar_u + s, 1);
-            mbar_init(bar_y + s, 1);
+        for (int i = 0; i < 3; ++i) {
+            mbar_init(bar_ld + i, 1);
+            mbar_init(bar_free + i, 1);
         }
-        mbar_init(bar_m, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_split + i, kWork);
+            mbar_init(bar_mma + i, 1);
+        }
+        mbar_init(bar_read, kWork);
         mbar_init_fence();
         tma_prefetch_desc(&p.tm_u);
         tma_prefetch_desc(&p.tm_y);
-        if (p.store_h) tma_prefetch_desc(&p.tm_h);
     }
-    for (int i = tid * 16; i < 8192; i += kThreads * 16)
-        *reinterpret_cast<uint4*>(sm + L::Z + i) = make_uint4(0u, 0u, 0u, 0u);
-    fence_async_smem();
     if (warp == 0) {
         tmem_alloc(tmem_slot, L::TMEM_COLS);
         tmem_relinquish();
@@ -642,129 +650,231 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_state_pass_kernel(cons
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tq = tmem_addr(tmem, quad * 32, 0);
-
     auto chunk_at = [&](int it) { return REVERSE ? (c_end - 1 - it) : (c_begin + it); };
-    auto load_a = [&](int c) {
-        const int t = c * 128 + tid;
-        return t < p.T ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f;
-    };
-    int pend = 0;                              // bit s: stage s has loads in flight
-    uint32_t ph_ld[2] = {0u, 0u};
-    uint32_t mph = 0;
-    bool pend_m = false;
-    auto issue = [&](int c, int s) {
-        const int t0 = c * 128;
-        uint8_t* u = sm + (s ? L::U1 : L::U0);
-        uint8_t* y = sm + (s ? L::Y1 : L::Y0);
-        mbar_arrive_expect_tx(bar_u + s, kTileQK);
-        for (int i = 0; i < 3; ++i) tma_load_4d(u + i * 8192, &p.tm_u, bar_u + s, i * 32, h, t0, b);
-        mbar_arrive_expect_tx(bar_y + s, kTileV);
-        for (int i = 0; i < 3; ++i) tma_load_4d(y + i * 16384, &p.tm_y, bar_y + s, i * 64, h, t0, b);
-        pend |= 1 << s;
-    };
 
-    if (issuer) {
-        if (nchunks > 0) issue(chunk_at(0), 0);
-        if (nchunks > 1) issue(chunk_at(1), 1);
-    }
-    float a_cur = (tid < 128 && nchunks > 0) ? load_a(chunk_at(0)) : 0.f;
-    if (srow) {
-        const float* src = p.s_init ? p.s_init + unit * p.init_unit_stride + seg * p.init_seg_stride +
-                                          row * kDv + half * 96
-                                    : nullptr;
-        state_to_tmem(src, tq + L::TM_S + half * 96);
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    bool failed = false, aborted = false;
-    float gsum2 = 0.f;
-    for (int it = 0; it < nchunks; ++it) {
-        const int c = chunk_at(it);
-        const int s = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        uint8_t* u = sm + (s ? L::U1 : L::U0);
-        const uint32_t ua = s ? L::U1 : L::U0, ya = s ? L::Y1 : L::Y0;
-        const float a_nxt = (tid < 128 && it + 1 < nchunks) ? load_a(chunk_at(it + 1)) : 0.f;
-
-        // (A) cumulative decay
-        if (tid < 128) b2s[tid] = chunk_cumsum(a_cur, wsum, warp, lane);
-        __syncthreads();
-        const float g2 = b2s[127];
-        gsum2 += g2;
-
-        // (B) store-copy (bf16) and decay of the state
-        if (srow)
-            state_copy_and_decay<false>(tq + L::TM_S + half * 96, row, half, exp2f(g2), sm + L::X,
-                                        nullptr, p.store_h != 0);
-
-        // (C) U~ = w U split into hi (in place) + lo
-        if (!mbar_wait(bar_u + s, ph, ctl)) failed = true;
-        if (!failed && worker) {
-            for (int idx = tid; idx < 384; idx += kWorkers) {
-                const int r = idx & 127, blk = idx >> 7;
-                const float f = REVERSE ? p.scale * exp2f(b2s[r]) : exp2f(g2 - b2s[r]);
-                split_row_sw64(u, sm + L::UL, r, blk, f);
+    if (producer) {
+        // -------------------------------------------------------- producer
+        // chunk it goes to stage it % 3 as soon as the MMAs of chunk it-3,
+        // the stage's previous user, are done
+        int n_ld[3] = {0, 0, 0};
+        for (int it = 0; it < nchunks; ++it) {
+            const int st = it % 3;
+            if (it >= 3 && !mbar_wait(bar_free + st, ((it - 3) / 3) & 1, ctl)) break;
+            const int t0 = chunk_at(it) * 128;
+            uint8_t* base = sm + st * L::STAGE;
+            mbar_arrive_expect_tx(bar_ld + st, kTileQK + kTileV);
+            for (int i = 0; i < 3; ++i) {
+                tma_load_4d(base + i * 8192, &p.tm_u, bar_ld + st, i * 32, h, t0, b);
+                tma_load_4d(base + L::Y + i * 16384, &p.tm_y, bar_ld + st, i * 64, h, t0, b);
             }
+            ++n_ld[st];
         }
-        fence_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(failed)) { aborted = true; break; }
-        tc_fence_after();
-
-        // (D) store the state copy; S += U~^T Y
-        if (issuer) {
-            if (p.store_h) {
-                for (int i = 0; i < 3; ++i)
-                    tma_store_3d(&p.tm_h, sm + L::X + i * 12288, i * 64, 0, unit * p.NC + c);
-                tma_store_commit();
-            }
-            if (mbar_wait(bar_y + s, ph, ctl)) {
-                pend &= ~(1 << s);
-                ph_ld[s] ^= 1;
-#pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    const uint32_t abase = part ? L::UL : ua;
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        umma_bf16(tmem + L::TM_S, smem_desc(sb + abase + ks * 1024, 8192, 512, kLayoutSW64),
-                                  smem_desc(sb + ya + ks * 2048, 16384, 1024, kLayoutSW128), kIdState, 1);
-                }
-                umma_commit(bar_m);
-                pend_m = true;
-            } else {
-                failed = true;
-            }
-        }
-
-        // (E) wait for the update; refill this stage with chunk it+2
-        if (!mbar_wait(bar_m, mph, ctl)) failed = true;
-        if (issuer && p.store_h) tma_store_wait_read();
-        if (__syncthreads_or(failed)) { aborted = true; break; }
-        if (issuer) pend_m = false;
-        mph ^= 1;
-        tc_fence_after();
-        if (issuer && it + 2 < nchunks) issue(chunk_at(it + 2), s);
-        a_cur = a_nxt;
-    }
-
-    if (!aborted) {
-        const bool write_state = p.s_out && (!p.out_last_only || seg == static_cast<int>(gridDim.x) - 1);
-        if (write_state && srow)
-            tmem_to_state(tq + L::TM_S + half * 96,
-                          p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + half * 96);
-        if (p.g2_out && tid == 0) p.g2_out[static_cast<int64_t>(unit) * p.g2_unit_stride + seg] = gsum2;
+        // at most one load per stage is ever outstanding: waiting for the last
+        // one issued waits for everything in flight
+        for (int i = 0; i < 3; ++i)
+            if (n_ld[i]) mbar_wait(bar_ld + i, (n_ld[i] - 1) & 1, ctl);
     } else if (issuer) {
-        for (int s = 0; s < 2; ++s)
-            if (pend & (1 << s)) {
-                mbar_wait(bar_u + s, ph_ld[s], ctl);
-                mbar_wait(bar_y + s, ph_ld[s], ctl);
+        // ---------------------------------------------------------- issuer
+        int n_mma[2] = {0, 0}, n_free[3] = {0, 0, 0};
+        for (int it = 0; it < nchunks; ++it) {
+            if (!mbar_wait(bar_split + (it & 1), (it >> 1) & 1, ctl)) break;
+            if (it >= 1 && !mbar_wait(bar_read, (it - 1) & 1, ctl)) break;
+            tc_fence_after();
+            const uint32_t ya = sb + (it % 3) * L::STAGE + L::Y;
+            const uint32_t ua = tmem + L::TM_U + (it & 1) * 128;
+            const uint64_t yd = smem_desc(ya, 16384, 1024, kLayoutSW128);
+#pragma unroll
+            for (int part = 0; part < 2; ++part)
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_bf16_ts(tmem + L::TM_DS, ua + part * 64 + ks * 8, desc_add(yd, ks * 2048), kIdStateTs,
+                                 (part | ks) > 0);
+            umma_commit(bar_mma + (it & 1));
+            umma_commit(bar_free + it % 3);
+            ++n_mma[it & 1];
+            ++n_free[it % 3];
+        }
+        // at most one phase of each barrier is ever outstanding
+        for (int i = 0; i < 2; ++i)
+            if (n_mma[i]) mbar_wait(bar_mma + i, (n_mma[i] - 1) & 1, ctl);
+        for (int i = 0; i < 3; ++i)
+            if (n_free[i]) mbar_wait(bar_free + i, (n_free[i] - 1) & 1, ctl);
+    } else if (worker) {
+        // ---------- state in registers (row `row`, columns 48 qt .. +47)
+        float S[48];
+        const float* src = p.s_init ? p.s_init + unit * p.init_unit_stride + seg * p.init_seg_stride +
+                                          row * kDv + qt * 48
+                                    : nullptr;
+#pragma unroll
+        for (int e = 0; e < 48; e += 4) {
+            const float4 v = src ? *reinterpret_cast<const float4*>(src + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+            S[e] = v.x;
+            S[e + 1] = v.y;
+            S[e + 2] = v.z;
+            S[e + 3] = v.w;
+        }
+        const uint32_t tq = tmem_addr(tmem, quad * 32, 0);
+        // this lane holds tokens 4*lane .. +3 of the chunk's decay scan
+        auto load_a = [&](int it, float (&x)[4]) {
+            const int c = chunk_at(it);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int t = c * 128 + lane * 4 + e;
+                x[e] = (it < nchunks && t < p.T) ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f;
             }
-        if (pend_m) mbar_wait(bar_m, mph, ctl);
+        };
+        // the chunk's per-token factors f (for U~ = f U) and its total log2-decay
+        auto scan = [&](const float (&x)[4], float (&f)[4]) {
+            float c4[4];
+            c4[0] = x[0] * kLog2e;
+#pragma unroll
+            for (int e = 1; e < 4; ++e) c4[e] = c4[e - 1] + x[e] * kLog2e;
+            float incl = c4[3];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const float up = __shfl_up_sync(0xffffffffu, incl, 1);
+            const float pre = lane ? up : 0.f;
+            const float g2 = __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) f[e] = REVERSE ? p.scale * exp2f(pre + c4[e]) : exp2f(g2 - (pre + c4[e]));
+            return g2;
+        };
+        // U~^T (row = dk index, columns = tokens 32 qt .. +31) -> TMEM buffer.
+        // Element (t, d) of the [3][128][32] SW64 tile sits at block d/32, byte
+        // 64 t + 16 ((d%32)/8 ^ (t/2)%4) + 2 (d%8); for t = 32 qt + 2 q the
+        // xor term is q % 4, so every load has a constant offset.
+        const uint32_t cb = lane >> 3;
+        const uint32_t sw[4] = {(cb ^ 0u) * 16 + (lane & 7) * 2, (cb ^ 1u) * 16 + (lane & 7) * 2,
+                                (cb ^ 2u) * 16 + (lane & 7) * 2, (cb ^ 3u) * 16 + (lane & 7) * 2};
+        auto split = [&](int it, const float (&f)[4]) {
+            const uint8_t* u = sm + (it % 3) * L::STAGE + quad * 8192 + qt * 32 * 64;
+            const uint32_t dst = tq + L::TM_U + (it & 1) * 128 + qt * 16;
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                uint32_t hi[8], lo[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int tl = g * 16 + 2 * q;           // token within this quarter
+                    const int t = qt * 32 + tl;
+                    const float f0 = __shfl_sync(0xffffffffu, f[tl & 3], t >> 2);
+                    const float f1 = __shfl_sync(0xffffffffu, f[(tl + 1) & 3], (t + 1) >> 2);
+                    const uint32_t o = sw[q & 3];
+                    const float k0 = __uint_as_float(
+                        static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(u + tl * 64 + o)) << 16);
+                    const float k1 = __uint_as_float(
+                        static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(u + tl * 64 + 64 + o)) << 16);
+                    const float v0 = k0 * f0, v1 = k1 * f1;
+                    const uint32_t hv = pack_bf16(v0, v1);
+                    hi[q] = hv;
+                    lo[q] = pack_bf16(v0 - bf16_lo(hv), v1 - bf16_hi(hv));
+                }
+                tmem_st8(dst + g * 8, hi);
+                tmem_st8(dst + 64 + g * 8, lo);
+            }
+            tmem_st_wait();
+        };
+        // bf16 copy of S (96 B of this thread's row) -> h_out, eight rows of the
+        // warp at a time through a shared-memory transpose so that each store
+        // instruction writes whole 96-byte row segments
+        uint8_t* xp = sm + L::XPOSE + ((warp >> 2) * 3 + quad) * 768;
+        auto store_h = [&](int it) {
+            uint8_t* hrow0 = static_cast<uint8_t*>(p.h_out) +
+                             ((static_cast<int64_t>(unit) * p.NC + chunk_at(it)) * kDk + quad * 32) * (kDv * 2) + qt * 96;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if ((lane >> 3) == k) {
+                    uint4* dst = reinterpret_cast<uint4*>(xp + (lane & 7) * 96);
+#pragma unroll
+                    for (int q = 0; q < 6; ++q)
+                        dst[q] = make_uint4(pack_bf16(S[8 * q], S[8 * q + 1]), pack_bf16(S[8 * q + 2], S[8 * q + 3]),
+                                            pack_bf16(S[8 * q + 4], S[8 * q + 5]),
+                                            pack_bf16(S[8 * q + 6], S[8 * q + 7]));
+                }
+                __syncwarp();
+#pragma unroll
+                for (int j0 = 0; j0 < 48; j0 += 32) {
+                    const int j = j0 + lane;       // piece j: row j / 6, 16-byte part j % 6
+                    if (j < 48)
+                        *reinterpret_cast<uint4*>(hrow0 + (8 * k + j / 6) * (kDv * 2) + (j % 6) * 16) =
+                            *reinterpret_cast<const uint4*>(xp + j * 16);
+                }
+                __syncwarp();
+            }
+        };
+
+        bool ok = true;
+        float gsum2 = 0.f;
+        float xa[4], f[4];
+        float g2 = 0.f;
+        if (nchunks > 0) {
+            load_a(0, xa);
+            g2 = scan(xa, f);
+            load_a(1, xa);
+            if (p.store_h) store_h(0);
+            if (mbar_wait(bar_ld, 0, ctl)) {
+                tc_fence_after();
+                split(0, f);
+                tc_fence_before();
+                mbar_arrive(bar_split);
+            } else {
+                ok = false;
+            }
+        }
+        for (int it = 0; ok && it < nchunks; ++it) {
+            const float g2_cur = g2;
+            if (it + 1 < nchunks) {
+                float fn[4];
+                g2 = scan(xa, fn);
+                load_a(it + 2, xa);
+                const int nx = it + 1;
+                if (!mbar_wait(bar_ld + nx % 3, (nx / 3) & 1, ctl) ||
+                    (it >= 1 && !mbar_wait(bar_mma + ((it - 1) & 1), ((it - 1) >> 1) & 1, ctl))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                split(nx, fn);
+                tc_fence_before();
+                mbar_arrive(bar_split + (nx & 1));
+            }
+            if (!mbar_wait(bar_mma + (it & 1), (it >> 1) & 1, ctl)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float fd = exp2f(g2_cur);
+            gsum2 += g2_cur;
+            {
+                uint32_t r0[16], r1[16], r2[16];
+                tmem_ld16(tq + L::TM_DS + qt * 48, r0);
+                tmem_ld16(tq + L::TM_DS + qt * 48 + 16, r1);
+                tmem_ld16(tq + L::TM_DS + qt * 48 + 32, r2);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    S[e] = fmaf(fd, S[e], __uint_as_float(r0[e]));
+                    S[16 + e] = fmaf(fd, S[16 + e], __uint_as_float(r1[e]));
+                    S[32 + e] = fmaf(fd, S[32 + e], __uint_as_float(r2[e]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar_read);
+            if (p.store_h && it + 1 < nchunks) store_h(it + 1);
+        }
+        if (ok) {
+            const bool write_state = p.s_out && (!p.out_last_only || seg == static_cast<int>(gridDim.x) - 1);
+            if (write_state) {
+                float* dst = p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + qt * 48;
+#pragma unroll
+                for (int e = 0; e < 48; e += 4)
+                    *reinterpret_cast<float4*>(dst + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+            }
+            if (p.g2_out && tid == 0) p.g2_out[static_cast<int64_t>(unit) * p.g2_unit_stride + seg] = gsum2;
+        }
     }
-    if (issuer) tma_store_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);

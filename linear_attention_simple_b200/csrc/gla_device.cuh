@@ -286,6 +286,13 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait()
 {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -310,6 +317,14 @@ __device__ __forceinline__ uint32_t tmem_addr(uint32_t base, uint32_t lane, uint
 // (64 B of elements per atom row for SW64, 128 B for SW128) and SBO the
 // distance between consecutive 8-row groups along K.
 enum : uint32_t { kLayoutSW128 = 2u, kLayoutSW64 = 4u, kLayoutSW32 = 6u };
+
+// A descriptor for `bytes` further on: the start address is the low 14-bit
+// field in 16-byte units, and shared-memory addresses stay below 256 KB, so
+// the add never carries out of the field.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes)
+{
+    return d + static_cast<uint64_t>(bytes >> 4);
+}
 
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
                                               uint32_t layout)

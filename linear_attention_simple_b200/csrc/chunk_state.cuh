@@ -31,11 +31,12 @@
 // gla_state_pass_kernel<REVERSE> -- state only: S (or D) = e^gamma S + U~^T Y
 //   per chunk with U~ split into bf16 hi + lo, optionally storing the bf16
 //   state before each chunk's update (the backward's h_c and D_c).  Twelve
-//   warps hold S in registers (dk row, a quarter of dv each); per chunk they write the
-//   next chunk's decayed U~^T (hi, lo) into one of two TMEM buffers while the
-//   current chunk's dS = U~^T Y runs on the tensor core with A read from
-//   TMEM, then fold dS into S and store the bf16 copy.  Warp 15 issues the
-//   loads (a three-stage ring, two chunks ahead) and the MMAs.
+//   warps hold S in registers (dk row, a quarter of dv each); per chunk they
+//   write the next chunk's decayed U~^T (hi, lo) into one of two TMEM buffers
+//   while the current chunk's dS = U~^T Y runs on the tensor core with A read
+//   from TMEM, then fold dS into S and store the bf16 copy.  Warp 3 scans the
+//   decays ahead into a ring of per-token factors, warp 11 issues the loads
+//   (a three-stage ring) and warp 15 the MMAs.
 //
 // Operand layouts (validated against the hardware): q and k tiles are
 // TMA-loaded as three 32-wide SW64 boxes ([3][128][32]; K-major for the
@@ -111,9 +112,9 @@ struct PassSmem {
     // three stages of (U [3][128][32] SW64, Y [3][128][64] SW128)
     static constexpr uint32_t STAGE = 73728, Y = 24576;
     static constexpr int kStages = 3;
-    static constexpr uint32_t MISC = kStages * STAGE;
-    static constexpr uint32_t XPOSE = MISC + 1024;       // [12 warps][8 rows][96 B] store transpose
-    static constexpr uint32_t BYTES = XPOSE + 12 * 768 + 1024;
+    static constexpr uint32_t MISC = kStages * STAGE;     // barriers, g2 ring
+    static constexpr uint32_t FRING = MISC + 256;         // [4][128] per-token decay factors
+    static constexpr uint32_t BYTES = FRING + 2048 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     // dS accumulator [192 cols]; U~^T hi (64 cols) + lo (64 cols) per buffer, two buffers
     static constexpr uint32_t TM_DS = 0, TM_U = 256;
@@ -613,7 +614,11 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
     uint64_t* bar_split = bar_ld + 6;                               // [2] U~^T buffer written (384)
     uint64_t* bar_mma = bar_ld + 8;                                 // [2] dS of chunk parity done
     uint64_t* bar_read = bar_ld + 10;                               // dS read by the workers (384)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ld + 11);
+    uint64_t* bar_f = bar_ld + 11;                                  // [4] decay factors ready (32)
+    uint64_t* bar_fdone = bar_ld + 15;                              // [4] decay factors used (384)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ld + 19);
+    float* g2s = reinterpret_cast<float*>(sm + L::MISC + 192);      // [4] chunk log2-decay
+    float* fring = reinterpret_cast<float*>(sm + L::FRING);
     constexpr uint32_t kWork = 384;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -627,6 +632,7 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
     const bool worker = warp < 15 && quad < 3;     // TMEM lanes 0..95: row = dk index
     const bool issuer = warp == 15 && lane == 0;
     const bool producer = warp == 11 && lane == 0;
+    const bool decay = warp == 3;
 
     if (issuer) {
         for (int i = 0; i < 3; ++i) {
@@ -638,6 +644,10 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
             mbar_init(bar_mma + i, 1);
         }
         mbar_init(bar_read, kWork);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(bar_f + i, 32);
+            mbar_init(bar_fdone + i, kWork);
+        }
         mbar_init_fence();
         tma_prefetch_desc(&p.tm_u);
         tma_prefetch_desc(&p.tm_y);
@@ -673,6 +683,45 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
         // one issued waits for everything in flight
         for (int i = 0; i < 3; ++i)
             if (n_ld[i]) mbar_wait(bar_ld + i, (n_ld[i] - 1) & 1, ctl);
+    } else if (decay) {
+        // ------------------------------------------------------ decay warp
+        // per chunk: f_t (U~ = f U) for the 128 tokens and the chunk's total
+        // log2-decay, into a four-slot ring; lane L scans tokens 4L .. 4L+3
+        auto load_a = [&](int it, float (&x)[4]) {
+            const int c = chunk_at(it);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int t = c * 128 + lane * 4 + e;
+                x[e] = (it < nchunks && t < p.T) ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f;
+            }
+        };
+        float xa[4];
+        load_a(0, xa);
+        for (int it = 0; it < nchunks; ++it) {
+            float c4[4];
+            c4[0] = xa[0] * kLog2e;
+#pragma unroll
+            for (int e = 1; e < 4; ++e) c4[e] = c4[e - 1] + xa[e] * kLog2e;
+            load_a(it + 1, xa);
+            float incl = c4[3];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const float up = __shfl_up_sync(0xffffffffu, incl, 1);
+            const float pre = lane ? up : 0.f;
+            const float g2 = __shfl_sync(0xffffffffu, incl, 31);
+            float f[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) f[e] = REVERSE ? p.scale * exp2f(pre + c4[e]) : exp2f(g2 - (pre + c4[e]));
+            const int slot = it & 3;
+            if (it >= 4 && !mbar_wait(bar_fdone + slot, ((it - 4) >> 2) & 1, ctl)) break;
+            *reinterpret_cast<float4*>(fring + slot * 128 + lane * 4) = make_float4(f[0], f[1], f[2], f[3]);
+            if (lane == 0) g2s[slot] = g2;
+            __syncwarp();
+            mbar_arrive(bar_f + slot);
+        }
     } else if (issuer) {
         // ---------------------------------------------------------- issuer
         int n_mma[2] = {0, 0}, n_free[3] = {0, 0, 0};
@@ -714,34 +763,6 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
             S[e + 3] = v.w;
         }
         const uint32_t tq = tmem_addr(tmem, quad * 32, 0);
-        // this lane holds tokens 4*lane .. +3 of the chunk's decay scan
-        auto load_a = [&](int it, float (&x)[4]) {
-            const int c = chunk_at(it);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int t = c * 128 + lane * 4 + e;
-                x[e] = (it < nchunks && t < p.T) ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f;
-            }
-        };
-        // the chunk's per-token factors f (for U~ = f U) and its total log2-decay
-        auto scan = [&](const float (&x)[4], float (&f)[4]) {
-            float c4[4];
-            c4[0] = x[0] * kLog2e;
-#pragma unroll
-            for (int e = 1; e < 4; ++e) c4[e] = c4[e - 1] + x[e] * kLog2e;
-            float incl = c4[3];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            const float up = __shfl_up_sync(0xffffffffu, incl, 1);
-            const float pre = lane ? up : 0.f;
-            const float g2 = __shfl_sync(0xffffffffu, incl, 31);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) f[e] = REVERSE ? p.scale * exp2f(pre + c4[e]) : exp2f(g2 - (pre + c4[e]));
-            return g2;
-        };
         // U~^T (row = dk index, columns = tokens 32 qt .. +31) -> TMEM buffer.
         // Element (t, d) of the [3][128][32] SW64 tile sits at block d/32, byte
         // 64 t + 16 ((d%32)/8 ^ (t/2)%4) + 2 (d%8); for t = 32 qt + 2 q the
@@ -749,24 +770,31 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
         const uint32_t cb = lane >> 3;
         const uint32_t sw[4] = {(cb ^ 0u) * 16 + (lane & 7) * 2, (cb ^ 1u) * 16 + (lane & 7) * 2,
                                 (cb ^ 2u) * 16 + (lane & 7) * 2, (cb ^ 3u) * 16 + (lane & 7) * 2};
-        auto split = [&](int it, const float (&f)[4]) {
+        auto split = [&](int it) {
             const uint8_t* u = sm + (it % 3) * L::STAGE + quad * 8192 + qt * 32 * 64;
+            const float* fs = fring + (it & 3) * 128 + qt * 32;
             const uint32_t dst = tq + L::TM_U + (it & 1) * 128 + qt * 16;
 #pragma unroll
             for (int g = 0; g < 2; ++g) {
+                float f[16];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 v = *reinterpret_cast<const float4*>(fs + g * 16 + 4 * i);
+                    f[4 * i] = v.x;
+                    f[4 * i + 1] = v.y;
+                    f[4 * i + 2] = v.z;
+                    f[4 * i + 3] = v.w;
+                }
                 uint32_t hi[8], lo[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const int tl = g * 16 + 2 * q;           // token within this quarter
-                    const int t = qt * 32 + tl;
-                    const float f0 = __shfl_sync(0xffffffffu, f[tl & 3], t >> 2);
-                    const float f1 = __shfl_sync(0xffffffffu, f[(tl + 1) & 3], (t + 1) >> 2);
                     const uint32_t o = sw[q & 3];
                     const float k0 = __uint_as_float(
                         static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(u + tl * 64 + o)) << 16);
                     const float k1 = __uint_as_float(
                         static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(u + tl * 64 + 64 + o)) << 16);
-                    const float v0 = k0 * f0, v1 = k1 * f1;
+                    const float v0 = k0 * f[2 * q], v1 = k1 * f[2 * q + 1];
                     const uint32_t hv = pack_bf16(v0, v1);
                     hi[q] = hv;
                     lo[q] = pack_bf16(v0 - bf16_lo(hv), v1 - bf16_hi(hv));
@@ -776,69 +804,46 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
             }
             tmem_st_wait();
         };
-        // bf16 copy of S (96 B of this thread's row) -> h_out, eight rows of the
-        // warp at a time through a shared-memory transpose so that each store
-        // instruction writes whole 96-byte row segments
-        uint8_t* xp = sm + L::XPOSE + ((warp >> 2) * 3 + quad) * 768;
+        // bf16 copy of S (96 B of this thread's row) -> h_out as three 32-byte
+        // stores: whole sectors, the row segment 32-byte aligned
         auto store_h = [&](int it) {
-            uint8_t* hrow0 = static_cast<uint8_t*>(p.h_out) +
-                             ((static_cast<int64_t>(unit) * p.NC + chunk_at(it)) * kDk + quad * 32) * (kDv * 2) + qt * 96;
+            uint8_t* dst = static_cast<uint8_t*>(p.h_out) +
+                           ((static_cast<int64_t>(unit) * p.NC + chunk_at(it)) * kDk + row) * (kDv * 2) + qt * 96;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                if ((lane >> 3) == k) {
-                    uint4* dst = reinterpret_cast<uint4*>(xp + (lane & 7) * 96);
+            for (int q = 0; q < 3; ++q) {
+                uint32_t w[8];
 #pragma unroll
-                    for (int q = 0; q < 6; ++q)
-                        dst[q] = make_uint4(pack_bf16(S[8 * q], S[8 * q + 1]), pack_bf16(S[8 * q + 2], S[8 * q + 3]),
-                                            pack_bf16(S[8 * q + 4], S[8 * q + 5]),
-                                            pack_bf16(S[8 * q + 6], S[8 * q + 7]));
-                }
-                __syncwarp();
-#pragma unroll
-                for (int j0 = 0; j0 < 48; j0 += 32) {
-                    const int j = j0 + lane;       // piece j: row j / 6, 16-byte part j % 6
-                    if (j < 48)
-                        *reinterpret_cast<uint4*>(hrow0 + (8 * k + j / 6) * (kDv * 2) + (j % 6) * 16) =
-                            *reinterpret_cast<const uint4*>(xp + j * 16);
-                }
-                __syncwarp();
+                for (int e = 0; e < 8; ++e) w[e] = pack_bf16(S[16 * q + 2 * e], S[16 * q + 2 * e + 1]);
+                st_global_v8(dst + 32 * q, w);
             }
         };
 
         bool ok = true;
         float gsum2 = 0.f;
-        float xa[4], f[4];
         float g2 = 0.f;
+        // split of chunk it: its decay factors and tiles are ready and the
+        // TMEM buffer's previous MMAs (chunk it-2) are done
+        auto do_split = [&](int it) {
+            if (!mbar_wait(bar_f + (it & 3), (it >> 2) & 1, ctl) || !mbar_wait(bar_ld + it % 3, (it / 3) & 1, ctl) ||
+                (it >= 2 && !mbar_wait(bar_mma + (it & 1), ((it - 2) >> 1) & 1, ctl)))
+                return false;
+            tc_fence_after();
+            split(it);
+            g2 = g2s[it & 3];
+            tc_fence_before();
+            mbar_arrive(bar_split + (it & 1));
+            mbar_arrive(bar_fdone + (it & 3));
+            return true;
+        };
         if (nchunks > 0) {
-            load_a(0, xa);
-            g2 = scan(xa, f);
-            load_a(1, xa);
             if (p.store_h) store_h(0);
-            if (mbar_wait(bar_ld, 0, ctl)) {
-                tc_fence_after();
-                split(0, f);
-                tc_fence_before();
-                mbar_arrive(bar_split);
-            } else {
-                ok = false;
-            }
+            ok = do_split(0);
         }
         for (int it = 0; ok && it < nchunks; ++it) {
             const float g2_cur = g2;
-            if (it + 1 < nchunks) {
-                float fn[4];
-                g2 = scan(xa, fn);
-                load_a(it + 2, xa);
-                const int nx = it + 1;
-                if (!mbar_wait(bar_ld + nx % 3, (nx / 3) & 1, ctl) ||
-                    (it >= 1 && !mbar_wait(bar_mma + ((it - 1) & 1), ((it - 1) >> 1) & 1, ctl))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                split(nx, fn);
-                tc_fence_before();
-                mbar_arrive(bar_split + (nx & 1));
+            if (it + 1 < nchunks && !do_split(it + 1)) {
+                ok = false;
+                break;
             }
             if (!mbar_wait(bar_mma + (it & 1), (it >> 1) & 1, ctl)) {
                 ok = false;

@@ -102,7 +102,7 @@ gla_status launch_state_kernel(bool with_o, bool reverse, const StateParams& p, 
 {
     if (with_o && !reverse)
         return launch_chunk_kernel(gla_fwd_fused_kernel, chunk::FusedSmem::BYTES,
-                                   "chunk_fwd_fused_kernel", p, grid, st);
+                                   "chunk_fwd_fused_kernel", p, grid, st, chunk::kFusedThreads);
     if (!with_o && !reverse)
         return launch_chunk_kernel(gla_state_pass_kernel<false>, chunk::PassSmem::BYTES,
                                    "chunk_state_fwd_kernel", p, grid, st, chunk::kPassThreads);
@@ -136,8 +136,7 @@ gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float
     if ((s = make_token_map(&p.tm_q, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64, 16)) != GLA_OK) return s;
     if ((s = make_token_map(&p.tm_u, pr.k, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&p.tm_y, pr.v, kDv, pr.H, pr.T, pr.B, pr.ld_v, 64, 128)) != GLA_OK) return s;
-    if ((s = make_token_map(&p.tm_o, o, kDv, pr.H, pr.T, pr.B, static_cast<int64_t>(pr.H) * kDv, 64,
-                            128)) != GLA_OK)
+    if ((s = make_token_map(&p.tm_o, o, kDv, pr.H, pr.T, pr.B, static_cast<int64_t>(pr.H) * kDv, 64, 128)) != GLA_OK)
         return s;
     p.a = pr.a;
     p.B = pr.B;

@@ -61,8 +61,8 @@ namespace gla {
 struct StateParams {
     CUtensorMap tm_q;       // q tile loads, 16-row boxes (fused forward)
     CUtensorMap tm_u;       // scaled operand: k (forward) or q (reverse)
-    CUtensorMap tm_y;       // v (forward) or dO (reverse)
-    CUtensorMap tm_o;       // o tile stores (fused forward)
+    CUtensorMap tm_y;
+    CUtensorMap tm_o;       // o tile stores (fused forward)       // v (forward) or dO (reverse)
     const float* a;         // [B, T, H] log-decay
     const float* s_init;    // initial state per (unit, seg) or null (zeros)
     float* s_out;           // state after the segment, or null
@@ -83,6 +83,7 @@ namespace chunk {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kWorkers = 256;
 constexpr int kThreads = kWorkers + 32;
+constexpr int kFusedThreads = kThreads + 32;   // + a producer warp
 // state pass: 16 warps; w % 4 < 3 for w < 15 are the 12 workers (TMEM lanes
 // 0..95 = the dk rows, four column quarters), warp 15 issues
 constexpr int kPassThreads = 512;
@@ -92,17 +93,18 @@ constexpr float kFactorRange = 100.0f;         // max log2 span for the factoris
 
 constexpr uint32_t kIdScores = idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint32_t kIdOut = idesc_bf16_f32(128, 192, 0, 1);
+constexpr uint32_t kIdOutTs = idesc_bf16_f32(128, 192, 0, 1);   // A from tensor memory
 constexpr uint32_t kIdState = idesc_bf16_f32(128, 192, 1, 1);
 constexpr uint32_t kIdStateTs = idesc_bf16_f32(128, 192, 0, 1);   // A from tensor memory
 
 // Shared-memory maps (bytes from a 1024-aligned base).
 struct FusedSmem {
     static constexpr uint32_t Q = 0;          // q tile, permuted rows
-    static constexpr uint32_t U = 24576;      // k tile, then K~ (its 4th M block is Y: finite)
-    static constexpr uint32_t Y = 49152;      // v tile
-    static constexpr uint32_t X = 98304;      // state copy hi, then P_hi
-    static constexpr uint32_t XL = 135168;    // state copy lo
-    static constexpr uint32_t O = 172032;     // P_lo, then output staging
+    static constexpr uint32_t U = 24576;      // k tile, then K~ (its 4th M block is X: finite)
+    static constexpr uint32_t X = 49152;      // state copy hi [3][96][64] SW128; with XL, o staging
+    static constexpr uint32_t XL = 86016;     // state copy lo
+    static constexpr uint32_t Y0 = 122880;    // v tiles, double buffered
+    static constexpr uint32_t Y1 = 172032;
     static constexpr uint32_t MISC = 221184;
     static constexpr uint32_t BYTES = MISC + 2048 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -130,6 +132,17 @@ __device__ __forceinline__ int row_token(int r) { return perm16(r >> 4) * 16 + (
 __device__ __forceinline__ void named_sync(int id, int n)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ void bar_sync(int id, int n) { named_sync(id, n); }
+
+// Named-barrier OR reduction over n threads (a __syncthreads_or on a subset).
+__device__ __forceinline__ bool bar_or(int id, int n, bool v)
+{
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %3, 0;\n\tbarrier.cta.red.or.pred q, %1, %2, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"(id), "r"(n), "r"(static_cast<uint32_t>(v)) : "memory");
+    return r != 0;
 }
 
 __device__ __forceinline__ uint4 scale8(uint4 v, float f)
@@ -293,7 +306,7 @@ __device__ __forceinline__ void state_copy_and_decay(uint32_t taddr, int row, in
 // =====================================================================
 // Fused forward.
 // =====================================================================
-__global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const __grid_constant__ StateParams p)
+__global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(const __grid_constant__ StateParams p)
 {
     using namespace chunk;
     using L = FusedSmem;
@@ -303,9 +316,11 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const
     const uint32_t sb = smem_u32(sm);
     uint64_t* bar_q = reinterpret_cast<uint64_t*>(sm + L::MISC);
     uint64_t* bar_u = bar_q + 1;
-    uint64_t* bar_y = bar_q + 2;
-    uint64_t* bar_m = bar_q + 3;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_q + 4);
+    uint64_t* bar_y = bar_q + 2;                                 // [2]
+    uint64_t* bar_m = bar_q + 4;                                 // scores; then all of the chunk's MMAs
+    uint64_t* bar_d = bar_q + 5;                                 // O = Q S_prev and the state update
+    uint64_t* bar_f = bar_q + 6;                                 // [2] all of a chunk's MMAs (producer)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_q + 8);
     float* b2s = reinterpret_cast<float*>(sm + L::MISC + 64);   // [128] by token
     float* cfac = b2s + 128;                                     // [128] 2^{-b_j}
     float* wsum = cfac + 128;                                    // [4]
@@ -325,6 +340,7 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const
     const bool worker = warp < 8;
     const bool srow = worker && quad < 3;
     const bool issuer = warp == 8 && lane == 0;
+    const bool producer = warp == 9 && lane == 0;   // TMA loads; outside the loop's named barrier
     // largest token among this lane quarter's rows (columns beyond it are masked)
     const int quad_max_tok = max(perm16(2 * quad), perm16(2 * quad + 1)) * 16 + 15;
 
@@ -332,7 +348,11 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const
         mbar_init(bar_q, 1);
         mbar_init(bar_u, 1);
         mbar_init(bar_y, 1);
+        mbar_init(bar_y + 1, 1);
         mbar_init(bar_m, 1);
+        mbar_init(bar_d, 1);
+        mbar_init(bar_f, 1);
+        mbar_init(bar_f + 1, 1);
         mbar_init_fence();
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_u);
@@ -353,32 +373,13 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const
         const int t = c * 128 + tid;
         return t < p.T ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f;
     };
-    bool pend_q = false, pend_u = false, pend_y = false, pend_m = false;
-    uint32_t ph_q = 0, ph_u = 0, ph_y = 0, mph = 0;
-    auto issue_qu = [&](int c) {
-        const int t0 = c * 128;
-        mbar_arrive_expect_tx(bar_q, kTileQK);
-        for (int i = 0; i < 3; ++i)
-            for (int r16 = 0; r16 < 8; ++r16)
-                tma_load_4d(sm + L::Q + i * 8192 + r16 * 1024, &p.tm_q, bar_q, i * 32, h,
-                            t0 + perm16(r16) * 16, b);
-        pend_q = true;
-        mbar_arrive_expect_tx(bar_u, kTileQK);
-        for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::U + i * 8192, &p.tm_u, bar_u, i * 32, h, t0, b);
-        pend_u = true;
-    };
-    auto issue_y = [&](int c) {
-        mbar_arrive_expect_tx(bar_y, kTileV);
-        for (int i = 0; i < 3; ++i)
-            tma_load_4d(sm + L::Y + i * 16384, &p.tm_y, bar_y, i * 64, h, c * 128, b);
-        pend_y = true;
-    };
+    // per barrier at most one phase is ever outstanding
+    uint32_t ph_q = 0, ph_u = 0, ph_y[2] = {0u, 0u}, mph = 0;
+    bool pend_m = false;
+    int n_d = 0, n_f[2] = {0, 0};   // commits issued to bar_d and bar_f[]
 
-    if (issuer && nchunks > 0) {
-        issue_qu(c_begin);
-        issue_y(c_begin);
-    }
     float a_cur = (tid < 128 && nchunks > 0) ? load_a(c_begin) : 0.f;
+    float a_nx = (tid < 128 && nchunks > 1) ? load_a(c_begin + 1) : 0.f;
     if (srow) {
         const float* src = p.s_init ? p.s_init + unit * p.init_unit_stride + seg * p.init_seg_stride +
                                           row * kDv + half * 96
@@ -389,9 +390,59 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const
     __syncthreads();
     tc_fence_after();
 
+    if (producer) {
+        // ----------------------------------------------------------- producer
+        // q, k of chunk it+1 once (D) of chunk it is done; v of chunk it+2
+        // into the buffer chunk it used once all of chunk it's MMAs are done
+        auto issue_qu = [&](int c) {
+            const int t0 = c * 128;
+            mbar_arrive_expect_tx(bar_q, kTileQK);
+            for (int i = 0; i < 3; ++i)
+                for (int r16 = 0; r16 < 8; ++r16)
+                    tma_load_4d(sm + L::Q + i * 8192 + r16 * 1024, &p.tm_q, bar_q, i * 32, h,
+                                t0 + perm16(r16) * 16, b);
+            mbar_arrive_expect_tx(bar_u, kTileQK);
+            for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::U + i * 8192, &p.tm_u, bar_u, i * 32, h, t0, b);
+        };
+        auto issue_y = [&](int c, int s) {
+            uint8_t* y = sm + (s ? L::Y1 : L::Y0);
+            mbar_arrive_expect_tx(bar_y + s, kTileV);
+            for (int i = 0; i < 3; ++i) tma_load_4d(y + i * 16384, &p.tm_y, bar_y + s, i * 64, h, c * 128, b);
+        };
+        int n_qu = 0, n_y[2] = {0, 0};
+        if (nchunks > 0) {
+            issue_qu(c_begin);
+            ++n_qu;
+            issue_y(c_begin, 0);
+            ++n_y[0];
+            if (nchunks > 1) {
+                issue_y(c_begin + 1, 1);
+                ++n_y[1];
+            }
+        }
+        for (int it = 0; it + 1 < nchunks; ++it) {
+            if (!mbar_wait(bar_d, it & 1, ctl)) break;
+            issue_qu(c_begin + it + 1);
+            ++n_qu;
+            if (it + 2 < nchunks) {
+                if (!mbar_wait(bar_f + (it & 1), (it >> 1) & 1, ctl)) break;
+                issue_y(c_begin + it + 2, it & 1);
+                ++n_y[it & 1];
+            }
+        }
+        if (n_qu) {
+            mbar_wait(bar_q, (n_qu - 1) & 1, ctl);
+            mbar_wait(bar_u, (n_qu - 1) & 1, ctl);
+        }
+        for (int i = 0; i < 2; ++i)
+            if (n_y[i]) mbar_wait(bar_y + i, (n_y[i] - 1) & 1, ctl);
+    }
+
     bool failed = false, aborted = false;
-    for (int it = 0; it < nchunks; ++it) {
+    for (int it = 0; warp < 9 && it < nchunks; ++it) {
         const int c = c_begin + it;
+        const int ys = it & 1;
+        const uint32_t ya = ys ? L::Y1 : L::Y0;
 
         // (A) cumulative decay (warps 0-3) and column factors; scores MMA
         if (tid < 128) {
@@ -401,23 +452,24 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const
         }
         if (issuer) {
             if (mbar_wait(bar_q, ph_q, ctl) && mbar_wait(bar_u, ph_u, ctl)) {
-                pend_q = pend_u = false;
                 ph_q ^= 1;
                 ph_u ^= 1;
                 tc_fence_after();
+                const uint64_t dq = smem_desc(sb + L::Q, 16, 512, kLayoutSW64);
+                const uint64_t du = smem_desc(sb + L::U, 16, 512, kLayoutSW64);
 #pragma unroll
                 for (int ks = 0; ks < 6; ++ks) {
                     const uint32_t off = (ks >> 1) * 8192 + (ks & 1) * 32;
-                    umma_bf16(tmem + L::TM_SC, smem_desc(sb + L::Q + off, 16, 512, kLayoutSW64),
-                              smem_desc(sb + L::U + off, 16, 512, kLayoutSW64), kIdScores, ks > 0);
+                    umma_bf16(tmem + L::TM_SC, desc_add(dq, off), desc_add(du, off), kIdScores, ks > 0);
                 }
                 umma_commit(bar_m);
                 pend_m = true;
             } else {
                 failed = true;
             }
+            tma_store_wait_read();   // the previous chunk's o staging (X, XL) is free
         }
-        if (__syncthreads_or(failed)) { aborted = true; break; }
+        if (bar_or(2, 288, failed)) { aborted = true; break; }
         const float g2 = b2s[127];
         const bool fast = -g2 <= kFactorRange;   // uniform: the factorised path is safe
 
@@ -429,7 +481,6 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const
         // (C) K~ = e^{gamma - b} K in place; on the exact path also
         // Q~ = scale e^{b} Q (rows in permuted token order)
         if (!mbar_wait(bar_m, mph, ctl)) failed = true;           // scores done: Q, K free
-        if (issuer) tma_store_wait_read();                          // o staging free (P_lo)
         if (!failed && worker) {
             for (int idx = tid; idx < 384; idx += kWorkers) {
                 const int r = idx & 127, blk = idx >> 7;
@@ -439,54 +490,55 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const
         }
         fence_async_smem();
         tc_fence_before();
-        if (__syncthreads_or(failed)) { aborted = true; break; }
+        if (bar_or(2, 288, failed)) { aborted = true; break; }
         tc_fence_after();
         if (issuer) pend_m = false;
         mph ^= 1;
 
         // (D) O = Q S_prev (hi, lo), S += K~^T V
         if (issuer) {
-            if (mbar_wait(bar_y, ph_y, ctl)) {
-                pend_y = false;
-                ph_y ^= 1;
+            if (mbar_wait(bar_y + ys, ph_y[ys], ctl)) {
+                ph_y[ys] ^= 1;
+                const uint64_t dq = smem_desc(sb + L::Q, 16, 512, kLayoutSW64);
+                const uint64_t dx = smem_desc(sb + L::X, 12288, 1024, kLayoutSW128);
+                const uint64_t dxl = smem_desc(sb + L::XL, 12288, 1024, kLayoutSW128);
+                const uint64_t dua = smem_desc(sb + L::U, 8192, 512, kLayoutSW64);
+                const uint64_t dy = smem_desc(sb + ya, 16384, 1024, kLayoutSW128);
 #pragma unroll
-                for (int part = 0; part < 2; ++part) {
-                    const uint32_t sbase = part ? L::XL : L::X;
+                for (int part = 0; part < 2; ++part)
 #pragma unroll
-                    for (int ks = 0; ks < 6; ++ks) {
-                        const uint32_t aoff = (ks >> 1) * 8192 + (ks & 1) * 32;
-                        umma_bf16(tmem + L::TM_O, smem_desc(sb + L::Q + aoff, 16, 512, kLayoutSW64),
-                                  smem_desc(sb + sbase + ks * 2048, 12288, 1024, kLayoutSW128), kIdOut,
-                                  (part | ks) > 0);
-                    }
-                }
+                    for (int ks = 0; ks < 6; ++ks)
+                        umma_bf16(tmem + L::TM_O, desc_add(dq, (ks >> 1) * 8192 + (ks & 1) * 32),
+                                  desc_add(part ? dxl : dx, ks * 2048), kIdOut, (part | ks) > 0);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    umma_bf16(tmem + L::TM_S, smem_desc(sb + L::U + ks * 1024, 8192, 512, kLayoutSW64),
-                              smem_desc(sb + L::Y + ks * 2048, 16384, 1024, kLayoutSW128), kIdState, 1);
-                umma_commit(bar_m);
-                pend_m = true;
+                    umma_bf16(tmem + L::TM_S, desc_add(dua, ks * 1024), desc_add(dy, ks * 2048), kIdState, 1);
+                umma_commit(bar_d);
+                ++n_d;
             } else {
                 failed = true;
             }
         }
 
-        // (E) P = P_hi + P_lo from the scores; P_lo to the output staging
-        // buffer at once, P_hi once O = Q S_prev has released the state copy
-        uint32_t pk[32];
+        // (E) scores -> P (hi, lo) in place in tensor memory: lane = row i,
+        // 32-token block kb holds hi in columns 32 kb .. +15 and lo in +16 .. +31.
+        // The epilogue's row factor is read here, before the next chunk's decays
+        // overwrite b2s.
+        float rf = 1.0f;
         if (worker) {
             const float b2r = b2s[tok];
-            uint8_t* plo = sm + L::O + half * 16384;
+            if (fast) rf = p.scale * exp2f(b2r);
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 const int j0 = half * 64 + q2 * 32;
-                uint32_t lo[16];
+                const uint32_t col = L::TM_SC + j0;
+                uint32_t hi[16], lo[16];
                 if (j0 > quad_max_tok) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[q2 * 16 + e] = lo[e] = 0u;
+                    for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
                 } else {
                     uint32_t r[32];
-                    tmem_ld32(tq + L::TM_SC + j0, r);
+                    tmem_ld32(tq + col, r);
                     tmem_ld_wait();
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
@@ -499,62 +551,46 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const
                             v0 = (j <= tok) ? p.scale * __uint_as_float(r[e]) * exp2f(b2r - b2s[j]) : 0.f;
                             v1 = (j + 1 <= tok) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2r - b2s[j + 1]) : 0.f;
                         }
-                        const uint32_t hi = pack_bf16(v0, v1);
-                        pk[q2 * 16 + e / 2] = hi;
-                        lo[e / 2] = pack_bf16(v0 - bf16_lo(hi), v1 - bf16_hi(hi));
+                        const uint32_t hv = pack_bf16(v0, v1);
+                        hi[e / 2] = hv;
+                        lo[e / 2] = pack_bf16(v0 - bf16_lo(hv), v1 - bf16_hi(hv));
                     }
                 }
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4)
-                    *reinterpret_cast<uint4*>(plo + swz_off(row, q2 * 4 + c4, 128)) =
-                        make_uint4(lo[c4 * 4], lo[c4 * 4 + 1], lo[c4 * 4 + 2], lo[c4 * 4 + 3]);
+                tmem_st16(tq + col, hi);
+                tmem_st16(tq + col + 16, lo);
             }
+            tmem_st_wait();
         }
-        if (!mbar_wait(bar_m, mph, ctl)) failed = true;               // O = Q S_prev, S update done
         tc_fence_before();
-        if (__syncthreads_or(failed)) { aborted = true; break; }
-        if (issuer) pend_m = false;
-        mph ^= 1;
-        if (worker) {
-            uint8_t* pb = sm + L::X + half * 16384;
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4*>(pb + swz_off(row, ch, 128)) =
-                    make_uint4(pk[ch * 4], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
+        if (bar_or(2, 288, failed)) { aborted = true; break; }
 
-        // (F) O += P V; prefetch the next q and k tiles and decays
+        // (F) O += P V with P from tensor memory; once (D) is done, q and k
+        // of the next chunk may load
         float a_next = 0.f;
         if (issuer) {
             tc_fence_after();
+            const uint64_t dy = smem_desc(sb + ya, 16384, 1024, kLayoutSW128);
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const uint32_t pbase = part ? L::O : L::X;
+            for (int part = 0; part < 2; ++part)
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t aoff = (ks >> 2) * 16384 + (ks & 3) * 32;
-                    umma_bf16(tmem + L::TM_O, smem_desc(sb + pbase + aoff, 16, 1024, kLayoutSW128),
-                              smem_desc(sb + L::Y + ks * 2048, 16384, 1024, kLayoutSW128), kIdOut, 1);
-                }
-            }
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_bf16_ts(tmem + L::TM_O, tmem + L::TM_SC + 32 * (ks >> 1) + 8 * (ks & 1) + 16 * part,
+                                 desc_add(dy, ks * 2048), kIdOutTs, 1);
             umma_commit(bar_m);
+            umma_commit(bar_f + ys);
             pend_m = true;
-            if (it + 1 < nchunks) issue_qu(c + 1);
+            ++n_f[ys];
         }
-        if (tid < 128 && it + 1 < nchunks) a_next = load_a(c + 1);
+        if (tid < 128 && it + 2 < nchunks) a_next = load_a(c + 2);
 
-        // (G) epilogue: o = r_i O_i -> bf16 staging (token order) -> TMA store
+        // (G) epilogue: o = r_i O_i -> bf16 staging in X, XL (token order,
+        // [3][128][64] SW128; the state copies are dead once (D) is done) -> TMA store
         if (!mbar_wait(bar_m, mph, ctl)) failed = true;
-        if (__syncthreads_or(failed)) { aborted = true; break; }
+        if (bar_or(2, 288, failed)) { aborted = true; break; }
         if (issuer) pend_m = false;
         mph ^= 1;
         tc_fence_after();
-        if (issuer && it + 1 < nchunks) issue_y(c + 1);
         if (worker) {
-            const float rf = fast ? p.scale * exp2f(b2s[tok]) : 1.0f;
 #pragma unroll
             for (int j = 0; j < 3; ++j) {
                 uint32_t r[32];
@@ -565,19 +601,20 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     const int n = half * 96 + j * 32 + q4 * 8;
-                    *reinterpret_cast<uint4*>(sm + L::O + (n >> 6) * 16384 +
-                                              swz_off(tok, (n & 63) >> 3, 128)) = pack8(r + q4 * 8);
+                    *reinterpret_cast<uint4*>(sm + L::X + (n >> 6) * 16384 + swz_off(tok, (n & 63) >> 3, 128)) =
+                        pack8(r + q4 * 8);
                 }
             }
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        bar_sync(2, 288);
         if (issuer) {
-            for (int i = 0; i < 3; ++i) tma_store_4d(&p.tm_o, sm + L::O + i * 16384, i * 64, h, c * 128, b);
+            for (int i = 0; i < 3; ++i) tma_store_4d(&p.tm_o, sm + L::X + i * 16384, i * 64, h, c * 128, b);
             tma_store_commit();
         }
-        a_cur = a_next;
+        a_cur = a_nx;
+        a_nx = a_next;
     }
 
     if (!aborted) {
@@ -585,11 +622,15 @@ __global__ void __launch_bounds__(chunk::kThreads, 1) gla_fwd_fused_kernel(const
         if (write_state && srow)
             tmem_to_state(tq + L::TM_S + half * 96,
                           p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + half * 96);
-    } else if (issuer) {
-        if (pend_q) mbar_wait(bar_q, ph_q, ctl);
-        if (pend_u) mbar_wait(bar_u, ph_u, ctl);
-        if (pend_y) mbar_wait(bar_y, ph_y, ctl);
-        if (pend_m) mbar_wait(bar_m, mph, ctl);
+    } else if (issuer && pend_m) {
+        mbar_wait(bar_m, mph, ctl);
+    }
+    if (issuer) {
+        // every commit's arrival has landed before the barriers go away: at
+        // most one phase of each is outstanding, so wait for the last one
+        if (n_d) mbar_wait(bar_d, (n_d - 1) & 1, ctl);
+        for (int i = 0; i < 2; ++i)
+            if (n_f[i]) mbar_wait(bar_f + i, (n_f[i] - 1) & 1, ctl);
     }
     if (issuer) tma_store_wait_all();
     tc_fence_before();

@@ -13,10 +13,20 @@ Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
 cuda synchronize, measured with CUDA events on the launching stream, max
 over ranks.  Inputs (about 0.6 GB per rank for the training step, 36 GB of
 decode state) are larger than the 126 MB L2, so no flush is needed.
-Roofline: libgla's own per-launch event tracing times every kernel inside
-the timed region; the dominant kernel's algorithmic bytes (or flops) per
-launch divided by its mean launch time, against MEASURED_PEAKS.json.
+Roofline: right after the timed region the same K steps run again with
+libgla's per-launch event tracing (events between launches cost a few
+percent, so they stay out of the headline region); the dominant kernel's
+algorithmic bytes (or flops) per launch divided by its mean launch time,
+against MEASURED_PEAKS.json.  Its
+"traffic" (DRAM bytes per launch) comes from the ncu capture summarised in
+profiles/dram_traffic.md, and only while the digest of the kernel's source
+files still matches the one recorded there; otherwise it is null.
+
+--skip-decode / --skip-e2e time only the training step: the command the
+profiles' ncu captures run (a few GB on the device instead of the 36 GB of
+decode state).
 """
+import hashlib
 import argparse
 import json
 import os
@@ -53,6 +63,8 @@ CHUNK_BYTES = {
     "chunk_state_rev_kernel": QK + VO + A + HS,
     # dq/dk: read q, k, v, dO, h, D, a; write dq, dk, q.dq and k.dk per token
     "bwd_dqdk_kernel": 2 * QK + 2 * VO + 2 * HS + A + 2 * QK + 2 * A,
+    # da: read q.dq, k.dk; write da
+    "da_finish_kernel": 3 * A,
     # dv: read q, k, dO, D, a; write dv
     "bwd_dv_kernel": 2 * QK + VO + HS + A + VO,
 }
@@ -60,6 +72,47 @@ CHUNK_FLOPS = {
     # 2*(128*128*96 + 128*192*96 + 128*192*128 + 96*192*128), dense tiles
     "chunk_fwd_fused_kernel": 2 * (128 * 128 * 96 + 128 * 192 * 96 + 128 * 192 * 128 + 96 * 192 * 128),
 }
+
+
+# Source files each kernel is built from (the digest that ties a recorded
+# ncu traffic figure to the code it was measured on).
+CSRC = os.path.join(ROOT, "linear_attention_simple_b200", "csrc")
+KERNEL_SOURCES = {
+    "chunk_fwd_fused_kernel": ("chunk_fwd.cu", "chunk_state.cuh", "gla_device.cuh"),
+    "chunk_state_fwd_kernel": ("chunk_fwd.cu", "chunk_state.cuh", "gla_device.cuh"),
+    "chunk_state_rev_kernel": ("chunk_fwd.cu", "chunk_state.cuh", "gla_device.cuh"),
+    "bwd_dqdk_kernel": ("chunk_bwd.cu", "chunk_state.cuh", "gla_device.cuh"),
+    "bwd_dv_kernel": ("chunk_bwd.cu", "chunk_state.cuh", "gla_device.cuh"),
+    "da_finish_kernel": ("chunk_bwd.cu",),
+}
+
+
+def kernel_digest(name):
+    files = KERNEL_SOURCES.get(name)
+    if not files:
+        return None
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(name):
+    """DRAM bytes per launch of `name` from profiles/dram_traffic.md, if the
+    row's source digest matches the current sources; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    dig = kernel_digest(name)
+    if dig is None or not os.path.exists(path):
+        return None
+    for line in open(path):
+        cells = [c.strip().strip("`") for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 5 and cells[0] == name and cells[1] == dig:
+            try:
+                return int(cells[4].replace(",", ""))
+            except ValueError:
+                return None
+    return None
 
 
 def load_peaks():
@@ -185,7 +238,8 @@ def kernel_roofline(summary, peaks, peak_kind, units_per_launch, B, H):
         roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                 "unit": "GB/s", "frac": round(achieved / peak, 4),
                 "bytes_per_launch": bytes_per_launch, "mean_launch_us": round(mean_s * 1e6, 2),
-                "traffic": None, "peak_source": "%s copy bandwidth" % peak_kind}
+                "traffic": recorded_traffic(name), "source_digest": kernel_digest(name),
+                "peak_source": "%s copy bandwidth" % peak_kind}
     else:
         roof = {"kernel": name, "bound": None, "achieved": None, "peak": None, "unit": None,
                 "frac": None, "traffic": None, "mean_launch_us": round(mean_s * 1e6, 2)}
@@ -263,7 +317,6 @@ def run_ours(args, ws, rank, local):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)                       # let the sampler come up
-    gla.gla_trace_enable(True)
     launches0 = gla.gla_launch_count()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(st)
@@ -272,17 +325,41 @@ def run_ours(args, ws, rank, local):
     ev1.record(st)
     ev1.synchronize()
     launches = gla.gla_launch_count() - launches0
-    summary = gla.gla_trace_summary()
-    gla.gla_trace_enable(False)
     torch.cuda.synchronize()
     barrier(ws)
     elapsed = max_over_ranks(ev0.elapsed_time(ev1) / 1e3, ws)
     ms_step = elapsed / args.steps * 1e3
     value = ws * w.B * w.T * args.steps / elapsed
+    # per-kernel times: the same steps again with libgla's per-launch events
+    # (kept out of the timed region above: the events themselves cost time)
+    gla.gla_trace_enable(True)
+    for _ in range(args.steps):
+        train_step(d)
+    summary = gla.gla_trace_summary()
+    gla.gla_trace_enable(False)
+    torch.cuda.synchronize()
     roof, shares = kernel_roofline([(n, c, t) for n, c, t in summary], peaks, peak_kind,
                                    units_per_launch, w.B, w.H)
 
     # ---- end to end through the public API with host buffers
+    e2e = None
+    if args.skip_e2e:
+        del d
+        torch.cuda.empty_cache()
+    else:
+        e2e = run_e2e(args, ws, d, st)
+        torch.cuda.empty_cache()
+
+    # ---- decode step at 1280 sequences x 24 layers
+    dec = None if args.skip_decode else run_decode(args, ws, peaks, peak_kind)
+    clk = clocks.stop()
+    if clk is not None:
+        clk["region"] = "fwd+bwd and decode timed regions"
+    run_tail(args, ws, rank, value, ms_step, roof, shares, e2e, launches, clk, dec)
+
+
+def run_e2e(args, ws, d, st):
+    w = TRAIN
     pin = {n: torch.empty_like(d[n], device="cpu").pin_memory() for n in ("q", "k", "v", "a", "dO")}
     for n in pin:
         pin[n].copy_(d[n])
@@ -309,17 +386,12 @@ def run_ours(args, ws, rank, local):
     e1.record(st)
     e1.synchronize()
     e_elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3, ws)
-    e2e = {"value": round(ws * w.B * w.T * e_steps / e_elapsed, 1), "unit": "tokens/s",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    del d, pin, outs
-    torch.cuda.empty_cache()
+    return {"value": round(ws * w.B * w.T * e_steps / e_elapsed, 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    # ---- decode step at 1280 sequences x 24 layers
-    dec = run_decode(args, ws, peaks, peak_kind)
-    clk = clocks.stop()
-    if clk is not None:
-        clk["region"] = "fwd+bwd and decode timed regions"
 
+def run_tail(args, ws, rank, value, ms_step, roof, shares, e2e, launches, clk, dec):
+    w = TRAIN
     # ---- oracle on the host cores (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -392,6 +464,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-decode", action="store_true", help="time the training step only (profiling)")
+    ap.add_argument("--skip-e2e", action="store_true", help="no host-buffer end-to-end leg (profiling)")
     args = ap.parse_args()
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -191,6 +191,31 @@ gla_status conv1d_silu_causal(const void* x, int apply_ln, const float* ln_gamma
                               cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Front end at decode time: conv1d_silu_causal at T = 1 for N sequences
+ * whose conv histories live in a pool of slots, updated in place -- the way
+ * gla_decode_step addresses the recurrent states (the serving wrapper links
+ * the state to the serving memory pool: "AWS serve Laplace 3B ...", section
+ * "Lo stato di Laplace 3B resta fisso durante l'inferenza").  For sequence n
+ * with slot s = slot_idx[n] (n when NULL):
+ *     xn       = LayerNorm(x[n]) as in conv1d_silu_causal if apply_ln, else x[n]
+ *     y[n,c]   = SiLU( sum_{j<W-1} w[c,j] * h[s,j,c] + w[c,W-1] * xn[c] + bias[c] )
+ *     h[s]    <- (h[s,1], ..., h[s,W-2], xn)        (in place)
+ *   x, y        [N, D] bf16, contiguous.
+ *   conv_state  [N_slots, W-1, D] fp32: h, the last W-1 conv inputs of each
+ *               slot, oldest first (the layout of conv1d_silu_causal's
+ *               conv_state_in / _out for one sequence), updated in place.
+ *   slot_idx    [N] int32 or NULL (identity, N_slots = N).  Slots must be
+ *               distinct within one call and < N_slots (not checked on the
+ *               device).
+ *   ln_gamma/beta, w, bias as in conv1d_silu_causal.
+ * Supported: W == 4, D % 8 == 0, 8 <= D <= 4096.
+ * ------------------------------------------------------------------------ */
+gla_status conv1d_silu_decode_step(const void* x, const int32_t* slot_idx, int apply_ln,
+                                   const float* ln_gamma, const float* ln_beta, float ln_eps,
+                                   const float* w, const float* bias, float* conv_state, void* y,
+                                   int N, int D, int W, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Device status.  gla_get_device_status SYNCHRONISES the stream, copies the
  * device status word of the current device (0 or a gla_status recorded by a
  * kernel, e.g. GLA_ERR_TIMEOUT) into *device_status and clears it.

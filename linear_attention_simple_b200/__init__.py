@@ -19,7 +19,7 @@ __all__ = [
     "gla_chunk_workspace_bytes", "gla_chunk_fwd", "gla_chunk_bwd", "gla_decode_step",
     "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
-    "gla_chunk_fwd_noalloc", "EXPORTED_SYMBOLS", "LIB_PATH",
+    "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step", "EXPORTED_SYMBOLS", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgla.so")
@@ -29,7 +29,7 @@ EXPORTED_SYMBOLS = (
     "gla_chunk_workspace_bytes", "gla_chunk_fwd", "gla_chunk_bwd", "gla_decode_step",
     "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
-    "gla_chunk_fwd_noalloc",
+    "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step",
 )
 
 GLA_BF16, GLA_F32 = 0, 1
@@ -84,6 +84,8 @@ def lib():
     L.conv1d_silu_causal.restype = _i
     L.conv1d_silu_causal.argtypes = [_vp, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _vp,
                                      _i, _i, _i, _i, _vp]
+    L.conv1d_silu_decode_step.restype = _i
+    L.conv1d_silu_decode_step.argtypes = [_vp, _vp, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]
     L.gla_get_device_status.restype = _i
     L.gla_get_device_status.argtypes = [_vp, ctypes.POINTER(_i)]
     L.gla_set_wait_limit_ns.restype = _i
@@ -294,6 +296,34 @@ def conv1d_silu_causal(x, w, apply_ln=True, ln_gamma=None, ln_beta=None, ln_eps=
                                   float(ln_eps), _ptr(w), _ptr(bias), _ptr(conv_state_in),
                                   _ptr(conv_state_out), _ptr(y), B, T, D, W, _stream(stream))
     _check("conv1d_silu_causal", st)
+    return y
+
+
+def conv1d_silu_decode_step(x, w, conv_state, slot_idx=None, apply_ln=True, ln_gamma=None,
+                            ln_beta=None, ln_eps=1e-5, bias=None, y=None, stream=None):
+    """Front end at decode time: one token per sequence.  x [N,D] bf16;
+    conv_state [N_slots,W-1,D] fp32 (oldest first), updated in place;
+    slot_idx [N] int32 or None.  Returns y [N,D] bf16."""
+    N, D = x.shape
+    W = w.shape[1]
+    _need(x, "x", torch.bfloat16, (N, D))
+    _need(w, "w", torch.float32, (D, W))
+    _need(ln_gamma, "ln_gamma", torch.float32, (D,))
+    _need(ln_beta, "ln_beta", torch.float32, (D,))
+    _need(bias, "bias", torch.float32, (D,))
+    n_slots = conv_state.shape[0] if conv_state is not None else N
+    _need(conv_state, "conv_state", torch.float32, (n_slots, W - 1, D))
+    if slot_idx is not None:
+        _need(slot_idx, "slot_idx", torch.int32, (N,))
+    elif n_slots != N:
+        raise ValueError("conv_state has %d slots for %d sequences and no slot_idx" % (n_slots, N))
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", torch.bfloat16, (N, D))
+    st = lib().conv1d_silu_decode_step(_ptr(x), _ptr(slot_idx), 1 if apply_ln else 0, _ptr(ln_gamma),
+                                       _ptr(ln_beta), float(ln_eps), _ptr(w), _ptr(bias), _ptr(conv_state),
+                                       _ptr(y), N, D, W, _stream(stream))
+    _check("conv1d_silu_decode_step", st)
     return y
 
 

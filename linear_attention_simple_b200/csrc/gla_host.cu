@@ -346,6 +346,23 @@ gla_status conv1d_silu_causal(const void* x, int apply_ln, const float* ln_gamma
                        conv_state_out, y, B, T, D, stream);
 }
 
+gla_status conv1d_silu_decode_step(const void* x, const int32_t* slot_idx, int apply_ln,
+                                   const float* ln_gamma, const float* ln_beta, float ln_eps,
+                                   const float* w, const float* bias, float* conv_state, void* y,
+                                   int N, int D, int W, cudaStream_t stream)
+{
+    if (N < 0 || D <= 0 || W <= 0) return GLA_ERR_INVALID_ARG;
+    if (apply_ln && !(ln_eps > 0.0f && std::isfinite(ln_eps))) return GLA_ERR_INVALID_ARG;
+    if (W != 4 || D % 8 != 0 || D > 4096) return GLA_ERR_UNSUPPORTED;
+    if (N == 0) return GLA_OK;
+    if (!x || !y || !w || !conv_state) return GLA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(w) || !aligned16(ln_gamma) || !aligned16(ln_beta) ||
+        !aligned16(bias) || !aligned16(conv_state))
+        return GLA_ERR_MISALIGNED;
+    return launch_conv_decode(x, slot_idx, apply_ln, ln_gamma, ln_beta, ln_eps, w, bias, conv_state, y, N, D,
+                              stream);
+}
+
 gla_status gla_get_device_status(cudaStream_t stream, int* device_status)
 {
     if (!device_status) return GLA_ERR_INVALID_ARG;

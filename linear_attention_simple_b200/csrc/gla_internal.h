@@ -48,6 +48,10 @@ gla_status launch_conv(const void* x, int apply_ln, const float* g, const float*
                        const float* w, const float* bias, const float* cs_in, float* cs_out,
                        void* y, int B, int T, int D, cudaStream_t st);
 
+gla_status launch_conv_decode(const void* x, const int32_t* slot_idx, int apply_ln, const float* g,
+                              const float* b, float eps, const float* w, const float* bias, float* hist,
+                              void* y, int N, int D, cudaStream_t st);
+
 gla_status launch_fwd_f32(const float* q, const float* k, const float* v, const float* a,
                           const float* s0, float* o, float* s_final, int B, int T, int H,
                           int64_t ld_qk, int64_t ld_v, float scale, const WaitCtl& ctl,

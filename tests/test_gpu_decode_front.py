@@ -165,6 +165,79 @@ def test_front_end_full_size_sampled():
     _front_check(np.stack(got), np.stack(ref))
 
 
+# ---------------------------------------------------- decode front end
+
+def _pool_inputs(N, D, n_slots, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = inputs.randn((N, D), seed, "cuda").to(torch.bfloat16)
+    w = inputs.randn((D, 4), seed + 1, "cuda", std=0.5)
+    pool = inputs.randn((n_slots, 3, D), seed + 2, "cuda")
+    idx = torch.randperm(n_slots, generator=g)[:N].to(torch.int32).cuda()
+    return x, w, pool, idx
+
+
+@pytest.mark.parametrize("N,D,affine", [(1, 8, False), (37, 256, True), (64, 4096, True), (5, 3072, False)])
+def test_decode_front_parity_with_slot_pool(N, D, affine):
+    n_slots = 2 * N + 3
+    x, w, pool, idx = _pool_inputs(N, D, n_slots, 60 + N)
+    g = b = bias = None
+    if affine:
+        g = inputs.randn((D,), 61, "cuda", std=0.5) + 1.0
+        b = inputs.randn((D,), 62, "cuda", std=0.5)
+        bias = inputs.randn((D,), 63, "cuda", std=0.5)
+    before = pool.clone()
+    y = gla.conv1d_silu_decode_step(x, w, pool, slot_idx=idx, ln_gamma=g, ln_beta=b, bias=bias)
+    hist = _np(before[idx.long()])                                  # [N, 3, D]
+    ref_y, ref_cs = recurrent.ln_conv_silu(_np(x)[:, None, :], _np(w), ln=True,
+                                           ln_gamma=None if g is None else _np(g),
+                                           ln_beta=None if b is None else _np(b),
+                                           bias=None if bias is None else _np(bias), conv_state=hist)
+    _front_check(_np(y), ref_y[:, 0])
+    after = pool[idx.long()]
+    assert rel(_np(after), ref_cs) <= 1e-5
+    # the two older rows move down unchanged (bit-exact); other slots untouched
+    assert torch.equal(after[:, :2], before[idx.long()][:, 1:])
+    untouched = sorted(set(range(n_slots)) - set(idx.cpu().tolist()))
+    assert torch.equal(pool[untouched], before[untouched])
+
+
+def test_decode_front_steps_equal_the_sequence_front_end():
+    """T decode steps from a given history reproduce the oracle's front end over
+    the T tokens, and leave the oracle's final history in the slots."""
+    N, D, T = 6, 512, 9
+    d = inputs.front_inputs(N, T, D, seed=64, device="cuda", with_state=True)
+    pool = d["conv_state"].clone()
+    ys = [gla.conv1d_silu_decode_step(d["x"][:, t].contiguous(), d["w"], pool) for t in range(T)]
+    ref_y, ref_cs = recurrent.ln_conv_silu(_np(d["x"]), _np(d["w"]), conv_state=_np(d["conv_state"]))
+    _front_check(np.stack([_np(y) for y in ys], axis=1), ref_y)
+    assert rel(_np(pool), ref_cs) <= 1e-5
+
+
+def test_decode_front_without_layernorm():
+    N, D = 16, 1024
+    x, w, pool, _ = _pool_inputs(N, D, N, 65)
+    before = pool.clone()
+    y = gla.conv1d_silu_decode_step(x, w, pool, apply_ln=False)
+    ref_y, ref_cs = recurrent.ln_conv_silu(_np(x)[:, None, :], _np(w), ln=False, conv_state=_np(before))
+    _front_check(_np(y), ref_y[:, 0])
+    assert rel(_np(pool), ref_cs) <= 1e-6
+
+
+def test_decode_front_full_size_sampled():
+    """1,280 sequences x D = 3,072 (one layer of the decode step's front end),
+    checked on sampled sequences."""
+    N, D = 1280, 3072
+    x, w, pool, idx = _pool_inputs(N, D, 2 * N, 1006)
+    before = pool.clone()
+    y = gla.conv1d_silu_decode_step(x, w, pool, slot_idx=idx)
+    g = torch.Generator().manual_seed(11)
+    pick = torch.cat([torch.randperm(N, generator=g)[:64], torch.tensor([0, N - 1])])
+    hist = _np(before[idx[pick].long()])
+    ref_y, ref_cs = recurrent.ln_conv_silu(_np(x[pick])[:, None, :], _np(w), conv_state=hist)
+    _front_check(_np(y[pick]), ref_y[:, 0])
+    assert rel(_np(pool[idx[pick].long()]), ref_cs) <= 1e-5
+
+
 # -------------------------------------------------------------- fp32 path
 
 @pytest.mark.parametrize("B,T,H,s0", [(1, 256, 1, False), (2, 77, 3, True), (1, 1, 1, True)])

@@ -43,7 +43,9 @@
  * residual vector passes LayerNorm, then a causal depthwise Conv1d of width 4
  * with SiLU): y[t,c] = SiLU(sum_j w[c,j] * xn[t-(W-1)+j, c] + bias[c]), with
  * xn the LayerNorm output (biased variance over D, eps inside the root) and
- * positions before t = 0 taken from conv_state (zeros when absent).
+ * positions before t = 0 taken from conv_state (zeros when absent).  Its
+ * backward (gla_oracle_ln_conv_silu_bwd) is the chain rule through those
+ * three stages, written out below.
  *
  * A fault switch (gla_oracle_set_fault) plants a known mistake so the tests
  * can show that each pin catches it.  It is 0 outside those tests.
@@ -67,7 +69,9 @@ enum {
     FAULT_BWD_DA_NO_EXP = 5,   /* da_t misses its exp(a_t) factor                 */
     FAULT_BWD_DK_SIGN = 6,     /* dk sign flipped                                 */
     FAULT_LN_NO_CENTER = 7,    /* LayerNorm forgets to subtract the mean          */
-    FAULT_CONV_TAP_FLIP = 8    /* conv taps applied in reverse order              */
+    FAULT_CONV_TAP_FLIP = 8,   /* conv taps applied in reverse order              */
+    FAULT_BWD_SILU_SIGMOID = 9, /* front-end backward uses sigmoid(u) as SiLU'(u)  */
+    FAULT_BWD_LN_NO_MEAN = 10  /* LayerNorm backward drops the mean(g) term        */
 };
 static int g_fault = 0;
 
@@ -347,5 +351,121 @@ void gla_oracle_ln_conv_silu(const double* x, const double* ln_gamma, const doub
                     conv_state_out[((size_t)b * (W - 1) + r) * D + c] =
                         xn[((size_t)T + r) * D + c];
         free(xn);
+    }
+}
+
+/*
+ * Backward of the front end above (the per-layer LayerNorm -> causal
+ * depthwise conv -> SiLU of "Como i14 ...", section "Diseno esencial de
+ * Laplace 3B"), by the chain rule, for a loss whose gradient with respect to
+ * y is dy.  With xn the conv inputs (history rows first), u the conv output
+ * before SiLU and s = 1 / (1 + exp(-u)):
+ *     du[t,c]     = dy[t,c] * s * (1 + u (1 - s))           SiLU'(u)
+ *     dbias[c]    = sum_{b,t} du[t,c]
+ *     dw[c,j]     = sum_{b,t} du[t,c] * xn[t-(W-1)+j, c]
+ *     dxn[p,c]    = sum_j w[c,j] * du[p+(W-1)-j, c]           (du = 0 outside 0..T-1)
+ *   rows p < 0 are the history: dconv_state_in[b, p+W-1, c] = dxn[p,c].
+ *   LayerNorm, xhat = (x - mean) * rstd, xn = xhat * gamma + beta:
+ *     dgamma[c]   = sum_{b,t} dxn * xhat      dbeta[c] = sum_{b,t} dxn
+ *     g           = dxn * gamma
+ *     dx          = rstd * (g - mean_c(g) - xhat * mean_c(g * xhat))
+ *   (without LayerNorm, dx = dxn and dgamma = dbeta = 0).  The conv state
+ *   out carries no gradient back.  All outputs are overwritten.
+ */
+void gla_oracle_ln_conv_silu_bwd(const double* x, const double* ln_gamma, const double* ln_beta,
+                                 double ln_eps, int do_ln, const double* w, const double* bias,
+                                 const double* conv_state_in, const double* dy, double* dx, double* dw,
+                                 double* dbias, double* dgamma, double* dbeta, double* dconv_state_in,
+                                 int B, int T, int D, int W)
+{
+    for (int c = 0; c < D; ++c) {
+        dbias[c] = dgamma[c] = dbeta[c] = 0.0;
+        for (int j = 0; j < W; ++j) dw[(size_t)c * W + j] = 0.0;
+    }
+    for (int b = 0; b < B; ++b) {
+        const size_t rows = (size_t)T + W - 1;
+        double* xn = (double*)malloc(sizeof(double) * rows * D);
+        double* xh = (double*)malloc(sizeof(double) * (size_t)T * D);
+        double* rs = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+        double* du = (double*)malloc(sizeof(double) * (size_t)T * D);
+        double* dxn = (double*)malloc(sizeof(double) * rows * D);
+        for (int r = 0; r < W - 1; ++r)
+            for (int c = 0; c < D; ++c)
+                xn[(size_t)r * D + c] = conv_state_in ? conv_state_in[((size_t)b * (W - 1) + r) * D + c] : 0.0;
+        /* forward again: LayerNorm rows, conv, SiLU'(u) */
+        for (int t = 0; t < T; ++t) {
+            const double* xr = x + ((size_t)b * T + t) * D;
+            double* out = xn + ((size_t)t + W - 1) * D;
+            double* h = xh + (size_t)t * D;
+            if (!do_ln) {
+                for (int c = 0; c < D; ++c) out[c] = h[c] = xr[c];
+                rs[t] = 1.0;
+                continue;
+            }
+            double mean = 0.0, var = 0.0;
+            for (int c = 0; c < D; ++c) mean += xr[c];
+            mean /= D;
+            for (int c = 0; c < D; ++c) var += (xr[c] - mean) * (xr[c] - mean);
+            var /= D;
+            rs[t] = 1.0 / sqrt(var + ln_eps);
+            for (int c = 0; c < D; ++c) {
+                h[c] = (xr[c] - mean) * rs[t];
+                out[c] = h[c] * (ln_gamma ? ln_gamma[c] : 1.0) + (ln_beta ? ln_beta[c] : 0.0);
+            }
+        }
+        for (int t = 0; t < T; ++t)
+            for (int c = 0; c < D; ++c) {
+                double u = bias ? bias[c] : 0.0;
+                for (int j = 0; j < W; ++j) u += w[(size_t)c * W + j] * xn[((size_t)t + j) * D + c];
+                const double sg = 1.0 / (1.0 + exp(-u));
+                const double dsilu = (g_fault == FAULT_BWD_SILU_SIGMOID) ? sg : sg * (1.0 + u * (1.0 - sg));
+                const double g = dy[((size_t)b * T + t) * D + c] * dsilu;
+                du[(size_t)t * D + c] = g;
+                dbias[c] += g;
+                for (int j = 0; j < W; ++j) dw[(size_t)c * W + j] += g * xn[((size_t)t + j) * D + c];
+            }
+        /* dxn over all rows, history included: row r = p + W - 1 */
+        for (size_t r = 0; r < rows; ++r)
+            for (int c = 0; c < D; ++c) {
+                double acc = 0.0;
+                for (int j = 0; j < W; ++j) {
+                    const long t = (long)r - j;           /* p + (W-1) - j with p = r - (W-1) */
+                    if (t >= 0 && t < T) acc += w[(size_t)c * W + j] * du[(size_t)t * D + c];
+                }
+                dxn[r * D + c] = acc;
+            }
+        if (dconv_state_in)
+            for (int r = 0; r < W - 1; ++r)
+                for (int c = 0; c < D; ++c)
+                    dconv_state_in[((size_t)b * (W - 1) + r) * D + c] = dxn[(size_t)r * D + c];
+        for (int t = 0; t < T; ++t) {
+            const double* d = dxn + ((size_t)t + W - 1) * D;
+            const double* h = xh + (size_t)t * D;
+            double* o = dx + ((size_t)b * T + t) * D;
+            if (!do_ln) {
+                for (int c = 0; c < D; ++c) o[c] = d[c];
+                continue;
+            }
+            double mg = 0.0, mgh = 0.0;
+            for (int c = 0; c < D; ++c) {
+                const double g = d[c] * (ln_gamma ? ln_gamma[c] : 1.0);
+                mg += g;
+                mgh += g * h[c];
+                dgamma[c] += d[c] * h[c];
+                dbeta[c] += d[c];
+            }
+            mg /= D;
+            mgh /= D;
+            if (g_fault == FAULT_BWD_LN_NO_MEAN) mg = 0.0;
+            for (int c = 0; c < D; ++c) {
+                const double g = d[c] * (ln_gamma ? ln_gamma[c] : 1.0);
+                o[c] = rs[t] * (g - mg - h[c] * mgh);
+            }
+        }
+        free(xn);
+        free(xh);
+        free(rs);
+        free(du);
+        free(dxn);
     }
 }

@@ -32,6 +32,7 @@ def _lib():
         lib.gla_oracle_bwd.restype = None
         lib.gla_oracle_decode.restype = None
         lib.gla_oracle_ln_conv_silu.restype = None
+        lib.gla_oracle_ln_conv_silu_bwd.restype = None
         lib.gla_oracle_set_fault.argtypes = [ctypes.c_int]
         lib.gla_oracle_get_fault.restype = ctypes.c_int
         lib.gla_oracle_max_threads.restype = ctypes.c_int
@@ -60,6 +61,8 @@ def max_threads() -> int:
 
 
 FAULTS = {
+    "bwd_silu_sigmoid": 9,
+    "bwd_ln_no_mean": 10,
     "no_decay": 1,
     "exclusive_state": 2,
     "double_scale": 3,
@@ -155,3 +158,28 @@ def ln_conv_silu(x, w, ln=True, ln_gamma=None, ln_beta=None, ln_eps=1e-5, bias=N
     _lib().gla_oracle_ln_conv_silu(xp, gp, bp, ctypes.c_double(ln_eps), 1 if ln else 0, wp, bip,
                                    csp, _ptr(cso), _ptr(y), B, T, D, W, 1 if silu else 0)
     return y, cso
+
+
+def ln_conv_silu_bwd(x, w, dy, ln=True, ln_gamma=None, ln_beta=None, ln_eps=1e-5, bias=None,
+                     conv_state=None):
+    """Backward of ln_conv_silu for the gradient dy of y.  Returns
+    (dx [B,T,D], dw [D,W], dbias [D], dgamma [D], dbeta [D], dconv_state [B,W-1,D])."""
+    x, xp = _in(x)
+    w, wp = _in(w)
+    dy, dyp = _in(dy)
+    g, gp = _in(ln_gamma)
+    be, bp = _in(ln_beta)
+    bi, bip = _in(bias)
+    cs, csp = _in(conv_state)
+    B, T, D = x.shape
+    W = w.shape[1]
+    dx = np.zeros_like(x)
+    dw = np.zeros((D, W), np.float64)
+    dbias = np.zeros(D, np.float64)
+    dgamma = np.zeros(D, np.float64)
+    dbeta = np.zeros(D, np.float64)
+    dcs = np.zeros((B, W - 1, D), np.float64)
+    _lib().gla_oracle_ln_conv_silu_bwd(xp, gp, bp, ctypes.c_double(ln_eps), 1 if ln else 0, wp, bip, csp,
+                                       dyp, _ptr(dx), _ptr(dw), _ptr(dbias), _ptr(dgamma), _ptr(dbeta),
+                                       _ptr(dcs), B, T, D, W)
+    return dx, dw, dbias, dgamma, dbeta, dcs

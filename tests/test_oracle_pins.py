@@ -249,6 +249,71 @@ def test_front_end_composes():
     assert _rel(y, pre * scipy.special.expit(pre)) < 1e-13
 
 
+# ------------------------------------------------ front-end backward pins
+
+def _front_bwd_case(seed=18, T=6, D=8, ln=True):
+    rng = np.random.default_rng(seed)
+    B, W = 2, 4
+    return dict(x=rng.standard_normal((B, T, D)) + 0.5, w=rng.standard_normal((D, W)) * 0.5,
+                dy=rng.standard_normal((B, T, D)), g=1.0 + 0.5 * rng.standard_normal(D),
+                be=0.5 * rng.standard_normal(D), bias=0.5 * rng.standard_normal(D),
+                hist=rng.standard_normal((B, W - 1, D)), ln=ln)
+
+
+def _front_loss(c, **over):
+    v = dict(c)
+    v.update(over)
+    y, _ = recurrent.ln_conv_silu(v["x"], v["w"], ln=v["ln"], ln_gamma=v["g"] if v["ln"] else None,
+                                  ln_beta=v["be"] if v["ln"] else None, bias=v["bias"], conv_state=v["hist"])
+    return float(np.sum(y * c["dy"]))
+
+
+def check_front_fd():
+    """Central differences of sum(dy * y) through the pinned forward, every
+    input element, against the oracle's backward; max relative error."""
+    worst = 0.0
+    for ln in (True, False):
+        c = _front_bwd_case(ln=ln)
+        dx, dw, dbias, dg, dbe, dcs = recurrent.ln_conv_silu_bwd(
+            c["x"], c["w"], c["dy"], ln=ln, ln_gamma=c["g"] if ln else None, ln_beta=c["be"] if ln else None,
+            bias=c["bias"], conv_state=c["hist"])
+        pairs = [("x", dx), ("w", dw), ("bias", dbias), ("hist", dcs)] + ([("g", dg), ("be", dbe)] if ln else [])
+        h = 1e-6
+        for name, grad in pairs:
+            num = np.zeros_like(grad)
+            base = c[name]
+            for idx in np.ndindex(base.shape):
+                p_, m_ = base.copy(), base.copy()
+                p_[idx] += h
+                m_[idx] -= h
+                num[idx] = (_front_loss(c, **{name: p_}) - _front_loss(c, **{name: m_})) / (2 * h)
+            worst = max(worst, _rel(grad, num))
+    return worst
+
+
+def test_front_end_backward_finite_differences():
+    assert check_front_fd() < 1e-6
+
+
+def test_front_end_backward_matches_torch_autograd():
+    """The oracle's hand-written backward against torch float64 autograd of an
+    independently written forward (layer_norm, a causal conv1d over the history,
+    silu)."""
+    import torch
+    c = _front_bwd_case(seed=19, T=9, D=16)
+    t = {k: torch.tensor(c[k], dtype=torch.float64, requires_grad=True) for k in ("x", "w", "g", "be", "bias", "hist")}
+    D = c["x"].shape[-1]
+    xn = torch.nn.functional.layer_norm(t["x"], (D,), t["g"], t["be"], eps=1e-5)
+    seq = torch.cat([t["hist"], xn], dim=1).transpose(1, 2)              # [B, D, W-1+T]
+    u = torch.nn.functional.conv1d(seq, t["w"].unsqueeze(1), t["bias"], groups=D).transpose(1, 2)
+    y = torch.nn.functional.silu(u)
+    (y * torch.tensor(c["dy"])).sum().backward()
+    dx, dw, dbias, dg, dbe, dcs = recurrent.ln_conv_silu_bwd(c["x"], c["w"], c["dy"], ln_gamma=c["g"],
+                                                             ln_beta=c["be"], bias=c["bias"], conv_state=c["hist"])
+    for ours, ref in ((dx, t["x"]), (dw, t["w"]), (dbias, t["bias"]), (dg, t["g"]), (dbe, t["be"]), (dcs, t["hist"])):
+        assert _rel(ours, ref.grad.numpy()) < 1e-12
+
+
 # ------------------------------------------------------------------ sizing pin
 
 def test_sizing_identities_from_the_pages():
@@ -273,6 +338,8 @@ PIN_FOR_FAULT = {
     "bwd_dk_sign": lambda: check_finite_differences() < 1e-6,
     "ln_no_center": lambda: check_ln_moments() < 1e-12,
     "conv_tap_flip": lambda: check_conv_vs_numpy() < 1e-13,
+    "bwd_silu_sigmoid": lambda: check_front_fd() < 1e-6,
+    "bwd_ln_no_mean": lambda: check_front_fd() < 1e-6,
 }
 
 

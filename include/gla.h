@@ -191,6 +191,37 @@ gla_status conv1d_silu_causal(const void* x, int apply_ln, const float* ln_gamma
                               cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Backward of conv1d_silu_causal, for training the mixer block: given dy,
+ * the gradient of a loss with respect to y, compute the gradients of x, of
+ * the conv weights and bias, of the LayerNorm affine and of conv_state_in.
+ * The forward is recomputed from x (nothing is saved between the calls);
+ * conv_state_out carries no gradient back.  With u the conv output before
+ * SiLU, s = sigmoid(u), xhat the normalised rows:
+ *     du      = dy * s * (1 + u (1 - s))
+ *     dxn[p]  = sum_j w[c,j] * du[p+W-1-j]            (rows p < 0: dconv_state_in)
+ *     dx      = rstd * (g - mean(g) - xhat * mean(g * xhat)),  g = dxn * gamma
+ *               (dx = dxn without LayerNorm)
+ *     dw[c,j] = sum_{b,t} du[t,c] * xn[t-(W-1)+j, c]     dbias = sum du
+ *     dln_gamma = sum dxn * xhat                           dln_beta = sum dxn
+ *   x, dy, dx       [B, T, D] bf16.   dw [D, W] fp32 (required).
+ *   dbias, dln_gamma, dln_beta [D] fp32, dconv_state_in [B, W-1, D] fp32:
+ *                   each NULL = not wanted.  Every output is overwritten.
+ *   ws              ws_bytes >= conv1d_silu_causal_bwd_workspace_bytes(B,T,D,W)
+ *                   (per-CTA partial sums, added in a fixed order: results do
+ *                   not depend on scheduling).
+ * Other arguments as in conv1d_silu_causal.  Supported: W == 4, D % 8 == 0,
+ * 8 <= D <= 4096, B <= 65535.
+ * ------------------------------------------------------------------------ */
+size_t conv1d_silu_causal_bwd_workspace_bytes(int B, int T, int D, int W);
+gla_status conv1d_silu_causal_bwd(const void* x, int apply_ln, const float* ln_gamma,
+                                  const float* ln_beta, float ln_eps, const float* w,
+                                  const float* bias, const float* conv_state_in, const void* dy,
+                                  void* dx, float* dw, float* dbias, float* dln_gamma,
+                                  float* dln_beta, float* dconv_state_in, void* ws,
+                                  size_t ws_bytes, int B, int T, int D, int W,
+                                  cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Front end at decode time: conv1d_silu_causal at T = 1 for N sequences
  * whose conv histories live in a pool of slots, updated in place -- the way
  * gla_decode_step addresses the recurrent states (the serving wrapper links

@@ -19,7 +19,8 @@ __all__ = [
     "gla_chunk_workspace_bytes", "gla_chunk_fwd", "gla_chunk_bwd", "gla_decode_step",
     "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
-    "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step", "EXPORTED_SYMBOLS", "LIB_PATH",
+    "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step", "conv1d_silu_causal_bwd",
+    "conv1d_silu_causal_bwd_workspace_bytes", "EXPORTED_SYMBOLS", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgla.so")
@@ -29,7 +30,8 @@ EXPORTED_SYMBOLS = (
     "gla_chunk_workspace_bytes", "gla_chunk_fwd", "gla_chunk_bwd", "gla_decode_step",
     "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
-    "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step",
+    "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step", "conv1d_silu_causal_bwd",
+    "conv1d_silu_causal_bwd_workspace_bytes",
 )
 
 GLA_BF16, GLA_F32 = 0, 1
@@ -84,6 +86,11 @@ def lib():
     L.conv1d_silu_causal.restype = _i
     L.conv1d_silu_causal.argtypes = [_vp, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _vp,
                                      _i, _i, _i, _i, _vp]
+    L.conv1d_silu_causal_bwd_workspace_bytes.restype = ctypes.c_size_t
+    L.conv1d_silu_causal_bwd_workspace_bytes.argtypes = [_i, _i, _i, _i]
+    L.conv1d_silu_causal_bwd.restype = _i
+    L.conv1d_silu_causal_bwd.argtypes = [_vp, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                         _vp, _vp, ctypes.c_size_t, _i, _i, _i, _i, _vp]
     L.conv1d_silu_decode_step.restype = _i
     L.conv1d_silu_decode_step.argtypes = [_vp, _vp, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]
     L.gla_get_device_status.restype = _i
@@ -297,6 +304,42 @@ def conv1d_silu_causal(x, w, apply_ln=True, ln_gamma=None, ln_beta=None, ln_eps=
                                   _ptr(conv_state_out), _ptr(y), B, T, D, W, _stream(stream))
     _check("conv1d_silu_causal", st)
     return y
+
+
+def conv1d_silu_causal_bwd_workspace_bytes(B, T, D, W=4):
+    return int(lib().conv1d_silu_causal_bwd_workspace_bytes(B, T, D, W))
+
+
+def conv1d_silu_causal_bwd(x, w, dy, apply_ln=True, ln_gamma=None, ln_beta=None, ln_eps=1e-5, bias=None,
+                           conv_state_in=None, want=("dx", "dw", "dbias", "dln_gamma", "dln_beta", "dconv_state_in"),
+                           ws=None, stream=None):
+    """Backward of conv1d_silu_causal.  Returns a dict with the gradients in
+    `want` (dx [B,T,D] bf16; dw [D,W], dbias, dln_gamma, dln_beta [D],
+    dconv_state_in [B,W-1,D] fp32)."""
+    B, T, D = x.shape
+    W = w.shape[1]
+    _need(x, "x", torch.bfloat16, (B, T, D))
+    _need(dy, "dy", torch.bfloat16, (B, T, D))
+    _need(w, "w", torch.float32, (D, W))
+    _need(ln_gamma, "ln_gamma", torch.float32, (D,))
+    _need(ln_beta, "ln_beta", torch.float32, (D,))
+    _need(bias, "bias", torch.float32, (D,))
+    _need(conv_state_in, "conv_state_in", torch.float32, (B, W - 1, D))
+    dev = x.device
+    out = {"dx": torch.empty_like(x), "dw": torch.empty((D, W), dtype=torch.float32, device=dev)}
+    for name, shape in (("dbias", (D,)), ("dln_gamma", (D,)), ("dln_beta", (D,)),
+                        ("dconv_state_in", (B, W - 1, D))):
+        out[name] = torch.empty(shape, dtype=torch.float32, device=dev) if name in want else None
+    need = conv1d_silu_causal_bwd_workspace_bytes(B, T, D, W)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    st = lib().conv1d_silu_causal_bwd(_ptr(x), 1 if apply_ln else 0, _ptr(ln_gamma), _ptr(ln_beta), float(ln_eps),
+                                      _ptr(w), _ptr(bias), _ptr(conv_state_in), _ptr(dy), _ptr(out["dx"]),
+                                      _ptr(out["dw"]), _ptr(out["dbias"]), _ptr(out["dln_gamma"]),
+                                      _ptr(out["dln_beta"]), _ptr(out["dconv_state_in"]), _ptr(ws),
+                                      ws.numel() * ws.element_size(), B, T, D, W, _stream(stream))
+    _check("conv1d_silu_causal_bwd", st)
+    return {k: v for k, v in out.items() if k in want or k in ("dx", "dw")}
 
 
 def conv1d_silu_decode_step(x, w, conv_state, slot_idx=None, apply_ln=True, ln_gamma=None,

@@ -363,6 +363,44 @@ gla_status conv1d_silu_decode_step(const void* x, const int32_t* slot_idx, int a
                               stream);
 }
 
+size_t conv1d_silu_causal_bwd_workspace_bytes(int B, int T, int D, int W)
+{
+    if (B <= 0 || T <= 0 || W != 4 || D <= 0 || D % 8 != 0 || D > 4096) return 0;
+    return conv_bwd_workspace_bytes(B, T, D);
+}
+
+gla_status conv1d_silu_causal_bwd(const void* x, int apply_ln, const float* ln_gamma, const float* ln_beta,
+                                  float ln_eps, const float* w, const float* bias, const float* conv_state_in,
+                                  const void* dy, void* dx, float* dw, float* dbias, float* dln_gamma,
+                                  float* dln_beta, float* dconv_state_in, void* ws, size_t ws_bytes, int B, int T,
+                                  int D, int W, cudaStream_t stream)
+{
+    if (B < 0 || T < 0 || D <= 0 || W <= 0) return GLA_ERR_INVALID_ARG;
+    if (apply_ln && !(ln_eps > 0.0f && std::isfinite(ln_eps))) return GLA_ERR_INVALID_ARG;
+    if (W != 4 || D % 8 != 0 || D > 4096) return GLA_ERR_UNSUPPORTED;
+    if (!w || !dw) return GLA_ERR_INVALID_ARG;
+    if (B > 65535) return GLA_ERR_UNSUPPORTED;
+    if (!aligned16(w) || !aligned16(ln_gamma) || !aligned16(ln_beta) || !aligned16(bias) ||
+        !aligned16(conv_state_in) || !aligned16(dw) || !aligned16(dbias) || !aligned16(dln_gamma) ||
+        !aligned16(dln_beta) || !aligned16(dconv_state_in) || !aligned16(ws))
+        return GLA_ERR_MISALIGNED;
+    if (B == 0 || T == 0) {
+        // no tokens: every gradient is zero
+        cudaError_t e = cudaMemsetAsync(dw, 0, static_cast<size_t>(D) * W * sizeof(float), stream);
+        if (e == cudaSuccess && dbias) e = cudaMemsetAsync(dbias, 0, D * sizeof(float), stream);
+        if (e == cudaSuccess && dln_gamma) e = cudaMemsetAsync(dln_gamma, 0, D * sizeof(float), stream);
+        if (e == cudaSuccess && dln_beta) e = cudaMemsetAsync(dln_beta, 0, D * sizeof(float), stream);
+        if (e == cudaSuccess && dconv_state_in && B > 0)
+            e = cudaMemsetAsync(dconv_state_in, 0, static_cast<size_t>(B) * (W - 1) * D * sizeof(float), stream);
+        return e == cudaSuccess ? GLA_OK : cuda_fail(e);
+    }
+    if (!x || !dy || !dx) return GLA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(dy) || !aligned16(dx)) return GLA_ERR_MISALIGNED;
+    if (!ws || ws_bytes < conv_bwd_workspace_bytes(B, T, D)) return GLA_ERR_INVALID_ARG;
+    return launch_conv_bwd(x, apply_ln, ln_gamma, ln_beta, ln_eps, w, bias, conv_state_in, dy, dx, dw, dbias,
+                           dln_gamma, dln_beta, dconv_state_in, ws, B, T, D, stream);
+}
+
 gla_status gla_get_device_status(cudaStream_t stream, int* device_status)
 {
     if (!device_status) return GLA_ERR_INVALID_ARG;

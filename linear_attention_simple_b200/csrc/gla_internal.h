@@ -52,6 +52,11 @@ gla_status launch_conv_decode(const void* x, const int32_t* slot_idx, int apply_
                               const float* b, float eps, const float* w, const float* bias, float* hist,
                               void* y, int N, int D, cudaStream_t st);
 
+size_t conv_bwd_workspace_bytes(int B, int T, int D);
+gla_status launch_conv_bwd(const void* x, int apply_ln, const float* g, const float* be, float eps, const float* w,
+                           const float* bias, const float* cs_in, const void* dy, void* dx, float* dw, float* dbias,
+                           float* dgamma, float* dbeta, float* dcs, void* ws, int B, int T, int D, cudaStream_t st);
+
 gla_status launch_fwd_f32(const float* q, const float* k, const float* v, const float* a,
                           const float* s0, float* o, float* s_final, int B, int T, int H,
                           int64_t ld_qk, int64_t ld_v, float scale, const WaitCtl& ctl,

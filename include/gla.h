@@ -100,6 +100,29 @@ gla_status gla_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          gla_dtype dt, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Chunked forward over a packed batch of sequences of different lengths
+ * (prefill of several requests at once): gla_chunk_fwd for each sequence n,
+ * whose tokens are rows cu_seqlens[n] .. cu_seqlens[n+1]-1 of q, k, v, a and
+ * o, each sequence with its own initial and final state.  The chunk grid
+ * restarts at every sequence; tokens of one sequence never enter another's
+ * state or output.
+ *   q, k        [total_T, H, 96], v [total_T, H, 192] bf16, token stride
+ *               ld_qkv as in gla_chunk_fwd (0 = packed).
+ *   a           [total_T, H] fp32.    o [total_T, H, 192] bf16.
+ *   cu_seqlens  DEVICE pointer, [N+1] int32, non-decreasing, cu_seqlens[0] >= 0,
+ *               cu_seqlens[N] <= total_T.  A sequence whose offsets fall
+ *               outside 0 .. total_T is skipped and GLA_ERR_INVALID_ARG is
+ *               recorded in the device status word (gla_get_device_status).
+ *   s0, s_final [N, H, 96, 192] fp32 or NULL (zeros / not wanted).
+ * Rows of o outside every sequence are not written.  dt must be GLA_BF16;
+ * N <= 65535.  No workspace.
+ * ------------------------------------------------------------------------ */
+gla_status gla_chunk_fwd_varlen(const void* q, const void* k, const void* v, const float* a,
+                                const int32_t* cu_seqlens, int N, const float* s0, void* o,
+                                float* s_final, int total_T, int H, int dk, int dv, int64_t ld_qkv,
+                                float scale, gla_dtype dt, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * gla_chunk_fwd for callers that cannot allocate device memory.  (The pages
  * have no counterpart to this call; it exists for library users.)
  *

@@ -20,7 +20,7 @@ __all__ = [
     "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
     "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step", "conv1d_silu_causal_bwd",
-    "conv1d_silu_causal_bwd_workspace_bytes", "EXPORTED_SYMBOLS", "LIB_PATH",
+    "conv1d_silu_causal_bwd_workspace_bytes", "gla_chunk_fwd_varlen", "EXPORTED_SYMBOLS", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgla.so")
@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = (
     "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
     "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step", "conv1d_silu_causal_bwd",
-    "conv1d_silu_causal_bwd_workspace_bytes",
+    "conv1d_silu_causal_bwd_workspace_bytes", "gla_chunk_fwd_varlen",
 )
 
 GLA_BF16, GLA_F32 = 0, 1
@@ -91,6 +91,9 @@ def lib():
     L.conv1d_silu_causal_bwd.restype = _i
     L.conv1d_silu_causal_bwd.argtypes = [_vp, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                          _vp, _vp, ctypes.c_size_t, _i, _i, _i, _i, _vp]
+    L.gla_chunk_fwd_varlen.restype = _i
+    L.gla_chunk_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i,
+                                       ctypes.c_longlong, _f, _i, _vp]
     L.conv1d_silu_decode_step.restype = _i
     L.conv1d_silu_decode_step.argtypes = [_vp, _vp, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]
     L.gla_get_device_status.restype = _i
@@ -304,6 +307,35 @@ def conv1d_silu_causal(x, w, apply_ln=True, ln_gamma=None, ln_beta=None, ln_eps=
                                   _ptr(conv_state_out), _ptr(y), B, T, D, W, _stream(stream))
     _check("conv1d_silu_causal", st)
     return y
+
+
+def gla_chunk_fwd_varlen(q, k, v, a, cu_seqlens, s0=None, o=None, s_final=None, scale=None,
+                         want_final_state=True, stream=None):
+    """Chunked forward over packed sequences: q, k [total,H,96], v [total,H,192]
+    bf16, a [total,H] fp32, cu_seqlens [N+1] int32 on the device.  Returns
+    (o [total,H,192] bf16, s_final [N,H,96,192] fp32 or None)."""
+    total, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype != torch.bfloat16:
+        raise TypeError("gla_chunk_fwd_varlen takes bf16 q, k, v")
+    _need(k, "k", torch.bfloat16, (total, H, dk))
+    _need(v, "v", torch.bfloat16, (total, H, dv))
+    _need(q, "q", torch.bfloat16, (total, H, dk))
+    _need(a, "a", torch.float32, (total, H))
+    N = cu_seqlens.numel() - 1
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,))
+    _need(s0, "s0", torch.float32, (N, H, dk, dv))
+    if o is None:
+        o = torch.empty((total, H, dv), dtype=torch.bfloat16, device=q.device)
+    _need(o, "o", torch.bfloat16, (total, H, dv))
+    if s_final is None and want_final_state:
+        s_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(s_final, "s_final", torch.float32, (N, H, dk, dv))
+    sc = dk ** -0.5 if scale is None else scale
+    st = lib().gla_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(cu_seqlens), N, _ptr(s0), _ptr(o),
+                                    _ptr(s_final), total, H, dk, dv, 0, float(sc), GLA_BF16, _stream(stream))
+    _check("gla_chunk_fwd_varlen", st)
+    return o, s_final
 
 
 def conv1d_silu_causal_bwd_workspace_bytes(B, T, D, W=4):

@@ -101,8 +101,10 @@ gla_status launch_state_kernel(bool with_o, bool reverse, const StateParams& p, 
                                cudaStream_t st)
 {
     if (with_o && !reverse)
-        return launch_chunk_kernel(gla_fwd_fused_kernel, chunk::FusedSmem::BYTES,
-                                   "chunk_fwd_fused_kernel", p, grid, st, chunk::kFusedThreads);
+        return p.cu_seqlens ? launch_chunk_kernel(gla_fwd_fused_kernel<true>, chunk::FusedSmem::BYTES,
+                                                  "chunk_fwd_varlen_kernel", p, grid, st, chunk::kFusedThreads)
+                            : launch_chunk_kernel(gla_fwd_fused_kernel<false>, chunk::FusedSmem::BYTES,
+                                                  "chunk_fwd_fused_kernel", p, grid, st, chunk::kFusedThreads);
     if (!with_o && !reverse)
         return launch_chunk_kernel(gla_state_pass_kernel<false>, chunk::PassSmem::BYTES,
                                    "chunk_state_fwd_kernel", p, grid, st, chunk::kPassThreads);
@@ -120,6 +122,36 @@ size_t fwd_workspace_bytes(int B, int T, int H)
     if (nseg == 1) return 0;
     return align256(static_cast<size_t>(units) * nseg * kSS * sizeof(float)) +
            align256(static_cast<size_t>(units) * nseg * sizeof(float));
+}
+
+gla_status run_chunk_fwd_varlen(const ChunkProblem& pr, const int* cu_seqlens, int N, const float* s0, void* o,
+                                float* s_final, const WaitCtl& ctl, cudaStream_t st)
+{
+    // pr.B == 1, pr.T == total tokens; one CTA per (sequence, head)
+    StateParams p;
+    memset(&p, 0, sizeof(p));
+    gla_status s;
+    if ((s = make_token_map(&p.tm_q, pr.q, kDk, pr.H, pr.T, 1, pr.ld_qk, 32, 64, 16)) != GLA_OK) return s;
+    if ((s = make_token_map(&p.tm_u, pr.k, kDk, pr.H, pr.T, 1, pr.ld_qk, 32, 64)) != GLA_OK) return s;
+    if ((s = make_token_map(&p.tm_y, pr.v, kDv, pr.H, pr.T, 1, pr.ld_v, 64, 128)) != GLA_OK) return s;
+    if ((s = make_token_map(&p.tm_o, o, kDv, pr.H, pr.T, 1, static_cast<int64_t>(pr.H) * kDv, 64, 128)) != GLA_OK)
+        return s;
+    p.a = pr.a;
+    p.B = N;
+    p.T = pr.T;
+    p.H = pr.H;
+    p.NC = num_chunks(pr.T);
+    p.chunks_per_seg = 1 << 30;
+    p.scale = pr.scale;
+    p.ctl = ctl;
+    p.cu_seqlens = cu_seqlens;
+    p.o_direct = o;
+    p.s_init = s0;
+    p.init_unit_stride = kSS;
+    p.s_out = s_final;
+    p.out_unit_stride = kSS;
+    p.out_last_only = 1;
+    return launch_state_kernel(true, false, p, dim3(1, pr.H, N), st);
 }
 
 gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float* s_final,

@@ -74,6 +74,8 @@ struct StateParams {
     int g2_unit_stride;     // segments per unit in g2_out
     int store_h;            // store the bf16 state entering each chunk into h_out
     void* h_out;            // bf16 [B*H*NC][96][192]
+    const int* cu_seqlens;  // varlen forward: [B+1] token offsets into batch row 0, or null
+    void* o_direct;         // varlen forward: o, for the direct stores of a sequence's last chunk
     float scale;
     WaitCtl ctl;
 };
@@ -306,6 +308,7 @@ __device__ __forceinline__ void state_copy_and_decay(uint32_t taddr, int row, in
 // =====================================================================
 // Fused forward.
 // =====================================================================
+template <bool VARLEN>
 __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(const __grid_constant__ StateParams p)
 {
     using namespace chunk;
@@ -328,8 +331,21 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int unit = b * p.H + h;
+    // varlen: blockIdx.z is a sequence, its tokens tb .. tb+Tn-1 of batch row
+    // 0; otherwise batch row b, tokens 0 .. T-1
+    int tb = 0, Tn = p.T, NCn = p.NC;
+    if constexpr (VARLEN) {
+        tb = p.cu_seqlens[b];
+        Tn = p.cu_seqlens[b + 1] - tb;
+        NCn = (Tn + 127) / 128;
+        if (tb < 0 || Tn < 0 || tb + Tn > p.T) {   // offsets out of range: touch nothing
+            if (threadIdx.x == 0) record_status(p.ctl.status, GLA_ERR_INVALID_ARG);
+            return;
+        }
+    }
+    const int bc = VARLEN ? 0 : b;                 // batch coordinate of the token tensors
     const int c_begin = seg * p.chunks_per_seg;
-    const int c_end = min(p.NC, c_begin + p.chunks_per_seg);
+    const int c_end = min(NCn, c_begin + p.chunks_per_seg);
     const int nchunks = c_end - c_begin;
     const WaitCtl ctl = p.ctl;
 
@@ -371,7 +387,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
 
     auto load_a = [&](int c) {
         const int t = c * 128 + tid;
-        return t < p.T ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f;
+        return t < Tn ? p.a[(static_cast<int64_t>(bc) * p.T + tb + t) * p.H + h] : 0.f;
     };
     // per barrier at most one phase is ever outstanding
     uint32_t ph_q = 0, ph_u = 0, ph_y[2] = {0u, 0u}, mph = 0;
@@ -400,14 +416,15 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             for (int i = 0; i < 3; ++i)
                 for (int r16 = 0; r16 < 8; ++r16)
                     tma_load_4d(sm + L::Q + i * 8192 + r16 * 1024, &p.tm_q, bar_q, i * 32, h,
-                                t0 + perm16(r16) * 16, b);
+                                tb + t0 + perm16(r16) * 16, bc);
             mbar_arrive_expect_tx(bar_u, kTileQK);
-            for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::U + i * 8192, &p.tm_u, bar_u, i * 32, h, t0, b);
+            for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::U + i * 8192, &p.tm_u, bar_u, i * 32, h, tb + t0, bc);
         };
         auto issue_y = [&](int c, int s) {
             uint8_t* y = sm + (s ? L::Y1 : L::Y0);
             mbar_arrive_expect_tx(bar_y + s, kTileV);
-            for (int i = 0; i < 3; ++i) tma_load_4d(y + i * 16384, &p.tm_y, bar_y + s, i * 64, h, c * 128, b);
+            for (int i = 0; i < 3; ++i)
+                tma_load_4d(y + i * 16384, &p.tm_y, bar_y + s, i * 64, h, tb + c * 128, bc);
         };
         int n_qu = 0, n_y[2] = {0, 0};
         if (nchunks > 0) {
@@ -482,9 +499,10 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         // Q~ = scale e^{b} Q (rows in permuted token order)
         if (!mbar_wait(bar_m, mph, ctl)) failed = true;           // scores done: Q, K free
         if (!failed && worker) {
+            const int live = Tn - c * 128;   // varlen: rows past the sequence (the next one's) add nothing
             for (int idx = tid; idx < 384; idx += kWorkers) {
                 const int r = idx & 127, blk = idx >> 7;
-                scale_row_sw64(sm + L::U, r, blk, exp2f(g2 - b2s[r]));
+                scale_row_sw64(sm + L::U, r, blk, (!VARLEN || r < live) ? exp2f(g2 - b2s[r]) : 0.f);
                 if (!fast) scale_row_sw64(sm + L::Q, r, blk, p.scale * exp2f(b2s[row_token(r)]));
             }
         }
@@ -590,7 +608,14 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         if (issuer) pend_m = false;
         mph ^= 1;
         tc_fence_after();
+        // a varlen sequence's last chunk writes its rows itself: a TMA store of
+        // the whole tile would also write the next sequence's rows
+        const bool direct = VARLEN && c * 128 + 128 > Tn;
         if (worker) {
+            const bool mine = VARLEN && tok < Tn - c * 128;
+            uint8_t* orow = VARLEN ? static_cast<uint8_t*>(p.o_direct) +
+                                         ((static_cast<int64_t>(tb) + c * 128 + tok) * p.H + h) * (kDv * 2) + half * 192
+                                   : nullptr;
 #pragma unroll
             for (int j = 0; j < 3; ++j) {
                 uint32_t r[32];
@@ -601,16 +626,20 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
                     const int n = half * 96 + j * 32 + q4 * 8;
-                    *reinterpret_cast<uint4*>(sm + L::X + (n >> 6) * 16384 + swz_off(tok, (n & 63) >> 3, 128)) =
-                        pack8(r + q4 * 8);
+                    if (!direct)
+                        *reinterpret_cast<uint4*>(sm + L::X + (n >> 6) * 16384 + swz_off(tok, (n & 63) >> 3, 128)) =
+                            pack8(r + q4 * 8);
+                    else if (mine)
+                        *reinterpret_cast<uint4*>(orow + (j * 32 + q4 * 8) * 2) = pack8(r + q4 * 8);
                 }
             }
         }
         fence_async_smem();
         tc_fence_before();
         bar_sync(2, 288);
-        if (issuer) {
-            for (int i = 0; i < 3; ++i) tma_store_4d(&p.tm_o, sm + L::X + i * 16384, i * 64, h, c * 128, b);
+        if (issuer && !direct) {
+            for (int i = 0; i < 3; ++i)
+                tma_store_4d(&p.tm_o, sm + L::X + i * 16384, i * 64, h, tb + c * 128, bc);
             tma_store_commit();
         }
         a_cur = a_nx;

@@ -265,6 +265,28 @@ gla_status gla_chunk_fwd(const void* q, const void* k, const void* v, const floa
     return run_chunk_fwd(p, s0, o, s_final, ws, ws_bytes, ctl, stream);
 }
 
+gla_status gla_chunk_fwd_varlen(const void* q, const void* k, const void* v, const float* a,
+                                const int32_t* cu_seqlens, int N, const float* s0, void* o, float* s_final,
+                                int total_T, int H, int dk, int dv, int64_t ld_qkv, float scale, gla_dtype dt,
+                                cudaStream_t stream)
+{
+    if (N < 0 || N > 65535) return N < 0 ? GLA_ERR_INVALID_ARG : GLA_ERR_UNSUPPORTED;
+    int64_t ld_qk = 0, ld_v = 0;
+    gla_status s = validate_chunk(q, k, v, a, 1, total_T, H, dk, dv, ld_qkv, scale, dt, &ld_qk, &ld_v);
+    if (s != GLA_OK) return s;
+    if (dt != GLA_BF16) return GLA_ERR_UNSUPPORTED;
+    if (!aligned16(s0) || !aligned16(s_final)) return GLA_ERR_MISALIGNED;
+    if (N == 0 || H == 0) return GLA_OK;
+    if (!cu_seqlens) return GLA_ERR_INVALID_ARG;
+    if (total_T > 0 && !o) return GLA_ERR_INVALID_ARG;
+    if (!aligned16(o)) return GLA_ERR_MISALIGNED;
+    gla_status se;
+    WaitCtl ctl = wait_ctl_for_current_device(&se);
+    if (se != GLA_OK) return se;
+    ChunkProblem p{q, k, v, a, 1, total_T, H, ld_qk, ld_v, scale};
+    return run_chunk_fwd_varlen(p, cu_seqlens, N, s0, o, s_final, ctl, stream);
+}
+
 gla_status gla_chunk_bwd(const void* q, const void* k, const void* v, const float* a,
                          const float* s0, const void* dO, const float* ds_final,
                          void* grad_q, void* grad_k, void* grad_v, float* grad_a,

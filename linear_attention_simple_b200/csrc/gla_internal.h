@@ -76,6 +76,8 @@ struct ChunkProblem {
 size_t fwd_workspace_bytes(int B, int T, int H);
 size_t bwd_workspace_bytes(int B, int T, int H);
 
+gla_status run_chunk_fwd_varlen(const ChunkProblem& pr, const int* cu_seqlens, int N, const float* s0, void* o,
+                                float* s_final, const WaitCtl& ctl, cudaStream_t st);
 gla_status run_chunk_fwd(const ChunkProblem& p, const float* s0, void* o, float* s_final,
                          void* ws, size_t ws_bytes, const WaitCtl& ctl, cudaStream_t st);
 

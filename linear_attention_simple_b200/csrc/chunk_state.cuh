@@ -106,9 +106,9 @@ struct FusedSmem {
     static constexpr uint32_t X = 49152;      // state copy hi [3][96][64] SW128; with XL, o staging
     static constexpr uint32_t XL = 86016;     // state copy lo
     static constexpr uint32_t Y0 = 122880;    // v tiles, double buffered
-    static constexpr uint32_t Y1 = 172032;
+    static constexpr uint32_t Y1 = 172032;    // (the o staging of a chunk, once its P V is done)
     static constexpr uint32_t MISC = 221184;
-    static constexpr uint32_t BYTES = MISC + 2048 + 1024;
+    static constexpr uint32_t BYTES = MISC + 3072 + 1024;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t TM_SC = 0, TM_O = 128, TM_S = 320;
 };
@@ -319,14 +319,15 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     const uint32_t sb = smem_u32(sm);
     uint64_t* bar_q = reinterpret_cast<uint64_t*>(sm + L::MISC);
     uint64_t* bar_u = bar_q + 1;
-    uint64_t* bar_y = bar_q + 2;                                 // [2]
-    uint64_t* bar_m = bar_q + 4;                                 // scores; then all of the chunk's MMAs
-    uint64_t* bar_d = bar_q + 5;                                 // O = Q S_prev and the state update
-    uint64_t* bar_f = bar_q + 6;                                 // [2] all of a chunk's MMAs (producer)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_q + 8);
-    float* b2s = reinterpret_cast<float*>(sm + L::MISC + 64);   // [128] by token
-    float* cfac = b2s + 128;                                     // [128] 2^{-b_j}
-    float* wsum = cfac + 128;                                    // [4]
+    uint64_t* bar_y = bar_q + 2;                                 // [2] v tile loaded
+    uint64_t* bar_sc = bar_q + 4;                                // scores done
+    uint64_t* bar_d = bar_q + 5;                                 // O = Q S_prev and the state update done
+    uint64_t* bar_fo = bar_q + 6;                                // O += P V done
+    uint64_t* bar_stg = bar_q + 7;                               // [2] o staged in the v buffer (256)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_q + 9);
+    float* b2s = reinterpret_cast<float*>(sm + L::MISC + 128);  // [2][128] by token, chunk parity
+    float* cfac = b2s + 256;                                     // [2][128] 2^{-b_j}
+    float* wsum = cfac + 256;                                    // [4]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -356,7 +357,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     const bool worker = warp < 8;
     const bool srow = worker && quad < 3;
     const bool issuer = warp == 8 && lane == 0;
-    const bool producer = warp == 9 && lane == 0;   // TMA loads; outside the loop's named barrier
+    const bool producer = warp == 9 && lane == 0;   // TMA loads and o stores; outside the loop's barriers
     // largest token among this lane quarter's rows (columns beyond it are masked)
     const int quad_max_tok = max(perm16(2 * quad), perm16(2 * quad + 1)) * 16 + 15;
 
@@ -365,10 +366,11 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         mbar_init(bar_u, 1);
         mbar_init(bar_y, 1);
         mbar_init(bar_y + 1, 1);
-        mbar_init(bar_m, 1);
+        mbar_init(bar_sc, 1);
         mbar_init(bar_d, 1);
-        mbar_init(bar_f, 1);
-        mbar_init(bar_f + 1, 1);
+        mbar_init(bar_fo, 1);
+        mbar_init(bar_stg, kWorkers);
+        mbar_init(bar_stg + 1, kWorkers);
         mbar_init_fence();
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_u);
@@ -389,13 +391,18 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         const int t = c * 128 + tid;
         return t < Tn ? p.a[(static_cast<int64_t>(bc) * p.T + tb + t) * p.H + h] : 0.f;
     };
-    // per barrier at most one phase is ever outstanding
-    uint32_t ph_q = 0, ph_u = 0, ph_y[2] = {0u, 0u}, mph = 0;
-    bool pend_m = false;
-    int n_d = 0, n_f[2] = {0, 0};   // commits issued to bar_d and bar_f[]
+    // cumulative log2-decay of a chunk and its column factors (warps 0-3)
+    auto decays = [&](float av, int par) {
+        if (tid < 128) {
+            const float x = chunk_cumsum(av, wsum, warp, lane);
+            b2s[par * 128 + tid] = x;
+            cfac[par * 128 + tid] = exp2f(-x);
+        }
+    };
 
-    float a_cur = (tid < 128 && nchunks > 0) ? load_a(c_begin) : 0.f;
+    // prologue: decays and state copy of the first chunk
     float a_nx = (tid < 128 && nchunks > 1) ? load_a(c_begin + 1) : 0.f;
+    if (nchunks > 0) decays(tid < 128 ? load_a(c_begin) : 0.f, 0);
     if (srow) {
         const float* src = p.s_init ? p.s_init + unit * p.init_unit_stride + seg * p.init_seg_stride +
                                           row * kDv + half * 96
@@ -405,11 +412,18 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (nchunks > 0 && srow)
+        state_copy_and_decay<true>(tq + L::TM_S + half * 96, row, half, exp2f(b2s[127]), sm + L::X, sm + L::XL,
+                                   true);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
     if (producer) {
         // ----------------------------------------------------------- producer
-        // q, k of chunk it+1 once (D) of chunk it is done; v of chunk it+2
-        // into the buffer chunk it used once all of chunk it's MMAs are done
+        // q, k of chunk it+1 once (D) of chunk it is done; the o tile of chunk
+        // it from its v buffer once staged, then v of chunk it+2 into it
         auto issue_qu = [&](int c) {
             const int t0 = c * 128;
             mbar_arrive_expect_tx(bar_q, kTileQK);
@@ -437,16 +451,28 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                 ++n_y[1];
             }
         }
-        for (int it = 0; it + 1 < nchunks; ++it) {
-            if (!mbar_wait(bar_d, it & 1, ctl)) break;
-            issue_qu(c_begin + it + 1);
-            ++n_qu;
+        for (int it = 0; it < nchunks; ++it) {
+            const int c = c_begin + it, ys = it & 1;
+            if (it + 1 < nchunks) {
+                if (!mbar_wait(bar_d, it & 1, ctl)) break;
+                issue_qu(c + 1);
+                ++n_qu;
+            }
+            if (!mbar_wait(bar_stg + ys, (it >> 1) & 1, ctl)) break;
+            const bool direct = VARLEN && c * 128 + 128 > Tn;
+            if (!direct) {
+                uint8_t* y = sm + (ys ? L::Y1 : L::Y0);
+                for (int i = 0; i < 3; ++i) tma_store_4d(&p.tm_o, y + i * 16384, i * 64, h, tb + c * 128, bc);
+                tma_store_commit();
+            }
             if (it + 2 < nchunks) {
-                if (!mbar_wait(bar_f + (it & 1), (it >> 1) & 1, ctl)) break;
-                issue_y(c_begin + it + 2, it & 1);
-                ++n_y[it & 1];
+                tma_store_wait_read();
+                issue_y(c + 2, ys);
+                ++n_y[ys];
             }
         }
+        tma_store_wait_all();
+        // at most one load per barrier is ever outstanding
         if (n_qu) {
             mbar_wait(bar_q, (n_qu - 1) & 1, ctl);
             mbar_wait(bar_u, (n_qu - 1) & 1, ctl);
@@ -455,20 +481,22 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             if (n_y[i]) mbar_wait(bar_y + i, (n_y[i] - 1) & 1, ctl);
     }
 
+    // -------------------------------------------------- workers and issuer
+    uint32_t ph_q = 0, ph_u = 0, ph_y[2] = {0u, 0u};
+    int n_sc = 0, n_d = 0, n_fo = 0;          // commits (issuer)
     bool failed = false, aborted = false;
     for (int it = 0; warp < 9 && it < nchunks; ++it) {
         const int c = c_begin + it;
-        const int ys = it & 1;
+        const int ys = it & 1, par = it & 1;
         const uint32_t ya = ys ? L::Y1 : L::Y0;
+        const float* b2c = b2s + par * 128;
+        const float* cfc = cfac + par * 128;
 
-        // (A) cumulative decay (warps 0-3) and column factors; scores MMA
-        if (tid < 128) {
-            const float x = chunk_cumsum(a_cur, wsum, warp, lane);
-            b2s[tid] = x;
-            cfac[tid] = exp2f(-x);
-        }
+        // (A) scores, once q and k are in and the last chunk's P V (which reads
+        // its P from the scores columns) is done
         if (issuer) {
-            if (mbar_wait(bar_q, ph_q, ctl) && mbar_wait(bar_u, ph_u, ctl)) {
+            if (mbar_wait(bar_q, ph_q, ctl) && mbar_wait(bar_u, ph_u, ctl) &&
+                (it == 0 || mbar_wait(bar_fo, (it - 1) & 1, ctl))) {
                 ph_q ^= 1;
                 ph_u ^= 1;
                 tc_fence_after();
@@ -479,39 +507,30 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                     const uint32_t off = (ks >> 1) * 8192 + (ks & 1) * 32;
                     umma_bf16(tmem + L::TM_SC, desc_add(dq, off), desc_add(du, off), kIdScores, ks > 0);
                 }
-                umma_commit(bar_m);
-                pend_m = true;
+                umma_commit(bar_sc);
+                ++n_sc;
             } else {
                 failed = true;
             }
-            tma_store_wait_read();   // the previous chunk's o staging (X, XL) is free
         }
-        if (bar_or(2, 288, failed)) { aborted = true; break; }
-        const float g2 = b2s[127];
+        const float g2 = b2c[127];
         const bool fast = -g2 <= kFactorRange;   // uniform: the factorised path is safe
-
-        // (B) state copy (bf16 hi + lo, the B operand of O = Q S_prev), decay
-        if (srow)
-            state_copy_and_decay<true>(tq + L::TM_S + half * 96, row, half, exp2f(g2), sm + L::X,
-                                       sm + L::XL, true);
 
         // (C) K~ = e^{gamma - b} K in place; on the exact path also
         // Q~ = scale e^{b} Q (rows in permuted token order)
-        if (!mbar_wait(bar_m, mph, ctl)) failed = true;           // scores done: Q, K free
+        if (worker && !failed && !mbar_wait(bar_sc, it & 1, ctl)) failed = true;
         if (!failed && worker) {
             const int live = Tn - c * 128;   // varlen: rows past the sequence (the next one's) add nothing
             for (int idx = tid; idx < 384; idx += kWorkers) {
                 const int r = idx & 127, blk = idx >> 7;
-                scale_row_sw64(sm + L::U, r, blk, (!VARLEN || r < live) ? exp2f(g2 - b2s[r]) : 0.f);
-                if (!fast) scale_row_sw64(sm + L::Q, r, blk, p.scale * exp2f(b2s[row_token(r)]));
+                scale_row_sw64(sm + L::U, r, blk, (!VARLEN || r < live) ? exp2f(g2 - b2c[r]) : 0.f);
+                if (!fast) scale_row_sw64(sm + L::Q, r, blk, p.scale * exp2f(b2c[row_token(r)]));
             }
         }
         fence_async_smem();
         tc_fence_before();
         if (bar_or(2, 288, failed)) { aborted = true; break; }
         tc_fence_after();
-        if (issuer) pend_m = false;
-        mph ^= 1;
 
         // (D) O = Q S_prev (hi, lo), S += K~^T V
         if (issuer) {
@@ -540,11 +559,9 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
 
         // (E) scores -> P (hi, lo) in place in tensor memory: lane = row i,
         // 32-token block kb holds hi in columns 32 kb .. +15 and lo in +16 .. +31.
-        // The epilogue's row factor is read here, before the next chunk's decays
-        // overwrite b2s.
         float rf = 1.0f;
         if (worker) {
-            const float b2r = b2s[tok];
+            const float b2r = b2c[tok];
             if (fast) rf = p.scale * exp2f(b2r);
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
@@ -563,11 +580,11 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                         const int j = j0 + e;
                         float v0, v1;
                         if (fast) {
-                            v0 = (j <= tok) ? __uint_as_float(r[e]) * cfac[j] : 0.f;
-                            v1 = (j + 1 <= tok) ? __uint_as_float(r[e + 1]) * cfac[j + 1] : 0.f;
+                            v0 = (j <= tok) ? __uint_as_float(r[e]) * cfc[j] : 0.f;
+                            v1 = (j + 1 <= tok) ? __uint_as_float(r[e + 1]) * cfc[j + 1] : 0.f;
                         } else {
-                            v0 = (j <= tok) ? p.scale * __uint_as_float(r[e]) * exp2f(b2r - b2s[j]) : 0.f;
-                            v1 = (j + 1 <= tok) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2r - b2s[j + 1]) : 0.f;
+                            v0 = (j <= tok) ? p.scale * __uint_as_float(r[e]) * exp2f(b2r - b2c[j]) : 0.f;
+                            v1 = (j + 1 <= tok) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2r - b2c[j + 1]) : 0.f;
                         }
                         const uint32_t hv = pack_bf16(v0, v1);
                         hi[e / 2] = hv;
@@ -582,9 +599,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         tc_fence_before();
         if (bar_or(2, 288, failed)) { aborted = true; break; }
 
-        // (F) O += P V with P from tensor memory; once (D) is done, q and k
-        // of the next chunk may load
-        float a_next = 0.f;
+        // (F) O += P V with P from tensor memory
         if (issuer) {
             tc_fence_after();
             const uint64_t dy = smem_desc(sb + ya, 16384, 1024, kLayoutSW128);
@@ -594,74 +609,76 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                 for (int ks = 0; ks < 8; ++ks)
                     umma_bf16_ts(tmem + L::TM_O, tmem + L::TM_SC + 32 * (ks >> 1) + 8 * (ks & 1) + 16 * part,
                                  desc_add(dy, ks * 2048), kIdOutTs, 1);
-            umma_commit(bar_m);
-            umma_commit(bar_f + ys);
-            pend_m = true;
-            ++n_f[ys];
+            umma_commit(bar_fo);
+            ++n_fo;
         }
-        if (tid < 128 && it + 2 < nchunks) a_next = load_a(c + 2);
+        const float a_next = (tid < 128 && it + 2 < nchunks) ? load_a(c + 2) : 0.f;
 
-        // (G) epilogue: o = r_i O_i -> bf16 staging in X, XL (token order,
-        // [3][128][64] SW128; the state copies are dead once (D) is done) -> TMA store
-        if (!mbar_wait(bar_m, mph, ctl)) failed = true;
-        if (bar_or(2, 288, failed)) { aborted = true; break; }
-        if (issuer) pend_m = false;
-        mph ^= 1;
-        tc_fence_after();
-        // a varlen sequence's last chunk writes its rows itself: a TMA store of
-        // the whole tile would also write the next sequence's rows
-        const bool direct = VARLEN && c * 128 + 128 > Tn;
+        // (B) while P V runs: the next chunk's decays, then -- once (D) has
+        // updated S and released the state copies -- its state copy and decay
+        if (worker && it + 1 < nchunks) {
+            decays(a_nx, par ^ 1);
+            named_sync(3, kWorkers);             // the next chunk's total decay is in b2s
+            if (!failed && !mbar_wait(bar_d, it & 1, ctl)) failed = true;
+            tc_fence_after();
+            if (srow && !failed)
+                state_copy_and_decay<true>(tq + L::TM_S + half * 96, row, half, exp2f(b2s[(par ^ 1) * 128 + 127]),
+                                           sm + L::X, sm + L::XL, true);
+            fence_async_smem();
+        }
+
+        // (G) epilogue: o = r_i O_i -> bf16 staging in this chunk's v buffer
+        // (token order, [3][128][64] SW128) -> the producer's TMA store; a
+        // varlen sequence's last chunk writes its rows itself
         if (worker) {
+            if (!failed && !mbar_wait(bar_fo, it & 1, ctl)) failed = true;
+            tc_fence_after();
+            const bool direct = VARLEN && c * 128 + 128 > Tn;
             const bool mine = VARLEN && tok < Tn - c * 128;
             uint8_t* orow = VARLEN ? static_cast<uint8_t*>(p.o_direct) +
                                          ((static_cast<int64_t>(tb) + c * 128 + tok) * p.H + h) * (kDv * 2) + half * 192
                                    : nullptr;
+            if (!failed) {
+                uint8_t* stg = sm + ya;
 #pragma unroll
-            for (int j = 0; j < 3; ++j) {
-                uint32_t r[32];
-                tmem_ld32(tq + L::TM_O + half * 96 + j * 32, r);
-                tmem_ld_wait();
+                for (int j = 0; j < 3; ++j) {
+                    uint32_t r[32];
+                    tmem_ld32(tq + L::TM_O + half * 96 + j * 32, r);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * rf);
+                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * rf);
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int n = half * 96 + j * 32 + q4 * 8;
-                    if (!direct)
-                        *reinterpret_cast<uint4*>(sm + L::X + (n >> 6) * 16384 + swz_off(tok, (n & 63) >> 3, 128)) =
-                            pack8(r + q4 * 8);
-                    else if (mine)
-                        *reinterpret_cast<uint4*>(orow + (j * 32 + q4 * 8) * 2) = pack8(r + q4 * 8);
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int n = half * 96 + j * 32 + q4 * 8;
+                        if (!direct)
+                            *reinterpret_cast<uint4*>(stg + (n >> 6) * 16384 + swz_off(tok, (n & 63) >> 3, 128)) =
+                                pack8(r + q4 * 8);
+                        else if (mine)
+                            *reinterpret_cast<uint4*>(orow + (j * 32 + q4 * 8) * 2) = pack8(r + q4 * 8);
+                    }
                 }
+                fence_async_smem();
+                mbar_arrive(bar_stg + ys);
             }
         }
-        fence_async_smem();
         tc_fence_before();
-        bar_sync(2, 288);
-        if (issuer && !direct) {
-            for (int i = 0; i < 3; ++i)
-                tma_store_4d(&p.tm_o, sm + L::X + i * 16384, i * 64, h, tb + c * 128, bc);
-            tma_store_commit();
-        }
-        a_cur = a_nx;
         a_nx = a_next;
     }
 
-    if (!aborted) {
+    if (!aborted && warp < 9) {
+        // all MMAs are done (the epilogue waited for the last P V): S is final
         const bool write_state = p.s_out && (!p.out_last_only || seg == static_cast<int>(gridDim.x) - 1);
-        if (write_state && srow)
+        if (write_state && srow && !failed)
             tmem_to_state(tq + L::TM_S + half * 96,
                           p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + half * 96);
-    } else if (issuer && pend_m) {
-        mbar_wait(bar_m, mph, ctl);
     }
     if (issuer) {
         // every commit's arrival has landed before the barriers go away: at
         // most one phase of each is outstanding, so wait for the last one
+        if (n_sc) mbar_wait(bar_sc, (n_sc - 1) & 1, ctl);
         if (n_d) mbar_wait(bar_d, (n_d - 1) & 1, ctl);
-        for (int i = 0; i < 2; ++i)
-            if (n_f[i]) mbar_wait(bar_f + i, (n_f[i] - 1) & 1, ctl);
+        if (n_fo) mbar_wait(bar_fo, (n_fo - 1) & 1, ctl);
     }
-    if (issuer) tma_store_wait_all();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, L::TMEM_COLS);

@@ -194,10 +194,11 @@ def barrier(ws):
         torch.distributed.barrier()
 
 
-def max_over_ranks(x, ws):
+def max_over_ranks(x, ws, device="cuda"):
+    """x maximised over all ranks (every rank gets the result)."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 

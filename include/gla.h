@@ -169,6 +169,60 @@ gla_status gla_chunk_bwd(const void* q, const void* k, const void* v, const floa
                          int dv, int64_t ld_qkv, float scale, gla_dtype dt, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Sequence split across ranks (long documents, "Como i14 ...", section "Por
+ * qué atención lineal importa": cost linear in T with a fixed-size state).
+ * A sequence cut into R consecutive segments, one per rank, is exact in
+ * three steps, because the state is linear in its inputs (section
+ * "Adaptaciones para AWS Trainium2", item 1: chunking only regroups the
+ * recurrence):
+ *   1. each rank: gla_segment_state_fwd on its own tokens -> (L_r, G_r), and
+ *      for the backward also gla_segment_state_bwd -> D_r;
+ *   2. exchange (an all_gather of those B*H*(dk*dv + 1) floats per rank);
+ *   3. each rank: gla_state_fold to get the state entering its segment
+ *      (entries 0 .. r-1, in order, from S_0) and, for the backward, the
+ *      state gradient at its end (entries r+1 .. R-1, right to left, from
+ *      dS_T); then gla_chunk_fwd / gla_chunk_bwd on its tokens with those
+ *      as s0 / ds_final.
+ *
+ * gla_segment_state_fwd: for every (b, h) of a segment of T tokens,
+ *     s_seg = sum_t exp(A_{T-1} - A_t) k_t^T v_t   (the end state from zero)
+ *     g_seg = A_{T-1} = sum_t a_t                  (natural log)
+ *   k [B,T,H,dk], v [B,T,H,dv] bf16 with token stride ld_qkv as in
+ *   gla_chunk_fwd; a [B,T,H] fp32; s_seg [B,H,dk,dv] fp32 (required);
+ *   g_seg [B,H] fp32 (NULL to skip).
+ * gla_segment_state_bwd: with zero state gradient at the segment's end,
+ *     ds_seg = dL/dS entering the segment
+ *            = sum_t scale exp(A_t) q_t^T dO_t     (A_t inclusive of a_t)
+ *   q [B,T,H,dk] bf16 (token stride ld_qkv); dO [B,T,H,dv] bf16 contiguous;
+ *   ds_seg [B,H,dk,dv] fp32 (required); g_seg as above.
+ * Both: dt must be GLA_BF16; ws_bytes >= gla_segment_workspace_bytes(B,T,H,
+ * dk,dv) (a scratch of per-sub-segment states; contents do not matter).
+ * T == 0 gives zeros.
+ *
+ * gla_state_fold: out = x after x <- exp(g[j]) x + s[j] for j = 0 .. n-1
+ * (j = n-1 .. 0 when reverse != 0), starting from x = s_in (zeros if NULL).
+ *   s [n][units][dk][dv] fp32, g [n][units] fp32 (natural log), s_in and
+ *   out [units][dk][dv] fp32; out may be s_in.  n == 0 copies s_in (or
+ *   zeros) to out.  units = B*H.
+ * All pointers are device memory, 16-byte aligned except g (4 bytes, so
+ * that g may start at any entry of a gathered array); every call is
+ * asynchronous on `stream`.
+ * ------------------------------------------------------------------------ */
+size_t gla_segment_workspace_bytes(int B, int T, int H, int dk, int dv);
+
+gla_status gla_segment_state_fwd(const void* k, const void* v, const float* a, float* s_seg,
+                                 float* g_seg, void* ws, size_t ws_bytes, int B, int T, int H,
+                                 int dk, int dv, int64_t ld_qkv, gla_dtype dt, cudaStream_t stream);
+
+gla_status gla_segment_state_bwd(const void* q, const void* dO, const float* a, float* ds_seg,
+                                 float* g_seg, void* ws, size_t ws_bytes, int B, int T, int H,
+                                 int dk, int dv, int64_t ld_qkv, float scale, gla_dtype dt,
+                                 cudaStream_t stream);
+
+gla_status gla_state_fold(const float* s, const float* g, int n, int reverse, const float* s_in,
+                          float* out, int units, int dk, int dv, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * One decode step for N sequences (the fixed per-sequence state of "AWS serve
  * Laplace 3B ...", section "Lo stato di Laplace 3B resta fisso durante
  * l'inferenza"; 1,280 concurrent sequences in "Como i14 ...", section

@@ -20,7 +20,8 @@ __all__ = [
     "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
     "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step", "conv1d_silu_causal_bwd",
-    "conv1d_silu_causal_bwd_workspace_bytes", "gla_chunk_fwd_varlen", "EXPORTED_SYMBOLS", "LIB_PATH",
+    "conv1d_silu_causal_bwd_workspace_bytes", "gla_chunk_fwd_varlen", "gla_segment_workspace_bytes",
+    "gla_segment_state_fwd", "gla_segment_state_bwd", "gla_state_fold", "EXPORTED_SYMBOLS", "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgla.so")
@@ -31,7 +32,8 @@ EXPORTED_SYMBOLS = (
     "conv1d_silu_causal", "gla_get_device_status", "gla_set_wait_limit_ns",
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
     "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step", "conv1d_silu_causal_bwd",
-    "conv1d_silu_causal_bwd_workspace_bytes", "gla_chunk_fwd_varlen",
+    "conv1d_silu_causal_bwd_workspace_bytes", "gla_chunk_fwd_varlen", "gla_segment_workspace_bytes",
+    "gla_segment_state_fwd", "gla_segment_state_bwd", "gla_state_fold",
 )
 
 GLA_BF16, GLA_F32 = 0, 1
@@ -94,6 +96,16 @@ def lib():
     L.gla_chunk_fwd_varlen.restype = _i
     L.gla_chunk_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i,
                                        ctypes.c_longlong, _f, _i, _vp]
+    L.gla_segment_workspace_bytes.restype = ctypes.c_size_t
+    L.gla_segment_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+    L.gla_segment_state_fwd.restype = _i
+    L.gla_segment_state_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _i, _i, _i, _i, _i,
+                                        _i64, _i, _vp]
+    L.gla_segment_state_bwd.restype = _i
+    L.gla_segment_state_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _i, _i, _i, _i, _i,
+                                        _i64, _f, _i, _vp]
+    L.gla_state_fold.restype = _i
+    L.gla_state_fold.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _i, _i, _i, _vp]
     L.conv1d_silu_decode_step.restype = _i
     L.conv1d_silu_decode_step.argtypes = [_vp, _vp, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]
     L.gla_get_device_status.restype = _i
@@ -336,6 +348,100 @@ def gla_chunk_fwd_varlen(q, k, v, a, cu_seqlens, s0=None, o=None, s_final=None, 
                                     _ptr(s_final), total, H, dk, dv, 0, float(sc), GLA_BF16, _stream(stream))
     _check("gla_chunk_fwd_varlen", st)
     return o, s_final
+
+
+def gla_segment_workspace_bytes(B, T, H, dk=96, dv=192):
+    return int(lib().gla_segment_workspace_bytes(B, T, H, dk, dv))
+
+
+def _segment_outputs(B, H, dk, dv, dev, s_seg, g_seg, want_g):
+    if s_seg is None:
+        s_seg = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    _need(s_seg, "s_seg", torch.float32, (B, H, dk, dv))
+    if g_seg is None and want_g:
+        g_seg = torch.empty((B, H), dtype=torch.float32, device=dev)
+    _need(g_seg, "g_seg", torch.float32, (B, H))
+    return s_seg, g_seg
+
+
+def _segment_ws(ws, B, T, H, dk, dv, dev):
+    need = gla_segment_workspace_bytes(B, T, H, dk, dv)
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    return ws
+
+
+def gla_segment_state_fwd(k, v, a, s_seg=None, g_seg=None, ws=None, want_decay=True, stream=None):
+    """State a segment of tokens leaves from a zero start, and its total
+    log-decay.  k [B,T,H,96], v [B,T,H,192] bf16; a [B,T,H] fp32.  Returns
+    (s_seg [B,H,96,192] fp32, g_seg [B,H] fp32 or None)."""
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    if k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("gla_segment_state_fwd takes bf16 k and v")
+    lk = _token_stride(k, B, T, H, dk)
+    lv = _token_stride(v, B, T, H, dv)
+    if lk == H * dk and lv == H * dv:
+        ld = 0
+    elif lk == lv:
+        ld = lk
+    else:
+        raise ValueError("k and v must share one token stride when not packed (got %d, %d)" % (lk, lv))
+    _need(a, "a", torch.float32, (B, T, H))
+    s_seg, g_seg = _segment_outputs(B, H, dk, dv, k.device, s_seg, g_seg, want_decay)
+    ws = _segment_ws(ws, B, T, H, dk, dv, k.device)
+    st = lib().gla_segment_state_fwd(_ptr(k), _ptr(v), _ptr(a), _ptr(s_seg), _ptr(g_seg), _ptr(ws),
+                                     0 if ws is None else ws.numel(), B, T, H, dk, dv, ld, GLA_BF16,
+                                     _stream(stream))
+    _check("gla_segment_state_fwd", st)
+    return s_seg, g_seg
+
+
+def gla_segment_state_bwd(q, dO, a, ds_seg=None, g_seg=None, ws=None, scale=None, want_decay=False,
+                          stream=None):
+    """Gradient of the state entering a segment from the segment's own
+    outputs (zero gradient at its end), and optionally its total log-decay.
+    q [B,T,H,96] bf16 (packed heads; any token stride), dO [B,T,H,192] bf16
+    contiguous; a [B,T,H] fp32.  Returns (ds_seg [B,H,96,192], g_seg or None)."""
+    B, T, H, dk = q.shape
+    dv = dO.shape[-1]
+    if q.dtype != torch.bfloat16:
+        raise TypeError("gla_segment_state_bwd takes bf16 q and dO")
+    lq = _token_stride(q, B, T, H, dk)
+    if lq != H * dk and lq < H * dv:
+        raise ValueError("an unpacked q needs a token stride >= H*dv (got %d)" % lq)
+    _need(dO, "dO", torch.bfloat16, (B, T, H, dv))
+    _need(a, "a", torch.float32, (B, T, H))
+    ds_seg, g_seg = _segment_outputs(B, H, dk, dv, q.device, ds_seg, g_seg, want_decay)
+    ws = _segment_ws(ws, B, T, H, dk, dv, q.device)
+    sc = dk ** -0.5 if scale is None else scale
+    st = lib().gla_segment_state_bwd(_ptr(q), _ptr(dO), _ptr(a), _ptr(ds_seg), _ptr(g_seg), _ptr(ws),
+                                     0 if ws is None else ws.numel(), B, T, H, dk, dv,
+                                     0 if lq == H * dk else lq, float(sc), GLA_BF16, _stream(stream))
+    _check("gla_segment_state_bwd", st)
+    return ds_seg, g_seg
+
+
+def gla_state_fold(s, g, reverse=False, s_in=None, out=None, stream=None):
+    """x <- exp(g[j]) x + s[j] over j = 0..n-1 (n-1..0 if reverse) from
+    x = s_in (zeros if None).  s [n, *U, 96, 192] fp32, g [n, *U] fp32 with U
+    the unit dims (e.g. B, H); s_in / out [*U, 96, 192].  Returns out."""
+    n = s.shape[0]
+    unit_shape = tuple(s.shape[1:-2])
+    dk, dv = s.shape[-2], s.shape[-1]
+    units = 1
+    for x in unit_shape:
+        units *= x
+    _need(s, "s", torch.float32)
+    _need(g, "g", torch.float32, (n,) + unit_shape)
+    _need(s_in, "s_in", torch.float32, unit_shape + (dk, dv))
+    if out is None:
+        out = torch.empty(unit_shape + (dk, dv), dtype=torch.float32, device=s.device)
+    _need(out, "out", torch.float32, unit_shape + (dk, dv))
+    st = lib().gla_state_fold(_ptr(s), _ptr(g), n, 1 if reverse else 0, _ptr(s_in), _ptr(out), units, dk, dv,
+                              _stream(stream))
+    _check("gla_state_fold", st)
+    return out
 
 
 def conv1d_silu_causal_bwd_workspace_bytes(B, T, D, W=4):

@@ -36,27 +36,46 @@ void segment_plan(int units, int NC, int* nseg, int* cps)
     *nseg = (NC + c - 1) / c;
 }
 
+// States entering every segment, in place: slot g holds L_g (the local end
+// state of segment g from zero) on entry and S_g on return.  The loads of a
+// batch of segments are issued before the dependent chain that uses them.
 __global__ void __launch_bounds__(256) seg_combine_kernel(float* __restrict__ states,
                                                           const float* __restrict__ g2,
                                                           const float* __restrict__ s0, int nseg,
                                                           int units)
 {
+    constexpr int kBatch = 8;
     const int64_t n4 = kSS / 4;
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= n4 * units) return;
     const int64_t unit = idx / n4, e4 = idx - unit * n4;
     float4* st = reinterpret_cast<float4*>(states);
     float4 x = s0 ? reinterpret_cast<const float4*>(s0)[unit * n4 + e4] : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int g = 0; g < nseg; ++g) {
-        float4* slot = st + (unit * nseg + g) * n4 + e4;
-        const float4 l = (g < nseg - 1) ? *slot : make_float4(0.f, 0.f, 0.f, 0.f);
-        *slot = x;
-        if (g < nseg - 1) {
-            const float f = exp2f(g2[unit * nseg + g]);
-            x.x = fmaf(f, x.x, l.x);
-            x.y = fmaf(f, x.y, l.y);
-            x.z = fmaf(f, x.z, l.z);
-            x.w = fmaf(f, x.w, l.w);
+    for (int g0 = 0; g0 < nseg; g0 += kBatch) {
+        float4 l[kBatch];
+        float f[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int g = g0 + u;
+            // the last segment's slot only receives its entering state
+            if (g < nseg - 1) {
+                l[u] = st[(unit * nseg + g) * n4 + e4];
+                f[u] = g2[unit * nseg + g];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int g = g0 + u;
+            if (g < nseg) {
+                st[(unit * nseg + g) * n4 + e4] = x;
+                if (g < nseg - 1) {
+                    const float e = exp2f(f[u]);
+                    x.x = fmaf(e, x.x, l[u].x);
+                    x.y = fmaf(e, x.y, l[u].y);
+                    x.z = fmaf(e, x.z, l[u].z);
+                    x.w = fmaf(e, x.w, l[u].w);
+                }
+            }
         }
     }
 }

@@ -324,6 +324,81 @@ gla_status gla_chunk_bwd(const void* q, const void* k, const void* v, const floa
                          ws_bytes, ctl, stream);
 }
 
+size_t gla_segment_workspace_bytes(int B, int T, int H, int dk, int dv)
+{
+    if (B <= 0 || T <= 0 || H <= 0 || dk != kDk || dv != kDv) return 0;
+    return segment_workspace_bytes(B, T, H);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Shared by gla_segment_state_fwd / _bwd: u = k or q (dk wide, token stride
+// ld_u), y = v or dO (dv wide, token stride ld_y).
+gla_status segment_state(const void* u, const void* y, const float* a, float* s_seg, float* g_seg, void* ws,
+                         size_t ws_bytes, int B, int T, int H, int dk, int dv, int64_t ld_u, int64_t ld_y,
+                         float scale, bool reverse, cudaStream_t stream)
+{
+    if (static_cast<int64_t>(B) * H == 0) return GLA_OK;
+    if (!s_seg) return GLA_ERR_INVALID_ARG;
+    if (!aligned16(s_seg) || !aligned16(g_seg) || !aligned16(ws)) return GLA_ERR_MISALIGNED;
+    if (T == 0) {
+        // an empty segment contributes nothing and does not decay
+        cudaError_t e = cudaMemsetAsync(s_seg, 0, static_cast<size_t>(B) * H * dk * dv * sizeof(float), stream);
+        if (e == cudaSuccess && g_seg) e = cudaMemsetAsync(g_seg, 0, static_cast<size_t>(B) * H * sizeof(float), stream);
+        return e == cudaSuccess ? GLA_OK : cuda_fail(e);
+    }
+    if (!ws || ws_bytes < segment_workspace_bytes(B, T, H)) return GLA_ERR_INVALID_ARG;
+    gla_status se;
+    WaitCtl ctl = wait_ctl_for_current_device(&se);
+    if (se != GLA_OK) return se;
+    return run_segment_state(u, y, a, B, T, H, ld_u, ld_y, scale, reverse, s_seg, g_seg, ws, ctl, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+gla_status gla_segment_state_fwd(const void* k, const void* v, const float* a, float* s_seg, float* g_seg,
+                                 void* ws, size_t ws_bytes, int B, int T, int H, int dk, int dv, int64_t ld_qkv,
+                                 gla_dtype dt, cudaStream_t stream)
+{
+    int64_t ld_qk = 0, ld_v = 0;
+    // q is not read: k stands in for it in the shared validation
+    gla_status s = validate_chunk(k, k, v, a, B, T, H, dk, dv, ld_qkv, 1.0f, dt, &ld_qk, &ld_v);
+    if (s != GLA_OK) return s;
+    if (dt != GLA_BF16) return GLA_ERR_UNSUPPORTED;
+    return segment_state(k, v, a, s_seg, g_seg, ws, ws_bytes, B, T, H, dk, dv, ld_qk, ld_v, 1.0f, false, stream);
+}
+
+gla_status gla_segment_state_bwd(const void* q, const void* dO, const float* a, float* ds_seg, float* g_seg,
+                                 void* ws, size_t ws_bytes, int B, int T, int H, int dk, int dv, int64_t ld_qkv,
+                                 float scale, gla_dtype dt, cudaStream_t stream)
+{
+    int64_t ld_qk = 0, ld_v = 0;
+    // dO is contiguous; the shared validation checks it in v's place, and its
+    // stride is the packed H*dv whatever ld_qkv is
+    gla_status s = validate_chunk(q, q, dO, a, B, T, H, dk, dv, ld_qkv, scale, dt, &ld_qk, &ld_v);
+    if (s != GLA_OK) return s;
+    if (dt != GLA_BF16) return GLA_ERR_UNSUPPORTED;
+    return segment_state(q, dO, a, ds_seg, g_seg, ws, ws_bytes, B, T, H, dk, dv, ld_qk,
+                         static_cast<int64_t>(H) * dv, scale, true, stream);
+}
+
+gla_status gla_state_fold(const float* s, const float* g, int n, int reverse, const float* s_in, float* out,
+                          int units, int dk, int dv, cudaStream_t stream)
+{
+    if (n < 0 || units < 0 || dk <= 0 || dv <= 0) return GLA_ERR_INVALID_ARG;
+    if (dk != kDk || dv != kDv) return GLA_ERR_UNSUPPORTED;
+    if (units == 0) return GLA_OK;
+    if (!out || (n > 0 && (!s || !g))) return GLA_ERR_INVALID_ARG;
+    // g is read one float at a time: 4-byte alignment suffices
+    if (!aligned16(s) || !aligned16(s_in) || !aligned16(out) || (reinterpret_cast<uintptr_t>(g) & 3u))
+        return GLA_ERR_MISALIGNED;
+    return launch_state_fold(s, g, n, units, reverse ? 1 : 0, s_in, out, stream);
+}
+
 gla_status gla_decode_step(float* state, const int32_t* slot_idx, const void* q, const void* k,
                            const void* v, const float* a, float* o, int N, int H, int dk, int dv,
                            float scale, cudaStream_t stream)

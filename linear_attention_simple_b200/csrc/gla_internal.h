@@ -88,6 +88,14 @@ gla_status run_chunk_bwd(const ChunkProblem& p, const float* s0, const void* dO,
 
 gla_status launch_wait_selftest(const WaitCtl& ctl, cudaStream_t st);
 
+// Sequence split across ranks (chunk_seg.cu).
+size_t segment_workspace_bytes(int B, int T, int H);
+gla_status run_segment_state(const void* u, const void* y, const float* a, int B, int T, int H, int64_t ld_u,
+                             int64_t ld_y, float scale, bool reverse, float* s_seg, float* g_seg, void* ws,
+                             const WaitCtl& ctl, cudaStream_t st);
+gla_status launch_state_fold(const float* s, const float* g, int n, int units, int reverse, const float* s_in,
+                             float* out, cudaStream_t st);
+
 // Shared by the forward and backward host code (chunk_fwd.cu).
 struct StateParams;   // chunk_state.cuh
 gla_status make_token_map(CUtensorMap* m, const void* base, int d, int H, int T, int B,

@@ -23,7 +23,8 @@
 //      as bf16 hi + lo and feed the next MMA from there; the epilogues also
 //      emit q.dq and k.dk per token and per chunk;
 //   4. da_finish_kernel: reverse cumulative sum over T (plus <dS_T, S_T>
-//      from state_dot_kernel when dS_T is given).
+//      from state_dot_kernel when dS_T is given), restarted every 16 chunks
+//      from the closed form <dS_a, S_a> (da_anchor_kernel).
 #include <cstring>
 
 #include "chunk_state.cuh"
@@ -628,23 +629,39 @@ done:
 //
 // da_t = sum_{m >= t} (q_m . dq_m - k_m . dk_m) + <dS_T, S_T>.  One CTA of
 // 128 threads per (chunk, batch x head): the reverse inclusive scan of the
-// chunk's own tokens, plus the totals of every later chunk, plus the state
-// term (dS_T given) that state_dot_kernel wrote per (batch, head).
+// chunk's own tokens, plus the totals of the later chunks up to the next
+// anchor, plus the anchor's value.
+//
+// Anchors.  Each chunk total carries the rounding of the bf16 state copies
+// the gradient kernels read, and a sum over every later chunk would let that
+// error grow like sqrt(T).  The sum over all tokens after chunk a has a
+// closed form, <dS_a, S_a> (the gradient of the state after chunk a with that
+// state: the same identity that gives <dS_T, S_T> for the tokens after T), so
+// every kDaAnchor chunks the sum restarts from that inner product
+// (da_anchor_kernel).  The last anchor is the dS_T term that state_dot_kernel
+// wrote per (batch, head), or zero.
 
 constexpr int kDaThreads = 128;
+constexpr int kDaAnchor = 16;      // chunks between anchors (2,048 tokens)
+
+__host__ __device__ inline int da_anchors(int NC) { return (NC - 1) / kDaAnchor; }
 
 __global__ void __launch_bounds__(kDaThreads) da_finish_kernel(float* __restrict__ da,
                                                                const float* __restrict__ delta,
                                                                const float* __restrict__ ctot,
-                                                               const float* __restrict__ base, int T, int H,
+                                                               const float* __restrict__ base,
+                                                               const float* __restrict__ anchor, int T, int H,
                                                                int NC, int units)
 {
     __shared__ float wtot[kDaThreads / 32], wsuf[kDaThreads / 32];
     const int unit = blockIdx.x, c = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t = c * kChunk + tid;
     const float* cu = ctot + static_cast<int64_t>(unit) * NC * 2;
+    // chunks c+1 .. last are summed; the anchor after `last` closes the sum
+    const int na = da_anchors(NC), j = c / kDaAnchor;
+    const int last = j < na ? (j + 1) * kDaAnchor - 1 : NC - 1;
     float suf = 0.f;
-    for (int cc = c + 1 + tid; cc < NC; cc += kDaThreads) suf += cu[2 * cc] - cu[2 * cc + 1];
+    for (int cc = c + 1 + tid; cc <= last; cc += kDaThreads) suf += cu[2 * cc] - cu[2 * cc + 1];
     float x = 0.f;
     if (t < T) x = delta[static_cast<int64_t>(unit) * T + t] - delta[(static_cast<int64_t>(units) + unit) * T + t];
 #pragma unroll
@@ -658,7 +675,7 @@ __global__ void __launch_bounds__(kDaThreads) da_finish_kernel(float* __restrict
         wsuf[warp] = suf;
     }
     __syncthreads();
-    float add = base ? base[unit] : 0.f;
+    float add = j < na ? anchor[static_cast<int64_t>(unit) * na + j] : (base ? base[unit] : 0.f);
     for (int w = 0; w < kDaThreads / 32; ++w) {
         add += wsuf[w];
         if (w > warp) add += wtot[w];
@@ -666,28 +683,82 @@ __global__ void __launch_bounds__(kDaThreads) da_finish_kernel(float* __restrict
     if (t < T) da[(static_cast<int64_t>(unit / H) * T + t) * H + unit % H] = x + add;
 }
 
-// <dS_T, S_T> per (batch, head), one CTA each.
-__global__ void __launch_bounds__(256) state_dot_kernel(float* __restrict__ out, const float* __restrict__ dsT,
-                                                        const float* __restrict__ sT)
+// Both inner products below are a few hundred KB per CTA at most, read by
+// 1,024 threads whose loads are all issued before the FMAs that use them, so
+// each thread waits about once instead of once per vector.
+constexpr int kDotThreads = 1024;
+
+__device__ __forceinline__ float block_sum_dot(float s, float* red)
 {
-    __shared__ float red[8];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+    __syncthreads();
+    float r = 0.f;
+    if (threadIdx.x == 0)
+        for (int i = 0; i < kDotThreads / 32; ++i) r += red[i];
+    return r;
+}
+
+// anchor[unit][j] = <D_a, h_{a+1}> for a = (j+1) kDaAnchor - 1: the bf16
+// gradient of the state after chunk a and the bf16 state after it (the
+// state entering chunk a+1), in fp32.  One CTA per anchor.
+__global__ void __launch_bounds__(kDotThreads) da_anchor_kernel(float* __restrict__ anchor,
+                                                                const __nv_bfloat16* __restrict__ dbuf,
+                                                                const __nv_bfloat16* __restrict__ hbuf, int NC)
+{
+    constexpr int kVec = static_cast<int>(kSS / 8);                       // 16-byte vectors per state
+    constexpr int kIt = (kVec + kDotThreads - 1) / kDotThreads;
+    __shared__ float red[kDotThreads / 32];
+    const int unit = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
+    const int a = (j + 1) * kDaAnchor - 1;
+    const uint4* x = reinterpret_cast<const uint4*>(dbuf + (static_cast<int64_t>(unit) * NC + a) * kSS);
+    const uint4* y = reinterpret_cast<const uint4*>(hbuf + (static_cast<int64_t>(unit) * NC + a + 1) * kSS);
+    uint4 u[kIt], v[kIt];
+#pragma unroll
+    for (int i = 0; i < kIt; ++i) {
+        const int e = tid + i * kDotThreads;
+        u[i] = e < kVec ? x[e] : make_uint4(0u, 0u, 0u, 0u);
+        v[i] = e < kVec ? y[e] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kIt; ++i) {
+        const uint32_t uw[4] = {u[i].x, u[i].y, u[i].z, u[i].w}, vw[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            s = fmaf(__uint_as_float(uw[w] << 16), __uint_as_float(vw[w] << 16), s);
+            s = fmaf(__uint_as_float(uw[w] & 0xffff0000u), __uint_as_float(vw[w] & 0xffff0000u), s);
+        }
+    }
+    const float r = block_sum_dot(s, red);
+    if (tid == 0) anchor[static_cast<int64_t>(unit) * gridDim.y + j] = r;
+}
+
+// out[unit] = <dS_T, S_T> in fp32 (the da term of the tokens after T).
+__global__ void __launch_bounds__(kDotThreads) state_dot_kernel(float* __restrict__ out,
+                                                                const float* __restrict__ dsT,
+                                                                const float* __restrict__ sT)
+{
+    constexpr int kVec = static_cast<int>(kSS / 4);                       // float4 per state
+    constexpr int kIt = (kVec + kDotThreads - 1) / kDotThreads;
+    __shared__ float red[kDotThreads / 32];
     const int unit = blockIdx.x, tid = threadIdx.x;
     const float4* x = reinterpret_cast<const float4*>(dsT + unit * kSS);
     const float4* y = reinterpret_cast<const float4*>(sT + unit * kSS);
-    float s = 0.f;
-    for (int e = tid; e < kSS / 4; e += 256) {
-        const float4 a = x[e], b = y[e];
-        s = fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, s))));
-    }
+    float4 u[kIt], v[kIt];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if ((tid & 31) == 0) red[tid >> 5] = s;
-    __syncthreads();
-    if (tid == 0) {
-        float r = 0.f;
-        for (int i = 0; i < 8; ++i) r += red[i];
-        out[unit] = r;
+    for (int i = 0; i < kIt; ++i) {
+        const int e = tid + i * kDotThreads;
+        u[i] = e < kVec ? x[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[i] = e < kVec ? y[e] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < kIt; ++i)
+        s = fmaf(u[i].x, v[i].x, fmaf(u[i].y, v[i].y, fmaf(u[i].z, v[i].z, fmaf(u[i].w, v[i].w, s))));
+    const float r = block_sum_dot(s, red);
+    if (tid == 0) out[unit] = r;
 }
 
 template <typename K>
@@ -705,12 +776,25 @@ gla_status launch_bwd_kernel(K kernel, uint32_t bytes, const BwdParams& p, dim3 
 
 }  // namespace
 
+// Segment scratch of the state passes when B*H is too small to fill the GPU:
+// per (unit, segment) an fp32 state and a log2-decay (none when nseg == 1).
+size_t seg_scratch_bytes(int units, int nseg)
+{
+    if (nseg <= 1) return 0;
+    return align256(static_cast<size_t>(units) * nseg * kSS * sizeof(float)) +
+           align256(static_cast<size_t>(units) * nseg * sizeof(float));
+}
+
 size_t bwd_workspace_bytes(int B, int T, int H)
 {
     const size_t units = static_cast<size_t>(B) * H, NC = num_chunks(T);
     const size_t states = align256(units * NC * kSS * 2);
+    int nseg, cps;
+    chunk_segment_plan(static_cast<int>(units), static_cast<int>(NC), &nseg, &cps);
     return 2 * states + align256(units * kSS * sizeof(float)) + align256(2 * units * T * sizeof(float)) +
-           align256(units * NC * 2 * sizeof(float)) + align256(units * sizeof(float));
+           align256(units * NC * 2 * sizeof(float)) + align256(units * sizeof(float)) +
+           align256(units * da_anchors(static_cast<int>(NC)) * sizeof(float)) +
+           seg_scratch_bytes(static_cast<int>(units), nseg);
 }
 
 gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO,
@@ -731,8 +815,36 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     float* ctot = reinterpret_cast<float*>(wsb + off);
     off += align256(static_cast<size_t>(units) * NC * 2 * sizeof(float));
     float* base = reinterpret_cast<float*>(wsb + off);
+    off += align256(static_cast<size_t>(units) * sizeof(float));
+    const int na = da_anchors(NC);
+    float* anchor = reinterpret_cast<float*>(wsb + off);
+    off += align256(static_cast<size_t>(units) * na * sizeof(float));
+    // segments of chunks per unit, each swept by its own CTA, when B*H alone
+    // cannot fill the GPU (long sequences, few heads); the state entering each
+    // segment comes from a state-only pre-pass and a fold (launch_seg_combine)
+    int nseg, cps;
+    chunk_segment_plan(units, NC, &nseg, &cps);
+    float* segst = reinterpret_cast<float*>(wsb + off);
+    float* segg2 = reinterpret_cast<float*>(wsb + off + align256(static_cast<size_t>(units) * nseg * kSS * sizeof(float)));
     const int64_t ldo = static_cast<int64_t>(pr.H) * kDv;
     gla_status s;
+    // state-only pass over `grid_segs` segments from zero into segst / segg2,
+    // then the fold that leaves the state entering each segment's sweep there
+    auto pre_pass = [&](const StateParams& base_p, bool reverse, int grid_segs, const float* edge) {
+        StateParams pre = base_p;
+        pre.store_h = 0;
+        pre.h_out = nullptr;
+        pre.s_init = nullptr;
+        pre.s_out = segst;
+        pre.out_unit_stride = static_cast<int64_t>(nseg) * kSS;
+        pre.out_seg_stride = kSS;
+        pre.out_last_only = 0;
+        pre.g2_out = segg2;
+        pre.g2_unit_stride = nseg;
+        gla_status r = launch_state_kernel(false, reverse, pre, dim3(grid_segs, pr.H, pr.B), st);
+        if (r != GLA_OK) return r;
+        return launch_seg_combine(segst, segg2, edge, nseg, units, reverse, st);
+    };
 
     // 1. h_c for every chunk (and S_T when dS_T is given)
     StateParams sp;
@@ -749,21 +861,38 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     sp.T = pr.T;
     sp.H = pr.H;
     sp.NC = NC;
-    sp.chunks_per_seg = NC;
+    sp.chunks_per_seg = cps;
     sp.store_h = 1;
     sp.h_out = hbuf;
     sp.scale = pr.scale;
     sp.ctl = ctl;
-    if ((s = launch_state_kernel(false, false, sp, dim3(1, pr.H, pr.B), st)) != GLA_OK) return s;
+    if (nseg > 1) {
+        // local end states of segments 0 .. nseg-2 (the last one's is not needed)
+        if ((s = pre_pass(sp, false, nseg - 1, s0)) != GLA_OK) return s;
+        sp.s_init = segst;
+        sp.init_unit_stride = static_cast<int64_t>(nseg) * kSS;
+        sp.init_seg_stride = kSS;
+    }
+    if ((s = launch_state_kernel(false, false, sp, dim3(nseg, pr.H, pr.B), st)) != GLA_OK) return s;
 
-    // 2. D_c for every chunk, dS_0
+    // 2. D_c for every chunk, dS_0 (written by segment 0, where the reverse sweep ends)
     StateParams rp = sp;
     if ((s = make_token_map(&rp.tm_u, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&rp.tm_y, dO, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
     rp.h_out = dbuf;
     rp.s_init = ds_final;
+    rp.init_unit_stride = kSS;
+    rp.init_seg_stride = 0;
+    if (nseg > 1) {
+        // local gradients of every segment (segment 0's is computed and not
+        // used: its CTAs run beside the others')
+        if ((s = pre_pass(rp, true, nseg, ds_final)) != GLA_OK) return s;
+        rp.s_init = segst;
+        rp.init_unit_stride = static_cast<int64_t>(nseg) * kSS;
+        rp.init_seg_stride = kSS;
+    }
     rp.s_out = ds0;
-    if ((s = launch_state_kernel(false, true, rp, dim3(1, pr.H, pr.B), st)) != GLA_OK) return s;
+    if ((s = launch_state_kernel(false, true, rp, dim3(nseg, pr.H, pr.B), st)) != GLA_OK) return s;
 
     // 3. dq, dk (+ per-token delta halves and chunk totals) and dv
     BwdParams bp;
@@ -799,14 +928,22 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     // 4. da = reverse cumulative sum of delta (+ <dS_T, S_T>)
     if (ds_final) {
         trace_begin(st);
-        state_dot_kernel<<<units, 256, 0, st>>>(base, ds_final, sT);
+        state_dot_kernel<<<units, kDotThreads, 0, st>>>(base, ds_final, sT);
         trace_end(st, "state_dot_kernel");
         count_launch();
         if ((s = check_launch("state_dot_kernel")) != GLA_OK) return s;
     }
+    if (na > 0) {
+        trace_begin(st);
+        da_anchor_kernel<<<dim3(units, na), kDotThreads, 0, st>>>(anchor, static_cast<const __nv_bfloat16*>(dbuf),
+                                                          static_cast<const __nv_bfloat16*>(hbuf), NC);
+        trace_end(st, "da_anchor_kernel");
+        count_launch();
+        if ((s = check_launch("da_anchor_kernel")) != GLA_OK) return s;
+    }
     trace_begin(st);
-    da_finish_kernel<<<dim3(units, NC), kDaThreads, 0, st>>>(da, delta, ctot, ds_final ? base : nullptr, pr.T, pr.H,
-                                                             NC, units);
+    da_finish_kernel<<<dim3(units, NC), kDaThreads, 0, st>>>(da, delta, ctot, ds_final ? base : nullptr, anchor,
+                                                             pr.T, pr.H, NC, units);
     trace_end(st, "da_finish_kernel");
     count_launch();
     return check_launch("da_finish_kernel");

@@ -27,22 +27,13 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 int num_chunks(int T) { return (T + kChunk - 1) / kChunk; }
 
-void segment_plan(int units, int NC, int* nseg, int* cps)
-{
-    int n = units >= kTargetCtas / 2 ? 1 : kTargetCtas / units;
-    n = n < 1 ? 1 : (n > NC ? NC : n);
-    int c = (NC + n - 1) / n;
-    *cps = c;
-    *nseg = (NC + c - 1) / c;
-}
-
-// States entering every segment, in place: slot g holds L_g (the local end
-// state of segment g from zero) on entry and S_g on return.  The loads of a
-// batch of segments are issued before the dependent chain that uses them.
+// States entering every segment's sweep, in place (launch_seg_combine).
+// The loads of a batch of segments are issued before the dependent chain that
+// uses them.
 __global__ void __launch_bounds__(256) seg_combine_kernel(float* __restrict__ states,
                                                           const float* __restrict__ g2,
-                                                          const float* __restrict__ s0, int nseg,
-                                                          int units)
+                                                          const float* __restrict__ s_edge, int nseg,
+                                                          int units, int reverse)
 {
     constexpr int kBatch = 8;
     const int64_t n4 = kSS / 4;
@@ -50,25 +41,25 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(float* __restrict__ st
     if (idx >= n4 * units) return;
     const int64_t unit = idx / n4, e4 = idx - unit * n4;
     float4* st = reinterpret_cast<float4*>(states);
-    float4 x = s0 ? reinterpret_cast<const float4*>(s0)[unit * n4 + e4] : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int g0 = 0; g0 < nseg; g0 += kBatch) {
+    float4 x = s_edge ? reinterpret_cast<const float4*>(s_edge)[unit * n4 + e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i0 = 0; i0 < nseg; i0 += kBatch) {
         float4 l[kBatch];
         float f[kBatch];
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
-            const int g = g0 + u;
-            // the last segment's slot only receives its entering state
-            if (g < nseg - 1) {
+            const int i = i0 + u, g = reverse ? nseg - 1 - i : i;
+            // the sweep's last segment only receives its entering state
+            if (i < nseg - 1) {
                 l[u] = st[(unit * nseg + g) * n4 + e4];
                 f[u] = g2[unit * nseg + g];
             }
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
-            const int g = g0 + u;
-            if (g < nseg) {
+            const int i = i0 + u, g = reverse ? nseg - 1 - i : i;
+            if (i < nseg) {
                 st[(unit * nseg + g) * n4 + e4] = x;
-                if (g < nseg - 1) {
+                if (i < nseg - 1) {
                     const float e = exp2f(f[u]);
                     x.x = fmaf(e, x.x, l[u].x);
                     x.y = fmaf(e, x.y, l[u].y);
@@ -94,6 +85,27 @@ gla_status launch_chunk_kernel(K kernel, uint32_t bytes, const char* name, const
 }
 
 }  // namespace
+
+void chunk_segment_plan(int units, int NC, int* nseg, int* cps)
+{
+    int n = units >= kTargetCtas / 2 ? 1 : kTargetCtas / units;
+    n = n < 1 ? 1 : (n > NC ? NC : n);
+    int c = (NC + n - 1) / n;
+    *cps = c;
+    *nseg = (NC + c - 1) / c;
+}
+
+gla_status launch_seg_combine(float* states, const float* g2, const float* s_edge, int nseg, int units,
+                              bool reverse, cudaStream_t st)
+{
+    const int64_t n4 = static_cast<int64_t>(units) * (kSS / 4);
+    trace_begin(st);
+    seg_combine_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(states, g2, s_edge, nseg, units,
+                                                                               reverse ? 1 : 0);
+    trace_end(st, "seg_combine_kernel");
+    count_launch();
+    return check_launch("seg_combine_kernel");
+}
 
 gla_status make_token_map(CUtensorMap* m, const void* base, int d, int H, int T, int B,
                           int64_t ld, int box_d, int swizzle, int box_rows)
@@ -137,7 +149,7 @@ size_t fwd_workspace_bytes(int B, int T, int H)
 {
     const int units = B * H, NC = num_chunks(T);
     int nseg, cps;
-    segment_plan(units, NC, &nseg, &cps);
+    chunk_segment_plan(units, NC, &nseg, &cps);
     if (nseg == 1) return 0;
     return align256(static_cast<size_t>(units) * nseg * kSS * sizeof(float)) +
            align256(static_cast<size_t>(units) * nseg * sizeof(float));
@@ -179,7 +191,7 @@ gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float
     (void)ws_bytes;
     const int units = pr.B * pr.H, NC = num_chunks(pr.T);
     int nseg, cps;
-    segment_plan(units, NC, &nseg, &cps);
+    chunk_segment_plan(units, NC, &nseg, &cps);
 
     StateParams p;
     memset(&p, 0, sizeof(p));
@@ -222,13 +234,7 @@ gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float
     pre.g2_unit_stride = nseg;
     if ((s = launch_state_kernel(false, false, pre, dim3(nseg - 1, pr.H, pr.B), st)) != GLA_OK) return s;
     // 2. states entering every segment
-    const int64_t n4 = static_cast<int64_t>(units) * (kSS / 4);
-    trace_begin(st);
-    seg_combine_kernel<<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(states, g2, s0, nseg,
-                                                                               units);
-    trace_end(st, "seg_combine_kernel");
-    count_launch();
-    if ((s = check_launch("seg_combine_kernel")) != GLA_OK) return s;
+    if ((s = launch_seg_combine(states, g2, s0, nseg, units, false, st)) != GLA_OK) return s;
     // 3. fused output pass
     p.s_init = states;
     p.init_unit_stride = nseg * kSS;

@@ -31,21 +31,11 @@
 namespace gla {
 namespace {
 
-constexpr int kTargetCtas = 148;
 constexpr int64_t kSS = static_cast<int64_t>(kDk) * kDv;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kFoldBatch = 8;      // entries whose loads are in flight together
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-
-void sub_segment_plan(int units, int NC, int* nseg, int* cps)
-{
-    int n = units >= kTargetCtas / 2 ? 1 : kTargetCtas / units;
-    n = n < 1 ? 1 : (n > NC ? NC : n);
-    const int c = (NC + n - 1) / n;
-    *cps = c;
-    *nseg = (NC + c - 1) / c;
-}
 
 // Fold of one unit's sub-segments, in order (forward) or right to left
 // (reverse), from a zero state: out = the segment's L (or D); g_out = the
@@ -138,7 +128,7 @@ size_t segment_workspace_bytes(int B, int T, int H)
 {
     const int units = B * H, NC = (T + kChunk - 1) / kChunk;
     int nseg, cps;
-    sub_segment_plan(units, NC, &nseg, &cps);
+    chunk_segment_plan(units, NC, &nseg, &cps);
     return align256(static_cast<size_t>(units) * nseg * kSS * sizeof(float)) +
            align256(static_cast<size_t>(units) * nseg * sizeof(float));
 }
@@ -149,7 +139,7 @@ gla_status run_segment_state(const void* u, const void* y, const float* a, int B
 {
     const int units = B * H, NC = (T + kChunk - 1) / kChunk;
     int nseg, cps;
-    sub_segment_plan(units, NC, &nseg, &cps);
+    chunk_segment_plan(units, NC, &nseg, &cps);
     float* parts = static_cast<float*>(ws);
     float* g2 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
                                          align256(static_cast<size_t>(units) * nseg * kSS * sizeof(float)));

@@ -70,7 +70,8 @@ struct StateParams {
     int64_t init_unit_stride, init_seg_stride;   // elements
     int64_t out_unit_stride, out_seg_stride;     // elements
     int B, T, H, NC, chunks_per_seg;
-    int out_last_only;      // write s_out only from the last segment
+    int out_last_only;      // write s_out only from the segment that ends the sweep
+                            // (the last one; segment 0 in the reverse pass)
     int g2_unit_stride;     // segments per unit in g2_out
     int store_h;            // store the bf16 state entering each chunk into h_out
     void* h_out;            // bf16 [B*H*NC][96][192]
@@ -957,7 +958,8 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
             if (p.store_h && it + 1 < nchunks) store_h(it + 1);
         }
         if (ok) {
-            const bool write_state = p.s_out && (!p.out_last_only || seg == static_cast<int>(gridDim.x) - 1);
+            const int sweep_end = REVERSE ? 0 : static_cast<int>(gridDim.x) - 1;
+            const bool write_state = p.s_out && (!p.out_last_only || seg == sweep_end);
             if (write_state) {
                 float* dst = p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + qt * 48;
 #pragma unroll

@@ -104,4 +104,14 @@ gla_status make_state_map(CUtensorMap* m, void* base, int64_t nstates, int box_c
 gla_status launch_state_kernel(bool with_o, bool reverse, const StateParams& p, dim3 grid,
                                cudaStream_t st);
 
+// Segment plan of a unit's chunks when B*H alone cannot fill the GPU: nseg
+// segments of cps chunks (the last may be shorter); nseg == 1 otherwise.
+void chunk_segment_plan(int units, int NC, int* nseg, int* cps);
+// In place over states [units][nseg][dk*dv]: slot g holds segment g's local
+// state from zero on entry (L_g, or D_g in reverse) and, on return, the state
+// entering segment g's sweep: S_0 folded forward over segments < g, or (reverse)
+// dS_T folded right to left over segments > g.  s_edge (S_0 or dS_T) may be null.
+gla_status launch_seg_combine(float* states, const float* g2, const float* s_edge, int nseg, int units,
+                              bool reverse, cudaStream_t st);
+
 }  // namespace gla

@@ -90,6 +90,20 @@ def test_chunk_bwd_parity(B, T, H, s0, dsT):
     check_bwd(d, grads, dsT=ds)
 
 
+@pytest.mark.parametrize("B,T,H", [(1, 12795, 3), (1, 16384, 16)])
+def test_chunk_bwd_long_sequence_few_heads(B, T, H):
+    """Few (batch, head) units and a long sequence: each unit's chunks are
+    swept as segments (one CTA each; 34 segments of 3 chunks with a
+    one-chunk tail at B*H = 3, 9 of 15 with an 8-chunk tail at B*H = 16),
+    the state entering each from a state-only pre-pass and a fold.  With s0
+    and dS_T; sampled heads against the oracle on the whole sequence."""
+    d = inputs.chunk_inputs(B, T, H, seed=250 + H, device="cuda", s0_std=0.1, with_dO=True)
+    ds = inputs.randn((B, H, 96, 192), 251 + H, "cuda", std=0.1)
+    grads = gla.gla_chunk_bwd(d["q"], d["k"], d["v"], d["a"], d["dO"], s0=d["s0"], ds_final=ds)
+    assert gla.gla_get_device_status() == 0
+    check_bwd(d, grads, units=[(0, 0), (0, H - 1)], dsT=ds)
+
+
 def test_chunk_bwd_fused_projection_stride():
     B, T, H = 2, 200, 16
     d = inputs.chunk_inputs(B, T, H, seed=220, device="cuda", s0_std=0.1, ld=9216, with_dO=True)

@@ -135,10 +135,106 @@ def test_conv_validation(L):
     assert conv(D=3070) == UNSUPPORTED
     assert conv(D=8192) == UNSUPPORTED
     assert conv(eps=0.0) == INVALID
-    assert conv(ln=0, eps=0.0) != INVALID      # eps only matters with LayerNorm
+    # eps only matters with LayerNorm: without it the call gets past the eps
+    # check to the (later) width check; nothing here reaches a launch
+    assert conv(ln=0, eps=0.0, W=3) == UNSUPPORTED
+    assert conv(ln=1, eps=0.0, W=3) == INVALID
     assert conv(csi=0x4000, cso=0x4000) == INVALID
     assert conv(y=0x3002) == MISALIGNED
     assert conv(B=0) == OK
+
+
+def test_varlen_validation(L):
+    def varlen(q=0x1000, k=0x2000, v=0x3000, a=0x4000, cu=0x5000, N=2, s0=None, o=0x6000, sf=None,
+               total=256, H=2, dk=96, dv=192, ld=0, scale=96 ** -0.5, dt=0):
+        return L.gla_chunk_fwd_varlen(P(q), P(k), P(v), P(a), P(cu), N, P(s0), P(o), P(sf), total, H, dk, dv,
+                                      ld, scale, dt, None)
+    assert varlen(N=-1) == INVALID
+    assert varlen(N=70000) == UNSUPPORTED
+    assert varlen(dt=1) == UNSUPPORTED           # bf16 only
+    assert varlen(cu=None) == INVALID
+    assert varlen(o=None) == INVALID
+    assert varlen(q=None) == INVALID
+    assert varlen(dk=64) == UNSUPPORTED
+    assert varlen(s0=0x7008) == MISALIGNED
+    assert varlen(N=0) == OK
+
+
+def test_conv_decode_and_backward_validation(L):
+    def dec(x=0x1000, slot=None, ln=1, g=None, b=None, eps=1e-5, w=0x2000, bias=None, cs=0x3000, y=0x4000,
+            N=4, D=3072, W=4):
+        return L.conv1d_silu_decode_step(P(x), P(slot), ln, P(g), P(b), eps, P(w), P(bias), P(cs), P(y), N, D, W,
+                                         None)
+    assert dec(x=None) == INVALID
+    assert dec(cs=None) == INVALID
+    assert dec(W=3) == UNSUPPORTED
+    assert dec(D=12) == UNSUPPORTED
+    assert dec(eps=-1.0) == INVALID
+    assert dec(cs=0x3004) == MISALIGNED
+    assert dec(N=0) == OK
+
+    need = gla.conv1d_silu_causal_bwd_workspace_bytes(1, 64, 3072)
+    assert need > 0
+    assert gla.conv1d_silu_causal_bwd_workspace_bytes(1, 64, 3072, 3) == 0
+
+    def bwd(x=0x1000, ln=1, g=None, b=None, eps=1e-5, w=0x2000, bias=None, csi=None, dy=0x3000, dx=0x4000,
+            dw=0x5000, dbias=None, dg=None, db=None, dcs=None, ws=0x6000, wsb=need, B=1, T=64, D=3072, W=4):
+        return L.conv1d_silu_causal_bwd(P(x), ln, P(g), P(b), eps, P(w), P(bias), P(csi), P(dy), P(dx), P(dw),
+                                        P(dbias), P(dg), P(db), P(dcs), P(ws), wsb, B, T, D, W, None)
+    assert bwd(dw=None) == INVALID
+    assert bwd(dy=None) == INVALID
+    assert bwd(B=70000) == UNSUPPORTED
+    assert bwd(W=5) == UNSUPPORTED
+    assert bwd(ws=None) == INVALID
+    assert bwd(wsb=need - 16) == INVALID
+    assert bwd(dx=0x4008) == MISALIGNED
+    assert bwd(dcs=0x7004) == MISALIGNED
+
+
+def test_segment_calls_validation(L):
+    """gla_segment_state_fwd / _bwd, gla_state_fold, gla_segment_workspace_bytes:
+    every case below is rejected on the host before any device work."""
+    need = gla.gla_segment_workspace_bytes(1, 1000, 2)
+    assert need > 0
+    assert gla.gla_segment_workspace_bytes(1, 1000, 2, 64, 192) == 0
+    assert gla.gla_segment_workspace_bytes(0, 1000, 2) == 0
+    # more (batch, head) pairs or a shorter sequence never need more scratch per token
+    assert gla.gla_segment_workspace_bytes(1, 8192, 16) >= gla.gla_segment_workspace_bytes(1, 4096, 16)
+
+    def seg(fn, u=0x1000, y=0x2000, a=0x3000, s=0x4000, g=0x5000, ws=0x6000, wsb=need, B=1, T=1000, H=2,
+            dk=96, dv=192, ld=0, scale=96 ** -0.5, dt=0):
+        if fn == "fwd":
+            return L.gla_segment_state_fwd(P(u), P(y), P(a), P(s), P(g), P(ws), wsb, B, T, H, dk, dv, ld, dt,
+                                           None)
+        return L.gla_segment_state_bwd(P(u), P(y), P(a), P(s), P(g), P(ws), wsb, B, T, H, dk, dv, ld, scale,
+                                       dt, None)
+    for fn in ("fwd", "bwd"):
+        assert seg(fn, u=None) == INVALID
+        assert seg(fn, a=None) == INVALID
+        assert seg(fn, s=None) == INVALID         # the segment state is required
+        assert seg(fn, ws=None) == INVALID
+        assert seg(fn, wsb=need - 16) == INVALID
+        assert seg(fn, dk=64) == UNSUPPORTED
+        assert seg(fn, dt=1) == UNSUPPORTED       # bf16 only
+        assert seg(fn, T=-1) == INVALID
+        assert seg(fn, s=0x4004) == MISALIGNED
+        assert seg(fn, g=0x5008) == MISALIGNED
+        assert seg(fn, y=0x2002) == MISALIGNED
+        assert seg(fn, B=0) == OK
+    assert seg("bwd", scale=0.0) == INVALID
+
+    def fold(s=0x1000, g=0x2000, n=3, rev=0, s_in=None, out=0x3000, units=4, dk=96, dv=192):
+        return L.gla_state_fold(P(s), P(g), n, rev, P(s_in), P(out), units, dk, dv, None)
+    assert fold(n=-1) == INVALID
+    assert fold(units=-1) == INVALID
+    assert fold(out=None) == INVALID
+    assert fold(s=None) == INVALID
+    assert fold(g=None) == INVALID
+    assert fold(dk=64) == UNSUPPORTED
+    assert fold(s=0x1008) == MISALIGNED
+    assert fold(g=0x2002) == MISALIGNED           # g needs 4-byte alignment only
+    assert fold(s_in=0x4004) == MISALIGNED
+    assert fold(units=0) == OK
 
 
 def test_wait_limit_setter(L):

@@ -6,8 +6,13 @@ the static CUDA runtime, into ``linear_attention_simple_b200/libgla.so``.
 The driver library is not linked: ``cuTensorMapEncodeTiled`` is fetched at
 run time through ``cudaGetDriverEntryPoint``, so the library loads on hosts
 without a GPU.
+
+Several processes may call build() at once (one per rank under torchrun):
+an exclusive lock on ``_build/.lock`` serialises them, and every object and
+the library are written under a temporary name and renamed into place.
 """
 import concurrent.futures
+import fcntl
 import os
 import shutil
 import subprocess
@@ -43,10 +48,12 @@ def _compile(src, verbose=False):
     if (os.path.exists(obj) and os.path.getmtime(obj) >= os.path.getmtime(src)
             and os.path.getmtime(obj) >= _headers_mtime()):
         return obj
-    cmd = [nvcc()] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
+    tmp = obj + ".tmp.%d" % os.getpid()
+    cmd = [nvcc()] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", tmp]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed for %s:\n%s\n%s" % (src, r.stdout, r.stderr))
+    os.replace(tmp, obj)
     if verbose:
         sys.stderr.write(r.stderr)
     return obj
@@ -54,6 +61,12 @@ def _compile(src, verbose=False):
 
 def build(verbose=False, force=False):
     os.makedirs(BUILD, exist_ok=True)
+    with open(os.path.join(BUILD, ".lock"), "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        return _build_locked(verbose, force)
+
+
+def _build_locked(verbose, force):
     if force:
         for f in os.listdir(BUILD):
             if f.endswith(".o"):

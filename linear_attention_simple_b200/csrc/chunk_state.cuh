@@ -435,6 +435,16 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             mbar_arrive_expect_tx(bar_u, kTileQK);
             for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::U + i * 8192, &p.tm_u, bar_u, i * 32, h, tb + t0, bc);
         };
+        // q, k of a later chunk into L2, so that its load (issued only once the
+        // current chunk's state update has released the tiles) hits L2
+        auto prefetch_qu = [&](int c) {
+            const int t0 = c * 128;
+            for (int i = 0; i < 3; ++i) {
+                for (int r16 = 0; r16 < 8; ++r16)
+                    tma_prefetch_l2_4d(&p.tm_q, i * 32, h, tb + t0 + r16 * 16, bc);
+                tma_prefetch_l2_4d(&p.tm_u, i * 32, h, tb + t0, bc);
+            }
+        };
         auto issue_y = [&](int c, int s) {
             uint8_t* y = sm + (s ? L::Y1 : L::Y0);
             mbar_arrive_expect_tx(bar_y + s, kTileV);
@@ -442,6 +452,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                 tma_load_4d(y + i * 16384, &p.tm_y, bar_y + s, i * 64, h, tb + c * 128, bc);
         };
         int n_qu = 0, n_y[2] = {0, 0};
+        if (nchunks > 1) prefetch_qu(c_begin + 1);
         if (nchunks > 0) {
             issue_qu(c_begin);
             ++n_qu;
@@ -454,6 +465,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         }
         for (int it = 0; it < nchunks; ++it) {
             const int c = c_begin + it, ys = it & 1;
+            if (it + 2 < nchunks) prefetch_qu(c + 2);
             if (it + 1 < nchunks) {
                 if (!mbar_wait(bar_d, it & 1, ctl)) break;
                 issue_qu(c + 1);
@@ -522,10 +534,16 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         if (worker && !failed && !mbar_wait(bar_sc, it & 1, ctl)) failed = true;
         if (!failed && worker) {
             const int live = Tn - c * 128;   // varlen: rows past the sequence (the next one's) add nothing
-            for (int idx = tid; idx < 384; idx += kWorkers) {
-                const int r = idx & 127, blk = idx >> 7;
-                scale_row_sw64(sm + L::U, r, blk, (!VARLEN || r < live) ? exp2f(g2 - b2c[r]) : 0.f);
-                if (!fast) scale_row_sw64(sm + L::Q, r, blk, p.scale * exp2f(b2c[row_token(r)]));
+            // 16-byte chunk idx % 4 of row (idx / 4) % 128 of block idx / 512: a
+            // warp covers 512 contiguous bytes, so no two lanes share a bank
+            for (int idx = tid; idx < 1536; idx += kWorkers) {
+                const int r = (idx >> 2) & 127, blk = idx >> 9, ch = idx & 3;
+                uint4* u = reinterpret_cast<uint4*>(sm + L::U + blk * 8192 + r * 64) + ch;
+                *u = scale8(*u, (!VARLEN || r < live) ? exp2f(g2 - b2c[r]) : 0.f);
+                if (!fast) {
+                    uint4* qq = reinterpret_cast<uint4*>(sm + L::Q + blk * 8192 + r * 64) + ch;
+                    *qq = scale8(*qq, p.scale * exp2f(b2c[row_token(r)]));
+                }
             }
         }
         fence_async_smem();

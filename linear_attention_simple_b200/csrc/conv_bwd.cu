@@ -10,14 +10,18 @@
 //   dw[c,j]   = sum_t du[t,c] xn[t-3+j, c]   dbias = sum du
 //   dgamma    = sum dxn xhat                  dbeta = sum dxn
 //
-// conv_bwd_kernel: one CTA per (128-token range, sequence), thread i owns
-// CH consecutive channels (4, or 8 when D > 3072) and walks the rows p = t0-3 .. t1+2 once: the
-// LayerNorm of row p (one block reduction of the shifted first and second
-// moments), then u and du of row p, then dxn and dx of row q = p-3 (one block
-// reduction of sum g and sum g xhat).  The last four rows of xn, xhat and du
-// sit in shared-memory rings private to each thread.  The sums over tokens
-// go to per-CTA partials; conv_bwd_reduce_kernel adds them in a fixed order
-// (deterministic).
+// Three passes, none with a block-wide barrier per row:
+//   ln_stats_kernel       mean and rstd of every row (a warp per row);
+//   conv_bwd_tile_kernel<false>  tiles of 256 rows x 512 channels, a thread per
+//                         2 channels walking the rows with register windows:
+//                         u, du, dxn, the per-(tile, channel) sums of dw,
+//                         dbias, dgamma, dbeta, the history gradient, and the
+//                         per-row sums of g and g xhat over the tile's
+//                         channels (dx itself when there is no LayerNorm);
+//   conv_bwd_tile_kernel<true>   the same walk again, finishing dx from the
+//                         row totals of those sums.
+// conv_bwd_reduce_kernel adds the per-tile partials in a fixed order, so
+// every output is deterministic.
 #include <cuda_bf16.h>
 
 #include "gla_device.cuh"
@@ -26,8 +30,12 @@
 namespace gla {
 namespace {
 
-constexpr int kRows = 128;       // tokens per CTA
+constexpr int kRows = 256;       // tokens per tile
+constexpr int kTileThreads = 256;
+constexpr int kTileCh = 2 * kTileThreads;   // channels per tile
 constexpr int kParts = 7;        // dw (4 taps), dbias, dgamma, dbeta
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 __device__ __forceinline__ float warp_sum_bwd(float v)
 {
@@ -36,281 +44,251 @@ __device__ __forceinline__ float warp_sum_bwd(float v)
     return v;
 }
 
-// Block sums of (a, b); every thread gets both.  Two buffers used in turn,
-// so one barrier per reduction suffices.
-__device__ __forceinline__ void block_sum2(float& a, float& b, float* red, int& turn)
+// stats[row] = (mean, rstd) of the row's D values; the moments are taken
+// about the row's first element (shifted), as the forward does.
+__global__ void __launch_bounds__(256) ln_stats_kernel(const __nv_bfloat16* __restrict__ x, int rows, int D,
+                                                       float eps, float2* __restrict__ stats)
 {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = (blockDim.x + 31) >> 5;
-    float* r = red + (turn & 1) * 64;
-    ++turn;
-    a = warp_sum_bwd(a);
-    b = warp_sum_bwd(b);
-    if (lane == 0) {
-        r[warp] = a;
-        r[32 + warp] = b;
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const __nv_bfloat16* xr = x + static_cast<int64_t>(row) * D;
+    const float x0 = __bfloat162float(xr[0]);
+    float s1 = 0.f, s2 = 0.f;
+    for (int v = lane; v < D / 8; v += 32) {
+        const uint4 q = *reinterpret_cast<const uint4*>(xr + v * 8);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float a = bf16_lo(w[i]) - x0, b = bf16_hi(w[i]) - x0;
+            s1 += a + b;
+            s2 = fmaf(a, a, fmaf(b, b, s2));
+        }
     }
-    __syncthreads();
-    // every warp reduces the per-warp partials again (same order in each)
-    a = warp_sum_bwd(lane < nw ? r[lane] : 0.f);
-    b = warp_sum_bwd(lane < nw ? r[32 + lane] : 0.f);
+    s1 = warp_sum_bwd(s1);
+    s2 = warp_sum_bwd(s2);
+    if (lane == 0) {
+        const float m1 = s1 / D;
+        const float var = fmaxf(s2 / D - m1 * m1, 0.f);
+        stats[row] = make_float2(x0 + m1, rsqrtf(var + eps));
+    }
 }
 
-// Raw bf16 words of CH channels (prefetched ahead of their use).
-template <int CH>
-struct RawRow {
-    uint32_t w[CH / 2];
+struct TileArgs {
+    const __nv_bfloat16* x;
+    const __nv_bfloat16* dy;
+    const float* gamma;
+    const float* beta;
+    const float* w;
+    const float* bias;
+    const float* cs_in;
+    const float2* stats;       // [B*T] (LayerNorm only)
+    float2* psum;              // [B*T][CB] per-row sums of g and g xhat over a tile's channels
+    float* part;               // [B * nrb][7][D]
+    float* dcs;
+    __nv_bfloat16* dx;
+    int T, D, CB, nrb, apply_ln;
 };
 
-template <int CH>
-__device__ __forceinline__ RawRow<CH> ld_raw(const __nv_bfloat16* p)
+// FINISH = false: sums (and dx without LayerNorm); FINISH = true: dx.
+template <bool FINISH>
+__global__ void __launch_bounds__(kTileThreads) conv_bwd_tile_kernel(const TileArgs a)
 {
-    RawRow<CH> r;
-    if constexpr (CH == 4) {
-        const uint2 u = *reinterpret_cast<const uint2*>(p);
-        r.w[0] = u.x;
-        r.w[1] = u.y;
-    } else {
-        const uint4 u = *reinterpret_cast<const uint4*>(p);
-        r.w[0] = u.x;
-        r.w[1] = u.y;
-        r.w[2] = u.z;
-        r.w[3] = u.w;
-    }
-    return r;
-}
-
-template <int CH>
-__device__ __forceinline__ void unpack_raw(const RawRow<CH>& r, float (&v)[CH])
-{
-#pragma unroll
-    for (int i = 0; i < CH / 2; ++i) {
-        v[2 * i] = bf16_lo(r.w[i]);
-        v[2 * i + 1] = bf16_hi(r.w[i]);
-    }
-}
-
-template <int CH>
-__device__ __forceinline__ void stv_bf16(__nv_bfloat16* p, const float (&v)[CH])
-{
-    if constexpr (CH == 4) {
-        *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]));
-    } else {
-        *reinterpret_cast<uint4*>(p) = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
-                                                  pack_bf16(v[6], v[7]));
-    }
-}
-
-template <int CH>
-__device__ __forceinline__ void ldv_f32(const float* p, float (&v)[CH])
-{
-#pragma unroll
-    for (int i = 0; i < CH; i += 4) {
-        const float4 q = *reinterpret_cast<const float4*>(p + i);
-        v[i] = q.x;
-        v[i + 1] = q.y;
-        v[i + 2] = q.z;
-        v[i + 3] = q.w;
-    }
-}
-
-template <int CH>
-__device__ __forceinline__ void stv_f32(float* p, const float (&v)[CH])
-{
-#pragma unroll
-    for (int i = 0; i < CH; i += 4) *reinterpret_cast<float4*>(p + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-}
-
-// CH channels per thread: 4 (at most 768 threads, D <= 3072) or 8 (D <= 4096).
-template <int CH>
-__global__ void __launch_bounds__(CH == 4 ? 768 : 512, 1) conv_bwd_kernel(
-    const __nv_bfloat16* __restrict__ x, int apply_ln, const float* __restrict__ gamma,
-    const float* __restrict__ beta, float eps, const float* __restrict__ w, const float* __restrict__ bias,
-    const float* __restrict__ cs_in, const __nv_bfloat16* __restrict__ dy, __nv_bfloat16* __restrict__ dx,
-    float* __restrict__ dcs, float* __restrict__ part, int T, int D)
-{
-    extern __shared__ float smf[];
-    float* xn_r = smf;               // [4][D]
-    float* xh_r = smf + 4 * D;       // [4][D]
-    float* du_r = smf + 8 * D;       // [4][D]
-    float* red = smf + 12 * D;       // [2][64]
-    float* aff = red + 128;          // CH == 4: [3][D] gamma, beta, bias (fewer live registers)
-    const int blk = blockIdx.x, b = blockIdx.y, c = threadIdx.x * CH;
-    const int t0 = blk * kRows, t1 = min(T, t0 + kRows);
+    __shared__ float2 rowsum[kRows][kTileThreads / 32];
+    __shared__ float2 total[kRows];
+    __shared__ float2 st_s[kRows + 6];     // LayerNorm statistics of rows t0-3 .. t1+2
+    const int rb = blockIdx.x, b = blockIdx.y, cb = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = cb * kTileCh + 2 * tid;
+    const bool live = c < a.D;
+    const int T = a.T, D = a.D;
+    const int t0 = rb * kRows, t1 = min(T, t0 + kRows);
     const int64_t row0 = static_cast<int64_t>(b) * T;
+    const bool ln = a.apply_ln != 0;
 
-    float wv[CH][4];
-    float aff_r[3][CH == 4 ? 1 : CH];
+    for (int i = tid; i < t1 - t0 + 6; i += kTileThreads) {
+        const int r = t0 - 3 + i;
+        st_s[i] = (ln && r >= 0 && r < T) ? a.stats[row0 + r] : make_float2(0.f, 1.f);
+    }
+    if (FINISH) {
+        // row totals of the tile's rows: the per-channel-block sums, in order
+        for (int i = tid; i < t1 - t0; i += kTileThreads) {
+            float sg = 0.f, sgh = 0.f;
+            for (int k = 0; k < a.CB; ++k) {
+                const float2 v = a.psum[(row0 + t0 + i) * a.CB + k];
+                sg += v.x;
+                sgh += v.y;
+            }
+            total[i] = make_float2(sg, sgh);
+        }
+    }
+    __syncthreads();
+
+    float wv[2][4], gm[2], bt[2], bi[2];
 #pragma unroll
-    for (int e = 0; e < CH; ++e) {
-        const float4 q = *reinterpret_cast<const float4*>(w + static_cast<int64_t>(c + e) * 4);
+    for (int e = 0; e < 2; ++e) {
+        const float4 q = live ? *reinterpret_cast<const float4*>(a.w + static_cast<int64_t>(c + e) * 4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
         wv[e][0] = q.x;
         wv[e][1] = q.y;
         wv[e][2] = q.z;
         wv[e][3] = q.w;
-        const float gv = gamma ? gamma[c + e] : 1.f, bv = beta ? beta[c + e] : 0.f, iv = bias ? bias[c + e] : 0.f;
-        if constexpr (CH == 4) {
-            aff[c + e] = gv;
-            aff[D + c + e] = bv;
-            aff[2 * D + c + e] = iv;
-        } else {
-            aff_r[0][e] = gv;
-            aff_r[1][e] = bv;
-            aff_r[2][e] = iv;
-        }
+        gm[e] = (live && a.gamma) ? a.gamma[c + e] : 1.f;
+        bt[e] = (live && a.beta) ? a.beta[c + e] : 0.f;
+        bi[e] = (live && a.bias) ? a.bias[c + e] : 0.f;
     }
-    // gamma, beta, bias of channel c+e (thread-private in shared memory when
-    // CH == 4, read as one 16-byte vector: conflict-free)
-    auto affv = [&](int k, int e) {
-        if constexpr (CH == 4) {
-            const float4 q = *reinterpret_cast<const float4*>(aff + k * D + c);
-            return e == 0 ? q.x : e == 1 ? q.y : e == 2 ? q.z : q.w;
-        } else {
-            return aff_r[k][e];
-        }
-    };
-    auto g4 = [&](int e) { return affv(0, e); };
-    auto be4 = [&](int e) { return affv(1, e); };
-    auto bi4 = [&](int e) { return affv(2, e); };
-    float pdw[4][CH] = {}, pdb[CH] = {}, pdg[CH] = {}, pdbe[CH] = {};
-    float rs_r[4] = {1.f, 1.f, 1.f, 1.f};
-    int turn = 0;
+    float pdw[4][2] = {}, pdb[2] = {}, pdg[2] = {}, pdbe[2] = {};
+    // windows over rows p-3 .. p (index 3 = row p)
+    float xn[4][2] = {}, xh[4][2] = {}, du[4][2] = {}, rs[4] = {1.f, 1.f, 1.f, 1.f};
 
-    // x (with its row's first element, the LayerNorm shift) and dy of rows
-    // p, p+1 and p+2 in registers: loads go out two rows ahead of their use
-    auto fetch = [&](int r, RawRow<CH>& xr, float& x0, RawRow<CH>& dr) {
-        if (r >= 0 && r < T) {
-            xr = ld_raw<CH>(x + (row0 + r) * D + c);
-            x0 = __bfloat162float(x[(row0 + r) * D]);
-            if (r >= t0) dr = ld_raw<CH>(dy + (row0 + r) * D + c);
+    // x and dy of a row (this thread's two channels), loaded a whole group of
+    // kGroup rows ahead of their use: kGroup rows of loads stay in flight
+    constexpr int kGroup = 4;
+    auto fetch = [&](int r) {
+        uint2 v = make_uint2(0u, 0u);
+        if (live && r >= 0 && r < T) {
+            v.x = *reinterpret_cast<const uint32_t*>(a.x + (row0 + r) * D + c);
+            if (r >= t0) v.y = *reinterpret_cast<const uint32_t*>(a.dy + (row0 + r) * D + c);
         }
+        return v;
     };
-    RawRow<CH> xr0 = {}, xr1 = {}, xr2 = {}, dr0 = {}, dr1 = {}, dr2 = {};
-    float x00 = 0.f, x01 = 0.f, x02 = 0.f;
-    fetch(t0 - 3, xr0, x00, dr0);
-    fetch(t0 - 2, xr1, x01, dr1);
+    uint2 cur[kGroup], nxt[kGroup];
+#pragma unroll
+    for (int i = 0; i < kGroup; ++i) cur[i] = fetch(t0 - 3 + i);
 
-    for (int p = t0 - 3; p <= t1 + 2; ++p) {
-        const int s = (p + 4) & 3;
-        fetch(p + 2, xr2, x02, dr2);
+    auto row = [&](int p, const uint2 f0) {
+        const float2 st = st_s[p - (t0 - 3)];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+            rs[j] = rs[j + 1];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                xn[j][e] = xn[j + 1][e];
+                xh[j][e] = xh[j + 1][e];
+                du[j][e] = du[j + 1][e];
+            }
+        }
         // (1) conv input of row p
-        float xnv[CH] = {}, xhv[CH] = {};
-        float rs = 1.f;
         if (p < 0) {
-            if (cs_in) ldv_f32<CH>(cs_in + (static_cast<int64_t>(b) * 3 + p + 3) * D + c, xnv);
+            const bool hv = live && a.cs_in;
+            const float* src = a.cs_in + (static_cast<int64_t>(b) * 3 + p + 3) * D + c;
+            xn[3][0] = hv ? src[0] : 0.f;
+            xn[3][1] = hv ? src[1] : 0.f;
+            xh[3][0] = xh[3][1] = 0.f;
+            rs[3] = 1.f;
         } else if (p < T) {
-            float v[CH];
-            unpack_raw<CH>(xr0, v);
-            if (apply_ln) {
-                const float x0 = x00;   // shift: the row's first element
-                float s1 = 0.f, s2 = 0.f;
-#pragma unroll
-                for (int e = 0; e < CH; ++e) {
-                    s1 += v[e] - x0;
-                    s2 = fmaf(v[e] - x0, v[e] - x0, s2);
-                }
-                block_sum2(s1, s2, red, turn);
-                const float m1 = s1 / D;
-                const float var = fmaxf(s2 / D - m1 * m1, 0.f);
-                const float mean = x0 + m1;
-                rs = rsqrtf(var + eps);
-#pragma unroll
-                for (int e = 0; e < CH; ++e) {
-                    xhv[e] = (v[e] - mean) * rs;
-                    xnv[e] = fmaf(xhv[e], g4(e), be4(e));
-                }
+            const float v0 = bf16_lo(f0.x), v1 = bf16_hi(f0.x);
+            if (ln) {
+                xh[3][0] = (v0 - st.x) * st.y;
+                xh[3][1] = (v1 - st.x) * st.y;
+                xn[3][0] = fmaf(xh[3][0], gm[0], bt[0]);
+                xn[3][1] = fmaf(xh[3][1], gm[1], bt[1]);
+                rs[3] = st.y;
             } else {
-#pragma unroll
-                for (int e = 0; e < CH; ++e) xnv[e] = xhv[e] = v[e];
+                xh[3][0] = xn[3][0] = v0;
+                xh[3][1] = xn[3][1] = v1;
+                rs[3] = 1.f;
             }
+        } else {
+            xn[3][0] = xn[3][1] = xh[3][0] = xh[3][1] = 0.f;
+            rs[3] = 1.f;
         }
-        rs_r[s] = rs;
-        stv_f32<CH>(xn_r + s * D + c, xnv);
-        stv_f32<CH>(xh_r + s * D + c, xhv);
-
         // (2) du of row p (rows t0 .. T-1; zero elsewhere)
-        float duv[CH] = {};
         if (p >= t0 && p < T) {
-            float dyv[CH];
-            unpack_raw<CH>(dr0, dyv);
-            float win[4][CH];   // xn of rows p-3 .. p: vector loads, conflict-free
+            const float dyv[2] = {bf16_lo(f0.y), bf16_hi(f0.y)};
 #pragma unroll
-            for (int j = 0; j < 3; ++j) ldv_f32<CH>(xn_r + ((p + 1 + j) & 3) * D + c, win[j]);
+            for (int e = 0; e < 2; ++e) {
+                float u = bi[e];
 #pragma unroll
-            for (int e = 0; e < CH; ++e) win[3][e] = xnv[e];
-#pragma unroll
-            for (int e = 0; e < CH; ++e) {
-                float u = bi4(e);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) u = fmaf(wv[e][j], win[j][e], u);
-                const float sg = 1.f / (1.f + expf(-u));
-                duv[e] = dyv[e] * sg * fmaf(u, 1.f - sg, 1.f);
+                for (int j = 0; j < 4; ++j) u = fmaf(wv[e][j], xn[j][e], u);
+                // sigmoid with the fast exponential and division intrinsics:
+                // about 2 ulp, far below the bf16 rounding of dx
+                const float sg = __fdividef(1.f, 1.f + __expf(-u));
+                du[3][e] = dyv[e] * sg * fmaf(u, 1.f - sg, 1.f);
             }
-            if (p < t1) {
+            if (!FINISH && p < t1) {
 #pragma unroll
-                for (int e = 0; e < CH; ++e) {
-                    pdb[e] += duv[e];
+                for (int e = 0; e < 2; ++e) {
+                    pdb[e] += du[3][e];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) pdw[j][e] = fmaf(duv[e], win[j][e], pdw[j][e]);
+                    for (int j = 0; j < 4; ++j) pdw[j][e] = fmaf(du[3][e], xn[j][e], pdw[j][e]);
                 }
             }
+        } else {
+            du[3][0] = du[3][1] = 0.f;
         }
-        stv_f32<CH>(du_r + s * D + c, duv);
-
-        // (3) dxn and dx of row q = p - 3
+        // (3) dxn of row q = p - 3, then its LayerNorm backward
         const int q = p - 3;
         const bool out_row = q >= t0 && q < t1;
         const bool hist_row = t0 == 0 && q < 0 && q >= -3;   // rows -3 .. -1: the history
         if (out_row || hist_row) {
-            float d4[3][CH];   // du of rows q .. q+2 (row q+3 = p is in registers)
+            float dxn[2];
 #pragma unroll
-            for (int j = 0; j < 3; ++j) ldv_f32<CH>(du_r + ((q + 4 + j) & 3) * D + c, d4[j]);
-            float dxn[CH];
-#pragma unroll
-            for (int e = 0; e < CH; ++e)
-                dxn[e] = wv[e][3] * d4[0][e] + wv[e][2] * d4[1][e] + wv[e][1] * d4[2][e] + wv[e][0] * duv[e];
+            for (int e = 0; e < 2; ++e)
+                dxn[e] = wv[e][3] * du[0][e] + wv[e][2] * du[1][e] + wv[e][1] * du[2][e] + wv[e][0] * du[3][e];
             if (hist_row) {
-                if (dcs) stv_f32<CH>(dcs + (static_cast<int64_t>(b) * 3 + q + 3) * D + c, dxn);
-            } else {
-                float o[CH];
-                if (apply_ln) {
-                    const int sq = (q + 4) & 3;
-                    float xh[CH];
-                    ldv_f32<CH>(xh_r + sq * D + c, xh);
-                    float sg = 0.f, sgh = 0.f, gg[CH];
+                if (!FINISH && live && a.dcs) {
+                    float* dst = a.dcs + (static_cast<int64_t>(b) * 3 + q + 3) * D + c;
+                    dst[0] = dxn[0];
+                    dst[1] = dxn[1];
+                }
+            } else if (ln) {
+                const float g0 = dxn[0] * gm[0], g1 = dxn[1] * gm[1];
+                if (!FINISH) {
+                    const float sgv = warp_sum_bwd(g0 + g1);
+                    const float sghv = warp_sum_bwd(fmaf(g0, xh[0][0], g1 * xh[0][1]));
+                    if (lane == 0) rowsum[q - t0][warp] = make_float2(sgv, sghv);
 #pragma unroll
-                    for (int e = 0; e < CH; ++e) {
-                        gg[e] = dxn[e] * g4(e);
-                        sg += gg[e];
-                        sgh = fmaf(gg[e], xh[e], sgh);
-                        pdg[e] = fmaf(dxn[e], xh[e], pdg[e]);
+                    for (int e = 0; e < 2; ++e) {
+                        pdg[e] = fmaf(dxn[e], xh[0][e], pdg[e]);
                         pdbe[e] += dxn[e];
                     }
-                    block_sum2(sg, sgh, red, turn);
-                    const float mg = sg / D, mgh = sgh / D, r = rs_r[sq];
-#pragma unroll
-                    for (int e = 0; e < CH; ++e) o[e] = r * (gg[e] - mg - xh[e] * mgh);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < CH; ++e) o[e] = dxn[e];
+                } else if (live) {
+                    const float2 tt = total[q - t0];
+                    const float mg = tt.x / D, mgh = tt.y / D;
+                    const float o0 = rs[0] * (g0 - mg - xh[0][0] * mgh);
+                    const float o1 = rs[0] * (g1 - mg - xh[0][1] * mgh);
+                    *reinterpret_cast<uint32_t*>(a.dx + (row0 + q) * D + c) = pack_bf16(o0, o1);
                 }
-                stv_bf16<CH>(dx + (row0 + q) * D + c, o);
+            } else if (!FINISH && live) {
+                *reinterpret_cast<uint32_t*>(a.dx + (row0 + q) * D + c) = pack_bf16(dxn[0], dxn[1]);
             }
         }
-        xr0 = xr1;
-        xr1 = xr2;
-        dr0 = dr1;
-        dr1 = dr2;
-        x00 = x01;
-        x01 = x02;
+    };
+
+    for (int p0 = t0 - 3; p0 <= t1 + 2; p0 += kGroup) {
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) nxt[i] = fetch(p0 + kGroup + i);
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i)
+            if (p0 + i <= t1 + 2) row(p0 + i, cur[i]);
+#pragma unroll
+        for (int i = 0; i < kGroup; ++i) cur[i] = nxt[i];
     }
 
-    // per-CTA partials: rows dw tap 0..3, dbias, dgamma, dbeta
-    float* pp = part + (static_cast<int64_t>(b) * gridDim.x + blk) * kParts * D + c;
+    if (!FINISH) {
+        // per-row sums over this tile's channels, in warp order
+        if (ln) {
+            __syncthreads();
+            for (int i = tid; i < t1 - t0; i += kTileThreads) {
+                float sg = 0.f, sgh = 0.f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) stv_f32<CH>(pp + j * D, pdw[j]);
-    stv_f32<CH>(pp + 4 * D, pdb);
-    stv_f32<CH>(pp + 5 * D, pdg);
-    stv_f32<CH>(pp + 6 * D, pdbe);
+                for (int k = 0; k < kTileThreads / 32; ++k) {
+                    sg += rowsum[i][k].x;
+                    sgh += rowsum[i][k].y;
+                }
+                a.psum[(row0 + t0 + i) * a.CB + cb] = make_float2(sg, sgh);
+            }
+        }
+        // per-tile partials: dw taps 0..3, dbias, dgamma, dbeta
+        if (live) {
+            float* pp = a.part + (static_cast<int64_t>(b) * a.nrb + rb) * kParts * D + c;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) *reinterpret_cast<float2*>(pp + j * D) = make_float2(pdw[j][0], pdw[j][1]);
+            *reinterpret_cast<float2*>(pp + 4 * D) = make_float2(pdb[0], pdb[1]);
+            *reinterpret_cast<float2*>(pp + 5 * D) = make_float2(pdg[0], pdg[1]);
+            *reinterpret_cast<float2*>(pp + 6 * D) = make_float2(pdbe[0], pdbe[1]);
+        }
+    }
 }
 
 // Sum of the per-CTA partials in CTA order: thread per (part, channel).
@@ -336,33 +314,67 @@ __global__ void __launch_bounds__(256) conv_bwd_reduce_kernel(const float* __res
 
 }  // namespace
 
+// part [B * nrb][7][D] | stats [B*T] float2 | psum [B*T][CB] float2
 size_t conv_bwd_workspace_bytes(int B, int T, int D)
 {
-    const size_t nblk = static_cast<size_t>((T + kRows - 1) / kRows);
-    return static_cast<size_t>(B) * nblk * kParts * D * sizeof(float);
+    const size_t nrb = static_cast<size_t>((T + kRows - 1) / kRows), CB = (D + kTileCh - 1) / kTileCh;
+    const size_t rows = static_cast<size_t>(B) * T;
+    return align256(static_cast<size_t>(B) * nrb * kParts * D * sizeof(float)) + align256(rows * sizeof(float2)) +
+           align256(rows * CB * sizeof(float2));
 }
 
 gla_status launch_conv_bwd(const void* x, int apply_ln, const float* g, const float* be, float eps, const float* w,
                            const float* bias, const float* cs_in, const void* dy, void* dx, float* dw, float* dbias,
                            float* dgamma, float* dbeta, float* dcs, void* ws, int B, int T, int D, cudaStream_t st)
 {
-    const int nblk = (T + kRows - 1) / kRows;
-    const size_t smem = ((D <= 3072 ? 15 : 12) * static_cast<size_t>(D) + 128) * sizeof(float);
-    const bool narrow = D <= 3072;
-    auto kern = narrow ? conv_bwd_kernel<4> : conv_bwd_kernel<8>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
-        return check_launch("cudaFuncSetAttribute");
-    float* part = static_cast<float*>(ws);
+    const int nrb = (T + kRows - 1) / kRows, CB = (D + kTileCh - 1) / kTileCh;
+    const size_t rows = static_cast<size_t>(B) * T;
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    TileArgs a;
+    a.x = static_cast<const __nv_bfloat16*>(x);
+    a.dy = static_cast<const __nv_bfloat16*>(dy);
+    a.gamma = g;
+    a.beta = be;
+    a.w = w;
+    a.bias = bias;
+    a.cs_in = cs_in;
+    a.part = reinterpret_cast<float*>(wsb);
+    size_t off = align256(static_cast<size_t>(B) * nrb * kParts * D * sizeof(float));
+    float2* stats = reinterpret_cast<float2*>(wsb + off);
+    off += align256(rows * sizeof(float2));
+    a.stats = stats;
+    a.psum = reinterpret_cast<float2*>(wsb + off);
+    a.dcs = dcs;
+    a.dx = static_cast<__nv_bfloat16*>(dx);
+    a.T = T;
+    a.D = D;
+    a.CB = CB;
+    a.nrb = nrb;
+    a.apply_ln = apply_ln;
+    gla_status s;
+    if (apply_ln) {
+        trace_begin(st);
+        ln_stats_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(a.x, static_cast<int>(rows), D, eps,
+                                                                              stats);
+        trace_end(st, "ln_stats_kernel");
+        count_launch();
+        if ((s = check_launch("ln_stats_kernel")) != GLA_OK) return s;
+    }
+    const dim3 grid(nrb, B, CB);
     trace_begin(st);
-    kern<<<dim3(nblk, B), D / (narrow ? 4 : 8), smem, st>>>(
-        static_cast<const __nv_bfloat16*>(x), apply_ln, g, be, eps, w, bias, cs_in,
-        static_cast<const __nv_bfloat16*>(dy), static_cast<__nv_bfloat16*>(dx), dcs, part, T, D);
-    trace_end(st, "conv_bwd_kernel");
+    conv_bwd_tile_kernel<false><<<grid, kTileThreads, 0, st>>>(a);
+    trace_end(st, "conv_bwd_tile_kernel");
     count_launch();
-    gla_status s = check_launch("conv_bwd_kernel");
-    if (s != GLA_OK) return s;
+    if ((s = check_launch("conv_bwd_tile_kernel")) != GLA_OK) return s;
+    if (apply_ln) {
+        trace_begin(st);
+        conv_bwd_tile_kernel<true><<<grid, kTileThreads, 0, st>>>(a);
+        trace_end(st, "conv_bwd_dx_kernel");
+        count_launch();
+        if ((s = check_launch("conv_bwd_dx_kernel")) != GLA_OK) return s;
+    }
     trace_begin(st);
-    conv_bwd_reduce_kernel<<<(kParts * D + 255) / 256, 256, 0, st>>>(part, B * nblk, D, dw, dbias, dgamma, dbeta);
+    conv_bwd_reduce_kernel<<<(kParts * D + 255) / 256, 256, 0, st>>>(a.part, B * nrb, D, dw, dbias, dgamma, dbeta);
     trace_end(st, "conv_bwd_reduce_kernel");
     count_launch();
     return check_launch("conv_bwd_reduce_kernel");

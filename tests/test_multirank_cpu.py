@@ -153,6 +153,6 @@ def _seqpar_rank(rank, world, lengths):
     np.testing.assert_allclose(grads[4].numpy(), ref[4], rtol=1e-9, atol=1e-11)
 
 
-@pytest.mark.parametrize("lengths", [[9, 14], [5, 0, 9], [1, 7, 3]])
+@pytest.mark.parametrize("lengths", [[9, 14], [5, 0, 9], [1, 7, 3], [3, 0, 5, 2]])
 def test_seqpar_split_over_gloo_ranks_matches_unsplit(lengths):
     _spawn(_seqpar_rank, len(lengths), lengths)

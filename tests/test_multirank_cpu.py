@@ -4,7 +4,7 @@
     every rank takes part in;
   * bench.py --impl reference under torchrun with two ranks: rank 0 alone
     runs the oracle and prints one JSON line, the other rank exits 0;
-  * the sequence split (linear_attention_simple_b200.seqpar) over 2 and 3
+  * the sequence split (linear_attention_simple_b200.seqpar) over 2, 3 and 4
     ranks, with an oracle-backed set of per-segment calls standing in for
     libgla's kernels, against the oracle run on the unsplit sequence.  This
     checks the exchange, the rank order and the direction of each fold; the

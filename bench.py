@@ -7,7 +7,9 @@ H = 16, dk = 96, dv = 192 in bf16: gla_chunk_fwd followed by gla_chunk_bwd
 chunk fwd+bwd tokens/s over all ranks.  The metric also names decode
 tokens/s at 1,280 sequences, so the same run times the 24-layer decode step
 (1,280 sequences x 24 layers x 16 heads, fp32 state in place) and reports
-it under "decode".
+it under "decode", and the long-context prefill (T = 65,536: the LayerNorm +
+conv + SiLU front end, then the chunked forward with S_0) under
+"long_prefill", each call against its HBM roofline.
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
 cuda synchronize, measured with CUDA events on the launching stream, max
@@ -24,7 +26,7 @@ files still matches the one recorded there; otherwise it is null.
 
 --skip-decode / --skip-e2e time only the training step: the command the
 profiles' ncu captures run (a few GB on the device instead of the 36 GB of
-decode state).
+decode state); --skip-decode also skips the long prefill.
 """
 import hashlib
 import argparse
@@ -48,6 +50,7 @@ from linear_attention_simple_b200.configs import WORKLOADS  # noqa: E402
 METRIC = "GLA chunk fwd+bwd tokens/s; decode tokens/s at 1280 seqs; % of roofline"
 TRAIN = WORKLOADS["train_fwd_bwd_b8_t2048"]
 DECODE = WORKLOADS["decode_n1280_l24"]
+LONG = WORKLOADS["long_prefill_t65536"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # Algorithmic bytes per unit (one (batch, head, 128-token chunk) unless
@@ -353,10 +356,17 @@ def run_ours(args, ws, rank, local):
 
     # ---- decode step at 1280 sequences x 24 layers
     dec = None if args.skip_decode else run_decode(args, ws, peaks, peak_kind)
+    # ---- long-context prefill: front end, then the chunked forward at T = 65,536
+    lp = None
+    if not args.skip_decode:
+        try:
+            lp = run_long_prefill(args, ws, peaks, peak_kind)
+        except Exception as e:          # reported, never at the cost of the lines above
+            lp = {"error": ("%s: %s" % (type(e).__name__, e))[:300]}
     clk = clocks.stop()
     if clk is not None:
-        clk["region"] = "fwd+bwd and decode timed regions"
-    run_tail(args, ws, rank, value, ms_step, roof, shares, e2e, launches, clk, dec)
+        clk["region"] = "fwd+bwd, decode and long-prefill timed regions"
+    run_tail(args, ws, rank, value, ms_step, roof, shares, e2e, launches, clk, dec, lp)
 
 
 def run_e2e(args, ws, d, st):
@@ -432,7 +442,7 @@ def run_e2e(args, ws, d, st):
             "steps": e_steps, "overlap": "copy-in, compute and copy-out of consecutive steps on three streams"}
 
 
-def run_tail(args, ws, rank, value, ms_step, roof, shares, e2e, launches, clk, dec):
+def run_tail(args, ws, rank, value, ms_step, roof, shares, e2e, launches, clk, dec, lp=None):
     w = TRAIN
     # ---- oracle on the host cores (rank 0, N = 1 only)
     cpu = None
@@ -458,7 +468,7 @@ def run_tail(args, ws, rank, value, ms_step, roof, shares, e2e, launches, clk, d
                            "heads": w.H, "dk": w.dk, "dv": w.dv, "parallelism": "dp%d" % ws,
                            "l2": "inputs larger than L2 (no flush)"},
                 "roofline": roof, "kernel_shares": shares, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches, "clocks": clk, "decode": dec}
+                "gpu_launches": launches, "clocks": clk, "decode": dec, "long_prefill": lp}
         print(json.dumps(line), flush=True)
 
 
@@ -495,6 +505,63 @@ def run_decode(args, ws, peaks, peak_kind):
                         "frac_of_8tbs": round(achieved / 8000.0, 4),
                         "peak_source": "%s copy bandwidth" % peak_kind}}
     del layers, outs
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_long_prefill(args, ws, peaks, peak_kind):
+    """Long-context prefill at T = 65,536 (B = 1, H = 16, D = 3,072): the
+    LayerNorm + conv + SiLU front end over x, then the chunked forward with
+    S_0 on independent q, k, v (their projection is not part of the path).
+    Each call is timed on its own, K launches between two events."""
+    w = LONG
+    st = torch.cuda.current_stream()
+    f = inputs.front_inputs(w.B, w.T, w.D, w.W, seed=w.seed, device="cuda")
+    y = torch.empty_like(f["x"])
+    d = inputs.chunk_inputs(w.B, w.T, w.H, w.dk, w.dv, seed=w.seed, device="cuda", s0_std=w.s0_std)
+    o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.bfloat16, device="cuda")
+    sf = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device="cuda")
+    wsf = torch.empty(max(1, gla.gla_chunk_workspace_bytes(w.B, w.T, w.H)), dtype=torch.uint8, device="cuda")
+
+    def front():
+        gla.conv1d_silu_causal(f["x"], f["w"], y=y)
+
+    def mixer():
+        gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], s0=d["s0"], o=o, s_final=sf, ws=wsf)
+
+    def timed(fn, n):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        barrier(ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(n):
+            fn()
+        e1.record(st)
+        e1.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1) / 1e3 / n, ws)
+
+    n = max(1, min(args.steps, 20))
+    t_front, t_mix = timed(front, n), timed(mixer, n)
+    front_bytes = w.B * w.T * w.D * 4                       # x in, y out (bf16)
+    units = w.B * w.H * ((w.T + 127) // 128)
+    mix_bytes = CHUNK_BYTES["chunk_fwd_fused_kernel"] * units + 2 * FS * w.B * w.H   # + S_0 in, S_T out
+
+    def roof(kernel, nbytes, t):
+        a = nbytes / t / 1e9
+        return {"kernel": kernel, "bound": "hbm", "achieved": round(a, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(a / peaks["hbm_gbs"], 4), "bytes_per_launch": nbytes,
+                "peak_source": "%s copy bandwidth" % peak_kind}
+
+    out = {"value": round(ws * w.B * w.T / (t_front + t_mix), 1), "unit": "tokens/s", "workload": w.name,
+           "ms_per_step": round((t_front + t_mix) * 1e3, 4),
+           "front_end": {"us_per_launch": round(t_front * 1e6, 2),
+                         "roofline": roof("ln_conv_silu_kernel", front_bytes, t_front)},
+           "gla_fwd": {"us_per_launch": round(t_mix * 1e6, 2),
+                       "roofline": roof("gla_chunk_fwd (segmented: state pre-pass, combine, fused pass)",
+                                        mix_bytes, t_mix)}}
+    del f, y, d, o, sf, wsf
     torch.cuda.empty_cache()
     return out
 

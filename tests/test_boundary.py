@@ -266,3 +266,32 @@ def test_product_does_not_import_the_oracle():
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
                 assert "gla_oracle" not in src, f
+
+
+def test_bindings_reject_host_tensors(L):
+    """Every binding refuses CPU tensors before any call into the library:
+    there is no host fallback for any step."""
+    import torch
+    bf = lambda *s: torch.zeros(s, dtype=torch.bfloat16)  # noqa: E731
+    f32 = lambda *s: torch.zeros(s, dtype=torch.float32)  # noqa: E731
+    B, T, H = 1, 4, 2
+    q, k, v, a = bf(B, T, H, 96), bf(B, T, H, 96), bf(B, T, H, 192), f32(B, T, H)
+    calls = [
+        lambda: gla.gla_chunk_fwd(q, k, v, a),
+        lambda: gla.gla_chunk_bwd(q, k, v, a, bf(B, T, H, 192)),
+        lambda: gla.gla_decode_step(f32(2, H, 96, 192), bf(2, H, 96), bf(2, H, 96), bf(2, H, 192), f32(2, H)),
+        lambda: gla.conv1d_silu_causal(bf(1, T, 64), f32(64, 4)),
+        lambda: gla.conv1d_silu_decode_step(bf(2, 64), f32(64, 4), f32(2, 3, 64)),
+        lambda: gla.conv1d_silu_causal_bwd(bf(1, T, 64), f32(64, 4), bf(1, T, 64)),
+        lambda: gla.gla_chunk_fwd_varlen(bf(T, H, 96), bf(T, H, 96), bf(T, H, 192), f32(T, H),
+                                         torch.tensor([0, T], dtype=torch.int32)),
+        lambda: gla.gla_segment_state_fwd(k, v, a),
+        lambda: gla.gla_segment_state_bwd(q, bf(B, T, H, 192), a),
+        lambda: gla.gla_state_fold(f32(2, B, H, 96, 192), f32(2, B, H)),
+        lambda: gla.gla_chunk_fwd_noalloc(q, k, v, a),
+    ]
+    for call in calls:
+        # rejected by the binding itself, not by the library (a GlaError would
+        # mean host pointers reached libgla)
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            call()

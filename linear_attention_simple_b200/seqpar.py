@@ -27,6 +27,10 @@ most, once per call.
 The two phases are separate functions (``fwd_local`` / ``fwd_finish``,
 ``bwd_local`` / ``bwd_finish``) so that callers can run the exchange
 themselves, e.g. all ranks' phases one after another on one device.
+
+``ops`` is the set of per-segment calls the phases make: ``LibglaOps``
+(libgla's kernels) unless a caller passes another.  The package defines no
+other set; the tests pass a host one to check the exchange on CPU ranks.
 """
 import torch
 import torch.distributed as dist

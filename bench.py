@@ -15,14 +15,23 @@ Timing: W untimed warm-up steps, then K steps bracketed by a barrier and
 cuda synchronize, measured with CUDA events on the launching stream, max
 over ranks.  Inputs (about 0.6 GB per rank for the training step, 36 GB of
 decode state) are larger than the 126 MB L2, so no flush is needed.
-Roofline: right after the timed region the same K steps run again with
-libgla's per-launch event tracing (events between launches cost a few
-percent, so they stay out of the headline region); the dominant kernel's
-algorithmic bytes (or flops) per launch divided by its mean launch time,
-against MEASURED_PEAKS.json.  Its
-"traffic" (DRAM bytes per launch) comes from the ncu capture summarised in
-profiles/dram_traffic.md, and only while the digest of the kernel's source
-files still matches the one recorded there; otherwise it is null.
+Rooflines, all against MEASURED_PEAKS.json:
+  roofline       the dominant kernel: right after the timed region the same K
+                 steps run again with libgla's per-launch event tracing
+                 (events between launches cost a few percent, so they stay
+                 out of the headline region); its method bytes (the inputs
+                 and outputs of the computation it reads or writes) per
+                 launch over its mean launch time against HBM copy bandwidth,
+                 with its design bytes (per-chunk states, partial sums) and
+                 its bf16 tensor-core fraction beside it;
+  roofline_step  the whole step: 3,084 method bytes per token-head (+ the
+                 final state) against HBM, 64.5 MF of algorithmic flops per
+                 (batch, head, chunk) against the sustained bf16 peak;
+  prefill_fwd    the forward alone at the same shape, both rooflines.
+The dominant kernel's "traffic" (DRAM bytes per launch) comes from the ncu
+capture summarised in profiles/dram_traffic.md, and only while the digest of
+the kernel's source files still matches the one recorded there; otherwise it
+is null.
 
 --skip-decode / --skip-e2e time only the training step: the command the
 profiles' ncu captures run (a few GB on the device instead of the 36 GB of
@@ -53,28 +62,50 @@ DECODE = WORKLOADS["decode_n1280_l24"]
 LONG = WORKLOADS["long_prefill_t65536"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# Algorithmic bytes per unit (one (batch, head, 128-token chunk) unless
-# stated), used for each kernel's roofline.  bf16 tiles: q, k 24,576 B; v, o,
-# dO 49,152 B; a 512 B; bf16 per-chunk state 36,864 B; fp32 state 73,728 B.
+# Byte and flop models per unit = one (batch, head, 128-token chunk).  bf16
+# tiles: q, k 24,576 B; v, o, dO 49,152 B; a 512 B; one bf16 plane of a
+# per-chunk state 36,864 B; an fp32 state 73,728 B.
 QK, VO, A, HS, FS = 24576, 49152, 512, 36864, 73728
-CHUNK_BYTES = {
-    # fused forward: read q, k, v, a; write o          (+ S_T per head)
-    "chunk_fwd_fused_kernel": 2 * QK + 2 * VO + A,
-    # state recompute: read k, v, a; write h_c          (+ S_T per head if dS_T)
-    "chunk_state_fwd_kernel": QK + VO + A + HS,
-    # state-gradient pass: read q, dO, a; write D_c     (+ dS_0 per head)
-    "chunk_state_rev_kernel": QK + VO + A + HS,
-    # dq/dk: read q, k, v, dO, h, D, a; write dq, dk, q.dq and k.dk per token
-    "bwd_dqdk_kernel": 2 * QK + 2 * VO + 2 * HS + A + 2 * QK + 2 * A,
-    # da: read q.dq, k.dk; write da
-    "da_finish_kernel": 3 * A,
-    # dv: read q, k, dO, D, a; write dv
-    "bwd_dv_kernel": 2 * QK + VO + HS + A + VO,
+# Method bytes: the inputs and outputs of the computation itself (q, k, v, a
+# in and o out forward; q, k, v, dO, a in and dq, dk, dv, da out backward),
+# counted for the kernel that reads or writes them.  The roofline fraction is
+# taken on these.
+METHOD_BYTES = {
+    "chunk_fwd_fused_kernel": 2 * QK + 2 * VO + A,      # q, k, v, a in; o out   (+ S_T per head)
+    "chunk_state_fwd_kernel": QK + VO + A,              # k, v, a in
+    "chunk_state_rev_kernel": QK + VO + A,              # q, dO, a in
+    "bwd_dqdk_kernel": 2 * QK + 2 * VO + A + 2 * QK,    # q, k, v, dO, a in; dq, dk out
+    "bwd_dv_kernel": 2 * QK + VO + A + VO,              # q, k, dO, a in; dv out
+    "da_finish_kernel": A,                              # da out
 }
+# Design bytes: intermediates the kernels exchange through HBM (the
+# per-chunk states as bf16 hi + lo planes, the per-token halves of the da
+# sum), reported beside the method bytes and not counted in the fraction.
+DESIGN_BYTES = {
+    "chunk_state_fwd_kernel": 2 * HS,                   # h_c written (hi, lo)
+    "chunk_state_rev_kernel": 2 * HS,                   # D_c written (hi, lo)
+    "bwd_dqdk_kernel": 2 * 2 * HS + 2 * A,              # h_c, D_c read (hi, lo); q.dq, k.dk written
+    "bwd_dv_kernel": HS,                                # D_c read (hi plane)
+    "da_finish_kernel": 2 * A,                          # q.dq, k.dk read
+}
+# Algorithmic flops per unit on dense 128-token tiles (2 m n k per product;
+# the hi + lo splits the kernels make for precision are not counted).
+MM = lambda m, n, k: 2 * m * n * k  # noqa: E731
 CHUNK_FLOPS = {
-    # 2*(128*128*96 + 128*192*96 + 128*192*128 + 96*192*128), dense tiles
-    "chunk_fwd_fused_kernel": 2 * (128 * 128 * 96 + 128 * 192 * 96 + 128 * 192 * 128 + 96 * 192 * 128),
+    # scores Q K^T, Q S_prev, P V, state update K~^T V
+    "chunk_fwd_fused_kernel": MM(128, 128, 96) + MM(128, 192, 96) + MM(128, 192, 128) + MM(96, 192, 128),
+    "chunk_state_fwd_kernel": MM(96, 192, 128),          # K~^T V
+    "chunk_state_rev_kernel": MM(96, 192, 128),          # Q~^T dO
+    # dP = dO V^T, dO h^T, dP K, V D^T, dP^T Q
+    "bwd_dqdk_kernel": MM(128, 128, 192) + 2 * MM(128, 96, 192) + 2 * MM(128, 96, 128),
+    # scores^T K Q^T, P~ dO, K D
+    "bwd_dv_kernel": MM(128, 128, 96) + MM(128, 192, 128) + MM(128, 192, 96),
 }
+# The whole training step per unit: forward (q, k, v, a in, o out) and
+# backward (q, k, v, dO, a in; dq, dk, dv, da out) method bytes, and the
+# forward + backward algorithmic flops.
+STEP_BYTES = (2 * QK + 2 * VO + A) + (2 * QK + 2 * VO + A + 2 * QK + VO + A)
+STEP_FLOPS = sum(CHUNK_FLOPS.values())
 
 
 # Source files each kernel is built from (the digest that ties a recorded
@@ -228,27 +259,57 @@ def train_step(d):
 
 
 def kernel_roofline(summary, peaks, peak_kind, units_per_launch, B, H):
-    """Roofline of the kernel with the largest summed time in the trace."""
+    """Roofline of the kernel with the largest summed time in the trace:
+    HBM on its method bytes (the fraction), with its design bytes and its
+    bf16 tensor-core fraction beside it."""
     if not summary:
         return None, None
     name, launches, total_ms = max(summary, key=lambda r: r[2])
     mean_s = total_ms / launches / 1e3
-    if name in CHUNK_BYTES:
-        bytes_per_launch = CHUNK_BYTES[name] * units_per_launch
+    if name in METHOD_BYTES:
+        bytes_per_launch = METHOD_BYTES[name] * units_per_launch
         if name in ("chunk_fwd_fused_kernel",):
             bytes_per_launch += FS * B * H          # final state written per head
+        design = DESIGN_BYTES.get(name, 0) * units_per_launch
         achieved = bytes_per_launch / mean_s / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                 "unit": "GB/s", "frac": round(achieved / peak, 4),
-                "bytes_per_launch": bytes_per_launch, "mean_launch_us": round(mean_s * 1e6, 2),
+                "bytes_per_launch": bytes_per_launch, "bytes": "method (inputs and outputs of the path)",
+                "design_bytes_per_launch": design,
+                "frac_incl_design_bytes": round((bytes_per_launch + design) / mean_s / 1e9 / peak, 4),
+                "mean_launch_us": round(mean_s * 1e6, 2),
                 "traffic": recorded_traffic(name), "source_digest": kernel_digest(name),
                 "peak_source": "%s copy bandwidth" % peak_kind}
+        if name in CHUNK_FLOPS:
+            tf = CHUNK_FLOPS[name] * units_per_launch / mean_s / 1e12
+            tpk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+            roof["tensor"] = {"achieved": round(tf, 1), "peak": tpk, "unit": "TFLOP/s",
+                              "frac": round(tf / tpk, 4),
+                              "flops_per_launch": CHUNK_FLOPS[name] * units_per_launch,
+                              "peak_source": "%s bf16 dense, sustained" % peak_kind}
     else:
         roof = {"kernel": name, "bound": None, "achieved": None, "peak": None, "unit": None,
                 "frac": None, "traffic": None, "mean_launch_us": round(mean_s * 1e6, 2)}
     shares = {n: round(t / sum(r[2] for r in summary), 4) for n, _, t in summary}
     return roof, shares
+
+
+def step_roofline(step_s, units, B, H, peaks, peak_kind):
+    """The training step as a whole against both rooflines: its method bytes
+    (+ the final state the forward writes) over HBM, its algorithmic flops
+    over the sustained bf16 tensor-core peak."""
+    nbytes = STEP_BYTES * units + FS * B * H
+    flops = STEP_FLOPS * units
+    gbs = nbytes / step_s / 1e9
+    tfs = flops / step_s / 1e12
+    tpk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    return {"hbm": {"achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_step": nbytes,
+                    "peak_source": "%s copy bandwidth" % peak_kind},
+            "tensor": {"achieved": round(tfs, 1), "peak": tpk, "unit": "TFLOP/s", "frac": round(tfs / tpk, 4),
+                       "flops_per_step": flops, "peak_source": "%s bf16 dense, sustained" % peak_kind},
+            "ms_per_step": round(step_s * 1e3, 4)}
 
 
 # ------------------------------------------------------------ oracle arm
@@ -344,6 +405,9 @@ def run_ours(args, ws, rank, local):
     torch.cuda.synchronize()
     roof, shares = kernel_roofline([(n, c, t) for n, c, t in summary], peaks, peak_kind,
                                    units_per_launch, w.B, w.H)
+    roof_step = step_roofline(elapsed / args.steps, units_per_launch, w.B, w.H, peaks, peak_kind)
+    # ---- prefill: the forward alone at the same shape
+    pre = run_prefill(args, ws, d, st, peaks, peak_kind, units_per_launch)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -366,7 +430,43 @@ def run_ours(args, ws, rank, local):
     clk = clocks.stop()
     if clk is not None:
         clk["region"] = "fwd+bwd, decode and long-prefill timed regions"
-    run_tail(args, ws, rank, value, ms_step, roof, shares, e2e, launches, clk, dec, lp)
+    run_tail(args, ws, rank, value, ms_step, roof, shares, e2e, launches, clk, dec, lp,
+             roof_step=roof_step, prefill=pre)
+
+
+def run_prefill(args, ws, d, st, peaks, peak_kind, units):
+    """Prefill forward alone (gla_chunk_fwd at B8 H16 T2048, S_T written),
+    K launches between two events on the launching stream: tokens/s and both
+    rooflines on its method bytes (q, k, v, a in, o and S_T out) and its
+    algorithmic flops."""
+    w = TRAIN
+
+    def fwd():
+        gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], o=d["o"], s_final=d["sf"], ws=d["ws_f"])
+
+    for _ in range(max(3, args.warmup)):
+        fwd()
+    torch.cuda.synchronize()
+    barrier(ws)
+    n = max(1, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(n):
+        fwd()
+    e1.record(st)
+    e1.synchronize()
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3 / n, ws)
+    nbytes = METHOD_BYTES["chunk_fwd_fused_kernel"] * units + FS * w.B * w.H
+    flops = CHUNK_FLOPS["chunk_fwd_fused_kernel"] * units
+    gbs, tfs = nbytes / t / 1e9, flops / t / 1e12
+    tpk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    return {"value": round(ws * w.B * w.T / t, 1), "unit": "tokens/s", "workload": "prefill_fwd_b8_t2048",
+            "us_per_launch": round(t * 1e6, 2), "launches": n,
+            "roofline": {"kernel": "chunk_fwd_fused_kernel", "bound": "hbm", "achieved": round(gbs, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "bytes_per_launch": nbytes, "peak_source": "%s copy bandwidth" % peak_kind},
+            "tensor": {"achieved": round(tfs, 1), "peak": tpk, "unit": "TFLOP/s", "frac": round(tfs / tpk, 4),
+                       "flops_per_launch": flops, "peak_source": "%s bf16 dense, sustained" % peak_kind}}
 
 
 def run_e2e(args, ws, d, st):
@@ -442,7 +542,8 @@ def run_e2e(args, ws, d, st):
             "steps": e_steps, "overlap": "copy-in, compute and copy-out of consecutive steps on three streams"}
 
 
-def run_tail(args, ws, rank, value, ms_step, roof, shares, e2e, launches, clk, dec, lp=None):
+def run_tail(args, ws, rank, value, ms_step, roof, shares, e2e, launches, clk, dec, lp=None,
+             roof_step=None, prefill=None):
     w = TRAIN
     # ---- oracle on the host cores (rank 0, N = 1 only)
     cpu = None
@@ -467,8 +568,9 @@ def run_tail(args, ws, rank, value, ms_step, roof, shares, e2e, launches, clk, d
                 "config": {"workload": w.name, "global_batch": w.B * ws, "seq_len": w.T,
                            "heads": w.H, "dk": w.dk, "dv": w.dv, "parallelism": "dp%d" % ws,
                            "l2": "inputs larger than L2 (no flush)"},
-                "roofline": roof, "kernel_shares": shares, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches, "clocks": clk, "decode": dec, "long_prefill": lp}
+                "roofline": roof, "roofline_step": roof_step, "kernel_shares": shares,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+                "prefill_fwd": prefill, "decode": dec, "long_prefill": lp}
         print(json.dumps(line), flush=True)
 
 
@@ -546,7 +648,7 @@ def run_long_prefill(args, ws, peaks, peak_kind):
     t_front, t_mix = timed(front, n), timed(mixer, n)
     front_bytes = w.B * w.T * w.D * 4                       # x in, y out (bf16)
     units = w.B * w.H * ((w.T + 127) // 128)
-    mix_bytes = CHUNK_BYTES["chunk_fwd_fused_kernel"] * units + 2 * FS * w.B * w.H   # + S_0 in, S_T out
+    mix_bytes = METHOD_BYTES["chunk_fwd_fused_kernel"] * units + 2 * FS * w.B * w.H   # + S_0 in, S_T out
 
     def roof(kernel, nbytes, t):
         a = nbytes / t / 1e9

@@ -67,6 +67,20 @@ int gla_last_cuda_error(void);
  * threads), for launch accounting by callers. */
 unsigned long long gla_launch_count(void);
 
+/* How this copy of the library was built: a bit mask of GLA_BUILD_* flags.
+ * GLA_BUILD_DEBUG_BOUNDS marks the checking build (libgla_debug.so, compiled
+ * with -DGLA_DEBUG_BOUNDS).  It has the same ABI and results as the normal
+ * build and additionally, without ever trapping:
+ *   - scans the inputs of every chunk, segment and decode call before its
+ *     kernels run: a_t <= 0 and finite, q/k/v/dO and fp32 states finite;
+ *   - checks the index of each direct global store in its kernels against
+ *     the tensor it writes, and skips a store that would fall outside;
+ * and records GLA_ERR_INVALID_ARG in the device status word on a violation
+ * (read it with gla_get_device_status).  The scans cost one extra read of
+ * the inputs per call. */
+#define GLA_BUILD_DEBUG_BOUNDS 1
+int gla_build_flags(void);
+
 /* ---------------------------------------------------------------------------
  * Chunked prefill / training forward.
  *
@@ -140,8 +154,9 @@ gla_status gla_chunk_fwd_varlen(const void* q, const void* k, const void* v, con
  *   - Calls that overlap on the GPU (e.g. on two streams at once) race on the
  *     shared array; order them.  The array's leftover contents never matter.
  *   - The first call on each device looks the array's device address up
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture starts.
+ *     (cudaGetSymbolAddress) with that device current, and so does the first
+ *     call after the device's current context has changed (cudaDeviceReset,
+ *     another context); make those calls before any stream capture starts.
  * Everything else (layouts, validation, status codes) is as gla_chunk_fwd.
  * ------------------------------------------------------------------------ */
 #define GLA_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
@@ -229,15 +244,18 @@ gla_status gla_state_fold(const float* s, const float* g, int n, int reverse, co
  * "Resultados de entrenamiento e inferencia").  For every (n, h):
  *     S <- exp(a[n,h]) * S + k[n,h]^T v[n,h]     (in place, fp32)
  *     o[n,h] = scale * q[n,h] S                   (the updated S)
- *   state    [N_slots, H, dk, dv] fp32, updated in place.
- *   slot_idx [N] int32: state slot of sequence n (NULL = identity, N_slots = N).
- *            Slots must be distinct within one call and < N_slots (not
- *            checked on the device).
+ *   state    [n_slots, H, dk, dv] fp32, updated in place.
+ *   slot_idx [N] int32: state slot of sequence n (NULL = identity).  Slots
+ *            must be distinct within one call.  A slot outside
+ *            [0, n_slots) is skipped (its state is not touched and o[n] is
+ *            not written) and GLA_ERR_INVALID_ARG is recorded in the device
+ *            status word (gla_get_device_status).
+ *   n_slots  number of slots in state; >= N when slot_idx is NULL.
  *   q, k     [N, H, dk] bf16;  v [N, H, dv] bf16;  a [N, H] fp32 (contiguous).
  *   o        [N, H, dv] fp32.
  * Supported: dk == 96, dv == 192.
  * ------------------------------------------------------------------------ */
-gla_status gla_decode_step(float* state, const int32_t* slot_idx, const void* q, const void* k,
+gla_status gla_decode_step(float* state, const int32_t* slot_idx, int n_slots, const void* q, const void* k,
                            const void* v, const float* a, float* o, int N, int H, int dk, int dv,
                            float scale, cudaStream_t stream);
 
@@ -309,16 +327,18 @@ gla_status conv1d_silu_causal_bwd(const void* x, int apply_ln, const float* ln_g
  *     y[n,c]   = SiLU( sum_{j<W-1} w[c,j] * h[s,j,c] + w[c,W-1] * xn[c] + bias[c] )
  *     h[s]    <- (h[s,1], ..., h[s,W-2], xn)        (in place)
  *   x, y        [N, D] bf16, contiguous.
- *   conv_state  [N_slots, W-1, D] fp32: h, the last W-1 conv inputs of each
+ *   conv_state  [n_slots, W-1, D] fp32: h, the last W-1 conv inputs of each
  *               slot, oldest first (the layout of conv1d_silu_causal's
  *               conv_state_in / _out for one sequence), updated in place.
- *   slot_idx    [N] int32 or NULL (identity, N_slots = N).  Slots must be
- *               distinct within one call and < N_slots (not checked on the
- *               device).
+ *   slot_idx    [N] int32 or NULL (identity).  Slots must be distinct within
+ *               one call.  A slot outside [0, n_slots) is skipped (nothing
+ *               read or written for that sequence) and GLA_ERR_INVALID_ARG is
+ *               recorded in the device status word.
+ *   n_slots     number of slots in conv_state; >= N when slot_idx is NULL.
  *   ln_gamma/beta, w, bias as in conv1d_silu_causal.
  * Supported: W == 4, D % 8 == 0, 8 <= D <= 4096.
  * ------------------------------------------------------------------------ */
-gla_status conv1d_silu_decode_step(const void* x, const int32_t* slot_idx, int apply_ln,
+gla_status conv1d_silu_decode_step(const void* x, const int32_t* slot_idx, int n_slots, int apply_ln,
                                    const float* ln_gamma, const float* ln_beta, float ln_eps,
                                    const float* w, const float* bias, float* conv_state, void* y,
                                    int N, int D, int W, cudaStream_t stream);

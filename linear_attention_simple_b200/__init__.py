@@ -8,6 +8,10 @@ Every step of the computation runs in the kernels of ``libgla.so``; there is
 no CPU or PyTorch fallback.  Importing this package does not load the
 library; the first call does, and raises ``GlaLibraryMissing`` when
 ``libgla.so`` has not been built (``python -m linear_attention_simple_b200.build``).
+With ``GLA_DEBUG_BOUNDS=1`` in the environment the first call loads the
+checking build ``libgla_debug.so`` instead (same ABI; input scans and index
+checks that record GLA_ERR_INVALID_ARG in the device status word; built by
+``python -m linear_attention_simple_b200.build --debug``).
 """
 import ctypes
 import os
@@ -21,10 +25,13 @@ __all__ = [
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
     "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step", "conv1d_silu_causal_bwd",
     "conv1d_silu_causal_bwd_workspace_bytes", "gla_chunk_fwd_varlen", "gla_segment_workspace_bytes",
-    "gla_segment_state_fwd", "gla_segment_state_bwd", "gla_state_fold", "EXPORTED_SYMBOLS", "LIB_PATH",
+    "gla_segment_state_fwd", "gla_segment_state_bwd", "gla_state_fold", "gla_build_flags", "EXPORTED_SYMBOLS",
+    "LIB_PATH", "LIB_DEBUG_PATH", "GLA_BUILD_DEBUG_BOUNDS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgla.so")
+LIB_DEBUG_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgla_debug.so")
+GLA_BUILD_DEBUG_BOUNDS = 1
 
 EXPORTED_SYMBOLS = (
     "gla_status_string", "gla_last_cuda_error", "gla_launch_count",
@@ -33,7 +40,7 @@ EXPORTED_SYMBOLS = (
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
     "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step", "conv1d_silu_causal_bwd",
     "conv1d_silu_causal_bwd_workspace_bytes", "gla_chunk_fwd_varlen", "gla_segment_workspace_bytes",
-    "gla_segment_state_fwd", "gla_segment_state_bwd", "gla_state_fold",
+    "gla_segment_state_fwd", "gla_segment_state_bwd", "gla_state_fold", "gla_build_flags",
 )
 
 GLA_BF16, GLA_F32 = 0, 1
@@ -63,14 +70,23 @@ _f = ctypes.c_float
 
 
 def lib():
-    """Load libgla.so (once).  Raises GlaLibraryMissing if it is not built."""
+    """Load libgla.so (once; libgla_debug.so when GLA_DEBUG_BOUNDS=1).
+    Raises GlaLibraryMissing if it is not built."""
     global _LIB
     if _LIB is not None:
         return _LIB
-    if not os.path.exists(LIB_PATH):
-        raise GlaLibraryMissing("libgla.so not found at %s; build it with "
-                                "`python -m linear_attention_simple_b200.build`" % LIB_PATH)
-    L = ctypes.CDLL(LIB_PATH)
+    debug = os.environ.get("GLA_DEBUG_BOUNDS", "0") not in ("", "0")
+    path = LIB_DEBUG_PATH if debug else LIB_PATH
+    if not os.path.exists(path):
+        raise GlaLibraryMissing("%s not found; build it with `python -m linear_attention_simple_b200.build%s`"
+                                % (path, " --debug" if debug else ""))
+    _LIB = declare(ctypes.CDLL(path))
+    return _LIB
+
+
+def declare(L):
+    """Set the ctypes signatures of every exported entry point on a loaded
+    copy of the library (the normal or the checking build); returns L."""
     L.gla_status_string.restype = ctypes.c_char_p
     L.gla_status_string.argtypes = [_i]
     L.gla_last_cuda_error.restype = _i
@@ -84,7 +100,7 @@ def lib():
     L.gla_chunk_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _vp, ctypes.c_size_t, _i, _i, _i, _i, _i, _i64, _f, _i, _vp]
     L.gla_decode_step.restype = _i
-    L.gla_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
+    L.gla_decode_step.argtypes = [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
     L.conv1d_silu_causal.restype = _i
     L.conv1d_silu_causal.argtypes = [_vp, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _vp,
                                      _i, _i, _i, _i, _vp]
@@ -107,7 +123,7 @@ def lib():
     L.gla_state_fold.restype = _i
     L.gla_state_fold.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _i, _i, _i, _vp]
     L.conv1d_silu_decode_step.restype = _i
-    L.conv1d_silu_decode_step.argtypes = [_vp, _vp, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]
+    L.conv1d_silu_decode_step.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _i, _i, _i, _vp]
     L.gla_get_device_status.restype = _i
     L.gla_get_device_status.argtypes = [_vp, ctypes.POINTER(_i)]
     L.gla_set_wait_limit_ns.restype = _i
@@ -123,7 +139,8 @@ def lib():
     L.gla_trace_summary.argtypes = [ctypes.POINTER(ctypes.c_char_p),
                                     ctypes.POINTER(ctypes.c_ulonglong),
                                     ctypes.POINTER(ctypes.c_double), _i]
-    _LIB = L
+    L.gla_build_flags.restype = _i
+    L.gla_build_flags.argtypes = []
     return L
 
 
@@ -181,6 +198,12 @@ def gla_status_string(status):
 
 def gla_launch_count():
     return int(lib().gla_launch_count())
+
+
+def gla_build_flags():
+    """Bit mask of how the loaded library was built (GLA_BUILD_DEBUG_BOUNDS
+    for the checking build)."""
+    return int(lib().gla_build_flags())
 
 
 def gla_chunk_workspace_bytes(B, T, H, dk=96, dv=192, for_bwd=False):
@@ -273,7 +296,8 @@ def gla_chunk_bwd(q, k, v, a, dO, s0=None, ds_final=None, grads=None, ws=None, s
 
 def gla_decode_step(state, q, k, v, a, o=None, slot_idx=None, scale=None, stream=None):
     """In-place decode step.  state [N_slots,H,dk,dv] fp32; q, k [N,H,dk] and
-    v [N,H,dv] bf16; a [N,H] fp32; slot_idx [N] int32 or None.  Returns o."""
+    v [N,H,dv] bf16; a [N,H] fp32; slot_idx [N] int32 or None (a slot outside
+    the pool is skipped and recorded in the device status word).  Returns o."""
     N, H, dk = q.shape
     dv = v.shape[-1]
     _need(state, "state", torch.float32)
@@ -291,7 +315,7 @@ def gla_decode_step(state, q, k, v, a, o=None, slot_idx=None, scale=None, stream
     _need(o, "o", torch.float32, (N, H, dv))
     if scale is None:
         scale = dk ** -0.5
-    st = lib().gla_decode_step(_ptr(state), _ptr(slot_idx), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+    st = lib().gla_decode_step(_ptr(state), _ptr(slot_idx), state.shape[0], _ptr(q), _ptr(k), _ptr(v), _ptr(a),
                                _ptr(o), N, H, dk, dv, float(scale), _stream(stream))
     _check("gla_decode_step", st)
     return o
@@ -501,7 +525,7 @@ def conv1d_silu_decode_step(x, w, conv_state, slot_idx=None, apply_ln=True, ln_g
     if y is None:
         y = torch.empty_like(x)
     _need(y, "y", torch.bfloat16, (N, D))
-    st = lib().conv1d_silu_decode_step(_ptr(x), _ptr(slot_idx), 1 if apply_ln else 0, _ptr(ln_gamma),
+    st = lib().conv1d_silu_decode_step(_ptr(x), _ptr(slot_idx), n_slots, 1 if apply_ln else 0, _ptr(ln_gamma),
                                        _ptr(ln_beta), float(ln_eps), _ptr(w), _ptr(bias), _ptr(conv_state),
                                        _ptr(y), N, D, W, _stream(stream))
     _check("conv1d_silu_decode_step", st)

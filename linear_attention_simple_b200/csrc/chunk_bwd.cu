@@ -39,10 +39,11 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 int num_chunks(int T) { return (T + kChunk - 1) / kChunk; }
 
 struct BwdParams {
-    CUtensorMap tm_q, tm_k, tm_v, tm_do;   // token tiles
-    CUtensorMap tm_h, tm_d;                // per-chunk bf16 states
-    CUtensorMap tm_dq, tm_dk, tm_dv;       // gradient stores
-    CUtensorMap tm_do32, tm_d32, tm_dv32;  // 32-column SW64 boxes (dv kernel)
+    CUtensorMap tm_q, tm_k;                // q, k tiles (32-column SW64 boxes)
+    CUtensorMap tm_dq, tm_dk;              // gradient stores
+    // 32-column SW64 boxes: dO, v, dv; per-chunk states [units*NC][2][96][192]
+    // (plane 0 hi, plane 1 lo) h and D
+    CUtensorMap tm_do32, tm_v32, tm_dv32, tm_h32, tm_d32;
     const float* a;
     float* delta;                          // [B*H, T]: q.dq per token (role 0), k.dk (role 1) after it
     float* ctot;                           // [B*H, NC, 2]: chunk totals of both halves
@@ -85,7 +86,7 @@ __device__ __forceinline__ void chunk_cumsum(float a, float* b2s, float* wsum, i
 
 // ------------------------------------------------------------ dq, dk kernel
 //
-// Two CTAs per chunk, role 0 (dq) and role 1 (dk), each 90 KB of shared
+// Two CTAs per chunk, role 0 (dq) and role 1 (dk), each 87 KB of shared
 // memory and 256 TMEM columns, so two share an SM.  With gamma the chunk's
 // total log-decay and T the masked tile of the dO / V products:
 //
@@ -93,23 +94,28 @@ __device__ __forceinline__ void chunk_cumsum(float a, float* b2s, float* wsum, i
 //   role 1:  dk_j = e^{gamma - b_j} ( v_j D^T + sum_{i >= j} s e^{b_i - gamma} (v_j . dO_i) q_i )
 //
 // The contraction over dv (T = dO V^T for role 0, V dO^T for role 1, and the
-// state product into the accumulator) streams through two shared-memory
-// slots in three 64-column slices; T is then turned in place, in tensor
-// memory, into the bf16 hi and lo halves of the decayed tile and used as the
-// A operand of the MMA against K (role 0) or Q (role 1); the row factor is
-// applied in the epilogue.  Chunks whose decay spans more than 2^100 take
-// the exact path: the tile carries s e^{b_i - b_j}, the state product is
-// scaled in place by the row factor before the tile MMA, row factor 1.
-// Each role also writes its half of the per-token delta of the da sum,
-// q.dq (role 0) or k.dk (role 1), and that half's chunk total.
+// state product into the accumulator) streams through three shared-memory
+// slots in six 32-column slices; each slice carries the state as its bf16
+// hi and lo planes, both multiplied into the accumulator, so the state
+// product keeps the fp32 state's precision (q.dq and k.dk, and through them
+// da, are sums that cancel to a small fraction of their terms).  T is then
+// turned in place, in tensor memory, into the bf16 hi and lo halves of the
+// decayed tile and used as the A operand of the MMA against K (role 0) or Q
+// (role 1); the row factor is applied in the epilogue.  Chunks whose decay
+// spans more than 2^100 take the exact path: the tile carries
+// s e^{b_i - b_j}, the state product is scaled in place by the row factor
+// before the tile MMA, row factor 1.  Each role also writes its half of the
+// per-token delta of the da sum, q.dq (role 0) or k.dk (role 1), and that
+// half's chunk total.
 
-namespace bq {   // dq / dk kernel shared-memory map
-constexpr uint32_t SLOT = 45056;         // dv slice: first [128][64], second [128][64], state [96][64], SW128
-constexpr uint32_t SECOND = 16384, STATE = 32768;
-constexpr uint32_t MISC = 2 * SLOT;
+namespace bq {   // dq / dk kernel shared-memory map (SW64 tiles, 32 columns wide)
+constexpr uint32_t SLOT = 28672;         // first [128][32], second [128][32], state hi, lo [96][32]
+constexpr uint32_t SECOND = 8192, STATE_HI = 16384, STATE_LO = 22528;
+constexpr int kSlots = 3, kSlices = 6;
+constexpr uint32_t MISC = kSlots * SLOT;
 constexpr uint32_t BYTES = MISC + 2048 + 1024;
 constexpr uint32_t TM_T = 0, TM_ACC = 128, TMEM_COLS = 256;
-constexpr uint32_t kSliceBytes = 2 * 16384 + 12288;
+constexpr uint32_t kSliceBytes = 2 * 8192 + 2 * 6144;
 constexpr uint32_t kTileBytes = 3 * 128 * 64;
 }  // namespace bq
 
@@ -143,10 +149,10 @@ __global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dqdk_kernel(const __grid_c
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(sm);
-    uint64_t* bar_full = reinterpret_cast<uint64_t*>(sm + bq::MISC);   // [2] slot loaded
-    uint64_t* bar_free = bar_full + 2;                                  // [2] slot consumed
-    uint64_t* bar_done = bar_full + 4;                                  // all MMAs so far done
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_full + 5);
+    uint64_t* bar_full = reinterpret_cast<uint64_t*>(sm + bq::MISC);   // [3] slot loaded
+    uint64_t* bar_free = bar_full + 3;                                  // [3] slot's MMAs done
+    uint64_t* bar_done = bar_full + 6;                                  // all MMAs so far done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_full + 7);
     float* b2s = reinterpret_cast<float*>(sm + bq::MISC + 64);
     float* cfs = b2s + 128;                  // [128] column factors of the fast path
     float* wsum = cfs + 128;
@@ -160,16 +166,17 @@ __global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dqdk_kernel(const __grid_c
     const bool worker = warp < 8;
     const bool issuer = warp == 8 && lane == 0;
     const WaitCtl ctl = p.ctl;
-    const CUtensorMap* tm_first = role ? &p.tm_v : &p.tm_do;
-    const CUtensorMap* tm_second = role ? &p.tm_do : &p.tm_v;
-    const CUtensorMap* tm_state = role ? &p.tm_d : &p.tm_h;
+    const CUtensorMap* tm_first = role ? &p.tm_v32 : &p.tm_do32;
+    const CUtensorMap* tm_second = role ? &p.tm_do32 : &p.tm_v32;
+    const CUtensorMap* tm_state = role ? &p.tm_d32 : &p.tm_h32;
     const CUtensorMap* tm_op = role ? &p.tm_q : &p.tm_k;      // B operand of the tile MMA
     const CUtensorMap* tm_dot = role ? &p.tm_k : &p.tm_q;     // partner of the delta dot
-    BarTrack tr_full[2], tr_free[2], tr_done;
+    const int state_idx = (unit * p.NC + c) * 2;              // hi plane; lo at + 1
+    BarTrack tr_full[bq::kSlots], tr_free[bq::kSlots], tr_done;
     bool failed = false;
 
     if (issuer) {
-        for (int i = 0; i < 5; ++i) mbar_init(bar_full + i, 1);
+        for (int i = 0; i < 7; ++i) mbar_init(bar_full + i, 1);
         mbar_init_fence();
     }
     if (warp == 0) {
@@ -183,12 +190,13 @@ __global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dqdk_kernel(const __grid_c
     const uint32_t tq = tmem_addr(tmem, quad * 32, 0);
 
     auto load_slice = [&](int sl) {
-        const int k = sl & 1;
+        const int k = sl % bq::kSlots;
         uint8_t* base = sm + k * bq::SLOT;
         mbar_arrive_expect_tx(bar_full + k, bq::kSliceBytes);
-        tma_load_4d(base, tm_first, bar_full + k, sl * 64, h, t0, b);
-        tma_load_4d(base + bq::SECOND, tm_second, bar_full + k, sl * 64, h, t0, b);
-        tma_load_3d(base + bq::STATE, tm_state, bar_full + k, sl * 64, 0, unit * p.NC + c);
+        tma_load_4d(base, tm_first, bar_full + k, sl * 32, h, t0, b);
+        tma_load_4d(base + bq::SECOND, tm_second, bar_full + k, sl * 32, h, t0, b);
+        tma_load_3d(base + bq::STATE_HI, tm_state, bar_full + k, sl * 32, 0, state_idx);
+        tma_load_3d(base + bq::STATE_LO, tm_state, bar_full + k, sl * 32, 0, state_idx + 1);
         ++tr_full[k].issued;
     };
     auto load_tile = [&](int k, const CUtensorMap* m) {
@@ -197,20 +205,25 @@ __global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dqdk_kernel(const __grid_c
         for (int i = 0; i < 3; ++i) tma_load_4d(base + i * 8192, m, bar_full + k, i * 32, h, t0, b);
         ++tr_full[k].issued;
     };
+    // slice sl: two K steps of 16 (32 bytes each) inside the 64-byte rows
     auto mma_slice = [&](int sl) {
-        const uint32_t base = sb + (sl & 1) * bq::SLOT;
-        for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t a = smem_desc(base + ks * 32, 16, 1024, kLayoutSW128);
-            umma_bf16(tmem + bq::TM_T, a, smem_desc(base + bq::SECOND + ks * 32, 16, 1024, kLayoutSW128),
-                      idesc_bf16_f32(128, 128, 0, 0), (sl | ks) > 0);
-            umma_bf16(tmem + bq::TM_ACC, a, smem_desc(base + bq::STATE + ks * 32, 16, 1024, kLayoutSW128),
-                      idesc_bf16_f32(128, 96, 0, 0), (sl | ks) > 0);
+        const uint32_t base = sb + (sl % bq::kSlots) * bq::SLOT;
+        const uint64_t da = smem_desc(base, 16, 512, kLayoutSW64);
+        const uint64_t db = smem_desc(base + bq::SECOND, 16, 512, kLayoutSW64);
+        const uint64_t dh = smem_desc(base + bq::STATE_HI, 16, 512, kLayoutSW64);
+        const uint64_t dl = smem_desc(base + bq::STATE_LO, 16, 512, kLayoutSW64);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            const uint64_t a = desc_add(da, ks * 32);
+            const uint32_t acc = (sl | ks) > 0;
+            umma_bf16(tmem + bq::TM_T, a, desc_add(db, ks * 32), idesc_bf16_f32(128, 128, 0, 0), acc);
+            umma_bf16(tmem + bq::TM_ACC, a, desc_add(dh, ks * 32), idesc_bf16_f32(128, 96, 0, 0), acc);
+            umma_bf16(tmem + bq::TM_ACC, a, desc_add(dl, ks * 32), idesc_bf16_f32(128, 96, 0, 0), 1);
         }
     };
 
     if (issuer) {
-        load_slice(0);
-        load_slice(1);
+        for (int sl = 0; sl < bq::kSlots; ++sl) load_slice(sl);
     }
     if (tid < 128) {
         const int t = t0 + tid;
@@ -224,41 +237,43 @@ __global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dqdk_kernel(const __grid_c
     const float g2 = b2s[127];
     const bool fast = -g2 <= chunk::kFactorRange;
 
-    // T and the state product over the three dv slices
+    // T and the state product over the six dv slices.  Slice sl uses slot
+    // sl % 3; once slice sl's MMAs are issued, the slot of slice sl-1 is
+    // refilled (with slice sl+2, then the tile operand, then the dot
+    // partner) as soon as its MMAs are done, so one slot's MMAs run while
+    // the next slot loads.
     if (issuer) {
-        bool ok = wait_next(bar_full, tr_full[0], ctl);
-        if (ok) {
+        bool ok = true;
+        for (int sl = 0; ok && sl < bq::kSlices; ++sl) {
+            const int k = sl % bq::kSlots;
+            if (!(ok = wait_next(bar_full + k, tr_full[k], ctl))) break;
             tc_fence_after();
-            mma_slice(0);
-            umma_commit(bar_free);
-            ++tr_free[0].issued;
-            ok = wait_next(bar_full + 1, tr_full[1], ctl);
+            mma_slice(sl);
+            if (sl + 1 < bq::kSlices) {
+                umma_commit(bar_free + k);
+                ++tr_free[k].issued;
+            } else {
+                umma_commit(bar_done);
+                ++tr_done.issued;
+            }
+            if (sl >= 1) {
+                const int kp = (sl - 1) % bq::kSlots;
+                if (!(ok = wait_next(bar_free + kp, tr_free[kp], ctl))) break;
+                if (sl + 2 < bq::kSlices)
+                    load_slice(sl + 2);
+                else if (sl + 2 == bq::kSlices)
+                    load_tile(kp, tm_op);    // slot 0, after slice 3
+                else
+                    load_tile(kp, tm_dot);   // slot 1, after slice 4
+            }
         }
-        if (ok) {
-            tc_fence_after();
-            mma_slice(1);
-            umma_commit(bar_free + 1);
-            ++tr_free[1].issued;
-            ok = wait_next(bar_free, tr_free[0], ctl);
-        }
-        if (ok) {
-            load_slice(2);
-            ok = wait_next(bar_free + 1, tr_free[1], ctl);
-        }
-        if (ok) {
-            load_tile(1, tm_op);
-            ok = wait_next(bar_full, tr_full[0], ctl);
-        }
-        if (ok) {
-            tc_fence_after();
-            mma_slice(2);
-            umma_commit(bar_done);
-            ++tr_done.issued;
-            ok = wait_next(bar_done, tr_done, ctl);
-        }
-        if (ok) load_tile(0, tm_dot);   // slot 0 is free once every slice MMA is done
+        // the issuer consumes every phase of bar_done in order, so that its
+        // parity never refers to a phase two ahead of the one it waits for
+        if (ok) ok = wait_next(bar_done, tr_done, ctl);
         failed = !ok;
-    } else if (!mbar_wait(bar_done, 0, ctl)) {
+    } else if (worker && !mbar_wait(bar_done, 0, ctl)) {
+        // (the issuer warp's other lanes wait at the block barrier instead of
+        // spinning beside the issuing lane)
         failed = true;
     }
     tc_fence_before();
@@ -321,26 +336,28 @@ __global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dqdk_kernel(const __grid_c
     // acc += tile (hi, lo) x K or Q, A from tensor memory
     if (issuer) {
         tc_fence_after();
-        bool ok = wait_next(bar_full + 1, tr_full[1], ctl);
+        // the tile operand sits in slot 0 (its third load), the dot partner in
+        // slot 1 (its third load: phase parity 0)
+        bool ok = wait_next(bar_full, tr_full[0], ctl);
         if (ok) {
             for (int part = 0; part < 2; ++part)
                 for (int ks = 0; ks < 8; ++ks)
                     umma_bf16_ts(tmem + bq::TM_ACC, tmem + ts_hi(bq::TM_T, ks) + 16 * part,
-                                 smem_desc(sb + bq::SLOT + ks * 1024, 8192, 512, kLayoutSW64),
+                                 smem_desc(sb + ks * 1024, 8192, 512, kLayoutSW64),
                                  idesc_bf16_f32(128, 96, 0, 1), 1);
             umma_commit(bar_done);
             ++tr_done.issued;
-            ok = wait_next(bar_done, tr_done, ctl) && wait_next(bar_full, tr_full[0], ctl);
+            ok = wait_next(bar_done, tr_done, ctl) && wait_next(bar_full + 1, tr_full[1], ctl);
         }
         failed = !ok;
-    } else if (!mbar_wait(bar_done, 1, ctl) || !mbar_wait(bar_full, 0, ctl)) {
+    } else if (worker && (!mbar_wait(bar_done, 1, ctl) || !mbar_wait(bar_full + 1, 0, ctl))) {
         failed = true;
     }
     tc_fence_before();
     if (__syncthreads_or(failed)) goto done;
     tc_fence_after();
     if (worker) {
-        // epilogue: out = f acc -> staging [3][128][32] SW64 in slot 1; delta partial
+        // epilogue: out = f acc -> staging [3][128][32] SW64 in slot 2; delta partial
         const float f = fast ? (role ? exp2f(g2 - b2s[row]) : p.scale * exp2f(b2s[row])) : 1.0f;
         float dsum = 0.f;
 #pragma unroll
@@ -353,7 +370,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dqdk_kernel(const __grid_c
             for (int g = 0; g < 2; ++g) {
                 const int n = n0 + g * 8;
                 const uint32_t off = (n >> 5) * 8192 + swz_off(row, (n & 31) >> 3, 64);
-                const uint4 w = *reinterpret_cast<const uint4*>(sm + off);   // q or k, slot 0
+                const uint4 w = *reinterpret_cast<const uint4*>(sm + bq::SLOT + off);   // q or k, slot 1
                 const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
                 uint32_t pk[4];
 #pragma unroll
@@ -364,7 +381,7 @@ __global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dqdk_kernel(const __grid_c
                     dsum = fmaf(bf16_hi(wv[e]), x1, dsum);
                     pk[e] = pack_bf16(x0, x1);
                 }
-                *reinterpret_cast<uint4*>(sm + bq::SLOT + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                *reinterpret_cast<uint4*>(sm + 2 * bq::SLOT + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
         }
         if (half) dpart[row] = dsum;
@@ -374,26 +391,27 @@ __global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dqdk_kernel(const __grid_c
         if (!half) {
             const bool live = t0 + row < p.T;
             float x = live ? dsum + dpart[row] : 0.f;
-            if (live) p.delta[(static_cast<int64_t>(role) * p.B * p.H + unit) * p.T + t0 + row] = x;
+            if (live && GLA_DCHECK(unit < p.B * p.H && c < p.NC, ctl.status))
+                p.delta[(static_cast<int64_t>(role) * p.B * p.H + unit) * p.T + t0 + row] = x;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
             if (lane == 0) wsum[quad] = x;
             named_sync128();
-            if (row == 0) p.ctot[(static_cast<int64_t>(unit) * p.NC + c) * 2 + role] = ((wsum[0] + wsum[1]) + wsum[2]) + wsum[3];
+            if (row == 0 && GLA_DCHECK(unit < p.B * p.H && c < p.NC, ctl.status)) p.ctot[(static_cast<int64_t>(unit) * p.NC + c) * 2 + role] = ((wsum[0] + wsum[1]) + wsum[2]) + wsum[3];
         }
     }
     __syncthreads();
     if (issuer) {
         const CUtensorMap* tm_out = role ? &p.tm_dk : &p.tm_dq;
-        for (int i = 0; i < 3; ++i) tma_store_4d(tm_out, sm + bq::SLOT + i * 8192, i * 32, h, t0, b);
+        for (int i = 0; i < 3; ++i) tma_store_4d(tm_out, sm + 2 * bq::SLOT + i * 8192, i * 32, h, t0, b);
         tma_store_commit();
     }
 done:
     if (issuer) {
-        drain(bar_full, tr_full[0], ctl);
-        drain(bar_full + 1, tr_full[1], ctl);
-        drain(bar_free, tr_free[0], ctl);
-        drain(bar_free + 1, tr_free[1], ctl);
+        for (int k = 0; k < bq::kSlots; ++k) {
+            drain(bar_full + k, tr_full[k], ctl);
+            drain(bar_free + k, tr_free[k], ctl);
+        }
         drain(bar_done, tr_done, ctl);
         tma_store_wait_all();
     }
@@ -532,7 +550,7 @@ __global__ void __launch_bounds__(dvp::kThreads, 1) bwd_dv_kernel(const __grid_c
             for (int i = 0; i < 3; ++i) {
                 tma_load_4d(st + dvp::DO + i * 8192, &p.tm_do32, bar_dd + s, w.dvh * 96 + i * 32, w.h, t0, w.b);
                 tma_load_3d(st + dvp::DS + i * 6144, &p.tm_d32, bar_dd + s, w.dvh * 96 + i * 32, 0,
-                            w.unit * p.NC + w.c);
+                            (w.unit * p.NC + w.c) * 2);   // hi plane
             }
             ++n_ld[s];
         }
@@ -746,7 +764,7 @@ __global__ void __launch_bounds__(kDaThreads) da_finish_kernel(float* __restrict
                                                                const float* __restrict__ ctot,
                                                                const float* __restrict__ base,
                                                                const float* __restrict__ anchor, int T, int H,
-                                                               int NC, int units)
+                                                               int NC, int units, int* __restrict__ status)
 {
     __shared__ float wtot[kDaThreads / 32], wsuf[kDaThreads / 32];
     const int unit = blockIdx.x, c = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -775,7 +793,7 @@ __global__ void __launch_bounds__(kDaThreads) da_finish_kernel(float* __restrict
         add += wsuf[w];
         if (w > warp) add += wtot[w];
     }
-    if (t < T) da[(static_cast<int64_t>(unit / H) * T + t) * H + unit % H] = x + add;
+    if (t < T && GLA_DCHECK(unit < units && c < NC, status)) da[(static_cast<int64_t>(unit / H) * T + t) * H + unit % H] = x + add;
 }
 
 // Both inner products below are a few hundred KB per CTA at most, read by
@@ -795,35 +813,42 @@ __device__ __forceinline__ float block_sum_dot(float s, float* red)
     return r;
 }
 
-// anchor[unit][j] = <D_a, h_{a+1}> for a = (j+1) kDaAnchor - 1: the bf16
-// gradient of the state after chunk a and the bf16 state after it (the
-// state entering chunk a+1), in fp32.  One CTA per anchor.
+// anchor[unit][j] = <D_a, h_{a+1}> for a = (j+1) kDaAnchor - 1: the
+// gradient of the state after chunk a and the state after it (the state
+// entering chunk a+1), each read as its bf16 hi + lo pair, in fp32.  One CTA
+// per anchor.
 __global__ void __launch_bounds__(kDotThreads) da_anchor_kernel(float* __restrict__ anchor,
                                                                 const __nv_bfloat16* __restrict__ dbuf,
                                                                 const __nv_bfloat16* __restrict__ hbuf, int NC)
 {
-    constexpr int kVec = static_cast<int>(kSS / 8);                       // 16-byte vectors per state
+    constexpr int kVec = static_cast<int>(kSS / 8);                       // 16-byte vectors per plane
     constexpr int kIt = (kVec + kDotThreads - 1) / kDotThreads;
     __shared__ float red[kDotThreads / 32];
     const int unit = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
     const int a = (j + 1) * kDaAnchor - 1;
-    const uint4* x = reinterpret_cast<const uint4*>(dbuf + (static_cast<int64_t>(unit) * NC + a) * kSS);
-    const uint4* y = reinterpret_cast<const uint4*>(hbuf + (static_cast<int64_t>(unit) * NC + a + 1) * kSS);
-    uint4 u[kIt], v[kIt];
+    const uint4* x = reinterpret_cast<const uint4*>(dbuf + (static_cast<int64_t>(unit) * NC + a) * 2 * kSS);
+    const uint4* y = reinterpret_cast<const uint4*>(hbuf + (static_cast<int64_t>(unit) * NC + a + 1) * 2 * kSS);
+    uint4 xh[kIt], xl[kIt], yh[kIt], yl[kIt];
 #pragma unroll
     for (int i = 0; i < kIt; ++i) {
         const int e = tid + i * kDotThreads;
-        u[i] = e < kVec ? x[e] : make_uint4(0u, 0u, 0u, 0u);
-        v[i] = e < kVec ? y[e] : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+        xh[i] = e < kVec ? x[e] : z;
+        xl[i] = e < kVec ? x[kVec + e] : z;
+        yh[i] = e < kVec ? y[e] : z;
+        yl[i] = e < kVec ? y[kVec + e] : z;
     }
     float s = 0.f;
 #pragma unroll
     for (int i = 0; i < kIt; ++i) {
-        const uint32_t uw[4] = {u[i].x, u[i].y, u[i].z, u[i].w}, vw[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+        const uint32_t a0[4] = {xh[i].x, xh[i].y, xh[i].z, xh[i].w}, a1[4] = {xl[i].x, xl[i].y, xl[i].z, xl[i].w};
+        const uint32_t b0[4] = {yh[i].x, yh[i].y, yh[i].z, yh[i].w}, b1[4] = {yl[i].x, yl[i].y, yl[i].z, yl[i].w};
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            s = fmaf(__uint_as_float(uw[w] << 16), __uint_as_float(vw[w] << 16), s);
-            s = fmaf(__uint_as_float(uw[w] & 0xffff0000u), __uint_as_float(vw[w] & 0xffff0000u), s);
+            const float u0 = bf16_lo(a0[w]) + bf16_lo(a1[w]), u1 = bf16_hi(a0[w]) + bf16_hi(a1[w]);
+            const float v0 = bf16_lo(b0[w]) + bf16_lo(b1[w]), v1 = bf16_hi(b0[w]) + bf16_hi(b1[w]);
+            s = fmaf(u0, v0, s);
+            s = fmaf(u1, v1, s);
         }
     }
     const float r = block_sum_dot(s, red);
@@ -883,7 +908,7 @@ size_t seg_scratch_bytes(int units, int nseg)
 size_t bwd_workspace_bytes(int B, int T, int H)
 {
     const size_t units = static_cast<size_t>(B) * H, NC = num_chunks(T);
-    const size_t states = align256(units * NC * kSS * 2);
+    const size_t states = align256(units * NC * kSS * 2 * 2);   // bf16 hi and lo planes
     int nseg, cps;
     chunk_segment_plan(static_cast<int>(units), static_cast<int>(NC), &nseg, &cps);
     return 2 * states + align256(units * kSS * sizeof(float)) + align256(2 * units * T * sizeof(float)) +
@@ -899,7 +924,7 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
 {
     (void)ws_bytes;
     const int units = pr.B * pr.H, NC = num_chunks(pr.T);
-    const size_t states = align256(static_cast<size_t>(units) * NC * kSS * 2);
+    const size_t states = align256(static_cast<size_t>(units) * NC * kSS * 2 * 2);   // bf16 hi and lo planes
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     void* hbuf = wsb;
     void* dbuf = wsb + states;
@@ -995,16 +1020,13 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     const int64_t ldk = static_cast<int64_t>(pr.H) * kDk;
     if ((s = make_token_map(&bp.tm_q, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&bp.tm_k, pr.k, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
-    if ((s = make_token_map(&bp.tm_v, pr.v, kDv, pr.H, pr.T, pr.B, pr.ld_v, 64, 128)) != GLA_OK) return s;
-    if ((s = make_token_map(&bp.tm_do, dO, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
     if ((s = make_token_map(&bp.tm_dq, dq, kDk, pr.H, pr.T, pr.B, ldk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&bp.tm_dk, dk, kDk, pr.H, pr.T, pr.B, ldk, 32, 64)) != GLA_OK) return s;
-    if ((s = make_token_map(&bp.tm_dv, dv, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
-    if ((s = make_state_map(&bp.tm_h, hbuf, static_cast<int64_t>(units) * NC)) != GLA_OK) return s;
-    if ((s = make_state_map(&bp.tm_d, dbuf, static_cast<int64_t>(units) * NC)) != GLA_OK) return s;
     if ((s = make_token_map(&bp.tm_do32, dO, kDv, pr.H, pr.T, pr.B, ldo, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&bp.tm_dv32, dv, kDv, pr.H, pr.T, pr.B, ldo, 32, 64)) != GLA_OK) return s;
-    if ((s = make_state_map(&bp.tm_d32, dbuf, static_cast<int64_t>(units) * NC, 32)) != GLA_OK) return s;
+    if ((s = make_token_map(&bp.tm_v32, pr.v, kDv, pr.H, pr.T, pr.B, pr.ld_v, 32, 64)) != GLA_OK) return s;
+    if ((s = make_state_map(&bp.tm_h32, hbuf, static_cast<int64_t>(units) * NC * 2, 32)) != GLA_OK) return s;
+    if ((s = make_state_map(&bp.tm_d32, dbuf, static_cast<int64_t>(units) * NC * 2, 32)) != GLA_OK) return s;
     bp.a = pr.a;
     bp.delta = delta;
     bp.ctot = ctot;
@@ -1046,7 +1068,7 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     }
     trace_begin(st);
     da_finish_kernel<<<dim3(units, NC), kDaThreads, 0, st>>>(da, delta, ctot, ds_final ? base : nullptr, anchor,
-                                                             pr.T, pr.H, NC, units);
+                                                             pr.T, pr.H, NC, units, ctl.status);
     trace_end(st, "da_finish_kernel");
     count_launch();
     return check_launch("da_finish_kernel");

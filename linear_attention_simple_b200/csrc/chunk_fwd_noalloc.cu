@@ -20,9 +20,11 @@
 //
 // In host code the array's name is only a host-side stand-in, not a device
 // address, so the host looks the device address up with
-// cudaGetSymbolAddress, once per device, with that device current, on the
-// first call made on it.  That first call must therefore come before any
-// stream capture begins.
+// cudaGetSymbolAddress, with that device current, on the first call made on
+// it, and again whenever the device's current context is no longer the one
+// the address was looked up in (after cudaDeviceReset, or from another
+// context).  The first call on a device (and the first after such a change)
+// must therefore come before any stream capture begins.
 #include <mutex>
 
 #include "gla_internal.h"
@@ -34,21 +36,25 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 void* g_scratch_addr[kMaxDevices] = {};
+const void* g_scratch_ctx[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device (looked up on
-// the first call per device).
+// Device address of the scratch array on the current device, looked up on
+// the first call per device and again when the device's current context
+// differs from the one the cached address belongs to.
 gla_status scratch_for_current_device(void** out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return check_launch("cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return GLA_ERR_UNSUPPORTED;
+    const void* ctx = current_cu_context();
     std::lock_guard<std::mutex> lk(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
+    if (!g_scratch_addr[dev] || g_scratch_ctx[dev] != ctx) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_fwd_noalloc_scratch) != cudaSuccess || !p)
             return check_launch("cudaGetSymbolAddress");
         g_scratch_addr[dev] = p;
+        g_scratch_ctx[dev] = ctx;
     }
     *out = g_scratch_addr[dev];
     return GLA_OK;

@@ -73,8 +73,8 @@ struct StateParams {
     int out_last_only;      // write s_out only from the segment that ends the sweep
                             // (the last one; segment 0 in the reverse pass)
     int g2_unit_stride;     // segments per unit in g2_out
-    int store_h;            // store the bf16 state entering each chunk into h_out
-    void* h_out;            // bf16 [B*H*NC][96][192]
+    int store_h;            // store the state entering each chunk into h_out
+    void* h_out;            // bf16 [B*H*NC][2][96][192]: plane 0 = bf16(S), plane 1 = bf16(S - plane 0)
     const int* cu_seqlens;  // varlen forward: [B+1] token offsets into batch row 0, or null
     void* o_direct;         // varlen forward: o, for the direct stores of a sequence's last chunk
     float scale;
@@ -672,7 +672,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                         if (!direct)
                             *reinterpret_cast<uint4*>(stg + (n >> 6) * 16384 + swz_off(tok, (n & 63) >> 3, 128)) =
                                 pack8(r + q4 * 8);
-                        else if (mine)
+                        else if (mine && GLA_DCHECK(tb + c * 128 + tok < p.T, p.ctl.status))
                             *reinterpret_cast<uint4*>(orow + (j * 32 + q4 * 8) * 2) = pack8(r + q4 * 8);
                     }
                 }
@@ -687,7 +687,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     if (!aborted && warp < 9) {
         // all MMAs are done (the epilogue waited for the last P V): S is final
         const bool write_state = p.s_out && (!p.out_last_only || seg == static_cast<int>(gridDim.x) - 1);
-        if (write_state && srow && !failed)
+        if (write_state && srow && !failed && GLA_DCHECK(unit < p.B * p.H, p.ctl.status))
             tmem_to_state(tq + L::TM_S + half * 96,
                           p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + half * 96);
     }
@@ -910,17 +910,27 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
             }
             tmem_st_wait();
         };
-        // bf16 copy of S (96 B of this thread's row) -> h_out as three 32-byte
-        // stores: whole sectors, the row segment 32-byte aligned
+        // S as a bf16 pair, hi = bf16(S) and lo = bf16(S - hi) (96 B of this
+        // thread's row in each plane) -> h_out as 32-byte stores: whole
+        // sectors, the row segments 32-byte aligned.  hi + lo carries S to
+        // about 2^-17 of its size, so the gradient terms read against the
+        // pair keep the precision of the fp32 state.
         auto store_h = [&](int it) {
+            if (!GLA_DCHECK(chunk_at(it) >= 0 && chunk_at(it) < p.NC && unit < p.B * p.H, p.ctl.status)) return;
             uint8_t* dst = static_cast<uint8_t*>(p.h_out) +
-                           ((static_cast<int64_t>(unit) * p.NC + chunk_at(it)) * kDk + row) * (kDv * 2) + qt * 96;
+                           (((static_cast<int64_t>(unit) * p.NC + chunk_at(it)) * 2) * kDk + row) * (kDv * 2) + qt * 96;
+            constexpr int64_t kPlane = static_cast<int64_t>(kDk) * kDv * 2;
 #pragma unroll
             for (int q = 0; q < 3; ++q) {
-                uint32_t w[8];
+                uint32_t w[8], l[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) w[e] = pack_bf16(S[16 * q + 2 * e], S[16 * q + 2 * e + 1]);
+                for (int e = 0; e < 8; ++e) {
+                    const float x0 = S[16 * q + 2 * e], x1 = S[16 * q + 2 * e + 1];
+                    w[e] = pack_bf16(x0, x1);
+                    l[e] = pack_bf16(x0 - bf16_lo(w[e]), x1 - bf16_hi(w[e]));
+                }
                 st_global_v8(dst + 32 * q, w);
+                st_global_v8(dst + kPlane + 32 * q, l);
             }
         };
 
@@ -978,7 +988,7 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
         if (ok) {
             const int sweep_end = REVERSE ? 0 : static_cast<int>(gridDim.x) - 1;
             const bool write_state = p.s_out && (!p.out_last_only || seg == sweep_end);
-            if (write_state) {
+            if (write_state && GLA_DCHECK(unit < p.B * p.H && row < kDk, p.ctl.status)) {
                 float* dst = p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + qt * 48;
 #pragma unroll
                 for (int e = 0; e < 48; e += 4)

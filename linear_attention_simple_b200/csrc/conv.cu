@@ -9,19 +9,20 @@
 //   y[t,c] = SiLU( sum_{j<4} w[c,j] xn[t-3+j, c] + bias[c] )
 //
 // HBM-bound: x is read once and y written once (2 x 2 bytes per element),
-// about 25 flop per element.  One CTA owns a contiguous token range of one
-// sequence.  x rows reach shared memory through a ring of bulk asynchronous
-// copies (cp.async.bulk, one copy of G contiguous rows per stage, completion
-// on an mbarrier), so up to kStages x G rows are in flight while the CTA
-// works; thread i owns CH consecutive channels (4, or 8 when D > 3072) and
-// reads one vector per row from shared memory.  Per stage one block reduction
-// gives every row's
-// mean and variance: each thread accumulates sums of (x - x0) and (x - x0)^2
-// with the row's first element x0 as shift, which keeps the one-pass
-// variance free of cancellation for shifted inputs.  The causal window of the
-// previous three normalised rows stays in registers; a CTA recomputes the
-// LayerNorm of the three rows before its range instead of exchanging them.
-// Every wait is bounded.
+// about 12 instructions per element.  One CTA owns a contiguous token range
+// of one sequence.  x rows reach shared memory through a ring of bulk
+// asynchronous copies (cp.async.bulk, one copy of G contiguous rows per
+// stage, completion on an mbarrier) issued by a producer warp, which refills
+// a slot as soon as every worker has released it (a per-slot "free"
+// mbarrier), so the workers meet at one block barrier per stage.  Per stage,
+// warp g computes the LayerNorm moments of row g over all D channels (sums
+// of (x - x0) and (x - x0)^2 with the row's first element x0 as shift, which
+// keeps the one-pass variance free of cancellation for shifted inputs, then
+// one warp reduction); then every worker thread, owning 8 consecutive
+// channels, normalises, convolves and writes its channels of the G rows.  The causal window of the previous three
+// normalised rows stays in registers; a CTA recomputes the LayerNorm of the
+// three rows before its range instead of exchanging them.  Every wait is
+// bounded.
 #include <cuda_bf16.h>
 
 #include "gla_device.cuh"
@@ -31,8 +32,7 @@ namespace {
 
 constexpr int kW = 4;
 constexpr int kG = 8;            // rows per stage
-constexpr int kStages = 3;
-constexpr int kMaxWarps = 32;    // up to 1024 threads
+constexpr int kMaxStages = 4;
 
 __device__ __forceinline__ float warp_sum(float v)
 {
@@ -71,42 +71,82 @@ struct Vec<8> {
     using T = uint4;
 };
 
-template <int CH>
-__device__ __forceinline__ void unpack(const typename Vec<CH>::T& v, float* f)
+template <int NCH>
+__device__ __forceinline__ void unpack(const typename Vec<NCH>::T& v, float* f)
 {
     const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
 #pragma unroll
-    for (int i = 0; i < CH / 2; ++i) {
+    for (int i = 0; i < NCH / 2; ++i) {
         f[2 * i] = __uint_as_float(w[i] << 16);
         f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
 }
 
-template <int CH>
-__global__ void __launch_bounds__(CH == 4 ? 768 : 512, 1)
+// OR of v over the n worker threads (named barrier 1; the producer warp is
+// not among them).
+__device__ __forceinline__ bool workers_or(bool v, int n)
+{
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %2, 0;\n\tbarrier.cta.red.or.pred q, 1, %1, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"(n), "r"(static_cast<uint32_t>(v)) : "memory");
+    return r != 0;
+}
+
+// LayerNorm moments of one row of D bf16 values by one warp: (mean, rstd).
+__device__ __forceinline__ float2 row_moments(const uint8_t* row, int D, float eps, int lane)
+{
+    const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(row));
+    float s1 = 0.f, s2 = 0.f;
+    for (int c = lane * 8; c < D; c += 256) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + c * 2);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float a = bf16_lo(w[i]) - x0, b = bf16_hi(w[i]) - x0;
+            s1 += a + b;
+            s2 = fmaf(a, a, fmaf(b, b, s2));
+        }
+    }
+    s1 = warp_sum(s1);
+    s2 = warp_sum(s2);
+    const float invD = 1.0f / static_cast<float>(D);
+    const float m1 = s1 * invD;
+    const float var = fmaxf(s2 * invD - m1 * m1, 0.f);
+    return make_float2(x0 + m1, 1.0f / sqrtf(var + eps));
+}
+
+// Block = D/8 worker threads (8 channels each, rounded up to whole warps) +
+// one producer warp, at most MAXT threads: 13 warps up to D = 3,072 (four a
+// sub-partition, so 128 registers a thread), 17 up to 4,096.  AFF: a
+// LayerNorm affine or a conv bias is given (otherwise their registers are
+// not needed).
+constexpr int CH = 8;
+template <bool AFF, int MAXT>
+__global__ void __launch_bounds__(MAXT, 1)
 ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
                     const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
                     const float* __restrict__ w, const float* __restrict__ bias,
                     const float* __restrict__ cs_in, float* __restrict__ cs_out,
-                    __nv_bfloat16* __restrict__ y, int T, int D, int tokens_per_cta, WaitCtl ctl)
+                    __nv_bfloat16* __restrict__ y, int T, int D, int tokens_per_cta, int stages, WaitCtl ctl)
 {
     using V = typename Vec<CH>::T;
     extern __shared__ __align__(16) uint8_t smem[];
     const size_t row_bytes = static_cast<size_t>(D) * 2;
-    uint8_t* ring = smem;                                                     // [kStages][kG][D]
-    float* red = reinterpret_cast<float*>(smem + kStages * kG * row_bytes);   // [kMaxWarps][kG][2]
-    float* stats = red + kMaxWarps * kG * 2;                                  // [kG][2]: mean, rstd
-    uint64_t* bars = reinterpret_cast<uint64_t*>(stats + kG * 2);
+    uint8_t* ring = smem;                                                        // [stages][kG][D]
+    float2* stats = reinterpret_cast<float2*>(smem + stages * kG * row_bytes);   // [kMaxStages][kG]
+    uint64_t* full = reinterpret_cast<uint64_t*>(stats + kMaxStages * kG);       // [kMaxStages]
+    uint64_t* freeb = full + kMaxStages;                                         // [kMaxStages]
 
     const int b = blockIdx.y;
     const int t_begin = blockIdx.x * tokens_per_cta;
     const int t_end = min(T, t_begin + tokens_per_cta);
     if (t_begin >= t_end) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nwarps = blockDim.x >> 5;
+    const int nwork = blockDim.x - 32;                 // worker threads
+    const int nwarps = nwork >> 5;
+    const bool producer = warp == nwarps;
     const int c0 = tid * CH;
-    const bool active = c0 < D;
-    const float invD = 1.0f / static_cast<float>(D);
+    const bool active = !producer && c0 < D;
 
     // positions p0 .. t_end-1 stream through the ring; p0 >= 0
     const int p0 = max(0, t_begin - (kW - 1));
@@ -115,30 +155,48 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
     __nv_bfloat16* yb = y + static_cast<int64_t>(b) * T * D;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(bars + s, 1);
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(freeb + s, nwork);
+        }
         mbar_init_fence();
     }
     __syncthreads();
-    auto issue = [&](int s) {
-        const int pos = p0 + s * kG;
-        const int rows = min(kG, t_end - pos);
-        uint64_t* bar = bars + (s % kStages);
-        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows * row_bytes));
-        bulk_load(ring + (s % kStages) * kG * row_bytes, xb + static_cast<int64_t>(pos) * D,
-                  static_cast<uint32_t>(rows * row_bytes), bar);
-    };
-    if (tid == 0)
-        for (int s = 0; s < min(kStages, nstages); ++s) issue(s);
 
-    float wr[CH][kW], ga[CH], be[CH], bi[CH];
+    if (producer) {
+        // -------------------------------------------------------- producer
+        if (lane == 0) {
+            int issued[kMaxStages] = {0, 0, 0, 0};
+            for (int s = 0; s < nstages; ++s) {
+                const int slot = s % stages;
+                // the slot's previous stage (s - stages) has been released by every worker
+                if (s >= stages && !mbar_wait(freeb + slot, ((s - stages) / stages) & 1, ctl)) break;
+                const int pos = p0 + s * kG;
+                const int rows = min(kG, t_end - pos);
+                mbar_arrive_expect_tx(full + slot, static_cast<uint32_t>(rows * row_bytes));
+                bulk_load(ring + slot * kG * row_bytes, xb + static_cast<int64_t>(pos) * D,
+                          static_cast<uint32_t>(rows * row_bytes), full + slot);
+                ++issued[slot];
+            }
+            // every copy in flight lands before the shared memory is released
+            for (int i = 0; i < stages; ++i)
+                if (issued[i]) mbar_wait(full + i, (issued[i] - 1) & 1, ctl);
+        }
+        return;
+    }
+
+    // ----------------------------------------------------------- workers
+    float wr[CH][kW], ga[AFF ? CH : 1], be[AFF ? CH : 1], bi[AFF ? CH : 1];
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
         const int ch = active ? c0 + c : 0;
 #pragma unroll
         for (int j = 0; j < kW; ++j) wr[c][j] = active ? w[ch * kW + j] : 0.f;
-        ga[c] = (gamma && active) ? gamma[ch] : 1.f;
-        be[c] = (beta && active) ? beta[ch] : 0.f;
-        bi[c] = (bias && active) ? bias[ch] : 0.f;
+        if constexpr (AFF) {
+            ga[c] = (gamma && active) ? gamma[ch] : 1.f;
+            be[c] = (beta && active) ? beta[ch] : 0.f;
+            bi[c] = (bias && active) ? bias[ch] : 0.f;
+        }
     }
 
     // window: the three positions before the stream start p0 (only negative
@@ -157,58 +215,26 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
 
     bool failed = false;
     for (int s = 0; s < nstages; ++s) {
-        const int slot = s % kStages;
+        const int slot = s % stages;
         const int pos0 = p0 + s * kG;
         const int rows = min(kG, t_end - pos0);
-        if (!mbar_wait(bars + slot, (s / kStages) & 1, ctl)) failed = true;
-        if (__syncthreads_or(failed)) break;
+        if (!failed && !mbar_wait(full + slot, (s / stages) & 1, ctl)) failed = true;
         const uint8_t* st = ring + slot * kG * row_bytes;
-
-        if (apply_ln) {
-            // per-row shifted sums -> warp partials -> one warp finalises
-#pragma unroll
-            for (int g = 0; g < kG; ++g) {
-                float s1 = 0.f, s2 = 0.f;
-                if (g < rows && active) {
-                    const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(st + g * row_bytes));
-                    float f[CH];
-                    unpack<CH>(*reinterpret_cast<const V*>(st + g * row_bytes + c0 * 2), f);
-#pragma unroll
-                    for (int c = 0; c < CH; ++c) {
-                        const float d = f[c] - x0;
-                        s1 += d;
-                        s2 = fmaf(d, d, s2);
-                    }
-                }
-                s1 = warp_sum(s1);
-                s2 = warp_sum(s2);
-                if (lane == 0) {
-                    red[(warp * kG + g) * 2] = s1;
-                    red[(warp * kG + g) * 2 + 1] = s2;
-                }
+        float2* sst = stats + slot * kG;
+        if (apply_ln && !failed)
+            for (int g = warp; g < rows; g += nwarps) {
+                const float2 m = row_moments(st + g * row_bytes, D, eps, lane);
+                if (lane == 0) sst[g] = m;
             }
-            __syncthreads();
-            if (warp == 0) {
-                // lane = 2 g + k: row g, k = 0 sum, k = 1 sum of squares
-                float v = 0.f;
-                if (lane < 2 * kG)
-                    for (int i = 0; i < nwarps; ++i) v += red[i * kG * 2 + lane];
-                const float other = __shfl_xor_sync(0xffffffffu, v, 1);
-                if (lane < 2 * kG && (lane & 1) == 0) {
-                    const int g = lane >> 1;
-                    const float x0 = g < rows
-                                         ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(st + g * row_bytes))
-                                         : 0.f;
-                    const float m1 = v * invD;
-                    const float var = fmaxf(other * invD - m1 * m1, 0.f);
-                    stats[2 * g] = x0 + m1;
-                    stats[2 * g + 1] = 1.0f / sqrtf(var + eps);
-                }
-            }
-            __syncthreads();
+        // moments visible to every worker; a timed-out wait stops the CTA
+        if (workers_or(failed, nwork)) {
+            failed = true;
+            break;
         }
 
-#pragma unroll
+        // fully unrolled (the window rotation becomes register renaming) where
+        // the registers allow it
+#pragma unroll(MAXT <= 416 ? kG : 2)
         for (int g = 0; g < kG; ++g) {
             if (g >= rows) break;
             const int p = pos0 + g;
@@ -216,15 +242,21 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
             if (active) {
                 unpack<CH>(*reinterpret_cast<const V*>(st + g * row_bytes + c0 * 2), xn);
                 if (apply_ln) {
-                    const float mean = stats[2 * g], rstd = stats[2 * g + 1];
+                    const float2 m = sst[g];
+                    if constexpr (AFF) {
 #pragma unroll
-                    for (int c = 0; c < CH; ++c) xn[c] = fmaf((xn[c] - mean) * rstd, ga[c], be[c]);
+                        for (int c = 0; c < CH; ++c) xn[c] = fmaf((xn[c] - m.x) * m.y, ga[c], be[c]);
+                    } else {
+                        const float sh = -m.x * m.y;
+#pragma unroll
+                        for (int c = 0; c < CH; ++c) xn[c] = fmaf(xn[c], m.y, sh);
+                    }
                 }
             } else {
 #pragma unroll
                 for (int c = 0; c < CH; ++c) xn[c] = 0.f;
             }
-            if (p >= t_begin && active) {
+            if (p >= t_begin && active && GLA_DCHECK(p < T && c0 + CH <= D, ctl.status)) {
                 V out;
                 uint32_t* ow = reinterpret_cast<uint32_t*>(&out);
 #pragma unroll
@@ -232,14 +264,14 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
                     float r[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        float acc = bi[c + e];
+                        float acc = AFF ? bi[AFF ? c + e : 0] : 0.f;
 #pragma unroll
                         for (int j = 0; j < kW - 1; ++j) acc = fmaf(wr[c + e][j], win[j][c + e], acc);
                         r[e] = silu(fmaf(wr[c + e][kW - 1], xn[c + e], acc));
                     }
                     ow[c / 2] = pack_bf16(r[0], r[1]);
                 }
-                *reinterpret_cast<V*>(yb + static_cast<int64_t>(p) * D + c0) = out;
+                __stcs(reinterpret_cast<V*>(yb + static_cast<int64_t>(p) * D + c0), out);
             }
 #pragma unroll
             for (int c = 0; c < CH; ++c) {
@@ -248,8 +280,7 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
                 win[2][c] = xn[c];
             }
         }
-        __syncthreads();                       // everyone is done with this slot
-        if (tid == 0 && s + kStages < nstages) issue(s + kStages);
+        mbar_arrive(freeb + slot);             // this worker is done with the slot
     }
 
     // The CTA that owns the end of the sequence hands the window on.
@@ -258,10 +289,6 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
         for (int r = 0; r < kW - 1; ++r)
 #pragma unroll
             for (int c = 0; c < CH; ++c) cs_out[(static_cast<int64_t>(b) * (kW - 1) + r) * D + c0 + c] = win[r][c];
-    }
-    if (failed && tid == 0) {
-        // drain in-flight copies (bounded) before the shared memory is released
-        for (int s = 0; s < kStages; ++s) mbar_wait(bars + s, 0, ctl) || mbar_wait(bars + s, 1, ctl);
     }
 }
 
@@ -275,9 +302,9 @@ gla_status launch_conv(const void* x, int apply_ln, const float* g, const float*
     gla_status se;
     const WaitCtl ctl = wait_ctl_for_current_device(&se);
     if (se != GLA_OK) return se;
-    // 4 channels per thread up to D = 3072 (768 threads), else 8 (512 threads)
-    const int ch = D <= 3072 ? 4 : 8;
-    const int threads = ((D / ch) + 31) / 32 * 32;
+    // 8 channels per worker thread (384 workers at D = 3,072); one more warp
+    // issues the copies
+    const int threads = ((D / CH) + 31) / 32 * 32 + 32;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -288,9 +315,16 @@ gla_status launch_conv(const void* x, int apply_ln, const float* g, const float*
     if (nx < 1) nx = 1;
     int per = (T + nx - 1) / nx;
     nx = (T + per - 1) / per;
-    const size_t smem = static_cast<size_t>(kStages) * kG * D * 2 +
-                        (kMaxWarps * kG * 2 + kG * 2) * sizeof(float) + kStages * sizeof(uint64_t);
-    auto kernel = ch == 4 ? ln_conv_silu_kernel<4> : ln_conv_silu_kernel<8>;
+    // as many ring stages (up to 4) as fit beside the moments and barriers
+    const size_t stage_bytes = static_cast<size_t>(kG) * D * 2;
+    const size_t fixed = kMaxStages * kG * sizeof(float2) + 2 * kMaxStages * sizeof(uint64_t);
+    int stages = static_cast<int>((200 * 1024 - fixed) / stage_bytes);
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < 2) stages = 2;
+    const size_t smem = stages * stage_bytes + fixed;
+    const bool aff = g || b || bias;
+    auto kernel = threads <= 416 ? (aff ? ln_conv_silu_kernel<true, 416> : ln_conv_silu_kernel<false, 416>)
+                                 : (aff ? ln_conv_silu_kernel<true, 544> : ln_conv_silu_kernel<false, 544>);
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return check_launch("cudaFuncSetAttribute");
@@ -298,7 +332,7 @@ gla_status launch_conv(const void* x, int apply_ln, const float* g, const float*
     trace_begin(st);
     kernel<<<grid, threads, smem, st>>>(static_cast<const __nv_bfloat16*>(x), apply_ln, g, b, eps, w,
                                         bias, cs_in, cs_out, static_cast<__nv_bfloat16*>(y), T, D, per,
-                                        ctl);
+                                        stages, ctl);
     trace_end(st, "ln_conv_silu_kernel");
     count_launch();
     return check_launch("ln_conv_silu_kernel");

@@ -19,6 +19,8 @@
 // One CTA per sequence, thread i owns channels 8i .. 8i+7: one 16-byte
 // vector of x and y, two of each history row.  The LayerNorm moments are two
 // block reductions (mean, then the centred second moment) over registers.
+// A slot outside [0, n_slots) is skipped (nothing read or written) and
+// GLA_ERR_INVALID_ARG is recorded in the device status word.
 #include <cuda_bf16.h>
 
 #include "gla_device.cuh"
@@ -75,11 +77,15 @@ __global__ void __launch_bounds__(kMaxThreads) conv_decode_kernel(
     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ slot_idx, int apply_ln,
     const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
     const float* __restrict__ w, const float* __restrict__ bias, float* __restrict__ hist,
-    __nv_bfloat16* __restrict__ y, int D)
+    __nv_bfloat16* __restrict__ y, int D, int n_slots, int* __restrict__ status)
 {
     __shared__ float red[kMaxThreads / 32];
     const int n = blockIdx.x, c0 = threadIdx.x * 8;
     const int s = slot_idx ? slot_idx[n] : n;
+    if (s < 0 || s >= n_slots) {                // a slot outside the pool: touch nothing
+        if (threadIdx.x == 0) record_status(status, GLA_ERR_INVALID_ARG);
+        return;
+    }
 
     const uint4 xv = __ldcs(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(n) * D + c0));
     const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
@@ -140,13 +146,13 @@ __global__ void __launch_bounds__(kMaxThreads) conv_decode_kernel(
 
 }  // namespace
 
-gla_status launch_conv_decode(const void* x, const int32_t* slot_idx, int apply_ln, const float* g,
+gla_status launch_conv_decode(const void* x, const int32_t* slot_idx, int n_slots, int apply_ln, const float* g,
                               const float* b, float eps, const float* w, const float* bias, float* hist,
-                              void* y, int N, int D, cudaStream_t st)
+                              void* y, int N, int D, int* status, cudaStream_t st)
 {
     trace_begin(st);
     conv_decode_kernel<<<N, D / 8, 0, st>>>(static_cast<const __nv_bfloat16*>(x), slot_idx, apply_ln, g, b, eps,
-                                            w, bias, hist, static_cast<__nv_bfloat16*>(y), D);
+                                            w, bias, hist, static_cast<__nv_bfloat16*>(y), D, n_slots, status);
     trace_end(st, "conv_decode_kernel");
     count_launch();
     return check_launch("conv_decode_kernel");

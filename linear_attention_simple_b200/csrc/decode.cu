@@ -13,7 +13,8 @@
 // contiguous bytes, so every load and store is fully coalesced, and each
 // thread keeps 24 independent 16-byte loads in flight before it computes.
 // The column sums of q S are reduced over the four row groups in shared
-// memory.
+// memory.  A slot outside [0, n_slots) is skipped (nothing read or written)
+// and GLA_ERR_INVALID_ARG is recorded in the device status word.
 #include <cuda_bf16.h>
 
 #include "gla_internal.h"
@@ -30,7 +31,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 decode_step_kernel(float* __restrict__ state, const int32_t* __restrict__ slot_idx,
                    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                    const __nv_bfloat16* __restrict__ v, const float* __restrict__ a,
-                   float* __restrict__ o, int H, float scale)
+                   float* __restrict__ o, int H, int n_slots, float scale, int* __restrict__ status)
 {
     __shared__ float s_q[kDk];
     __shared__ float s_k[kDk];
@@ -44,6 +45,10 @@ decode_step_kernel(float* __restrict__ state, const int32_t* __restrict__ slot_i
     const int rg = t / kC4;
 
     const int64_t slot = slot_idx ? static_cast<int64_t>(slot_idx[n]) : static_cast<int64_t>(n);
+    if (slot < 0 || slot >= n_slots) {          // a slot outside the pool: touch nothing
+        if (t == 0 && status) atomicCAS(status, 0, static_cast<int>(GLA_ERR_INVALID_ARG));
+        return;
+    }
     float4* S = reinterpret_cast<float4*>(state + (slot * H + h) * (int64_t)(kDk * kDv));
 
     // Issue the whole state slice of this thread first (24 x 16 B in flight).
@@ -96,9 +101,9 @@ decode_step_kernel(float* __restrict__ state, const int32_t* __restrict__ slot_i
 
 }  // namespace
 
-gla_status launch_decode(float* state, const int32_t* slot_idx, const void* q, const void* k,
+gla_status launch_decode(float* state, const int32_t* slot_idx, int n_slots, const void* q, const void* k,
                          const void* v, const float* a, float* o, int N, int H, float scale,
-                         cudaStream_t st)
+                         int* status, cudaStream_t st)
 {
     const int64_t units = static_cast<int64_t>(N) * H;
     if (units == 0) return GLA_OK;
@@ -107,7 +112,7 @@ gla_status launch_decode(float* state, const int32_t* slot_idx, const void* q, c
     decode_step_kernel<<<static_cast<unsigned>(units), kThreads, 0, st>>>(
         state, slot_idx, static_cast<const __nv_bfloat16*>(q),
         static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), a, o, H,
-        scale);
+        n_slots, scale, status);
     trace_end(st, "decode_step_kernel");
     count_launch();
     return check_launch("decode_step_kernel");

@@ -33,6 +33,17 @@ __device__ __forceinline__ void record_status(int* status, int code)
     if (status) atomicCAS(status, 0, code);
 }
 
+// Index checks compiled in only with -DGLA_DEBUG_BOUNDS (libgla_debug.so): a
+// failed check records GLA_ERR_INVALID_ARG in the device status word and the
+// guarded access is skipped -- no trap, the context stays usable.  In the
+// normal build a check is the constant true and its condition is not
+// evaluated.
+#ifdef GLA_DEBUG_BOUNDS
+#define GLA_DCHECK(cond, status) ((cond) ? true : (::gla::record_status((status), GLA_ERR_INVALID_ARG), false))
+#else
+#define GLA_DCHECK(cond, status) true
+#endif
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)

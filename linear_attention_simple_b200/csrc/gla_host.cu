@@ -24,6 +24,7 @@ std::atomic<unsigned long long> g_wait_limit_ns{0};
 constexpr unsigned long long kDefaultWaitNs = 2000000000ull;  // 2 s
 constexpr int kMaxDevices = 64;
 int* g_status_addr[kMaxDevices] = {};
+const void* g_status_ctx[kMaxDevices] = {};
 std::mutex g_status_mu;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -34,6 +35,30 @@ gla_status cuda_fail(cudaError_t e)
     return GLA_ERR_CUDA;
 }
 
+}  // namespace
+
+// The driver context current on this thread (an opaque handle; null when it
+// cannot be read), fetched through the runtime's driver entry point so that
+// the library need not link the driver library.
+const void* current_cu_context()
+{
+    typedef CUresult (*GetCtxFn)(CUcontext*);
+    static GetCtxFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<GetCtxFn>(p);
+    });
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+namespace {
+
 int* status_addr_current(gla_status* err)
 {
     int dev = 0;
@@ -42,8 +67,11 @@ int* status_addr_current(gla_status* err)
         *err = cuda_fail(e == cudaSuccess ? cudaErrorInvalidDevice : e);
         return nullptr;
     }
+    const void* ctx = current_cu_context();
     std::lock_guard<std::mutex> lk(g_status_mu);
-    if (!g_status_addr[dev]) {
+    // looked up again whenever the device's current context is not the one
+    // the cached address belongs to (a reset device, another context)
+    if (!g_status_addr[dev] || g_status_ctx[dev] != ctx) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_device_status);
         if (e != cudaSuccess) {
@@ -51,6 +79,7 @@ int* status_addr_current(gla_status* err)
             return nullptr;
         }
         g_status_addr[dev] = static_cast<int*>(p);
+        g_status_ctx[dev] = ctx;
     }
     *err = GLA_OK;
     return g_status_addr[dev];
@@ -205,6 +234,28 @@ gla_status validate_chunk(const void* q, const void* k, const void* v, const flo
     return GLA_OK;
 }
 
+// The checking build's scan of a chunked call's inputs (no-op otherwise):
+// q, k [rows = B*T][H*96] and v [rows][H*192] at token stride ld, dO packed.
+gla_status scan_chunk_inputs(const void* q, const void* k, const void* v, const float* a, const void* dO,
+                             const float* s0, const float* s_extra, int B, int T, int H, int64_t ld_qk,
+                             int64_t ld_v, int* status, cudaStream_t st)
+{
+    DebugScan d;
+    const int64_t rows = static_cast<int64_t>(B) * T;
+    d.a = a;
+    d.na = rows * H;
+    d.bf16[0] = {q, rows, ld_qk, static_cast<int64_t>(H) * kDk};
+    d.bf16[1] = {k, rows, ld_qk, static_cast<int64_t>(H) * kDk};
+    d.bf16[2] = {v, rows, ld_v, static_cast<int64_t>(H) * kDv};
+    d.bf16[3] = {dO, rows, static_cast<int64_t>(H) * kDv, static_cast<int64_t>(H) * kDv};
+    const int64_t ns = static_cast<int64_t>(B) * H * kDk * kDv;
+    d.f32[0] = s0;
+    d.nf32[0] = s0 ? ns : 0;
+    d.f32[1] = s_extra;
+    d.nf32[1] = s_extra ? ns : 0;
+    return debug_scan(d, status, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -261,6 +312,9 @@ gla_status gla_chunk_fwd(const void* q, const void* k, const void* v, const floa
                               s_final, B, T, H, ld_qk, ld_v, scale, ctl, stream);
     const size_t need = fwd_workspace_bytes(B, T, H);
     if (need > 0 && (!ws || ws_bytes < need)) return GLA_ERR_INVALID_ARG;
+    if ((s = scan_chunk_inputs(q, k, v, a, nullptr, s0, nullptr, B, T, H, ld_qk, ld_v, ctl.status, stream)) !=
+        GLA_OK)
+        return s;
     ChunkProblem p{q, k, v, a, B, T, H, ld_qk, ld_v, scale};
     return run_chunk_fwd(p, s0, o, s_final, ws, ws_bytes, ctl, stream);
 }
@@ -283,6 +337,9 @@ gla_status gla_chunk_fwd_varlen(const void* q, const void* k, const void* v, con
     gla_status se;
     WaitCtl ctl = wait_ctl_for_current_device(&se);
     if (se != GLA_OK) return se;
+    if ((s = scan_chunk_inputs(q, k, v, a, nullptr, nullptr, nullptr, 1, total_T, H, ld_qk, ld_v, ctl.status,
+                               stream)) != GLA_OK)
+        return s;
     ChunkProblem p{q, k, v, a, 1, total_T, H, ld_qk, ld_v, scale};
     return run_chunk_fwd_varlen(p, cu_seqlens, N, s0, o, s_final, ctl, stream);
 }
@@ -319,6 +376,9 @@ gla_status gla_chunk_bwd(const void* q, const void* k, const void* v, const floa
     gla_status se;
     WaitCtl ctl = wait_ctl_for_current_device(&se);
     if (se != GLA_OK) return se;
+    if ((s = scan_chunk_inputs(q, k, v, a, dO, s0, ds_final, B, T, H, ld_qk, ld_v, ctl.status, stream)) !=
+        GLA_OK)
+        return s;
     ChunkProblem p{q, k, v, a, B, T, H, ld_qk, ld_v, scale};
     return run_chunk_bwd(p, s0, dO, ds_final, grad_q, grad_k, grad_v, grad_a, grad_s0, ws,
                          ws_bytes, ctl, stream);
@@ -353,6 +413,14 @@ gla_status segment_state(const void* u, const void* y, const float* a, float* s_
     gla_status se;
     WaitCtl ctl = wait_ctl_for_current_device(&se);
     if (se != GLA_OK) return se;
+    DebugScan d;
+    const int64_t rows = static_cast<int64_t>(B) * T;
+    d.a = a;
+    d.na = rows * H;
+    d.bf16[0] = {u, rows, ld_u, static_cast<int64_t>(H) * dk};
+    d.bf16[1] = {y, rows, ld_y, static_cast<int64_t>(H) * dv};
+    gla_status s = debug_scan(d, ctl.status, stream);
+    if (s != GLA_OK) return s;
     return run_segment_state(u, y, a, B, T, H, ld_u, ld_y, scale, reverse, s_seg, g_seg, ws, ctl, stream);
 }
 
@@ -399,11 +467,12 @@ gla_status gla_state_fold(const float* s, const float* g, int n, int reverse, co
     return launch_state_fold(s, g, n, units, reverse ? 1 : 0, s_in, out, stream);
 }
 
-gla_status gla_decode_step(float* state, const int32_t* slot_idx, const void* q, const void* k,
+gla_status gla_decode_step(float* state, const int32_t* slot_idx, int n_slots, const void* q, const void* k,
                            const void* v, const float* a, float* o, int N, int H, int dk, int dv,
                            float scale, cudaStream_t stream)
 {
     if (N < 0 || H < 0 || dk <= 0 || dv <= 0) return GLA_ERR_INVALID_ARG;
+    if (n_slots < 0 || (!slot_idx && n_slots < N)) return GLA_ERR_INVALID_ARG;
     if (bad_scale(scale)) return GLA_ERR_INVALID_ARG;
     if (dk != kDk || dv != kDv) return GLA_ERR_UNSUPPORTED;
     if (static_cast<int64_t>(N) * H == 0) return GLA_OK;
@@ -411,7 +480,18 @@ gla_status gla_decode_step(float* state, const int32_t* slot_idx, const void* q,
     if (!aligned16(state) || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(a) ||
         !aligned16(o) || !aligned16(slot_idx))
         return GLA_ERR_MISALIGNED;
-    return launch_decode(state, slot_idx, q, k, v, a, o, N, H, scale, stream);
+    gla_status se;
+    WaitCtl ctl = wait_ctl_for_current_device(&se);
+    if (se != GLA_OK) return se;
+    DebugScan d;
+    d.a = a;
+    d.na = static_cast<int64_t>(N) * H;
+    d.bf16[0] = {q, static_cast<int64_t>(N) * H, dk, dk};
+    d.bf16[1] = {k, static_cast<int64_t>(N) * H, dk, dk};
+    d.bf16[2] = {v, static_cast<int64_t>(N) * H, dv, dv};
+    gla_status s = debug_scan(d, ctl.status, stream);
+    if (s != GLA_OK) return s;
+    return launch_decode(state, slot_idx, n_slots, q, k, v, a, o, N, H, scale, ctl.status, stream);
 }
 
 gla_status conv1d_silu_causal(const void* x, int apply_ln, const float* ln_gamma,
@@ -443,12 +523,13 @@ gla_status conv1d_silu_causal(const void* x, int apply_ln, const float* ln_gamma
                        conv_state_out, y, B, T, D, stream);
 }
 
-gla_status conv1d_silu_decode_step(const void* x, const int32_t* slot_idx, int apply_ln,
+gla_status conv1d_silu_decode_step(const void* x, const int32_t* slot_idx, int n_slots, int apply_ln,
                                    const float* ln_gamma, const float* ln_beta, float ln_eps,
                                    const float* w, const float* bias, float* conv_state, void* y,
                                    int N, int D, int W, cudaStream_t stream)
 {
     if (N < 0 || D <= 0 || W <= 0) return GLA_ERR_INVALID_ARG;
+    if (n_slots < 0 || (!slot_idx && n_slots < N)) return GLA_ERR_INVALID_ARG;
     if (apply_ln && !(ln_eps > 0.0f && std::isfinite(ln_eps))) return GLA_ERR_INVALID_ARG;
     if (W != 4 || D % 8 != 0 || D > 4096) return GLA_ERR_UNSUPPORTED;
     if (N == 0) return GLA_OK;
@@ -456,8 +537,11 @@ gla_status conv1d_silu_decode_step(const void* x, const int32_t* slot_idx, int a
     if (!aligned16(x) || !aligned16(y) || !aligned16(w) || !aligned16(ln_gamma) || !aligned16(ln_beta) ||
         !aligned16(bias) || !aligned16(conv_state))
         return GLA_ERR_MISALIGNED;
-    return launch_conv_decode(x, slot_idx, apply_ln, ln_gamma, ln_beta, ln_eps, w, bias, conv_state, y, N, D,
-                              stream);
+    gla_status se;
+    WaitCtl ctl = wait_ctl_for_current_device(&se);
+    if (se != GLA_OK) return se;
+    return launch_conv_decode(x, slot_idx, n_slots, apply_ln, ln_gamma, ln_beta, ln_eps, w, bias, conv_state, y, N,
+                              D, ctl.status, stream);
 }
 
 size_t conv1d_silu_causal_bwd_workspace_bytes(int B, int T, int D, int W)

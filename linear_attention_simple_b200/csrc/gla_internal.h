@@ -25,6 +25,9 @@ constexpr int kDv = 192;
 
 // Host-side helpers implemented in gla_host.cu.
 WaitCtl wait_ctl_for_current_device(gla_status* err);
+// The driver context current on this thread (opaque; null if unreadable):
+// device addresses cached per device are valid only within it.
+const void* current_cu_context();
 gla_status check_launch(const char* what);
 void count_launch(unsigned n = 1);
 
@@ -40,17 +43,17 @@ gla_status make_tmap(CUtensorMap* map, const void* base, int rank, const uint64_
                      int swizzle_bytes);
 
 // ---- launchers (one per kernel family), all asynchronous on `st`.
-gla_status launch_decode(float* state, const int32_t* slot_idx, const void* q, const void* k,
+gla_status launch_decode(float* state, const int32_t* slot_idx, int n_slots, const void* q, const void* k,
                          const void* v, const float* a, float* o, int N, int H, float scale,
-                         cudaStream_t st);
+                         int* status, cudaStream_t st);
 
 gla_status launch_conv(const void* x, int apply_ln, const float* g, const float* b, float eps,
                        const float* w, const float* bias, const float* cs_in, float* cs_out,
                        void* y, int B, int T, int D, cudaStream_t st);
 
-gla_status launch_conv_decode(const void* x, const int32_t* slot_idx, int apply_ln, const float* g,
+gla_status launch_conv_decode(const void* x, const int32_t* slot_idx, int n_slots, int apply_ln, const float* g,
                               const float* b, float eps, const float* w, const float* bias, float* hist,
-                              void* y, int N, int D, cudaStream_t st);
+                              void* y, int N, int D, int* status, cudaStream_t st);
 
 size_t conv_bwd_workspace_bytes(int B, int T, int D);
 gla_status launch_conv_bwd(const void* x, int apply_ln, const float* g, const float* be, float eps, const float* w,
@@ -87,6 +90,23 @@ gla_status run_chunk_bwd(const ChunkProblem& p, const float* s0, const void* dO,
                          cudaStream_t st);
 
 gla_status launch_wait_selftest(const WaitCtl& ctl, cudaStream_t st);
+
+// Inputs of one call for the checking build's precondition scan
+// (debug_checks.cu): the decay a (<= 0 and finite), bf16 token tensors and
+// fp32 states (finite).  debug_scan launches nothing in the normal build.
+struct DebugScan {
+    static constexpr int kMaxBf16 = 4, kMaxF32 = 2;
+    struct Rows {
+        const void* base;          // bf16; rows of `width` values, `ld` elements apart
+        int64_t rows, ld, width;
+    };
+    const float* a = nullptr;
+    int64_t na = 0;
+    Rows bf16[kMaxBf16] = {};
+    const float* f32[kMaxF32] = {};
+    int64_t nf32[kMaxF32] = {};
+};
+gla_status debug_scan(const DebugScan& s, int* status, cudaStream_t st);
 
 // Sequence split across ranks (chunk_seg.cu).
 size_t segment_workspace_bytes(int B, int T, int H);

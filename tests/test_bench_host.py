@@ -8,39 +8,70 @@ import pytest
 import bench
 
 
-def test_algorithmic_bytes_per_chunk():
+def test_method_and_design_bytes_per_chunk():
     # bf16 tiles of one (batch, head, 128-token chunk): q, k 128x96x2; v, o, dO
-    # 128x192x2; a 128x4; a bf16 96x192 state 36,864; q.dq and k.dk 128x4 each
-    q = k = 128 * 96 * 2
-    v = o = dO = 128 * 192 * 2
-    a = 128 * 4
+    # 128x192x2; a 128x4; one bf16 plane of a 96x192 state 36,864; q.dq and
+    # k.dk 128x4 each
+    q = k = dq = dk = 128 * 96 * 2
+    v = o = dO = dv = 128 * 192 * 2
+    a = da = 128 * 4
     h = 96 * 192 * 2
-    assert bench.CHUNK_BYTES["chunk_fwd_fused_kernel"] == q + k + v + o + a == 147_968
-    assert bench.CHUNK_BYTES["chunk_state_fwd_kernel"] == k + v + a + h == 111_104
-    assert bench.CHUNK_BYTES["chunk_state_rev_kernel"] == q + dO + a + h == 111_104
-    # dq/dk: q, k, v, dO, h, D, a in; dq, dk, q.dq, k.dk out
-    assert bench.CHUNK_BYTES["bwd_dqdk_kernel"] == q + k + v + dO + 2 * h + a + q + k + 2 * a == 271_872
-    # dv: q, k, dO, D, a in; dv out
-    assert bench.CHUNK_BYTES["bwd_dv_kernel"] == q + k + dO + h + a + v == 184_832
-    assert bench.CHUNK_BYTES["da_finish_kernel"] == 3 * a
+    M, D = bench.METHOD_BYTES, bench.DESIGN_BYTES
+    assert M["chunk_fwd_fused_kernel"] == q + k + v + o + a == 147_968
+    assert M["chunk_state_fwd_kernel"] == k + v + a and D["chunk_state_fwd_kernel"] == 2 * h
+    assert M["chunk_state_rev_kernel"] == q + dO + a and D["chunk_state_rev_kernel"] == 2 * h
+    # dq/dk: q, k, v, dO, a in; dq, dk out (+ h and D as hi, lo planes; q.dq, k.dk)
+    assert M["bwd_dqdk_kernel"] == q + k + v + dO + a + dq + dk == 197_120
+    assert D["bwd_dqdk_kernel"] == 4 * h + 2 * a
+    # dv: q, k, dO, a in; dv out (+ the hi plane of D)
+    assert M["bwd_dv_kernel"] == q + k + dO + a + dv == 147_968
+    assert D["bwd_dv_kernel"] == h
+    assert M["da_finish_kernel"] == da
+    # the step: forward and backward inputs and outputs, 3,084 B per token-head
+    assert bench.STEP_BYTES == (q + k + v + a + o) + (q + k + v + dO + a + dq + dk + dv + da)
+    assert bench.STEP_BYTES == 3084 * 128
+
+
+def test_algorithmic_flops_per_chunk():
+    mm = lambda m, n, kk: 2 * m * n * kk  # noqa: E731
+    F = bench.CHUNK_FLOPS
+    assert F["chunk_fwd_fused_kernel"] == 18_874_368
+    assert F["chunk_state_fwd_kernel"] == F["chunk_state_rev_kernel"] == mm(96, 192, 128)
+    assert F["bwd_dqdk_kernel"] == mm(128, 128, 192) + 2 * mm(128, 96, 192) + 2 * mm(128, 96, 128)
+    assert F["bwd_dv_kernel"] == mm(128, 128, 96) + mm(128, 192, 128) + mm(128, 192, 96)
+    # forward 18.9 MF and backward 45.6 MF per chunk-head: 132 GF at B8 H16 T2048
+    assert bench.STEP_FLOPS * 8 * 16 * 16 == pytest.approx(132.07e9, rel=1e-4)
 
 
 def test_roofline_takes_the_dominant_kernel():
-    peaks = {"hbm_gbs": 6539.5}
+    peaks = {"hbm_gbs": 6539.5, "bf16_tflops": 1624.7, "bf16_tflops_sustained": 1376.7}
     units = 8 * 16 * 16
     summary = [("chunk_fwd_fused_kernel", 3, 3 * 0.108), ("bwd_dqdk_kernel", 3, 3 * 0.155),
                ("bwd_dv_kernel", 3, 3 * 0.092)]
     roof, shares = bench.kernel_roofline(summary, peaks, "measured", units, 8, 16)
     assert roof["kernel"] == "bwd_dqdk_kernel"
-    by = bench.CHUNK_BYTES["bwd_dqdk_kernel"] * units
+    by = bench.METHOD_BYTES["bwd_dqdk_kernel"] * units
     assert roof["bytes_per_launch"] == by
+    assert roof["design_bytes_per_launch"] == bench.DESIGN_BYTES["bwd_dqdk_kernel"] * units
     assert roof["achieved"] == pytest.approx(by / 155e-6 / 1e9, rel=1e-3)
     assert roof["frac"] == pytest.approx(roof["achieved"] / 6539.5, rel=1e-3)
     assert roof["bound"] == "hbm" and roof["unit"] == "GB/s"
+    fl = bench.CHUNK_FLOPS["bwd_dqdk_kernel"] * units
+    assert roof["tensor"]["achieved"] == pytest.approx(fl / 155e-6 / 1e12, rel=1e-3)
+    assert roof["tensor"]["frac"] == pytest.approx(roof["tensor"]["achieved"] / 1376.7, rel=1e-3)
     assert sum(shares.values()) == pytest.approx(1.0, abs=1e-3)
     # the fused forward also writes the final state of every head
     roof_f, _ = bench.kernel_roofline(summary[:1], peaks, "measured", units, 8, 16)
-    assert roof_f["bytes_per_launch"] == bench.CHUNK_BYTES["chunk_fwd_fused_kernel"] * units + 73_728 * 8 * 16
+    assert roof_f["bytes_per_launch"] == bench.METHOD_BYTES["chunk_fwd_fused_kernel"] * units + 73_728 * 8 * 16
+
+
+def test_step_roofline():
+    peaks = {"hbm_gbs": 6539.5, "bf16_tflops": 1624.7, "bf16_tflops_sustained": 1376.7}
+    r = bench.step_roofline(0.4568e-3, 8 * 16 * 16, 8, 16, peaks, "measured")
+    # 808.5 MB of inputs and outputs + 9.4 MB of final state per step
+    assert r["hbm"]["bytes_per_step"] == 3084 * 262_144 + 73_728 * 128
+    assert r["hbm"]["frac"] == pytest.approx(817.9e6 / 0.4568e-3 / 6539.5e9, rel=1e-3)
+    assert r["tensor"]["frac"] == pytest.approx(132.07e9 / 0.4568e-3 / 1376.7e12, rel=1e-3)
 
 
 def test_recorded_traffic_only_for_the_profiled_sources(monkeypatch):

@@ -110,9 +110,9 @@ def test_chunk_bwd_validation(L):
 
 
 def test_decode_validation(L):
-    def dec(state=0x1000, slot=None, q=0x2000, k=0x3000, v=0x4000, a=0x5000, o=0x6000, N=4,
+    def dec(state=0x1000, slot=None, ns=4, q=0x2000, k=0x3000, v=0x4000, a=0x5000, o=0x6000, N=4,
             H=16, dk=96, dv=192, scale=96 ** -0.5):
-        return L.gla_decode_step(P(state), P(slot), P(q), P(k), P(v), P(a), P(o), N, H, dk, dv,
+        return L.gla_decode_step(P(state), P(slot), ns, P(q), P(k), P(v), P(a), P(o), N, H, dk, dv,
                                  scale, None)
     assert dec(state=None) == INVALID
     assert dec(o=None) == INVALID
@@ -121,6 +121,8 @@ def test_decode_validation(L):
     assert dec(scale=0.0) == INVALID
     assert dec(state=0x1004) == MISALIGNED
     assert dec(slot=0x7002) == MISALIGNED
+    assert dec(ns=-1) == INVALID
+    assert dec(ns=3) == INVALID                 # identity slots need N_slots >= N
     assert dec(N=0) == OK
 
 
@@ -161,16 +163,17 @@ def test_varlen_validation(L):
 
 
 def test_conv_decode_and_backward_validation(L):
-    def dec(x=0x1000, slot=None, ln=1, g=None, b=None, eps=1e-5, w=0x2000, bias=None, cs=0x3000, y=0x4000,
+    def dec(x=0x1000, slot=None, ns=4, ln=1, g=None, b=None, eps=1e-5, w=0x2000, bias=None, cs=0x3000, y=0x4000,
             N=4, D=3072, W=4):
-        return L.conv1d_silu_decode_step(P(x), P(slot), ln, P(g), P(b), eps, P(w), P(bias), P(cs), P(y), N, D, W,
-                                         None)
+        return L.conv1d_silu_decode_step(P(x), P(slot), ns, ln, P(g), P(b), eps, P(w), P(bias), P(cs), P(y), N, D,
+                                         W, None)
     assert dec(x=None) == INVALID
     assert dec(cs=None) == INVALID
     assert dec(W=3) == UNSUPPORTED
     assert dec(D=12) == UNSUPPORTED
     assert dec(eps=-1.0) == INVALID
     assert dec(cs=0x3004) == MISALIGNED
+    assert dec(ns=2) == INVALID                 # identity slots need N_slots >= N
     assert dec(N=0) == OK
 
     need = gla.conv1d_silu_causal_bwd_workspace_bytes(1, 64, 3072)

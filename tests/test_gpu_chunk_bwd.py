@@ -3,10 +3,10 @@ reverse recurrence (itself pinned by finite differences on the CPU).
 
 Tolerances (tests/tolerances.py):
   dq, dk, dv (bf16)   rel L2 <= 1e-2, max-abs <= 5e-2 beyond bf16 storage rounding
-  da (fp32)           rel L2 <= 1e-2, max-abs <= 5e-2 * max(1, max|da|)
+  da (fp32)           rel L2 <= 1e-2, max-abs <= 5e-2
   dS_0 (fp32 state)   rel L2 <= 5e-3
-da is a reverse cumulative sum over the whole sequence, so its magnitude
-grows with T; its absolute bound scales with its own size (stated reading).
+Every case prints, per gradient, the relative L2 and the raw max-abs error
+(and for the bf16 gradients the max-abs beyond storage rounding).
 """
 import numpy as np
 import pytest
@@ -61,15 +61,17 @@ def check_bwd(d, grads, units=None, dsT=None):
         report[name] = assert_bf16_close(g, r, name)
     e_da = rel_l2(got[3], ra)
     m_da = float(np.max(np.abs(got[3] - ra)))
-    assert e_da <= REL_BF16, "da rel L2 %.3g" % e_da
-    assert m_da <= ABS_BF16 * max(1.0, float(np.max(np.abs(ra)))), "da max-abs %.3g" % m_da
     report["da"] = (e_da, m_da, float(np.max(np.abs(ra))))
+    print("(rel L2, raw max-abs, beyond-rounding max-abs) per bf16 gradient; da: (rel L2, raw max-abs, max|da|)")
+    print(" ".join("%s=%s" % (k, tuple(float("%.4g" % x) for x in v)) for k, v in report.items()))
+    assert e_da <= REL_BF16, "da rel L2 %.3g" % e_da
+    assert m_da <= ABS_BF16, "da max-abs %.3g" % m_da
     if got[4] is not None:
         e = rel_l2(got[4], rs0)
         assert e <= REL_STATE, "dS0 rel L2 %.3g" % e
         report["ds0"] = e
-    print(" ".join("%s=%s" % (k, tuple(round(x, 5) for x in v) if isinstance(v, tuple) else round(v, 6))
-                   for k, v in report.items()))
+    if "ds0" in report:
+        print("ds0 rel L2 %.4g" % report["ds0"])
     return report
 
 
@@ -131,10 +133,14 @@ def test_chunk_bwd_strong_decay_and_no_decay(mean):
 
     da is a sum of terms that cancel: under a ~ -8 the diagonal parts of q.dq
     and k.dk cancel, and <dS_T, S_T> cancels k_T . (dS_T v_T), leaving da some
-    three orders of magnitude below the terms.  The per-chunk state copies the
-    kernels read are bf16, so da's absolute error is bounded by their rounding
-    of those terms; its bound is max-abs <= 1e-2 * the larger of max|da| and
-    the largest cancelling term (max |q.dq|, |k.dk|, |<dS_T, S_T>|)."""
+    two to three orders of magnitude below the terms.  Every case meets the
+    absolute max-abs <= 5e-2 of the workloads.  With a = 0 and the mixed
+    decays da also keeps rel L2 <= 1e-2.  Under a ~ -8 its error is set by
+    the precision of the cancelling terms themselves: they are products with
+    one operand carried as a bf16 hi + lo pair (within 2^-17 of its value)
+    summed in fp32, so the bound is max-abs <= 2^-15 (four such roundings) of
+    the largest cancelling term (max |q.dq|, |k.dk|, |<dS_T, S_T>|); its rel
+    L2 is printed."""
     B, T, H = 2, 512, 2
     seed = 230 if mean is None else 231 + int(mean * 10)
     d = inputs.chunk_inputs(B, T, H, seed=seed, device="cuda", s0_std=0.1, with_dO=True)
@@ -154,4 +160,11 @@ def test_chunk_bwd_strong_decay_and_no_decay(mean):
                 np.max(np.abs(np.einsum("bthd,bthd->bth", k, ref[1]))),
                 np.max(np.abs(np.einsum("bhij,bhij->bh", _np(ds), s_T))))
     err = np.max(np.abs(_np(grads[3]) - ref[3]))
-    assert err <= 1e-2 * max(np.max(np.abs(ref[3])), terms), "da max-abs %.3g (terms %.3g)" % (err, terms)
+    e_da = rel_l2(_np(grads[3]), ref[3])
+    print("da: rel L2 %.4g, raw max-abs %.4g, max|da| %.4g, largest cancelling term %.4g"
+          % (e_da, err, np.max(np.abs(ref[3])), terms))
+    assert err <= ABS_BF16, "da max-abs %.3g" % err
+    if mean == -8.0:
+        assert err <= 2.0 ** -15 * terms, "da max-abs %.3g (terms %.3g)" % (err, terms)
+    else:
+        assert e_da <= REL_BF16, "da rel L2 %.3g" % e_da

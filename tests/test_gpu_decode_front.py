@@ -61,6 +61,47 @@ def test_decode_slot_indirection_leaves_other_slots_untouched():
     assert torch.equal(d["state"][untouched], before[untouched])      # bit-exact
 
 
+def test_decode_slot_outside_the_pool_is_skipped_and_reported():
+    """A slot map entry outside [0, N_slots) (here N_slots and -1) touches no
+    state and no output and records GLA_ERR_INVALID_ARG in the device status
+    word; every other sequence is updated as usual.  The kernel checks the
+    slot before any access, so the bad entries never address memory."""
+    N, H, slots = 6, 2, 8
+    d = inputs.decode_inputs(N, H, seed=32, device="cuda", n_slots=slots)[0]
+    idx = torch.tensor([3, slots, 0, -1, 7, 5], dtype=torch.int32, device="cuda")
+    good = [0, 2, 4, 5]
+    before = d["state"].clone()
+    o = torch.full((N, H, 192), 1234.5, dtype=torch.float32, device="cuda")
+    gla.gla_decode_step(d["state"], d["q"], d["k"], d["v"], d["a"], o=o, slot_idx=idx)
+    assert gla.gla_get_device_status() == 1                 # GLA_ERR_INVALID_ARG
+    assert gla.gla_get_device_status() == 0                 # read clears it
+    g = torch.tensor(good)
+    ref_state, ref_o = recurrent.decode(_np(before), _np(d["q"][g]), _np(d["k"][g]), _np(d["v"][g]),
+                                        _np(d["a"][g]), slot_idx=idx[g].cpu().numpy())
+    assert rel(_np(d["state"]), ref_state) <= 1e-5
+    assert rel(_np(o[g]), ref_o) <= 1e-5
+    assert torch.all(o[[1, 3]] == 1234.5)                    # skipped rows not written
+    untouched = sorted(set(range(slots)) - set(idx[g].cpu().tolist()))
+    assert torch.equal(d["state"][untouched], before[untouched])
+
+
+def test_decode_front_slot_outside_the_pool_is_skipped_and_reported():
+    N, D, n_slots = 4, 256, 5
+    x, w, pool, _ = _pool_inputs(N, D, n_slots, 66)
+    idx = torch.tensor([1, n_slots, 4, -2], dtype=torch.int32, device="cuda")
+    before = pool.clone()
+    y = torch.full((N, D), 7.0, dtype=torch.bfloat16, device="cuda")
+    gla.conv1d_silu_decode_step(x, w, pool, slot_idx=idx, y=y)
+    assert gla.gla_get_device_status() == 1
+    good = torch.tensor([0, 2])
+    hist = _np(before[idx[good].long()])
+    ref_y, ref_cs = recurrent.ln_conv_silu(_np(x[good])[:, None, :], _np(w), conv_state=hist)
+    _front_check(_np(y[good]), ref_y[:, 0])
+    assert rel(_np(pool[idx[good].long()]), ref_cs) <= 1e-5
+    assert torch.all(y[[1, 3]] == 7.0)
+    assert torch.equal(pool[[0, 2, 3]], before[[0, 2, 3]])
+
+
 def test_decode_repeated_steps_match_recurrence():
     """T decode steps from S_0 equal the forward recurrence over T tokens."""
     N, H, T = 8, 2, 5

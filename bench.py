@@ -2,8 +2,10 @@
 """Benchmark of the Simple GLA mixer hot path on B200.
 
 One step = one training step of one Laplace-layer mixer at B = 8, T = 2048,
-H = 16, dk = 96, dv = 192 in bf16: gla_chunk_fwd followed by gla_chunk_bwd
-(dO ~ N(0,1), zero gradient on the final state).  The headline value is
+H = 16, dk = 96, dv = 192 in bf16: the chunked forward followed by the
+chunked backward (dO ~ N(0,1), zero gradient on the final state), as the
+library's training pair gla_chunk_fwd_train (which keeps the state entering
+every chunk) and gla_chunk_bwd_saved (which reads them).  The headline value is
 chunk fwd+bwd tokens/s over all ranks.  The metric also names decode
 tokens/s at 1,280 sequences, so the same run times the 24-layer decode step
 (1,280 sequences x 24 layers x 16 heads, fp32 state in place) and reports
@@ -82,6 +84,7 @@ METHOD_BYTES = {
 # per-chunk states as bf16 hi + lo planes, the per-token halves of the da
 # sum), reported beside the method bytes and not counted in the fraction.
 DESIGN_BYTES = {
+    "chunk_fwd_fused_kernel": 2 * HS,                   # training forward: h_c kept (hi, lo)
     "chunk_state_fwd_kernel": 2 * HS,                   # h_c written (hi, lo)
     "chunk_state_rev_kernel": 2 * HS,                   # D_c written (hi, lo)
     "bwd_dqdk_kernel": 2 * 2 * HS + 2 * A,              # h_c, D_c read (hi, lo); q.dq, k.dk written
@@ -103,7 +106,8 @@ CHUNK_FLOPS = {
 }
 # The whole training step per unit: forward (q, k, v, a in, o out) and
 # backward (q, k, v, dO, a in; dq, dk, dv, da out) method bytes, and the
-# forward + backward algorithmic flops.
+# forward + backward algorithmic flops (18.9 + 45.6 MF: the backward counted
+# with both state scans, whichever kernel runs them).
 STEP_BYTES = (2 * QK + 2 * VO + A) + (2 * QK + 2 * VO + A + 2 * QK + VO + A)
 STEP_FLOPS = sum(CHUNK_FLOPS.values())
 
@@ -247,15 +251,19 @@ def train_buffers(seed, device="cuda"):
                   torch.empty_like(d["a"]), None)
     d["ws_f"] = torch.empty(max(1, gla.gla_chunk_workspace_bytes(w.B, w.T, w.H)), dtype=torch.uint8,
                             device=dev)
-    d["ws_b"] = torch.empty(gla.gla_chunk_workspace_bytes(w.B, w.T, w.H, for_bwd=True),
+    d["ws_b"] = torch.empty(gla.gla_chunk_workspace_bytes(w.B, w.T, w.H, for_bwd=True, from_saved=True),
                             dtype=torch.uint8, device=dev)
+    d["saved"] = torch.empty(gla.gla_chunk_saved_state_bytes(w.B, w.T, w.H), dtype=torch.uint8, device=dev)
     return d
 
 
 def train_step(d):
-    gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], o=d["o"], s_final=d["sf"], ws=d["ws_f"])
-    gla.gla_chunk_bwd(d["q"], d["k"], d["v"], d["a"], d["dO"], grads=d["grads"], ws=d["ws_b"],
-                      want_grad_s0=False)
+    """One training step of the mixer: the forward that keeps the per-chunk
+    states, then the backward that reads them."""
+    gla.gla_chunk_fwd_train(d["q"], d["k"], d["v"], d["a"], o=d["o"], s_final=d["sf"], saved=d["saved"],
+                            ws=d["ws_f"])
+    gla.gla_chunk_bwd_saved(d["q"], d["k"], d["v"], d["a"], d["saved"], d["dO"], grads=d["grads"], ws=d["ws_b"],
+                            want_grad_s0=False)
 
 
 def kernel_roofline(summary, peaks, peak_kind, units_per_launch, B, H):
@@ -488,6 +496,7 @@ def run_e2e(args, ws, d, st):
         second[n] = torch.empty_like(d[n])
     second["o"] = torch.empty_like(d["o"])
     second["sf"] = torch.empty_like(d["sf"])
+    second["saved"] = torch.empty_like(d["saved"])
     second["grads"] = tuple(None if g is None else torch.empty_like(g) for g in d["grads"])
     sets = (d, second)
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
@@ -628,6 +637,13 @@ def run_long_prefill(args, ws, peaks, peak_kind):
     def front():
         gla.conv1d_silu_causal(f["x"], f["w"], y=y)
 
+    dy = inputs.randn((w.B, w.T, w.D), w.seed + 3, "cuda", dtype=torch.bfloat16)
+    wsb = torch.empty(max(16, gla.conv1d_silu_causal_bwd_workspace_bytes(w.B, w.T, w.D, w.W)), dtype=torch.uint8,
+                      device="cuda")
+
+    def front_bwd():
+        gla.conv1d_silu_causal_bwd(f["x"], f["w"], dy, ws=wsb, want=("dx", "dw"))
+
     def mixer():
         gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], s0=d["s0"], o=o, s_final=sf, ws=wsf)
 
@@ -646,7 +662,9 @@ def run_long_prefill(args, ws, peaks, peak_kind):
 
     n = max(1, min(args.steps, 20))
     t_front, t_mix = timed(front, n), timed(mixer, n)
+    t_fbwd = timed(front_bwd, max(1, min(n, 10)))
     front_bytes = w.B * w.T * w.D * 4                       # x in, y out (bf16)
+    front_bwd_bytes = w.B * w.T * w.D * 6                   # x, dy in, dx out (bf16)
     units = w.B * w.H * ((w.T + 127) // 128)
     mix_bytes = METHOD_BYTES["chunk_fwd_fused_kernel"] * units + 2 * FS * w.B * w.H   # + S_0 in, S_T out
 
@@ -660,10 +678,13 @@ def run_long_prefill(args, ws, peaks, peak_kind):
            "ms_per_step": round((t_front + t_mix) * 1e3, 4),
            "front_end": {"us_per_launch": round(t_front * 1e6, 2),
                          "roofline": roof("ln_conv_silu_kernel", front_bytes, t_front)},
+           "front_end_bwd": {"us_per_launch": round(t_fbwd * 1e6, 2),
+                             "roofline": roof("conv1d_silu_causal_bwd (row statistics, two tile passes, reduction)",
+                                              front_bwd_bytes, t_fbwd)},
            "gla_fwd": {"us_per_launch": round(t_mix * 1e6, 2),
                        "roofline": roof("gla_chunk_fwd (segmented: state pre-pass, combine, fused pass)",
                                         mix_bytes, t_mix)}}
-    del f, y, d, o, sf, wsf
+    del f, y, d, o, sf, wsf, dy, wsb
     torch.cuda.empty_cache()
     return out
 

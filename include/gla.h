@@ -99,7 +99,8 @@ int gla_build_flags(void);
  *   s_final [B, H, dk, dv] fp32     final state S_T; NULL to skip.
  *   ws      workspace of ws_bytes >= gla_chunk_workspace_bytes(B,T,H,dk,dv,0)
  *           (may be NULL when that size is 0).  Its contents on entry do not
- *           matter and are undefined on return.
+ *           matter and are undefined on return.  (for_bwd: 0 forward, 1
+ *           gla_chunk_bwd, 2 gla_chunk_bwd_saved.)
  *   scale   multiplies q once (normally dk^-1/2); must be > 0 and finite.
  *   dt      GLA_BF16 (tensor-core path: fp32 accumulation, fp32 state) or
  *           GLA_F32 (fp32 CUDA-core path, for small problems).
@@ -112,6 +113,40 @@ gla_status gla_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          const float* s0, void* o, float* s_final, void* ws, size_t ws_bytes,
                          int B, int T, int H, int dk, int dv, int64_t ld_qkv, float scale,
                          gla_dtype dt, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Training pair: a forward that also keeps what the backward needs, and the
+ * backward that reads it instead of recomputing it.  The backward needs the
+ * state entering every chunk (the states of the recurrence at the chunk
+ * boundaries, "Como i14 ...", section "Adaptaciones para AWS Trainium2",
+ * item 1); the forward computes them anyway, so it can write them out.
+ *
+ * gla_chunk_fwd_train: gla_chunk_fwd (same arguments and results) that also
+ * writes the state entering each chunk c of every (b, h) into `saved`:
+ *   saved   [B, H, NC, 2, dk, dv] bf16, NC = ceil(T / 128): plane 0 holds
+ *           bf16(S), plane 1 bf16(S - plane 0), together within 2^-17 of the
+ *           fp32 state; saved_bytes >= gla_chunk_saved_state_bytes(B,T,H,dk,dv).
+ * gla_chunk_bwd_saved: gla_chunk_bwd given those states (and, when ds_final is
+ * given, the forward's s_final, which the dS_T term of da needs) in place of
+ * s0; it skips the backward's own state-recompute pass.  Its workspace is
+ * gla_chunk_workspace_bytes(B,T,H,dk,dv, 2) (smaller than the plain
+ * backward's: no state planes of its own).  Results equal gla_chunk_bwd's.
+ * Both: dt must be GLA_BF16; other arguments, layouts and status codes as
+ * gla_chunk_fwd / gla_chunk_bwd.
+ * ------------------------------------------------------------------------ */
+size_t gla_chunk_saved_state_bytes(int B, int T, int H, int dk, int dv);
+
+gla_status gla_chunk_fwd_train(const void* q, const void* k, const void* v, const float* a,
+                               const float* s0, void* o, float* s_final, void* saved, size_t saved_bytes,
+                               void* ws, size_t ws_bytes, int B, int T, int H, int dk, int dv,
+                               int64_t ld_qkv, float scale, gla_dtype dt, cudaStream_t stream);
+
+gla_status gla_chunk_bwd_saved(const void* q, const void* k, const void* v, const float* a,
+                               const void* saved, size_t saved_bytes, const float* s_final,
+                               const void* dO, const float* ds_final, void* grad_q, void* grad_k,
+                               void* grad_v, float* grad_a, float* grad_s0, void* ws, size_t ws_bytes,
+                               int B, int T, int H, int dk, int dv, int64_t ld_qkv, float scale,
+                               gla_dtype dt, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Chunked forward over a packed batch of sequences of different lengths
@@ -128,13 +163,24 @@ gla_status gla_chunk_fwd(const void* q, const void* k, const void* v, const floa
  *               outside 0 .. total_T is skipped and GLA_ERR_INVALID_ARG is
  *               recorded in the device status word (gla_get_device_status).
  *   s0, s_final [N, H, 96, 192] fp32 or NULL (zeros / not wanted).
+ *   ws          workspace of ws_bytes >= gla_chunk_varlen_workspace_bytes(N,
+ *               total_T, H, dk, dv), or NULL.  With it, sequences longer than a
+ *               segment (a length the library derives from total_T and H)
+ *               are cut into segments that run in parallel (state-only
+ *               pre-pass, fp32 fold, output pass), so one long sequence no
+ *               longer sets the time; without it (or when the size is 0) each
+ *               (sequence, head) is one sweep.  Contents on entry do not
+ *               matter.  When cu_seqlens is invalid and a workspace is given,
+ *               the outputs of the valid sequences are undefined as well.
  * Rows of o outside every sequence are not written.  dt must be GLA_BF16;
- * N <= 65535.  No workspace.
+ * N <= 65535.
  * ------------------------------------------------------------------------ */
+size_t gla_chunk_varlen_workspace_bytes(int N, int total_T, int H, int dk, int dv);
+
 gla_status gla_chunk_fwd_varlen(const void* q, const void* k, const void* v, const float* a,
                                 const int32_t* cu_seqlens, int N, const float* s0, void* o,
-                                float* s_final, int total_T, int H, int dk, int dv, int64_t ld_qkv,
-                                float scale, gla_dtype dt, cudaStream_t stream);
+                                float* s_final, void* ws, size_t ws_bytes, int total_T, int H, int dk,
+                                int dv, int64_t ld_qkv, float scale, gla_dtype dt, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
  * gla_chunk_fwd for callers that cannot allocate device memory.  (The pages

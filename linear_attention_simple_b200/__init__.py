@@ -25,7 +25,9 @@ __all__ = [
     "gla_selftest_wait_timeout", "gla_trace_enable", "gla_trace_summary",
     "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step", "conv1d_silu_causal_bwd",
     "conv1d_silu_causal_bwd_workspace_bytes", "gla_chunk_fwd_varlen", "gla_segment_workspace_bytes",
-    "gla_segment_state_fwd", "gla_segment_state_bwd", "gla_state_fold", "gla_build_flags", "EXPORTED_SYMBOLS",
+    "gla_segment_state_fwd", "gla_segment_state_bwd", "gla_state_fold", "gla_build_flags",
+    "gla_chunk_varlen_workspace_bytes", "gla_chunk_saved_state_bytes", "gla_chunk_fwd_train",
+    "gla_chunk_bwd_saved", "EXPORTED_SYMBOLS",
     "LIB_PATH", "LIB_DEBUG_PATH", "GLA_BUILD_DEBUG_BOUNDS",
 ]
 
@@ -41,6 +43,8 @@ EXPORTED_SYMBOLS = (
     "gla_chunk_fwd_noalloc", "conv1d_silu_decode_step", "conv1d_silu_causal_bwd",
     "conv1d_silu_causal_bwd_workspace_bytes", "gla_chunk_fwd_varlen", "gla_segment_workspace_bytes",
     "gla_segment_state_fwd", "gla_segment_state_bwd", "gla_state_fold", "gla_build_flags",
+    "gla_chunk_varlen_workspace_bytes", "gla_chunk_saved_state_bytes", "gla_chunk_fwd_train",
+    "gla_chunk_bwd_saved",
 )
 
 GLA_BF16, GLA_F32 = 0, 1
@@ -99,6 +103,14 @@ def declare(L):
     L.gla_chunk_bwd.restype = _i
     L.gla_chunk_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _vp, ctypes.c_size_t, _i, _i, _i, _i, _i, _i64, _f, _i, _vp]
+    L.gla_chunk_saved_state_bytes.restype = ctypes.c_size_t
+    L.gla_chunk_saved_state_bytes.argtypes = [_i, _i, _i, _i, _i]
+    L.gla_chunk_fwd_train.restype = _i
+    L.gla_chunk_fwd_train.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp,
+                                      ctypes.c_size_t, _i, _i, _i, _i, _i, _i64, _f, _i, _vp]
+    L.gla_chunk_bwd_saved.restype = _i
+    L.gla_chunk_bwd_saved.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp, _vp,
+                                      _vp, _vp, _vp, ctypes.c_size_t, _i, _i, _i, _i, _i, _i64, _f, _i, _vp]
     L.gla_decode_step.restype = _i
     L.gla_decode_step.argtypes = [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _vp]
     L.conv1d_silu_causal.restype = _i
@@ -110,8 +122,10 @@ def declare(L):
     L.conv1d_silu_causal_bwd.argtypes = [_vp, _i, _vp, _vp, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                          _vp, _vp, ctypes.c_size_t, _i, _i, _i, _i, _vp]
     L.gla_chunk_fwd_varlen.restype = _i
-    L.gla_chunk_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _i, _i, _i, _i,
-                                       ctypes.c_longlong, _f, _i, _vp]
+    L.gla_chunk_fwd_varlen.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, ctypes.c_size_t, _i,
+                                       _i, _i, _i, ctypes.c_longlong, _f, _i, _vp]
+    L.gla_chunk_varlen_workspace_bytes.restype = ctypes.c_size_t
+    L.gla_chunk_varlen_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
     L.gla_segment_workspace_bytes.restype = ctypes.c_size_t
     L.gla_segment_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
     L.gla_segment_state_fwd.restype = _i
@@ -206,8 +220,15 @@ def gla_build_flags():
     return int(lib().gla_build_flags())
 
 
-def gla_chunk_workspace_bytes(B, T, H, dk=96, dv=192, for_bwd=False):
-    return int(lib().gla_chunk_workspace_bytes(B, T, H, dk, dv, 1 if for_bwd else 0))
+def gla_chunk_workspace_bytes(B, T, H, dk=96, dv=192, for_bwd=False, from_saved=False):
+    """Workspace bytes of gla_chunk_fwd (default), gla_chunk_bwd (for_bwd) or
+    gla_chunk_bwd_saved (for_bwd and from_saved)."""
+    mode = (2 if from_saved else 1) if for_bwd else 0
+    return int(lib().gla_chunk_workspace_bytes(B, T, H, dk, dv, mode))
+
+
+def gla_chunk_saved_state_bytes(B, T, H, dk=96, dv=192):
+    return int(lib().gla_chunk_saved_state_bytes(B, T, H, dk, dv))
 
 
 def _qkv_strides(q, k, v):
@@ -294,6 +315,78 @@ def gla_chunk_bwd(q, k, v, a, dO, s0=None, ds_final=None, grads=None, ws=None, s
     return gq, gk, gv, ga, gs0
 
 
+def gla_chunk_fwd_train(q, k, v, a, s0=None, o=None, s_final=None, saved=None, ws=None, scale=None,
+                        stream=None):
+    """gla_chunk_fwd that also keeps the state entering every chunk (bf16 hi
+    and lo planes) for gla_chunk_bwd_saved.  Returns (o, s_final, saved);
+    saved is a uint8 tensor of gla_chunk_saved_state_bytes bytes."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype != torch.bfloat16:
+        raise TypeError("gla_chunk_fwd_train takes bf16 q, k, v")
+    ld = _qkv_strides(q, k, v)
+    _need(a, "a", torch.float32, (B, T, H))
+    _need(s0, "s0", torch.float32, (B, H, dk, dv))
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    _need(o, "o", q.dtype, (B, T, H, dv))
+    if s_final is None:
+        s_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    _need(s_final, "s_final", torch.float32, (B, H, dk, dv))
+    nsv = gla_chunk_saved_state_bytes(B, T, H, dk, dv)
+    if saved is None:
+        saved = torch.empty(max(nsv, 16), dtype=torch.uint8, device=q.device)
+    _need(saved, "saved", torch.uint8)
+    need = gla_chunk_workspace_bytes(B, T, H, dk, dv)
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    sc = dk ** -0.5 if scale is None else scale
+    st = lib().gla_chunk_fwd_train(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(s0), _ptr(o), _ptr(s_final),
+                                   _ptr(saved), saved.numel(), _ptr(ws), 0 if ws is None else ws.numel(),
+                                   B, T, H, dk, dv, ld, float(sc), GLA_BF16, _stream(stream))
+    _check("gla_chunk_fwd_train", st)
+    return o, s_final, saved
+
+
+def gla_chunk_bwd_saved(q, k, v, a, saved, dO, s_final=None, ds_final=None, grads=None, ws=None, scale=None,
+                        want_grad_s0=True, stream=None):
+    """gla_chunk_bwd from the states gla_chunk_fwd_train kept (s_final is
+    needed only with ds_final).  Returns (dq, dk, dv, da, ds0)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if q.dtype != torch.bfloat16:
+        raise TypeError("gla_chunk_bwd_saved takes bf16 q, k, v")
+    ld = _qkv_strides(q, k, v)
+    _need(a, "a", torch.float32, (B, T, H))
+    _need(dO, "dO", q.dtype, (B, T, H, dv))
+    _need(saved, "saved", torch.uint8)
+    _need(s_final, "s_final", torch.float32, (B, H, dk, dv))
+    _need(ds_final, "ds_final", torch.float32, (B, H, dk, dv))
+    dev = q.device
+    if grads is None:
+        grads = (torch.empty((B, T, H, dk), dtype=q.dtype, device=dev),
+                 torch.empty((B, T, H, dk), dtype=q.dtype, device=dev),
+                 torch.empty((B, T, H, dv), dtype=q.dtype, device=dev),
+                 torch.empty((B, T, H), dtype=torch.float32, device=dev),
+                 torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev) if want_grad_s0 else None)
+    gq, gk, gv, ga, gs0 = grads
+    _need(gq, "grad_q", q.dtype, (B, T, H, dk))
+    _need(gk, "grad_k", q.dtype, (B, T, H, dk))
+    _need(gv, "grad_v", q.dtype, (B, T, H, dv))
+    _need(ga, "grad_a", torch.float32, (B, T, H))
+    _need(gs0, "grad_s0", torch.float32, (B, H, dk, dv))
+    need = gla_chunk_workspace_bytes(B, T, H, dk, dv, for_bwd=True, from_saved=True)
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    sc = dk ** -0.5 if scale is None else scale
+    st = lib().gla_chunk_bwd_saved(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(saved), saved.numel(), _ptr(s_final),
+                                   _ptr(dO), _ptr(ds_final), _ptr(gq), _ptr(gk), _ptr(gv), _ptr(ga), _ptr(gs0),
+                                   _ptr(ws), 0 if ws is None else ws.numel(), B, T, H, dk, dv, ld, float(sc),
+                                   GLA_BF16, _stream(stream))
+    _check("gla_chunk_bwd_saved", st)
+    return gq, gk, gv, ga, gs0
+
+
 def gla_decode_step(state, q, k, v, a, o=None, slot_idx=None, scale=None, stream=None):
     """In-place decode step.  state [N_slots,H,dk,dv] fp32; q, k [N,H,dk] and
     v [N,H,dv] bf16; a [N,H] fp32; slot_idx [N] int32 or None (a slot outside
@@ -345,10 +438,16 @@ def conv1d_silu_causal(x, w, apply_ln=True, ln_gamma=None, ln_beta=None, ln_eps=
     return y
 
 
+def gla_chunk_varlen_workspace_bytes(N, total_T, H, dk=96, dv=192):
+    return int(lib().gla_chunk_varlen_workspace_bytes(N, total_T, H, dk, dv))
+
+
 def gla_chunk_fwd_varlen(q, k, v, a, cu_seqlens, s0=None, o=None, s_final=None, scale=None,
-                         want_final_state=True, stream=None):
+                         want_final_state=True, ws=None, segmented=True, stream=None):
     """Chunked forward over packed sequences: q, k [total,H,96], v [total,H,192]
-    bf16, a [total,H] fp32, cu_seqlens [N+1] int32 on the device.  Returns
+    bf16, a [total,H] fp32, cu_seqlens [N+1] int32 on the device.  With
+    segmented (the default) a workspace is allocated when the caller passes
+    none, so long sequences are cut into parallel segments.  Returns
     (o [total,H,192] bf16, s_final [N,H,96,192] fp32 or None)."""
     total, H, dk = q.shape
     dv = v.shape[-1]
@@ -368,8 +467,13 @@ def gla_chunk_fwd_varlen(q, k, v, a, cu_seqlens, s0=None, o=None, s_final=None, 
         s_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
     _need(s_final, "s_final", torch.float32, (N, H, dk, dv))
     sc = dk ** -0.5 if scale is None else scale
+    if ws is None and segmented:
+        need = gla_chunk_varlen_workspace_bytes(N, total, H, dk, dv)
+        if need > 0:
+            ws = torch.empty(need, dtype=torch.uint8, device=q.device)
     st = lib().gla_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(cu_seqlens), N, _ptr(s0), _ptr(o),
-                                    _ptr(s_final), total, H, dk, dv, 0, float(sc), GLA_BF16, _stream(stream))
+                                    _ptr(s_final), _ptr(ws), 0 if ws is None else ws.numel(), total, H, dk, dv,
+                                    0, float(sc), GLA_BF16, _stream(stream))
     _check("gla_chunk_fwd_varlen", st)
     return o, s_final
 

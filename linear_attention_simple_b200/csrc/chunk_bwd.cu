@@ -905,13 +905,17 @@ size_t seg_scratch_bytes(int units, int nseg)
            align256(static_cast<size_t>(units) * nseg * sizeof(float));
 }
 
-size_t bwd_workspace_bytes(int B, int T, int H)
+// Layout: [h_c planes (not with saved states)] [D_c planes] [S_T (not with
+// saved states)] [q.dq, k.dk] [chunk totals] [<dS_T, S_T>] [anchors]
+// [segment scratch].
+size_t bwd_workspace_bytes(int B, int T, int H, bool from_saved)
 {
     const size_t units = static_cast<size_t>(B) * H, NC = num_chunks(T);
     const size_t states = align256(units * NC * kSS * 2 * 2);   // bf16 hi and lo planes
     int nseg, cps;
     chunk_segment_plan(static_cast<int>(units), static_cast<int>(NC), &nseg, &cps);
-    return 2 * states + align256(units * kSS * sizeof(float)) + align256(2 * units * T * sizeof(float)) +
+    const size_t own = from_saved ? 0 : states + align256(units * kSS * sizeof(float));
+    return own + states + align256(2 * units * T * sizeof(float)) +
            align256(units * NC * 2 * sizeof(float)) + align256(units * sizeof(float)) +
            align256(units * da_anchors(static_cast<int>(NC)) * sizeof(float)) +
            seg_scratch_bytes(static_cast<int>(units), nseg);
@@ -920,16 +924,22 @@ size_t bwd_workspace_bytes(int B, int T, int H)
 gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO,
                          const float* ds_final, void* dq, void* dk, void* dv, float* da,
                          float* ds0, void* ws, size_t ws_bytes, const WaitCtl& ctl,
-                         cudaStream_t st)
+                         cudaStream_t st, const void* saved, const float* s_final)
 {
     (void)ws_bytes;
     const int units = pr.B * pr.H, NC = num_chunks(pr.T);
     const size_t states = align256(static_cast<size_t>(units) * NC * kSS * 2 * 2);   // bf16 hi and lo planes
     uint8_t* wsb = static_cast<uint8_t*>(ws);
-    void* hbuf = wsb;
-    void* dbuf = wsb + states;
-    float* sT = reinterpret_cast<float*>(wsb + 2 * states);
-    size_t off = 2 * states + align256(static_cast<size_t>(units) * kSS * sizeof(float));
+    // with the forward's saved states (gla_chunk_fwd_train) h_c is read from
+    // there and S_T is the forward's final state; otherwise both are computed
+    // here by a state-only pass
+    size_t off = 0;
+    void* hbuf = saved ? const_cast<void*>(saved) : wsb;
+    if (!saved) off += states;
+    void* dbuf = wsb + off;
+    off += states;
+    float* sT = saved ? const_cast<float*>(s_final) : reinterpret_cast<float*>(wsb + off);
+    if (!saved) off += align256(static_cast<size_t>(units) * kSS * sizeof(float));
     float* delta = reinterpret_cast<float*>(wsb + off);
     off += align256(2 * static_cast<size_t>(units) * pr.T * sizeof(float));
     float* ctot = reinterpret_cast<float*>(wsb + off);
@@ -986,14 +996,16 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     sp.h_out = hbuf;
     sp.scale = pr.scale;
     sp.ctl = ctl;
-    if (nseg > 1) {
-        // local end states of segments 0 .. nseg-2 (the last one's is not needed)
-        if ((s = pre_pass(sp, false, nseg - 1, s0)) != GLA_OK) return s;
-        sp.s_init = segst;
-        sp.init_unit_stride = static_cast<int64_t>(nseg) * kSS;
-        sp.init_seg_stride = kSS;
+    if (!saved) {
+        if (nseg > 1) {
+            // local end states of segments 0 .. nseg-2 (the last one's is not needed)
+            if ((s = pre_pass(sp, false, nseg - 1, s0)) != GLA_OK) return s;
+            sp.s_init = segst;
+            sp.init_unit_stride = static_cast<int64_t>(nseg) * kSS;
+            sp.init_seg_stride = kSS;
+        }
+        if ((s = launch_state_kernel(false, false, sp, dim3(nseg, pr.H, pr.B), st)) != GLA_OK) return s;
     }
-    if ((s = launch_state_kernel(false, false, sp, dim3(nseg, pr.H, pr.B), st)) != GLA_OK) return s;
 
     // 2. D_c for every chunk, dS_0 (written by segment 0, where the reverse sweep ends)
     StateParams rp = sp;
@@ -1036,13 +1048,19 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     bp.NC = NC;
     bp.scale = pr.scale;
     bp.ctl = ctl;
-    if ((s = launch_bwd_kernel(bwd_dqdk_kernel, bq::BYTES, bp, dim3(2 * NC, pr.H, pr.B), st, "bwd_dqdk_kernel")) !=
-        GLA_OK)
-        return s;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    {
+        // persistent: one CTA per SM over the (batch, head, chunk) items
+        const int items = units * NC;
+        const int grid = items < sms ? items : sms;
+        (void)grid;
+        if ((s = launch_bwd_kernel(bwd_dqdk_kernel, bq::BYTES, bp, dim3(2 * NC, pr.H, pr.B), st,
+                                   "bwd_dqdk_kernel")) != GLA_OK)
+            return s;
+    }
     {
         // persistent: one CTA per SM over the (batch, head, chunk, dv half) items
-        int dev = 0, sms = 148;
-        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const int items = units * NC * 2;
         const int grid = items < sms ? items : sms;
         if ((s = launch_bwd_kernel(bwd_dv_kernel, dvp::BYTES, bp, dim3(grid), st, "bwd_dv_kernel", dvp::kThreads)) !=

@@ -71,6 +71,43 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(float* __restrict__ st
     }
 }
 
+// Segmented varlen forward: the state entering every segment of every
+// sequence, in place over the scratch slots.  On entry slot(n, s) holds the
+// pre-pass end state of segment s from zero (s < nseg_n - 1); on return it
+// holds the state entering segment s (s >= 1; segment 0 starts from s0).
+// One thread per (sequence, head, float4 of the state), walking the
+// sequence's segments in order.
+__global__ void __launch_bounds__(256) seg_combine_varlen_kernel(float* __restrict__ states,
+                                                                 const float* __restrict__ g2,
+                                                                 const float* __restrict__ s0,
+                                                                 const int* __restrict__ cu, int N, int H,
+                                                                 int total_T, int cps)
+{
+    const int64_t n4 = kSS / 4;
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= n4 * N * H) return;
+    const int64_t u = idx / n4, e4 = idx - u * n4;
+    const int n = static_cast<int>(u / H), h = static_cast<int>(u - static_cast<int64_t>(n) * H);
+    const int tb = cu[n], Tn = cu[n + 1] - tb;
+    if (tb < 0 || Tn < 0 || tb + Tn > total_T) return;   // reported by the pre-pass
+    const int nseg = max(1, ((Tn + 127) / 128 + cps - 1) / cps);
+    if (nseg == 1) return;
+    float4* st = reinterpret_cast<float4*>(states);
+    const int64_t slot0 = static_cast<int64_t>(n) + tb / (128 * cps);
+    float4 x = s0 ? reinterpret_cast<const float4*>(s0)[u * n4 + e4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sgm = 0; sgm < nseg - 1; ++sgm) {
+        const int64_t at = ((slot0 + sgm) * H + h) * n4 + e4;
+        const float4 l = st[at];
+        const float f = exp2f(g2[(slot0 + sgm) * H + h]);
+        if (sgm > 0) st[at] = x;
+        x.x = fmaf(f, x.x, l.x);
+        x.y = fmaf(f, x.y, l.y);
+        x.z = fmaf(f, x.z, l.z);
+        x.w = fmaf(f, x.w, l.w);
+    }
+    st[((slot0 + nseg - 1) * H + h) * n4 + e4] = x;
+}
+
 template <typename K>
 gla_status launch_chunk_kernel(K kernel, uint32_t bytes, const char* name, const StateParams& p,
                                dim3 grid, cudaStream_t st, int threads = chunk::kThreads)
@@ -155,10 +192,36 @@ size_t fwd_workspace_bytes(int B, int T, int H)
            align256(static_cast<size_t>(units) * nseg * sizeof(float));
 }
 
-gla_status run_chunk_fwd_varlen(const ChunkProblem& pr, const int* cu_seqlens, int N, const float* s0, void* o,
-                                float* s_final, const WaitCtl& ctl, cudaStream_t st)
+// Segment plan of the packed forward: chunks per segment such that the
+// (sequence, head, segment) CTAs number about four per SM if the tokens were
+// spread evenly (the lengths differ, so small pieces balance the waves; each
+// extra segment costs a pre-pass sweep), at least 4 chunks; 0 when no
+// sequence can be longer than one segment (total_T within it), i.e. no
+// segmenting.
+int varlen_chunks_per_seg(int total_T, int H)
 {
-    // pr.B == 1, pr.T == total tokens; one CTA per (sequence, head)
+    const int64_t per_cta = (static_cast<int64_t>(total_T) * H + 4 * kTargetCtas - 1) / (4 * kTargetCtas);
+    int cps = static_cast<int>((per_cta + 127) / 128);
+    if (cps < 4) cps = 4;
+    return static_cast<int64_t>(total_T) <= static_cast<int64_t>(cps) * 128 ? 0 : cps;
+}
+
+size_t varlen_workspace_bytes(int N, int total_T, int H)
+{
+    const int cps = varlen_chunks_per_seg(total_T, H);
+    if (cps == 0) return 0;
+    const int64_t L = static_cast<int64_t>(cps) * 128;
+    const int64_t slots = N + (total_T + L - 1) / L + 1;
+    return align256(static_cast<size_t>(slots) * H * kSS * sizeof(float)) +
+           align256(static_cast<size_t>(slots) * H * sizeof(float));
+}
+
+gla_status run_chunk_fwd_varlen(const ChunkProblem& pr, const int* cu_seqlens, int N, const float* s0, void* o,
+                                float* s_final, void* ws, size_t ws_bytes, const WaitCtl& ctl, cudaStream_t st)
+{
+    // pr.B == 1, pr.T == total tokens; one CTA per (sequence, head, segment)
+    const int cps = varlen_chunks_per_seg(pr.T, pr.H);
+    const bool segmented = cps > 0 && ws && ws_bytes >= varlen_workspace_bytes(N, pr.T, pr.H);
     StateParams p;
     memset(&p, 0, sizeof(p));
     gla_status s;
@@ -182,11 +245,44 @@ gla_status run_chunk_fwd_varlen(const ChunkProblem& pr, const int* cu_seqlens, i
     p.s_out = s_final;
     p.out_unit_stride = kSS;
     p.out_last_only = 1;
-    return launch_state_kernel(true, false, p, dim3(1, pr.H, N), st);
+    if (!segmented) return launch_state_kernel(true, false, p, dim3(1, pr.H, N), st);
+
+    // segments of cps chunks: state-only pre-pass from zero over every
+    // segment but each sequence's last, the fold that leaves the state
+    // entering each segment in its slot, then the fused pass per segment
+    const int64_t L = static_cast<int64_t>(cps) * 128;
+    const int max_segs = static_cast<int>((pr.T + L - 1) / L);
+    const int64_t slots = N + (pr.T + L - 1) / L + 1;
+    float* states = static_cast<float*>(ws);
+    float* g2 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                         align256(static_cast<size_t>(slots) * pr.H * kSS * sizeof(float)));
+    StateParams pre = p;
+    pre.chunks_per_seg = cps;
+    pre.seg_states = states;
+    pre.seg_g2 = g2;
+    pre.varlen_segs = 1;
+    pre.pre_pass = 1;
+    pre.s_init = nullptr;
+    pre.s_out = states;                 // written at each segment's slot
+    pre.out_last_only = 0;
+    if ((s = launch_state_kernel(false, false, pre, dim3(max_segs, pr.H, N), st)) != GLA_OK) return s;
+    {
+        const int64_t n = static_cast<int64_t>(N) * pr.H * (kSS / 4);
+        trace_begin(st);
+        seg_combine_varlen_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(states, g2, s0, cu_seqlens,
+                                                                                        N, pr.H, pr.T, cps);
+        trace_end(st, "seg_combine_varlen_kernel");
+        count_launch();
+        if ((s = check_launch("seg_combine_varlen_kernel")) != GLA_OK) return s;
+    }
+    p.chunks_per_seg = cps;
+    p.seg_states = states;
+    p.varlen_segs = 1;
+    return launch_state_kernel(true, false, p, dim3(max_segs, pr.H, N), st);
 }
 
 gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float* s_final,
-                         void* ws, size_t ws_bytes, const WaitCtl& ctl, cudaStream_t st)
+                         void* ws, size_t ws_bytes, const WaitCtl& ctl, cudaStream_t st, void* h_save)
 {
     (void)ws_bytes;
     const int units = pr.B * pr.H, NC = num_chunks(pr.T);
@@ -210,6 +306,7 @@ gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float
     p.scale = pr.scale;
     p.ctl = ctl;
     p.store_h = 0;
+    p.h_save = h_save;
 
     if (nseg == 1) {
         p.s_init = s0;
@@ -225,6 +322,7 @@ gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float
                                          align256(static_cast<size_t>(units) * nseg * kSS * sizeof(float)));
     // 1. local end states of segments 0..nseg-2
     StateParams pre = p;
+    pre.h_save = nullptr;
     pre.s_init = nullptr;
     pre.s_out = states;
     pre.out_unit_stride = nseg * kSS;

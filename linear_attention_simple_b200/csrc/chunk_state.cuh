@@ -14,9 +14,10 @@
 // Two kernels:
 //
 // gla_fwd_fused_kernel -- forward with the output fused in.  Per chunk:
-//   scores = Q K^T (tcgen05, 128x128x96); O = Q S_prev (128x192x96, the bf16
-//   state copy split into hi + lo terms); S += K~^T V (K~ = e^{gamma-b} K);
-//   O += P V (P split into bf16 hi + lo); epilogue o = r_i O_i.
+//   scores = Q K^T (tcgen05, 128x128x96); O = Q S_prev (128x192x96, against a
+//   bf16 copy of the state); S += K~^T V (K~ = e^{gamma-b} K split into bf16
+//   hi + lo, so the fp32 state keeps its precision); O += P V (P split into
+//   bf16 hi + lo); epilogue o = r_i O_i.
 //   Decay factorisation: while the chunk's total decay spans at most 2^100,
 //   e^{b_i - b_j} = e^{b_i} e^{-b_j} is split into a column factor folded
 //   into P (P'_ij = (q_i.k_j) 2^{-b_j}) and a row factor applied in the
@@ -77,6 +78,15 @@ struct StateParams {
     void* h_out;            // bf16 [B*H*NC][2][96][192]: plane 0 = bf16(S), plane 1 = bf16(S - plane 0)
     const int* cu_seqlens;  // varlen forward: [B+1] token offsets into batch row 0, or null
     void* o_direct;         // varlen forward: o, for the direct stores of a sequence's last chunk
+    // varlen forward cut into segments of chunks_per_seg chunks: segment s of
+    // sequence n owns scratch slot n + cu_seqlens[n] / (128 chunks_per_seg) + s
+    // (distinct for every (n, s), fewer than N + total / (128 chunks_per_seg) + 1)
+    float* seg_states;      // [slots][H][96][192] fp32: pre-pass end states, then entering states
+    float* seg_g2;          // [slots][H] total log2-decay of each segment (pre-pass)
+    int varlen_segs;        // 1: segmented varlen (chunks_per_seg chunks per segment)
+    int pre_pass;           // state pass: only segments 0 .. nseg_n - 2 of each sequence
+    void* h_save;           // fused forward: the state entering each chunk, [B*H*NC][2][96][192]
+                            // bf16 (hi, lo planes), for the backward; null = not saved
     float scale;
     WaitCtl ctl;
 };
@@ -104,8 +114,9 @@ constexpr uint32_t kIdStateTs = idesc_bf16_f32(128, 192, 0, 1);   // A from tens
 struct FusedSmem {
     static constexpr uint32_t Q = 0;          // q tile, permuted rows
     static constexpr uint32_t U = 24576;      // k tile, then K~ (its 4th M block is X: finite)
-    static constexpr uint32_t X = 49152;      // state copy hi [3][96][64] SW128; with XL, o staging
-    static constexpr uint32_t XL = 86016;     // state copy lo
+    static constexpr uint32_t X = 49152;      // bf16 state copy [3][96][64] SW128
+    static constexpr uint32_t KL = 86016;     // lo half of K~ [3][128][32] SW64 (hi: K~ in place in U)
+    static constexpr uint32_t KL_PAD = 110592;   // [8192] zeros: the 4th M block (dk 96..127) of KL
     static constexpr uint32_t Y0 = 122880;    // v tiles, double buffered
     static constexpr uint32_t Y1 = 172032;    // (the o staging of a chunk, once its P V is done)
     static constexpr uint32_t MISC = 221184;
@@ -124,6 +135,12 @@ struct PassSmem {
     // dS accumulator [192 cols]; U~^T hi (64 cols) + lo (64 cols) per buffer, two buffers
     static constexpr uint32_t TM_DS = 0, TM_U = 256;
 };
+
+// Scratch slot of segment s of sequence n in the segmented varlen forward.
+__device__ __forceinline__ int64_t varlen_slot(const int* cu, int n, int s, int chunks_per_seg)
+{
+    return static_cast<int64_t>(n) + cu[n] / (128 * chunks_per_seg) + s;
+}
 
 // Token held by row r of the permuted q tile: 16-row block r/16 holds token
 // block perm16(r/16) (0, 7, 1, 6, 2, 5, 3, 4), so lane quarter q (rows
@@ -269,15 +286,32 @@ __device__ __forceinline__ void tmem_to_state(uint32_t taddr, float* dst)
 
 // State copy into [3][96][64] SW128 (row = dk index, n = dv column), for the
 // 96 columns half*96 .. +95 of this thread's row; then decay the state.
+// With gsave, the same 96 values also go to global memory as a bf16 hi plane
+// (gsave) and lo plane (gsave + plane_bytes), 32-byte stores.
 template <bool SPLIT>
 __device__ __forceinline__ void state_copy_and_decay(uint32_t taddr, int row, int half, float f,
-                                                     uint8_t* hi, uint8_t* lo, bool copy)
+                                                     uint8_t* hi, uint8_t* lo, bool copy,
+                                                     uint8_t* gsave = nullptr, int64_t plane_bytes = 0)
 {
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
         uint32_t r[32];
         tmem_ld32(taddr + j * 32, r);
         tmem_ld_wait();
+        if (gsave) {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t w[8], l[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float x0 = __uint_as_float(r[16 * h2 + 2 * e]), x1 = __uint_as_float(r[16 * h2 + 2 * e + 1]);
+                    w[e] = pack_bf16(x0, x1);
+                    l[e] = pack_bf16(x0 - bf16_lo(w[e]), x1 - bf16_hi(w[e]));
+                }
+                st_global_v8(gsave + j * 64 + h2 * 32, w);
+                st_global_v8(gsave + plane_bytes + j * 64 + h2 * 32, l);
+            }
+        }
         if (copy) {
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
@@ -347,8 +381,14 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     }
     const int bc = VARLEN ? 0 : b;                 // batch coordinate of the token tensors
     const int c_begin = seg * p.chunks_per_seg;
+    // segmented varlen: a grid slot past this sequence's last segment has
+    // nothing to do (segment 0 always runs: an empty sequence still passes
+    // its initial state on)
+    if (VARLEN && seg > 0 && c_begin >= NCn) return;
     const int c_end = min(NCn, c_begin + p.chunks_per_seg);
     const int nchunks = c_end - c_begin;
+    const int last_seg = VARLEN ? max(1, (NCn + p.chunks_per_seg - 1) / p.chunks_per_seg) - 1
+                                : static_cast<int>(gridDim.x) - 1;
     const WaitCtl ctl = p.ctl;
 
     const int quad = warp & 3;
@@ -392,6 +432,13 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         const int t = c * 128 + tid;
         return t < Tn ? p.a[(static_cast<int64_t>(bc) * p.T + tb + t) * p.H + h] : 0.f;
     };
+    // this thread's row of the saved state entering chunk c (hi plane), or null
+    constexpr int64_t kStatePlane = static_cast<int64_t>(kDk) * kDv * 2;
+    auto save_row = [&](int c) -> uint8_t* {
+        if (VARLEN || !p.h_save || !GLA_DCHECK(c < p.NC && unit < p.B * p.H, p.ctl.status)) return nullptr;
+        return static_cast<uint8_t*>(p.h_save) + ((static_cast<int64_t>(unit) * p.NC + c) * 2) * kStatePlane +
+               static_cast<int64_t>(row) * (kDv * 2) + half * 192;
+    };
     // cumulative log2-decay of a chunk and its column factors (warps 0-3)
     auto decays = [&](float av, int par) {
         if (tid < 128) {
@@ -401,6 +448,11 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         }
     };
 
+    // the rows dk 96..127 of the K~ lo operand (the padding of M to 128; they
+    // feed only accumulator lanes that are never read): zeros
+    for (int i = tid; i < 512; i += blockDim.x)
+        reinterpret_cast<uint4*>(sm + L::KL_PAD)[i] = make_uint4(0u, 0u, 0u, 0u);
+
     // prologue: decays and state copy of the first chunk
     float a_nx = (tid < 128 && nchunks > 1) ? load_a(c_begin + 1) : 0.f;
     if (nchunks > 0) decays(tid < 128 ? load_a(c_begin) : 0.f, 0);
@@ -408,14 +460,17 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         const float* src = p.s_init ? p.s_init + unit * p.init_unit_stride + seg * p.init_seg_stride +
                                           row * kDv + half * 96
                                     : nullptr;
+        if (VARLEN && seg > 0)    // a later segment of a sequence: the state the combine left for it
+            src = p.seg_states + (varlen_slot(p.cu_seqlens, b, seg, p.chunks_per_seg) * p.H + h) * (kDk * kDv) +
+                  row * kDv + half * 96;
         state_to_tmem(src, tq + L::TM_S + half * 96);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (nchunks > 0 && srow)
-        state_copy_and_decay<true>(tq + L::TM_S + half * 96, row, half, exp2f(b2s[127]), sm + L::X, sm + L::XL,
-                                   true);
+        state_copy_and_decay<false>(tq + L::TM_S + half * 96, row, half, exp2f(b2s[127]), sm + L::X, nullptr,
+                                    true, save_row(c_begin), kStatePlane);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -529,8 +584,9 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         const float g2 = b2c[127];
         const bool fast = -g2 <= kFactorRange;   // uniform: the factorised path is safe
 
-        // (C) K~ = e^{gamma - b} K in place; on the exact path also
-        // Q~ = scale e^{b} Q (rows in permuted token order)
+        // (C) K~ = e^{gamma - b} K as a bf16 pair: hi in place, lo (K~ - hi) in
+        // KL, so that the state update keeps the fp32 state's precision; on
+        // the exact path also Q~ = scale e^{b} Q (rows in permuted token order)
         if (worker && !failed && !mbar_wait(bar_sc, it & 1, ctl)) failed = true;
         if (!failed && worker) {
             const int live = Tn - c * 128;   // varlen: rows past the sequence (the next one's) add nothing
@@ -539,7 +595,10 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             for (int idx = tid; idx < 1536; idx += kWorkers) {
                 const int r = (idx >> 2) & 127, blk = idx >> 9, ch = idx & 3;
                 uint4* u = reinterpret_cast<uint4*>(sm + L::U + blk * 8192 + r * 64) + ch;
-                *u = scale8(*u, (!VARLEN || r < live) ? exp2f(g2 - b2c[r]) : 0.f);
+                uint4 hi, lo;
+                scale8_split(*u, (!VARLEN || r < live) ? exp2f(g2 - b2c[r]) : 0.f, hi, lo);
+                *u = hi;
+                *(reinterpret_cast<uint4*>(sm + L::KL + blk * 8192 + r * 64) + ch) = lo;
                 if (!fast) {
                     uint4* qq = reinterpret_cast<uint4*>(sm + L::Q + blk * 8192 + r * 64) + ch;
                     *qq = scale8(*qq, p.scale * exp2f(b2c[row_token(r)]));
@@ -551,24 +610,25 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         if (bar_or(2, 288, failed)) { aborted = true; break; }
         tc_fence_after();
 
-        // (D) O = Q S_prev (hi, lo), S += K~^T V
+        // (D) O = Q S_prev, S += K~^T V (K~ as hi + lo)
         if (issuer) {
             if (mbar_wait(bar_y + ys, ph_y[ys], ctl)) {
                 ph_y[ys] ^= 1;
                 const uint64_t dq = smem_desc(sb + L::Q, 16, 512, kLayoutSW64);
                 const uint64_t dx = smem_desc(sb + L::X, 12288, 1024, kLayoutSW128);
-                const uint64_t dxl = smem_desc(sb + L::XL, 12288, 1024, kLayoutSW128);
                 const uint64_t dua = smem_desc(sb + L::U, 8192, 512, kLayoutSW64);
+                const uint64_t dul = smem_desc(sb + L::KL, 8192, 512, kLayoutSW64);
                 const uint64_t dy = smem_desc(sb + ya, 16384, 1024, kLayoutSW128);
+#pragma unroll
+                for (int ks = 0; ks < 6; ++ks)
+                    umma_bf16(tmem + L::TM_O, desc_add(dq, (ks >> 1) * 8192 + (ks & 1) * 32),
+                              desc_add(dx, ks * 2048), kIdOut, ks > 0);
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
 #pragma unroll
-                    for (int ks = 0; ks < 6; ++ks)
-                        umma_bf16(tmem + L::TM_O, desc_add(dq, (ks >> 1) * 8192 + (ks & 1) * 32),
-                                  desc_add(part ? dxl : dx, ks * 2048), kIdOut, (part | ks) > 0);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    umma_bf16(tmem + L::TM_S, desc_add(dua, ks * 1024), desc_add(dy, ks * 2048), kIdState, 1);
+                    for (int ks = 0; ks < 8; ++ks)
+                        umma_bf16(tmem + L::TM_S, desc_add(part ? dul : dua, ks * 1024), desc_add(dy, ks * 2048),
+                                  kIdState, 1);
                 umma_commit(bar_d);
                 ++n_d;
             } else {
@@ -641,8 +701,8 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             if (!failed && !mbar_wait(bar_d, it & 1, ctl)) failed = true;
             tc_fence_after();
             if (srow && !failed)
-                state_copy_and_decay<true>(tq + L::TM_S + half * 96, row, half, exp2f(b2s[(par ^ 1) * 128 + 127]),
-                                           sm + L::X, sm + L::XL, true);
+                state_copy_and_decay<false>(tq + L::TM_S + half * 96, row, half, exp2f(b2s[(par ^ 1) * 128 + 127]),
+                                            sm + L::X, nullptr, true, save_row(c + 1), kStatePlane);
             fence_async_smem();
         }
 
@@ -686,7 +746,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
 
     if (!aborted && warp < 9) {
         // all MMAs are done (the epilogue waited for the last P V): S is final
-        const bool write_state = p.s_out && (!p.out_last_only || seg == static_cast<int>(gridDim.x) - 1);
+        const bool write_state = p.s_out && (!p.out_last_only || seg == last_seg);
         if (write_state && srow && !failed && GLA_DCHECK(unit < p.B * p.H, p.ctl.status))
             tmem_to_state(tq + L::TM_S + half * 96,
                           p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + half * 96);
@@ -730,8 +790,24 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int unit = b * p.H + h;
+    // varlen (segmented pre-pass of the packed forward): blockIdx.z is a
+    // sequence, its tokens tb .. tb+Tn-1 of batch row 0; the segments are
+    // the sequence's own, and the pre-pass sweeps all but its last
+    int tb = 0, Tn = p.T, NCn = p.NC;
+    if (p.cu_seqlens) {
+        tb = p.cu_seqlens[b];
+        Tn = p.cu_seqlens[b + 1] - tb;
+        if (tb < 0 || Tn < 0 || tb + Tn > p.T) {   // offsets out of range: touch nothing
+            if (threadIdx.x == 0) record_status(p.ctl.status, GLA_ERR_INVALID_ARG);
+            return;
+        }
+        NCn = (Tn + 127) / 128;
+        const int nseg_n = max(1, (NCn + p.chunks_per_seg - 1) / p.chunks_per_seg);
+        if (seg >= nseg_n - (p.pre_pass ? 1 : 0)) return;
+    }
+    const int bc = p.cu_seqlens ? 0 : b;         // batch coordinate of the token tensors
     const int c_begin = seg * p.chunks_per_seg;
-    const int c_end = min(p.NC, c_begin + p.chunks_per_seg);
+    const int c_end = min(NCn, c_begin + p.chunks_per_seg);
     const int nchunks = c_end - c_begin;
     const WaitCtl ctl = p.ctl;
     const int quad = warp & 3, row = quad * 32 + lane, qt = warp >> 2;
@@ -776,12 +852,12 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
         for (int it = 0; it < nchunks; ++it) {
             const int st = it % 3;
             if (it >= 3 && !mbar_wait(bar_free + st, ((it - 3) / 3) & 1, ctl)) break;
-            const int t0 = chunk_at(it) * 128;
+            const int t0 = tb + chunk_at(it) * 128;
             uint8_t* base = sm + st * L::STAGE;
             mbar_arrive_expect_tx(bar_ld + st, kTileQK + kTileV);
             for (int i = 0; i < 3; ++i) {
-                tma_load_4d(base + i * 8192, &p.tm_u, bar_ld + st, i * 32, h, t0, b);
-                tma_load_4d(base + L::Y + i * 16384, &p.tm_y, bar_ld + st, i * 64, h, t0, b);
+                tma_load_4d(base + i * 8192, &p.tm_u, bar_ld + st, i * 32, h, t0, bc);
+                tma_load_4d(base + L::Y + i * 16384, &p.tm_y, bar_ld + st, i * 64, h, t0, bc);
             }
             ++n_ld[st];
         }
@@ -798,7 +874,7 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int t = c * 128 + lane * 4 + e;
-                x[e] = (it < nchunks && t < p.T) ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f;
+                x[e] = (it < nchunks && t < Tn) ? p.a[(static_cast<int64_t>(bc) * p.T + tb + t) * p.H + h] : 0.f;
             }
         };
         float xa[4];
@@ -821,6 +897,13 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
             float f[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) f[e] = REVERSE ? p.scale * exp2f(pre + c4[e]) : exp2f(g2 - (pre + c4[e]));
+            if (p.cu_seqlens) {
+                // rows past the sequence (the next sequence's tokens) add nothing
+                const int t = chunk_at(it) * 128 + lane * 4;
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (t + e >= Tn) f[e] = 0.f;
+            }
             const int slot = it & 3;
             if (it >= 4 && !mbar_wait(bar_fdone + slot, ((it - 4) >> 2) & 1, ctl)) break;
             *reinterpret_cast<float4*>(fring + slot * 128 + lane * 4) = make_float4(f[0], f[1], f[2], f[3]);
@@ -989,12 +1072,19 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
             const int sweep_end = REVERSE ? 0 : static_cast<int>(gridDim.x) - 1;
             const bool write_state = p.s_out && (!p.out_last_only || seg == sweep_end);
             if (write_state && GLA_DCHECK(unit < p.B * p.H && row < kDk, p.ctl.status)) {
-                float* dst = p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + qt * 48;
+                float* dst = p.cu_seqlens
+                                 ? p.seg_states +
+                                       (varlen_slot(p.cu_seqlens, b, seg, p.chunks_per_seg) * p.H + h) * (kDk * kDv) +
+                                       row * kDv + qt * 48
+                                 : p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + qt * 48;
 #pragma unroll
                 for (int e = 0; e < 48; e += 4)
                     *reinterpret_cast<float4*>(dst + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
             }
-            if (p.g2_out && tid == 0) p.g2_out[static_cast<int64_t>(unit) * p.g2_unit_stride + seg] = gsum2;
+            if (p.cu_seqlens && tid == 0)
+                p.seg_g2[varlen_slot(p.cu_seqlens, b, seg, p.chunks_per_seg) * p.H + h] = gsum2;
+            else if (p.g2_out && tid == 0)
+                p.g2_out[static_cast<int64_t>(unit) * p.g2_unit_stride + seg] = gsum2;
         }
     }
     tc_fence_before();

@@ -50,13 +50,15 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
         : "memory");
 }
 
-// SiLU(x) = x * sigmoid(x), with sigmoid(x) = (1 + tanh(x / 2)) / 2 and the
-// hardware tanh approximation: one special-function op per element.
-__device__ __forceinline__ float silu(float x)
+// SiLU(u) = u sigmoid(u) = h + h tanh(h) with h = u / 2 (sigmoid(u) =
+// (1 + tanh(u / 2)) / 2), on the hardware tanh approximation.  The kernel
+// folds the 1/2 into the conv weights and bias, so it convolves straight to
+// h: one special-function op and one FMA per element.
+__device__ __forceinline__ float silu_of_half(float h)
 {
     float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
-    return x * fmaf(0.5f, t, 0.5f);
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
 }
 
 // CH channels (one 2*CH-byte vector) per thread.
@@ -191,11 +193,11 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
     for (int c = 0; c < CH; ++c) {
         const int ch = active ? c0 + c : 0;
 #pragma unroll
-        for (int j = 0; j < kW; ++j) wr[c][j] = active ? w[ch * kW + j] : 0.f;
+        for (int j = 0; j < kW; ++j) wr[c][j] = active ? 0.5f * w[ch * kW + j] : 0.f;   // halved: see silu_of_half
         if constexpr (AFF) {
             ga[c] = (gamma && active) ? gamma[ch] : 1.f;
             be[c] = (beta && active) ? beta[ch] : 0.f;
-            bi[c] = (bias && active) ? bias[ch] : 0.f;
+            bi[c] = (bias && active) ? 0.5f * bias[ch] : 0.f;
         }
     }
 
@@ -232,12 +234,9 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
             break;
         }
 
-        // fully unrolled (the window rotation becomes register renaming) where
-        // the registers allow it
-#pragma unroll(MAXT <= 416 ? kG : 2)
-        for (int g = 0; g < kG; ++g) {
-            if (g >= rows) break;
-            const int p = pos0 + g;
+        // one row: normalise, convolve with the window, SiLU, write y (when the
+        // row is an output of this CTA), shift the window
+        auto do_row = [&](int g, int p, bool out) {
             float xn[CH];
             if (active) {
                 unpack<CH>(*reinterpret_cast<const V*>(st + g * row_bytes + c0 * 2), xn);
@@ -256,9 +255,9 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
 #pragma unroll
                 for (int c = 0; c < CH; ++c) xn[c] = 0.f;
             }
-            if (p >= t_begin && active && GLA_DCHECK(p < T && c0 + CH <= D, ctl.status)) {
-                V out;
-                uint32_t* ow = reinterpret_cast<uint32_t*>(&out);
+            if (out && GLA_DCHECK(p < T && c0 + CH <= D, ctl.status)) {
+                V o;
+                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
                 for (int c = 0; c < CH; c += 2) {
                     float r[2];
@@ -267,11 +266,11 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
                         float acc = AFF ? bi[AFF ? c + e : 0] : 0.f;
 #pragma unroll
                         for (int j = 0; j < kW - 1; ++j) acc = fmaf(wr[c + e][j], win[j][c + e], acc);
-                        r[e] = silu(fmaf(wr[c + e][kW - 1], xn[c + e], acc));
+                        r[e] = silu_of_half(fmaf(wr[c + e][kW - 1], xn[c + e], acc));
                     }
                     ow[c / 2] = pack_bf16(r[0], r[1]);
                 }
-                __stcs(reinterpret_cast<V*>(yb + static_cast<int64_t>(p) * D + c0), out);
+                __stcs(reinterpret_cast<V*>(yb + static_cast<int64_t>(p) * D + c0), o);
             }
 #pragma unroll
             for (int c = 0; c < CH; ++c) {
@@ -279,6 +278,16 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
                 win[1][c] = win[2][c];
                 win[2][c] = xn[c];
             }
+        };
+        if (rows == kG && pos0 >= t_begin && active) {
+            // an interior stage: eight output rows and no branch between them,
+            // so the rows' dependency chains interleave (and, unrolled, the
+            // window rotation becomes register renaming)
+#pragma unroll(MAXT <= 416 ? kG : 2)
+            for (int g = 0; g < kG; ++g) do_row(g, pos0 + g, true);
+        } else {
+#pragma unroll 1
+            for (int g = 0; g < rows; ++g) do_row(g, pos0 + g, pos0 + g >= t_begin && active);
         }
         mbar_arrive(freeb + slot);             // this worker is done with the slot
     }

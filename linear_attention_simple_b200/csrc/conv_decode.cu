@@ -17,8 +17,11 @@
 // HBM-bound: per sequence x and y (2 B per channel each) and the history
 // read and written (12 B each); the weights stay in L2 across sequences.
 // One CTA per sequence, thread i owns channels 8i .. 8i+7: one 16-byte
-// vector of x and y, two of each history row.  The LayerNorm moments are two
-// block reductions (mean, then the centred second moment) over registers.
+// vector of x and y, two of each history row.  The history rows are loaded
+// with x, before the LayerNorm, so their latency overlaps the moments (the
+// weights and bias, L2-resident, come after); the two moments (sums of
+// (x - x0) and (x - x0)^2, shifted by the row's first element x0 as the
+// sequence front end does) come from one block reduction.
 // A slot outside [0, n_slots) is skipped (nothing read or written) and
 // GLA_ERR_INVALID_ARG is recorded in the device status word.
 #include <cuda_bf16.h>
@@ -38,16 +41,19 @@ __device__ __forceinline__ float warp_sum_dec(float v)
     return v;
 }
 
-// Sum over the block; every thread gets the result.
-__device__ __forceinline__ float block_sum(float v, float* red)
+// Sums of a and b over the block; every thread gets both.
+__device__ __forceinline__ float2 block_sum2(float a, float b, float2* red)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = (blockDim.x + 31) >> 5;
-    v = warp_sum_dec(v);
-    __syncthreads();                     // red is free (an earlier sum may still read it)
-    if (lane == 0) red[warp] = v;
+    a = warp_sum_dec(a);
+    b = warp_sum_dec(b);
+    if (lane == 0) red[warp] = make_float2(a, b);
     __syncthreads();
-    float s = 0.f;
-    for (int i = 0; i < nw; ++i) s += red[i];
+    float2 s = make_float2(0.f, 0.f);
+    for (int i = 0; i < nw; ++i) {
+        s.x += red[i].x;
+        s.y += red[i].y;
+    }
     return s;
 }
 
@@ -67,27 +73,32 @@ __device__ __forceinline__ void load8(const float* p, float (&v)[8])
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-__device__ __forceinline__ void store8(float* p, const float (&v)[8])
-{
-    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
-    *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
-}
-
-__global__ void __launch_bounds__(kMaxThreads) conv_decode_kernel(
+// At most 80 registers, so that two CTAs of 384 threads (D = 3,072) share
+// an SM.
+__global__ void __maxnreg__(80) conv_decode_kernel(
     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ slot_idx, int apply_ln,
     const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
     const float* __restrict__ w, const float* __restrict__ bias, float* __restrict__ hist,
     __nv_bfloat16* __restrict__ y, int D, int n_slots, int* __restrict__ status)
 {
-    __shared__ float red[kMaxThreads / 32];
+    __shared__ float2 red[kMaxThreads / 32];
     const int n = blockIdx.x, c0 = threadIdx.x * 8;
     const int s = slot_idx ? slot_idx[n] : n;
     if (s < 0 || s >= n_slots) {                // a slot outside the pool: touch nothing
         if (threadIdx.x == 0) record_status(status, GLA_ERR_INVALID_ARG);
         return;
     }
-
+    // the loads from HBM first: x and the three history rows
     const uint4 xv = __ldcs(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(n) * D + c0));
+    float* hs = hist + static_cast<int64_t>(s) * 3 * D + c0;
+    float4 hv[3][2];
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+        hv[r][0] = __ldcs(reinterpret_cast<const float4*>(hs + r * D));
+        hv[r][1] = __ldcs(reinterpret_cast<const float4*>(hs + r * D + 4));
+    }
+    const float x0 = __bfloat162float(x[static_cast<int64_t>(n) * D]);
+
     const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
     float v[8];
 #pragma unroll
@@ -96,14 +107,17 @@ __global__ void __launch_bounds__(kMaxThreads) conv_decode_kernel(
         v[2 * i + 1] = bf16_hi(xw[i]);
     }
     if (apply_ln) {
-        float sum = 0.f;
+        float s1 = 0.f, s2 = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) sum += v[e];
-        const float mean = block_sum(sum, red) / D;
-        float sq = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sq = fmaf(v[e] - mean, v[e] - mean, sq);
-        const float rstd = rsqrtf(block_sum(sq, red) / D + eps);
+        for (int e = 0; e < 8; ++e) {
+            const float d = v[e] - x0;
+            s1 += d;
+            s2 = fmaf(d, d, s2);
+        }
+        const float2 m = block_sum2(s1, s2, red);
+        const float m1 = m.x / D;
+        const float var = fmaxf(m.y / D - m1 * m1, 0.f);
+        const float mean = x0 + m1, rstd = rsqrtf(var + eps);
         float g[8], bt[8];
         if (gamma) load8(gamma + c0, g);
         if (beta) load8(beta + c0, bt);
@@ -116,11 +130,11 @@ __global__ void __launch_bounds__(kMaxThreads) conv_decode_kernel(
         }
     }
 
-    float* hs = hist + static_cast<int64_t>(s) * 3 * D + c0;
-    float h0[8], h1[8], h2[8], bi[8];
-    load8(hs, h0);
-    load8(hs + D, h1);
-    load8(hs + 2 * D, h2);
+    const float h0[8] = {hv[0][0].x, hv[0][0].y, hv[0][0].z, hv[0][0].w, hv[0][1].x, hv[0][1].y, hv[0][1].z, hv[0][1].w};
+    const float h1[8] = {hv[1][0].x, hv[1][0].y, hv[1][0].z, hv[1][0].w, hv[1][1].x, hv[1][1].y, hv[1][1].z, hv[1][1].w};
+    const float h2[8] = {hv[2][0].x, hv[2][0].y, hv[2][0].z, hv[2][0].w, hv[2][1].x, hv[2][1].y, hv[2][1].z, hv[2][1].w};
+    // the weights and the bias are L2-resident across sequences
+    float bi[8];
     if (bias) load8(bias + c0, bi);
     uint32_t out[4];
 #pragma unroll
@@ -139,9 +153,12 @@ __global__ void __launch_bounds__(kMaxThreads) conv_decode_kernel(
         out[e / 2] = pack_bf16(r[0], r[1]);
     }
     __stcs(reinterpret_cast<uint4*>(y + static_cast<int64_t>(n) * D + c0), make_uint4(out[0], out[1], out[2], out[3]));
-    store8(hs, h1);
-    store8(hs + D, h2);
-    store8(hs + 2 * D, v);
+    __stcs(reinterpret_cast<float4*>(hs), hv[1][0]);
+    __stcs(reinterpret_cast<float4*>(hs + 4), hv[1][1]);
+    __stcs(reinterpret_cast<float4*>(hs + D), hv[2][0]);
+    __stcs(reinterpret_cast<float4*>(hs + D + 4), hv[2][1]);
+    __stcs(reinterpret_cast<float4*>(hs + 2 * D), make_float4(v[0], v[1], v[2], v[3]));
+    __stcs(reinterpret_cast<float4*>(hs + 2 * D + 4), make_float4(v[4], v[5], v[6], v[7]));
 }
 
 }  // namespace

@@ -280,7 +280,15 @@ unsigned long long gla_launch_count(void) { return g_launches.load(); }
 size_t gla_chunk_workspace_bytes(int B, int T, int H, int dk, int dv, int for_bwd)
 {
     if (B <= 0 || T <= 0 || H <= 0 || dk != kDk || dv != kDv) return 0;
+    if (for_bwd == 2) return bwd_workspace_bytes(B, T, H, true);
     return for_bwd ? bwd_workspace_bytes(B, T, H) : fwd_workspace_bytes(B, T, H);
+}
+
+size_t gla_chunk_saved_state_bytes(int B, int T, int H, int dk, int dv)
+{
+    if (B <= 0 || T <= 0 || H <= 0 || dk != kDk || dv != kDv) return 0;
+    const size_t NC = (static_cast<size_t>(T) + kChunk - 1) / kChunk;
+    return static_cast<size_t>(B) * H * NC * 2 * kDk * kDv * 2;
 }
 
 gla_status gla_chunk_fwd(const void* q, const void* k, const void* v, const float* a,
@@ -319,17 +327,49 @@ gla_status gla_chunk_fwd(const void* q, const void* k, const void* v, const floa
     return run_chunk_fwd(p, s0, o, s_final, ws, ws_bytes, ctl, stream);
 }
 
+size_t gla_chunk_varlen_workspace_bytes(int N, int total_T, int H, int dk, int dv)
+{
+    if (N <= 0 || total_T <= 0 || H <= 0 || dk != kDk || dv != kDv) return 0;
+    return varlen_workspace_bytes(N, total_T, H);
+}
+
+gla_status gla_chunk_fwd_train(const void* q, const void* k, const void* v, const float* a,
+                               const float* s0, void* o, float* s_final, void* saved, size_t saved_bytes,
+                               void* ws, size_t ws_bytes, int B, int T, int H, int dk, int dv, int64_t ld_qkv,
+                               float scale, gla_dtype dt, cudaStream_t stream)
+{
+    int64_t ld_qk = 0, ld_v = 0;
+    gla_status s = validate_chunk(q, k, v, a, B, T, H, dk, dv, ld_qkv, scale, dt, &ld_qk, &ld_v);
+    if (s != GLA_OK) return s;
+    if (dt != GLA_BF16) return GLA_ERR_UNSUPPORTED;
+    if (!aligned16(s0) || !aligned16(s_final) || !aligned16(ws) || !aligned16(saved)) return GLA_ERR_MISALIGNED;
+    if (static_cast<int64_t>(B) * T * H == 0) return gla_chunk_fwd(q, k, v, a, s0, o, s_final, ws, ws_bytes, B, T,
+                                                                     H, dk, dv, ld_qkv, scale, dt, stream);
+    if (!o || !saved || saved_bytes < gla_chunk_saved_state_bytes(B, T, H, dk, dv)) return GLA_ERR_INVALID_ARG;
+    if (!aligned16(o)) return GLA_ERR_MISALIGNED;
+    const size_t need = fwd_workspace_bytes(B, T, H);
+    if (need > 0 && (!ws || ws_bytes < need)) return GLA_ERR_INVALID_ARG;
+    gla_status se;
+    WaitCtl ctl = wait_ctl_for_current_device(&se);
+    if (se != GLA_OK) return se;
+    if ((s = scan_chunk_inputs(q, k, v, a, nullptr, s0, nullptr, B, T, H, ld_qk, ld_v, ctl.status, stream)) !=
+        GLA_OK)
+        return s;
+    ChunkProblem p{q, k, v, a, B, T, H, ld_qk, ld_v, scale};
+    return run_chunk_fwd(p, s0, o, s_final, ws, ws_bytes, ctl, stream, saved);
+}
+
 gla_status gla_chunk_fwd_varlen(const void* q, const void* k, const void* v, const float* a,
                                 const int32_t* cu_seqlens, int N, const float* s0, void* o, float* s_final,
-                                int total_T, int H, int dk, int dv, int64_t ld_qkv, float scale, gla_dtype dt,
-                                cudaStream_t stream)
+                                void* ws, size_t ws_bytes, int total_T, int H, int dk, int dv, int64_t ld_qkv,
+                                float scale, gla_dtype dt, cudaStream_t stream)
 {
     if (N < 0 || N > 65535) return N < 0 ? GLA_ERR_INVALID_ARG : GLA_ERR_UNSUPPORTED;
     int64_t ld_qk = 0, ld_v = 0;
     gla_status s = validate_chunk(q, k, v, a, 1, total_T, H, dk, dv, ld_qkv, scale, dt, &ld_qk, &ld_v);
     if (s != GLA_OK) return s;
     if (dt != GLA_BF16) return GLA_ERR_UNSUPPORTED;
-    if (!aligned16(s0) || !aligned16(s_final)) return GLA_ERR_MISALIGNED;
+    if (!aligned16(s0) || !aligned16(s_final) || !aligned16(ws)) return GLA_ERR_MISALIGNED;
     if (N == 0 || H == 0) return GLA_OK;
     if (!cu_seqlens) return GLA_ERR_INVALID_ARG;
     if (total_T > 0 && !o) return GLA_ERR_INVALID_ARG;
@@ -341,7 +381,7 @@ gla_status gla_chunk_fwd_varlen(const void* q, const void* k, const void* v, con
                                stream)) != GLA_OK)
         return s;
     ChunkProblem p{q, k, v, a, 1, total_T, H, ld_qk, ld_v, scale};
-    return run_chunk_fwd_varlen(p, cu_seqlens, N, s0, o, s_final, ctl, stream);
+    return run_chunk_fwd_varlen(p, cu_seqlens, N, s0, o, s_final, ws, ws_bytes, ctl, stream);
 }
 
 gla_status gla_chunk_bwd(const void* q, const void* k, const void* v, const float* a,
@@ -382,6 +422,40 @@ gla_status gla_chunk_bwd(const void* q, const void* k, const void* v, const floa
     ChunkProblem p{q, k, v, a, B, T, H, ld_qk, ld_v, scale};
     return run_chunk_bwd(p, s0, dO, ds_final, grad_q, grad_k, grad_v, grad_a, grad_s0, ws,
                          ws_bytes, ctl, stream);
+}
+
+gla_status gla_chunk_bwd_saved(const void* q, const void* k, const void* v, const float* a, const void* saved,
+                               size_t saved_bytes, const float* s_final, const void* dO, const float* ds_final,
+                               void* grad_q, void* grad_k, void* grad_v, float* grad_a, float* grad_s0, void* ws,
+                               size_t ws_bytes, int B, int T, int H, int dk, int dv, int64_t ld_qkv, float scale,
+                               gla_dtype dt, cudaStream_t stream)
+{
+    int64_t ld_qk = 0, ld_v = 0;
+    gla_status s = validate_chunk(q, k, v, a, B, T, H, dk, dv, ld_qkv, scale, dt, &ld_qk, &ld_v);
+    if (s != GLA_OK) return s;
+    if (dt != GLA_BF16) return GLA_ERR_UNSUPPORTED;
+    if (!aligned16(saved) || !aligned16(s_final) || !aligned16(ds_final) || !aligned16(grad_s0) || !aligned16(ws))
+        return GLA_ERR_MISALIGNED;
+    if (static_cast<int64_t>(B) * H == 0) return GLA_OK;
+    if (T == 0)   // no chunks, nothing saved: the plain backward's empty case
+        return gla_chunk_bwd(q, k, v, a, nullptr, dO, ds_final, grad_q, grad_k, grad_v, grad_a, grad_s0, ws,
+                             ws_bytes, B, T, H, dk, dv, ld_qkv, scale, dt, stream);
+    if (!saved || saved_bytes < gla_chunk_saved_state_bytes(B, T, H, dk, dv)) return GLA_ERR_INVALID_ARG;
+    if (ds_final && !s_final) return GLA_ERR_INVALID_ARG;   // <dS_T, S_T> needs the final state
+    if (!dO || !grad_q || !grad_k || !grad_v || !grad_a) return GLA_ERR_INVALID_ARG;
+    if (!aligned16(dO) || !aligned16(grad_q) || !aligned16(grad_k) || !aligned16(grad_v) || !aligned16(grad_a))
+        return GLA_ERR_MISALIGNED;
+    const size_t need = bwd_workspace_bytes(B, T, H, true);
+    if (need > 0 && (!ws || ws_bytes < need)) return GLA_ERR_INVALID_ARG;
+    gla_status se;
+    WaitCtl ctl = wait_ctl_for_current_device(&se);
+    if (se != GLA_OK) return se;
+    if ((s = scan_chunk_inputs(q, k, v, a, dO, s_final, ds_final, B, T, H, ld_qk, ld_v, ctl.status, stream)) !=
+        GLA_OK)
+        return s;
+    ChunkProblem p{q, k, v, a, B, T, H, ld_qk, ld_v, scale};
+    return run_chunk_bwd(p, nullptr, dO, ds_final, grad_q, grad_k, grad_v, grad_a, grad_s0, ws, ws_bytes, ctl,
+                         stream, saved, s_final);
 }
 
 size_t gla_segment_workspace_bytes(int B, int T, int H, int dk, int dv)

@@ -77,17 +77,23 @@ struct ChunkProblem {
 };
 
 size_t fwd_workspace_bytes(int B, int T, int H);
-size_t bwd_workspace_bytes(int B, int T, int H);
+size_t bwd_workspace_bytes(int B, int T, int H, bool from_saved = false);
 
+size_t varlen_workspace_bytes(int N, int total_T, int H);
 gla_status run_chunk_fwd_varlen(const ChunkProblem& pr, const int* cu_seqlens, int N, const float* s0, void* o,
-                                float* s_final, const WaitCtl& ctl, cudaStream_t st);
+                                float* s_final, void* ws, size_t ws_bytes, const WaitCtl& ctl, cudaStream_t st);
+// h_save (optional): the state entering each chunk as bf16 hi + lo planes,
+// [B*H*NC][2][96][192], for gla_chunk_bwd from saved states.
 gla_status run_chunk_fwd(const ChunkProblem& p, const float* s0, void* o, float* s_final,
-                         void* ws, size_t ws_bytes, const WaitCtl& ctl, cudaStream_t st);
+                         void* ws, size_t ws_bytes, const WaitCtl& ctl, cudaStream_t st,
+                         void* h_save = nullptr);
 
+// saved / s_final (optional): the forward's saved states and final state;
+// with them the forward state pass is skipped.
 gla_status run_chunk_bwd(const ChunkProblem& p, const float* s0, const void* dO,
                          const float* ds_final, void* dq, void* dk, void* dv, float* da,
                          float* ds0, void* ws, size_t ws_bytes, const WaitCtl& ctl,
-                         cudaStream_t st);
+                         cudaStream_t st, const void* saved = nullptr, const float* s_final = nullptr);
 
 gla_status launch_wait_selftest(const WaitCtl& ctl, cudaStream_t st);
 

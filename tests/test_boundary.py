@@ -109,6 +109,34 @@ def test_chunk_bwd_validation(L):
     assert bwd(B=0) == OK
 
 
+def test_training_pair_validation(L):
+    saved = gla.gla_chunk_saved_state_bytes(1, 300, 2)
+    assert saved == 2 * 3 * 2 * 96 * 192 * 2
+    assert gla.gla_chunk_saved_state_bytes(1, 300, 2, dk=64) == 0
+    assert 0 < gla.gla_chunk_workspace_bytes(8, 2048, 16, for_bwd=True, from_saved=True) < \
+        gla.gla_chunk_workspace_bytes(8, 2048, 16, for_bwd=True)
+
+    def fwd(q=0x1000, o=0x5000, sv=0x9000, svb=saved, dt=0, T=300):
+        return L.gla_chunk_fwd_train(P(q), P(0x2000), P(0x3000), P(0x4000), None, P(o), None, P(sv), svb, None, 0,
+                                     1, T, 2, 96, 192, 0, 96 ** -0.5, dt, None)
+    assert fwd(sv=None) == INVALID
+    assert fwd(svb=saved - 16) == INVALID
+    assert fwd(sv=0x9008) == MISALIGNED
+    assert fwd(dt=1) == UNSUPPORTED
+    assert fwd(q=None) == INVALID
+
+    def bwd(sv=0x9000, svb=saved, sf=None, dsT=None, dO=0x6000, ws=0xA000, wsb=1 << 30):
+        return L.gla_chunk_bwd_saved(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(sv), svb, P(sf), P(dO), P(dsT),
+                                     P(0x7000), P(0x7100), P(0x7200), P(0x7300), None, P(ws), wsb, 1, 300, 2, 96, 192,
+                                     0, 96 ** -0.5, 0, None)
+    assert bwd(sv=None) == INVALID
+    assert bwd(svb=saved - 1) == INVALID
+    assert bwd(dsT=0xB000) == INVALID               # dS_T given without the final state
+    assert bwd(dO=None) == INVALID
+    assert bwd(ws=None, wsb=0) == INVALID
+    assert bwd(sf=0xB004, dsT=0xB000) == MISALIGNED
+
+
 def test_decode_validation(L):
     def dec(state=0x1000, slot=None, ns=4, q=0x2000, k=0x3000, v=0x4000, a=0x5000, o=0x6000, N=4,
             H=16, dk=96, dv=192, scale=96 ** -0.5):
@@ -148,9 +176,9 @@ def test_conv_validation(L):
 
 def test_varlen_validation(L):
     def varlen(q=0x1000, k=0x2000, v=0x3000, a=0x4000, cu=0x5000, N=2, s0=None, o=0x6000, sf=None,
-               total=256, H=2, dk=96, dv=192, ld=0, scale=96 ** -0.5, dt=0):
-        return L.gla_chunk_fwd_varlen(P(q), P(k), P(v), P(a), P(cu), N, P(s0), P(o), P(sf), total, H, dk, dv,
-                                      ld, scale, dt, None)
+               ws=None, wsb=0, total=256, H=2, dk=96, dv=192, ld=0, scale=96 ** -0.5, dt=0):
+        return L.gla_chunk_fwd_varlen(P(q), P(k), P(v), P(a), P(cu), N, P(s0), P(o), P(sf), P(ws), wsb, total,
+                                      H, dk, dv, ld, scale, dt, None)
     assert varlen(N=-1) == INVALID
     assert varlen(N=70000) == UNSUPPORTED
     assert varlen(dt=1) == UNSUPPORTED           # bf16 only
@@ -159,7 +187,13 @@ def test_varlen_validation(L):
     assert varlen(q=None) == INVALID
     assert varlen(dk=64) == UNSUPPORTED
     assert varlen(s0=0x7008) == MISALIGNED
+    assert varlen(ws=0x7004, wsb=4096) == MISALIGNED
     assert varlen(N=0) == OK
+    # the segment scratch: none for a short total, grows with the tokens
+    assert gla.gla_chunk_varlen_workspace_bytes(8, 256, 16) == 0
+    small = gla.gla_chunk_varlen_workspace_bytes(8, 16384, 16)
+    assert small > 0 and gla.gla_chunk_varlen_workspace_bytes(8, 65536, 16) >= small
+    assert gla.gla_chunk_varlen_workspace_bytes(8, 16384, 16, dk=64) == 0
 
 
 def test_conv_decode_and_backward_validation(L):

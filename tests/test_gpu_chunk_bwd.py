@@ -122,6 +122,16 @@ def test_chunk_bwd_training_full_size_sampled():
     check_bwd(d, grads, units=[(0, 0), (4, 7), (7, 15)])
 
 
+def test_chunk_bwd_training_full_tensor():
+    """The training step's backward (B = 8, T = 2048, H = 16, zero gradient on
+    the final state) on every (batch, head) against the oracle: whole dq,
+    dk, dv and da tensors."""
+    d = inputs.chunk_inputs(8, 2048, 16, seed=1013, device="cuda", with_dO=True)
+    grads = gla.gla_chunk_bwd(d["q"], d["k"], d["v"], d["a"], d["dO"])
+    assert gla.gla_get_device_status() == 0
+    check_bwd(d, grads)
+
+
 @pytest.mark.parametrize("mean", [None, -8.0, 0.6])
 def test_chunk_bwd_strong_decay_and_no_decay(mean):
     """Decays outside the workload distribution: a = 0 (no decay), a ~ -8 per
@@ -168,3 +178,47 @@ def test_chunk_bwd_strong_decay_and_no_decay(mean):
         assert err <= 2.0 ** -15 * terms, "da max-abs %.3g (terms %.3g)" % (err, terms)
     else:
         assert e_da <= REL_BF16, "da rel L2 %.3g" % e_da
+
+
+@pytest.mark.parametrize("B,T,H,s0,dsT", [(2, 300, 3, True, True), (1, 4096, 3, True, False), (8, 2048, 16, False, False)])
+def test_training_pair_saved_states_and_backward(B, T, H, s0, dsT):
+    """gla_chunk_fwd_train keeps the state entering every chunk as bf16 hi + lo
+    planes: checked against the oracle's state after each chunk boundary
+    (prefix runs) on sampled heads, to 1e-5 relative L2.  gla_chunk_bwd_saved
+    then gives the gradients of the plain backward (to 1e-3: the states come
+    from the fused forward instead of the state-only pass) and of the oracle
+    (the usual bounds).  The second case is segmented (few heads, long T);
+    the third is the training workload."""
+    d = inputs.chunk_inputs(B, T, H, seed=260 + H, device="cuda", s0_std=0.1 if s0 else None, with_dO=True)
+    ds = inputs.randn((B, H, 96, 192), 261 + H, "cuda", std=0.1) if dsT else None
+    o, sf, saved = gla.gla_chunk_fwd_train(d["q"], d["k"], d["v"], d["a"], s0=d["s0"])
+    o_ref, sf_ref = gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"], s0=d["s0"])
+    assert gla.gla_get_device_status() == 0
+    assert torch.equal(o, o_ref) and torch.equal(sf, sf_ref)      # the same forward, plus the saving
+    NC = (T + 127) // 128
+    planes = saved[:B * H * NC * 2 * 96 * 192 * 2].view(torch.bfloat16).view(B, H, NC, 2, 96, 192).float()
+    states = (planes[:, :, :, 0] + planes[:, :, :, 1]).double()
+    units = [(0, 0), (B - 1, H - 1)]
+    for b, h in units:
+        for c in sorted({0, 1, NC // 2, NC - 1}):
+            t = 128 * c
+            s0n = None if d["s0"] is None else _np(d["s0"][b, h])[None, None]
+            if t == 0:
+                ref = np.zeros((96, 192)) if s0n is None else s0n[0, 0]
+            else:
+                _, rs = recurrent.fwd(_np(d["q"][b:b + 1, :t, h:h + 1]), _np(d["k"][b:b + 1, :t, h:h + 1]),
+                                      _np(d["v"][b:b + 1, :t, h:h + 1]), _np(d["a"][b:b + 1, :t, h:h + 1]), s0n)
+                ref = rs[0, 0]
+            got = states[b, h, c].cpu().numpy()
+            if np.linalg.norm(ref) > 0:
+                e = rel_l2(got, ref)
+                assert e <= 1e-5, "saved state (%d, %d, chunk %d) rel L2 %.3g" % (b, h, c, e)
+            else:
+                assert np.abs(got).max() == 0.0
+    g1 = gla.gla_chunk_bwd_saved(d["q"], d["k"], d["v"], d["a"], saved, d["dO"], s_final=sf, ds_final=ds)
+    g0 = gla.gla_chunk_bwd(d["q"], d["k"], d["v"], d["a"], d["dO"], s0=d["s0"], ds_final=ds)
+    assert gla.gla_get_device_status() == 0
+    for name, x, y in zip(("dq", "dk", "dv", "da", "ds0"), g1, g0):
+        e = rel_l2(_np(x), _np(y))
+        assert e <= 1e-3, "%s: saved-state backward vs plain, rel L2 %.3g" % (name, e)
+    check_bwd(d, g1, units=None if B * T * H <= 4096 else units, dsT=ds)

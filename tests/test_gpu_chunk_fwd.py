@@ -123,6 +123,16 @@ def test_chunk_fwd_prefill_full_size_sampled():
     check_fwd(d, o, sf, units=[(0, 0), (3, 5), (7, 15), (5, 9)])
 
 
+def test_chunk_fwd_prefill_full_tensor():
+    """The prefill workload (B = 8, T = 2048, H = 16) on every (batch, head)
+    against the oracle: the whole o and S_T tensors, so a fault confined to
+    the CTAs of some batch rows or heads cannot hide between samples."""
+    d = inputs.chunk_inputs(8, 2048, 16, seed=1012, device="cuda")
+    o, sf = gla.gla_chunk_fwd(d["q"], d["k"], d["v"], d["a"])
+    assert gla.gla_get_device_status() == 0
+    check_fwd(d, o, sf)
+
+
 def test_chunk_fwd_long_prefill_full_size_sampled():
     """B = 1, T = 65536, H = 16 with S_0 ~ N(0, 0.1^2) (the long-context
     prefill, segmented path), on two sampled heads."""

@@ -96,3 +96,63 @@ def test_varlen_prefill_size_sampled():
                                _np(s0[n, h])[None, None])
         assert_bf16_close(_np(o[lo:hi, h]), ro[0, :, 0], "o (%d, %d)" % (n, h))
         assert rel_l2(_np(sf[n, h]), rs[0, 0]) <= REL_STATE
+
+
+def test_varlen_long_sequence_among_short_ones_is_segmented():
+    """One 16,384-token sequence among short ones, with initial states: the
+    long sequence is cut into segments (pre-pass, fold, output pass) and
+    every sequence still matches the oracle run on it alone; the result also
+    matches the unsegmented sweep (the fold only regroups the sums)."""
+    lengths = [3, 16384, 128, 700, 1, 2000]
+    H = 4
+    q, k, v, a, cu, s0 = _packed(lengths, H, seed=93)
+    total = q.shape[0]
+    assert gla.gla_chunk_varlen_workspace_bytes(len(lengths), total, H) > 0
+    o, sf = gla.gla_chunk_fwd_varlen(q, k, v, a, cu, s0=s0)
+    assert gla.gla_get_device_status() == 0
+    c = cu.cpu().numpy()
+    for n in range(len(lengths)):
+        lo, hi = int(c[n]), int(c[n + 1])
+        ro, rs = recurrent.fwd(_np(q[lo:hi])[None], _np(k[lo:hi])[None], _np(v[lo:hi])[None],
+                               _np(a[lo:hi])[None], _np(s0[n])[None])
+        r = assert_bf16_close(_np(o[lo:hi]), ro[0], "o of sequence %d" % n)
+        es = rel_l2(_np(sf[n]), rs[0])
+        assert es <= REL_STATE, "S_T of sequence %d rel L2 %.3g" % (n, es)
+        print("sequence %d (%d tokens): o rel %.3g raw-max %.3g beyond-rounding %.3g, S_T rel %.3g"
+              % ((n, hi - lo) + r + (es,)))
+    o1, sf1 = gla.gla_chunk_fwd_varlen(q, k, v, a, cu, s0=s0, segmented=False)
+    assert rel_l2(_np(o), _np(o1)) <= 1e-3
+    assert rel_l2(_np(sf), _np(sf1)) <= 1e-3
+
+
+def test_varlen_segmented_time_16k_tokens():
+    """16,384 tokens in 8 sequences of 1 to 5,610 tokens at H = 16: the
+    segmented and the one-sweep-per-sequence forward, timed with CUDA events
+    (printed), and equal to each other."""
+    lengths = [5610, 1, 3000, 2048, 777, 129, 4000, 819]
+    H = 16
+    q, k, v, a, cu, s0 = _packed(lengths, H, seed=94)
+    ws = torch.empty(max(1, gla.gla_chunk_varlen_workspace_bytes(len(lengths), q.shape[0], H)),
+                     dtype=torch.uint8, device="cuda")
+    o = torch.empty((q.shape[0], H, 192), dtype=torch.bfloat16, device="cuda")
+    sf = torch.empty((len(lengths), H, 96, 192), dtype=torch.float32, device="cuda")
+    times = {}
+    outs = {}
+    for seg in (False, True):
+        run = lambda: gla.gla_chunk_fwd_varlen(q, k, v, a, cu, s0=s0, o=o, s_final=sf,  # noqa: E731
+                                               ws=ws if seg else None, segmented=seg)
+        for _ in range(3):
+            run()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(10):
+            run()
+        e1.record()
+        e1.synchronize()
+        times[seg] = e0.elapsed_time(e1) / 10 * 1e3
+        outs[seg] = (o.clone(), sf.clone())
+    assert gla.gla_get_device_status() == 0
+    print("packed forward, 16,384 tokens, H = 16: one sweep per sequence %.1f us, segmented %.1f us"
+          % (times[False], times[True]))
+    assert rel_l2(_np(outs[True][0]), _np(outs[False][0])) <= 1e-3
+    assert rel_l2(_np(outs[True][1]), _np(outs[False][1])) <= 1e-3

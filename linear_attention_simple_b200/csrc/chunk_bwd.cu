@@ -14,14 +14,15 @@
 //   da_t = sum_{m >= t} (q_m . dq_m - k_m . dk_m) + <dS_T, S_T>
 //
 // Passes (all on the caller's stream):
-//   1. state kernel, forward, state-only: h_c (bf16) for every chunk, and
-//      S_T when an upstream dS_T is given;
-//   2. state kernel, reverse: D_c (bf16) for every chunk, dS_0 = D_{-1};
-//   3. bwd_dqdk_kernel (two CTAs per chunk: dq, dk) and bwd_dv_kernel (two
-//      CTAs per chunk: the halves of dv), fully parallel, tcgen05 for every
-//      contraction; the masked, decayed dP / P tiles stay in tensor memory
-//      as bf16 hi + lo and feed the next MMA from there; the epilogues also
-//      emit q.dq and k.dk per token and per chunk;
+//   1. state kernel, forward, state-only: h_c for every chunk (bf16 hi + lo
+//      planes), and S_T when an upstream dS_T is given -- skipped when the
+//      forward kept the states (gla_chunk_fwd_train / gla_chunk_bwd_saved);
+//   2. state kernel, reverse: D_c for every chunk (hi + lo), dS_0 = D_{-1};
+//   3. bwd_dqdk_persistent_kernel (dq and dk of a chunk in one CTA, one CTA
+//      per SM) and bwd_dv_kernel (the halves of dv, one CTA per SM), tcgen05
+//      for every contraction; the masked, decayed dP / P tiles stay in tensor
+//      memory as bf16 hi + lo and feed the next MMA from there; the dq / dk
+//      epilogues also emit q.dq and k.dk per token and per chunk;
 //   4. da_finish_kernel: reverse cumulative sum over T (plus <dS_T, S_T>
 //      from state_dot_kernel when dS_T is given), restarted every 16 chunks
 //      from the closed form <dS_a, S_a> (da_anchor_kernel).
@@ -54,17 +55,10 @@ struct BwdParams {
 
 
 
-// Threads: warps 0-7 are workers; warp 8 only issues TMA and tcgen05.mma.
-constexpr int kThreadsBwd = 288;
 
 __device__ __forceinline__ void named_sync128()
 {
     asm volatile("bar.sync 1, 128;" ::: "memory");
-}
-
-__device__ __forceinline__ void named_sync256()
-{
-    asm volatile("bar.sync 2, 256;" ::: "memory");
 }
 
 // Inclusive cumulative log2-decay of the chunk's tokens, warps 0-3.
@@ -84,41 +78,6 @@ __device__ __forceinline__ void chunk_cumsum(float a, float* b2s, float* wsum, i
     b2s[tid] = x + pre;
 }
 
-// ------------------------------------------------------------ dq, dk kernel
-//
-// Two CTAs per chunk, role 0 (dq) and role 1 (dk), each 87 KB of shared
-// memory and 256 TMEM columns, so two share an SM.  With gamma the chunk's
-// total log-decay and T the masked tile of the dO / V products:
-//
-//   role 0:  dq_i = s e^{b_i} ( dO_i h^T + sum_{j <= i} (dO_i . v_j) e^{-b_j} k_j )
-//   role 1:  dk_j = e^{gamma - b_j} ( v_j D^T + sum_{i >= j} s e^{b_i - gamma} (v_j . dO_i) q_i )
-//
-// The contraction over dv (T = dO V^T for role 0, V dO^T for role 1, and the
-// state product into the accumulator) streams through three shared-memory
-// slots in six 32-column slices; each slice carries the state as its bf16
-// hi and lo planes, both multiplied into the accumulator, so the state
-// product keeps the fp32 state's precision (q.dq and k.dk, and through them
-// da, are sums that cancel to a small fraction of their terms).  T is then
-// turned in place, in tensor memory, into the bf16 hi and lo halves of the
-// decayed tile and used as the A operand of the MMA against K (role 0) or Q
-// (role 1); the row factor is applied in the epilogue.  Chunks whose decay
-// spans more than 2^100 take the exact path: the tile carries
-// s e^{b_i - b_j}, the state product is scaled in place by the row factor
-// before the tile MMA, row factor 1.  Each role also writes its half of the
-// per-token delta of the da sum, q.dq (role 0) or k.dk (role 1), and that
-// half's chunk total.
-
-namespace bq {   // dq / dk kernel shared-memory map (SW64 tiles, 32 columns wide)
-constexpr uint32_t SLOT = 28672;         // first [128][32], second [128][32], state hi, lo [96][32]
-constexpr uint32_t SECOND = 8192, STATE_HI = 16384, STATE_LO = 22528;
-constexpr int kSlots = 3, kSlices = 6;
-constexpr uint32_t MISC = kSlots * SLOT;
-constexpr uint32_t BYTES = MISC + 2048 + 1024;
-constexpr uint32_t TM_T = 0, TM_ACC = 128, TMEM_COLS = 256;
-constexpr uint32_t kSliceBytes = 2 * 8192 + 2 * 6144;
-constexpr uint32_t kTileBytes = 3 * 128 * 64;
-}  // namespace bq
-
 // TMEM column of the hi words of K step ks (16 tokens) of a tile kept as
 // [32-token block: 16 hi columns, 16 lo columns]; the lo words are 16 further.
 __device__ __forceinline__ uint32_t ts_hi(uint32_t base, int ks)
@@ -126,298 +85,376 @@ __device__ __forceinline__ uint32_t ts_hi(uint32_t base, int ks)
     return base + 32 * (ks >> 1) + 8 * (ks & 1);
 }
 
-// Phases of one mbarrier issued and waited for by the issuing thread.
-struct BarTrack {
-    int issued = 0, waited = 0;
-};
+// ------------------------------------------------------------ dq, dk kernel
+//
+// With gamma the chunk's total log-decay and T the masked tile of the dO / V
+// products:
+//
+//   dq_i = s e^{b_i} ( dO_i h^T + sum_{j <= i} (dO_i . v_j) e^{-b_j} k_j )
+//   dk_j = e^{gamma - b_j} ( v_j D^T + sum_{i >= j} s e^{b_i - gamma} (v_j . dO_i) q_i )
+//
+// The contraction over dv (T_q = dO V^T, T_k = V dO^T and the state products)
+// streams in six 32-column slices; each slice carries h and D as their bf16
+// hi and lo planes, both multiplied into the accumulators, so the state
+// products keep the fp32 states' precision (q.dq and k.dk, and through them
+// da, are sums that cancel to a small fraction of their terms).  The T tiles
+// are then turned in place, in tensor memory, into the bf16 hi and lo halves
+// of the decayed tiles and used as A operands against K (dq) and Q (dk); the
+// row factors are applied in the epilogues.  Chunks whose decay spans more
+// than 2^100 take the exact path: the tiles carry s e^{b_i - b_j}, the state
+// products are scaled in place by the row factors first, row factor 1.  Each
+// gradient also yields its half of the per-token delta of the da sum, q.dq
+// or k.dk, and that half's chunk total.
+//
+// Persistent: both gradients of a chunk in one CTA, one CTA per SM walking
+// the chunks blockIdx.x, + gridDim.x, ...: every input of a chunk is read
+// into the SM once, and the next chunk's loads run under this chunk's
+// conversion and epilogues.
+//
+//   producer warp   per chunk: dv slices 0..2 into the ring as slots free,
+//                   then Q and K once the previous chunk is done with them,
+//                   then slices 3..5; every slice carries dO, V and the
+//                   hi / lo planes of h and D (40 KB, six per chunk)
+//   issuer thread   per slice: T_q += dO V^T, T_k += V dO^T, A_q += dO h^T
+//                   (hi, lo), A_k += V D^T (hi, lo); then, once the tiles
+//                   are converted and Q, K are in, A_q += dP K and
+//                   A_k += dP^T Q (A from tensor memory, hi and lo)
+//   workers 0-7     T_q -> dP in place (bf16 hi + lo), the dq epilogue and
+//                   q.dq; workers 8-15 the same for T_k -> dP^T, dk, k.dk
+// Tensor memory: T_q at 0, A_q at 128, T_k at 256, A_k at 384 (448 of 512
+// columns): one chunk at a time, so a chunk's slice MMAs start once the
+// previous chunk's accumulators are read (the "done" barrier).
 
-__device__ __forceinline__ bool wait_next(uint64_t* bar, BarTrack& t, const WaitCtl& ctl)
-{
-    if (!mbar_wait(bar, t.waited & 1, ctl)) return false;
-    ++t.waited;
-    return true;
-}
+namespace bqp {   // persistent dq / dk kernel shared-memory map
+constexpr uint32_t SLOT = 40960;    // dO [128][32] | V [128][32] | h hi, lo | D hi, lo [96][32], SW64
+constexpr uint32_t S_V = 8192, S_HH = 16384, S_HL = 22528, S_DH = 28672, S_DL = 34816;
+constexpr int kSlots = 3, kSlices = 6;
+constexpr uint32_t QT = kSlots * SLOT;          // q tile [3][128][32] SW64
+constexpr uint32_t KT = QT + 24576;             // k tile
+constexpr uint32_t SQ = KT + 24576;             // dq staging [3][128][32]
+constexpr uint32_t SK = SQ + 24576;             // dk staging
+constexpr uint32_t MISC = SK + 24576;          // barriers, tmem slot, decays, delta partials: 4,288 B
+constexpr uint32_t BYTES = MISC + 4608 + 1024;
+constexpr uint32_t TM_TQ = 0, TM_AQ = 128, TM_TK = 256, TM_AK = 384, TMEM_COLS = 512;
+constexpr uint32_t kSliceBytes = 2 * 8192 + 4 * 6144;
+constexpr int kWorkers = 512;
+constexpr int kThreads = kWorkers + 64;
+}  // namespace bqp
 
-__device__ __forceinline__ void drain(uint64_t* bar, BarTrack& t, const WaitCtl& ctl)
+__global__ void __launch_bounds__(bqp::kThreads, 1) bwd_dqdk_persistent_kernel(const __grid_constant__ BwdParams p)
 {
-    for (; t.waited < t.issued; ++t.waited) mbar_wait(bar, t.waited & 1, ctl);
-}
-
-__global__ void __launch_bounds__(kThreadsBwd, 2) bwd_dqdk_kernel(const __grid_constant__ BwdParams p)
-{
+    using namespace bqp;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(sm);
-    uint64_t* bar_full = reinterpret_cast<uint64_t*>(sm + bq::MISC);   // [3] slot loaded
-    uint64_t* bar_free = bar_full + 3;                                  // [3] slot's MMAs done
-    uint64_t* bar_done = bar_full + 6;                                  // all MMAs so far done
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_full + 7);
-    float* b2s = reinterpret_cast<float*>(sm + bq::MISC + 64);
-    float* cfs = b2s + 128;                  // [128] column factors of the fast path
-    float* wsum = cfs + 128;
-    float* dpart = wsum + 8;                 // [128] delta partial of column half 1
+    uint64_t* bar_full = reinterpret_cast<uint64_t*>(sm + MISC);   // [3] slot loaded
+    uint64_t* bar_empty = bar_full + 3;                           // [3] slot's MMAs done
+    uint64_t* bar_qk = bar_full + 6;                              // q, k tiles loaded
+    uint64_t* bar_sl = bar_full + 7;                              // a chunk's slice MMAs done
+    uint64_t* bar_cv = bar_full + 8;                              // both tiles converted (512)
+    uint64_t* bar_tl = bar_full + 9;                              // tile MMAs done
+    uint64_t* bar_free = bar_full + 10;                           // accumulators and q, k tiles read (512)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_full + 11);
+    float* b2s = reinterpret_cast<float*>(sm + MISC + 128);       // [2][128] by chunk parity
+    float* cfq = b2s + 256;                                       // [2][128] 2^{-b_j}
+    float* cfk = cfq + 256;                                       // [2][128] s 2^{b_i - gamma}
+    float* wsum = cfk + 256;                                      // [8]
+    float* dpart = wsum + 8;                                      // [2][128] delta partial of column half 1
+    float* rsum = dpart + 256;                                    // [2][4] chunk-total partials
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x >> 1, role = blockIdx.x & 1, h = blockIdx.y, b = blockIdx.z;
-    const int unit = b * p.H + h;
-    const int t0 = c * kChunk;
+    const bool worker = warp < 16;
+    const bool issuer = warp == 16 && lane == 0;
+    const bool producer = warp == 17 && lane == 0;
+    const int role = (warp >> 3) & 1;                    // workers: 0 dq, 1 dk
     const int quad = warp & 3, half = (warp >> 2) & 1, row = quad * 32 + lane;
-    const bool worker = warp < 8;
-    const bool issuer = warp == 8 && lane == 0;
+    const int wtid = tid & 255;                          // thread index within the role's 256
     const WaitCtl ctl = p.ctl;
-    const CUtensorMap* tm_first = role ? &p.tm_v32 : &p.tm_do32;
-    const CUtensorMap* tm_second = role ? &p.tm_do32 : &p.tm_v32;
-    const CUtensorMap* tm_state = role ? &p.tm_d32 : &p.tm_h32;
-    const CUtensorMap* tm_op = role ? &p.tm_q : &p.tm_k;      // B operand of the tile MMA
-    const CUtensorMap* tm_dot = role ? &p.tm_k : &p.tm_q;     // partner of the delta dot
-    const int state_idx = (unit * p.NC + c) * 2;              // hi plane; lo at + 1
-    BarTrack tr_full[bq::kSlots], tr_free[bq::kSlots], tr_done;
-    bool failed = false;
+
+    const int total = p.B * p.H * p.NC;
+    const int first = blockIdx.x, stride = gridDim.x;
+    const int n = first < total ? (total - first + stride - 1) / stride : 0;
+    struct Item {
+        int b, h, c, unit;
+    };
+    auto item = [&](int k) {
+        const int it = first + k * stride;
+        Item r;
+        r.unit = it / p.NC;
+        r.c = it - r.unit * p.NC;
+        r.b = r.unit / p.H;
+        r.h = r.unit - r.b * p.H;
+        return r;
+    };
 
     if (issuer) {
-        for (int i = 0; i < 7; ++i) mbar_init(bar_full + i, 1);
+        for (int i = 0; i < 11; ++i) mbar_init(bar_full + i, (i == 8 || i == 10) ? kWorkers : 1);
         mbar_init_fence();
+        tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_k);
+        tma_prefetch_desc(&p.tm_do32);
+        tma_prefetch_desc(&p.tm_v32);
+        tma_prefetch_desc(&p.tm_h32);
+        tma_prefetch_desc(&p.tm_d32);
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, bq::TMEM_COLS);
+        tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tq = tmem_addr(tmem, quad * 32, 0);
 
-    auto load_slice = [&](int sl) {
-        const int k = sl % bq::kSlots;
-        uint8_t* base = sm + k * bq::SLOT;
-        mbar_arrive_expect_tx(bar_full + k, bq::kSliceBytes);
-        tma_load_4d(base, tm_first, bar_full + k, sl * 32, h, t0, b);
-        tma_load_4d(base + bq::SECOND, tm_second, bar_full + k, sl * 32, h, t0, b);
-        tma_load_3d(base + bq::STATE_HI, tm_state, bar_full + k, sl * 32, 0, state_idx);
-        tma_load_3d(base + bq::STATE_LO, tm_state, bar_full + k, sl * 32, 0, state_idx + 1);
-        ++tr_full[k].issued;
-    };
-    auto load_tile = [&](int k, const CUtensorMap* m) {
-        uint8_t* base = sm + k * bq::SLOT;
-        mbar_arrive_expect_tx(bar_full + k, bq::kTileBytes);
-        for (int i = 0; i < 3; ++i) tma_load_4d(base + i * 8192, m, bar_full + k, i * 32, h, t0, b);
-        ++tr_full[k].issued;
-    };
-    // slice sl: two K steps of 16 (32 bytes each) inside the 64-byte rows
-    auto mma_slice = [&](int sl) {
-        const uint32_t base = sb + (sl % bq::kSlots) * bq::SLOT;
-        const uint64_t da = smem_desc(base, 16, 512, kLayoutSW64);
-        const uint64_t db = smem_desc(base + bq::SECOND, 16, 512, kLayoutSW64);
-        const uint64_t dh = smem_desc(base + bq::STATE_HI, 16, 512, kLayoutSW64);
-        const uint64_t dl = smem_desc(base + bq::STATE_LO, 16, 512, kLayoutSW64);
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-            const uint64_t a = desc_add(da, ks * 32);
-            const uint32_t acc = (sl | ks) > 0;
-            umma_bf16(tmem + bq::TM_T, a, desc_add(db, ks * 32), idesc_bf16_f32(128, 128, 0, 0), acc);
-            umma_bf16(tmem + bq::TM_ACC, a, desc_add(dh, ks * 32), idesc_bf16_f32(128, 96, 0, 0), acc);
-            umma_bf16(tmem + bq::TM_ACC, a, desc_add(dl, ks * 32), idesc_bf16_f32(128, 96, 0, 0), 1);
-        }
-    };
-
-    if (issuer) {
-        for (int sl = 0; sl < bq::kSlots; ++sl) load_slice(sl);
-    }
-    if (tid < 128) {
-        const int t = t0 + tid;
-        chunk_cumsum(t < p.T ? p.a[(static_cast<int64_t>(b) * p.T + t) * p.H + h] : 0.f, b2s, wsum, tid, warp,
-                     lane);
-        const float g2 = ((wsum[0] + wsum[1]) + wsum[2]) + wsum[3];   // the order b2s[127] sums in
-        const float b2 = b2s[tid];
-        cfs[tid] = role ? p.scale * exp2f(b2 - g2) : exp2f(-b2);
-    }
-    __syncthreads();
-    const float g2 = b2s[127];
-    const bool fast = -g2 <= chunk::kFactorRange;
-
-    // T and the state product over the six dv slices.  Slice sl uses slot
-    // sl % 3; once slice sl's MMAs are issued, the slot of slice sl-1 is
-    // refilled (with slice sl+2, then the tile operand, then the dot
-    // partner) as soon as its MMAs are done, so one slot's MMAs run while
-    // the next slot loads.
-    if (issuer) {
+    if (producer) {
+        // ----------------------------------------------------------- loads
+        int n_full[kSlots] = {0, 0, 0}, n_qk = 0, sidx = 0;
         bool ok = true;
-        for (int sl = 0; ok && sl < bq::kSlices; ++sl) {
-            const int k = sl % bq::kSlots;
-            if (!(ok = wait_next(bar_full + k, tr_full[k], ctl))) break;
-            tc_fence_after();
-            mma_slice(sl);
-            if (sl + 1 < bq::kSlices) {
-                umma_commit(bar_free + k);
-                ++tr_free[k].issued;
-            } else {
-                umma_commit(bar_done);
-                ++tr_done.issued;
+        auto load_slice = [&](const Item& w, int sl) {
+            const int slot = sidx % kSlots;
+            if (sidx >= kSlots && !mbar_wait(bar_empty + slot, ((sidx - kSlots) / kSlots) & 1, ctl)) return false;
+            uint8_t* base = sm + slot * SLOT;
+            const int t0 = w.c * kChunk, si = (w.unit * p.NC + w.c) * 2;
+            mbar_arrive_expect_tx(bar_full + slot, kSliceBytes);
+            tma_load_4d(base, &p.tm_do32, bar_full + slot, sl * 32, w.h, t0, w.b);
+            tma_load_4d(base + S_V, &p.tm_v32, bar_full + slot, sl * 32, w.h, t0, w.b);
+            tma_load_3d(base + S_HH, &p.tm_h32, bar_full + slot, sl * 32, 0, si);
+            tma_load_3d(base + S_HL, &p.tm_h32, bar_full + slot, sl * 32, 0, si + 1);
+            tma_load_3d(base + S_DH, &p.tm_d32, bar_full + slot, sl * 32, 0, si);
+            tma_load_3d(base + S_DL, &p.tm_d32, bar_full + slot, sl * 32, 0, si + 1);
+            ++n_full[slot];
+            ++sidx;
+            return true;
+        };
+        for (int k = 0; ok && k < n; ++k) {
+            const Item w = item(k);
+            for (int sl = 0; ok && sl < 3; ++sl) ok = load_slice(w, sl);
+            // q, k of this chunk once the previous chunk has read its tiles
+            if (ok && k >= 1 && !mbar_wait(bar_free, (k - 1) & 1, ctl)) ok = false;
+            if (ok) {
+                const int t0 = w.c * kChunk;
+                mbar_arrive_expect_tx(bar_qk, 2 * 24576);
+                for (int i = 0; i < 3; ++i) {
+                    tma_load_4d(sm + QT + i * 8192, &p.tm_q, bar_qk, i * 32, w.h, t0, w.b);
+                    tma_load_4d(sm + KT + i * 8192, &p.tm_k, bar_qk, i * 32, w.h, t0, w.b);
+                }
+                ++n_qk;
             }
-            if (sl >= 1) {
-                const int kp = (sl - 1) % bq::kSlots;
-                if (!(ok = wait_next(bar_free + kp, tr_free[kp], ctl))) break;
-                if (sl + 2 < bq::kSlices)
-                    load_slice(sl + 2);
-                else if (sl + 2 == bq::kSlices)
-                    load_tile(kp, tm_op);    // slot 0, after slice 3
-                else
-                    load_tile(kp, tm_dot);   // slot 1, after slice 4
-            }
+            for (int sl = 3; ok && sl < kSlices; ++sl) ok = load_slice(w, sl);
         }
-        // the issuer consumes every phase of bar_done in order, so that its
-        // parity never refers to a phase two ahead of the one it waits for
-        if (ok) ok = wait_next(bar_done, tr_done, ctl);
-        failed = !ok;
-    } else if (worker && !mbar_wait(bar_done, 0, ctl)) {
-        // (the issuer warp's other lanes wait at the block barrier instead of
-        // spinning beside the issuing lane)
-        failed = true;
-    }
-    tc_fence_before();
-    if (__syncthreads_or(failed)) goto done;
-    tc_fence_after();
+        // at most one load per barrier is ever outstanding
+        for (int i = 0; i < kSlots; ++i)
+            if (n_full[i]) mbar_wait(bar_full + i, (n_full[i] - 1) & 1, ctl);
+        if (n_qk) mbar_wait(bar_qk, (n_qk - 1) & 1, ctl);
+    } else if (issuer) {
+        // ------------------------------------------------------------ MMAs
+        const uint32_t idT = idesc_bf16_f32(128, 128, 0, 0), idA = idesc_bf16_f32(128, 96, 0, 0);
+        const uint32_t idB = idesc_bf16_f32(128, 96, 0, 1);
+        int n_empty[kSlots] = {0, 0, 0}, n_sl = 0, n_tl = 0, sidx = 0;
+        bool ok = true;
+        for (int k = 0; ok && k < n; ++k) {
+            // the previous chunk's accumulators have been read out
+            if (k >= 1 && !mbar_wait(bar_free, (k - 1) & 1, ctl)) break;
+            tc_fence_after();
+            for (int sl = 0; sl < kSlices; ++sl, ++sidx) {
+                const int slot = sidx % kSlots;
+                if (!mbar_wait(bar_full + slot, (sidx / kSlots) & 1, ctl)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t base = sb + slot * SLOT;
+                const uint64_t ddo = smem_desc(base, 16, 512, kLayoutSW64);
+                const uint64_t dv = smem_desc(base + S_V, 16, 512, kLayoutSW64);
+                const uint64_t dhh = smem_desc(base + S_HH, 16, 512, kLayoutSW64);
+                const uint64_t dhl = smem_desc(base + S_HL, 16, 512, kLayoutSW64);
+                const uint64_t ddh = smem_desc(base + S_DH, 16, 512, kLayoutSW64);
+                const uint64_t ddl = smem_desc(base + S_DL, 16, 512, kLayoutSW64);
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    const uint32_t o = ks * 32, acc = (sl | ks) > 0;
+                    umma_bf16(tmem + TM_TQ, desc_add(ddo, o), desc_add(dv, o), idT, acc);
+                    umma_bf16(tmem + TM_TK, desc_add(dv, o), desc_add(ddo, o), idT, acc);
+                    umma_bf16(tmem + TM_AQ, desc_add(ddo, o), desc_add(dhh, o), idA, acc);
+                    umma_bf16(tmem + TM_AQ, desc_add(ddo, o), desc_add(dhl, o), idA, 1);
+                    umma_bf16(tmem + TM_AK, desc_add(dv, o), desc_add(ddh, o), idA, acc);
+                    umma_bf16(tmem + TM_AK, desc_add(dv, o), desc_add(ddl, o), idA, 1);
+                }
+                umma_commit(bar_empty + slot);
+                ++n_empty[slot];
+            }
+            if (!ok) break;
+            umma_commit(bar_sl);
+            ++n_sl;
+            // the tiles: dP (hi, lo) against K, dP^T against Q
+            if (!mbar_wait(bar_cv, k & 1, ctl) || !mbar_wait(bar_qk, k & 1, ctl)) break;
+            tc_fence_after();
+            const uint64_t dk = smem_desc(sb + KT, 8192, 512, kLayoutSW64);
+            const uint64_t dq = smem_desc(sb + QT, 8192, 512, kLayoutSW64);
+#pragma unroll
+            for (int part = 0; part < 2; ++part)
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    umma_bf16_ts(tmem + TM_AQ, tmem + ts_hi(TM_TQ, ks) + 16 * part, desc_add(dk, ks * 1024), idB, 1);
+                    umma_bf16_ts(tmem + TM_AK, tmem + ts_hi(TM_TK, ks) + 16 * part, desc_add(dq, ks * 1024), idB, 1);
+                }
+            umma_commit(bar_tl);
+            ++n_tl;
+        }
+        // every commit's arrival has landed before the barriers go away
+        for (int i = 0; i < kSlots; ++i)
+            if (n_empty[i]) mbar_wait(bar_empty + i, (n_empty[i] - 1) & 1, ctl);
+        if (n_sl) mbar_wait(bar_sl, (n_sl - 1) & 1, ctl);
+        if (n_tl) mbar_wait(bar_tl, (n_tl - 1) & 1, ctl);
+    } else if (worker) {
+        // --------------------------------------------------------- workers
+        const uint32_t tq = tmem_addr(tmem, quad * 32, 0);
+        const uint32_t TT = role ? TM_TK : TM_TQ, TA = role ? TM_AK : TM_AQ;
+        uint8_t* stg = sm + (role ? SK : SQ);
+        const uint8_t* dot = sm + (role ? KT : QT);      // partner of the delta dot: k (dk) or q (dq)
+        float* dp = dpart + role * 128;
+        bool ok = true;
+        for (int k = 0; ok && k < n; ++k) {
+            const Item w = item(k);
+            const int par = k & 1, t0 = w.c * kChunk;
+            float* bz = b2s + par * 128;
+            // decays of this chunk (warps 0-3); the buffers of parity par were
+            // last read by chunk k-2, finished before chunk k-1's barriers
+            if (tid < 128) {
+                const int t = t0 + tid;
+                chunk_cumsum(t < p.T ? p.a[(static_cast<int64_t>(w.b) * p.T + t) * p.H + w.h] : 0.f, bz, wsum, tid,
+                             warp, lane);
+                const float g2 = ((wsum[0] + wsum[1]) + wsum[2]) + wsum[3];
+                cfq[par * 128 + tid] = exp2f(-bz[tid]);
+                cfk[par * 128 + tid] = p.scale * exp2f(bz[tid] - g2);
+            }
+            chunk::named_sync(2, kWorkers);
+            const float g2 = bz[127];
+            const bool fast = -g2 <= chunk::kFactorRange;
+            const float* cfs = (role ? cfk : cfq) + par * 128;
+            const float b2r = bz[row];
+            const float rowf = role ? exp2f(g2 - b2r) : p.scale * exp2f(b2r);
 
-    if (worker) {
-        const float b2r = b2s[row];
-        const float rowf = role ? exp2f(g2 - b2r) : p.scale * exp2f(b2r);
+            // T -> decayed tile (hi, lo) in place; on the exact path also the
+            // state product's row factor
+            const bool got = mbar_wait(bar_sl, k & 1, ctl);
+            if (chunk::bar_or(2, kWorkers, !got)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
 #pragma unroll
-        for (int kb2 = 0; kb2 < 2; ++kb2) {
-            const int c0 = half * 64 + kb2 * 32;
-            const uint32_t col = bq::TM_T + c0;
-            const bool dead = role ? (c0 + 31 < quad * 32) : (c0 > quad * 32 + 31);
-            uint32_t hi[16], lo[16];
-            if (dead) {
+            for (int kb2 = 0; kb2 < 2; ++kb2) {
+                const int c0 = half * 64 + kb2 * 32;
+                const uint32_t col = TT + c0;
+                const bool dead = role ? (c0 + 31 < quad * 32) : (c0 > quad * 32 + 31);
+                uint32_t hi[16], lo[16];
+                if (dead) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
-            } else {
-                uint32_t r[32];
-                tmem_ld32(tq + col, r);
-                tmem_ld_wait();
+                    for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
+                } else {
+                    uint32_t r[32];
+                    tmem_ld32(tq + col, r);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float v[2];
+                    for (int e = 0; e < 32; e += 2) {
+                        float v[2];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int cc = c0 + e + u;
-                        const bool keep = role ? (cc >= row) : (cc <= row);
-                        const float f = fast ? cfs[cc]
-                                             : p.scale * exp2f(role ? b2s[cc] - b2r : b2r - b2s[cc]);
-                        v[u] = keep ? __uint_as_float(r[e + u]) * f : 0.f;
+                        for (int u = 0; u < 2; ++u) {
+                            const int cc = c0 + e + u;
+                            const bool keep = role ? (cc >= row) : (cc <= row);
+                            const float f = fast ? cfs[cc] : p.scale * exp2f(role ? bz[cc] - b2r : b2r - bz[cc]);
+                            v[u] = keep ? __uint_as_float(r[e + u]) * f : 0.f;
+                        }
+                        const uint32_t hv = pack_bf16(v[0], v[1]);
+                        hi[e / 2] = hv;
+                        lo[e / 2] = pack_bf16(v[0] - bf16_lo(hv), v[1] - bf16_hi(hv));
                     }
-                    const uint32_t hv = pack_bf16(v[0], v[1]);
-                    hi[e / 2] = hv;
-                    lo[e / 2] = pack_bf16(v[0] - bf16_lo(hv), v[1] - bf16_hi(hv));
+                }
+                tmem_st16(tq + col, hi);
+                tmem_st16(tq + col + 16, lo);
+            }
+            if (!fast) {
+#pragma unroll
+                for (int j = 0; j < 3; ++j) {
+                    const uint32_t col = TA + half * 48 + j * 16;
+                    uint32_t u[16];
+                    tmem_ld16(tq + col, u);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(rowf * __uint_as_float(u[e]));
+                    tmem_st16(tq + col, u);
                 }
             }
-            tmem_st16(tq + col, hi);
-            tmem_st16(tq + col + 16, lo);
-        }
-        if (!fast) {
-            // exact path: the state product takes its row factor now
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bar_cv);
+
+            // epilogue: out = f acc -> staging; delta partial against q or k
+            const bool got2 = mbar_wait(bar_tl, k & 1, ctl);
+            if (wtid == 0) tma_store_wait_read();      // the staging's previous store has read it
+            if (chunk::bar_or(2, kWorkers, !got2)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float f = fast ? rowf : 1.0f;
+            uint32_t u[3][16];
+#pragma unroll
+            for (int j = 0; j < 3; ++j) tmem_ld16(tq + TA + half * 48 + j * 16, u[j]);
+            tmem_ld_wait();
+            float dsum = 0.f;
 #pragma unroll
             for (int j = 0; j < 3; ++j) {
-                const uint32_t col = bq::TM_ACC + half * 48 + j * 16;
-                uint32_t u[16];
-                tmem_ld16(tq + col, u);
-                tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(rowf * __uint_as_float(u[e]));
-                tmem_st16(tq + col, u);
-            }
-        }
-        tmem_st_wait();
-    }
-    tc_fence_before();
-    __syncthreads();
-
-    // acc += tile (hi, lo) x K or Q, A from tensor memory
-    if (issuer) {
-        tc_fence_after();
-        // the tile operand sits in slot 0 (its third load), the dot partner in
-        // slot 1 (its third load: phase parity 0)
-        bool ok = wait_next(bar_full, tr_full[0], ctl);
-        if (ok) {
-            for (int part = 0; part < 2; ++part)
-                for (int ks = 0; ks < 8; ++ks)
-                    umma_bf16_ts(tmem + bq::TM_ACC, tmem + ts_hi(bq::TM_T, ks) + 16 * part,
-                                 smem_desc(sb + ks * 1024, 8192, 512, kLayoutSW64),
-                                 idesc_bf16_f32(128, 96, 0, 1), 1);
-            umma_commit(bar_done);
-            ++tr_done.issued;
-            ok = wait_next(bar_done, tr_done, ctl) && wait_next(bar_full + 1, tr_full[1], ctl);
-        }
-        failed = !ok;
-    } else if (worker && (!mbar_wait(bar_done, 1, ctl) || !mbar_wait(bar_full + 1, 0, ctl))) {
-        failed = true;
-    }
-    tc_fence_before();
-    if (__syncthreads_or(failed)) goto done;
-    tc_fence_after();
-    if (worker) {
-        // epilogue: out = f acc -> staging [3][128][32] SW64 in slot 2; delta partial
-        const float f = fast ? (role ? exp2f(g2 - b2s[row]) : p.scale * exp2f(b2s[row])) : 1.0f;
-        float dsum = 0.f;
+                for (int g = 0; g < 2; ++g) {
+                    const int nn = half * 48 + j * 16 + g * 8;
+                    const uint32_t off = (nn >> 5) * 8192 + swz_off(row, (nn & 31) >> 3, 64);
+                    const uint4 wv4 = *reinterpret_cast<const uint4*>(dot + off);
+                    const uint32_t wv[4] = {wv4.x, wv4.y, wv4.z, wv4.w};
+                    uint32_t pk[4];
 #pragma unroll
-        for (int j = 0; j < 3; ++j) {
-            const int n0 = half * 48 + j * 16;
-            uint32_t u[16];
-            tmem_ld16(tq + bq::TM_ACC + n0, u);
-            tmem_ld_wait();
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
-                const int n = n0 + g * 8;
-                const uint32_t off = (n >> 5) * 8192 + swz_off(row, (n & 31) >> 3, 64);
-                const uint4 w = *reinterpret_cast<const uint4*>(sm + bq::SLOT + off);   // q or k, slot 1
-                const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-                uint32_t pk[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float x0 = f * __uint_as_float(u[g * 8 + 2 * e]);
-                    const float x1 = f * __uint_as_float(u[g * 8 + 2 * e + 1]);
-                    dsum = fmaf(bf16_lo(wv[e]), x0, dsum);
-                    dsum = fmaf(bf16_hi(wv[e]), x1, dsum);
-                    pk[e] = pack_bf16(x0, x1);
+                    for (int e = 0; e < 4; ++e) {
+                        const float x0 = f * __uint_as_float(u[j][g * 8 + 2 * e]);
+                        const float x1 = f * __uint_as_float(u[j][g * 8 + 2 * e + 1]);
+                        dsum = fmaf(bf16_lo(wv[e]), x0, dsum);
+                        dsum = fmaf(bf16_hi(wv[e]), x1, dsum);
+                        pk[e] = pack_bf16(x0, x1);
+                    }
+                    *reinterpret_cast<uint4*>(stg + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
-                *reinterpret_cast<uint4*>(sm + 2 * bq::SLOT + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+            // accumulators and the q, k tiles are read: the next chunk may start
+            tc_fence_before();
+            mbar_arrive(bar_free);
+            if (half) dp[row] = dsum;
+            fence_async_smem();
+            chunk::named_sync(3 + role, 256);
+            if (!half) {
+                const bool live = t0 + row < p.T;
+                float x = live ? dsum + dp[row] : 0.f;
+                if (live && GLA_DCHECK(w.unit < p.B * p.H && w.c < p.NC, ctl.status))
+                    p.delta[(static_cast<int64_t>(role) * p.B * p.H + w.unit) * p.T + t0 + row] = x;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+                if (lane == 0) rsum[role * 4 + quad] = x;
+            }
+            chunk::named_sync(3 + role, 256);
+            if (wtid == 0) {
+                if (GLA_DCHECK(w.unit < p.B * p.H && w.c < p.NC, ctl.status))
+                    p.ctot[(static_cast<int64_t>(w.unit) * p.NC + w.c) * 2 + role] =
+                        ((rsum[role * 4] + rsum[role * 4 + 1]) + rsum[role * 4 + 2]) + rsum[role * 4 + 3];
+                const CUtensorMap* tm_out = role ? &p.tm_dk : &p.tm_dq;
+                for (int i = 0; i < 3; ++i) tma_store_4d(tm_out, stg + i * 8192, i * 32, w.h, t0, w.b);
+                tma_store_commit();
             }
         }
-        if (half) dpart[row] = dsum;
-        fence_async_smem();
-        tc_fence_before();
-        named_sync256();
-        if (!half) {
-            const bool live = t0 + row < p.T;
-            float x = live ? dsum + dpart[row] : 0.f;
-            if (live && GLA_DCHECK(unit < p.B * p.H && c < p.NC, ctl.status))
-                p.delta[(static_cast<int64_t>(role) * p.B * p.H + unit) * p.T + t0 + row] = x;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-            if (lane == 0) wsum[quad] = x;
-            named_sync128();
-            if (row == 0 && GLA_DCHECK(unit < p.B * p.H && c < p.NC, ctl.status)) p.ctot[(static_cast<int64_t>(unit) * p.NC + c) * 2 + role] = ((wsum[0] + wsum[1]) + wsum[2]) + wsum[3];
-        }
-    }
-    __syncthreads();
-    if (issuer) {
-        const CUtensorMap* tm_out = role ? &p.tm_dk : &p.tm_dq;
-        for (int i = 0; i < 3; ++i) tma_store_4d(tm_out, sm + 2 * bq::SLOT + i * 8192, i * 32, h, t0, b);
-        tma_store_commit();
-    }
-done:
-    if (issuer) {
-        for (int k = 0; k < bq::kSlots; ++k) {
-            drain(bar_full + k, tr_full[k], ctl);
-            drain(bar_free + k, tr_free[k], ctl);
-        }
-        drain(bar_done, tr_done, ctl);
-        tma_store_wait_all();
+        if (wtid == 0) tma_store_wait_all();
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, bq::TMEM_COLS);
+    if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 // ----------------------------------------------------------------- dv kernel
@@ -883,7 +920,7 @@ __global__ void __launch_bounds__(kDotThreads) state_dot_kernel(float* __restric
 
 template <typename K>
 gla_status launch_bwd_kernel(K kernel, uint32_t bytes, const BwdParams& p, dim3 grid, cudaStream_t st,
-                             const char* name, int threads = kThreadsBwd)
+                             const char* name, int threads)
 {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
         return check_launch(name);
@@ -1054,9 +1091,8 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
         // persistent: one CTA per SM over the (batch, head, chunk) items
         const int items = units * NC;
         const int grid = items < sms ? items : sms;
-        (void)grid;
-        if ((s = launch_bwd_kernel(bwd_dqdk_kernel, bq::BYTES, bp, dim3(2 * NC, pr.H, pr.B), st,
-                                   "bwd_dqdk_kernel")) != GLA_OK)
+        if ((s = launch_bwd_kernel(bwd_dqdk_persistent_kernel, bqp::BYTES, bp, dim3(grid), st, "bwd_dqdk_kernel",
+                                   bqp::kThreads)) != GLA_OK)
             return s;
     }
     {

@@ -41,6 +41,7 @@ decode state); --skip-decode also skips the long prefill.
 """
 import hashlib
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -375,6 +376,12 @@ def run_ours(args, ws, rank, local):
     build.build()
     gla.lib()
     peaks, peak_kind = load_peaks()
+    if args.only:
+        leg = run_decode if args.only == "decode" else run_long_prefill
+        rec = leg(args, ws, peaks, peak_kind)
+        if rank == 0:
+            print(json.dumps({"only": args.only, args.only: rec}), flush=True)
+        return
     st = torch.cuda.current_stream()
     w = TRAIN
     d = train_buffers(seed=w.seed + 97 * rank)
@@ -656,6 +663,8 @@ def run_long_prefill(args, ws, peaks, peak_kind):
     S_0 on independent q, k, v (their projection is not part of the path).
     Each call is timed on its own, K launches between two events."""
     w = LONG
+    if getattr(args, "lp_tokens", None):            # a smaller case of the same leg (profiling)
+        w = dataclasses.replace(LONG, T=args.lp_tokens, name="long_prefill_t%d" % args.lp_tokens)
     st = torch.cuda.current_stream()
     f = inputs.front_inputs(w.B, w.T, w.D, w.W, seed=w.seed, device="cuda")
     y = torch.empty_like(f["x"])
@@ -709,7 +718,7 @@ def run_long_prefill(args, ws, peaks, peak_kind):
            "front_end": {"us_per_launch": round(t_front * 1e6, 2),
                          "roofline": roof("ln_conv_silu_kernel", front_bytes, t_front)},
            "front_end_bwd": {"us_per_launch": round(t_fbwd * 1e6, 2),
-                             "roofline": roof("conv1d_silu_causal_bwd (row statistics, two tile passes, reduction)",
+                             "roofline": roof("conv1d_silu_causal_bwd (one row pass by clusters of 4 CTAs, reduction)",
                                               front_bwd_bytes, t_fbwd)},
            "gla_fwd": {"us_per_launch": round(t_mix * 1e6, 2),
                        "roofline": roof("gla_chunk_fwd (segmented: state pre-pass, combine, fused pass)",
@@ -728,6 +737,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--skip-decode", action="store_true", help="time the training step only (profiling)")
     ap.add_argument("--skip-e2e", action="store_true", help="no host-buffer end-to-end leg (profiling)")
+    ap.add_argument("--only", choices=["decode", "long_prefill"],
+                    help="run that leg alone and print its record (profiling; no headline line)")
+    ap.add_argument("--lp-tokens", type=int, default=None,
+                    help="sequence length of the long-prefill leg (default 65,536; profiling)")
     args = ap.parse_args()
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -123,7 +123,9 @@ __device__ __forceinline__ uint32_t ts_hi(uint32_t base, int ks)
 //                   q.dq; workers 8-15 the same for T_k -> dP^T, dk, k.dk
 // Tensor memory: T_q at 0, A_q at 128, T_k at 256, A_k at 384 (448 of 512
 // columns): one chunk at a time, so a chunk's slice MMAs start once the
-// previous chunk's accumulators are read (the "done" barrier).
+// previous chunk's accumulators are in the workers' registers (the "acc"
+// barrier, at the start of the epilogue; the producer's next q, k load waits
+// for the end of it, the "free" barrier).
 
 namespace bqp {   // persistent dq / dk kernel shared-memory map
 constexpr uint32_t SLOT = 40960;    // dO [128][32] | V [128][32] | h hi, lo | D hi, lo [96][32], SW64
@@ -154,8 +156,9 @@ __global__ void __launch_bounds__(bqp::kThreads, 1) bwd_dqdk_persistent_kernel(c
     uint64_t* bar_sl = bar_full + 7;                              // a chunk's slice MMAs done
     uint64_t* bar_cv = bar_full + 8;                              // both tiles converted (512)
     uint64_t* bar_tl = bar_full + 9;                              // tile MMAs done
-    uint64_t* bar_free = bar_full + 10;                           // accumulators and q, k tiles read (512)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_full + 11);
+    uint64_t* bar_free = bar_full + 10;                           // q, k tiles read (512)
+    uint64_t* bar_acc = bar_full + 11;                            // accumulators read out of TMEM (512)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_full + 12);
     float* b2s = reinterpret_cast<float*>(sm + MISC + 128);       // [2][128] by chunk parity
     float* cfq = b2s + 256;                                       // [2][128] 2^{-b_j}
     float* cfk = cfq + 256;                                       // [2][128] s 2^{b_i - gamma}
@@ -178,18 +181,22 @@ __global__ void __launch_bounds__(bqp::kThreads, 1) bwd_dqdk_persistent_kernel(c
     struct Item {
         int b, h, c, unit;
     };
+    // chunk-major from chunk 0: the reverse state pass that runs just before
+    // ends on the first chunks of every sequence, so the first items find
+    // their D_c and q, dO tiles still in L2
+    const int units = p.B * p.H;
     auto item = [&](int k) {
         const int it = first + k * stride;
         Item r;
-        r.unit = it / p.NC;
-        r.c = it - r.unit * p.NC;
+        r.c = it / units;
+        r.unit = it - r.c * units;
         r.b = r.unit / p.H;
         r.h = r.unit - r.b * p.H;
         return r;
     };
 
     if (issuer) {
-        for (int i = 0; i < 11; ++i) mbar_init(bar_full + i, (i == 8 || i == 10) ? kWorkers : 1);
+        for (int i = 0; i < 12; ++i) mbar_init(bar_full + i, (i == 8 || i >= 10) ? kWorkers : 1);
         mbar_init_fence();
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_k);
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(bqp::kThreads, 1) bwd_dqdk_persistent_kernel(c
         bool ok = true;
         for (int k = 0; ok && k < n; ++k) {
             // the previous chunk's accumulators have been read out
-            if (k >= 1 && !mbar_wait(bar_free, (k - 1) & 1, ctl)) break;
+            if (k >= 1 && !mbar_wait(bar_acc, (k - 1) & 1, ctl)) break;
             tc_fence_after();
             for (int sl = 0; sl < kSlices; ++sl, ++sidx) {
                 const int slot = sidx % kSlots;
@@ -404,6 +411,9 @@ __global__ void __launch_bounds__(bqp::kThreads, 1) bwd_dqdk_persistent_kernel(c
 #pragma unroll
             for (int j = 0; j < 3; ++j) tmem_ld16(tq + TA + half * 48 + j * 16, u[j]);
             tmem_ld_wait();
+            // the accumulators are in registers: the next chunk's MMAs may start
+            tc_fence_before();
+            mbar_arrive(bar_acc);
             float dsum = 0.f;
 #pragma unroll
             for (int j = 0; j < 3; ++j) {
@@ -425,8 +435,7 @@ __global__ void __launch_bounds__(bqp::kThreads, 1) bwd_dqdk_persistent_kernel(c
                     *reinterpret_cast<uint4*>(stg + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
             }
-            // accumulators and the q, k tiles are read: the next chunk may start
-            tc_fence_before();
+            // the q, k tiles are read: the producer may load the next chunk's
             mbar_arrive(bar_free);
             if (half) dp[row] = dsum;
             fence_async_smem();
@@ -534,12 +543,16 @@ __global__ void __launch_bounds__(dvp::kThreads, 1) bwd_dv_kernel(const __grid_c
     struct Item {
         int b, h, c, dvh, unit;
     };
+    // chunk-major from the last chunk (the two halves of a chunk side by
+    // side): the dq / dk kernel before it ends on the last chunks, so the
+    // first items find their q, k, dO and D tiles still in L2
+    const int units = p.B * p.H;
     auto item = [&](int k) {
-        const int it = first + k * stride;
+        const int it = total - 1 - (first + k * stride);
         Item r;
-        r.unit = it / (2 * p.NC);
-        const int rem = it - r.unit * 2 * p.NC;
-        r.c = rem >> 1;
+        r.c = it / (2 * units);
+        const int rem = it - r.c * 2 * units;
+        r.unit = rem >> 1;
         r.dvh = rem & 1;
         r.b = r.unit / p.H;
         r.h = r.unit - r.b * p.H;

@@ -64,7 +64,6 @@ struct StateParams {
     CUtensorMap tm_u;       // scaled operand: k (forward) or q (reverse)
     CUtensorMap tm_y;
     CUtensorMap tm_o;       // o tile stores (fused forward)       // v (forward) or dO (reverse)
-    CUtensorMap tm_save;    // h_save as [B*H*NC*2][96][192] bf16, 64-column SW128 boxes (fused forward)
     const float* a;         // [B, T, H] log-decay
     const float* s_init;    // initial state per (unit, seg) or null (zeros)
     float* s_out;           // state after the segment, or null
@@ -87,8 +86,7 @@ struct StateParams {
     int varlen_segs;        // 1: segmented varlen (chunks_per_seg chunks per segment)
     int pre_pass;           // state pass: only segments 0 .. nseg_n - 2 of each sequence
     void* h_save;           // fused forward: the state entering each chunk, [B*H*NC][2][96][192]
-                            // bf16 (hi, lo planes), for the backward; null = not saved (TMA-stored
-                            // from the state copy in shared memory through tm_save)
+                            // bf16 (hi, lo planes), for the backward; null = not saved
     float scale;
     WaitCtl ctl;
 };
@@ -118,11 +116,7 @@ struct FusedSmem {
     static constexpr uint32_t U = 24576;      // k tile, then K~ (its 4th M block is X: finite)
     static constexpr uint32_t X = 49152;      // bf16 state copy [3][96][64] SW128
     static constexpr uint32_t KL = 86016;     // lo half of K~ [3][128][32] SW64 (hi: K~ in place in U)
-    static constexpr uint32_t KL_PAD = 110592;   // [8192]: the 4th M block (dk 96..127) of KL
-    static constexpr uint32_t XL = 86016;
-    // XL, training forward: the lo plane of the state copy [3][96][64] SW128,
-    // over KL and KL_PAD (36,864 B up to Y0), between the state update that
-    // reads KL and the next chunk's K~ split that writes it
+    static constexpr uint32_t KL_PAD = 110592;   // [8192] zeros: the 4th M block (dk 96..127) of KL
     static constexpr uint32_t Y0 = 122880;    // v tiles, double buffered
     static constexpr uint32_t Y1 = 172032;    // (the o staging of a chunk, once its P V is done)
     static constexpr uint32_t MISC = 221184;
@@ -292,16 +286,32 @@ __device__ __forceinline__ void tmem_to_state(uint32_t taddr, float* dst)
 
 // State copy into [3][96][64] SW128 (row = dk index, n = dv column), for the
 // 96 columns half*96 .. +95 of this thread's row; then decay the state.
-// With SPLIT the copy is a bf16 hi (in `hi`) + lo (in `lo`) pair.
+// With gsave, the same 96 values also go to global memory as a bf16 hi plane
+// (gsave) and lo plane (gsave + plane_bytes), 32-byte stores.
 template <bool SPLIT>
 __device__ __forceinline__ void state_copy_and_decay(uint32_t taddr, int row, int half, float f,
-                                                     uint8_t* hi, uint8_t* lo, bool copy)
+                                                     uint8_t* hi, uint8_t* lo, bool copy,
+                                                     uint8_t* gsave = nullptr, int64_t plane_bytes = 0)
 {
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
         uint32_t r[32];
         tmem_ld32(taddr + j * 32, r);
         tmem_ld_wait();
+        if (gsave) {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t w[8], l[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float x0 = __uint_as_float(r[16 * h2 + 2 * e]), x1 = __uint_as_float(r[16 * h2 + 2 * e + 1]);
+                    w[e] = pack_bf16(x0, x1);
+                    l[e] = pack_bf16(x0 - bf16_lo(w[e]), x1 - bf16_hi(w[e]));
+                }
+                st_global_v8(gsave + j * 64 + h2 * 32, w);
+                st_global_v8(gsave + plane_bytes + j * 64 + h2 * 32, l);
+            }
+        }
         if (copy) {
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
@@ -350,7 +360,6 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     uint64_t* bar_fo = bar_q + 6;                                // O += P V done
     uint64_t* bar_stg = bar_q + 7;                               // [2] o staged in the v buffer (256)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_q + 9);
-    uint64_t* bar_cps = bar_q + 10;                              // a chunk's state copy stored (training)
     float* b2s = reinterpret_cast<float*>(sm + L::MISC + 128);  // [2][128] by token, chunk parity
     float* cfac = b2s + 256;                                     // [2][128] 2^{-b_j}
     float* wsum = cfac + 256;                                    // [4]
@@ -403,7 +412,6 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         mbar_init(bar_fo, 1);
         mbar_init(bar_stg, kWorkers);
         mbar_init(bar_stg + 1, kWorkers);
-        mbar_init(bar_cps, 1);
         mbar_init_fence();
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_u);
@@ -424,14 +432,12 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         const int t = c * 128 + tid;
         return t < Tn ? p.a[(static_cast<int64_t>(bc) * p.T + tb + t) * p.H + h] : 0.f;
     };
-    // training forward: every chunk's state copy (hi in X, lo in XL) is also
-    // TMA-stored by the producer into h_save, plane 0 and plane 1
-    const bool save = !VARLEN && p.h_save != nullptr;
-    auto copy_state = [&](float f) {
-        if (save)
-            state_copy_and_decay<true>(tq + L::TM_S + half * 96, row, half, f, sm + L::X, sm + L::XL, true);
-        else
-            state_copy_and_decay<false>(tq + L::TM_S + half * 96, row, half, f, sm + L::X, nullptr, true);
+    // this thread's row of the saved state entering chunk c (hi plane), or null
+    constexpr int64_t kStatePlane = static_cast<int64_t>(kDk) * kDv * 2;
+    auto save_row = [&](int c) -> uint8_t* {
+        if (VARLEN || !p.h_save || !GLA_DCHECK(c < p.NC && unit < p.B * p.H, p.ctl.status)) return nullptr;
+        return static_cast<uint8_t*>(p.h_save) + ((static_cast<int64_t>(unit) * p.NC + c) * 2) * kStatePlane +
+               static_cast<int64_t>(row) * (kDv * 2) + half * 192;
     };
     // cumulative log2-decay of a chunk and its column factors (warps 0-3)
     auto decays = [&](float av, int par) {
@@ -462,7 +468,9 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (nchunks > 0 && srow) copy_state(exp2f(b2s[127]));
+    if (nchunks > 0 && srow)
+        state_copy_and_decay<false>(tq + L::TM_S + half * 96, row, half, exp2f(b2s[127]), sm + L::X, nullptr,
+                                    true, save_row(c_begin), kStatePlane);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -498,21 +506,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             for (int i = 0; i < 3; ++i)
                 tma_load_4d(y + i * 16384, &p.tm_y, bar_y + s, i * 64, h, tb + c * 128, bc);
         };
-        // the state copy entering chunk c (X: hi, XL: lo) -> h_save; once its
-        // reads are done the workers may write the next K~ lo over XL
-        auto store_copy = [&](int c) {
-            const int si = (unit * p.NC + c) * 2;
-            if (GLA_DCHECK(c < p.NC && unit < p.B * p.H, p.ctl.status))
-                for (int j = 0; j < 3; ++j) {
-                    tma_store_3d(&p.tm_save, sm + L::X + j * 12288, j * 64, 0, si);
-                    tma_store_3d(&p.tm_save, sm + L::XL + j * 12288, j * 64, 0, si + 1);
-                }
-            tma_store_commit();
-            tma_store_wait_read();
-            mbar_arrive(bar_cps);
-        };
         int n_qu = 0, n_y[2] = {0, 0};
-        if (save && nchunks > 0) store_copy(c_begin);
         if (nchunks > 1) prefetch_qu(c_begin + 1);
         if (nchunks > 0) {
             issue_qu(c_begin);
@@ -539,9 +533,6 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                 for (int i = 0; i < 3; ++i) tma_store_4d(&p.tm_o, y + i * 16384, i * 64, h, tb + c * 128, bc);
                 tma_store_commit();
             }
-            // every worker has staged chunk it's o, so the copy of chunk it+1
-            // made before it is complete
-            if (save && it + 1 < nchunks) store_copy(c + 1);
             if (it + 2 < nchunks) {
                 tma_store_wait_read();
                 issue_y(c + 2, ys);
@@ -601,10 +592,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             const int live = Tn - c * 128;   // varlen: rows past the sequence (the next one's) add nothing
             // 16-byte chunk idx % 4 of row (idx / 4) % 128 of block idx / 512: a
             // warp covers 512 contiguous bytes, so no two lanes share a bank
-            // training forward: XL (under KL) holds this chunk's state copy
-            // until the producer's store has read it
-            if (save && !mbar_wait(bar_cps, it & 1, ctl)) failed = true;
-            for (int idx = tid; !failed && idx < 1536; idx += kWorkers) {
+            for (int idx = tid; idx < 1536; idx += kWorkers) {
                 const int r = (idx >> 2) & 127, blk = idx >> 9, ch = idx & 3;
                 uint4* u = reinterpret_cast<uint4*>(sm + L::U + blk * 8192 + r * 64) + ch;
                 uint4 hi, lo;
@@ -712,7 +700,9 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             named_sync(3, kWorkers);             // the next chunk's total decay is in b2s
             if (!failed && !mbar_wait(bar_d, it & 1, ctl)) failed = true;
             tc_fence_after();
-            if (srow && !failed) copy_state(exp2f(b2s[(par ^ 1) * 128 + 127]));
+            if (srow && !failed)
+                state_copy_and_decay<false>(tq + L::TM_S + half * 96, row, half, exp2f(b2s[(par ^ 1) * 128 + 127]),
+                                            sm + L::X, nullptr, true, save_row(c + 1), kStatePlane);
             fence_async_smem();
         }
 

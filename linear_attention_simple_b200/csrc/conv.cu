@@ -54,11 +54,11 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 // (1 + tanh(u / 2)) / 2), on the hardware tanh approximation.  The kernel
 // folds the 1/2 into the conv weights and bias, so it convolves straight to
 // h: one special-function op and one FMA per element.
-__device__ __forceinline__ float silu_of_half(float h)
+__device__ __forceinline__ float tanh_approx(float h)
 {
     float t;
     asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
-    return fmaf(h, t, h);
+    return t;
 }
 
 // CH channels (one 2*CH-byte vector) per thread.
@@ -73,17 +73,6 @@ struct Vec<8> {
     using T = uint4;
 };
 
-template <int NCH>
-__device__ __forceinline__ void unpack(const typename Vec<NCH>::T& v, float* f)
-{
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(&v);
-#pragma unroll
-    for (int i = 0; i < NCH / 2; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
-
 // OR of v over the n worker threads (named barrier 1; the producer warp is
 // not among them).
 __device__ __forceinline__ bool workers_or(bool v, int n)
@@ -95,25 +84,27 @@ __device__ __forceinline__ bool workers_or(bool v, int n)
 }
 
 // LayerNorm moments of one row of D bf16 values by one warp: (mean, rstd).
+// The sums run on fp32 pairs (even and odd channels), added at the end.
 __device__ __forceinline__ float2 row_moments(const uint8_t* row, int D, float eps, int lane)
 {
     const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(row));
-    float s1 = 0.f, s2 = 0.f;
+    const f2 x02 = f2_splat(x0);
+    f2 s1 = f2_splat(0.f), s2 = f2_splat(0.f);
     for (int c = lane * 8; c < D; c += 256) {
         const uint4 v = *reinterpret_cast<const uint4*>(row + c * 2);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float a = bf16_lo(w[i]) - x0, b = bf16_hi(w[i]) - x0;
-            s1 += a + b;
-            s2 = fmaf(a, a, fmaf(b, b, s2));
+            const f2 d = f2_sub(f2_from_bf16x2(w[i]), x02);
+            s1 = f2_add(s1, d);
+            s2 = f2_fma(d, d, s2);
         }
     }
-    s1 = warp_sum(s1);
-    s2 = warp_sum(s2);
+    const float2 a = f2_get(s1), b = f2_get(s2);
+    const float t1 = warp_sum(a.x + a.y), t2 = warp_sum(b.x + b.y);
     const float invD = 1.0f / static_cast<float>(D);
-    const float m1 = s1 * invD;
-    const float var = fmaxf(s2 * invD - m1 * m1, 0.f);
+    const float m1 = t1 * invD;
+    const float var = fmaxf(t2 * invD - m1 * m1, 0.f);
     return make_float2(x0 + m1, 1.0f / sqrtf(var + eps));
 }
 
@@ -188,31 +179,34 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
     }
 
     // ----------------------------------------------------------- workers
-    float wr[CH][kW], ga[AFF ? CH : 1], be[AFF ? CH : 1], bi[AFF ? CH : 1];
+    // channels in pairs (c0 + 2i, c0 + 2i + 1): every product below is one
+    // fp32-pair instruction
+    constexpr int NP = CH / 2;
+    f2 wr[NP][kW], ga[AFF ? NP : 1], be[AFF ? NP : 1], bi[AFF ? NP : 1];
 #pragma unroll
-    for (int c = 0; c < CH; ++c) {
-        const int ch = active ? c0 + c : 0;
+    for (int i = 0; i < NP; ++i) {
+        const int ch = active ? c0 + 2 * i : 0;
 #pragma unroll
-        for (int j = 0; j < kW; ++j) wr[c][j] = active ? 0.5f * w[ch * kW + j] : 0.f;   // halved: see silu_of_half
+        for (int j = 0; j < kW; ++j)   // halved: see tanh_approx
+            wr[i][j] = active ? f2_make(0.5f * w[ch * kW + j], 0.5f * w[(ch + 1) * kW + j]) : f2_splat(0.f);
         if constexpr (AFF) {
-            ga[c] = (gamma && active) ? gamma[ch] : 1.f;
-            be[c] = (beta && active) ? beta[ch] : 0.f;
-            bi[c] = (bias && active) ? 0.5f * bias[ch] : 0.f;
+            ga[i] = (gamma && active) ? f2_make(gamma[ch], gamma[ch + 1]) : f2_splat(1.f);
+            be[i] = (beta && active) ? f2_make(beta[ch], beta[ch + 1]) : f2_splat(0.f);
+            bi[i] = (bias && active) ? f2_make(0.5f * bias[ch], 0.5f * bias[ch + 1]) : f2_splat(0.f);
         }
     }
 
     // window: the three positions before the stream start p0 (only negative
     // positions matter -- they come from the conv history; the others are
     // shifted out before any output uses them)
-    float win[kW - 1][CH];
+    f2 win[kW - 1][NP];
 #pragma unroll
     for (int r = 0; r < kW - 1; ++r) {
         const int p = p0 - (kW - 1) + r;
+        const float* src = cs_in + (static_cast<int64_t>(b) * (kW - 1) + (kW - 1) + p) * D + c0;
 #pragma unroll
-        for (int c = 0; c < CH; ++c)
-            win[r][c] = (p < 0 && cs_in && active)
-                            ? cs_in[(static_cast<int64_t>(b) * (kW - 1) + (kW - 1) + p) * D + c0 + c]
-                            : 0.f;
+        for (int i = 0; i < NP; ++i)
+            win[r][i] = (p < 0 && cs_in && active) ? f2_make(src[2 * i], src[2 * i + 1]) : f2_splat(0.f);
     }
 
     bool failed = false;
@@ -237,46 +231,47 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
         // one row: normalise, convolve with the window, SiLU, write y (when the
         // row is an output of this CTA), shift the window
         auto do_row = [&](int g, int p, bool out) {
-            float xn[CH];
+            f2 xn[NP];
             if (active) {
-                unpack<CH>(*reinterpret_cast<const V*>(st + g * row_bytes + c0 * 2), xn);
+                const V xv = *reinterpret_cast<const V*>(st + g * row_bytes + c0 * 2);
+                const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xv);
+#pragma unroll
+                for (int i = 0; i < NP; ++i) xn[i] = f2_from_bf16x2(xw[i]);
                 if (apply_ln) {
                     const float2 m = sst[g];
                     if constexpr (AFF) {
+                        const f2 mu = f2_splat(m.x), rs = f2_splat(m.y);
 #pragma unroll
-                        for (int c = 0; c < CH; ++c) xn[c] = fmaf((xn[c] - m.x) * m.y, ga[c], be[c]);
+                        for (int i = 0; i < NP; ++i) xn[i] = f2_fma(f2_mul(f2_sub(xn[i], mu), rs), ga[i], be[i]);
                     } else {
-                        const float sh = -m.x * m.y;
+                        const f2 rs = f2_splat(m.y), sh = f2_splat(-m.x * m.y);
 #pragma unroll
-                        for (int c = 0; c < CH; ++c) xn[c] = fmaf(xn[c], m.y, sh);
+                        for (int i = 0; i < NP; ++i) xn[i] = f2_fma(xn[i], rs, sh);
                     }
                 }
             } else {
 #pragma unroll
-                for (int c = 0; c < CH; ++c) xn[c] = 0.f;
+                for (int i = 0; i < NP; ++i) xn[i] = f2_splat(0.f);
             }
             if (out && GLA_DCHECK(p < T && c0 + CH <= D, ctl.status)) {
                 V o;
                 uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
-                for (int c = 0; c < CH; c += 2) {
-                    float r[2];
+                for (int i = 0; i < NP; ++i) {
+                    f2 acc = AFF ? bi[AFF ? i : 0] : f2_splat(0.f);
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        float acc = AFF ? bi[AFF ? c + e : 0] : 0.f;
-#pragma unroll
-                        for (int j = 0; j < kW - 1; ++j) acc = fmaf(wr[c + e][j], win[j][c + e], acc);
-                        r[e] = silu_of_half(fmaf(wr[c + e][kW - 1], xn[c + e], acc));
-                    }
-                    ow[c / 2] = pack_bf16(r[0], r[1]);
+                    for (int j = 0; j < kW - 1; ++j) acc = f2_fma(wr[i][j], win[j][i], acc);
+                    const f2 h = f2_fma(wr[i][kW - 1], xn[i], acc);
+                    const float2 hh = f2_get(h);
+                    ow[i] = f2_to_bf16x2(f2_fma(h, f2_make(tanh_approx(hh.x), tanh_approx(hh.y)), h));
                 }
                 __stcs(reinterpret_cast<V*>(yb + static_cast<int64_t>(p) * D + c0), o);
             }
 #pragma unroll
-            for (int c = 0; c < CH; ++c) {
-                win[0][c] = win[1][c];
-                win[1][c] = win[2][c];
-                win[2][c] = xn[c];
+            for (int i = 0; i < NP; ++i) {
+                win[0][i] = win[1][i];
+                win[1][i] = win[2][i];
+                win[2][i] = xn[i];
             }
         };
         if (rows == kG && pos0 >= t_begin && active) {
@@ -297,7 +292,12 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
 #pragma unroll
         for (int r = 0; r < kW - 1; ++r)
 #pragma unroll
-            for (int c = 0; c < CH; ++c) cs_out[(static_cast<int64_t>(b) * (kW - 1) + r) * D + c0 + c] = win[r][c];
+            for (int i = 0; i < NP; ++i) {
+                const float2 v = f2_get(win[r][i]);
+                float* dst = cs_out + (static_cast<int64_t>(b) * (kW - 1) + r) * D + c0 + 2 * i;
+                dst[0] = v.x;
+                dst[1] = v.y;
+            }
     }
 }
 

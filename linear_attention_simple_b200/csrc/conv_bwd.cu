@@ -10,19 +10,42 @@
 //   dw[c,j]   = sum_t du[t,c] xn[t-3+j, c]   dbias = sum du
 //   dgamma    = sum dxn xhat                  dbeta = sum dxn
 //
-// Three passes, none with a block-wide barrier per row:
-//   ln_stats_kernel       mean and rstd of every row (a warp per row);
-//   conv_bwd_tile_kernel<false>  tiles of 256 rows x 512 channels, a thread per
-//                         2 channels walking the rows with register windows:
-//                         u, du, dxn, the per-(tile, channel) sums of dw,
-//                         dbias, dgamma, dbeta, the history gradient, and the
-//                         per-row sums of g and g xhat over the tile's
-//                         channels (dx itself when there is no LayerNorm);
-//   conv_bwd_tile_kernel<true>   the same walk again, finishing dx from the
-//                         row totals of those sums.
-// conv_bwd_reduce_kernel adds the per-tile partials in a fixed order, so
-// every output is deterministic.
+// One pass over the rows.  A cluster of CL CTAs (CL = 2 up to D = 2,048, 4
+// above) owns a contiguous token range of one sequence, and CTA r of the
+// cluster owns the r-th block of channels (whole 8-channel units).  Every
+// per-channel quantity -- the conv weights, the windows of the last three
+// rows' xn, xhat and du, the sums of dw, dbias, dgamma, dbeta -- stays in the
+// registers of the thread that owns the channel (4 channels a thread) for
+// the whole range.  A producer warp streams the rows of x and dy through a
+// ring of shared-memory stages of kG rows (bulk asynchronous copies, one per
+// row and tensor, completion on the stage's mbarrier).
+//
+// The LayerNorm needs two reductions over all D channels of a row: the
+// moments of x (before the row can be normalised) and the sums of g and
+// g xhat (before its dx can be written).  Per stage, each CTA reduces its
+// channels' part of both (a 16-value butterfly in each warp, then the warps
+// in a fixed order) and pushes the 24 numbers to every CTA of the cluster
+// with st.async into their shared memory, completing bytes on their
+// exchange mbarrier.  The exchange sent at stage s carries the g sums of the
+// rows that stage finished (q = p - 3) and the moments of the rows two
+// stages ahead; it is combined at stage s + 1, after that stage's rows are
+// done, so the cluster round trip hides under a stage of work.  The rows'
+// g and xhat wait in shared memory (fp32) for their dx until then.  The
+// moments are taken about the first channel of CTA 0 (the row's first
+// element, as the forward does), each CTA's shifted sums being moved to that
+// shift before they are added.
+//
+// The channel sums go out as per-(range, CTA) partials [B * nx][7][D] that
+// conv_bwd_reduce_kernel adds in a fixed order, so every output is
+// deterministic.  The SiLU derivative runs on h = u / 2 with the hardware
+// tanh (sigmoid(u) = (1 + tanh h) / 2); the kernel carries du2 = 2 du, so
+// the conv weights are halved and dw, dbias halved at the end.  Every wait
+// is bounded; on a timeout the CTAs record GLA_ERR_TIMEOUT and leave
+// through the same final cluster barrier.
 #include <cuda_bf16.h>
+
+#include <algorithm>
+#include <type_traits>
 
 #include "gla_device.cuh"
 #include "gla_internal.h"
@@ -30,50 +53,76 @@
 namespace gla {
 namespace {
 
-constexpr int kRows = 256;       // tokens per tile
-constexpr int kTileThreads = 256;
-constexpr int kTileCh = 2 * kTileThreads;   // channels per tile
-constexpr int kParts = 7;        // dw (4 taps), dbias, dgamma, dbeta
+constexpr int kW = 4;
+constexpr int kG = 4;           // rows per stage
+constexpr int kRing = 8;        // ring stages: s, s+1, s+2 (moments) and five in flight
+constexpr int kXch = 4;         // exchange buffers (a CTA runs at most two exchanges ahead)
+constexpr int kMsg = 24;        // floats per CTA per exchange
+constexpr int kStRing = 16;     // rows of LayerNorm statistics kept
+constexpr int kParts = 7;       // dw (4 taps), dbias, dgamma, dbeta
+constexpr int kMaxSlices = 128; // token ranges per sequence
+constexpr int kMinRows = 64;    // rows per range at least
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-__device__ __forceinline__ float warp_sum_bwd(float v)
+__device__ __forceinline__ void bulk_load_bwd(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
 {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
 }
 
-// stats[row] = (mean, rstd) of the row's D values; the moments are taken
-// about the row's first element (shifted), as the forward does.
-__global__ void __launch_bounds__(256) ln_stats_kernel(const __nv_bfloat16* __restrict__ x, int rows, int D,
-                                                       float eps, float2* __restrict__ stats)
+// Barrier over the n worker threads (named barrier 1) returning the OR of v.
+__device__ __forceinline__ bool workers_or_bwd(bool v, int n)
 {
-    const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    const __nv_bfloat16* xr = x + static_cast<int64_t>(row) * D;
-    const float x0 = __bfloat162float(xr[0]);
-    float s1 = 0.f, s2 = 0.f;
-    for (int v = lane; v < D / 8; v += 32) {
-        const uint4 q = *reinterpret_cast<const uint4*>(xr + v * 8);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float a = bf16_lo(w[i]) - x0, b = bf16_hi(w[i]) - x0;
-            s1 += a + b;
-            s2 = fmaf(a, a, fmaf(b, b, s2));
-        }
-    }
-    s1 = warp_sum_bwd(s1);
-    s2 = warp_sum_bwd(s2);
-    if (lane == 0) {
-        const float m1 = s1 / D;
-        const float var = fmaxf(s2 / D - m1 * m1, 0.f);
-        stats[row] = make_float2(x0 + m1, rsqrtf(var + eps));
-    }
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %2, 0;\n\tbarrier.cta.red.or.pred q, 1, %1, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"(n), "r"(static_cast<uint32_t>(v)) : "memory");
+    return r != 0;
 }
 
-struct TileArgs {
+__device__ __forceinline__ float tanh_hw(float h)
+{
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return t;
+}
+
+// Sums over the 32 lanes of a warp of each of v[0..15], by halving: at each
+// step a lane keeps one half of its values and adds the partner lane's copy
+// of that half.  Lanes 2k and 2k+1 end with the total of value k (bits 4..1
+// of the lane number are the value index).
+__device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane)
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const bool up = lane & 16;
+        const float send = up ? v[i] : v[i + 8], keep = up ? v[i + 8] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool up = lane & 8;
+        const float send = up ? v[i] : v[i + 4], keep = up ? v[i + 4] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool up = lane & 4;
+        const float send = up ? v[i] : v[i + 2], keep = up ? v[i + 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+    {
+        const bool up = lane & 2;
+        const float send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
+struct BwdArgs {
     const __nv_bfloat16* x;
     const __nv_bfloat16* dy;
     const float* gamma;
@@ -81,217 +130,479 @@ struct TileArgs {
     const float* w;
     const float* bias;
     const float* cs_in;
-    const float2* stats;       // [B*T] (LayerNorm only)
-    float2* psum;              // [B*T][CB] per-row sums of g and g xhat over a tile's channels
-    float* part;               // [B * nrb][7][D]
-    float* dcs;
     __nv_bfloat16* dx;
-    int T, D, CB, nrb, apply_ln;
+    float* part;       // [B * nx][7][D]
+    float* dcs;        // [B][3][D] or null
+    int T, D, nx, rps, upc, apply_ln;
+    float eps;
+    WaitCtl ctl;
 };
 
-// FINISH = false: sums (and dx without LayerNorm); FINISH = true: dx.
-template <bool FINISH>
-__global__ void __launch_bounds__(kTileThreads) conv_bwd_tile_kernel(const TileArgs a)
+// Shared-memory map (bytes), the same in every CTA of the cluster.
+struct BwdSmem {
+    uint32_t segb, ring, fin, red, xbuf, st, tot, bars, total;
+    __host__ __device__ BwdSmem(int upc, int nwork)
+    {
+        segb = 16u * upc;                                  // one row of a CTA's channels
+        ring = 0;
+        fin = ring + kRing * 2 * kG * segb;                // [2][kG][nwork][8] fp32: g, xhat
+        red = fin + 2 * kG * nwork * 32;                   // [warps][16]
+        xbuf = red + (nwork / 32) * 64;                    // [kXch][CL max 4][kMsg]
+        st = xbuf + kXch * 4 * kMsg * 4;                   // [kStRing] (mean, rstd)
+        tot = st + kStRing * 8;                            // [kG] (mean g, mean g xhat)
+        bars = tot + kG * 8;                               // full[kRing], free[kRing], xbar[kXch]
+        total = bars + (2 * kRing + kXch) * 8;
+    }
+};
+
+template <bool AFF, int CL, int MAXT>
+__global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_constant__ BwdArgs a)
 {
-    __shared__ float2 rowsum[kRows][kTileThreads / 32];
-    __shared__ float2 total[kRows];
-    __shared__ float2 st_s[kRows + 6];     // LayerNorm statistics of rows t0-3 .. t1+2
-    const int rb = blockIdx.x, b = blockIdx.y, cb = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = cb * kTileCh + 2 * tid;
-    const bool live = c < a.D;
-    const int T = a.T, D = a.D;
-    const int t0 = rb * kRows, t1 = min(T, t0 + kRows);
-    const int64_t row0 = static_cast<int64_t>(b) * T;
+    static_assert(CL >= 2 && CL <= 4, "the rows' channels are split over 2 to 4 CTAs");
+    static_assert(kMsg == 16 + 2 * kG, "a message: 16 sums, then 2 kG first elements");
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nwork = blockDim.x - 32, nwarps = nwork >> 5;
+    const BwdSmem L(a.upc, nwork);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
+    uint64_t* freeb = full + kRing;
+    uint64_t* xbar = freeb + kRing;
+    float* red = reinterpret_cast<float*>(smem + L.red);
+    float* xbuf = reinterpret_cast<float*>(smem + L.xbuf);
+    float2* st_ring = reinterpret_cast<float2*>(smem + L.st);
+    float2* tot = reinterpret_cast<float2*>(smem + L.tot);
+    const WaitCtl ctl = a.ctl;
+
+    const int T = a.T, D = a.D, P = D / 8;
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int ubase = (rank * P) / CL, nu = ((rank + 1) * P) / CL - ubase;
+    const int slice = blockIdx.x / CL, b = blockIdx.y;
+    const int t_b = slice * a.rps, t_e = min(T, t_b + a.rps);
+    const int p_s = t_b - 3;                                   // stream rows p_s .. t_e + 2
+    const int S = (t_e - t_b + 6 + kG - 1) / kG;
+    const int p_load = min(T, t_e + 3);                        // rows [max(0, p_s), p_load) are loaded
     const bool ln = a.apply_ln != 0;
+    const int64_t row0 = static_cast<int64_t>(b) * T;
 
-    for (int i = tid; i < t1 - t0 + 6; i += kTileThreads) {
-        const int r = t0 - 3 + i;
-        st_s[i] = (ln && r >= 0 && r < T) ? a.stats[row0 + r] : make_float2(0.f, 1.f);
+    if (tid == 0) {
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(full + i, 1);
+            mbar_init(freeb + i, nwork);
+        }
+        for (int i = 0; i < kXch; ++i) mbar_init(xbar + i, 1);
+        mbar_init_fence();
     }
-    if (FINISH) {
-        // row totals of the tile's rows: the per-channel-block sums, in order
-        for (int i = tid; i < t1 - t0; i += kTileThreads) {
-            float sg = 0.f, sgh = 0.f;
-            for (int k = 0; k < a.CB; ++k) {
-                const float2 v = a.psum[(row0 + t0 + i) * a.CB + k];
-                sg += v.x;
-                sgh += v.y;
-            }
-            total[i] = make_float2(sg, sgh);
-        }
-    }
-    __syncthreads();
+    // every CTA's barriers exist before any CTA of the cluster sends to them
+    cluster_sync_all();
 
-    float wv[2][4], gm[2], bt[2], bi[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-        const float4 q = live ? *reinterpret_cast<const float4*>(a.w + static_cast<int64_t>(c + e) * 4)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-        wv[e][0] = q.x;
-        wv[e][1] = q.y;
-        wv[e][2] = q.z;
-        wv[e][3] = q.w;
-        gm[e] = (live && a.gamma) ? a.gamma[c + e] : 1.f;
-        bt[e] = (live && a.beta) ? a.beta[c + e] : 0.f;
-        bi[e] = (live && a.bias) ? a.bias[c + e] : 0.f;
-    }
-    float pdw[4][2] = {}, pdb[2] = {}, pdg[2] = {}, pdbe[2] = {};
-    // windows over rows p-3 .. p (index 3 = row p)
-    float xn[4][2] = {}, xh[4][2] = {}, du[4][2] = {}, rs[4] = {1.f, 1.f, 1.f, 1.f};
+    auto ring_x = [&](int stage, int g) { return smem + L.ring + ((stage % kRing) * 2 * kG + g) * L.segb; };
+    auto ring_dy = [&](int stage, int g) { return smem + L.ring + ((stage % kRing) * 2 * kG + kG + g) * L.segb; };
 
-    // x and dy of a row (this thread's two channels), loaded a whole group of
-    // kGroup rows ahead of their use: kGroup rows of loads stay in flight
-    constexpr int kGroup = 4;
-    auto fetch = [&](int r) {
-        uint2 v = make_uint2(0u, 0u);
-        if (live && r >= 0 && r < T) {
-            v.x = *reinterpret_cast<const uint32_t*>(a.x + (row0 + r) * D + c);
-            if (r >= t0) v.y = *reinterpret_cast<const uint32_t*>(a.dy + (row0 + r) * D + c);
-        }
-        return v;
-    };
-    uint2 cur[kGroup], nxt[kGroup];
+    if (warp == nwarps) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            const uint32_t nbytes = 16u * nu;
+            int armed[kRing] = {};
+            for (int s = 0; s < S; ++s) {
+                const int slot = s % kRing;
+                if (s >= kRing && !mbar_wait(freeb + slot, ((s - kRing) / kRing) & 1, ctl)) break;
+                uint32_t bytes = 0;
 #pragma unroll
-    for (int i = 0; i < kGroup; ++i) cur[i] = fetch(t0 - 3 + i);
-
-    auto row = [&](int p, const uint2 f0) {
-        const float2 st = st_s[p - (t0 - 3)];
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-            rs[j] = rs[j + 1];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                xn[j][e] = xn[j + 1][e];
-                xh[j][e] = xh[j + 1][e];
-                du[j][e] = du[j + 1][e];
-            }
-        }
-        // (1) conv input of row p
-        if (p < 0) {
-            const bool hv = live && a.cs_in;
-            const float* src = a.cs_in + (static_cast<int64_t>(b) * 3 + p + 3) * D + c;
-            xn[3][0] = hv ? src[0] : 0.f;
-            xn[3][1] = hv ? src[1] : 0.f;
-            xh[3][0] = xh[3][1] = 0.f;
-            rs[3] = 1.f;
-        } else if (p < T) {
-            const float v0 = bf16_lo(f0.x), v1 = bf16_hi(f0.x);
-            if (ln) {
-                xh[3][0] = (v0 - st.x) * st.y;
-                xh[3][1] = (v1 - st.x) * st.y;
-                xn[3][0] = fmaf(xh[3][0], gm[0], bt[0]);
-                xn[3][1] = fmaf(xh[3][1], gm[1], bt[1]);
-                rs[3] = st.y;
-            } else {
-                xh[3][0] = xn[3][0] = v0;
-                xh[3][1] = xn[3][1] = v1;
-                rs[3] = 1.f;
-            }
-        } else {
-            xn[3][0] = xn[3][1] = xh[3][0] = xh[3][1] = 0.f;
-            rs[3] = 1.f;
-        }
-        // (2) du of row p (rows t0 .. T-1; zero elsewhere)
-        if (p >= t0 && p < T) {
-            const float dyv[2] = {bf16_lo(f0.y), bf16_hi(f0.y)};
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float u = bi[e];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) u = fmaf(wv[e][j], xn[j][e], u);
-                // sigmoid with the fast exponential and division intrinsics:
-                // about 2 ulp, far below the bf16 rounding of dx
-                const float sg = __fdividef(1.f, 1.f + __expf(-u));
-                du[3][e] = dyv[e] * sg * fmaf(u, 1.f - sg, 1.f);
-            }
-            if (!FINISH && p < t1) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    pdb[e] += du[3][e];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) pdw[j][e] = fmaf(du[3][e], xn[j][e], pdw[j][e]);
+                for (int g = 0; g < kG; ++g) {
+                    const int p = p_s + s * kG + g;
+                    if (nu > 0 && p >= 0 && p < p_load) bytes += (p >= t_b ? 2 : 1) * nbytes;
                 }
-            }
-        } else {
-            du[3][0] = du[3][1] = 0.f;
-        }
-        // (3) dxn of row q = p - 3, then its LayerNorm backward
-        const int q = p - 3;
-        const bool out_row = q >= t0 && q < t1;
-        const bool hist_row = t0 == 0 && q < 0 && q >= -3;   // rows -3 .. -1: the history
-        if (out_row || hist_row) {
-            float dxn[2];
+                if (bytes == 0) {
+                    mbar_arrive(full + slot);
+                } else {
+                    mbar_arrive_expect_tx(full + slot, bytes);
 #pragma unroll
-            for (int e = 0; e < 2; ++e)
-                dxn[e] = wv[e][3] * du[0][e] + wv[e][2] * du[1][e] + wv[e][1] * du[2][e] + wv[e][0] * du[3][e];
-            if (hist_row) {
-                if (!FINISH && live && a.dcs) {
-                    float* dst = a.dcs + (static_cast<int64_t>(b) * 3 + q + 3) * D + c;
-                    dst[0] = dxn[0];
-                    dst[1] = dxn[1];
-                }
-            } else if (ln) {
-                const float g0 = dxn[0] * gm[0], g1 = dxn[1] * gm[1];
-                if (!FINISH) {
-                    const float sgv = warp_sum_bwd(g0 + g1);
-                    const float sghv = warp_sum_bwd(fmaf(g0, xh[0][0], g1 * xh[0][1]));
-                    if (lane == 0) rowsum[q - t0][warp] = make_float2(sgv, sghv);
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        pdg[e] = fmaf(dxn[e], xh[0][e], pdg[e]);
-                        pdbe[e] += dxn[e];
+                    for (int g = 0; g < kG; ++g) {
+                        const int p = p_s + s * kG + g;
+                        if (nu > 0 && p >= 0 && p < p_load) {
+                            const int64_t off = (row0 + p) * D + 8 * ubase;
+                            bulk_load_bwd(ring_x(s, g), a.x + off, nbytes, full + slot);
+                            if (p >= t_b) bulk_load_bwd(ring_dy(s, g), a.dy + off, nbytes, full + slot);
+                        }
                     }
-                } else if (live) {
-                    const float2 tt = total[q - t0];
-                    const float mg = tt.x / D, mgh = tt.y / D;
-                    const float o0 = rs[0] * (g0 - mg - xh[0][0] * mgh);
-                    const float o1 = rs[0] * (g1 - mg - xh[0][1] * mgh);
-                    *reinterpret_cast<uint32_t*>(a.dx + (row0 + q) * D + c) = pack_bf16(o0, o1);
                 }
-            } else if (!FINISH && live) {
-                *reinterpret_cast<uint32_t*>(a.dx + (row0 + q) * D + c) = pack_bf16(dxn[0], dxn[1]);
+                ++armed[slot];
+            }
+            for (int i = 0; i < kRing; ++i)
+                if (armed[i]) mbar_wait(full + i, (armed[i] - 1) & 1, ctl);
+        }
+    } else {
+        // ------------------------------------------------------------- workers
+        const int u = tid >> 1, half = tid & 1;
+        const bool active = u < nu;
+        const int c = 8 * (ubase + u) + 4 * half;                // this thread's channels c .. c+3
+        const uint32_t seg_off = 16u * u + 8u * half;            // their bytes in a ring row
+
+        f2 wr[2][kW], ga[AFF ? 2 : 1], be[AFF ? 2 : 1], bi[AFF ? 2 : 1];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int ch = active ? c + 2 * i : 0;
+#pragma unroll
+            for (int j = 0; j < kW; ++j)
+                wr[i][j] = active ? f2_make(0.5f * a.w[ch * kW + j], 0.5f * a.w[(ch + 1) * kW + j]) : f2_splat(0.f);
+            if constexpr (AFF) {
+                ga[i] = (a.gamma && active) ? f2_make(a.gamma[ch], a.gamma[ch + 1]) : f2_splat(1.f);
+                be[i] = (a.beta && active) ? f2_make(a.beta[ch], a.beta[ch + 1]) : f2_splat(0.f);
+                bi[i] = (a.bias && active) ? f2_make(0.5f * a.bias[ch], 0.5f * a.bias[ch + 1]) : f2_splat(0.f);
             }
         }
-    };
+        const f2 zero = f2_splat(0.f), one = f2_splat(1.f);
+        f2 wxn[3][2], wxh[3][2], wdu[3][2];     // windows: rows p-3, p-2, p-1
+        f2 dw[kW][2], db[2], dg[2], dbe[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+#pragma unroll
+            for (int r = 0; r < 3; ++r) wxn[r][i] = wxh[r][i] = wdu[r][i] = zero;
+#pragma unroll
+            for (int j = 0; j < kW; ++j) dw[j][i] = zero;
+            db[i] = dg[i] = dbe[i] = zero;
+        }
+        float gs[2 * kG] = {};                   // this thread's g and g xhat sums of the stage's output rows
+        const float invD = 1.0f / static_cast<float>(D);
+        float* fin = reinterpret_cast<float*>(smem + L.fin);
+        auto fin_at = [&](int par, int g) { return fin + ((par * kG + g) * nwork + tid) * 8; };
 
-    for (int p0 = t0 - 3; p0 <= t1 + 2; p0 += kGroup) {
+        // moments of this CTA's channels of stream row p about the row's
+        // first element here: (sum d, sum d^2) for this thread's channels
+        auto moments = [&](int stage, int g, int p, float& m1, float& m2) {
+            m1 = m2 = 0.f;
+            if (active && p >= 0 && p < p_load) {
+                const uint8_t* row = ring_x(stage, g);
+                const f2 x0 = f2_splat(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(row)));
+                const uint2 xv = *reinterpret_cast<const uint2*>(row + seg_off);
+                const f2 d0 = f2_sub(f2_from_bf16x2(xv.x), x0), d1 = f2_sub(f2_from_bf16x2(xv.y), x0);
+                const float2 s1 = f2_get(f2_add(d0, d1)), s2 = f2_get(f2_fma(d1, d1, f2_mul(d0, d0)));
+                m1 = s1.x + s1.y;
+                m2 = s2.x + s2.y;
+            }
+        };
+        // the row's first element of this CTA's channels (0 without channels)
+        auto first_x = [&](int stage, int g, int p) {
+            return (nu > 0 && p >= 0 && p < p_load)
+                       ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ring_x(stage, g)))
+                       : 0.f;
+        };
+        auto xch_addr = [&](int e, int from, int k) { return xbuf + ((e % kXch) * 4 + from) * kMsg + k; };
+        // value k of this CTA's message e, into every CTA of the cluster
+        auto push = [&](int e, int k, float val) {
+            const uint32_t la = smem_u32(xch_addr(e, rank, k)), lb = smem_u32(xbar + e % kXch);
 #pragma unroll
-        for (int i = 0; i < kGroup; ++i) nxt[i] = fetch(p0 + kGroup + i);
-#pragma unroll
-        for (int i = 0; i < kGroup; ++i)
-            if (p0 + i <= t1 + 2) row(p0 + i, cur[i]);
-#pragma unroll
-        for (int i = 0; i < kGroup; ++i) cur[i] = nxt[i];
-    }
+            for (int r = 0; r < CL; ++r) st_async_f32(mapa_shared(la, r), val, mapa_shared(lb, r));
+        };
+        // LayerNorm statistics of a row from the CTAs' shifted sums
+        auto combine_stats = [&](int e, int i_s1, int i_s2, int i_x0) {
+            const float A = *xch_addr(e, 0, i_x0);
+            float S1 = 0.f, S2 = 0.f;
+            for (int r = 0; r < CL; ++r) {
+                const float n = static_cast<float>(8 * (((r + 1) * P) / CL - (r * P) / CL));
+                const float s1 = *xch_addr(e, r, i_s1), s2 = *xch_addr(e, r, i_s2);
+                const float dlt = *xch_addr(e, r, i_x0) - A;
+                S1 += fmaf(n, dlt, s1);
+                S2 += fmaf(n * dlt, dlt, fmaf(2.f * dlt, s1, s2));
+            }
+            const float m1 = S1 * invD;
+            const float var = fmaxf(S2 * invD - m1 * m1, 0.f);
+            return make_float2(A + m1, 1.0f / sqrtf(var + a.eps));
+        };
+        // exchange e: armed once by this CTA for the bytes of all CL messages
+        auto arm = [&](int e) {
+            if (tid == 0) mbar_arrive_expect_tx(xbar + e % kXch, CL * kMsg * 4);
+        };
+        auto wait_x = [&](int e) { return mbar_wait_cluster(xbar + e % kXch, (e / kXch) & 1, ctl); };
 
-    if (!FINISH) {
-        // per-row sums over this tile's channels, in warp order
+        bool failed = false;
+
+        // one stream row: xn, xhat, du (when p is a du row of this range),
+        // the sums, and for q = p - 3 its dxn (g and xhat to fin, or dx).
+        // INNER: a row with 0 <= p - 3, t_b <= p - 3 and p < min(T, t_e), so
+        // that no range check is needed.
+        auto do_row = [&](auto inner_tag, int stage, int g, int p) {
+            constexpr bool INNER = decltype(inner_tag)::value;
+            f2 xn[2], xh[2], du[2];
+            if (!INNER && p < 0) {
+                const bool hv = active && a.cs_in;
+                const float* src = a.cs_in + (static_cast<int64_t>(b) * 3 + p + 3) * D + c;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    xn[i] = hv ? f2_make(src[2 * i], src[2 * i + 1]) : zero;
+                    xh[i] = zero;
+                }
+            } else if ((INNER || p < T) && active) {
+                const uint2 xv = *reinterpret_cast<const uint2*>(ring_x(stage, g) + seg_off);
+                xn[0] = f2_from_bf16x2(xv.x);
+                xn[1] = f2_from_bf16x2(xv.y);
+                if (ln) {
+                    const float2 m = st_ring[(p - p_s) & (kStRing - 1)];
+                    if constexpr (AFF) {
+                        const f2 mu = f2_splat(m.x), rs = f2_splat(m.y);
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            xh[i] = f2_mul(f2_sub(xn[i], mu), rs);
+                            xn[i] = f2_fma(xh[i], ga[i], be[i]);
+                        }
+                    } else {
+                        const f2 rs = f2_splat(m.y), sh = f2_splat(-m.x * m.y);
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) xh[i] = xn[i] = f2_fma(xn[i], rs, sh);
+                    }
+                } else {
+                    xh[0] = xn[0];
+                    xh[1] = xn[1];
+                }
+            } else {
+                xn[0] = xn[1] = xh[0] = xh[1] = zero;
+            }
+            if ((INNER || (p >= t_b && p < T)) && active) {
+                const uint2 dv = *reinterpret_cast<const uint2*>(ring_dy(stage, g) + seg_off);
+                const f2 dyv[2] = {f2_from_bf16x2(dv.x), f2_from_bf16x2(dv.y)};
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    f2 acc = AFF ? bi[AFF ? i : 0] : zero;
+#pragma unroll
+                    for (int j = 0; j < kW - 1; ++j) acc = f2_fma(wr[i][j], wxn[j][i], acc);
+                    const f2 h = f2_fma(wr[i][kW - 1], xn[i], acc);
+                    const float2 hh = f2_get(h);
+                    const f2 t = f2_make(tanh_hw(hh.x), tanh_hw(hh.y));
+                    // du2 = 2 du = dy (1 + t) (1 + h (1 - t))
+                    du[i] = f2_mul(f2_mul(dyv[i], f2_add(one, t)), f2_fma(h, f2_sub(one, t), one));
+                }
+                if (INNER || p < t_e) {
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+#pragma unroll
+                        for (int j = 0; j < kW - 1; ++j) dw[j][i] = f2_fma(du[i], wxn[j][i], dw[j][i]);
+                        dw[kW - 1][i] = f2_fma(du[i], xn[i], dw[kW - 1][i]);
+                        db[i] = f2_add(db[i], du[i]);
+                    }
+                }
+            } else {
+                du[0] = du[1] = zero;
+            }
+            const int q = p - 3;
+            const bool out = INNER || (q >= t_b && q < t_e);
+            const bool hist = !INNER && t_b == 0 && q < 0 && q >= -3 && a.dcs;
+            if (out || hist) {
+                f2 dxn[2];
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    dxn[i] = f2_fma(wr[i][0], du[i],
+                                    f2_fma(wr[i][1], wdu[2][i], f2_fma(wr[i][2], wdu[1][i], f2_mul(wr[i][3], wdu[0][i]))));
+                if (hist) {
+                    if (active) {
+                        float* dst = a.dcs + (static_cast<int64_t>(b) * 3 + q + 3) * D + c;
+                        const float2 v0 = f2_get(dxn[0]), v1 = f2_get(dxn[1]);
+                        *reinterpret_cast<float4*>(dst) = make_float4(v0.x, v0.y, v1.x, v1.y);
+                    }
+                } else if (ln) {
+                    f2 gg[2];
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        gg[i] = AFF ? f2_mul(dxn[i], ga[AFF ? i : 0]) : dxn[i];
+                        dg[i] = f2_fma(dxn[i], wxh[0][i], dg[i]);
+                        dbe[i] = f2_add(dbe[i], dxn[i]);
+                    }
+                    const float2 s1 = f2_get(f2_add(gg[0], gg[1]));
+                    const float2 s2 = f2_get(f2_fma(gg[1], wxh[0][1], f2_mul(gg[0], wxh[0][0])));
+                    gs[g] += s1.x + s1.y;
+                    gs[kG + g] += s2.x + s2.y;
+                    float* fp = fin_at(stage & 1, g);
+                    const float2 a0 = f2_get(gg[0]), a1 = f2_get(gg[1]);
+                    const float2 h0 = f2_get(wxh[0][0]), h1 = f2_get(wxh[0][1]);
+                    *reinterpret_cast<float4*>(fp) = make_float4(a0.x, a0.y, a1.x, a1.y);
+                    *reinterpret_cast<float4*>(fp + 4) = make_float4(h0.x, h0.y, h1.x, h1.y);
+                } else if (active) {
+                    *reinterpret_cast<uint2*>(a.dx + (row0 + q) * D + c) =
+                        make_uint2(f2_to_bf16x2(dxn[0]), f2_to_bf16x2(dxn[1]));
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                wxn[0][i] = wxn[1][i];
+                wxn[1][i] = wxn[2][i];
+                wxn[2][i] = xn[i];
+                wxh[0][i] = wxh[1][i];
+                wxh[1][i] = wxh[2][i];
+                wxh[2][i] = xh[i];
+                wdu[0][i] = wdu[1][i];
+                wdu[1][i] = wdu[2][i];
+                wdu[2][i] = du[i];
+            }
+        };
+
+        // dx of the output rows of stage s (their g, xhat in fin)
+        auto finish = [&](int s) {
+#pragma unroll
+            for (int g = 0; g < kG; ++g) {
+                const int q = p_s + s * kG + g - 3;
+                if (q >= t_b && q < t_e && active) {
+                    const float rstd = st_ring[(q - p_s) & (kStRing - 1)].y;
+                    const float2 mt = tot[g];
+                    const f2 rs = f2_splat(rstd), na = f2_splat(-rstd * mt.x), nb = f2_splat(-rstd * mt.y);
+                    const float* fp = fin_at(s & 1, g);
+                    const float4 g4 = *reinterpret_cast<const float4*>(fp);
+                    const float4 h4 = *reinterpret_cast<const float4*>(fp + 4);
+                    const f2 o0 = f2_fma(f2_make(h4.x, h4.y), nb, f2_fma(f2_make(g4.x, g4.y), rs, na));
+                    const f2 o1 = f2_fma(f2_make(h4.z, h4.w), nb, f2_fma(f2_make(g4.z, g4.w), rs, na));
+                    *reinterpret_cast<uint2*>(a.dx + (row0 + q) * D + c) = make_uint2(f2_to_bf16x2(o0), f2_to_bf16x2(o1));
+                }
+            }
+        };
+
+        // ---- prologue: statistics of the rows of stages 0 and 1
         if (ln) {
-            __syncthreads();
-            for (int i = tid; i < t1 - t0; i += kTileThreads) {
-                float sg = 0.f, sgh = 0.f;
+            if (!mbar_wait(full + 0, 0, ctl)) failed = true;
+            if (S > 1 && !failed && !mbar_wait(full + 1, 0, ctl)) failed = true;
+            float v[16];
 #pragma unroll
-                for (int k = 0; k < kTileThreads / 32; ++k) {
-                    sg += rowsum[i][k].x;
-                    sgh += rowsum[i][k].y;
-                }
-                a.psum[(row0 + t0 + i) * a.CB + cb] = make_float2(sg, sgh);
+            for (int i = 0; i < 2 * kG; ++i) {
+                const int p = p_s + i;
+                if (!failed) moments(i / kG, i % kG, p, v[i], v[2 * kG + i]);
+                else v[i] = v[2 * kG + i] = 0.f;
             }
+            const float r = warp_reduce16(v, lane);
+            if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = r;
+            if (!workers_or_bwd(failed, nwork)) {
+                arm(0);
+                if (tid < 16) {
+                    float t = 0.f;
+                    for (int w = 0; w < nwarps; ++w) t += red[w * 16 + tid];
+                    push(0, tid, t);
+                } else if (tid < kMsg) {
+                    const int i = tid - 16;
+                    push(0, tid, first_x(i / kG, i % kG, p_s + i));
+                }
+                if (warp == 0) {
+                    if (!wait_x(0)) failed = true;
+                    if (!failed && lane < 2 * kG) st_ring[lane] = combine_stats(0, lane, 2 * kG + lane, 16 + lane);
+                }
+            } else {
+                failed = true;
+            }
+            if (workers_or_bwd(failed, nwork)) failed = true;
         }
-        // per-tile partials: dw taps 0..3, dbias, dgamma, dbeta
-        if (live) {
-            float* pp = a.part + (static_cast<int64_t>(b) * a.nrb + rb) * kParts * D + c;
+
+        // ---- the stages (every exit from the loop follows a barrier, so
+        // that all workers leave together)
+        for (int s = 0; s < S && !failed; ++s) {
+            const int slot = s % kRing;
+            bool ok = mbar_wait(full + slot, (s / kRing) & 1, ctl);
+            if (ln && ok && s + 2 < S) ok = mbar_wait(full + (s + 2) % kRing, ((s + 2) / kRing) & 1, ctl);
+            if (!ok) failed = true;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) *reinterpret_cast<float2*>(pp + j * D) = make_float2(pdw[j][0], pdw[j][1]);
-            *reinterpret_cast<float2*>(pp + 4 * D) = make_float2(pdb[0], pdb[1]);
-            *reinterpret_cast<float2*>(pp + 5 * D) = make_float2(pdg[0], pdg[1]);
-            *reinterpret_cast<float2*>(pp + 6 * D) = make_float2(pdbe[0], pdbe[1]);
+            for (int i = 0; i < 2 * kG; ++i) gs[i] = 0.f;
+            const int pos0 = p_s + s * kG;
+            if (!failed) {
+                if (pos0 >= t_b + 3 && pos0 + kG <= min(T, t_e)) {
+#pragma unroll
+                    for (int g = 0; g < kG; ++g) do_row(std::true_type{}, s, g, pos0 + g);
+                } else {
+#pragma unroll
+                    for (int g = 0; g < kG; ++g)
+                        if (pos0 + g <= t_e + 2) do_row(std::false_type{}, s, g, pos0 + g);
+                }
+            }
+            mbar_arrive(freeb + slot);          // this worker is done with the stage's rows
+            if (!ln) {
+                if (workers_or_bwd(failed, nwork)) {
+                    failed = true;
+                    break;
+                }
+                continue;
+            }
+
+            // moments of the rows two stages ahead, the g sums of this stage
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 2 * kG; ++i) v[i] = gs[i];
+#pragma unroll
+            for (int g = 0; g < kG; ++g) {
+                if (!failed && s + 2 < S) moments(s + 2, g, pos0 + 2 * kG + g, v[2 * kG + g], v[3 * kG + g]);
+                else v[2 * kG + g] = v[3 * kG + g] = 0.f;
+            }
+            const float r = warp_reduce16(v, lane);
+            if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = r;
+            if (workers_or_bwd(failed, nwork)) {
+                failed = true;
+                break;
+            }
+            arm(s + 1);
+            if (tid < 16) {
+                float t = 0.f;
+                for (int w = 0; w < nwarps; ++w) t += red[w * 16 + tid];
+                push(s + 1, tid, t);
+            } else if (tid < kMsg) {
+                // every message is kMsg values (the arm counts them): the
+                // first elements of the rows two stages ahead, then zeros
+                const int g = tid - 16;
+                push(s + 1, tid, (g < kG && s + 2 < S) ? first_x(s + 2, g, pos0 + 2 * kG + g) : 0.f);
+            }
+            if (s >= 1 && warp == 0) {
+                // exchange s: the g sums of stage s-1's output rows and the
+                // statistics of stage s+1's rows
+                if (!wait_x(s)) failed = true;
+                if (!failed) {
+                    if (lane < kG) {
+                        float sg = 0.f, sgx = 0.f;
+                        for (int r2 = 0; r2 < CL; ++r2) {
+                            sg += *xch_addr(s, r2, lane);
+                            sgx += *xch_addr(s, r2, kG + lane);
+                        }
+                        tot[lane] = make_float2(sg * invD, sgx * invD);
+                    } else if (lane < 2 * kG) {
+                        const int g = lane - kG;
+                        st_ring[(pos0 + kG + g - p_s) & (kStRing - 1)] =
+                            combine_stats(s, 2 * kG + g, 3 * kG + g, 16 + g);
+                    }
+                }
+            }
+            if (workers_or_bwd(failed, nwork)) {
+                failed = true;
+                break;
+            }
+            if (s >= 1) finish(s - 1);
+        }
+        // the last stage's output rows
+        if (ln && !failed && S > 0) {
+            if (warp == 0) {
+                if (!wait_x(S)) failed = true;
+                if (!failed && lane < kG) {
+                    float sg = 0.f, sgx = 0.f;
+                    for (int r2 = 0; r2 < CL; ++r2) {
+                        sg += *xch_addr(S, r2, lane);
+                        sgx += *xch_addr(S, r2, kG + lane);
+                    }
+                    tot[lane] = make_float2(sg * invD, sgx * invD);
+                }
+            }
+            if (!workers_or_bwd(failed, nwork)) finish(S - 1);
+            else failed = true;
+        }
+
+        // per-(range, CTA) partial sums
+        if (!failed && active) {
+            float* pp = a.part + (static_cast<int64_t>(b) * a.nx + slice) * kParts * D + c;
+            auto put = [&](int k, const f2 (&v)[2]) {
+                const float2 v0 = f2_get(v[0]), v1 = f2_get(v[1]);
+                *reinterpret_cast<float4*>(pp + k * D) = make_float4(v0.x, v0.y, v1.x, v1.y);
+            };
+#pragma unroll
+            for (int j = 0; j < kW; ++j) put(j, dw[j]);
+            put(4, db);
+            put(5, dg);
+            put(6, dbe);
         }
     }
+    // no CTA leaves while another may still write into its shared memory
+    cluster_sync_all();
 }
 
-// Sum of the per-CTA partials in CTA order: thread per (part, channel).
+// Sum of the per-range partials in range order: thread per (part, channel).
+// dw and dbias were summed from 2 du.
 __global__ void __launch_bounds__(256) conv_bwd_reduce_kernel(const float* __restrict__ part, int nparts, int D,
                                                               float* __restrict__ dw, float* __restrict__ dbias,
                                                               float* __restrict__ dgamma, float* __restrict__ dbeta)
@@ -302,9 +613,9 @@ __global__ void __launch_bounds__(256) conv_bwd_reduce_kernel(const float* __res
     float s = 0.f;
     for (int n = 0; n < nparts; ++n) s += part[static_cast<int64_t>(n) * kParts * D + i];
     if (k < 4)
-        dw[static_cast<int64_t>(ch) * 4 + k] = s;
+        dw[static_cast<int64_t>(ch) * 4 + k] = 0.5f * s;
     else if (k == 4) {
-        if (dbias) dbias[ch] = s;
+        if (dbias) dbias[ch] = 0.5f * s;
     } else if (k == 5) {
         if (dgamma) dgamma[ch] = s;
     } else if (dbeta) {
@@ -312,25 +623,86 @@ __global__ void __launch_bounds__(256) conv_bwd_reduce_kernel(const float* __res
     }
 }
 
+// At most 256 workers a CTA (4 channels each) and one producer warp, so
+// that the per-channel registers fit without spilling.
+constexpr int kBwdThreads = 288;
+
+struct BwdPlan {
+    int CL, upc, threads, nx, rps;
+};
+
+// clusters: how many clusters of CL CTAs the device runs at once
+BwdPlan plan_bwd(int B, int T, int D, int clusters)
+{
+    BwdPlan pl;
+    const int P = D / 8;
+    pl.CL = D <= 2048 ? 2 : 4;
+    pl.upc = (P + pl.CL - 1) / pl.CL;
+    pl.threads = (2 * pl.upc + 31) / 32 * 32 + 32;
+    int nx = clusters / (B > 0 ? B : 1);
+    if (nx < 1) nx = 1;
+    if (nx > kMaxSlices) nx = kMaxSlices;
+    const int max_nx = (T + kMinRows - 1) / kMinRows;
+    if (nx > max_nx) nx = max_nx;
+    if (nx < 1) nx = 1;
+    pl.rps = (T + nx - 1) / nx;
+    pl.nx = (T + pl.rps - 1) / pl.rps;
+    return pl;
+}
+
 }  // namespace
 
-// part [B * nrb][7][D] | stats [B*T] float2 | psum [B*T][CB] float2
+// part [B * nx][7][D] with nx at most min(128, ceil(T / 64)) ranges a sequence
 size_t conv_bwd_workspace_bytes(int B, int T, int D)
 {
-    const size_t nrb = static_cast<size_t>((T + kRows - 1) / kRows), CB = (D + kTileCh - 1) / kTileCh;
-    const size_t rows = static_cast<size_t>(B) * T;
-    return align256(static_cast<size_t>(B) * nrb * kParts * D * sizeof(float)) + align256(rows * sizeof(float2)) +
-           align256(rows * CB * sizeof(float2));
+    const size_t nx_max = std::min<size_t>(kMaxSlices, (static_cast<size_t>(T) + kMinRows - 1) / kMinRows);
+    return align256(static_cast<size_t>(B) * (nx_max > 0 ? nx_max : 1) * kParts * D * sizeof(float));
 }
 
 gla_status launch_conv_bwd(const void* x, int apply_ln, const float* g, const float* be, float eps, const float* w,
                            const float* bias, const float* cs_in, const void* dy, void* dx, float* dw, float* dbias,
                            float* dgamma, float* dbeta, float* dcs, void* ws, int B, int T, int D, cudaStream_t st)
 {
-    const int nrb = (T + kRows - 1) / kRows, CB = (D + kTileCh - 1) / kTileCh;
-    const size_t rows = static_cast<size_t>(B) * T;
-    uint8_t* wsb = static_cast<uint8_t*>(ws);
-    TileArgs a;
+    gla_status se;
+    const WaitCtl ctl = wait_ctl_for_current_device(&se);
+    if (se != GLA_OK) return se;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int CL = D <= 2048 ? 2 : 4;
+    const bool aff = g || be || bias;
+    void (*kernel)(BwdArgs);
+    if (CL == 2)
+        kernel = aff ? ln_conv_silu_bwd_kernel<true, 2, kBwdThreads> : ln_conv_silu_bwd_kernel<false, 2, kBwdThreads>;
+    else
+        kernel = aff ? ln_conv_silu_bwd_kernel<true, 4, kBwdThreads> : ln_conv_silu_bwd_kernel<false, 4, kBwdThreads>;
+    BwdPlan pl = plan_bwd(B, T, D, sms / CL);
+    const BwdSmem L(pl.upc, pl.threads - 32);
+    const size_t smem = L.total;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+        cudaSuccess)
+        return check_launch("cudaFuncSetAttribute");
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.blockDim = dim3(pl.threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    // as many token ranges as clusters run at once (a GPC may hold a
+    // number of SMs that is not a multiple of CL)
+    cfg.gridDim = dim3(pl.nx * CL, B);
+    int active = 0;
+    if (cudaOccupancyMaxActiveClusters(&active, kernel, &cfg) == cudaSuccess && active > 0)
+        pl = plan_bwd(B, T, D, active);
+    else
+        cudaGetLastError();
+    cfg.gridDim = dim3(pl.nx * CL, B);
+    BwdArgs a;
     a.x = static_cast<const __nv_bfloat16*>(x);
     a.dy = static_cast<const __nv_bfloat16*>(dy);
     a.gamma = g;
@@ -338,43 +710,26 @@ gla_status launch_conv_bwd(const void* x, int apply_ln, const float* g, const fl
     a.w = w;
     a.bias = bias;
     a.cs_in = cs_in;
-    a.part = reinterpret_cast<float*>(wsb);
-    size_t off = align256(static_cast<size_t>(B) * nrb * kParts * D * sizeof(float));
-    float2* stats = reinterpret_cast<float2*>(wsb + off);
-    off += align256(rows * sizeof(float2));
-    a.stats = stats;
-    a.psum = reinterpret_cast<float2*>(wsb + off);
-    a.dcs = dcs;
     a.dx = static_cast<__nv_bfloat16*>(dx);
+    a.part = static_cast<float*>(ws);
+    a.dcs = dcs;
     a.T = T;
     a.D = D;
-    a.CB = CB;
-    a.nrb = nrb;
+    a.nx = pl.nx;
+    a.rps = pl.rps;
+    a.upc = pl.upc;
     a.apply_ln = apply_ln;
-    gla_status s;
-    if (apply_ln) {
-        trace_begin(st);
-        ln_stats_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(a.x, static_cast<int>(rows), D, eps,
-                                                                              stats);
-        trace_end(st, "ln_stats_kernel");
-        count_launch();
-        if ((s = check_launch("ln_stats_kernel")) != GLA_OK) return s;
-    }
-    const dim3 grid(nrb, B, CB);
+    a.eps = eps;
+    a.ctl = ctl;
     trace_begin(st);
-    conv_bwd_tile_kernel<false><<<grid, kTileThreads, 0, st>>>(a);
-    trace_end(st, "conv_bwd_tile_kernel");
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, a);
+    trace_end(st, "ln_conv_silu_bwd_kernel");
     count_launch();
-    if ((s = check_launch("conv_bwd_tile_kernel")) != GLA_OK) return s;
-    if (apply_ln) {
-        trace_begin(st);
-        conv_bwd_tile_kernel<true><<<grid, kTileThreads, 0, st>>>(a);
-        trace_end(st, "conv_bwd_dx_kernel");
-        count_launch();
-        if ((s = check_launch("conv_bwd_dx_kernel")) != GLA_OK) return s;
-    }
+    if (e != cudaSuccess) return status_of(e);
+    gla_status s;
+    if ((s = check_launch("ln_conv_silu_bwd_kernel")) != GLA_OK) return s;
     trace_begin(st);
-    conv_bwd_reduce_kernel<<<(kParts * D + 255) / 256, 256, 0, st>>>(a.part, B * nrb, D, dw, dbias, dgamma, dbeta);
+    conv_bwd_reduce_kernel<<<(kParts * D + 255) / 256, 256, 0, st>>>(a.part, B * pl.nx, D, dw, dbias, dgamma, dbeta);
     trace_end(st, "conv_bwd_reduce_kernel");
     count_launch();
     return check_launch("conv_bwd_reduce_kernel");

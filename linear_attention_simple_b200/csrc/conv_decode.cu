@@ -15,15 +15,20 @@
 //   h[s]   <- (h[s,1], h[s,2], xn)                  (in place)
 //
 // HBM-bound: per sequence x and y (2 B per channel each) and the history
-// read and written (12 B each); the weights stay in L2 across sequences.
-// One CTA per sequence, thread i owns channels 8i .. 8i+7: one 16-byte
-// vector of x and y, two of each history row.  The history rows are loaded
-// with x, before the LayerNorm, so their latency overlaps the moments (the
-// weights and bias, L2-resident, come after); the two moments (sums of
-// (x - x0) and (x - x0)^2, shifted by the row's first element x0 as the
-// sequence front end does) come from one block reduction.
+// read and written (12 B each).  One CTA per SM walks the sequences
+// blockIdx.x, + gridDim.x, ...: a producer warp brings each sequence's
+// history rows and x row into a ring of shared-memory stages with bulk
+// asynchronous copies (cp.async.bulk, completion on the stage's mbarrier)
+// and refills a stage as soon as every worker has released it, so the loads
+// of the next sequences are in flight while the workers finish this one.
+// Worker thread i owns channels 8i .. 8i+7 and keeps their conv weights (and
+// LayerNorm affine and bias) in registers for the whole launch.  The two
+// moments (sums of (x - x0) and (x - x0)^2, shifted by the row's first
+// element x0 as the sequence front end does) come from one reduction over
+// the workers.  The outputs go out as streaming vector stores.
 // A slot outside [0, n_slots) is skipped (nothing read or written) and
-// GLA_ERR_INVALID_ARG is recorded in the device status word.
+// GLA_ERR_INVALID_ARG is recorded in the device status word.  Every wait is
+// bounded.
 #include <cuda_bf16.h>
 
 #include "gla_device.cuh"
@@ -32,7 +37,8 @@
 namespace gla {
 namespace {
 
-constexpr int kMaxThreads = 512;   // D <= 4096
+constexpr int kMaxStages = 4;
+constexpr int kCh = 8;
 
 __device__ __forceinline__ float warp_sum_dec(float v)
 {
@@ -41,29 +47,32 @@ __device__ __forceinline__ float warp_sum_dec(float v)
     return v;
 }
 
-// Sums of a and b over the block; every thread gets both.
-__device__ __forceinline__ float2 block_sum2(float a, float b, float2* red)
+__device__ __forceinline__ void bulk_load_dec(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
 {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = (blockDim.x + 31) >> 5;
-    a = warp_sum_dec(a);
-    b = warp_sum_dec(b);
-    if (lane == 0) red[warp] = make_float2(a, b);
-    __syncthreads();
-    float2 s = make_float2(0.f, 0.f);
-    for (int i = 0; i < nw; ++i) {
-        s.x += red[i].x;
-        s.y += red[i].y;
-    }
-    return s;
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
 }
 
-// SiLU(x) = x sigmoid(x) with sigmoid(x) = (1 + tanh(x / 2)) / 2 on the
-// hardware tanh approximation.
-__device__ __forceinline__ float silu_dec(float x)
+// Barrier over the n worker threads (named barrier 1) that also returns the
+// OR of v over them.
+__device__ __forceinline__ bool workers_or_dec(bool v, int n)
+{
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %2, 0;\n\tbarrier.cta.red.or.pred q, 1, %1, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r) : "r"(n), "r"(static_cast<uint32_t>(v)) : "memory");
+    return r != 0;
+}
+
+// SiLU(u) with h = u / 2 (the weights and bias are halved on load):
+// u sigmoid(u) = h (1 + tanh h), on the hardware tanh approximation.
+__device__ __forceinline__ float silu_of_half_dec(float h)
 {
     float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
-    return x * fmaf(0.5f, t, 0.5f);
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+    return fmaf(h, t, h);
 }
 
 __device__ __forceinline__ void load8(const float* p, float (&v)[8])
@@ -73,103 +82,222 @@ __device__ __forceinline__ void load8(const float* p, float (&v)[8])
     v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// At most 80 registers, so that two CTAs of 384 threads (D = 3,072) share
-// an SM.
-__global__ void __maxnreg__(80) conv_decode_kernel(
+// Stage layout: the slot's three history rows [3][D] fp32, then the x row
+// [D] bf16 (14 D bytes, a multiple of 16 since D % 8 == 0).  After the
+// stages: full[kMaxStages], free[kMaxStages] mbarriers, the slot of each
+// stage (-1: skipped), and the moments' partials [2][warps] by parity.
+// AFF: a LayerNorm affine or a conv bias is given (otherwise their
+// registers are not needed).
+template <bool AFF, int MAXT>
+__global__ void __launch_bounds__(MAXT, 1) conv_decode_kernel(
     const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ slot_idx, int apply_ln,
     const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
     const float* __restrict__ w, const float* __restrict__ bias, float* __restrict__ hist,
-    __nv_bfloat16* __restrict__ y, int D, int n_slots, int* __restrict__ status)
+    __nv_bfloat16* __restrict__ y, int N, int D, int n_slots, int stages, WaitCtl ctl)
 {
-    __shared__ float2 red[kMaxThreads / 32];
-    const int n = blockIdx.x, c0 = threadIdx.x * 8;
-    const int s = slot_idx ? slot_idx[n] : n;
-    if (s < 0 || s >= n_slots) {                // a slot outside the pool: touch nothing
-        if (threadIdx.x == 0) record_status(status, GLA_ERR_INVALID_ARG);
+    extern __shared__ __align__(16) uint8_t smem[];
+    const uint32_t hbytes = 12u * D, xbytes = 2u * D, stage_bytes = hbytes + xbytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(stages) * stage_bytes);
+    uint64_t* freeb = full + kMaxStages;
+    int* sslot = reinterpret_cast<int*>(freeb + kMaxStages);                 // [kMaxStages]
+    float2* red = reinterpret_cast<float2*>(sslot + kMaxStages);              // [2][MAXT / 32]
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nwork = blockDim.x - 32, nwarps = nwork >> 5;
+    const bool producer = warp == nwarps;
+    const int c0 = tid * kCh;
+    const bool active = !producer && c0 < D;
+    const int nseq = blockIdx.x < N ? (N - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < stages; ++i) {
+            mbar_init(full + i, 1);
+            mbar_init(freeb + i, nwork);
+        }
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    if (producer) {
+        // -------------------------------------------------------- producer
+        if (lane == 0) {
+            int armed[kMaxStages] = {0, 0, 0, 0};
+            for (int k = 0; k < nseq; ++k) {
+                const int st = k % stages;
+                // the stage's previous sequence has been released by every worker
+                if (k >= stages && !mbar_wait(freeb + st, ((k - stages) / stages) & 1, ctl)) break;
+                const int n = blockIdx.x + k * gridDim.x;
+                const int s = slot_idx ? slot_idx[n] : n;
+                const bool valid = s >= 0 && s < n_slots;
+                sslot[st] = valid ? s : -1;
+                uint8_t* base = smem + static_cast<size_t>(st) * stage_bytes;
+                if (valid) {
+                    mbar_arrive_expect_tx(full + st, stage_bytes);
+                    bulk_load_dec(base, hist + static_cast<int64_t>(s) * 3 * D, hbytes, full + st);
+                    bulk_load_dec(base + hbytes, x + static_cast<int64_t>(n) * D, xbytes, full + st);
+                } else {
+                    mbar_arrive(full + st);
+                }
+                ++armed[st];
+            }
+            // every copy in flight lands before the shared memory is released
+            for (int i = 0; i < stages; ++i)
+                if (armed[i]) mbar_wait(full + i, (armed[i] - 1) & 1, ctl);
+        }
         return;
     }
-    // the loads from HBM first: x and the three history rows
-    const uint4 xv = __ldcs(reinterpret_cast<const uint4*>(x + static_cast<int64_t>(n) * D + c0));
-    float* hs = hist + static_cast<int64_t>(s) * 3 * D + c0;
-    float4 hv[3][2];
-#pragma unroll
-    for (int r = 0; r < 3; ++r) {
-        hv[r][0] = __ldcs(reinterpret_cast<const float4*>(hs + r * D));
-        hv[r][1] = __ldcs(reinterpret_cast<const float4*>(hs + r * D + 4));
-    }
-    const float x0 = __bfloat162float(x[static_cast<int64_t>(n) * D]);
 
-    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-    float v[8];
+    // ------------------------------------------------------------- workers
+    float wr[kCh][4], ga[AFF ? kCh : 1], be[AFF ? kCh : 1], bi[AFF ? kCh : 1];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        v[2 * i] = bf16_lo(xw[i]);
-        v[2 * i + 1] = bf16_hi(xw[i]);
+    for (int e = 0; e < kCh; ++e) {
+        const float4 q = active ? *reinterpret_cast<const float4*>(w + static_cast<int64_t>(c0 + e) * 4)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        wr[e][0] = 0.5f * q.x;      // halved: see silu_of_half_dec
+        wr[e][1] = 0.5f * q.y;
+        wr[e][2] = 0.5f * q.z;
+        wr[e][3] = 0.5f * q.w;
     }
-    if (apply_ln) {
+    if constexpr (AFF) {
+        if (active && gamma) load8(gamma + c0, ga);
+        else
+            for (int e = 0; e < kCh; ++e) ga[e] = 1.f;
+        if (active && beta) load8(beta + c0, be);
+        else
+            for (int e = 0; e < kCh; ++e) be[e] = 0.f;
+        if (active && bias) {
+            load8(bias + c0, bi);
+            for (int e = 0; e < kCh; ++e) bi[e] *= 0.5f;
+        } else {
+            for (int e = 0; e < kCh; ++e) bi[e] = 0.f;
+        }
+    }
+    const float invD = 1.0f / static_cast<float>(D);
+
+    for (int k = 0; k < nseq; ++k) {
+        const int st = k % stages;
+        const bool got = mbar_wait(full + st, (k / stages) & 1, ctl);
+        const uint8_t* base = smem + static_cast<size_t>(st) * stage_bytes;
+        const int s = got ? sslot[st] : -1;
+        float v[kCh];
         float s1 = 0.f, s2 = 0.f;
+        if (s >= 0 && active) {
+            const uint4 xv = *reinterpret_cast<const uint4*>(base + hbytes + c0 * 2);
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float d = v[e] - x0;
-            s1 += d;
-            s2 = fmaf(d, d, s2);
-        }
-        const float2 m = block_sum2(s1, s2, red);
-        const float m1 = m.x / D;
-        const float var = fmaxf(m.y / D - m1 * m1, 0.f);
-        const float mean = x0 + m1, rstd = rsqrtf(var + eps);
-        float g[8], bt[8];
-        if (gamma) load8(gamma + c0, g);
-        if (beta) load8(beta + c0, bt);
+            for (int i = 0; i < 4; ++i) {
+                v[2 * i] = bf16_lo(xw[i]);
+                v[2 * i + 1] = bf16_hi(xw[i]);
+            }
+            if (apply_ln) {
+                const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + hbytes));
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            float t = (v[e] - mean) * rstd;
-            if (gamma) t *= g[e];
-            if (beta) t += bt[e];
-            v[e] = t;
+                for (int e = 0; e < kCh; ++e) {
+                    const float d = v[e] - x0;
+                    s1 += d;
+                    s2 = fmaf(d, d, s2);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < kCh; ++e) v[e] = 0.f;
         }
+        float2* rp = red + (k & 1) * (MAXT / 32);
+        if (apply_ln) {
+            s1 = warp_sum_dec(s1);
+            s2 = warp_sum_dec(s2);
+            if (lane == 0) rp[warp] = make_float2(s1, s2);
+        }
+        // the partials are visible to every worker (the buffer of this parity
+        // was last read before the previous sequence's barrier); a timed-out
+        // wait stops every worker here
+        if (workers_or_dec(!got, nwork)) break;
+        if (s < 0) {
+            if (tid == 0) record_status(ctl.status, GLA_ERR_INVALID_ARG);
+            mbar_arrive(freeb + st);
+            continue;
+        }
+        if (apply_ln) {
+            float m1 = 0.f, m2 = 0.f;
+            for (int i = 0; i < nwarps; ++i) {
+                m1 += rp[i].x;
+                m2 += rp[i].y;
+            }
+            const float x0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + hbytes));
+            const float mu = m1 * invD;
+            const float var = fmaxf(m2 * invD - mu * mu, 0.f);
+            const float mean = x0 + mu, rstd = rsqrtf(var + eps);
+#pragma unroll
+            for (int e = 0; e < kCh; ++e) {
+                const float t = (v[e] - mean) * rstd;
+                if constexpr (AFF) v[e] = fmaf(t, ga[e], be[e]);
+                else v[e] = t;
+            }
+        }
+        if (active) {
+            const float* hs = reinterpret_cast<const float*>(base);
+            float h0[kCh], h1[kCh], h2[kCh];
+            load8(hs + c0, h0);
+            load8(hs + D + c0, h1);
+            load8(hs + 2 * D + c0, h2);
+            uint32_t out[4];
+#pragma unroll
+            for (int e = 0; e < kCh; e += 2) {
+                float r[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    float acc = AFF ? bi[AFF ? e + u : 0] : 0.f;
+                    acc = fmaf(wr[e + u][0], h0[e + u], acc);
+                    acc = fmaf(wr[e + u][1], h1[e + u], acc);
+                    acc = fmaf(wr[e + u][2], h2[e + u], acc);
+                    r[u] = silu_of_half_dec(fmaf(wr[e + u][3], v[e + u], acc));
+                }
+                out[e / 2] = pack_bf16(r[0], r[1]);
+            }
+            const int n = blockIdx.x + k * gridDim.x;
+            float* hg = hist + static_cast<int64_t>(s) * 3 * D + c0;
+            __stcs(reinterpret_cast<uint4*>(y + static_cast<int64_t>(n) * D + c0),
+                   make_uint4(out[0], out[1], out[2], out[3]));
+            __stcs(reinterpret_cast<float4*>(hg), make_float4(h1[0], h1[1], h1[2], h1[3]));
+            __stcs(reinterpret_cast<float4*>(hg + 4), make_float4(h1[4], h1[5], h1[6], h1[7]));
+            __stcs(reinterpret_cast<float4*>(hg + D), make_float4(h2[0], h2[1], h2[2], h2[3]));
+            __stcs(reinterpret_cast<float4*>(hg + D + 4), make_float4(h2[4], h2[5], h2[6], h2[7]));
+            __stcs(reinterpret_cast<float4*>(hg + 2 * D), make_float4(v[0], v[1], v[2], v[3]));
+            __stcs(reinterpret_cast<float4*>(hg + 2 * D + 4), make_float4(v[4], v[5], v[6], v[7]));
+        }
+        mbar_arrive(freeb + st);             // this worker is done with the stage
     }
-
-    const float h0[8] = {hv[0][0].x, hv[0][0].y, hv[0][0].z, hv[0][0].w, hv[0][1].x, hv[0][1].y, hv[0][1].z, hv[0][1].w};
-    const float h1[8] = {hv[1][0].x, hv[1][0].y, hv[1][0].z, hv[1][0].w, hv[1][1].x, hv[1][1].y, hv[1][1].z, hv[1][1].w};
-    const float h2[8] = {hv[2][0].x, hv[2][0].y, hv[2][0].z, hv[2][0].w, hv[2][1].x, hv[2][1].y, hv[2][1].z, hv[2][1].w};
-    // the weights and the bias are L2-resident across sequences
-    float bi[8];
-    if (bias) load8(bias + c0, bi);
-    uint32_t out[4];
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-        float r[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const float4 wc = *reinterpret_cast<const float4*>(w + static_cast<int64_t>(c0 + e + u) * 4);
-            float acc = bias ? bi[e + u] : 0.f;
-            acc = fmaf(wc.x, h0[e + u], acc);
-            acc = fmaf(wc.y, h1[e + u], acc);
-            acc = fmaf(wc.z, h2[e + u], acc);
-            acc = fmaf(wc.w, v[e + u], acc);
-            r[u] = silu_dec(acc);
-        }
-        out[e / 2] = pack_bf16(r[0], r[1]);
-    }
-    __stcs(reinterpret_cast<uint4*>(y + static_cast<int64_t>(n) * D + c0), make_uint4(out[0], out[1], out[2], out[3]));
-    __stcs(reinterpret_cast<float4*>(hs), hv[1][0]);
-    __stcs(reinterpret_cast<float4*>(hs + 4), hv[1][1]);
-    __stcs(reinterpret_cast<float4*>(hs + D), hv[2][0]);
-    __stcs(reinterpret_cast<float4*>(hs + D + 4), hv[2][1]);
-    __stcs(reinterpret_cast<float4*>(hs + 2 * D), make_float4(v[0], v[1], v[2], v[3]));
-    __stcs(reinterpret_cast<float4*>(hs + 2 * D + 4), make_float4(v[4], v[5], v[6], v[7]));
 }
 
 }  // namespace
 
 gla_status launch_conv_decode(const void* x, const int32_t* slot_idx, int n_slots, int apply_ln, const float* g,
                               const float* b, float eps, const float* w, const float* bias, float* hist,
-                              void* y, int N, int D, int* status, cudaStream_t st)
+                              void* y, int N, int D, WaitCtl ctl, cudaStream_t st)
 {
+    // 8 channels per worker thread (384 workers at D = 3,072) and one warp
+    // that issues the copies; one CTA per SM (or per sequence, if fewer)
+    const int threads = ((D / kCh) + 31) / 32 * 32 + 32;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = N < sms ? N : sms;
+    // as many stages (up to 4) as fit in 200 KB beside the barriers
+    const size_t stage_bytes = static_cast<size_t>(14) * D;
+    const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + kMaxStages * sizeof(int) + 2 * 32 * sizeof(float2);
+    int stages = static_cast<int>((200 * 1024 - fixed) / stage_bytes);
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages > N) stages = N > 1 ? N : 1;
+    const size_t smem = stages * stage_bytes + fixed;
+    const bool aff = g || b || bias;
+    auto kernel = threads <= 416 ? (aff ? conv_decode_kernel<true, 416> : conv_decode_kernel<false, 416>)
+                                 : (aff ? conv_decode_kernel<true, 544> : conv_decode_kernel<false, 544>);
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+        cudaSuccess)
+        return check_launch("cudaFuncSetAttribute");
     trace_begin(st);
-    conv_decode_kernel<<<N, D / 8, 0, st>>>(static_cast<const __nv_bfloat16*>(x), slot_idx, apply_ln, g, b, eps,
-                                            w, bias, hist, static_cast<__nv_bfloat16*>(y), D, n_slots, status);
+    kernel<<<grid, threads, smem, st>>>(static_cast<const __nv_bfloat16*>(x), slot_idx, apply_ln, g, b, eps, w, bias,
+                                        hist, static_cast<__nv_bfloat16*>(y), N, D, n_slots, stages, ctl);
     trace_end(st, "conv_decode_kernel");
     count_launch();
     return check_launch("conv_decode_kernel");

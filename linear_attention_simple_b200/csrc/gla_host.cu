@@ -158,6 +158,8 @@ WaitCtl wait_ctl_for_current_device(gla_status* err)
     return c;
 }
 
+gla_status status_of(cudaError_t e) { return e == cudaSuccess ? GLA_OK : cuda_fail(e); }
+
 gla_status check_launch(const char* what)
 {
     (void)what;
@@ -615,7 +617,7 @@ gla_status conv1d_silu_decode_step(const void* x, const int32_t* slot_idx, int n
     WaitCtl ctl = wait_ctl_for_current_device(&se);
     if (se != GLA_OK) return se;
     return launch_conv_decode(x, slot_idx, n_slots, apply_ln, ln_gamma, ln_beta, ln_eps, w, bias, conv_state, y, N,
-                              D, ctl.status, stream);
+                              D, ctl, stream);
 }
 
 size_t conv1d_silu_causal_bwd_workspace_bytes(int B, int T, int D, int W)

@@ -29,6 +29,8 @@ WaitCtl wait_ctl_for_current_device(gla_status* err);
 // device addresses cached per device are valid only within it.
 const void* current_cu_context();
 gla_status check_launch(const char* what);
+// GLA_ERR_CUDA for a failed runtime call, its code kept for gla_last_cuda_error.
+gla_status status_of(cudaError_t e);
 void count_launch(unsigned n = 1);
 
 // Tracing: trace_begin() before a launch, trace_end() after it; both are
@@ -53,7 +55,7 @@ gla_status launch_conv(const void* x, int apply_ln, const float* g, const float*
 
 gla_status launch_conv_decode(const void* x, const int32_t* slot_idx, int n_slots, int apply_ln, const float* g,
                               const float* b, float eps, const float* w, const float* bias, float* hist,
-                              void* y, int N, int D, int* status, cudaStream_t st);
+                              void* y, int N, int D, WaitCtl ctl, cudaStream_t st);
 
 size_t conv_bwd_workspace_bytes(int B, int T, int D);
 gla_status launch_conv_bwd(const void* x, int apply_ln, const float* g, const float* be, float eps, const float* w,

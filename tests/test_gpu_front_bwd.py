@@ -70,6 +70,9 @@ def _check(d, ln, want_hist=True):
     (3, 129, 64, False, False, True),
     (2, 5, 512, True, False, True),
     (1, 130, 4096, True, True, True),
+    (2, 200, 2056, True, True, True),
+    (1, 700, 2048, True, False, True),
+    (1, 7, 3072, False, True, True),
 ])
 def test_front_bwd_parity(B, T, D, ln, affine, hist):
     _check(_case(B, T, D, affine, hist, seed=70 + T + D), ln)

@@ -624,7 +624,11 @@ __global__ void __launch_bounds__(256) conv_bwd_reduce_kernel(const float* __res
 }
 
 // At most 256 workers a CTA (4 channels each) and one producer warp, so
-// that the per-channel registers fit without spilling.
+// that the per-channel registers fit without spilling.  (Workers of 2
+// channels -- 13 warps a CTA at 128 registers -- measured slower at
+// D = 3,072, 1.46 ms against 1.38 ms: the kernel is bound by instruction
+// issue, and a narrower thread repeats the per-row work that does not
+// scale with its channels.)
 constexpr int kBwdThreads = 288;
 
 struct BwdPlan {

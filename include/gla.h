@@ -165,10 +165,13 @@ gla_status gla_chunk_bwd_saved(const void* q, const void* k, const void* v, cons
  *   s0, s_final [N, H, 96, 192] fp32 or NULL (zeros / not wanted).
  *   ws          workspace of ws_bytes >= gla_chunk_varlen_workspace_bytes(N,
  *               total_T, H, dk, dv), or NULL.  With it, sequences longer than a
- *               segment (a length the library derives from total_T and H)
- *               are cut into segments that run in parallel (state-only
- *               pre-pass, fp32 fold, output pass), so one long sequence no
- *               longer sets the time; without it (or when the size is 0) each
+ *               segment (about total_T H / (148 x 128) chunks, so that the
+ *               segments of all sequences make about one wave of CTAs) are cut
+ *               into segments that run in parallel (state-only pre-pass, fp32
+ *               fold, output pass), so one long sequence no longer sets the
+ *               time; a small kernel reads the lengths on the device and
+ *               splits only when the longest sequence spans at least two
+ *               segments.  Without it (or when the size is 0) each
  *               (sequence, head) is one sweep.  Contents on entry do not
  *               matter.  When cu_seqlens is invalid and a workspace is given,
  *               the outputs of the valid sequences are undefined as well.

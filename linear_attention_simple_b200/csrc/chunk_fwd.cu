@@ -81,8 +81,9 @@ __global__ void __launch_bounds__(256) seg_combine_varlen_kernel(float* __restri
                                                                  const float* __restrict__ g2,
                                                                  const float* __restrict__ s0,
                                                                  const int* __restrict__ cu, int N, int H,
-                                                                 int total_T, int cps)
+                                                                 int total_T, const int* __restrict__ cps_dev)
 {
+    const int cps = *cps_dev;
     const int64_t n4 = kSS / 4;
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= n4 * N * H) return;
@@ -198,12 +199,105 @@ size_t fwd_workspace_bytes(int B, int T, int H)
 // extra segment costs a pre-pass sweep), at least 4 chunks; 0 when no
 // sequence can be longer than one segment (total_T within it), i.e. no
 // segmenting.
+// Segment length of the packed forward: about one wave of CTAs over all the
+// chunks (total_T H / (148 x 128) chunks a segment, at least 4).  Measured
+// on 16,384 to 36,000 tokens at H = 16 with one or more long sequences,
+// this length was within 10% of the best of 4 to 64 chunks (four waves of
+// 4-chunk segments: up to 1.8x slower).  0: nothing to split.
 int varlen_chunks_per_seg(int total_T, int H)
 {
-    const int64_t per_cta = (static_cast<int64_t>(total_T) * H + 4 * kTargetCtas - 1) / (4 * kTargetCtas);
+    const int64_t per_cta = (static_cast<int64_t>(total_T) * H + kTargetCtas - 1) / kTargetCtas;
     int cps = static_cast<int>((per_cta + 127) / 128);
     if (cps < 4) cps = 4;
     return static_cast<int64_t>(total_T) <= static_cast<int64_t>(cps) * 128 ? 0 : cps;
+}
+
+// Whether to split at all, decided on the device from the sequence lengths:
+// the segment length above when the longest sequence has at least twice as
+// many chunks, else a length no sequence reaches (one segment each: equal
+// lengths gain nothing from the pre-pass).  The kernel also lists the
+// (sequence, segment) items of the output pass and of the pre-pass (every
+// segment but a sequence's last), so those grids hold only work.  One CTA;
+// plan = {chunks per segment, output items, pre-pass items}.
+constexpr int kNoSplit = 1 << 20;
+constexpr int kPlanThreads = 1024;
+
+// Upper bound of the items of either list: N + (all chunks + N) / cps + 1.
+int64_t varlen_max_items(int N, int total_T, int cps)
+{
+    const int64_t chunks = (static_cast<int64_t>(total_T) + 127) / 128;
+    return N + (chunks + N) / cps + 1;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) varlen_plan_kernel(const int* __restrict__ cu, int N, int total_T,
+                                                                   int cps, int* __restrict__ plan,
+                                                                   int2* __restrict__ work_out,
+                                                                   int2* __restrict__ work_pre)
+{
+    __shared__ int s_w[kPlanThreads / 32][2];
+    __shared__ int s_cps, s_carry[2];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    auto length = [&](int n) {
+        const int tb = cu[n], Tn = cu[n + 1] - tb;
+        return (tb >= 0 && Tn >= 0 && tb + Tn <= total_T) ? Tn : -1;   // -1: invalid (one item, reported later)
+    };
+    int m = 0;
+    for (int n = tid; n < N; n += kPlanThreads) m = max(m, length(n));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) s_w[warp][0] = m;
+    __syncthreads();
+    if (tid == 0) {
+        int mm = 0;
+        for (int w = 0; w < kPlanThreads / 32; ++w) mm = max(mm, s_w[w][0]);
+        s_cps = (mm + 127) / 128 >= 2 * cps ? cps : kNoSplit;
+        s_carry[0] = s_carry[1] = 0;
+    }
+    __syncthreads();
+    const int c = s_cps;
+    for (int base = 0; base < N; base += kPlanThreads) {
+        const int n = base + tid;
+        int segs = 0;
+        if (n < N) {
+            const int len = length(n);
+            segs = len < 0 ? 1 : max(1, ((len + 127) / 128 + c - 1) / c);
+        }
+        const int pre = segs > 0 ? segs - 1 : 0;
+        // inclusive scans of segs and pre over the block
+        int a = segs, q = pre;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int ya = __shfl_up_sync(0xffffffffu, a, o), yq = __shfl_up_sync(0xffffffffu, q, o);
+            if (lane >= o) {
+                a += ya;
+                q += yq;
+            }
+        }
+        if (lane == 31) {
+            s_w[warp][0] = a;
+            s_w[warp][1] = q;
+        }
+        __syncthreads();
+        int wa = 0, wq = 0;
+        for (int w = 0; w < warp; ++w) {
+            wa += s_w[w][0];
+            wq += s_w[w][1];
+        }
+        const int off_a = s_carry[0] + wa + a - segs, off_q = s_carry[1] + wq + q - pre;
+        for (int sg = 0; sg < segs; ++sg) work_out[off_a + sg] = make_int2(n, sg);
+        for (int sg = 0; sg < pre; ++sg) work_pre[off_q + sg] = make_int2(n, sg);
+        __syncthreads();
+        if (tid == kPlanThreads - 1) {
+            s_carry[0] = off_a + segs;
+            s_carry[1] = off_q + pre;
+        }
+        __syncthreads();
+    }
+    if (tid == 0) {
+        plan[0] = c;
+        plan[1] = s_carry[0];
+        plan[2] = s_carry[1];
+    }
 }
 
 size_t varlen_workspace_bytes(int N, int total_T, int H)
@@ -212,8 +306,10 @@ size_t varlen_workspace_bytes(int N, int total_T, int H)
     if (cps == 0) return 0;
     const int64_t L = static_cast<int64_t>(cps) * 128;
     const int64_t slots = N + (total_T + L - 1) / L + 1;
+    const int64_t items = varlen_max_items(N, total_T, cps);
     return align256(static_cast<size_t>(slots) * H * kSS * sizeof(float)) +
-           align256(static_cast<size_t>(slots) * H * sizeof(float));
+           align256(static_cast<size_t>(slots) * H * sizeof(float)) + 256 +   // + the plan
+           2 * align256(static_cast<size_t>(items) * sizeof(int2));            // + the two item lists
 }
 
 gla_status run_chunk_fwd_varlen(const ChunkProblem& pr, const int* cu_seqlens, int N, const float* s0, void* o,
@@ -251,13 +347,27 @@ gla_status run_chunk_fwd_varlen(const ChunkProblem& pr, const int* cu_seqlens, i
     // segment but each sequence's last, the fold that leaves the state
     // entering each segment in its slot, then the fused pass per segment
     const int64_t L = static_cast<int64_t>(cps) * 128;
-    const int max_segs = static_cast<int>((pr.T + L - 1) / L);
     const int64_t slots = N + (pr.T + L - 1) / L + 1;
     float* states = static_cast<float*>(ws);
     float* g2 = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
                                          align256(static_cast<size_t>(slots) * pr.H * kSS * sizeof(float)));
+    int* plan = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(g2) +
+                                       align256(static_cast<size_t>(slots) * pr.H * sizeof(float)));
+    const int64_t items = varlen_max_items(N, pr.T, cps);
+    int2* work_out = reinterpret_cast<int2*>(reinterpret_cast<uint8_t*>(plan) + 256);
+    int2* work_pre = reinterpret_cast<int2*>(reinterpret_cast<uint8_t*>(work_out) +
+                                             align256(static_cast<size_t>(items) * sizeof(int2)));
+    const int* cps_dev = plan;
+    trace_begin(st);
+    varlen_plan_kernel<<<1, kPlanThreads, 0, st>>>(cu_seqlens, N, pr.T, cps, plan, work_out, work_pre);
+    trace_end(st, "varlen_plan_kernel");
+    count_launch();
+    if ((s = check_launch("varlen_plan_kernel")) != GLA_OK) return s;
     StateParams pre = p;
     pre.chunks_per_seg = cps;
+    pre.cps_dev = cps_dev;
+    pre.work = work_pre;
+    pre.work_count = plan + 2;
     pre.seg_states = states;
     pre.seg_g2 = g2;
     pre.varlen_segs = 1;
@@ -265,20 +375,24 @@ gla_status run_chunk_fwd_varlen(const ChunkProblem& pr, const int* cu_seqlens, i
     pre.s_init = nullptr;
     pre.s_out = states;                 // written at each segment's slot
     pre.out_last_only = 0;
-    if ((s = launch_state_kernel(false, false, pre, dim3(max_segs, pr.H, N), st)) != GLA_OK) return s;
+    if ((s = launch_state_kernel(false, false, pre, dim3(static_cast<unsigned>(items), pr.H, 1), st)) != GLA_OK)
+        return s;
     {
         const int64_t n = static_cast<int64_t>(N) * pr.H * (kSS / 4);
         trace_begin(st);
         seg_combine_varlen_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(states, g2, s0, cu_seqlens,
-                                                                                        N, pr.H, pr.T, cps);
+                                                                                        N, pr.H, pr.T, cps_dev);
         trace_end(st, "seg_combine_varlen_kernel");
         count_launch();
         if ((s = check_launch("seg_combine_varlen_kernel")) != GLA_OK) return s;
     }
     p.chunks_per_seg = cps;
+    p.cps_dev = cps_dev;
+    p.work = work_out;
+    p.work_count = plan + 1;
     p.seg_states = states;
     p.varlen_segs = 1;
-    return launch_state_kernel(true, false, p, dim3(max_segs, pr.H, N), st);
+    return launch_state_kernel(true, false, p, dim3(static_cast<unsigned>(items), pr.H, 1), st);
 }
 
 gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float* s_final,

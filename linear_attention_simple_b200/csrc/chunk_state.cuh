@@ -84,6 +84,10 @@ struct StateParams {
     float* seg_states;      // [slots][H][96][192] fp32: pre-pass end states, then entering states
     float* seg_g2;          // [slots][H] total log2-decay of each segment (pre-pass)
     int varlen_segs;        // 1: segmented varlen (chunks_per_seg chunks per segment)
+    const int* cps_dev;     // segmented varlen: the chunks per segment the device planned
+                            // (read instead of chunks_per_seg when set)
+    const int2* work;       // segmented varlen: the (sequence, segment) of grid item x;
+    const int* work_count;  // items past *work_count exit (null: the grid's own indices)
     int pre_pass;           // state pass: only segments 0 .. nseg_n - 2 of each sequence
     void* h_save;           // fused forward: the state entering each chunk, [B*H*NC][2][96][192]
                             // bf16 (hi, lo planes), for the backward; null = not saved
@@ -365,10 +369,17 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     float* wsum = cfac + 256;                                    // [4]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.y;
+    int seg = blockIdx.x, b = blockIdx.z;
+    if (VARLEN && p.work) {                        // the device-planned segment list
+        if (static_cast<int>(blockIdx.x) >= *p.work_count) return;
+        const int2 w = p.work[blockIdx.x];
+        b = w.x;
+        seg = w.y;
+    }
     const int unit = b * p.H + h;
-    // varlen: blockIdx.z is a sequence, its tokens tb .. tb+Tn-1 of batch row
-    // 0; otherwise batch row b, tokens 0 .. T-1
+    // varlen: b is a sequence, its tokens tb .. tb+Tn-1 of batch row 0;
+    // otherwise batch row b, tokens 0 .. T-1
     int tb = 0, Tn = p.T, NCn = p.NC;
     if constexpr (VARLEN) {
         tb = p.cu_seqlens[b];
@@ -380,14 +391,15 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         }
     }
     const int bc = VARLEN ? 0 : b;                 // batch coordinate of the token tensors
-    const int c_begin = seg * p.chunks_per_seg;
+    const int cps = p.cps_dev ? *p.cps_dev : p.chunks_per_seg;
+    const int c_begin = seg * cps;
     // segmented varlen: a grid slot past this sequence's last segment has
     // nothing to do (segment 0 always runs: an empty sequence still passes
     // its initial state on)
     if (VARLEN && seg > 0 && c_begin >= NCn) return;
-    const int c_end = min(NCn, c_begin + p.chunks_per_seg);
+    const int c_end = min(NCn, c_begin + cps);
     const int nchunks = c_end - c_begin;
-    const int last_seg = VARLEN ? max(1, (NCn + p.chunks_per_seg - 1) / p.chunks_per_seg) - 1
+    const int last_seg = VARLEN ? max(1, (NCn + cps - 1) / cps) - 1
                                 : static_cast<int>(gridDim.x) - 1;
     const WaitCtl ctl = p.ctl;
 
@@ -461,7 +473,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                                           row * kDv + half * 96
                                     : nullptr;
         if (VARLEN && seg > 0)    // a later segment of a sequence: the state the combine left for it
-            src = p.seg_states + (varlen_slot(p.cu_seqlens, b, seg, p.chunks_per_seg) * p.H + h) * (kDk * kDv) +
+            src = p.seg_states + (varlen_slot(p.cu_seqlens, b, seg, cps) * p.H + h) * (kDk * kDv) +
                   row * kDv + half * 96;
         state_to_tmem(src, tq + L::TM_S + half * 96);
     }
@@ -788,9 +800,17 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
     constexpr uint32_t kWork = 384;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int seg = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.y;
+    int seg = blockIdx.x, b = blockIdx.z;
+    if (p.cu_seqlens && p.work) {                  // the device-planned segment list
+        if (static_cast<int>(blockIdx.x) >= *p.work_count) return;
+        const int2 w = p.work[blockIdx.x];
+        b = w.x;
+        seg = w.y;
+    }
     const int unit = b * p.H + h;
-    // varlen (segmented pre-pass of the packed forward): blockIdx.z is a
+    const int cps = p.cps_dev ? *p.cps_dev : p.chunks_per_seg;
+    // varlen (segmented pre-pass of the packed forward): b is a
     // sequence, its tokens tb .. tb+Tn-1 of batch row 0; the segments are
     // the sequence's own, and the pre-pass sweeps all but its last
     int tb = 0, Tn = p.T, NCn = p.NC;
@@ -802,12 +822,12 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
             return;
         }
         NCn = (Tn + 127) / 128;
-        const int nseg_n = max(1, (NCn + p.chunks_per_seg - 1) / p.chunks_per_seg);
+        const int nseg_n = max(1, (NCn + cps - 1) / cps);
         if (seg >= nseg_n - (p.pre_pass ? 1 : 0)) return;
     }
     const int bc = p.cu_seqlens ? 0 : b;         // batch coordinate of the token tensors
-    const int c_begin = seg * p.chunks_per_seg;
-    const int c_end = min(NCn, c_begin + p.chunks_per_seg);
+    const int c_begin = seg * cps;
+    const int c_end = min(NCn, c_begin + cps);
     const int nchunks = c_end - c_begin;
     const WaitCtl ctl = p.ctl;
     const int quad = warp & 3, row = quad * 32 + lane, qt = warp >> 2;
@@ -1074,7 +1094,7 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
             if (write_state && GLA_DCHECK(unit < p.B * p.H && row < kDk, p.ctl.status)) {
                 float* dst = p.cu_seqlens
                                  ? p.seg_states +
-                                       (varlen_slot(p.cu_seqlens, b, seg, p.chunks_per_seg) * p.H + h) * (kDk * kDv) +
+                                       (varlen_slot(p.cu_seqlens, b, seg, cps) * p.H + h) * (kDk * kDv) +
                                        row * kDv + qt * 48
                                  : p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + qt * 48;
 #pragma unroll
@@ -1082,7 +1102,7 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
                     *reinterpret_cast<float4*>(dst + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
             }
             if (p.cu_seqlens && tid == 0)
-                p.seg_g2[varlen_slot(p.cu_seqlens, b, seg, p.chunks_per_seg) * p.H + h] = gsum2;
+                p.seg_g2[varlen_slot(p.cu_seqlens, b, seg, cps) * p.H + h] = gsum2;
             else if (p.g2_out && tid == 0)
                 p.g2_out[static_cast<int64_t>(unit) * p.g2_unit_stride + seg] = gsum2;
         }

@@ -125,11 +125,16 @@ def test_varlen_long_sequence_among_short_ones_is_segmented():
     assert rel_l2(_np(sf), _np(sf1)) <= 1e-3
 
 
-def test_varlen_segmented_time_16k_tokens():
-    """16,384 tokens in 8 sequences of 1 to 5,610 tokens at H = 16: the
-    segmented and the one-sweep-per-sequence forward, timed with CUDA events
-    (printed), and equal to each other."""
-    lengths = [5610, 1, 3000, 2048, 777, 129, 4000, 819]
+@pytest.mark.parametrize("name,lengths", [
+    ("8 sequences of 1 to 5,610 tokens", [5610, 1, 3000, 2048, 777, 129, 4000, 819]),
+    ("one 16,384-token sequence among 7 short ones", [16384, 500, 300, 1000, 200, 700, 100, 50]),
+    ("8 equal sequences of 2,048 tokens", [2048] * 8),
+])
+def test_varlen_segmented_time(name, lengths):
+    """Packed sequences at H = 16: the segmented and the one-sweep-per-sequence
+    forward, timed with CUDA events (printed), and equal to each other.  With
+    equal lengths the device plan does not split (both paths do the same
+    work)."""
     H = 16
     q, k, v, a, cu, s0 = _packed(lengths, H, seed=94)
     ws = torch.empty(max(1, gla.gla_chunk_varlen_workspace_bytes(len(lengths), q.shape[0], H)),
@@ -152,7 +157,7 @@ def test_varlen_segmented_time_16k_tokens():
         times[seg] = e0.elapsed_time(e1) / 10 * 1e3
         outs[seg] = (o.clone(), sf.clone())
     assert gla.gla_get_device_status() == 0
-    print("packed forward, 16,384 tokens, H = 16: one sweep per sequence %.1f us, segmented %.1f us"
-          % (times[False], times[True]))
+    print("packed forward, %s (%d tokens), H = 16: one sweep per sequence %.1f us, segmented %.1f us"
+          % (name, sum(lengths), times[False], times[True]))
     assert rel_l2(_np(outs[True][0]), _np(outs[False][0])) <= 1e-3
     assert rel_l2(_np(outs[True][1]), _np(outs[False][1])) <= 1e-3

@@ -58,7 +58,7 @@ constexpr int kG = 4;           // rows per stage
 constexpr int kRing = 8;        // ring stages: s, s+1, s+2 (moments) and five in flight
 constexpr int kXch = 4;         // exchange buffers (a CTA runs at most two exchanges ahead)
 constexpr int kMsg = 24;        // floats per CTA per exchange
-constexpr int kStRing = 16;     // rows of LayerNorm statistics kept
+constexpr int kStRing = 32;     // rows of LayerNorm statistics kept
 constexpr int kParts = 7;       // dw (4 taps), dbias, dgamma, dbeta
 constexpr int kMaxSlices = 128; // token ranges per sequence
 constexpr int kMinRows = 64;    // rows per range at least
@@ -146,11 +146,11 @@ struct BwdSmem {
         segb = 16u * upc;                                  // one row of a CTA's channels
         ring = 0;
         fin = ring + kRing * 2 * kG * segb;                // [2][kG][nwork][8] fp32: g, xhat
-        red = fin + 2 * kG * nwork * 32;                   // [warps][16]
-        xbuf = red + (nwork / 32) * 64;                    // [kXch][CL max 4][kMsg]
+        red = fin + 2 * kG * nwork * 32;                   // [2][warps][16] by stage parity
+        xbuf = red + 2 * (nwork / 32) * 64;                // [kXch][CL max 4][kMsg]
         st = xbuf + kXch * 4 * kMsg * 4;                   // [kStRing] (mean, rstd)
-        tot = st + kStRing * 8;                            // [kG] (mean g, mean g xhat)
-        bars = tot + kG * 8;                               // full[kRing], free[kRing], xbar[kXch]
+        tot = st + kStRing * 8;                            // [2][kG] (mean g, mean g xhat) by stage parity
+        bars = tot + 2 * kG * 8;                           // full[kRing], free[kRing], xbar[kXch]
         total = bars + (2 * kRing + kXch) * 8;
     }
 };
@@ -441,7 +441,7 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
                 const int q = p_s + s * kG + g - 3;
                 if (q >= t_b && q < t_e && active) {
                     const float rstd = st_ring[(q - p_s) & (kStRing - 1)].y;
-                    const float2 mt = tot[g];
+                    const float2 mt = tot[(s & 1) * kG + g];
                     const f2 rs = f2_splat(rstd), na = f2_splat(-rstd * mt.x), nb = f2_splat(-rstd * mt.y);
                     const float* fp = fin_at(s & 1, g);
                     const float4 g4 = *reinterpret_cast<const float4*>(fp);
@@ -489,13 +489,33 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
         // ---- the stages (every exit from the loop follows a barrier, so
         // that all workers leave together)
         for (int s = 0; s < S && !failed; ++s) {
+            const int pos0 = p_s + s * kG;
+            if (ln && s >= 1 && warp == 0) {
+                // exchange s (sent after stage s-1): the g sums of stage
+                // s-1's output rows and the statistics of stage s+1's rows,
+                // published to the other workers by this stage's barrier
+                if (!wait_x(s)) failed = true;
+                if (!failed) {
+                    if (lane < kG) {
+                        float sg = 0.f, sgx = 0.f;
+                        for (int r2 = 0; r2 < CL; ++r2) {
+                            sg += *xch_addr(s, r2, lane);
+                            sgx += *xch_addr(s, r2, kG + lane);
+                        }
+                        tot[((s - 1) & 1) * kG + lane] = make_float2(sg * invD, sgx * invD);
+                    } else if (lane < 2 * kG) {
+                        const int g = lane - kG;
+                        st_ring[(pos0 + kG + g - p_s) & (kStRing - 1)] =
+                            combine_stats(s, 2 * kG + g, 3 * kG + g, 16 + g);
+                    }
+                }
+            }
             const int slot = s % kRing;
-            bool ok = mbar_wait(full + slot, (s / kRing) & 1, ctl);
+            bool ok = !failed && mbar_wait(full + slot, (s / kRing) & 1, ctl);
             if (ln && ok && s + 2 < S) ok = mbar_wait(full + (s + 2) % kRing, ((s + 2) / kRing) & 1, ctl);
             if (!ok) failed = true;
 #pragma unroll
             for (int i = 0; i < 2 * kG; ++i) gs[i] = 0.f;
-            const int pos0 = p_s + s * kG;
             if (!failed) {
                 if (pos0 >= t_b + 3 && pos0 + kG <= min(T, t_e)) {
 #pragma unroll
@@ -524,8 +544,9 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
                 if (!failed && s + 2 < S) moments(s + 2, g, pos0 + 2 * kG + g, v[2 * kG + g], v[3 * kG + g]);
                 else v[2 * kG + g] = v[3 * kG + g] = 0.f;
             }
+            float* rd = red + (s & 1) * nwarps * 16;
             const float r = warp_reduce16(v, lane);
-            if ((lane & 1) == 0) red[warp * 16 + (lane >> 1)] = r;
+            if ((lane & 1) == 0) rd[warp * 16 + (lane >> 1)] = r;
             if (workers_or_bwd(failed, nwork)) {
                 failed = true;
                 break;
@@ -533,36 +554,13 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
             arm(s + 1);
             if (tid < 16) {
                 float t = 0.f;
-                for (int w = 0; w < nwarps; ++w) t += red[w * 16 + tid];
+                for (int w = 0; w < nwarps; ++w) t += rd[w * 16 + tid];
                 push(s + 1, tid, t);
             } else if (tid < kMsg) {
                 // every message is kMsg values (the arm counts them): the
                 // first elements of the rows two stages ahead, then zeros
                 const int g = tid - 16;
                 push(s + 1, tid, (g < kG && s + 2 < S) ? first_x(s + 2, g, pos0 + 2 * kG + g) : 0.f);
-            }
-            if (s >= 1 && warp == 0) {
-                // exchange s: the g sums of stage s-1's output rows and the
-                // statistics of stage s+1's rows
-                if (!wait_x(s)) failed = true;
-                if (!failed) {
-                    if (lane < kG) {
-                        float sg = 0.f, sgx = 0.f;
-                        for (int r2 = 0; r2 < CL; ++r2) {
-                            sg += *xch_addr(s, r2, lane);
-                            sgx += *xch_addr(s, r2, kG + lane);
-                        }
-                        tot[lane] = make_float2(sg * invD, sgx * invD);
-                    } else if (lane < 2 * kG) {
-                        const int g = lane - kG;
-                        st_ring[(pos0 + kG + g - p_s) & (kStRing - 1)] =
-                            combine_stats(s, 2 * kG + g, 3 * kG + g, 16 + g);
-                    }
-                }
-            }
-            if (workers_or_bwd(failed, nwork)) {
-                failed = true;
-                break;
             }
             if (s >= 1) finish(s - 1);
         }
@@ -576,7 +574,7 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
                         sg += *xch_addr(S, r2, lane);
                         sgx += *xch_addr(S, r2, kG + lane);
                     }
-                    tot[lane] = make_float2(sg * invD, sgx * invD);
+                    tot[((S - 1) & 1) * kG + lane] = make_float2(sg * invD, sgx * invD);
                 }
             }
             if (!workers_or_bwd(failed, nwork)) finish(S - 1);

@@ -155,7 +155,12 @@ struct BwdSmem {
     }
 };
 
-template <bool AFF, int CL, int MAXT>
+// LN: the LayerNorm is applied (its statistics and row sums are exchanged).
+// FULL: every worker thread of every CTA owns channels (the 8-channel units
+// split evenly over the cluster into whole warps), so no thread is idle.
+// Both are template parameters: their tests would otherwise be branches in
+// the row loop (measured 9% of the kernel's time for the LayerNorm flag).
+template <bool AFF, bool LN, bool FULL, int CL, int MAXT>
 __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_constant__ BwdArgs a)
 {
     static_assert(CL >= 2 && CL <= 4, "the rows' channels are split over 2 to 4 CTAs");
@@ -181,7 +186,7 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
     const int p_s = t_b - 3;                                   // stream rows p_s .. t_e + 2
     const int S = (t_e - t_b + 6 + kG - 1) / kG;
     const int p_load = min(T, t_e + 3);                        // rows [max(0, p_s), p_load) are loaded
-    const bool ln = a.apply_ln != 0;
+    constexpr bool ln = LN;
     const int64_t row0 = static_cast<int64_t>(b) * T;
 
     if (tid == 0) {
@@ -234,7 +239,7 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
     } else {
         // ------------------------------------------------------------- workers
         const int u = tid >> 1, half = tid & 1;
-        const bool active = u < nu;
+        const bool active = FULL || u < nu;
         const int c = 8 * (ubase + u) + 4 * half;                // this thread's channels c .. c+3
         const uint32_t seg_off = 16u * u + 8u * half;            // their bytes in a ring row
 
@@ -269,9 +274,10 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
 
         // moments of this CTA's channels of stream row p about the row's
         // first element here: (sum d, sum d^2) for this thread's channels
-        auto moments = [&](int stage, int g, int p, float& m1, float& m2) {
+        auto moments = [&](auto inner_tag, int stage, int g, int p, float& m1, float& m2) {
+            constexpr bool INNER = decltype(inner_tag)::value;   // p is a loaded row
             m1 = m2 = 0.f;
-            if (active && p >= 0 && p < p_load) {
+            if (active && (INNER || (p >= 0 && p < p_load))) {
                 const uint8_t* row = ring_x(stage, g);
                 const f2 x0 = f2_splat(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(row)));
                 const uint2 xv = *reinterpret_cast<const uint2*>(row + seg_off);
@@ -436,20 +442,27 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
 
         // dx of the output rows of stage s (their g, xhat in fin)
         auto finish = [&](int s) {
+            auto one = [&](int g, int q) {
+                const float rstd = st_ring[(q - p_s) & (kStRing - 1)].y;
+                const float2 mt = tot[(s & 1) * kG + g];
+                const f2 rs = f2_splat(rstd), na = f2_splat(-rstd * mt.x), nb = f2_splat(-rstd * mt.y);
+                const float* fp = fin_at(s & 1, g);
+                const float4 g4 = *reinterpret_cast<const float4*>(fp);
+                const float4 h4 = *reinterpret_cast<const float4*>(fp + 4);
+                const f2 o0 = f2_fma(f2_make(h4.x, h4.y), nb, f2_fma(f2_make(g4.x, g4.y), rs, na));
+                const f2 o1 = f2_fma(f2_make(h4.z, h4.w), nb, f2_fma(f2_make(g4.z, g4.w), rs, na));
+                *reinterpret_cast<uint2*>(a.dx + (row0 + q) * D + c) = make_uint2(f2_to_bf16x2(o0), f2_to_bf16x2(o1));
+            };
+            const int q0 = p_s + s * kG - 3;
+            if (q0 >= t_b && q0 + kG <= t_e) {     // every row of the stage is an output row
+                if (active) {
 #pragma unroll
-            for (int g = 0; g < kG; ++g) {
-                const int q = p_s + s * kG + g - 3;
-                if (q >= t_b && q < t_e && active) {
-                    const float rstd = st_ring[(q - p_s) & (kStRing - 1)].y;
-                    const float2 mt = tot[(s & 1) * kG + g];
-                    const f2 rs = f2_splat(rstd), na = f2_splat(-rstd * mt.x), nb = f2_splat(-rstd * mt.y);
-                    const float* fp = fin_at(s & 1, g);
-                    const float4 g4 = *reinterpret_cast<const float4*>(fp);
-                    const float4 h4 = *reinterpret_cast<const float4*>(fp + 4);
-                    const f2 o0 = f2_fma(f2_make(h4.x, h4.y), nb, f2_fma(f2_make(g4.x, g4.y), rs, na));
-                    const f2 o1 = f2_fma(f2_make(h4.z, h4.w), nb, f2_fma(f2_make(g4.z, g4.w), rs, na));
-                    *reinterpret_cast<uint2*>(a.dx + (row0 + q) * D + c) = make_uint2(f2_to_bf16x2(o0), f2_to_bf16x2(o1));
+                    for (int g = 0; g < kG; ++g) one(g, q0 + g);
                 }
+            } else {
+#pragma unroll
+                for (int g = 0; g < kG; ++g)
+                    if (q0 + g >= t_b && q0 + g < t_e && active) one(g, q0 + g);
             }
         };
 
@@ -461,7 +474,7 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
 #pragma unroll
             for (int i = 0; i < 2 * kG; ++i) {
                 const int p = p_s + i;
-                if (!failed) moments(i / kG, i % kG, p, v[i], v[2 * kG + i]);
+                if (!failed) moments(std::false_type{}, i / kG, i % kG, p, v[i], v[2 * kG + i]);
                 else v[i] = v[2 * kG + i] = 0.f;
             }
             const float r = warp_reduce16(v, lane);
@@ -527,42 +540,48 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
                 }
             }
             mbar_arrive(freeb + slot);          // this worker is done with the stage's rows
-            if (!ln) {
+            if constexpr (!LN) {
                 if (workers_or_bwd(failed, nwork)) {
                     failed = true;
                     break;
                 }
-                continue;
-            }
-
-            // moments of the rows two stages ahead, the g sums of this stage
-            float v[16];
+            } else {
+                // moments of the rows two stages ahead, the g sums of this stage
+                float v[16];
+    #pragma unroll
+                for (int i = 0; i < 2 * kG; ++i) v[i] = gs[i];
+                    const int pm = pos0 + 2 * kG;           // the rows of stage s + 2
+                if (!failed && s + 2 < S && pm >= 0 && pm + kG <= p_load) {
 #pragma unroll
-            for (int i = 0; i < 2 * kG; ++i) v[i] = gs[i];
+                    for (int g = 0; g < kG; ++g)
+                        moments(std::true_type{}, s + 2, g, pm + g, v[2 * kG + g], v[3 * kG + g]);
+                } else {
 #pragma unroll
-            for (int g = 0; g < kG; ++g) {
-                if (!failed && s + 2 < S) moments(s + 2, g, pos0 + 2 * kG + g, v[2 * kG + g], v[3 * kG + g]);
-                else v[2 * kG + g] = v[3 * kG + g] = 0.f;
+                    for (int g = 0; g < kG; ++g) {
+                        if (!failed && s + 2 < S) moments(std::false_type{}, s + 2, g, pm + g, v[2 * kG + g], v[3 * kG + g]);
+                        else v[2 * kG + g] = v[3 * kG + g] = 0.f;
+                    }
+                }
+                float* rd = red + (s & 1) * nwarps * 16;
+                const float r = warp_reduce16(v, lane);
+                if ((lane & 1) == 0) rd[warp * 16 + (lane >> 1)] = r;
+                if (workers_or_bwd(failed, nwork)) {
+                    failed = true;
+                    break;
+                }
+                arm(s + 1);
+                if (tid < 16) {
+                    float t = 0.f;
+                    for (int w = 0; w < nwarps; ++w) t += rd[w * 16 + tid];
+                    push(s + 1, tid, t);
+                } else if (tid < kMsg) {
+                    // every message is kMsg values (the arm counts them): the
+                    // first elements of the rows two stages ahead, then zeros
+                    const int g = tid - 16;
+                    push(s + 1, tid, (g < kG && s + 2 < S) ? first_x(s + 2, g, pos0 + 2 * kG + g) : 0.f);
+                }
+                if (s >= 1) finish(s - 1);
             }
-            float* rd = red + (s & 1) * nwarps * 16;
-            const float r = warp_reduce16(v, lane);
-            if ((lane & 1) == 0) rd[warp * 16 + (lane >> 1)] = r;
-            if (workers_or_bwd(failed, nwork)) {
-                failed = true;
-                break;
-            }
-            arm(s + 1);
-            if (tid < 16) {
-                float t = 0.f;
-                for (int w = 0; w < nwarps; ++w) t += rd[w * 16 + tid];
-                push(s + 1, tid, t);
-            } else if (tid < kMsg) {
-                // every message is kMsg values (the arm counts them): the
-                // first elements of the rows two stages ahead, then zeros
-                const int g = tid - 16;
-                push(s + 1, tid, (g < kG && s + 2 < S) ? first_x(s + 2, g, pos0 + 2 * kG + g) : 0.f);
-            }
-            if (s >= 1) finish(s - 1);
         }
         // the last stage's output rows
         if (ln && !failed && S > 0) {
@@ -674,10 +693,20 @@ gla_status launch_conv_bwd(const void* x, int apply_ln, const float* g, const fl
     const int CL = D <= 2048 ? 2 : 4;
     const bool aff = g || be || bias;
     void (*kernel)(BwdArgs);
-    if (CL == 2)
-        kernel = aff ? ln_conv_silu_bwd_kernel<true, 2, kBwdThreads> : ln_conv_silu_bwd_kernel<false, 2, kBwdThreads>;
-    else
-        kernel = aff ? ln_conv_silu_bwd_kernel<true, 4, kBwdThreads> : ln_conv_silu_bwd_kernel<false, 4, kBwdThreads>;
+    const bool ln = apply_ln != 0;
+    const int P = D / 8;
+    const bool full = P % CL == 0 && (2 * (P / CL)) % 32 == 0;
+    // the 16 forms: affine or not, LayerNorm or not, every thread owning
+    // channels or not, 2 or 4 CTAs a cluster
+    using KFn = void (*)(BwdArgs);
+#define GLA_BWD_FORM(A, N, F) {ln_conv_silu_bwd_kernel<A, N, F, 2, kBwdThreads>, ln_conv_silu_bwd_kernel<A, N, F, 4, kBwdThreads>}
+    static const KFn forms[2][2][2][2] = {
+        {{GLA_BWD_FORM(false, false, false), GLA_BWD_FORM(false, false, true)},
+         {GLA_BWD_FORM(false, true, false), GLA_BWD_FORM(false, true, true)}},
+        {{GLA_BWD_FORM(true, false, false), GLA_BWD_FORM(true, false, true)},
+         {GLA_BWD_FORM(true, true, false), GLA_BWD_FORM(true, true, true)}}};
+#undef GLA_BWD_FORM
+    kernel = forms[aff][ln][full][CL == 4];
     BwdPlan pl = plan_bwd(B, T, D, sms / CL);
     const BwdSmem L(pl.upc, pl.threads - 32);
     const size_t smem = L.total;

@@ -114,9 +114,11 @@ __device__ __forceinline__ float2 row_moments(const uint8_t* row, int D, float e
 // LayerNorm affine or a conv bias is given (otherwise their registers are
 // not needed).
 constexpr int CH = 8;
-template <bool AFF, int MAXT>
+// LN: the LayerNorm is applied (a template parameter, so that the row loop
+// holds no test of it).
+template <bool AFF, bool LN, int MAXT>
 __global__ void __launch_bounds__(MAXT, 1)
-ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
+ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x,
                     const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
                     const float* __restrict__ w, const float* __restrict__ bias,
                     const float* __restrict__ cs_in, float* __restrict__ cs_out,
@@ -217,7 +219,7 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
         if (!failed && !mbar_wait(full + slot, (s / stages) & 1, ctl)) failed = true;
         const uint8_t* st = ring + slot * kG * row_bytes;
         float2* sst = stats + slot * kG;
-        if (apply_ln && !failed)
+        if (LN && !failed)
             for (int g = warp; g < rows; g += nwarps) {
                 const float2 m = row_moments(st + g * row_bytes, D, eps, lane);
                 if (lane == 0) sst[g] = m;
@@ -237,7 +239,7 @@ ln_conv_silu_kernel(const __nv_bfloat16* __restrict__ x, int apply_ln,
                 const uint32_t* xw = reinterpret_cast<const uint32_t*>(&xv);
 #pragma unroll
                 for (int i = 0; i < NP; ++i) xn[i] = f2_from_bf16x2(xw[i]);
-                if (apply_ln) {
+                if constexpr (LN) {
                     const float2 m = sst[g];
                     if constexpr (AFF) {
                         const f2 mu = f2_splat(m.x), rs = f2_splat(m.y);
@@ -332,14 +334,19 @@ gla_status launch_conv(const void* x, int apply_ln, const float* g, const float*
     if (stages < 2) stages = 2;
     const size_t smem = stages * stage_bytes + fixed;
     const bool aff = g || b || bias;
-    auto kernel = threads <= 416 ? (aff ? ln_conv_silu_kernel<true, 416> : ln_conv_silu_kernel<false, 416>)
-                                 : (aff ? ln_conv_silu_kernel<true, 544> : ln_conv_silu_kernel<false, 544>);
+    using KFn = decltype(&ln_conv_silu_kernel<true, true, 416>);
+    static const KFn forms[2][2][2] = {
+        {{ln_conv_silu_kernel<false, false, 416>, ln_conv_silu_kernel<false, false, 544>},
+         {ln_conv_silu_kernel<false, true, 416>, ln_conv_silu_kernel<false, true, 544>}},
+        {{ln_conv_silu_kernel<true, false, 416>, ln_conv_silu_kernel<true, false, 544>},
+         {ln_conv_silu_kernel<true, true, 416>, ln_conv_silu_kernel<true, true, 544>}}};
+    auto kernel = forms[aff][apply_ln != 0][threads > 416];
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return check_launch("cudaFuncSetAttribute");
     dim3 grid(nx, B);
     trace_begin(st);
-    kernel<<<grid, threads, smem, st>>>(static_cast<const __nv_bfloat16*>(x), apply_ln, g, b, eps, w,
+    kernel<<<grid, threads, smem, st>>>(static_cast<const __nv_bfloat16*>(x), g, b, eps, w,
                                         bias, cs_in, cs_out, static_cast<__nv_bfloat16*>(y), T, D, per,
                                         stages, ctl);
     trace_end(st, "ln_conv_silu_kernel");

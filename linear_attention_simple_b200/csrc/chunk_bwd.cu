@@ -27,6 +27,7 @@
 //      from state_dot_kernel when dS_T is given), restarted every 16 chunks
 //      from the closed form <dS_a, S_a> (da_anchor_kernel).
 #include <cstring>
+#include <type_traits>
 
 #include "chunk_state.cuh"
 
@@ -367,19 +368,31 @@ __global__ void __launch_bounds__(bqp::kThreads, 1) bwd_dqdk_persistent_kernel(c
                     uint32_t r[32];
                     tmem_ld32(tq + col, r);
                     tmem_ld_wait();
+                    // one loop per path (factorised or exact) and gradient, so
+                    // that no element computes the factor of the other path
+                    auto convert = [&](auto role_tag, auto fast_tag) {
+                        constexpr bool DK = decltype(role_tag)::value, FAST = decltype(fast_tag)::value;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        float v[2];
+                        for (int e = 0; e < 32; e += 2) {
+                            float v[2];
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int cc = c0 + e + u;
-                            const bool keep = role ? (cc >= row) : (cc <= row);
-                            const float f = fast ? cfs[cc] : p.scale * exp2f(role ? bz[cc] - b2r : b2r - bz[cc]);
-                            v[u] = keep ? __uint_as_float(r[e + u]) * f : 0.f;
+                            for (int u = 0; u < 2; ++u) {
+                                const int cc = c0 + e + u;
+                                const bool keep = DK ? (cc >= row) : (cc <= row);
+                                const float f = FAST ? cfs[cc] : p.scale * exp2f(DK ? bz[cc] - b2r : b2r - bz[cc]);
+                                v[u] = keep ? __uint_as_float(r[e + u]) * f : 0.f;
+                            }
+                            const uint32_t hv = pack_bf16(v[0], v[1]);
+                            hi[e / 2] = hv;
+                            lo[e / 2] = pack_bf16(v[0] - bf16_lo(hv), v[1] - bf16_hi(hv));
                         }
-                        const uint32_t hv = pack_bf16(v[0], v[1]);
-                        hi[e / 2] = hv;
-                        lo[e / 2] = pack_bf16(v[0] - bf16_lo(hv), v[1] - bf16_hi(hv));
+                    };
+                    if (role) {
+                        if (fast) convert(std::true_type{}, std::true_type{});
+                        else convert(std::true_type{}, std::false_type{});
+                    } else {
+                        if (fast) convert(std::false_type{}, std::true_type{});
+                        else convert(std::false_type{}, std::false_type{});
                     }
                 }
                 tmem_st16(tq + col, hi);
@@ -705,21 +718,27 @@ __global__ void __launch_bounds__(dvp::kThreads, 1) bwd_dv_kernel(const __grid_c
                 uint32_t r[32];
                 tmem_ld32(tq + col, r);
                 tmem_ld_wait();
+                // one loop per path, so that no element computes the other's factor
+                auto conv = [&](auto fast_tag) {
+                    constexpr bool FAST = decltype(fast_tag)::value;
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int i = i0 + e;
-                    float v0, v1;
-                    if (fast) {
-                        v0 = (i >= row) ? __uint_as_float(r[e]) * cf[i] : 0.f;
-                        v1 = (i + 1 >= row) ? __uint_as_float(r[e + 1]) * cf[i + 1] : 0.f;
-                    } else {
-                        v0 = (i >= row) ? p.scale * __uint_as_float(r[e]) * exp2f(b2[i] - b2j) : 0.f;
-                        v1 = (i + 1 >= row) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2[i + 1] - b2j) : 0.f;
+                    for (int e = 0; e < 32; e += 2) {
+                        const int i = i0 + e;
+                        float v0, v1;
+                        if constexpr (FAST) {
+                            v0 = (i >= row) ? __uint_as_float(r[e]) * cf[i] : 0.f;
+                            v1 = (i + 1 >= row) ? __uint_as_float(r[e + 1]) * cf[i + 1] : 0.f;
+                        } else {
+                            v0 = (i >= row) ? p.scale * __uint_as_float(r[e]) * exp2f(b2[i] - b2j) : 0.f;
+                            v1 = (i + 1 >= row) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2[i + 1] - b2j) : 0.f;
+                        }
+                        const uint32_t hv = pack_bf16(v0, v1);
+                        hi[e / 2] = hv;
+                        lo[e / 2] = pack_bf16(v0 - bf16_lo(hv), v1 - bf16_hi(hv));
                     }
-                    const uint32_t hv = pack_bf16(v0, v1);
-                    hi[e / 2] = hv;
-                    lo[e / 2] = pack_bf16(v0 - bf16_lo(hv), v1 - bf16_hi(hv));
-                }
+                };
+                if (fast) conv(std::true_type{});
+                else conv(std::false_type{});
             }
             tmem_st16(tq + col, hi);
             tmem_st16(tq + col + 16, lo);

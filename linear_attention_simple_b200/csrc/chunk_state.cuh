@@ -55,6 +55,8 @@
 // memory and returns with GLA_ERR_TIMEOUT recorded.
 #pragma once
 
+#include <type_traits>
+
 #include "gla_device.cuh"
 
 namespace gla {
@@ -666,21 +668,29 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                     uint32_t r[32];
                     tmem_ld32(tq + col, r);
                     tmem_ld_wait();
+                    // one loop per path, so that no element computes the
+                    // other path's factor
+                    auto conv = [&](auto fast_tag) {
+                        constexpr bool FAST = decltype(fast_tag)::value;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int j = j0 + e;
-                        float v0, v1;
-                        if (fast) {
-                            v0 = (j <= tok) ? __uint_as_float(r[e]) * cfc[j] : 0.f;
-                            v1 = (j + 1 <= tok) ? __uint_as_float(r[e + 1]) * cfc[j + 1] : 0.f;
-                        } else {
-                            v0 = (j <= tok) ? p.scale * __uint_as_float(r[e]) * exp2f(b2r - b2c[j]) : 0.f;
-                            v1 = (j + 1 <= tok) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2r - b2c[j + 1]) : 0.f;
+                        for (int e = 0; e < 32; e += 2) {
+                            const int j = j0 + e;
+                            float v0, v1;
+                            if constexpr (FAST) {
+                                v0 = (j <= tok) ? __uint_as_float(r[e]) * cfc[j] : 0.f;
+                                v1 = (j + 1 <= tok) ? __uint_as_float(r[e + 1]) * cfc[j + 1] : 0.f;
+                            } else {
+                                v0 = (j <= tok) ? p.scale * __uint_as_float(r[e]) * exp2f(b2r - b2c[j]) : 0.f;
+                                v1 = (j + 1 <= tok) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2r - b2c[j + 1])
+                                                    : 0.f;
+                            }
+                            const uint32_t hv = pack_bf16(v0, v1);
+                            hi[e / 2] = hv;
+                            lo[e / 2] = pack_bf16(v0 - bf16_lo(hv), v1 - bf16_hi(hv));
                         }
-                        const uint32_t hv = pack_bf16(v0, v1);
-                        hi[e / 2] = hv;
-                        lo[e / 2] = pack_bf16(v0 - bf16_lo(hv), v1 - bf16_hi(hv));
-                    }
+                    };
+                    if (fast) conv(std::true_type{});
+                    else conv(std::false_type{});
                 }
                 tmem_st16(tq + col, hi);
                 tmem_st16(tq + col + 16, lo);

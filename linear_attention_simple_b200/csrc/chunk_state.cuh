@@ -47,9 +47,9 @@
 // SW128 boxes ([3][128][64], MN-major B); state copies are [3][96][64] SW128;
 // P tiles are [2][128][64] SW128 (K-major A).
 //
-// Threads: warps 0-7 are workers (warp w reads TMEM lanes 32*(w%4) .. +31,
-// column half (w/4)); warp 8 only issues TMA copies and tcgen05.mma, so the
-// workers never stall behind the tensor core's issue queue.  Every wait is
+// Threads: warps 0-15 are workers (warp w reads TMEM lanes 32*(w%4) .. +31,
+// column quarter w/4); warp 16 only issues tcgen05.mma, so the workers never
+// stall behind the tensor core's issue queue, and warp 17 the TMA copies.  Every wait is
 // bounded; on timeout the CTA stops at the next block-wide barrier, drains
 // its in-flight copies and tensor-core work (bounded), frees its tensor
 // memory and returns with GLA_ERR_TIMEOUT recorded.
@@ -100,7 +100,10 @@ struct StateParams {
 namespace chunk {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kWorkers = 256;
+// fused forward: 16 worker warps, warp w on TMEM lane quarter w % 4 and
+// column quarter w / 4 (of the 128 score, 192 output and state columns)
+constexpr int kWorkerWarps = 16;
+constexpr int kWorkers = kWorkerWarps * 32;
 constexpr int kThreads = kWorkers + 32;
 constexpr int kFusedThreads = kThreads + 32;   // + a producer warp
 // state pass: 16 warps; w % 4 < 3 for w < 15 are the 12 workers (TMEM lanes
@@ -255,87 +258,78 @@ __device__ __forceinline__ float chunk_cumsum(float a, float* wsum, int warp, in
     return x + pre;
 }
 
-// Load a [96][192] fp32 state (row `row`, columns half*96 .. +95) into TMEM.
+// This thread's NCOL columns of its row of a [96][192] fp32 state (src
+// points at the first; null = zeros) into TMEM.
+template <int NCOL>
 __device__ __forceinline__ void state_to_tmem(const float* src, uint32_t taddr)
 {
 #pragma unroll
-    for (int j = 0; j < 3; ++j) {
-        uint32_t r[32];
+    for (int j = 0; j < NCOL / 16; ++j) {
+        uint32_t r[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-            const float4 v = src ? *reinterpret_cast<const float4*>(src + j * 32 + e)
+        for (int e = 0; e < 16; e += 4) {
+            const float4 v = src ? *reinterpret_cast<const float4*>(src + j * 16 + e)
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
             r[e] = __float_as_uint(v.x);
             r[e + 1] = __float_as_uint(v.y);
             r[e + 2] = __float_as_uint(v.z);
             r[e + 3] = __float_as_uint(v.w);
         }
-        tmem_st32(taddr + j * 32, r);
+        tmem_st16(taddr + j * 16, r);
     }
     tmem_st_wait();
 }
 
+template <int NCOL>
 __device__ __forceinline__ void tmem_to_state(uint32_t taddr, float* dst)
 {
+    uint32_t r[NCOL / 16][16];
 #pragma unroll
-    for (int j = 0; j < 3; ++j) {
-        uint32_t r[32];
-        tmem_ld32(taddr + j * 32, r);
-        tmem_ld_wait();
+    for (int j = 0; j < NCOL / 16; ++j) tmem_ld16(taddr + j * 16, r[j]);
+    tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + j * 32 + e) =
-                make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                            __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
-    }
+    for (int j = 0; j < NCOL / 16; ++j)
+#pragma unroll
+        for (int e = 0; e < 16; e += 4)
+            *reinterpret_cast<float4*>(dst + j * 16 + e) =
+                make_float4(__uint_as_float(r[j][e]), __uint_as_float(r[j][e + 1]),
+                            __uint_as_float(r[j][e + 2]), __uint_as_float(r[j][e + 3]));
 }
 
-// State copy into [3][96][64] SW128 (row = dk index, n = dv column), for the
-// 96 columns half*96 .. +95 of this thread's row; then decay the state.
-// With gsave, the same 96 values also go to global memory as a bf16 hi plane
-// (gsave) and lo plane (gsave + plane_bytes), 32-byte stores.
-template <bool SPLIT>
-__device__ __forceinline__ void state_copy_and_decay(uint32_t taddr, int row, int half, float f,
-                                                     uint8_t* hi, uint8_t* lo, bool copy,
+// State copy into [3][96][64] SW128 (row = dk index, n = dv column) of this
+// thread's NCOL columns col0 .. col0+NCOL-1 of its row; then decay the state
+// in TMEM by f.  With gsave, the same values also go to global memory as a
+// bf16 hi plane (gsave) and lo plane (gsave + plane_bytes), 32-byte stores.
+template <int NCOL>
+__device__ __forceinline__ void state_copy_and_decay(uint32_t taddr, int row, int col0, float f, uint8_t* copy,
                                                      uint8_t* gsave = nullptr, int64_t plane_bytes = 0)
 {
+    uint32_t r[NCOL / 16][16];
 #pragma unroll
-    for (int j = 0; j < 3; ++j) {
-        uint32_t r[32];
-        tmem_ld32(taddr + j * 32, r);
-        tmem_ld_wait();
+    for (int j = 0; j < NCOL / 16; ++j) tmem_ld16(taddr + j * 16, r[j]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < NCOL / 16; ++j) {
         if (gsave) {
+            uint32_t w[8], l[8];
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                uint32_t w[8], l[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float x0 = __uint_as_float(r[16 * h2 + 2 * e]), x1 = __uint_as_float(r[16 * h2 + 2 * e + 1]);
-                    w[e] = pack_bf16(x0, x1);
-                    l[e] = pack_bf16(x0 - bf16_lo(w[e]), x1 - bf16_hi(w[e]));
-                }
-                st_global_v8(gsave + j * 64 + h2 * 32, w);
-                st_global_v8(gsave + plane_bytes + j * 64 + h2 * 32, l);
+            for (int e = 0; e < 8; ++e) {
+                const float x0 = __uint_as_float(r[j][2 * e]), x1 = __uint_as_float(r[j][2 * e + 1]);
+                w[e] = pack_bf16(x0, x1);
+                l[e] = pack_bf16(x0 - bf16_lo(w[e]), x1 - bf16_hi(w[e]));
             }
-        }
-        if (copy) {
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                const int n = half * 96 + j * 32 + q4 * 8;
-                const uint32_t off = (n >> 6) * 12288 + swz_off(row, (n & 63) >> 3, 128);
-                if (SPLIT) {
-                    uint4 h, l;
-                    pack8_split(r + q4 * 8, h, l);
-                    *reinterpret_cast<uint4*>(hi + off) = h;
-                    *reinterpret_cast<uint4*>(lo + off) = l;
-                } else {
-                    *reinterpret_cast<uint4*>(hi + off) = pack8(r + q4 * 8);
-                }
-            }
+            st_global_v8(gsave + j * 32, w);
+            st_global_v8(gsave + plane_bytes + j * 32, l);
         }
 #pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
-        tmem_st32(taddr + j * 32, r);
+        for (int h8 = 0; h8 < 2; ++h8) {
+            const int n = col0 + j * 16 + h8 * 8;
+            *reinterpret_cast<uint4*>(copy + (n >> 6) * 12288 + swz_off(row, (n & 63) >> 3, 128)) =
+                pack8(r[j] + h8 * 8);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) r[j][e] = __float_as_uint(__uint_as_float(r[j][e]) * f);
+        tmem_st16(taddr + j * 16, r[j]);
     }
     tmem_st_wait();
 }
@@ -408,11 +402,12 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     const int quad = warp & 3;
     const int row = quad * 32 + lane;         // TMEM lane = tile row (permuted token order)
     const int tok = row_token(row);           // token of this row
-    const int half = (warp >> 2) & 1;
-    const bool worker = warp < 8;
+    const int cq = warp >> 2;                 // column quarter (workers)
+    constexpr int kOC = kDv / 4;              // output and state columns per worker: 48
+    const bool worker = warp < kWorkerWarps;
     const bool srow = worker && quad < 3;
-    const bool issuer = warp == 8 && lane == 0;
-    const bool producer = warp == 9 && lane == 0;   // TMA loads and o stores; outside the loop's barriers
+    const bool issuer = warp == kWorkerWarps && lane == 0;
+    const bool producer = warp == kWorkerWarps + 1 && lane == 0;   // TMA loads and o stores; outside the loop's barriers
     // largest token among this lane quarter's rows (columns beyond it are masked)
     const int quad_max_tok = max(perm16(2 * quad), perm16(2 * quad + 1)) * 16 + 15;
 
@@ -451,7 +446,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     auto save_row = [&](int c) -> uint8_t* {
         if (VARLEN || !p.h_save || !GLA_DCHECK(c < p.NC && unit < p.B * p.H, p.ctl.status)) return nullptr;
         return static_cast<uint8_t*>(p.h_save) + ((static_cast<int64_t>(unit) * p.NC + c) * 2) * kStatePlane +
-               static_cast<int64_t>(row) * (kDv * 2) + half * 192;
+               static_cast<int64_t>(row) * (kDv * 2) + cq * (kOC * 2);
     };
     // cumulative log2-decay of a chunk and its column factors (warps 0-3)
     auto decays = [&](float av, int par) {
@@ -472,19 +467,19 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     if (nchunks > 0) decays(tid < 128 ? load_a(c_begin) : 0.f, 0);
     if (srow) {
         const float* src = p.s_init ? p.s_init + unit * p.init_unit_stride + seg * p.init_seg_stride +
-                                          row * kDv + half * 96
+                                          row * kDv + cq * kOC
                                     : nullptr;
         if (VARLEN && seg > 0)    // a later segment of a sequence: the state the combine left for it
             src = p.seg_states + (varlen_slot(p.cu_seqlens, b, seg, cps) * p.H + h) * (kDk * kDv) +
-                  row * kDv + half * 96;
-        state_to_tmem(src, tq + L::TM_S + half * 96);
+                  row * kDv + cq * kOC;
+        state_to_tmem<kOC>(src, tq + L::TM_S + cq * kOC);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (nchunks > 0 && srow)
-        state_copy_and_decay<false>(tq + L::TM_S + half * 96, row, half, exp2f(b2s[127]), sm + L::X, nullptr,
-                                    true, save_row(c_begin), kStatePlane);
+        state_copy_and_decay<kOC>(tq + L::TM_S + cq * kOC, row, cq * kOC, exp2f(b2s[127]), sm + L::X,
+                                  save_row(c_begin), kStatePlane);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -567,7 +562,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     uint32_t ph_q = 0, ph_u = 0, ph_y[2] = {0u, 0u};
     int n_sc = 0, n_d = 0, n_fo = 0;          // commits (issuer)
     bool failed = false, aborted = false;
-    for (int it = 0; warp < 9 && it < nchunks; ++it) {
+    for (int it = 0; warp <= kWorkerWarps && it < nchunks; ++it) {
         const int c = c_begin + it;
         const int ys = it & 1, par = it & 1;
         const uint32_t ya = ys ? L::Y1 : L::Y0;
@@ -621,7 +616,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         }
         fence_async_smem();
         tc_fence_before();
-        if (bar_or(2, 288, failed)) { aborted = true; break; }
+        if (bar_or(2, kThreads, failed)) { aborted = true; break; }
         tc_fence_after();
 
         // (D) O = Q S_prev, S += K~^T V (K~ as hi + lo)
@@ -656,9 +651,8 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         if (worker) {
             const float b2r = b2c[tok];
             if (fast) rf = p.scale * exp2f(b2r);
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                const int j0 = half * 64 + q2 * 32;
+            {
+                const int j0 = cq * 32;               // this warp's 32-token block
                 const uint32_t col = L::TM_SC + j0;
                 uint32_t hi[16], lo[16];
                 if (j0 > quad_max_tok) {
@@ -698,7 +692,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             tmem_st_wait();
         }
         tc_fence_before();
-        if (bar_or(2, 288, failed)) { aborted = true; break; }
+        if (bar_or(2, kThreads, failed)) { aborted = true; break; }
 
         // (F) O += P V with P from tensor memory
         if (issuer) {
@@ -723,8 +717,8 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             if (!failed && !mbar_wait(bar_d, it & 1, ctl)) failed = true;
             tc_fence_after();
             if (srow && !failed)
-                state_copy_and_decay<false>(tq + L::TM_S + half * 96, row, half, exp2f(b2s[(par ^ 1) * 128 + 127]),
-                                            sm + L::X, nullptr, true, save_row(c + 1), kStatePlane);
+                state_copy_and_decay<kOC>(tq + L::TM_S + cq * kOC, row, cq * kOC, exp2f(b2s[(par ^ 1) * 128 + 127]),
+                                          sm + L::X, save_row(c + 1), kStatePlane);
             fence_async_smem();
         }
 
@@ -737,25 +731,26 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             const bool direct = VARLEN && c * 128 + 128 > Tn;
             const bool mine = VARLEN && tok < Tn - c * 128;
             uint8_t* orow = VARLEN ? static_cast<uint8_t*>(p.o_direct) +
-                                         ((static_cast<int64_t>(tb) + c * 128 + tok) * p.H + h) * (kDv * 2) + half * 192
+                                         ((static_cast<int64_t>(tb) + c * 128 + tok) * p.H + h) * (kDv * 2) + cq * (kOC * 2)
                                    : nullptr;
             if (!failed) {
                 uint8_t* stg = sm + ya;
+                uint32_t r[kOC / 16][16];
 #pragma unroll
-                for (int j = 0; j < 3; ++j) {
-                    uint32_t r[32];
-                    tmem_ld32(tq + L::TM_O + half * 96 + j * 32, r);
-                    tmem_ld_wait();
+                for (int j = 0; j < kOC / 16; ++j) tmem_ld16(tq + L::TM_O + cq * kOC + j * 16, r[j]);
+                tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * rf);
+                for (int j = 0; j < kOC / 16; ++j) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int n = half * 96 + j * 32 + q4 * 8;
+                    for (int e = 0; e < 16; ++e) r[j][e] = __float_as_uint(__uint_as_float(r[j][e]) * rf);
+#pragma unroll
+                    for (int h8 = 0; h8 < 2; ++h8) {
+                        const int n = cq * kOC + j * 16 + h8 * 8;
                         if (!direct)
                             *reinterpret_cast<uint4*>(stg + (n >> 6) * 16384 + swz_off(tok, (n & 63) >> 3, 128)) =
-                                pack8(r + q4 * 8);
+                                pack8(r[j] + h8 * 8);
                         else if (mine && GLA_DCHECK(tb + c * 128 + tok < p.T, p.ctl.status))
-                            *reinterpret_cast<uint4*>(orow + (j * 32 + q4 * 8) * 2) = pack8(r + q4 * 8);
+                            *reinterpret_cast<uint4*>(orow + (j * 16 + h8 * 8) * 2) = pack8(r[j] + h8 * 8);
                     }
                 }
                 fence_async_smem();
@@ -766,12 +761,12 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         a_nx = a_next;
     }
 
-    if (!aborted && warp < 9) {
+    if (!aborted && warp <= kWorkerWarps) {
         // all MMAs are done (the epilogue waited for the last P V): S is final
         const bool write_state = p.s_out && (!p.out_last_only || seg == last_seg);
         if (write_state && srow && !failed && GLA_DCHECK(unit < p.B * p.H, p.ctl.status))
-            tmem_to_state(tq + L::TM_S + half * 96,
-                          p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + half * 96);
+            tmem_to_state<kOC>(tq + L::TM_S + cq * kOC,
+                               p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + cq * kOC);
     }
     if (issuer) {
         // every commit's arrival has landed before the barriers go away: at

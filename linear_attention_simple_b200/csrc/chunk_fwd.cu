@@ -321,7 +321,7 @@ gla_status run_chunk_fwd_varlen(const ChunkProblem& pr, const int* cu_seqlens, i
     StateParams p;
     memset(&p, 0, sizeof(p));
     gla_status s;
-    if ((s = make_token_map(&p.tm_q, pr.q, kDk, pr.H, pr.T, 1, pr.ld_qk, 32, 64, 16)) != GLA_OK) return s;
+    if ((s = make_token_map(&p.tm_q, pr.q, kDk, pr.H, pr.T, 1, pr.ld_qk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&p.tm_u, pr.k, kDk, pr.H, pr.T, 1, pr.ld_qk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&p.tm_y, pr.v, kDv, pr.H, pr.T, 1, pr.ld_v, 64, 128)) != GLA_OK) return s;
     if ((s = make_token_map(&p.tm_o, o, kDv, pr.H, pr.T, 1, static_cast<int64_t>(pr.H) * kDv, 64, 128)) != GLA_OK)
@@ -406,7 +406,7 @@ gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float
     StateParams p;
     memset(&p, 0, sizeof(p));
     gla_status s;
-    if ((s = make_token_map(&p.tm_q, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64, 16)) != GLA_OK) return s;
+    if ((s = make_token_map(&p.tm_q, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&p.tm_u, pr.k, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&p.tm_y, pr.v, kDv, pr.H, pr.T, pr.B, pr.ld_v, 64, 128)) != GLA_OK) return s;
     if ((s = make_token_map(&p.tm_o, o, kDv, pr.H, pr.T, pr.B, static_cast<int64_t>(pr.H) * kDv, 64, 128)) != GLA_OK)

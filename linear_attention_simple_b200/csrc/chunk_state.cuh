@@ -25,9 +25,11 @@
 //   per-element exponential or scaled copy of Q is needed.  Chunks with a
 //   steeper decay take the exact per-element path (P_ij with 2^{b_i - b_j},
 //   Q scaled by scale e^{b_i} in place, r_i = 1).
-//   The rows of the Q tile are permuted in 16-row blocks so that each of
-//   the four TMEM lane quarters (each owned by one SM sub-partition) gets an
-//   equal share of the causal triangle.
+//   Q tile row i = token i (natural order, three TMA boxes per tile: each
+//   TMA instruction costs the issuing thread about 90 cycles, so the tile is
+//   loaded in as few boxes as its swizzle allows).  Each worker warp converts
+//   one 32-token block of P, so the causal triangle's imbalance between
+//   lane quarters costs at most one block per warp.
 //
 // gla_state_pass_kernel<REVERSE> -- state only: S (or D) = e^gamma S + U~^T Y
 //   per chunk with U~ split into bf16 hi + lo, optionally storing the bf16
@@ -62,7 +64,7 @@
 namespace gla {
 
 struct StateParams {
-    CUtensorMap tm_q;       // q tile loads, 16-row boxes (fused forward)
+    CUtensorMap tm_q;       // q tile loads (fused forward)
     CUtensorMap tm_u;       // scaled operand: k (forward) or q (reverse)
     CUtensorMap tm_y;
     CUtensorMap tm_o;       // o tile stores (fused forward)       // v (forward) or dO (reverse)
@@ -121,7 +123,7 @@ constexpr uint32_t kIdStateTs = idesc_bf16_f32(128, 192, 0, 1);   // A from tens
 
 // Shared-memory maps (bytes from a 1024-aligned base).
 struct FusedSmem {
-    static constexpr uint32_t Q = 0;          // q tile, permuted rows
+    static constexpr uint32_t Q = 0;          // q tile
     static constexpr uint32_t U = 24576;      // k tile, then K~ (its 4th M block is X: finite)
     static constexpr uint32_t X = 49152;      // bf16 state copy [3][96][64] SW128
     static constexpr uint32_t KL = 86016;     // lo half of K~ [3][128][32] SW64 (hi: K~ in place in U)
@@ -150,13 +152,6 @@ __device__ __forceinline__ int64_t varlen_slot(const int* cu, int n, int s, int 
 {
     return static_cast<int64_t>(n) + cu[n] / (128 * chunks_per_seg) + s;
 }
-
-// Token held by row r of the permuted q tile: 16-row block r/16 holds token
-// block perm16(r/16) (0, 7, 1, 6, 2, 5, 3, 4), so lane quarter q (rows
-// 32q..32q+31) holds token blocks {q, 7-q} and every quarter has the same
-// number of causal (i, j) pairs.
-__device__ __forceinline__ int perm16(int blk) { return (0x43526170u >> (4 * blk)) & 15; }
-__device__ __forceinline__ int row_token(int r) { return perm16(r >> 4) * 16 + (r & 15); }
 
 __device__ __forceinline__ void named_sync(int id, int n)
 {
@@ -400,8 +395,8 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     const WaitCtl ctl = p.ctl;
 
     const int quad = warp & 3;
-    const int row = quad * 32 + lane;         // TMEM lane = tile row (permuted token order)
-    const int tok = row_token(row);           // token of this row
+    const int row = quad * 32 + lane;         // TMEM lane = tile row = token in the chunk
+    const int tok = row;
     const int cq = warp >> 2;                 // column quarter (workers)
     constexpr int kOC = kDv / 4;              // output and state columns per worker: 48
     const bool worker = warp < kWorkerWarps;
@@ -409,7 +404,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     const bool issuer = warp == kWorkerWarps && lane == 0;
     const bool producer = warp == kWorkerWarps + 1 && lane == 0;   // TMA loads and o stores; outside the loop's barriers
     // largest token among this lane quarter's rows (columns beyond it are masked)
-    const int quad_max_tok = max(perm16(2 * quad), perm16(2 * quad + 1)) * 16 + 15;
+    const int quad_max_tok = quad * 32 + 31;
 
     if (issuer) {
         mbar_init(bar_q, 1);
@@ -492,10 +487,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         auto issue_qu = [&](int c) {
             const int t0 = c * 128;
             mbar_arrive_expect_tx(bar_q, kTileQK);
-            for (int i = 0; i < 3; ++i)
-                for (int r16 = 0; r16 < 8; ++r16)
-                    tma_load_4d(sm + L::Q + i * 8192 + r16 * 1024, &p.tm_q, bar_q, i * 32, h,
-                                tb + t0 + perm16(r16) * 16, bc);
+            for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::Q + i * 8192, &p.tm_q, bar_q, i * 32, h, tb + t0, bc);
             mbar_arrive_expect_tx(bar_u, kTileQK);
             for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::U + i * 8192, &p.tm_u, bar_u, i * 32, h, tb + t0, bc);
         };
@@ -504,8 +496,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         auto prefetch_qu = [&](int c) {
             const int t0 = c * 128;
             for (int i = 0; i < 3; ++i) {
-                for (int r16 = 0; r16 < 8; ++r16)
-                    tma_prefetch_l2_4d(&p.tm_q, i * 32, h, tb + t0 + r16 * 16, bc);
+                tma_prefetch_l2_4d(&p.tm_q, i * 32, h, tb + t0, bc);
                 tma_prefetch_l2_4d(&p.tm_u, i * 32, h, tb + t0, bc);
             }
         };
@@ -595,7 +586,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
 
         // (C) K~ = e^{gamma - b} K as a bf16 pair: hi in place, lo (K~ - hi) in
         // KL, so that the state update keeps the fp32 state's precision; on
-        // the exact path also Q~ = scale e^{b} Q (rows in permuted token order)
+        // the exact path also Q~ = scale e^{b} Q
         if (worker && !failed && !mbar_wait(bar_sc, it & 1, ctl)) failed = true;
         if (!failed && worker) {
             const int live = Tn - c * 128;   // varlen: rows past the sequence (the next one's) add nothing
@@ -610,7 +601,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                 *(reinterpret_cast<uint4*>(sm + L::KL + blk * 8192 + r * 64) + ch) = lo;
                 if (!fast) {
                     uint4* qq = reinterpret_cast<uint4*>(sm + L::Q + blk * 8192 + r * 64) + ch;
-                    *qq = scale8(*qq, p.scale * exp2f(b2c[row_token(r)]));
+                    *qq = scale8(*qq, p.scale * exp2f(b2c[r]));
                 }
             }
         }

@@ -44,8 +44,9 @@ struct BwdParams {
     CUtensorMap tm_q, tm_k;                // q, k tiles (32-column SW64 boxes)
     CUtensorMap tm_dq, tm_dk;              // gradient stores
     // 32-column SW64 boxes: dO, v, dv; per-chunk states [units*NC][2][96][192]
-    // (plane 0 hi, plane 1 lo) h and D
-    CUtensorMap tm_do32, tm_v32, tm_dv32, tm_h32, tm_d32;
+    // (plane 0 hi, plane 1 lo) h and D: tm_h2, tm_d2 load a state's two
+    // planes in one box, tm_d32 one plane
+    CUtensorMap tm_do32, tm_v32, tm_dv32, tm_h2, tm_d2, tm_d32;
     const float* a;
     float* delta;                          // [B*H, T]: q.dq per token (role 0), k.dk (role 1) after it
     float* ctot;                           // [B*H, NC, 2]: chunk totals of both halves
@@ -206,8 +207,8 @@ __global__ void __launch_bounds__(bqp::kThreads, 1) bwd_dqdk_persistent_kernel(c
         tma_prefetch_desc(&p.tm_k);
         tma_prefetch_desc(&p.tm_do32);
         tma_prefetch_desc(&p.tm_v32);
-        tma_prefetch_desc(&p.tm_h32);
-        tma_prefetch_desc(&p.tm_d32);
+        tma_prefetch_desc(&p.tm_h2);
+        tma_prefetch_desc(&p.tm_d2);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -230,10 +231,8 @@ __global__ void __launch_bounds__(bqp::kThreads, 1) bwd_dqdk_persistent_kernel(c
             mbar_arrive_expect_tx(bar_full + slot, kSliceBytes);
             tma_load_4d(base, &p.tm_do32, bar_full + slot, sl * 32, w.h, t0, w.b);
             tma_load_4d(base + S_V, &p.tm_v32, bar_full + slot, sl * 32, w.h, t0, w.b);
-            tma_load_3d(base + S_HH, &p.tm_h32, bar_full + slot, sl * 32, 0, si);
-            tma_load_3d(base + S_HL, &p.tm_h32, bar_full + slot, sl * 32, 0, si + 1);
-            tma_load_3d(base + S_DH, &p.tm_d32, bar_full + slot, sl * 32, 0, si);
-            tma_load_3d(base + S_DL, &p.tm_d32, bar_full + slot, sl * 32, 0, si + 1);
+            tma_load_3d(base + S_HH, &p.tm_h2, bar_full + slot, sl * 32, 0, si);   // hi, then lo at S_HL
+            tma_load_3d(base + S_DH, &p.tm_d2, bar_full + slot, sl * 32, 0, si);   // hi, then lo at S_DL
             ++n_full[slot];
             ++sidx;
             return true;
@@ -1109,7 +1108,8 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     if ((s = make_token_map(&bp.tm_do32, dO, kDv, pr.H, pr.T, pr.B, ldo, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&bp.tm_dv32, dv, kDv, pr.H, pr.T, pr.B, ldo, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&bp.tm_v32, pr.v, kDv, pr.H, pr.T, pr.B, pr.ld_v, 32, 64)) != GLA_OK) return s;
-    if ((s = make_state_map(&bp.tm_h32, hbuf, static_cast<int64_t>(units) * NC * 2, 32)) != GLA_OK) return s;
+    if ((s = make_state_map(&bp.tm_h2, hbuf, static_cast<int64_t>(units) * NC * 2, 32, 2)) != GLA_OK) return s;
+    if ((s = make_state_map(&bp.tm_d2, dbuf, static_cast<int64_t>(units) * NC * 2, 32, 2)) != GLA_OK) return s;
     if ((s = make_state_map(&bp.tm_d32, dbuf, static_cast<int64_t>(units) * NC * 2, 32)) != GLA_OK) return s;
     bp.a = pr.a;
     bp.delta = delta;

@@ -156,13 +156,14 @@ gla_status make_token_map(CUtensorMap* m, const void* base, int d, int H, int T,
     return make_tmap(m, base, 4, dims, strides, box, 2, swizzle);
 }
 
-gla_status make_state_map(CUtensorMap* m, void* base, int64_t nstates, int box_cols)
+gla_status make_state_map(CUtensorMap* m, void* base, int64_t nstates, int box_cols, int box_states)
 {
     const uint64_t dims[3] = {static_cast<uint64_t>(kDv), static_cast<uint64_t>(kDk),
                               static_cast<uint64_t>(nstates)};
     const uint64_t strides[3] = {2, static_cast<uint64_t>(kDv) * 2,
                                  static_cast<uint64_t>(kDk) * kDv * 2};
-    const uint32_t box[3] = {static_cast<uint32_t>(box_cols), static_cast<uint32_t>(kDk), 1};
+    const uint32_t box[3] = {static_cast<uint32_t>(box_cols), static_cast<uint32_t>(kDk),
+                             static_cast<uint32_t>(box_states)};
     return make_tmap(m, base, 3, dims, strides, box, 2, box_cols * 2);
 }
 

@@ -128,7 +128,9 @@ gla_status launch_state_fold(const float* s, const float* g, int n, int units, i
 struct StateParams;   // chunk_state.cuh
 gla_status make_token_map(CUtensorMap* m, const void* base, int d, int H, int T, int B,
                           int64_t ld, int box_d, int swizzle, int box_rows = 128);
-gla_status make_state_map(CUtensorMap* m, void* base, int64_t nstates, int box_cols = 64);
+// [nstates][96][192] bf16 states; a box is box_states consecutive states
+// (e.g. a state's hi and lo planes) of box_cols columns.
+gla_status make_state_map(CUtensorMap* m, void* base, int64_t nstates, int box_cols = 64, int box_states = 1);
 gla_status launch_state_kernel(bool with_o, bool reverse, const StateParams& p, dim3 grid,
                                cudaStream_t st);
 

@@ -422,6 +422,10 @@ gla_status run_chunk_fwd(const ChunkProblem& pr, const float* s0, void* o, float
     p.ctl = ctl;
     p.store_h = 0;
     p.h_save = h_save;
+    // the hi plane of each saved state goes out from the kernel's bf16 state
+    // copy ([3][96][64] SW128 in shared memory) by TMA
+    if (h_save && (s = make_state_map(&p.tm_h, h_save, static_cast<int64_t>(units) * NC * 2, 64)) != GLA_OK)
+        return s;
 
     if (nseg == 1) {
         p.s_init = s0;

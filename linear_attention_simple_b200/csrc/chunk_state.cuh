@@ -67,7 +67,8 @@ struct StateParams {
     CUtensorMap tm_q;       // q tile loads (fused forward)
     CUtensorMap tm_u;       // scaled operand: k (forward) or q (reverse)
     CUtensorMap tm_y;
-    CUtensorMap tm_o;       // o tile stores (fused forward)       // v (forward) or dO (reverse)
+    CUtensorMap tm_o;       // o tile stores (fused forward)
+    CUtensorMap tm_h;       // saved states, 64-column boxes of one plane (fused forward with h_save)       // v (forward) or dO (reverse)
     const float* a;         // [B, T, H] log-decay
     const float* s_init;    // initial state per (unit, seg) or null (zeros)
     float* s_out;           // state after the segment, or null
@@ -293,11 +294,11 @@ __device__ __forceinline__ void tmem_to_state(uint32_t taddr, float* dst)
 
 // State copy into [3][96][64] SW128 (row = dk index, n = dv column) of this
 // thread's NCOL columns col0 .. col0+NCOL-1 of its row; then decay the state
-// in TMEM by f.  With gsave, the same values also go to global memory as a
-// bf16 hi plane (gsave) and lo plane (gsave + plane_bytes), 32-byte stores.
+// in TMEM by f.  The same values also go to global memory as a bf16 hi plane
+// (ghi) and lo plane (glo, the remainder), 32-byte stores, where given.
 template <int NCOL>
 __device__ __forceinline__ void state_copy_and_decay(uint32_t taddr, int row, int col0, float f, uint8_t* copy,
-                                                     uint8_t* gsave = nullptr, int64_t plane_bytes = 0)
+                                                     uint8_t* ghi = nullptr, uint8_t* glo = nullptr)
 {
     uint32_t r[NCOL / 16][16];
 #pragma unroll
@@ -305,7 +306,7 @@ __device__ __forceinline__ void state_copy_and_decay(uint32_t taddr, int row, in
     tmem_ld_wait();
 #pragma unroll
     for (int j = 0; j < NCOL / 16; ++j) {
-        if (gsave) {
+        if (ghi || glo) {
             uint32_t w[8], l[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -313,8 +314,8 @@ __device__ __forceinline__ void state_copy_and_decay(uint32_t taddr, int row, in
                 w[e] = pack_bf16(x0, x1);
                 l[e] = pack_bf16(x0 - bf16_lo(w[e]), x1 - bf16_hi(w[e]));
             }
-            st_global_v8(gsave + j * 32, w);
-            st_global_v8(gsave + plane_bytes + j * 32, l);
+            if (ghi) st_global_v8(ghi + j * 32, w);
+            if (glo) st_global_v8(glo + j * 32, l);
         }
 #pragma unroll
         for (int h8 = 0; h8 < 2; ++h8) {
@@ -355,6 +356,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     uint64_t* bar_fo = bar_q + 6;                                // O += P V done
     uint64_t* bar_stg = bar_q + 7;                               // [2] o staged in the v buffer (256)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_q + 9);
+    uint64_t* bar_xfree = bar_q + 10;                            // the saved-state store has read X
     float* b2s = reinterpret_cast<float*>(sm + L::MISC + 128);  // [2][128] by token, chunk parity
     float* cfac = b2s + 256;                                     // [2][128] 2^{-b_j}
     float* wsum = cfac + 256;                                    // [4]
@@ -416,11 +418,13 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         mbar_init(bar_fo, 1);
         mbar_init(bar_stg, kWorkers);
         mbar_init(bar_stg + 1, kWorkers);
+        mbar_init(bar_xfree, 1);
         mbar_init_fence();
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_u);
         tma_prefetch_desc(&p.tm_y);
         tma_prefetch_desc(&p.tm_o);
+        if (p.h_save) tma_prefetch_desc(&p.tm_h);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, L::TMEM_COLS);
@@ -443,6 +447,9 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         return static_cast<uint8_t*>(p.h_save) + ((static_cast<int64_t>(unit) * p.NC + c) * 2) * kStatePlane +
                static_cast<int64_t>(row) * (kDv * 2) + cq * (kOC * 2);
     };
+    // saved states: the lo plane from the workers' registers, the hi plane
+    // from the bf16 copy X by the producer's TMA store
+    const bool tma_save = !VARLEN && p.h_save != nullptr;
     // cumulative log2-decay of a chunk and its column factors (warps 0-3)
     auto decays = [&](float av, int par) {
         if (tid < 128) {
@@ -472,9 +479,11 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (nchunks > 0 && srow)
-        state_copy_and_decay<kOC>(tq + L::TM_S + cq * kOC, row, cq * kOC, exp2f(b2s[127]), sm + L::X,
-                                  save_row(c_begin), kStatePlane);
+    if (nchunks > 0 && srow) {
+        uint8_t* g = save_row(c_begin);
+        state_copy_and_decay<kOC>(tq + L::TM_S + cq * kOC, row, cq * kOC, exp2f(b2s[127]), sm + L::X, g,
+                                  g ? g + kStatePlane : nullptr);
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -533,10 +542,21 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                 for (int i = 0; i < 3; ++i) tma_store_4d(&p.tm_o, y + i * 16384, i * 64, h, tb + c * 128, bc);
                 tma_store_commit();
             }
-            if (it + 2 < nchunks) {
+            // the state entering chunk c+1, whose bf16 copy X the workers wrote
+            // before this epilogue, goes out as its saved hi plane
+            const bool save_x = tma_save && it + 1 < nchunks;
+            if (save_x) {
+                const int si = (unit * p.NC + c + 1) * 2;
+                for (int i = 0; i < 3; ++i) tma_store_3d(&p.tm_h, sm + L::X + i * 12288, i * 64, 0, si);
+                tma_store_commit();
+            }
+            if (it + 2 < nchunks || save_x) {
                 tma_store_wait_read();
-                issue_y(c + 2, ys);
-                ++n_y[ys];
+                if (save_x) mbar_arrive(bar_xfree);
+                if (it + 2 < nchunks) {
+                    issue_y(c + 2, ys);
+                    ++n_y[ys];
+                }
             }
         }
         tma_store_wait_all();
@@ -706,10 +726,14 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             decays(a_nx, par ^ 1);
             named_sync(3, kWorkers);             // the next chunk's total decay is in b2s
             if (!failed && !mbar_wait(bar_d, it & 1, ctl)) failed = true;
+            // the producer's store of the last copy has read X
+            if (!failed && tma_save && it >= 1 && !mbar_wait(bar_xfree, (it - 1) & 1, ctl)) failed = true;
             tc_fence_after();
-            if (srow && !failed)
+            if (srow && !failed) {
+                uint8_t* g = save_row(c + 1);
                 state_copy_and_decay<kOC>(tq + L::TM_S + cq * kOC, row, cq * kOC, exp2f(b2s[(par ^ 1) * 128 + 127]),
-                                          sm + L::X, save_row(c + 1), kStatePlane);
+                                          sm + L::X, tma_save ? nullptr : g, g ? g + kStatePlane : nullptr);
+            }
             fence_async_smem();
         }
 

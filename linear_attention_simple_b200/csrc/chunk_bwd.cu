@@ -1078,7 +1078,35 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
         if ((s = launch_state_kernel(false, false, sp, dim3(nseg, pr.H, pr.B), st)) != GLA_OK) return s;
     }
 
-    // 2. D_c for every chunk, dS_0 (written by segment 0, where the reverse sweep ends)
+    // 2. D_c for every chunk, dS_0 (written by segment 0, where the reverse sweep ends);
+    // with one segment per head the reverse sweep also yields dv: the fused
+    // forward kernel run backwards (k in q's place, q in k's, dO in v's, dv
+    // out), D_c saved as hi and lo planes like the forward's entering states
+    const bool rev_fused = nseg == 1;
+    if (rev_fused) {
+        StateParams fp;
+        memset(&fp, 0, sizeof(fp));
+        if ((s = make_token_map(&fp.tm_q, pr.k, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
+        if ((s = make_token_map(&fp.tm_u, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
+        if ((s = make_token_map(&fp.tm_y, dO, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
+        if ((s = make_token_map(&fp.tm_o, dv, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
+        if ((s = make_state_map(&fp.tm_h, dbuf, static_cast<int64_t>(units) * NC * 2, 64)) != GLA_OK) return s;
+        fp.a = pr.a;
+        fp.s_init = ds_final;
+        fp.init_unit_stride = kSS;
+        fp.s_out = ds0;
+        fp.out_unit_stride = kSS;
+        fp.out_last_only = 1;
+        fp.B = pr.B;
+        fp.T = pr.T;
+        fp.H = pr.H;
+        fp.NC = NC;
+        fp.chunks_per_seg = cps;
+        fp.h_save = dbuf;
+        fp.scale = pr.scale;
+        fp.ctl = ctl;
+        if ((s = launch_state_kernel(true, true, fp, dim3(1, pr.H, pr.B), st)) != GLA_OK) return s;
+    }
     StateParams rp = sp;
     if ((s = make_token_map(&rp.tm_u, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&rp.tm_y, dO, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
@@ -1086,16 +1114,16 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     rp.s_init = ds_final;
     rp.init_unit_stride = kSS;
     rp.init_seg_stride = 0;
-    if (nseg > 1) {
+    if (!rev_fused) {
         // local gradients of every segment (segment 0's is computed and not
         // used: its CTAs run beside the others')
         if ((s = pre_pass(rp, true, nseg, ds_final)) != GLA_OK) return s;
         rp.s_init = segst;
         rp.init_unit_stride = static_cast<int64_t>(nseg) * kSS;
         rp.init_seg_stride = kSS;
+        rp.s_out = ds0;
+        if ((s = launch_state_kernel(false, true, rp, dim3(nseg, pr.H, pr.B), st)) != GLA_OK) return s;
     }
-    rp.s_out = ds0;
-    if ((s = launch_state_kernel(false, true, rp, dim3(nseg, pr.H, pr.B), st)) != GLA_OK) return s;
 
     // 3. dq, dk (+ per-token delta halves and chunk totals) and dv
     BwdParams bp;
@@ -1130,7 +1158,7 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
                                    bqp::kThreads)) != GLA_OK)
             return s;
     }
-    {
+    if (!rev_fused) {
         // persistent: one CTA per SM over the (batch, head, chunk, dv half) items
         const int items = units * NC * 2;
         const int grid = items < sms ? items : sms;

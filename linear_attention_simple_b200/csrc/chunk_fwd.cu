@@ -171,9 +171,9 @@ gla_status launch_state_kernel(bool with_o, bool reverse, const StateParams& p, 
                                cudaStream_t st)
 {
     if (with_o && !reverse)
-        return p.cu_seqlens ? launch_chunk_kernel(gla_fwd_fused_kernel<true>, chunk::FusedSmem::BYTES,
+        return p.cu_seqlens ? launch_chunk_kernel(gla_fwd_fused_kernel<true, false>, chunk::FusedSmem::BYTES,
                                                   "chunk_fwd_varlen_kernel", p, grid, st, chunk::kFusedThreads)
-                            : launch_chunk_kernel(gla_fwd_fused_kernel<false>, chunk::FusedSmem::BYTES,
+                            : launch_chunk_kernel(gla_fwd_fused_kernel<false, false>, chunk::FusedSmem::BYTES,
                                                   "chunk_fwd_fused_kernel", p, grid, st, chunk::kFusedThreads);
     if (!with_o && !reverse)
         return launch_chunk_kernel(gla_state_pass_kernel<false>, chunk::PassSmem::BYTES,
@@ -181,7 +181,9 @@ gla_status launch_state_kernel(bool with_o, bool reverse, const StateParams& p, 
     if (!with_o && reverse)
         return launch_chunk_kernel(gla_state_pass_kernel<true>, chunk::PassSmem::BYTES,
                                    "chunk_state_rev_kernel", p, grid, st, chunk::kPassThreads);
-    return GLA_ERR_UNSUPPORTED;
+    // reverse sweep with the output fused in: the backward's D_c and dv
+    return launch_chunk_kernel(gla_fwd_fused_kernel<false, true>, chunk::FusedSmem::BYTES, "chunk_rev_fused_kernel",
+                               p, grid, st, chunk::kFusedThreads);
 }
 
 size_t fwd_workspace_bytes(int B, int T, int H)

@@ -339,7 +339,7 @@ __device__ __forceinline__ void state_copy_and_decay(uint32_t taddr, int row, in
 // =====================================================================
 // Fused forward.
 // =====================================================================
-template <bool VARLEN>
+template <bool VARLEN, bool REV>
 __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(const __grid_constant__ StateParams p)
 {
     using namespace chunk;
@@ -392,6 +392,10 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     if (VARLEN && seg > 0 && c_begin >= NCn) return;
     const int c_end = min(NCn, c_begin + cps);
     const int nchunks = c_end - c_begin;
+    // the chunk of step it: forward in order; the reverse sweep from the last
+    constexpr int dc = REV ? -1 : 1;          // chunk step
+    const int c_first = REV ? c_end - 1 : c_begin;
+    auto chunk_at = [c_first](int it) { return c_first + dc * it; };
     const int last_seg = VARLEN ? max(1, (NCn + cps - 1) / cps) - 1
                                 : static_cast<int>(gridDim.x) - 1;
     const WaitCtl ctl = p.ctl;
@@ -405,8 +409,9 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     const bool srow = worker && quad < 3;
     const bool issuer = warp == kWorkerWarps && lane == 0;
     const bool producer = warp == kWorkerWarps + 1 && lane == 0;   // TMA loads and o stores; outside the loop's barriers
-    // largest token among this lane quarter's rows (columns beyond it are masked)
-    const int quad_max_tok = quad * 32 + 31;
+    // this lane quarter's rows span tokens 32 quad .. +31: a 32-token column
+    // block past them (forward) or before them (reverse) is masked whole
+    const int quad_max_tok = quad * 32 + 31, quad_min_tok = quad * 32;
 
     if (issuer) {
         mbar_init(bar_q, 1);
@@ -450,12 +455,18 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     // saved states: the lo plane from the workers' registers, the hi plane
     // from the bf16 copy X by the producer's TMA store
     const bool tma_save = !VARLEN && p.h_save != nullptr;
-    // cumulative log2-decay of a chunk and its column factors (warps 0-3)
+    // cumulative log2-decay b of a chunk and its column factors (warps 0-3):
+    // 2^{-b_j} forward, scale 2^{b_i - gamma} in the reverse sweep
     auto decays = [&](float av, int par) {
         if (tid < 128) {
             const float x = chunk_cumsum(av, wsum, warp, lane);
             b2s[par * 128 + tid] = x;
-            cfac[par * 128 + tid] = exp2f(-x);
+            if constexpr (REV) {
+                const float g = ((wsum[0] + wsum[1]) + wsum[2]) + wsum[3];
+                cfac[par * 128 + tid] = p.scale * exp2f(x - g);
+            } else {
+                cfac[par * 128 + tid] = exp2f(-x);
+            }
         }
     };
 
@@ -465,8 +476,8 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         reinterpret_cast<uint4*>(sm + L::KL_PAD)[i] = make_uint4(0u, 0u, 0u, 0u);
 
     // prologue: decays and state copy of the first chunk
-    float a_nx = (tid < 128 && nchunks > 1) ? load_a(c_begin + 1) : 0.f;
-    if (nchunks > 0) decays(tid < 128 ? load_a(c_begin) : 0.f, 0);
+    float a_nx = (tid < 128 && nchunks > 1) ? load_a(chunk_at(1)) : 0.f;
+    if (nchunks > 0) decays(tid < 128 ? load_a(chunk_at(0)) : 0.f, 0);
     if (srow) {
         const float* src = p.s_init ? p.s_init + unit * p.init_unit_stride + seg * p.init_seg_stride +
                                           row * kDv + cq * kOC
@@ -480,7 +491,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     __syncthreads();
     tc_fence_after();
     if (nchunks > 0 && srow) {
-        uint8_t* g = save_row(c_begin);
+        uint8_t* g = save_row(chunk_at(0));
         state_copy_and_decay<kOC>(tq + L::TM_S + cq * kOC, row, cq * kOC, exp2f(b2s[127]), sm + L::X, g,
                                   g ? g + kStatePlane : nullptr);
     }
@@ -516,23 +527,23 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                 tma_load_4d(y + i * 16384, &p.tm_y, bar_y + s, i * 64, h, tb + c * 128, bc);
         };
         int n_qu = 0, n_y[2] = {0, 0};
-        if (nchunks > 1) prefetch_qu(c_begin + 1);
+        if (nchunks > 1) prefetch_qu(chunk_at(1));
         if (nchunks > 0) {
-            issue_qu(c_begin);
+            issue_qu(chunk_at(0));
             ++n_qu;
-            issue_y(c_begin, 0);
+            issue_y(chunk_at(0), 0);
             ++n_y[0];
             if (nchunks > 1) {
-                issue_y(c_begin + 1, 1);
+                issue_y(chunk_at(1), 1);
                 ++n_y[1];
             }
         }
         for (int it = 0; it < nchunks; ++it) {
-            const int c = c_begin + it, ys = it & 1;
-            if (it + 2 < nchunks) prefetch_qu(c + 2);
+            const int c = chunk_at(it), ys = it & 1;
+            if (it + 2 < nchunks) prefetch_qu(c + 2 * dc);
             if (it + 1 < nchunks) {
                 if (!mbar_wait(bar_d, it & 1, ctl)) break;
-                issue_qu(c + 1);
+                issue_qu(c + dc);
                 ++n_qu;
             }
             if (!mbar_wait(bar_stg + ys, (it >> 1) & 1, ctl)) break;
@@ -546,7 +557,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             // before this epilogue, goes out as its saved hi plane
             const bool save_x = tma_save && it + 1 < nchunks;
             if (save_x) {
-                const int si = (unit * p.NC + c + 1) * 2;
+                const int si = (unit * p.NC + c + dc) * 2;
                 for (int i = 0; i < 3; ++i) tma_store_3d(&p.tm_h, sm + L::X + i * 12288, i * 64, 0, si);
                 tma_store_commit();
             }
@@ -554,7 +565,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                 tma_store_wait_read();
                 if (save_x) mbar_arrive(bar_xfree);
                 if (it + 2 < nchunks) {
-                    issue_y(c + 2, ys);
+                    issue_y(c + 2 * dc, ys);
                     ++n_y[ys];
                 }
             }
@@ -574,7 +585,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     int n_sc = 0, n_d = 0, n_fo = 0;          // commits (issuer)
     bool failed = false, aborted = false;
     for (int it = 0; warp <= kWorkerWarps && it < nchunks; ++it) {
-        const int c = c_begin + it;
+        const int c = chunk_at(it);
         const int ys = it & 1, par = it & 1;
         const uint32_t ya = ys ? L::Y1 : L::Y0;
         const float* b2c = b2s + par * 128;
@@ -616,12 +627,14 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                 const int r = (idx >> 2) & 127, blk = idx >> 9, ch = idx & 3;
                 uint4* u = reinterpret_cast<uint4*>(sm + L::U + blk * 8192 + r * 64) + ch;
                 uint4 hi, lo;
-                scale8_split(*u, (!VARLEN || r < live) ? exp2f(g2 - b2c[r]) : 0.f, hi, lo);
+                // forward K~ = 2^{gamma - b} K; reverse Q~ = scale 2^{b} Q (in the U tile)
+                const float fu = REV ? p.scale * exp2f(b2c[r]) : exp2f(g2 - b2c[r]);
+                scale8_split(*u, (!VARLEN || r < live) ? fu : 0.f, hi, lo);
                 *u = hi;
                 *(reinterpret_cast<uint4*>(sm + L::KL + blk * 8192 + r * 64) + ch) = lo;
                 if (!fast) {
                     uint4* qq = reinterpret_cast<uint4*>(sm + L::Q + blk * 8192 + r * 64) + ch;
-                    *qq = scale8(*qq, p.scale * exp2f(b2c[r]));
+                    *qq = scale8(*qq, REV ? exp2f(g2 - b2c[r]) : p.scale * exp2f(b2c[r]));
                 }
             }
         }
@@ -661,12 +674,12 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         float rf = 1.0f;
         if (worker) {
             const float b2r = b2c[tok];
-            if (fast) rf = p.scale * exp2f(b2r);
+            if (fast) rf = REV ? exp2f(g2 - b2r) : p.scale * exp2f(b2r);
             {
                 const int j0 = cq * 32;               // this warp's 32-token block
                 const uint32_t col = L::TM_SC + j0;
                 uint32_t hi[16], lo[16];
-                if (j0 > quad_max_tok) {
+                if (REV ? j0 + 31 < quad_min_tok : j0 > quad_max_tok) {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
                 } else {
@@ -681,12 +694,20 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
                         for (int e = 0; e < 32; e += 2) {
                             const int j = j0 + e;
                             float v0, v1;
-                            if constexpr (FAST) {
+                            // causal: column j <= row (forward), j >= row (reverse)
+                            if constexpr (FAST && !REV) {
                                 v0 = (j <= tok) ? __uint_as_float(r[e]) * cfc[j] : 0.f;
                                 v1 = (j + 1 <= tok) ? __uint_as_float(r[e + 1]) * cfc[j + 1] : 0.f;
-                            } else {
+                            } else if constexpr (!REV) {
                                 v0 = (j <= tok) ? p.scale * __uint_as_float(r[e]) * exp2f(b2r - b2c[j]) : 0.f;
                                 v1 = (j + 1 <= tok) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2r - b2c[j + 1])
+                                                    : 0.f;
+                            } else if constexpr (FAST) {
+                                v0 = (j >= tok) ? __uint_as_float(r[e]) * cfc[j] : 0.f;
+                                v1 = (j + 1 >= tok) ? __uint_as_float(r[e + 1]) * cfc[j + 1] : 0.f;
+                            } else {
+                                v0 = (j >= tok) ? p.scale * __uint_as_float(r[e]) * exp2f(b2c[j] - b2r) : 0.f;
+                                v1 = (j + 1 >= tok) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2c[j + 1] - b2r)
                                                     : 0.f;
                             }
                             const uint32_t hv = pack_bf16(v0, v1);
@@ -718,7 +739,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             umma_commit(bar_fo);
             ++n_fo;
         }
-        const float a_next = (tid < 128 && it + 2 < nchunks) ? load_a(c + 2) : 0.f;
+        const float a_next = (tid < 128 && it + 2 < nchunks) ? load_a(c + 2 * dc) : 0.f;
 
         // (B) while P V runs: the next chunk's decays, then -- once (D) has
         // updated S and released the state copies -- its state copy and decay
@@ -730,7 +751,7 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
             if (!failed && tma_save && it >= 1 && !mbar_wait(bar_xfree, (it - 1) & 1, ctl)) failed = true;
             tc_fence_after();
             if (srow && !failed) {
-                uint8_t* g = save_row(c + 1);
+                uint8_t* g = save_row(c + dc);
                 state_copy_and_decay<kOC>(tq + L::TM_S + cq * kOC, row, cq * kOC, exp2f(b2s[(par ^ 1) * 128 + 127]),
                                           sm + L::X, tma_save ? nullptr : g, g ? g + kStatePlane : nullptr);
             }

@@ -82,8 +82,13 @@ def check_bwd(d, grads, units=None, dsT=None):
     (1, 257, 2, False, False),
     (3, 129, 5, True, False),
     (2, 640, 40, False, True),
+    (1, 1000, 80, True, True),
+    (2, 130, 40, True, False),
 ])
 def test_chunk_bwd_parity(B, T, H, s0, dsT):
+    """Small shapes run the backward in segments per head; from B*H = 74 up
+    (the last three cases, ragged T among them) one reverse sweep per head
+    also yields dv."""
     d = inputs.chunk_inputs(B, T, H, seed=200 + T + H, device="cuda", s0_std=0.1 if s0 else None,
                             with_dO=True)
     ds = inputs.randn((B, H, 96, 192), 300 + T, "cuda", std=0.1) if dsT else None
@@ -132,8 +137,9 @@ def test_chunk_bwd_training_full_tensor():
     check_bwd(d, grads)
 
 
+@pytest.mark.parametrize("B,T,H", [(2, 512, 2), (1, 300, 80)])
 @pytest.mark.parametrize("mean", [None, -8.0, 0.6])
-def test_chunk_bwd_strong_decay_and_no_decay(mean):
+def test_chunk_bwd_strong_decay_and_no_decay(mean, B, T, H):
     """Decays outside the workload distribution: a = 0 (no decay), a ~ -8 per
     token (every chunk's decay spans far more than 2^100, the kernels' exact
     path), and logsigmoid(N(0.6, 1)) (chunk decays between 2^-111 and 2^-93,
@@ -150,9 +156,9 @@ def test_chunk_bwd_strong_decay_and_no_decay(mean):
     one operand carried as a bf16 hi + lo pair (within 2^-17 of its value)
     summed in fp32, so the bound is max-abs <= 2^-15 (four such roundings) of
     the largest cancelling term (max |q.dq|, |k.dk|, |<dS_T, S_T>|); its rel
-    L2 is printed."""
-    B, T, H = 2, 512, 2
-    seed = 230 if mean is None else 231 + int(mean * 10)
+    L2 is printed.  B*H = 4 sweeps each head in segments, B*H = 80 in one
+    reverse sweep that also yields dv (ragged T = 300)."""
+    seed = (230 if mean is None else 231 + int(mean * 10)) + (500 if B * H >= 74 else 0)
     d = inputs.chunk_inputs(B, T, H, seed=seed, device="cuda", s0_std=0.1, with_dO=True)
     d["a"] = (torch.zeros_like(d["a"]) if mean is None
               else inputs.log_decay((B, T, H), seed, "cuda", mean=mean))

@@ -113,10 +113,10 @@ __device__ __forceinline__ uint32_t ts_hi(uint32_t base, int ks)
 // into the SM once, and the next chunk's loads run under this chunk's
 // conversion and epilogues.
 //
-//   producer warp   per chunk: dv slices 0..2 into the ring as slots free,
-//                   then Q and K once the previous chunk is done with them,
-//                   then slices 3..5; every slice carries dO, V and the
-//                   hi / lo planes of h and D (40 KB, six per chunk)
+//   producer warp   per chunk: the six dv slices into the ring as slots
+//                   free, then Q and K once the previous chunk is done with
+//                   them; every slice carries dO, V and the hi / lo planes
+//                   of h and D (40 KB)
 //   issuer thread   per slice: T_q += dO V^T, T_k += V dO^T, A_q += dO h^T
 //                   (hi, lo), A_k += V D^T (hi, lo); then, once the tiles
 //                   are converted and Q, K are in, A_q += dP K and
@@ -239,8 +239,11 @@ __global__ void __launch_bounds__(bqp::kThreads, 1) bwd_dqdk_persistent_kernel(c
         };
         for (int k = 0; ok && k < n; ++k) {
             const Item w = item(k);
-            for (int sl = 0; ok && sl < 3; ++sl) ok = load_slice(w, sl);
-            // q, k of this chunk once the previous chunk has read its tiles
+            // the slices first: they wait only for ring slots, and the slice
+            // MMAs need nothing else
+            for (int sl = 0; ok && sl < kSlices; ++sl) ok = load_slice(w, sl);
+            // q, k of this chunk (needed from the tile MMAs on) once the
+            // previous chunk's epilogue has read its tiles
             if (ok && k >= 1 && !mbar_wait(bar_free, (k - 1) & 1, ctl)) ok = false;
             if (ok) {
                 const int t0 = w.c * kChunk;
@@ -251,7 +254,6 @@ __global__ void __launch_bounds__(bqp::kThreads, 1) bwd_dqdk_persistent_kernel(c
                 }
                 ++n_qk;
             }
-            for (int sl = 3; ok && sl < kSlices; ++sl) ok = load_slice(w, sl);
         }
         // at most one load per barrier is ever outstanding
         for (int i = 0; i < kSlots; ++i)

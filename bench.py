@@ -78,7 +78,6 @@ METHOD_BYTES = {
     "chunk_state_fwd_kernel": QK + VO + A,              # k, v, a in
     "chunk_state_rev_kernel": QK + VO + A,              # q, dO, a in
     "bwd_dqdk_kernel": 2 * QK + 2 * VO + A + 2 * QK,    # q, k, v, dO, a in; dq, dk out
-    "bwd_dv_kernel": 2 * QK + VO + A + VO,              # q, k, dO, a in; dv out
     "chunk_rev_fused_kernel": 2 * QK + VO + A + VO,     # q, k, dO, a in; dv out (reverse sweep + dv)
     "da_finish_kernel": A,                              # da out
 }
@@ -90,7 +89,6 @@ DESIGN_BYTES = {
     "chunk_state_fwd_kernel": 2 * HS,                   # h_c written (hi, lo)
     "chunk_state_rev_kernel": 2 * HS,                   # D_c written (hi, lo)
     "bwd_dqdk_kernel": 2 * 2 * HS + 2 * A,              # h_c, D_c read (hi, lo); q.dq, k.dk written
-    "bwd_dv_kernel": HS,                                # D_c read (hi plane)
     "chunk_rev_fused_kernel": 2 * HS,                   # D_c written (hi, lo)
     "da_finish_kernel": 2 * A,                          # q.dq, k.dk read
 }
@@ -104,9 +102,7 @@ CHUNK_FLOPS = {
     "chunk_state_rev_kernel": MM(96, 192, 128),          # Q~^T dO
     # dP = dO V^T, dO h^T, dP K, V D^T, dP^T Q
     "bwd_dqdk_kernel": MM(128, 128, 192) + 2 * MM(128, 96, 192) + 2 * MM(128, 96, 128),
-    # scores^T K Q^T, P~ dO, K D
-    "bwd_dv_kernel": MM(128, 128, 96) + MM(128, 192, 128) + MM(128, 192, 96),
-    # the reverse sweep with dv fused in: K Q^T, K D, P~ dO, Q~^T dO
+    # the reverse sweep with dv fused in: scores^T K Q^T, K D, P~ dO, and Q~^T dO
     "chunk_rev_fused_kernel": MM(128, 128, 96) + MM(128, 192, 96) + MM(128, 192, 128) + MM(96, 192, 128),
 }
 # The whole training step per unit: forward (q, k, v, a in, o out) and
@@ -115,7 +111,7 @@ CHUNK_FLOPS = {
 # with both state scans, whichever kernel runs them).
 STEP_BYTES = (2 * QK + 2 * VO + A) + (2 * QK + 2 * VO + A + 2 * QK + VO + A)
 STEP_FLOPS = sum(CHUNK_FLOPS[k] for k in ("chunk_fwd_fused_kernel", "chunk_state_fwd_kernel",
-                                           "chunk_state_rev_kernel", "bwd_dqdk_kernel", "bwd_dv_kernel"))
+                                           "chunk_rev_fused_kernel", "bwd_dqdk_kernel"))
 
 
 # Source files each kernel is built from (the digest that ties a recorded
@@ -126,7 +122,6 @@ KERNEL_SOURCES = {
     "chunk_state_fwd_kernel": ("chunk_fwd.cu", "chunk_state.cuh", "gla_device.cuh"),
     "chunk_state_rev_kernel": ("chunk_fwd.cu", "chunk_state.cuh", "gla_device.cuh"),
     "bwd_dqdk_kernel": ("chunk_bwd.cu", "chunk_state.cuh", "gla_device.cuh"),
-    "bwd_dv_kernel": ("chunk_bwd.cu", "chunk_state.cuh", "gla_device.cuh"),
     "chunk_rev_fused_kernel": ("chunk_fwd.cu", "chunk_state.cuh", "gla_device.cuh"),
     "da_finish_kernel": ("chunk_bwd.cu",),
 }

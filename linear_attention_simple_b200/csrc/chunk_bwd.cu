@@ -17,12 +17,15 @@
 //   1. state kernel, forward, state-only: h_c for every chunk (bf16 hi + lo
 //      planes), and S_T when an upstream dS_T is given -- skipped when the
 //      forward kept the states (gla_chunk_fwd_train / gla_chunk_bwd_saved);
-//   2. state kernel, reverse: D_c for every chunk (hi + lo), dS_0 = D_{-1};
+//   2. the reverse sweep with dv fused in (the fused forward kernel run
+//      backwards, chunk_state.cuh): D_c for every chunk (hi + lo), dS_0 =
+//      D_{-1}, and dv = P^T dO + diag(e^{gamma - b}) K D (after a state-only
+//      reverse pre-pass and a fold when a head's chunks are cut into
+//      segments);
 //   3. bwd_dqdk_persistent_kernel (dq and dk of a chunk in one CTA, one CTA
-//      per SM) and bwd_dv_kernel (the halves of dv, one CTA per SM), tcgen05
-//      for every contraction; the masked, decayed dP / P tiles stay in tensor
-//      memory as bf16 hi + lo and feed the next MMA from there; the dq / dk
-//      epilogues also emit q.dq and k.dk per token and per chunk;
+//      per SM), tcgen05 for every contraction; the masked, decayed dP tiles
+//      stay in tensor memory as bf16 hi + lo and feed the next MMA from
+//      there; the epilogues also emit q.dq and k.dk per token and per chunk;
 //   4. da_finish_kernel: reverse cumulative sum over T (plus <dS_T, S_T>
 //      from state_dot_kernel when dS_T is given), restarted every 16 chunks
 //      from the closed form <dS_a, S_a> (da_anchor_kernel).
@@ -43,10 +46,9 @@ int num_chunks(int T) { return (T + kChunk - 1) / kChunk; }
 struct BwdParams {
     CUtensorMap tm_q, tm_k;                // q, k tiles (32-column SW64 boxes)
     CUtensorMap tm_dq, tm_dk;              // gradient stores
-    // 32-column SW64 boxes: dO, v, dv; per-chunk states [units*NC][2][96][192]
-    // (plane 0 hi, plane 1 lo) h and D: tm_h2, tm_d2 load a state's two
-    // planes in one box, tm_d32 one plane
-    CUtensorMap tm_do32, tm_v32, tm_dv32, tm_h2, tm_d2, tm_d32;
+    // 32-column SW64 boxes: dO, v; per-chunk states [units*NC][2][96][192]
+    // (plane 0 hi, plane 1 lo) h and D, a state's two planes in one box
+    CUtensorMap tm_do32, tm_v32, tm_h2, tm_d2;
     const float* a;
     float* delta;                          // [B*H, T]: q.dq per token (role 0), k.dk (role 1) after it
     float* ctot;                           // [B*H, NC, 2]: chunk totals of both halves
@@ -483,334 +485,6 @@ __global__ void __launch_bounds__(bqp::kThreads, 1) bwd_dqdk_persistent_kernel(c
     if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-// ----------------------------------------------------------------- dv kernel
-//
-// Work item = (batch, head, chunk, half of dv).  With gamma the chunk's
-// total log-decay:
-//
-//   dv_j = e^{gamma - b_j} ( sum_{i >= j} P~_ji dO_i + k_j D )
-//   P~_ji = scale e^{b_i - gamma} (k_j . q_i)          (factorised path)
-//
-// scores^T = K Q^T lands in TMEM with lanes = j; the workers turn it in place
-// into the bf16 hi and lo halves of P~ (the A operand of a tcgen05.mma
-// straight from tensor memory), and k_j D shares the accumulator because
-// both terms carry the same row factor.  Chunks whose decay spans more than
-// 2^100 take the exact path: P_ji = scale e^{b_i - b_j} (k_j . q_i), K rows
-// scaled by e^{gamma - b_j} in place before K D, row factor 1.
-//
-// TMEM tile layout of P~ for one lane: K (token i) block kb = i / 32 holds
-// the hi words in columns 32 kb .. +15 and the lo words in 32 kb + 16 .. +31
-// (two bf16 per 32-bit column, even index in the low half).
-//
-// Persistent: one CTA per SM walks the items blockIdx.x, + gridDim.x, ...
-// through two stages (shared-memory tiles and TMEM columns), so that item
-// k+1's loads and scores^T run while the workers convert item k and write
-// item k-1's dv:
-//   producer warp   load(k) into stage k%2 once dv(k-2) has consumed it
-//                   (q, k and the dv operands on two barriers)
-//   issuer thread   scores(k+1) after dv(k); dv(k) once P~(k) is in TMEM
-//   16 worker warps P~(k+1) (conversion), then the epilogue of item k
-//                   (row factor, bf16 staging, TMA store by worker 0)
-// Warp w of the workers reads TMEM lanes 32 (w % 4) .. +31 and column
-// quarter w / 4.  Worker-side waits on mbarriers are bounded and followed
-// by a barrier OR-reduction, so that all workers leave together on a timeout.
-
-namespace dvp {   // persistent dv kernel shared-memory map
-constexpr uint32_t STAGE = 92160;                  // per stage:
-constexpr uint32_t Q = 0, K = 24576, DO = 49152, DS = 73728;   // DO [3][128][32], DS [3][96][32] SW64
-constexpr uint32_t OUT = 2 * STAGE;                // dv staging [3][128][32] SW64
-constexpr uint32_t MISC = OUT + 24576;
-constexpr uint32_t BYTES = MISC + 3072 + 1024;
-constexpr uint32_t TMEM_COLS = 512;                // per stage 256: T at 0, DV (96 columns) at 128
-constexpr int kWorkerWarps = 16;
-constexpr int kWorkers = kWorkerWarps * 32;
-constexpr int kThreads = kWorkers + 64;            // + issuer warp + producer warp
-constexpr uint32_t kQkBytes = 2 * chunk::kTileQK;           // q, k tiles (scores^T)
-constexpr uint32_t kDdBytes = 24576 + 18432;                 // dO, D halves (dv)
-}  // namespace dvp
-
-__global__ void __launch_bounds__(dvp::kThreads, 1) bwd_dv_kernel(const __grid_constant__ BwdParams p)
-{
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-    const uint32_t sb = smem_u32(sm);
-    uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + dvp::MISC);   // [2] stage's q, k loaded
-    uint64_t* bar_g1 = bar_ld + 2;                                    // [2] scores^T done
-    uint64_t* bar_g2 = bar_ld + 4;                                    // [2] dv done: stage and T free
-    uint64_t* bar_cv = bar_ld + 6;                                    // [2] P~ in TMEM (all workers)
-    uint64_t* bar_dd = bar_ld + 8;                                    // [2] stage's dO, D loaded
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_ld + 10);
-    float* b2s = reinterpret_cast<float*>(sm + dvp::MISC + 128);      // [2][128] by stage
-    float* cfs = b2s + 256;                                           // [2][128] scale 2^{b_i - gamma}
-    float* wsum = cfs + 256;
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const bool worker = warp < dvp::kWorkerWarps;
-    const bool issuer = warp == dvp::kWorkerWarps && lane == 0;
-    const bool producer = warp == dvp::kWorkerWarps + 1 && lane == 0;
-    const int quad = warp & 3, colq = (warp >> 2) & 3, row = quad * 32 + lane;
-    const WaitCtl ctl = p.ctl;
-    const uint32_t idT = idesc_bf16_f32(128, 128, 0, 0);
-    const uint32_t idV = idesc_bf16_f32(128, 96, 0, 1);
-
-    const int total = p.B * p.H * p.NC * 2;
-    const int first = blockIdx.x, stride = gridDim.x;
-    const int n = first < total ? (total - first + stride - 1) / stride : 0;
-    struct Item {
-        int b, h, c, dvh, unit;
-    };
-    // chunk-major from the last chunk (the two halves of a chunk side by
-    // side): the dq / dk kernel before it ends on the last chunks, so the
-    // first items find their q, k, dO and D tiles still in L2
-    const int units = p.B * p.H;
-    auto item = [&](int k) {
-        const int it = total - 1 - (first + k * stride);
-        Item r;
-        r.c = it / (2 * units);
-        const int rem = it - r.c * 2 * units;
-        r.unit = rem >> 1;
-        r.dvh = rem & 1;
-        r.b = r.unit / p.H;
-        r.h = r.unit - r.b * p.H;
-        return r;
-    };
-
-    if (issuer) {
-        for (int i = 0; i < 6; ++i) mbar_init(bar_ld + i, 1);
-        mbar_init(bar_dd, 1);
-        mbar_init(bar_dd + 1, 1);
-        mbar_init(bar_cv, dvp::kWorkers);
-        mbar_init(bar_cv + 1, dvp::kWorkers);
-        mbar_init_fence();
-        tma_prefetch_desc(&p.tm_q);
-        tma_prefetch_desc(&p.tm_k);
-        tma_prefetch_desc(&p.tm_do32);
-        tma_prefetch_desc(&p.tm_d32);
-        tma_prefetch_desc(&p.tm_dv32);
-    }
-    if (warp == 0) {
-        tmem_alloc(tmem_slot, dvp::TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    if (producer) {
-        // ----------------------------------------------------------- loads
-        int n_ld[2] = {0, 0};
-        for (int k = 0; k < n; ++k) {
-            const int s = k & 1;
-            if (k >= 2 && !mbar_wait(bar_g2 + s, ((k - 2) >> 1) & 1, ctl)) break;
-            const Item w = item(k);
-            const int t0 = w.c * kChunk;
-            uint8_t* st = sm + s * dvp::STAGE;
-            // q, k first (the scores need only them), then the dv operands
-            mbar_arrive_expect_tx(bar_ld + s, dvp::kQkBytes);
-            for (int i = 0; i < 3; ++i) {
-                tma_load_4d(st + dvp::Q + i * 8192, &p.tm_q, bar_ld + s, i * 32, w.h, t0, w.b);
-                tma_load_4d(st + dvp::K + i * 8192, &p.tm_k, bar_ld + s, i * 32, w.h, t0, w.b);
-            }
-            mbar_arrive_expect_tx(bar_dd + s, dvp::kDdBytes);
-            for (int i = 0; i < 3; ++i) {
-                tma_load_4d(st + dvp::DO + i * 8192, &p.tm_do32, bar_dd + s, w.dvh * 96 + i * 32, w.h, t0, w.b);
-                tma_load_3d(st + dvp::DS + i * 6144, &p.tm_d32, bar_dd + s, w.dvh * 96 + i * 32, 0,
-                            (w.unit * p.NC + w.c) * 2);   // hi plane
-            }
-            ++n_ld[s];
-        }
-        // at most one load per stage and barrier is ever outstanding
-        for (int s = 0; s < 2; ++s)
-            if (n_ld[s]) {
-                mbar_wait(bar_ld + s, (n_ld[s] - 1) & 1, ctl);
-                mbar_wait(bar_dd + s, (n_ld[s] - 1) & 1, ctl);
-            }
-    } else if (issuer) {
-        // ------------------------------------------------------------ MMAs
-        int n_g1[2] = {0, 0}, n_g2[2] = {0, 0};
-        auto scores = [&](int k) {
-            const int s = k & 1;
-            if (!mbar_wait(bar_ld + s, (k >> 1) & 1, ctl)) return false;
-            tc_fence_after();
-            const uint32_t base = sb + s * dvp::STAGE;
-            const uint64_t dk = smem_desc(base + dvp::K, 16, 512, kLayoutSW64);
-            const uint64_t dq = smem_desc(base + dvp::Q, 16, 512, kLayoutSW64);
-#pragma unroll
-            for (int ks = 0; ks < 6; ++ks) {
-                const uint32_t off = (ks >> 1) * 8192 + (ks & 1) * 32;
-                umma_bf16(tmem + s * 256, desc_add(dk, off), desc_add(dq, off), idT, ks > 0);
-            }
-            umma_commit(bar_g1 + s);
-            ++n_g1[s];
-            return true;
-        };
-        bool ok = n > 0 ? scores(0) : true;
-        for (int k = 0; ok && k < n; ++k) {
-            const int s = k & 1;
-            if (!mbar_wait(bar_cv + s, (k >> 1) & 1, ctl) || !mbar_wait(bar_dd + s, (k >> 1) & 1, ctl)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            // dv = K~ D + P~ dO (K~ = K on the factorised path)
-            const uint32_t base = sb + s * dvp::STAGE;
-            const uint64_t dk = smem_desc(base + dvp::K, 16, 512, kLayoutSW64);
-            const uint64_t dd = smem_desc(base + dvp::DS, 6144, 512, kLayoutSW64);
-            const uint64_t dg = smem_desc(base + dvp::DO, 8192, 512, kLayoutSW64);
-            const uint32_t acc = tmem + s * 256 + 128;
-#pragma unroll
-            for (int ks = 0; ks < 6; ++ks)
-                umma_bf16(acc, desc_add(dk, (ks >> 1) * 8192 + (ks & 1) * 32), desc_add(dd, ks * 1024), idV, ks > 0);
-#pragma unroll
-            for (int part = 0; part < 2; ++part)
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    umma_bf16_ts(acc, tmem + s * 256 + ts_hi(0, ks) + 16 * part, desc_add(dg, ks * 1024), idV, 1);
-            umma_commit(bar_g2 + s);
-            ++n_g2[s];
-            if (k + 1 < n) ok = scores(k + 1);
-        }
-        // every commit's arrival has landed before the barriers go away
-        for (int s = 0; s < 2; ++s) {
-            if (n_g1[s]) mbar_wait(bar_g1 + s, (n_g1[s] - 1) & 1, ctl);
-            if (n_g2[s]) mbar_wait(bar_g2 + s, (n_g2[s] - 1) & 1, ctl);
-        }
-    } else if (worker) {
-        // --------------------------------------------------------- workers
-        const uint32_t tq = tmem_addr(tmem, quad * 32, 0);
-        auto load_a = [&](int k) {
-            if (tid >= 128 || k >= n) return 0.f;
-            const Item w = item(k);
-            const int t = w.c * kChunk + tid;
-            return t < p.T ? p.a[(static_cast<int64_t>(w.b) * p.T + t) * p.H + w.h] : 0.f;
-        };
-        // decays of item k into stage k%2 (the stage's previous item, k-2, has
-        // finished its epilogue: every worker passed the first barrier)
-        auto decays = [&](int k, float av) {
-            const int s = k & 1;
-            chunk::named_sync(2, dvp::kWorkers);
-            if (tid < 128) {
-                chunk_cumsum(av, b2s + s * 128, wsum, tid, warp, lane);
-                named_sync128();
-                cfs[s * 128 + tid] = p.scale * exp2f(b2s[s * 128 + tid] - b2s[s * 128 + 127]);
-            }
-            chunk::named_sync(2, dvp::kWorkers);
-        };
-        // P~ of item k in place in TMEM (and on the exact path K~ in place)
-        auto convert = [&](int k) {
-            const int s = k & 1;
-            const bool got = mbar_wait(bar_g1 + s, (k >> 1) & 1, ctl);
-            if (chunk::bar_or(2, dvp::kWorkers, !got)) return false;
-            tc_fence_after();
-            const float* b2 = b2s + s * 128;
-            const float* cf = cfs + s * 128;
-            const float g2 = b2[127];
-            const bool fast = -g2 <= chunk::kFactorRange;
-            const float b2j = b2[row];
-            const int i0 = colq * 32;
-            const uint32_t col = s * 256 + i0;
-            uint32_t hi[16], lo[16];
-            if (i0 + 31 < quad * 32) {            // every i < j here: masked
-#pragma unroll
-                for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
-            } else {
-                uint32_t r[32];
-                tmem_ld32(tq + col, r);
-                tmem_ld_wait();
-                // one loop per path, so that no element computes the other's factor
-                auto conv = [&](auto fast_tag) {
-                    constexpr bool FAST = decltype(fast_tag)::value;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int i = i0 + e;
-                        float v0, v1;
-                        if constexpr (FAST) {
-                            v0 = (i >= row) ? __uint_as_float(r[e]) * cf[i] : 0.f;
-                            v1 = (i + 1 >= row) ? __uint_as_float(r[e + 1]) * cf[i + 1] : 0.f;
-                        } else {
-                            v0 = (i >= row) ? p.scale * __uint_as_float(r[e]) * exp2f(b2[i] - b2j) : 0.f;
-                            v1 = (i + 1 >= row) ? p.scale * __uint_as_float(r[e + 1]) * exp2f(b2[i + 1] - b2j) : 0.f;
-                        }
-                        const uint32_t hv = pack_bf16(v0, v1);
-                        hi[e / 2] = hv;
-                        lo[e / 2] = pack_bf16(v0 - bf16_lo(hv), v1 - bf16_hi(hv));
-                    }
-                };
-                if (fast) conv(std::true_type{});
-                else conv(std::false_type{});
-            }
-            tmem_st16(tq + col, hi);
-            tmem_st16(tq + col + 16, lo);
-            tmem_st_wait();
-            if (!fast && tid < 384) {
-                // exact path: K rows scaled by e^{gamma - b_j} in place for K D
-                const int r = tid & 127, blk = tid >> 7;
-                chunk::scale_row_sw64(sm + s * dvp::STAGE + dvp::K, r, blk, exp2f(g2 - b2[r]));
-                fence_async_smem();
-            }
-            tc_fence_before();
-            mbar_arrive(bar_cv + s);
-            return true;
-        };
-        // dv_j = f_j acc_j -> bf16 staging [3][128][32] SW64 -> TMA store
-        auto epilogue = [&](int k) {
-            const int s = k & 1;
-            const bool got = mbar_wait(bar_g2 + s, (k >> 1) & 1, ctl);
-            if (tid == 0) tma_store_wait_read();      // the staging's previous store has read it
-            if (chunk::bar_or(2, dvp::kWorkers, !got)) return false;
-            tc_fence_after();
-            const float* b2 = b2s + s * 128;
-            const float g2 = b2[127];
-            const float f = -g2 <= chunk::kFactorRange ? exp2f(g2 - b2[row]) : 1.0f;
-            uint32_t u[3][8];
-#pragma unroll
-            for (int g = 0; g < 3; ++g) tmem_ld8(tq + s * 256 + 128 + colq * 24 + g * 8, u[g]);
-            tmem_ld_wait();
-#pragma unroll
-            for (int g = 0; g < 3; ++g) {
-                const int nn = colq * 24 + g * 8;
-                uint32_t pk[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    pk[e] = pack_bf16(f * __uint_as_float(u[g][2 * e]), f * __uint_as_float(u[g][2 * e + 1]));
-                *reinterpret_cast<uint4*>(sm + dvp::OUT + (nn >> 5) * 8192 + swz_off(row, (nn & 31) >> 3, 64)) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
-            fence_async_smem();
-            chunk::named_sync(2, dvp::kWorkers);
-            if (tid == 0) {
-                const Item w = item(k);
-                for (int i = 0; i < 3; ++i)
-                    tma_store_4d(&p.tm_dv32, sm + dvp::OUT + i * 8192, w.dvh * 96 + i * 32, w.h, w.c * kChunk, w.b);
-                tma_store_commit();
-            }
-            return true;
-        };
-
-        float a_next = load_a(0);
-        bool ok = true;
-        if (n > 0) {
-            decays(0, a_next);
-            a_next = load_a(1);
-            ok = convert(0);
-        }
-        for (int k = 0; ok && k < n; ++k) {
-            if (k + 1 < n) {
-                decays(k + 1, a_next);
-                a_next = load_a(k + 2);
-                if (!(ok = convert(k + 1))) break;
-            }
-            ok = epilogue(k);
-        }
-        if (tid == 0) tma_store_wait_all();
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, dvp::TMEM_COLS);
-}
-
 // ------------------------------------------------------------------ da
 //
 // da_t = sum_{m >= t} (q_m . dq_m - k_m . dk_m) + <dS_T, S_T>.  One CTA of
@@ -1080,54 +754,47 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
         if ((s = launch_state_kernel(false, false, sp, dim3(nseg, pr.H, pr.B), st)) != GLA_OK) return s;
     }
 
-    // 2. D_c for every chunk, dS_0 (written by segment 0, where the reverse sweep ends);
-    // with one segment per head the reverse sweep also yields dv: the fused
-    // forward kernel run backwards (k in q's place, q in k's, dO in v's, dv
-    // out), D_c saved as hi and lo planes like the forward's entering states
-    const bool rev_fused = nseg == 1;
-    if (rev_fused) {
-        StateParams fp;
-        memset(&fp, 0, sizeof(fp));
-        if ((s = make_token_map(&fp.tm_q, pr.k, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
-        if ((s = make_token_map(&fp.tm_u, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
-        if ((s = make_token_map(&fp.tm_y, dO, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
-        if ((s = make_token_map(&fp.tm_o, dv, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
-        if ((s = make_state_map(&fp.tm_h, dbuf, static_cast<int64_t>(units) * NC * 2, 64)) != GLA_OK) return s;
-        fp.a = pr.a;
-        fp.s_init = ds_final;
-        fp.init_unit_stride = kSS;
-        fp.s_out = ds0;
-        fp.out_unit_stride = kSS;
-        fp.out_last_only = 1;
-        fp.B = pr.B;
-        fp.T = pr.T;
-        fp.H = pr.H;
-        fp.NC = NC;
-        fp.chunks_per_seg = cps;
-        fp.h_save = dbuf;
-        fp.scale = pr.scale;
-        fp.ctl = ctl;
-        if ((s = launch_state_kernel(true, true, fp, dim3(1, pr.H, pr.B), st)) != GLA_OK) return s;
-    }
-    StateParams rp = sp;
-    if ((s = make_token_map(&rp.tm_u, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
-    if ((s = make_token_map(&rp.tm_y, dO, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
-    rp.h_out = dbuf;
-    rp.s_init = ds_final;
-    rp.init_unit_stride = kSS;
-    rp.init_seg_stride = 0;
-    if (!rev_fused) {
-        // local gradients of every segment (segment 0's is computed and not
-        // used: its CTAs run beside the others')
+    // 2. D_c for every chunk, dS_0 (written by segment 0, where the reverse
+    // sweep ends) and dv, in one reverse sweep: the fused forward kernel run
+    // backwards (k in q's place, q in k's, dO in v's, dv out), D_c kept as hi
+    // and lo planes like the forward's entering states.  With several
+    // segments per head, a state-only reverse pre-pass from zero and the
+    // right-to-left fold give each segment's sweep its entering D first.
+    StateParams fp;
+    memset(&fp, 0, sizeof(fp));
+    if ((s = make_token_map(&fp.tm_q, pr.k, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
+    if ((s = make_token_map(&fp.tm_u, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
+    if ((s = make_token_map(&fp.tm_y, dO, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
+    if ((s = make_token_map(&fp.tm_o, dv, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
+    if ((s = make_state_map(&fp.tm_h, dbuf, static_cast<int64_t>(units) * NC * 2, 64)) != GLA_OK) return s;
+    fp.a = pr.a;
+    fp.s_init = ds_final;
+    fp.init_unit_stride = kSS;
+    fp.s_out = ds0;
+    fp.out_unit_stride = kSS;
+    fp.out_last_only = 1;
+    fp.B = pr.B;
+    fp.T = pr.T;
+    fp.H = pr.H;
+    fp.NC = NC;
+    fp.chunks_per_seg = cps;
+    fp.h_save = dbuf;
+    fp.scale = pr.scale;
+    fp.ctl = ctl;
+    if (nseg > 1) {
+        // local gradients of every segment from zero (segment 0's is computed
+        // and not used: its CTAs run beside the others'), then the fold
+        StateParams rp = sp;
+        if ((s = make_token_map(&rp.tm_u, pr.q, kDk, pr.H, pr.T, pr.B, pr.ld_qk, 32, 64)) != GLA_OK) return s;
+        if ((s = make_token_map(&rp.tm_y, dO, kDv, pr.H, pr.T, pr.B, ldo, 64, 128)) != GLA_OK) return s;
         if ((s = pre_pass(rp, true, nseg, ds_final)) != GLA_OK) return s;
-        rp.s_init = segst;
-        rp.init_unit_stride = static_cast<int64_t>(nseg) * kSS;
-        rp.init_seg_stride = kSS;
-        rp.s_out = ds0;
-        if ((s = launch_state_kernel(false, true, rp, dim3(nseg, pr.H, pr.B), st)) != GLA_OK) return s;
+        fp.s_init = segst;
+        fp.init_unit_stride = static_cast<int64_t>(nseg) * kSS;
+        fp.init_seg_stride = kSS;
     }
+    if ((s = launch_state_kernel(true, true, fp, dim3(nseg, pr.H, pr.B), st)) != GLA_OK) return s;
 
-    // 3. dq, dk (+ per-token delta halves and chunk totals) and dv
+    // 3. dq, dk (+ per-token delta halves and chunk totals)
     BwdParams bp;
     memset(&bp, 0, sizeof(bp));
     const int64_t ldk = static_cast<int64_t>(pr.H) * kDk;
@@ -1136,11 +803,9 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
     if ((s = make_token_map(&bp.tm_dq, dq, kDk, pr.H, pr.T, pr.B, ldk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&bp.tm_dk, dk, kDk, pr.H, pr.T, pr.B, ldk, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&bp.tm_do32, dO, kDv, pr.H, pr.T, pr.B, ldo, 32, 64)) != GLA_OK) return s;
-    if ((s = make_token_map(&bp.tm_dv32, dv, kDv, pr.H, pr.T, pr.B, ldo, 32, 64)) != GLA_OK) return s;
     if ((s = make_token_map(&bp.tm_v32, pr.v, kDv, pr.H, pr.T, pr.B, pr.ld_v, 32, 64)) != GLA_OK) return s;
     if ((s = make_state_map(&bp.tm_h2, hbuf, static_cast<int64_t>(units) * NC * 2, 32, 2)) != GLA_OK) return s;
     if ((s = make_state_map(&bp.tm_d2, dbuf, static_cast<int64_t>(units) * NC * 2, 32, 2)) != GLA_OK) return s;
-    if ((s = make_state_map(&bp.tm_d32, dbuf, static_cast<int64_t>(units) * NC * 2, 32)) != GLA_OK) return s;
     bp.a = pr.a;
     bp.delta = delta;
     bp.ctot = ctot;
@@ -1158,14 +823,6 @@ gla_status run_chunk_bwd(const ChunkProblem& pr, const float* s0, const void* dO
         const int grid = items < sms ? items : sms;
         if ((s = launch_bwd_kernel(bwd_dqdk_persistent_kernel, bqp::BYTES, bp, dim3(grid), st, "bwd_dqdk_kernel",
                                    bqp::kThreads)) != GLA_OK)
-            return s;
-    }
-    if (!rev_fused) {
-        // persistent: one CTA per SM over the (batch, head, chunk, dv half) items
-        const int items = units * NC * 2;
-        const int grid = items < sms ? items : sms;
-        if ((s = launch_bwd_kernel(bwd_dv_kernel, dvp::BYTES, bp, dim3(grid), st, "bwd_dv_kernel", dvp::kThreads)) !=
-            GLA_OK)
             return s;
     }
 

@@ -396,8 +396,10 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     constexpr int dc = REV ? -1 : 1;          // chunk step
     const int c_first = REV ? c_end - 1 : c_begin;
     auto chunk_at = [c_first](int it) { return c_first + dc * it; };
-    const int last_seg = VARLEN ? max(1, (NCn + cps - 1) / cps) - 1
-                                : static_cast<int>(gridDim.x) - 1;
+    // the segment where the sweep ends (the reverse sweep ends on segment 0)
+    const int last_seg = REV ? 0
+                             : VARLEN ? max(1, (NCn + cps - 1) / cps) - 1
+                                      : static_cast<int>(gridDim.x) - 1;
     const WaitCtl ctl = p.ctl;
 
     const int quad = warp & 3;

@@ -23,9 +23,9 @@ def test_method_and_design_bytes_per_chunk():
     # dq/dk: q, k, v, dO, a in; dq, dk out (+ h and D as hi, lo planes; q.dq, k.dk)
     assert M["bwd_dqdk_kernel"] == q + k + v + dO + a + dq + dk == 197_120
     assert D["bwd_dqdk_kernel"] == 4 * h + 2 * a
-    # dv: q, k, dO, a in; dv out (+ the hi plane of D)
-    assert M["bwd_dv_kernel"] == q + k + dO + a + dv == 147_968
-    assert D["bwd_dv_kernel"] == h
+    # the reverse sweep with dv: q, k, dO, a in; dv out (+ D_c as hi, lo planes)
+    assert M["chunk_rev_fused_kernel"] == q + k + dO + a + dv == 147_968
+    assert D["chunk_rev_fused_kernel"] == 2 * h
     assert M["da_finish_kernel"] == da
     # the step: forward and backward inputs and outputs, 3,084 B per token-head
     assert bench.STEP_BYTES == (q + k + v + a + o) + (q + k + v + dO + a + dq + dk + dv + da)
@@ -38,7 +38,9 @@ def test_algorithmic_flops_per_chunk():
     assert F["chunk_fwd_fused_kernel"] == 18_874_368
     assert F["chunk_state_fwd_kernel"] == F["chunk_state_rev_kernel"] == mm(96, 192, 128)
     assert F["bwd_dqdk_kernel"] == mm(128, 128, 192) + 2 * mm(128, 96, 192) + 2 * mm(128, 96, 128)
-    assert F["bwd_dv_kernel"] == mm(128, 128, 96) + mm(128, 192, 128) + mm(128, 192, 96)
+    # reverse sweep with dv: scores^T, K D, P~ dO (dv) and the state update Q~^T dO
+    assert F["chunk_rev_fused_kernel"] == (mm(128, 128, 96) + mm(128, 192, 128) + mm(128, 192, 96)
+                                           + F["chunk_state_rev_kernel"])
     # forward 18.9 MF and backward 45.6 MF per chunk-head: 132 GF at B8 H16 T2048
     assert bench.STEP_FLOPS * 8 * 16 * 16 == pytest.approx(132.07e9, rel=1e-4)
 

@@ -56,6 +56,10 @@ namespace {
 constexpr int kW = 4;
 constexpr int kG = 4;           // rows per stage
 constexpr int kRing = 8;        // ring stages: s, s+1, s+2 (moments) and five in flight
+// 8-channel workers hold half a row a CTA: four stages (s .. s+2 and one in
+// flight) keep the ring and the g / xhat rows within shared memory; a stage
+// takes microseconds, far longer than its load
+constexpr int ring_stages(int np) { return np == 4 ? 4 : kRing; }
 constexpr int kXch = 4;         // exchange buffers (a CTA runs at most two exchanges ahead)
 constexpr int kMsg = 24;        // floats per CTA per exchange
 constexpr int kStRing = 32;     // rows of LayerNorm statistics kept
@@ -141,12 +145,13 @@ struct BwdArgs {
 // Shared-memory map (bytes), the same in every CTA of the cluster.
 struct BwdSmem {
     uint32_t segb, ring, fin, red, xbuf, st, tot, bars, total;
-    __host__ __device__ BwdSmem(int upc, int nwork)
+    // np: fp32 pairs (channel pairs) a worker owns
+    __host__ __device__ BwdSmem(int upc, int nwork, int np)
     {
         segb = 16u * upc;                                  // one row of a CTA's channels
         ring = 0;
-        fin = ring + kRing * 2 * kG * segb;                // [2][kG][nwork][8] fp32: g, xhat
-        red = fin + 2 * kG * nwork * 32;                   // [2][warps][16] by stage parity
+        fin = ring + ring_stages(np) * 2 * kG * segb;     // [2][kG][nwork][4 np] fp32: g, xhat
+        red = fin + 2 * kG * nwork * 16 * np;              // [2][warps][16] by stage parity
         xbuf = red + 2 * (nwork / 32) * 64;                // [kXch][CL max 4][kMsg]
         st = xbuf + kXch * 4 * kMsg * 4;                   // [kStRing] (mean, rstd)
         tot = st + kStRing * 8;                            // [2][kG] (mean g, mean g xhat) by stage parity
@@ -160,15 +165,18 @@ struct BwdSmem {
 // split evenly over the cluster into whole warps), so no thread is idle.
 // Both are template parameters: their tests would otherwise be branches in
 // the row loop (measured 9% of the kernel's time for the LayerNorm flag).
-template <bool AFF, bool LN, bool FULL, int CL, int MAXT>
+// NP: fp32 pairs a worker owns, 2 (4 channels: two workers an 8-channel
+// unit) or 4 (the whole unit).
+template <bool AFF, bool LN, bool FULL, int CL, int NP, int MAXT>
 __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_constant__ BwdArgs a)
 {
     static_assert(CL >= 2 && CL <= 4, "the rows' channels are split over 2 to 4 CTAs");
+    static_assert(NP == 2 || NP == 4, "a worker owns 4 or 8 channels");
     static_assert(kMsg == 16 + 2 * kG, "a message: 16 sums, then 2 kG first elements");
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nwork = blockDim.x - 32, nwarps = nwork >> 5;
-    const BwdSmem L(a.upc, nwork);
+    const BwdSmem L(a.upc, nwork, NP);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
     uint64_t* freeb = full + kRing;
     uint64_t* xbar = freeb + kRing;
@@ -200,17 +208,18 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
     // every CTA's barriers exist before any CTA of the cluster sends to them
     cluster_sync_all();
 
-    auto ring_x = [&](int stage, int g) { return smem + L.ring + ((stage % kRing) * 2 * kG + g) * L.segb; };
-    auto ring_dy = [&](int stage, int g) { return smem + L.ring + ((stage % kRing) * 2 * kG + kG + g) * L.segb; };
+    constexpr int RING = ring_stages(NP);
+    auto ring_x = [&](int stage, int g) { return smem + L.ring + ((stage % RING) * 2 * kG + g) * L.segb; };
+    auto ring_dy = [&](int stage, int g) { return smem + L.ring + ((stage % RING) * 2 * kG + kG + g) * L.segb; };
 
     if (warp == nwarps) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             const uint32_t nbytes = 16u * nu;
-            int armed[kRing] = {};
+            int armed[RING] = {};
             for (int s = 0; s < S; ++s) {
-                const int slot = s % kRing;
-                if (s >= kRing && !mbar_wait(freeb + slot, ((s - kRing) / kRing) & 1, ctl)) break;
+                const int slot = s % RING;
+                if (s >= RING && !mbar_wait(freeb + slot, ((s - RING) / RING) & 1, ctl)) break;
                 uint32_t bytes = 0;
 #pragma unroll
                 for (int g = 0; g < kG; ++g) {
@@ -233,19 +242,19 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
                 }
                 ++armed[slot];
             }
-            for (int i = 0; i < kRing; ++i)
+            for (int i = 0; i < RING; ++i)
                 if (armed[i]) mbar_wait(full + i, (armed[i] - 1) & 1, ctl);
         }
     } else {
         // ------------------------------------------------------------- workers
-        const int u = tid >> 1, half = tid & 1;
+        const int u = NP == 4 ? tid : tid >> 1, half = NP == 4 ? 0 : tid & 1;
         const bool active = FULL || u < nu;
-        const int c = 8 * (ubase + u) + 4 * half;                // this thread's channels c .. c+3
+        const int c = 8 * (ubase + u) + 4 * half;                // this thread's channels c .. c + 2 NP - 1
         const uint32_t seg_off = 16u * u + 8u * half;            // their bytes in a ring row
 
-        f2 wr[2][kW], ga[AFF ? 2 : 1], be[AFF ? 2 : 1], bi[AFF ? 2 : 1];
+        f2 wr[NP][kW], ga[AFF ? NP : 1], be[AFF ? NP : 1], bi[AFF ? NP : 1];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NP; ++i) {
             const int ch = active ? c + 2 * i : 0;
 #pragma unroll
             for (int j = 0; j < kW; ++j)
@@ -257,10 +266,10 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
             }
         }
         const f2 zero = f2_splat(0.f), one = f2_splat(1.f);
-        f2 wxn[3][2], wxh[3][2], wdu[3][2];     // windows: rows p-3, p-2, p-1
-        f2 dw[kW][2], db[2], dg[2], dbe[2];
+        f2 wxn[3][NP], wxh[3][NP], wdu[3][NP];     // windows: rows p-3, p-2, p-1
+        f2 dw[kW][NP], db[NP], dg[NP], dbe[NP];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NP; ++i) {
 #pragma unroll
             for (int r = 0; r < 3; ++r) wxn[r][i] = wxh[r][i] = wdu[r][i] = zero;
 #pragma unroll
@@ -270,7 +279,36 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
         float gs[2 * kG] = {};                   // this thread's g and g xhat sums of the stage's output rows
         const float invD = 1.0f / static_cast<float>(D);
         float* fin = reinterpret_cast<float*>(smem + L.fin);
-        auto fin_at = [&](int par, int g) { return fin + ((par * kG + g) * nwork + tid) * 8; };
+        auto fin_at = [&](int par, int g) { return fin + ((par * kG + g) * nwork + tid) * (4 * NP); };
+        // this thread's channels of a ring row as NP fp32 pairs
+        auto load_pairs = [&](const uint8_t* ring_row, f2 (&v)[NP]) {
+            if constexpr (NP == 2) {
+                const uint2 w = *reinterpret_cast<const uint2*>(ring_row + seg_off);
+                v[0] = f2_from_bf16x2(w.x);
+                v[1] = f2_from_bf16x2(w.y);
+            } else {
+                const uint4 w = *reinterpret_cast<const uint4*>(ring_row + seg_off);
+                v[0] = f2_from_bf16x2(w.x);
+                v[1] = f2_from_bf16x2(w.y);
+                v[2] = f2_from_bf16x2(w.z);
+                v[3] = f2_from_bf16x2(w.w);
+            }
+        };
+        // NP pairs to global memory as bf16 (8 or 16 bytes) or fp32 (16 bytes a 2 pairs)
+        auto store_bf16 = [&](__nv_bfloat16* dst, const f2 (&v)[NP]) {
+            if constexpr (NP == 2)
+                *reinterpret_cast<uint2*>(dst) = make_uint2(f2_to_bf16x2(v[0]), f2_to_bf16x2(v[1]));
+            else
+                *reinterpret_cast<uint4*>(dst) = make_uint4(f2_to_bf16x2(v[0]), f2_to_bf16x2(v[1]),
+                                                            f2_to_bf16x2(v[2]), f2_to_bf16x2(v[3]));
+        };
+        auto store_f32 = [&](float* dst, const f2 (&v)[NP]) {
+#pragma unroll
+            for (int i = 0; i < NP; i += 2) {
+                const float2 v0 = f2_get(v[i]), v1 = f2_get(v[i + 1]);
+                *reinterpret_cast<float4*>(dst + 2 * i) = make_float4(v0.x, v0.y, v1.x, v1.y);
+            }
+        };
 
         // moments of this CTA's channels of stream row p about the row's
         // first element here: (sum d, sum d^2) for this thread's channels
@@ -280,9 +318,16 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
             if (active && (INNER || (p >= 0 && p < p_load))) {
                 const uint8_t* row = ring_x(stage, g);
                 const f2 x0 = f2_splat(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(row)));
-                const uint2 xv = *reinterpret_cast<const uint2*>(row + seg_off);
-                const f2 d0 = f2_sub(f2_from_bf16x2(xv.x), x0), d1 = f2_sub(f2_from_bf16x2(xv.y), x0);
-                const float2 s1 = f2_get(f2_add(d0, d1)), s2 = f2_get(f2_fma(d1, d1, f2_mul(d0, d0)));
+                f2 xv[NP];
+                load_pairs(row, xv);
+                f2 a1 = f2_sub(xv[0], x0), a2 = f2_mul(a1, a1);
+#pragma unroll
+                for (int i = 1; i < NP; ++i) {
+                    const f2 d = f2_sub(xv[i], x0);
+                    a1 = f2_add(a1, d);
+                    a2 = f2_fma(d, d, a2);
+                }
+                const float2 s1 = f2_get(a1), s2 = f2_get(a2);
                 m1 = s1.x + s1.y;
                 m2 = s2.x + s2.y;
             }
@@ -329,45 +374,44 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
         // that no range check is needed.
         auto do_row = [&](auto inner_tag, int stage, int g, int p) {
             constexpr bool INNER = decltype(inner_tag)::value;
-            f2 xn[2], xh[2], du[2];
+            f2 xn[NP], xh[NP], du[NP];
             if (!INNER && p < 0) {
                 const bool hv = active && a.cs_in;
                 const float* src = a.cs_in + (static_cast<int64_t>(b) * 3 + p + 3) * D + c;
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
+                for (int i = 0; i < NP; ++i) {
                     xn[i] = hv ? f2_make(src[2 * i], src[2 * i + 1]) : zero;
                     xh[i] = zero;
                 }
             } else if ((INNER || p < T) && active) {
-                const uint2 xv = *reinterpret_cast<const uint2*>(ring_x(stage, g) + seg_off);
-                xn[0] = f2_from_bf16x2(xv.x);
-                xn[1] = f2_from_bf16x2(xv.y);
+                load_pairs(ring_x(stage, g), xn);
                 if (ln) {
                     const float2 m = st_ring[(p - p_s) & (kStRing - 1)];
                     if constexpr (AFF) {
                         const f2 mu = f2_splat(m.x), rs = f2_splat(m.y);
 #pragma unroll
-                        for (int i = 0; i < 2; ++i) {
+                        for (int i = 0; i < NP; ++i) {
                             xh[i] = f2_mul(f2_sub(xn[i], mu), rs);
                             xn[i] = f2_fma(xh[i], ga[i], be[i]);
                         }
                     } else {
                         const f2 rs = f2_splat(m.y), sh = f2_splat(-m.x * m.y);
 #pragma unroll
-                        for (int i = 0; i < 2; ++i) xh[i] = xn[i] = f2_fma(xn[i], rs, sh);
+                        for (int i = 0; i < NP; ++i) xh[i] = xn[i] = f2_fma(xn[i], rs, sh);
                     }
                 } else {
-                    xh[0] = xn[0];
-                    xh[1] = xn[1];
+#pragma unroll
+                    for (int i = 0; i < NP; ++i) xh[i] = xn[i];
                 }
             } else {
-                xn[0] = xn[1] = xh[0] = xh[1] = zero;
+#pragma unroll
+                for (int i = 0; i < NP; ++i) xn[i] = xh[i] = zero;
             }
             if ((INNER || (p >= t_b && p < T)) && active) {
-                const uint2 dv = *reinterpret_cast<const uint2*>(ring_dy(stage, g) + seg_off);
-                const f2 dyv[2] = {f2_from_bf16x2(dv.x), f2_from_bf16x2(dv.y)};
+                f2 dyv[NP];
+                load_pairs(ring_dy(stage, g), dyv);
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
+                for (int i = 0; i < NP; ++i) {
                     f2 acc = AFF ? bi[AFF ? i : 0] : zero;
 #pragma unroll
                     for (int j = 0; j < kW - 1; ++j) acc = f2_fma(wr[i][j], wxn[j][i], acc);
@@ -379,7 +423,7 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
                 }
                 if (INNER || p < t_e) {
 #pragma unroll
-                    for (int i = 0; i < 2; ++i) {
+                    for (int i = 0; i < NP; ++i) {
 #pragma unroll
                         for (int j = 0; j < kW - 1; ++j) dw[j][i] = f2_fma(du[i], wxn[j][i], dw[j][i]);
                         dw[kW - 1][i] = f2_fma(du[i], xn[i], dw[kW - 1][i]);
@@ -387,47 +431,48 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
                     }
                 }
             } else {
-                du[0] = du[1] = zero;
+#pragma unroll
+                for (int i = 0; i < NP; ++i) du[i] = zero;
             }
             const int q = p - 3;
             const bool out = INNER || (q >= t_b && q < t_e);
             const bool hist = !INNER && t_b == 0 && q < 0 && q >= -3 && a.dcs;
             if (out || hist) {
-                f2 dxn[2];
+                f2 dxn[NP];
 #pragma unroll
-                for (int i = 0; i < 2; ++i)
+                for (int i = 0; i < NP; ++i)
                     dxn[i] = f2_fma(wr[i][0], du[i],
                                     f2_fma(wr[i][1], wdu[2][i], f2_fma(wr[i][2], wdu[1][i], f2_mul(wr[i][3], wdu[0][i]))));
                 if (hist) {
                     if (active) {
-                        float* dst = a.dcs + (static_cast<int64_t>(b) * 3 + q + 3) * D + c;
-                        const float2 v0 = f2_get(dxn[0]), v1 = f2_get(dxn[1]);
-                        *reinterpret_cast<float4*>(dst) = make_float4(v0.x, v0.y, v1.x, v1.y);
+                        store_f32(a.dcs + (static_cast<int64_t>(b) * 3 + q + 3) * D + c, dxn);
                     }
                 } else if (ln) {
-                    f2 gg[2];
+                    f2 gg[NP];
 #pragma unroll
-                    for (int i = 0; i < 2; ++i) {
+                    for (int i = 0; i < NP; ++i) {
                         gg[i] = AFF ? f2_mul(dxn[i], ga[AFF ? i : 0]) : dxn[i];
                         dg[i] = f2_fma(dxn[i], wxh[0][i], dg[i]);
                         dbe[i] = f2_add(dbe[i], dxn[i]);
                     }
-                    const float2 s1 = f2_get(f2_add(gg[0], gg[1]));
-                    const float2 s2 = f2_get(f2_fma(gg[1], wxh[0][1], f2_mul(gg[0], wxh[0][0])));
+                    f2 sg = gg[0], sgx = f2_mul(gg[0], wxh[0][0]);
+#pragma unroll
+                    for (int i = 1; i < NP; ++i) {
+                        sg = f2_add(sg, gg[i]);
+                        sgx = f2_fma(gg[i], wxh[0][i], sgx);
+                    }
+                    const float2 s1 = f2_get(sg), s2 = f2_get(sgx);
                     gs[g] += s1.x + s1.y;
                     gs[kG + g] += s2.x + s2.y;
                     float* fp = fin_at(stage & 1, g);
-                    const float2 a0 = f2_get(gg[0]), a1 = f2_get(gg[1]);
-                    const float2 h0 = f2_get(wxh[0][0]), h1 = f2_get(wxh[0][1]);
-                    *reinterpret_cast<float4*>(fp) = make_float4(a0.x, a0.y, a1.x, a1.y);
-                    *reinterpret_cast<float4*>(fp + 4) = make_float4(h0.x, h0.y, h1.x, h1.y);
+                    store_f32(fp, gg);
+                    store_f32(fp + 2 * NP, wxh[0]);
                 } else if (active) {
-                    *reinterpret_cast<uint2*>(a.dx + (row0 + q) * D + c) =
-                        make_uint2(f2_to_bf16x2(dxn[0]), f2_to_bf16x2(dxn[1]));
+                    store_bf16(a.dx + (row0 + q) * D + c, dxn);
                 }
             }
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
+            for (int i = 0; i < NP; ++i) {
                 wxn[0][i] = wxn[1][i];
                 wxn[1][i] = wxn[2][i];
                 wxn[2][i] = xn[i];
@@ -447,11 +492,15 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
                 const float2 mt = tot[(s & 1) * kG + g];
                 const f2 rs = f2_splat(rstd), na = f2_splat(-rstd * mt.x), nb = f2_splat(-rstd * mt.y);
                 const float* fp = fin_at(s & 1, g);
-                const float4 g4 = *reinterpret_cast<const float4*>(fp);
-                const float4 h4 = *reinterpret_cast<const float4*>(fp + 4);
-                const f2 o0 = f2_fma(f2_make(h4.x, h4.y), nb, f2_fma(f2_make(g4.x, g4.y), rs, na));
-                const f2 o1 = f2_fma(f2_make(h4.z, h4.w), nb, f2_fma(f2_make(g4.z, g4.w), rs, na));
-                *reinterpret_cast<uint2*>(a.dx + (row0 + q) * D + c) = make_uint2(f2_to_bf16x2(o0), f2_to_bf16x2(o1));
+                f2 o[NP];
+#pragma unroll
+                for (int i = 0; i < NP; i += 2) {
+                    const float4 g4 = *reinterpret_cast<const float4*>(fp + 2 * i);
+                    const float4 h4 = *reinterpret_cast<const float4*>(fp + 2 * NP + 2 * i);
+                    o[i] = f2_fma(f2_make(h4.x, h4.y), nb, f2_fma(f2_make(g4.x, g4.y), rs, na));
+                    o[i + 1] = f2_fma(f2_make(h4.z, h4.w), nb, f2_fma(f2_make(g4.z, g4.w), rs, na));
+                }
+                store_bf16(a.dx + (row0 + q) * D + c, o);
             };
             const int q0 = p_s + s * kG - 3;
             if (q0 >= t_b && q0 + kG <= t_e) {     // every row of the stage is an output row
@@ -523,9 +572,9 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
                     }
                 }
             }
-            const int slot = s % kRing;
-            bool ok = !failed && mbar_wait(full + slot, (s / kRing) & 1, ctl);
-            if (ln && ok && s + 2 < S) ok = mbar_wait(full + (s + 2) % kRing, ((s + 2) / kRing) & 1, ctl);
+            const int slot = s % RING;
+            bool ok = !failed && mbar_wait(full + slot, (s / RING) & 1, ctl);
+            if (ln && ok && s + 2 < S) ok = mbar_wait(full + (s + 2) % RING, ((s + 2) / RING) & 1, ctl);
             if (!ok) failed = true;
 #pragma unroll
             for (int i = 0; i < 2 * kG; ++i) gs[i] = 0.f;
@@ -603,10 +652,7 @@ __global__ void __launch_bounds__(MAXT, 1) ln_conv_silu_bwd_kernel(const __grid_
         // per-(range, CTA) partial sums
         if (!failed && active) {
             float* pp = a.part + (static_cast<int64_t>(b) * a.nx + slice) * kParts * D + c;
-            auto put = [&](int k, const f2 (&v)[2]) {
-                const float2 v0 = f2_get(v[0]), v1 = f2_get(v[1]);
-                *reinterpret_cast<float4*>(pp + k * D) = make_float4(v0.x, v0.y, v1.x, v1.y);
-            };
+            auto put = [&](int k, const f2 (&v)[NP]) { store_f32(pp + k * D, v); };
 #pragma unroll
             for (int j = 0; j < kW; ++j) put(j, dw[j]);
             put(4, db);
@@ -647,19 +693,28 @@ __global__ void __launch_bounds__(256) conv_bwd_reduce_kernel(const float* __res
 // issue, and a narrower thread repeats the per-row work that does not
 // scale with its channels.)
 constexpr int kBwdThreads = 288;
+constexpr int kBwdThreads8 = 224;   // 8-channel workers: at most 7 warps a CTA
 
 struct BwdPlan {
-    int CL, upc, threads, nx, rps;
+    int CL, NP, upc, threads, nx, rps;
 };
 
-// clusters: how many clusters of CL CTAs the device runs at once
+// Clusters of 2 CTAs where they fit: every SM can hold one (clusters of 4
+// left 16 of 148 SMs idle, a GPC's SM count not being a multiple of 4).  Up
+// to D = 2,048 a worker owns 4 channels; up to D = 3,072, 8 (at most 192
+// workers + the producer: a thread may keep 255 registers, and the 4-stage
+// ring and the g / xhat rows take 197 KB), which also spreads the per-row
+// work that does not scale with the channels over twice as many; above,
+// clusters of 4 CTAs with 4-channel workers.  clusters: how many clusters
+// the device runs at once.
 BwdPlan plan_bwd(int B, int T, int D, int clusters)
 {
     BwdPlan pl;
     const int P = D / 8;
-    pl.CL = D <= 2048 ? 2 : 4;
+    pl.CL = D <= 3072 ? 2 : 4;
+    pl.NP = D <= 2048 || D > 3072 ? 2 : 4;
     pl.upc = (P + pl.CL - 1) / pl.CL;
-    pl.threads = (2 * pl.upc + 31) / 32 * 32 + 32;
+    pl.threads = ((pl.NP == 4 ? 1 : 2) * pl.upc + 31) / 32 * 32 + 32;
     int nx = clusters / (B > 0 ? B : 1);
     if (nx < 1) nx = 1;
     if (nx > kMaxSlices) nx = kMaxSlices;
@@ -690,25 +745,28 @@ gla_status launch_conv_bwd(const void* x, int apply_ln, const float* g, const fl
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int CL = D <= 2048 ? 2 : 4;
+    BwdPlan pl = plan_bwd(B, T, D, sms / (D <= 3072 ? 2 : 4));
+    const int CL = pl.CL;
     const bool aff = g || be || bias;
     void (*kernel)(BwdArgs);
     const bool ln = apply_ln != 0;
     const int P = D / 8;
-    const bool full = P % CL == 0 && (2 * (P / CL)) % 32 == 0;
-    // the 16 forms: affine or not, LayerNorm or not, every thread owning
-    // channels or not, 2 or 4 CTAs a cluster
+    const bool full = P % CL == 0 && ((pl.NP == 4 ? 1 : 2) * (P / CL)) % 32 == 0;
+    // the 24 forms: affine or not, LayerNorm or not, every thread owning
+    // channels or not; 4-channel workers in clusters of 2 or 4 CTAs, or
+    // 8-channel workers in clusters of 2
     using KFn = void (*)(BwdArgs);
-#define GLA_BWD_FORM(A, N, F) {ln_conv_silu_bwd_kernel<A, N, F, 2, kBwdThreads>, ln_conv_silu_bwd_kernel<A, N, F, 4, kBwdThreads>}
-    static const KFn forms[2][2][2][2] = {
+#define GLA_BWD_FORM(A, N, F)                                                                            \
+    {ln_conv_silu_bwd_kernel<A, N, F, 2, 2, kBwdThreads>, ln_conv_silu_bwd_kernel<A, N, F, 4, 2, kBwdThreads>, \
+     ln_conv_silu_bwd_kernel<A, N, F, 2, 4, kBwdThreads8>}
+    static const KFn forms[2][2][2][3] = {
         {{GLA_BWD_FORM(false, false, false), GLA_BWD_FORM(false, false, true)},
          {GLA_BWD_FORM(false, true, false), GLA_BWD_FORM(false, true, true)}},
         {{GLA_BWD_FORM(true, false, false), GLA_BWD_FORM(true, false, true)},
          {GLA_BWD_FORM(true, true, false), GLA_BWD_FORM(true, true, true)}}};
 #undef GLA_BWD_FORM
-    kernel = forms[aff][ln][full][CL == 4];
-    BwdPlan pl = plan_bwd(B, T, D, sms / CL);
-    const BwdSmem L(pl.upc, pl.threads - 32);
+    kernel = forms[aff][ln][full][pl.NP == 4 ? 2 : (CL == 4 ? 1 : 0)];
+    const BwdSmem L(pl.upc, pl.threads - 32, pl.NP);
     const size_t smem = L.total;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
         cudaSuccess)

@@ -73,8 +73,13 @@ def _check(d, ln, want_hist=True):
     (2, 200, 2056, True, True, True),
     (1, 700, 2048, True, False, True),
     (1, 7, 3072, False, True, True),
+    (2, 160, 2560, True, False, False),
+    (1, 90, 3064, True, True, False),
 ])
 def test_front_bwd_parity(B, T, D, ln, affine, hist):
+    """Up to D = 2,048 and above D = 3,072 a worker owns 4 channels; in
+    between 8, in clusters of 2 CTAs (2,056 and 3,064: the channel units do
+    not split evenly over the cluster; 2,560 and 3,072: they do)."""
     _check(_case(B, T, D, affine, hist, seed=70 + T + D), ln)
 
 

@@ -13,7 +13,13 @@
 //
 // Two kernels:
 //
-// gla_fwd_fused_kernel -- forward with the output fused in.  Per chunk:
+// gla_fwd_fused_kernel<VARLEN, REV> -- forward with the output fused in.
+//   REV runs it as the backward's reverse sweep: chunks from the last, k in
+//   q's place (the tile rows), q in k's (the scaled operand of the update
+//   D = e^gamma D_next + (scale e^b q)^T dO), dO in v's and dv out:
+//     dv_i = e^{gamma - b_i} ( k_i D_next + sum_{j >= i} scale e^{b_j - gamma} (k_i.q_j) dO_j )
+//   i.e. the same tiles with the causal mask mirrored and the decay factors
+//   of the two sides swapped.  Per chunk (forward names):
 //   scores = Q K^T (tcgen05, 128x128x96); O = Q S_prev (128x192x96, against a
 //   bf16 copy of the state); S += K~^T V (K~ = e^{gamma-b} K split into bf16
 //   hi + lo, so the fp32 state keeps its precision); O += P V (P split into

@@ -10,13 +10,13 @@
 //   dw[c,j]   = sum_t du[t,c] xn[t-3+j, c]   dbias = sum du
 //   dgamma    = sum dxn xhat                  dbeta = sum dxn
 //
-// One pass over the rows.  A cluster of CL CTAs (CL = 2 up to D = 2,048, 4
+// One pass over the rows.  A cluster of CL CTAs (CL = 2 up to D = 3,072, 4
 // above) owns a contiguous token range of one sequence, and CTA r of the
 // cluster owns the r-th block of channels (whole 8-channel units).  Every
 // per-channel quantity -- the conv weights, the windows of the last three
 // rows' xn, xhat and du, the sums of dw, dbias, dgamma, dbeta -- stays in the
-// registers of the thread that owns the channel (4 channels a thread) for
-// the whole range.  A producer warp streams the rows of x and dy through a
+// registers of the thread that owns the channel (4 channels a thread, or 8
+// for 2,048 < D <= 3,072) for the whole range.  A producer warp streams the rows of x and dy through a
 // ring of shared-memory stages of kG rows (bulk asynchronous copies, one per
 // row and tensor, completion on the stage's mbarrier).
 //

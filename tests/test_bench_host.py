@@ -97,6 +97,14 @@ def test_kernel_digest_follows_the_sources():
     assert bench.kernel_digest("no_such_kernel") is None
 
 
+def test_digest_ignores_comments_only():
+    src = 'int a = 1; // one\n/* block\n comment */ const char* s = "//x";\n\nint b = 2;\n'
+    same = 'int a = 1;\n const char* s = "//x";\nint b = 2; // two\n'
+    assert bench.strip_comments(src) == bench.strip_comments(same)
+    assert bench.strip_comments(src) != bench.strip_comments(src.replace("b = 2", "b = 3"))
+    assert '"//x"' in bench.strip_comments(src)
+
+
 class _FakeProc:
     def terminate(self):
         pass

@@ -31,11 +31,11 @@
 //   per-element exponential or scaled copy of Q is needed.  Chunks with a
 //   steeper decay take the exact per-element path (P_ij with 2^{b_i - b_j},
 //   Q scaled by scale e^{b_i} in place, r_i = 1).
-//   Q tile row i = token i (natural order, three TMA boxes per tile: each
-//   TMA instruction costs the issuing thread about 90 cycles, so the tile is
-//   loaded in as few boxes as its swizzle allows).  Each worker warp converts
-//   one 32-token block of P, so the causal triangle's imbalance between
-//   lane quarters costs at most one block per warp.
+//   Q tile row i = token i (natural order, three TMA boxes per tile: issuing
+//   a tile as 24 permuted 16-row boxes kept the producer busy for about
+//   2.5k cycles).  Each worker warp converts one 32-token block of P, so the
+//   causal triangle's imbalance between lane quarters costs at most one
+//   block per warp.
 //
 // gla_state_pass_kernel<REVERSE> -- state only: S (or D) = e^gamma S + U~^T Y
 //   per chunk with U~ split into bf16 hi + lo, optionally storing the bf16
@@ -74,7 +74,7 @@ struct StateParams {
     CUtensorMap tm_u;       // scaled operand: k (forward) or q (reverse)
     CUtensorMap tm_y;
     CUtensorMap tm_o;       // o tile stores (fused forward)
-    CUtensorMap tm_h;       // saved states, 64-column boxes of one plane (fused forward with h_save)       // v (forward) or dO (reverse)
+    CUtensorMap tm_h;       // saved states, 64-column boxes of one plane (fused forward with h_save)
     const float* a;         // [B, T, H] log-decay
     const float* s_init;    // initial state per (unit, seg) or null (zeros)
     float* s_out;           // state after the segment, or null

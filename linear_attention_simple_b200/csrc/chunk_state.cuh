@@ -70,10 +70,10 @@
 namespace gla {
 
 struct StateParams {
-    CUtensorMap tm_q;       // q tile loads (fused forward)
+    CUtensorMap tm_q;       // tile rows of the fused kernel: q (forward) or k (reverse sweep)
     CUtensorMap tm_u;       // scaled operand: k (forward) or q (reverse)
-    CUtensorMap tm_y;
-    CUtensorMap tm_o;       // o tile stores (fused forward)
+    CUtensorMap tm_y;       // v (forward) or dO (reverse)
+    CUtensorMap tm_o;       // output tile stores of the fused kernel: o (forward) or dv (reverse sweep)
     CUtensorMap tm_h;       // saved states, 64-column boxes of one plane (fused forward with h_save)
     const float* a;         // [B, T, H] log-decay
     const float* s_init;    // initial state per (unit, seg) or null (zeros)

@@ -25,15 +25,16 @@ Rooflines, all against MEASURED_PEAKS.json:
                  and outputs of the computation it reads or writes) per
                  launch over its mean launch time against HBM copy bandwidth,
                  with its design bytes (per-chunk states, partial sums) and
-                 its bf16 tensor-core fraction beside it;
+                 its bf16 tensor-core fraction beside it, and under
+                 "per_kernel" the same fractions for every kernel of the step;
   roofline_step  the whole step: 3,084 method bytes per token-head (+ the
                  final state) against HBM, 64.5 MF of algorithmic flops per
                  (batch, head, chunk) against the sustained bf16 peak;
   prefill_fwd    the forward alone at the same shape, both rooflines.
 The dominant kernel's "traffic" (DRAM bytes per launch) comes from the ncu
 capture summarised in profiles/dram_traffic.md, and only while the digest of
-the kernel's source files still matches the one recorded there; otherwise it
-is null.
+the kernel's source files (their code, comments removed) still matches the
+one recorded there; otherwise it is null.
 
 --skip-decode / --skip-e2e time only the training step: the command the
 profiles' ncu captures run (a few GB on the device instead of the 36 GB of
@@ -329,6 +330,27 @@ def kernel_roofline(summary, peaks, peak_kind, units_per_launch, B, H):
     return roof, shares
 
 
+def kernel_rooflines(summary, peaks, units_per_launch, B, H):
+    """Every traced kernel with a byte model: mean launch time, HBM fraction
+    on its method bytes and with its design bytes, and its bf16 tensor
+    fraction where it has an algorithmic flop count."""
+    out = {}
+    tpk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    for name, launches, total_ms in summary:
+        if name not in METHOD_BYTES or launches <= 0:
+            continue
+        mean_s = total_ms / launches / 1e3
+        nb = METHOD_BYTES[name] * units_per_launch + (FS * B * H if name == "chunk_fwd_fused_kernel" else 0)
+        design = DESIGN_BYTES.get(name, 0) * units_per_launch
+        e = {"mean_launch_us": round(mean_s * 1e6, 2),
+             "frac": round(nb / mean_s / 1e9 / peaks["hbm_gbs"], 4),
+             "frac_incl_design_bytes": round((nb + design) / mean_s / 1e9 / peaks["hbm_gbs"], 4)}
+        if name in CHUNK_FLOPS:
+            e["tensor_frac"] = round(CHUNK_FLOPS[name] * units_per_launch / mean_s / 1e12 / tpk, 4)
+        out[name] = e
+    return out
+
+
 def step_roofline(step_s, units, B, H, peaks, peak_kind):
     """The training step as a whole against both rooflines: its method bytes
     (+ the final state the forward writes) over HBM, its algorithmic flops
@@ -445,6 +467,8 @@ def run_ours(args, ws, rank, local):
     torch.cuda.synchronize()
     roof, shares = kernel_roofline([(n, c, t) for n, c, t in summary], peaks, peak_kind,
                                    units_per_launch, w.B, w.H)
+    if roof is not None:
+        roof["per_kernel"] = kernel_rooflines(summary, peaks, units_per_launch, w.B, w.H)
     roof_step = step_roofline(elapsed / args.steps, units_per_launch, w.B, w.H, peaks, peak_kind)
     # ---- prefill: the forward alone at the same shape
     pre = run_prefill(args, ws, d, st, peaks, peak_kind, units_per_launch)
@@ -743,7 +767,7 @@ def run_long_prefill(args, ws, peaks, peak_kind):
            "front_end": {"us_per_launch": round(t_front * 1e6, 2),
                          "roofline": roof("ln_conv_silu_kernel", front_bytes, t_front)},
            "front_end_bwd": {"us_per_launch": round(t_fbwd * 1e6, 2),
-                             "roofline": roof("conv1d_silu_causal_bwd (one row pass by clusters of 4 CTAs, reduction)",
+                             "roofline": roof("conv1d_silu_causal_bwd (one row pass by clusters of 2 CTAs, reduction)",
                                               front_bwd_bytes, t_fbwd)},
            "gla_fwd": {"us_per_launch": round(t_mix * 1e6, 2),
                        "roofline": roof("gla_chunk_fwd (segmented: state pre-pass, combine, fused pass)",

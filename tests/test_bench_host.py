@@ -140,3 +140,16 @@ def test_clock_record_flags_slowdowns(tmp_path):
     out = s.stop()
     assert out["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
     assert out["sm_mhz"] == 1200.0
+
+
+def test_per_kernel_rooflines():
+    peaks = dict(bench.FALLBACK_PEAKS)
+    units = 8 * 16 * 16
+    summary = [("chunk_fwd_fused_kernel", 10, 1.0), ("bwd_dqdk_kernel", 10, 1.5), ("unmodelled_kernel", 3, 0.1)]
+    r = bench.kernel_rooflines(summary, peaks, units, 8, 16)
+    assert set(r) == {"chunk_fwd_fused_kernel", "bwd_dqdk_kernel"}
+    e = r["bwd_dqdk_kernel"]
+    assert e["mean_launch_us"] == 150.0
+    mb = bench.METHOD_BYTES["bwd_dqdk_kernel"] * units
+    assert e["frac"] == pytest.approx(mb / 150e-6 / 1e9 / peaks["hbm_gbs"], abs=1e-4)
+    assert e["frac_incl_design_bytes"] > e["frac"] and 0 < e["tensor_frac"] < 1

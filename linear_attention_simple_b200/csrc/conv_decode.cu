@@ -37,7 +37,10 @@
 namespace gla {
 namespace {
 
-constexpr int kMaxStages = 4;
+// three stages: measured against two (24.6 us a launch), four (24.7) and
+// five (26.6) at 1,280 sequences x D = 3,072 with inputs beyond L2: 23.9 us
+constexpr int kMaxStages = 3;
+constexpr int kSlotInts = (kMaxStages + 1) & ~1;   // the stages' slots, padded so the partials stay 8-byte aligned
 constexpr int kCh = 8;
 
 __device__ __forceinline__ float warp_sum_dec(float v)
@@ -100,7 +103,7 @@ __global__ void __launch_bounds__(MAXT, 1) conv_decode_kernel(
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(stages) * stage_bytes);
     uint64_t* freeb = full + kMaxStages;
     int* sslot = reinterpret_cast<int*>(freeb + kMaxStages);                 // [kMaxStages]
-    float2* red = reinterpret_cast<float2*>(sslot + kMaxStages);              // [2][MAXT / 32]
+    float2* red = reinterpret_cast<float2*>(sslot + kSlotInts);               // [2][MAXT / 32]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nwork = blockDim.x - 32, nwarps = nwork >> 5;
@@ -121,7 +124,7 @@ __global__ void __launch_bounds__(MAXT, 1) conv_decode_kernel(
     if (producer) {
         // -------------------------------------------------------- producer
         if (lane == 0) {
-            int armed[kMaxStages] = {0, 0, 0, 0};
+            int armed[kMaxStages] = {};
             for (int k = 0; k < nseq; ++k) {
                 const int st = k % stages;
                 // the stage's previous sequence has been released by every worker
@@ -282,10 +285,10 @@ gla_status launch_conv_decode(const void* x, const int32_t* slot_idx, int n_slot
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = N < sms ? N : sms;
-    // as many stages (up to 4) as fit in 200 KB beside the barriers
+    // as many stages (up to 3) as fit in 216 KB beside the barriers
     const size_t stage_bytes = static_cast<size_t>(14) * D;
-    const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + kMaxStages * sizeof(int) + 2 * 32 * sizeof(float2);
-    int stages = static_cast<int>((200 * 1024 - fixed) / stage_bytes);
+    const size_t fixed = 2 * kMaxStages * sizeof(uint64_t) + kSlotInts * sizeof(int) + 2 * 32 * sizeof(float2);
+    int stages = static_cast<int>((216 * 1024 - fixed) / stage_bytes);
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages > N) stages = N > 1 ? N : 1;
     const size_t smem = stages * stage_bytes + fixed;

@@ -282,6 +282,10 @@ __device__ __forceinline__ void state_to_tmem(const float* src, uint32_t taddr)
     tmem_st_wait();
 }
 
+// This thread's NCOL columns of its row of the state, from TMEM to dst.
+// Every thread writes a different row (rows 768 B apart), so whole 32-byte
+// sectors go out where dst allows it: half the store transactions of
+// 16-byte stores, none of them a partial sector.
 template <int NCOL>
 __device__ __forceinline__ void tmem_to_state(uint32_t taddr, float* dst)
 {
@@ -289,13 +293,25 @@ __device__ __forceinline__ void tmem_to_state(uint32_t taddr, float* dst)
 #pragma unroll
     for (int j = 0; j < NCOL / 16; ++j) tmem_ld16(taddr + j * 16, r[j]);
     tmem_ld_wait();
+    if ((reinterpret_cast<uintptr_t>(dst) & 31) == 0) {
 #pragma unroll
-    for (int j = 0; j < NCOL / 16; ++j)
+        for (int j = 0; j < NCOL / 16; ++j)
 #pragma unroll
-        for (int e = 0; e < 16; e += 4)
-            *reinterpret_cast<float4*>(dst + j * 16 + e) =
-                make_float4(__uint_as_float(r[j][e]), __uint_as_float(r[j][e + 1]),
-                            __uint_as_float(r[j][e + 2]), __uint_as_float(r[j][e + 3]));
+            for (int e = 0; e < 16; e += 8) {
+                uint32_t w[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w[i] = r[j][e + i];
+                st_global_v8(dst + j * 16 + e, w);
+            }
+    } else {
+#pragma unroll
+        for (int j = 0; j < NCOL / 16; ++j)
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+                *reinterpret_cast<float4*>(dst + j * 16 + e) =
+                    make_float4(__uint_as_float(r[j][e]), __uint_as_float(r[j][e + 1]),
+                                __uint_as_float(r[j][e + 2]), __uint_as_float(r[j][e + 3]));
+    }
 }
 
 // State copy into [3][96][64] SW128 (row = dk index, n = dv column) of this

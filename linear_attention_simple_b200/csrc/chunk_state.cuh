@@ -1162,9 +1162,19 @@ __global__ void __launch_bounds__(chunk::kPassThreads, 1) gla_state_pass_kernel(
                                        (varlen_slot(p.cu_seqlens, b, seg, cps) * p.H + h) * (kDk * kDv) +
                                        row * kDv + qt * 48
                                  : p.s_out + unit * p.out_unit_stride + seg * p.out_seg_stride + row * kDv + qt * 48;
+                if ((reinterpret_cast<uintptr_t>(dst) & 31) == 0) {
 #pragma unroll
-                for (int e = 0; e < 48; e += 4)
-                    *reinterpret_cast<float4*>(dst + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+                    for (int e = 0; e < 48; e += 8) {
+                        uint32_t w[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(S[e + i]);
+                        st_global_v8(dst + e, w);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 48; e += 4)
+                        *reinterpret_cast<float4*>(dst + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+                }
             }
             if (p.cu_seqlens && tid == 0)
                 p.seg_g2[varlen_slot(p.cu_seqlens, b, seg, cps) * p.H + h] = gsum2;

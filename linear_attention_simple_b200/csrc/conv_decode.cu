@@ -261,12 +261,27 @@ __global__ void __launch_bounds__(MAXT, 1) conv_decode_kernel(
             float* hg = hist + static_cast<int64_t>(s) * 3 * D + c0;
             __stcs(reinterpret_cast<uint4*>(y + static_cast<int64_t>(n) * D + c0),
                    make_uint4(out[0], out[1], out[2], out[3]));
-            __stcs(reinterpret_cast<float4*>(hg), make_float4(h1[0], h1[1], h1[2], h1[3]));
-            __stcs(reinterpret_cast<float4*>(hg + 4), make_float4(h1[4], h1[5], h1[6], h1[7]));
-            __stcs(reinterpret_cast<float4*>(hg + D), make_float4(h2[0], h2[1], h2[2], h2[3]));
-            __stcs(reinterpret_cast<float4*>(hg + D + 4), make_float4(h2[4], h2[5], h2[6], h2[7]));
-            __stcs(reinterpret_cast<float4*>(hg + 2 * D), make_float4(v[0], v[1], v[2], v[3]));
-            __stcs(reinterpret_cast<float4*>(hg + 2 * D + 4), make_float4(v[4], v[5], v[6], v[7]));
+            if ((reinterpret_cast<uintptr_t>(hist) & 31) == 0) {
+                // each row's 8 channels as one 32-byte store: whole sectors
+                // (c0 and the row stride 4 D are multiples of 32 bytes)
+                uint32_t w8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w8[i] = __float_as_uint(h1[i]);
+                st_global_cs_v8(hg, w8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w8[i] = __float_as_uint(h2[i]);
+                st_global_cs_v8(hg + D, w8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w8[i] = __float_as_uint(v[i]);
+                st_global_cs_v8(hg + 2 * D, w8);
+            } else {
+                __stcs(reinterpret_cast<float4*>(hg), make_float4(h1[0], h1[1], h1[2], h1[3]));
+                __stcs(reinterpret_cast<float4*>(hg + 4), make_float4(h1[4], h1[5], h1[6], h1[7]));
+                __stcs(reinterpret_cast<float4*>(hg + D), make_float4(h2[0], h2[1], h2[2], h2[3]));
+                __stcs(reinterpret_cast<float4*>(hg + D + 4), make_float4(h2[4], h2[5], h2[6], h2[7]));
+                __stcs(reinterpret_cast<float4*>(hg + 2 * D), make_float4(v[0], v[1], v[2], v[3]));
+                __stcs(reinterpret_cast<float4*>(hg + 2 * D + 4), make_float4(v[4], v[5], v[6], v[7]));
+            }
         }
         mbar_arrive(freeb + st);             // this worker is done with the stage
     }

@@ -416,6 +416,15 @@ __device__ __forceinline__ void st_global_v8(void* dst, const uint32_t (&w)[8])
                  : "memory");
 }
 
+// The same with the streaming cache hint (.cs: evict first), for data not
+// read again by this kernel.
+__device__ __forceinline__ void st_global_cs_v8(void* dst, const uint32_t (&w)[8])
+{
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]),
+                 "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+
 // A descriptor for `bytes` further on: the start address is the low 14-bit
 // field in 16-byte units, and shared-memory addresses stay below 256 KB, so
 // the add never carries out of the field.

@@ -499,6 +499,40 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
     for (int i = tid; i < 512; i += blockDim.x)
         reinterpret_cast<uint4*>(sm + L::KL_PAD)[i] = make_uint4(0u, 0u, 0u, 0u);
 
+    // The producer's loads (q, k single, v double buffered).  Those of the
+    // first chunks go out before the prologue: they fill Q, U, Y0 and Y1,
+    // which the prologue does not touch (it writes KL_PAD, X and MISC).
+    auto issue_qu = [&](int c) {
+        const int t0 = c * 128;
+        mbar_arrive_expect_tx(bar_q, kTileQK);
+        for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::Q + i * 8192, &p.tm_q, bar_q, i * 32, h, tb + t0, bc);
+        mbar_arrive_expect_tx(bar_u, kTileQK);
+        for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::U + i * 8192, &p.tm_u, bar_u, i * 32, h, tb + t0, bc);
+    };
+    // q, k of a later chunk into L2, so that its load (issued only once the
+    // current chunk's state update has released the tiles) hits L2
+    auto prefetch_qu = [&](int c) {
+        const int t0 = c * 128;
+        for (int i = 0; i < 3; ++i) {
+            tma_prefetch_l2_4d(&p.tm_q, i * 32, h, tb + t0, bc);
+            tma_prefetch_l2_4d(&p.tm_u, i * 32, h, tb + t0, bc);
+        }
+    };
+    auto issue_y = [&](int c, int s) {
+        uint8_t* y = sm + (s ? L::Y1 : L::Y0);
+        mbar_arrive_expect_tx(bar_y + s, kTileV);
+        for (int i = 0; i < 3; ++i)
+            tma_load_4d(y + i * 16384, &p.tm_y, bar_y + s, i * 64, h, tb + c * 128, bc);
+    };
+    if (producer) {
+        if (nchunks > 1) prefetch_qu(chunk_at(1));
+        if (nchunks > 0) {
+            issue_qu(chunk_at(0));
+            issue_y(chunk_at(0), 0);
+            if (nchunks > 1) issue_y(chunk_at(1), 1);
+        }
+    }
+
     // prologue: decays and state copy of the first chunk
     float a_nx = (tid < 128 && nchunks > 1) ? load_a(chunk_at(1)) : 0.f;
     if (nchunks > 0) decays(tid < 128 ? load_a(chunk_at(0)) : 0.f, 0);
@@ -528,40 +562,8 @@ __global__ void __launch_bounds__(chunk::kFusedThreads, 1) gla_fwd_fused_kernel(
         // ----------------------------------------------------------- producer
         // q, k of chunk it+1 once (D) of chunk it is done; the o tile of chunk
         // it from its v buffer once staged, then v of chunk it+2 into it
-        auto issue_qu = [&](int c) {
-            const int t0 = c * 128;
-            mbar_arrive_expect_tx(bar_q, kTileQK);
-            for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::Q + i * 8192, &p.tm_q, bar_q, i * 32, h, tb + t0, bc);
-            mbar_arrive_expect_tx(bar_u, kTileQK);
-            for (int i = 0; i < 3; ++i) tma_load_4d(sm + L::U + i * 8192, &p.tm_u, bar_u, i * 32, h, tb + t0, bc);
-        };
-        // q, k of a later chunk into L2, so that its load (issued only once the
-        // current chunk's state update has released the tiles) hits L2
-        auto prefetch_qu = [&](int c) {
-            const int t0 = c * 128;
-            for (int i = 0; i < 3; ++i) {
-                tma_prefetch_l2_4d(&p.tm_q, i * 32, h, tb + t0, bc);
-                tma_prefetch_l2_4d(&p.tm_u, i * 32, h, tb + t0, bc);
-            }
-        };
-        auto issue_y = [&](int c, int s) {
-            uint8_t* y = sm + (s ? L::Y1 : L::Y0);
-            mbar_arrive_expect_tx(bar_y + s, kTileV);
-            for (int i = 0; i < 3; ++i)
-                tma_load_4d(y + i * 16384, &p.tm_y, bar_y + s, i * 64, h, tb + c * 128, bc);
-        };
-        int n_qu = 0, n_y[2] = {0, 0};
-        if (nchunks > 1) prefetch_qu(chunk_at(1));
-        if (nchunks > 0) {
-            issue_qu(chunk_at(0));
-            ++n_qu;
-            issue_y(chunk_at(0), 0);
-            ++n_y[0];
-            if (nchunks > 1) {
-                issue_y(chunk_at(1), 1);
-                ++n_y[1];
-            }
-        }
+        // (loads issued so far: those of the first chunks, before the prologue)
+        int n_qu = nchunks > 0 ? 1 : 0, n_y[2] = {nchunks > 0 ? 1 : 0, nchunks > 1 ? 1 : 0};
         for (int it = 0; it < nchunks; ++it) {
             const int c = chunk_at(it), ys = it & 1;
             if (it + 2 < nchunks) prefetch_qu(c + 2 * dc);
